@@ -1,0 +1,264 @@
+/*
+ * pi_oracle.c -- plain, slow CPU oracle for the activation-sparse decode FFN.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  The product path (the
+ * CUDA library) never calls it, links it or shares code with it.
+ *
+ * Every value is decoded from the exact bytes the caller passes (fp32, fp16
+ * or Q4_0 split planes) by the code in this file, and all arithmetic is done
+ * in IEEE double.  There is no blocking, fusion or reordering: each sum runs
+ * over its index in ascending order.  OpenMP, when compiled in, only splits
+ * independent outputs between threads, so results do not depend on the
+ * thread count.
+ *
+ * Pages followed (titles as published):
+ *   [GN] GeekNews, "Serving model bahasa besar berkecepatan tinggi pada PC
+ *        dengan GPU konsumen"
+ *   [AB] aibars.net, "PowerInfer - Hochgeschwindigkeits-Inferenz-Engine für
+ *        große Sprachmodelle"
+ *   [UA] unite.ai, "PowerInfer: Tüketici Düzeyinde bir GPU ile Hızlı Büyük
+ *        Dil Modeli Sunucusu"
+ *
+ * Readings of points the pages leave open:
+ *   - predictor = low-rank GEMV -> ReLU -> GEMV (+ optional bias) -> strict
+ *     threshold, scoring cold neurons only; hot neurons are always computed;
+ *   - the batch mask is the union over the tokens of the block, and every
+ *     token is computed over that same union;
+ *   - the active-index list is ascending;
+ *   - squared ReLU is non-gated; the activation stays un-rounded (here: double);
+ *   - Q4_0 nibble order: in each 32-element block, byte k holds element k in
+ *     its low nibble and element k+16 in its high nibble; x = s * (q - 8);
+ *   - stack glue between layers: x = h + y, h' = x / sqrt(mean(x^2) + eps).
+ *
+ * Pinning: every function here is checked by the CPU test suite against
+ * hand-worked examples (tests/golden), closed forms, identities, brute force
+ * over all masks of tiny layers, and library routines for special cases.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* element types (this file's own numbering; the Python wrapper maps names) */
+enum { ORC_F32 = 0, ORC_F16 = 1, ORC_Q4_0 = 2 };
+/* activations: [GN] "Keterbatasan dan FAQ" names ReLU, ReGLU and squared ReLU */
+enum { ORC_RELU = 0, ORC_REGLU = 1, ORC_RELU2 = 2 };
+
+void orc_set_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
+int orc_get_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+/* IEEE 754 binary16 -> double, from the bit fields. */
+double orc_half_to_double(uint16_t bits) {
+  int sign = (bits >> 15) & 1;
+  int expo = (bits >> 10) & 0x1f;
+  int mant = bits & 0x3ff;
+  double v;
+  if (expo == 0) {
+    v = ldexp((double)mant, -24); /* subnormal: mant * 2^-14 / 2^10 */
+  } else if (expo == 31) {
+    v = mant ? NAN : INFINITY;
+  } else {
+    v = ldexp((double)(mant | 0x400), expo - 25); /* (1 + mant/2^10) * 2^(expo-15) */
+  }
+  return sign ? -v : v;
+}
+
+/*
+ * One element (row, col) of a row-major [rows, d] matrix stored as `type`.
+ * Q4_0 ([GN] "Kuantisasi dan kompatibilitas": INT4 Q4_0, 32-element blocks
+ * with an fp16 scale) uses split planes: qs [rows, d/2] bytes and
+ * sc [rows, d/32] fp16.
+ */
+double orc_elem(int type, const void *data, const void *scales, int64_t row, int64_t col, int64_t d) {
+  if (type == ORC_F32) {
+    return (double)((const float *)data)[row * d + col];
+  }
+  if (type == ORC_F16) {
+    return orc_half_to_double(((const uint16_t *)data)[row * d + col]);
+  }
+  /* Q4_0 */
+  const uint8_t *qs = (const uint8_t *)data + row * (d / 2);
+  const uint16_t *sc = (const uint16_t *)scales + row * (d / 32);
+  int64_t blk = col / 32;
+  int64_t k = col % 32;
+  uint8_t byte = qs[blk * 16 + (k % 16)];
+  int q = (k < 16) ? (byte & 0x0f) : (byte >> 4);
+  return orc_half_to_double(sc[blk]) * (double)(q - 8);
+}
+
+/* Decode a whole token block h [batch, d] into doubles. */
+static double *decode_tokens(int htype, const void *h, int batch, int d) {
+  double *out = (double *)malloc(sizeof(double) * (size_t)batch * (size_t)d);
+  for (int b = 0; b < batch; ++b)
+    for (int i = 0; i < d; ++i) out[(size_t)b * d + i] = orc_elem(htype, h, NULL, b, i, d);
+  return out;
+}
+
+/*
+ * Predictor ([UA] "Adaptif Sparsite Predictor’ları": a per-layer predictor
+ * picks the neurons that will fire; only those are computed).
+ *   u[b,k] = max(0, sum_i P1[k,i] h[b,i])                 k < rank
+ *   s[b,c] = sum_k P2[c,k] u[b,k] + bp[c]                  c < ffn - n_hot
+ *   active(c) = OR_b (s[b,c] > thr)
+ *   idx = ascending { n_hot + c : active(c) }
+ * Any output pointer may be NULL.  Returns the number of active neurons.
+ */
+int64_t orc_predict(int d, int ffn, int n_hot, int rank, int htype, int ptype, int batch,
+                    const void *h, const void *P1, const void *P2, const float *bp, double thr,
+                    double *u_out, double *s_out, uint8_t *mask_out, int32_t *idx_out) {
+  const int n_cold = ffn - n_hot;
+  double *hd = decode_tokens(htype, h, batch, d);
+  double *u = (double *)malloc(sizeof(double) * (size_t)batch * (size_t)rank);
+  double *s = (double *)malloc(sizeof(double) * (size_t)batch * (size_t)(n_cold > 0 ? n_cold : 1));
+
+  for (int b = 0; b < batch; ++b) {
+#pragma omp parallel for schedule(static)
+    for (int k = 0; k < rank; ++k) {
+      double acc = 0.0;
+      for (int i = 0; i < d; ++i) acc += orc_elem(ptype, P1, NULL, k, i, d) * hd[(size_t)b * d + i];
+      u[(size_t)b * rank + k] = acc > 0.0 ? acc : 0.0;
+    }
+  }
+  for (int b = 0; b < batch; ++b) {
+#pragma omp parallel for schedule(static)
+    for (int c = 0; c < n_cold; ++c) {
+      double acc = 0.0;
+      for (int k = 0; k < rank; ++k) acc += orc_elem(ptype, P2, NULL, c, k, rank) * u[(size_t)b * rank + k];
+      if (bp) acc += (double)bp[c];
+      s[(size_t)b * n_cold + c] = acc;
+    }
+  }
+  int64_t count = 0;
+  for (int c = 0; c < n_cold; ++c) {
+    int on = 0;
+    for (int b = 0; b < batch; ++b) on |= (s[(size_t)b * n_cold + c] > thr);
+    if (mask_out) mask_out[c] = (uint8_t)on;
+    if (on) {
+      if (idx_out) idx_out[count] = n_hot + c;
+      ++count;
+    }
+  }
+  if (u_out) memcpy(u_out, u, sizeof(double) * (size_t)batch * (size_t)rank);
+  if (s_out) memcpy(s_out, s, sizeof(double) * (size_t)batch * (size_t)n_cold);
+  free(hd);
+  free(u);
+  free(s);
+  return count;
+}
+
+/* Pre-activation of neuron j for token row hb (the bias sits on the gate
+ * for ReGLU and on the single up projection otherwise). */
+static double preact(const void *w, const void *w_sc, int wtype, const float *b1, int64_t j, const double *hb, int d) {
+  double acc = 0.0;
+  for (int i = 0; i < d; ++i) acc += orc_elem(wtype, w, w_sc, j, i, d) * hb[i];
+  if (b1) acc += (double)b1[j];
+  return acc;
+}
+
+/* Activation value of neuron j for one token ([GN] "Keterbatasan dan FAQ"). */
+static double neuron_act(int act, int wtype, const void *wg, const void *wg_sc, const void *wu, const void *wu_sc,
+                         const float *b1, int64_t j, const double *hb, int d) {
+  if (act == ORC_REGLU) {
+    double g = preact(wg, wg_sc, wtype, b1, j, hb, d);
+    double v = preact(wu, wu_sc, wtype, NULL, j, hb, d);
+    return (g > 0.0 ? g : 0.0) * v;
+  }
+  double z = preact(wu, wu_sc, wtype, b1, j, hb, d);
+  double r = z > 0.0 ? z : 0.0;
+  return act == ORC_RELU2 ? r * r : r;
+}
+
+/*
+ * Masked FFN ([UA] "Nöron Bilinçli Operatör": the operator works on single
+ * rows of the up/gate matrices and single columns of the down matrix; the
+ * down columns are stored neuron-major as the rows of W_downT).
+ *   list = [0, n_hot) ++ idx[0, count)            (idx ascending, each >= n_hot)
+ *   y[b,e] = b2[e] + sum_{j in list, in list order} a[b,j] * W_downT[j,e]
+ * The same list is used for every token of the block.  cols / ncols select
+ * which columns e to compute (cols == NULL: all d, y is [batch, d]; else y is
+ * [batch, ncols]).  a_out, if given, receives a[b, position in list].
+ */
+void orc_masked_ffn(int d, int ffn, int n_hot, int wtype, int act, int htype, int batch, const void *h,
+                    const int32_t *idx, int64_t count, const void *wg, const void *wg_sc, const void *wu,
+                    const void *wu_sc, const void *wd, const void *wd_sc, const float *b1, const float *b2,
+                    const int32_t *cols, int ncols, double *y_out, double *a_out) {
+  (void)ffn;
+  const int64_t n_list = (int64_t)n_hot + count;
+  double *hd = decode_tokens(htype, h, batch, d);
+  double *a = (double *)malloc(sizeof(double) * (size_t)batch * (size_t)(n_list > 0 ? n_list : 1));
+  for (int b = 0; b < batch; ++b) {
+#pragma omp parallel for schedule(static)
+    for (int64_t p = 0; p < n_list; ++p) {
+      int64_t j = p < n_hot ? p : (int64_t)idx[p - n_hot];
+      a[(size_t)b * n_list + p] = neuron_act(act, wtype, wg, wg_sc, wu, wu_sc, b1, j, hd + (size_t)b * d, d);
+    }
+  }
+  const int n_out = cols ? ncols : d;
+  for (int b = 0; b < batch; ++b) {
+#pragma omp parallel for schedule(static)
+    for (int o = 0; o < n_out; ++o) {
+      int64_t e = cols ? cols[o] : o;
+      double acc = b2 ? (double)b2[e] : 0.0;
+      for (int64_t p = 0; p < n_list; ++p) {
+        int64_t j = p < n_hot ? p : (int64_t)idx[p - n_hot];
+        acc += a[(size_t)b * n_list + p] * orc_elem(wtype, wd, wd_sc, j, e, d);
+      }
+      y_out[(size_t)b * n_out + o] = acc;
+    }
+  }
+  if (a_out) memcpy(a_out, a, sizeof(double) * (size_t)batch * (size_t)n_list);
+  free(hd);
+  free(a);
+}
+
+/*
+ * True activation support: support[b, j] = 1 iff neuron j's (gate, for
+ * ReGLU; else up) pre-activation including b1 is > 0 for token b.
+ */
+void orc_true_support(int d, int ffn, int wtype, int act, int htype, int batch, const void *h, const void *wg,
+                      const void *wg_sc, const void *wu, const void *wu_sc, const float *b1, uint8_t *support) {
+  double *hd = decode_tokens(htype, h, batch, d);
+  const void *w = act == ORC_REGLU ? wg : wu;
+  const void *w_sc = act == ORC_REGLU ? wg_sc : wu_sc;
+  for (int b = 0; b < batch; ++b) {
+#pragma omp parallel for schedule(static)
+    for (int j = 0; j < ffn; ++j)
+      support[(size_t)b * ffn + j] = (uint8_t)(preact(w, w_sc, wtype, b1, j, hd + (size_t)b * d, d) > 0.0);
+  }
+  free(hd);
+}
+
+/*
+ * Stack glue between layers (the pages are silent; residual + RMSNorm with
+ * unit gain): x = h + y;  out = x / sqrt(mean_e x[e]^2 + eps).
+ */
+void orc_residual_rmsnorm(int batch, int d, int htype, const void *h, const double *y, double eps, double *out) {
+  double *hd = decode_tokens(htype, h, batch, d);
+  for (int b = 0; b < batch; ++b) {
+    double ss = 0.0;
+    for (int e = 0; e < d; ++e) {
+      double x = hd[(size_t)b * d + e] + y[(size_t)b * d + e];
+      ss += x * x;
+    }
+    double inv = 1.0 / sqrt(ss / (double)d + eps);
+    for (int e = 0; e < d; ++e) out[(size_t)b * d + e] = (hd[(size_t)b * d + e] + y[(size_t)b * d + e]) * inv;
+  }
+  free(hd);
+}

@@ -1,0 +1,295 @@
+"""Seeded synthetic workloads for the activation-sparse decode FFN.
+
+This module only *makes inputs*: weights, predictor matrices, biases and token
+blocks with the shapes and statistics of the five benchmark workloads.  It
+holds none of the method's arithmetic (no predictor evaluation, no FFN, no
+decoding of Q4_0); both the CUDA path and the CPU oracle consume what it
+makes, and neither is imported here.
+
+Statistics (the pages give none of these numerically; each choice is the
+plainest one that reproduces the property the pages describe):
+
+* Power-law neuron activity ([AB] "Hot-Cold-Neuron-Mechanismus"; [UA]
+  "Offline Aşama"): neuron of Zipf rank k fires with probability
+  p_k = min(0.99, c * k^-alpha), c bisected so that mean_k p_k = 1 - sparsity.
+  The rank -> neuron-id map is a seeded random permutation.
+* The firing rate is set through the bias b1 = Phi^-1(p) on the gate (ReGLU)
+  or the up projection (ReLU, squared ReLU): with ||h||^2 = d and rows of
+  variance 1/d, w.h ~ N(0, 1), so P(w.h + b1 > 0) = p.
+* Predictor: W_gate (or W_up) = U V + sqrt(1 - rho) E with U ~ N(0, rho/r'),
+  V ~ N(0, 1/d), E ~ N(0, 1/d), r' = rank / 2, rho = 0.9.  P1 = [V; -V] and
+  P2 = [U, -U] (cold rows only), bp = b1 + thr, so that
+  P2 ReLU(P1 h) + bp - thr = U V h + b1, the low-rank part of the true
+  pre-activation.
+* Hot set: the top ceil(hot_frac * ffn) neurons by firing probability.  The
+  offline layout stores them first ([UA] "Nöron Yerleştirme ve Yönetimi":
+  a neuron table maps each placed neuron back to its original row); ``perm``
+  is that table (storage row -> original row).
+* Q4_0 ([GN] "Kuantisasi dan kompatibilitas"): 32-element blocks along d,
+  scale s = m / -8 where m is the block element of largest magnitude (sign
+  kept), rounded to fp16; q = clamp(round_half_away(x / s) + 8, 0, 15); byte k
+  of a block holds q[k] (low nibble) and q[k + 16] (high nibble).  Split
+  planes: qs [rows, d/2] uint8 and sc [rows, d/32] fp16.
+* Tokens: h ~ N(0, 1)^d, scaled so that ||h||^2 = d.
+
+Pages: [GN] GeekNews "Serving model bahasa besar berkecepatan tinggi pada PC
+dengan GPU konsumen"; [AB] aibars.net "PowerInfer - Hochgeschwindigkeits-
+Inferenz-Engine für große Sprachmodelle"; [UA] unite.ai "PowerInfer: Tüketici
+Düzeyinde bir GPU ile Hızlı Büyük Dil Modeli Sunucusu".
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, List, Optional
+
+import numpy as np
+import torch
+
+RHO = 0.9
+THRESHOLD = 0.5
+RMS_EPS = 1e-6
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    cfg_id: int
+    d: int
+    ffn: int
+    layers: int
+    act: str          # "relu" | "reglu" | "relu2"
+    wtype: str        # "f32" | "f16" | "q4_0"
+    ptype: str        # "f32" | "f16" (predictor and token dtype)
+    sparsity: float
+    alpha: float
+    hot_frac: float
+    rank: int
+    batches: tuple
+    steps: int
+    has_b2: bool = False
+    thr: float = THRESHOLD
+
+    @property
+    def n_hot(self) -> int:
+        return int(math.ceil(self.hot_frac * self.ffn - 1e-9))
+
+    @property
+    def n_cold(self) -> int:
+        return self.ffn - self.n_hot
+
+    @property
+    def gated(self) -> bool:
+        return self.act == "reglu"
+
+    def with_(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+# The five synthetic workloads (shapes of OPT-tiny, ReluLLaMA-7B, Llama2-13B,
+# Falcon-40B and Llama2-70B FFNs).  Steps for the last three are not fixed by
+# their statement; 512 / 128 / 128 bound the run time.
+WORKLOADS: Dict[str, Workload] = {
+    "tiny-relu-fp32": Workload("tiny-relu-fp32", 1, 512, 2048, 2, "relu", "f32", "f32", 0.90, 1.1, 0.05, 64,
+                               (1,), 256, has_b2=True),
+    "7b-reglu-fp16": Workload("7b-reglu-fp16", 2, 4096, 11008, 32, "reglu", "f16", "f16", 0.88, 1.2, 0.10, 1024,
+                              (1,), 512),
+    "13b-reglu-q4_0": Workload("13b-reglu-q4_0", 3, 5120, 13824, 40, "reglu", "q4_0", "f16", 0.90, 1.2, 0.10, 1024,
+                               (1,), 512),
+    "40b-relu-fp16": Workload("40b-relu-fp16", 4, 8192, 32768, 60, "relu", "f16", "f16", 0.92, 1.3, 0.08, 1536,
+                              (1, 8), 128),
+    "70b-reglu-fp16": Workload("70b-reglu-fp16", 5, 8192, 28672, 80, "reglu", "f16", "f16", 0.90, 1.2, 0.10, 2048,
+                               (1, 4, 16), 128),
+}
+SPARSITY_SWEEP_70B = (0.80, 0.90, 0.95)
+
+_TORCH_DT = {"f32": torch.float32, "f16": torch.float16}
+
+
+def _seed(w: Workload, layer: int, tensor: int) -> int:
+    key = (w.cfg_id * 1_000_003 + int(round(w.sparsity * 1000))) * 10_007 + layer
+    return (key * 131 + tensor) & 0x7FFF_FFFF_FFFF
+
+
+def _gen(device, seed: int) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def zipf_probs(n: int, alpha: float, mean: float, pmax: float = 0.99) -> np.ndarray:
+    """p[k-1] = min(pmax, c k^-alpha) for Zipf rank k = 1..n with mean(p) = mean (bisection on c)."""
+    base = np.arange(1, n + 1, dtype=np.float64) ** (-alpha)
+    lo, hi = 0.0, 1.0 / base[-1]
+    for _ in range(200):
+        c = 0.5 * (lo + hi)
+        if np.minimum(pmax, c * base).mean() < mean:
+            lo = c
+        else:
+            hi = c
+    return np.minimum(pmax, 0.5 * (lo + hi) * base)
+
+
+def neuron_layout(w: Workload, layer: int):
+    """Firing probabilities and the hot-first neuron table for one layer.
+
+    Returns (p_orig [ffn] float64 by original neuron id, perm [ffn] int64 with
+    perm[storage row] = original id: hot ids ascending, then cold ids ascending).
+    """
+    p_rank = zipf_probs(w.ffn, w.alpha, 1.0 - w.sparsity)
+    rng = np.random.default_rng(_seed(w, layer, 1))
+    rank_to_id = rng.permutation(w.ffn)
+    p_orig = np.empty(w.ffn, np.float64)
+    p_orig[rank_to_id] = p_rank
+    hot_ids = np.sort(rank_to_id[: w.n_hot])
+    is_hot = np.zeros(w.ffn, bool)
+    is_hot[hot_ids] = True
+    perm = np.concatenate([hot_ids, np.nonzero(~is_hot)[0]]).astype(np.int64)
+    return p_orig, perm
+
+
+def quantize_q4_0(x: torch.Tensor):
+    """Q4_0 split planes of a [rows, d] tensor (d % 32 == 0): (qs uint8 [rows, d/2], sc fp16 [rows, d/32])."""
+    rows, d = x.shape
+    assert d % 32 == 0
+    blk = x.float().reshape(rows, d // 32, 32)
+    amax_i = blk.abs().argmax(dim=-1, keepdim=True)
+    m = torch.gather(blk, -1, amax_i)
+    s16 = (m / -8.0).to(torch.float16)
+    s = s16.float()
+    safe = torch.where(s == 0, torch.ones_like(s), s)
+    v = blk / safe
+    q = torch.sign(v) * torch.floor(v.abs() + 0.5) + 8.0
+    q = torch.where(s == 0, torch.full_like(q, 8.0), q).clamp_(0, 15).to(torch.uint8)
+    qs = (q[..., :16] | (q[..., 16:] << 4)).reshape(rows, d // 2).contiguous()
+    sc = s16.reshape(rows, d // 32).contiguous()
+    return qs, sc
+
+
+def _as_wtype(x: torch.Tensor, wtype: str):
+    if wtype == "q4_0":
+        return quantize_q4_0(x.to(torch.float16))
+    return x.to(_TORCH_DT[wtype]).contiguous()
+
+
+def make_layer(w: Workload, layer: int, device="cpu") -> dict:
+    """All tensors of one layer in storage (hot-first) order, on `device`.
+
+    Keys: Wg (ReGLU only), Wu, WdT (each a tensor [ffn, d] or a Q4_0 pair),
+    b1 fp32 [ffn], b2 fp32 [d] or None, P1 [rank, d], P2 [n_cold, rank], bp fp32
+    [n_cold], perm int64 [ffn], p fp64 [ffn] (storage order), thr.
+    """
+    d, F, r = w.d, w.ffn, w.rank
+    assert r % 2 == 0
+    rh = r // 2
+    p_orig, perm = neuron_layout(w, layer)
+    perm_t = torch.as_tensor(perm, device=device)
+    inv_sd = 1.0 / math.sqrt(d)
+
+    U = torch.randn(F, rh, generator=_gen(device, _seed(w, layer, 2)), device=device) * math.sqrt(RHO / rh)
+    V = torch.randn(rh, d, generator=_gen(device, _seed(w, layer, 3)), device=device) * inv_sd
+    E = torch.randn(F, d, generator=_gen(device, _seed(w, layer, 4)), device=device) * inv_sd
+    W_pred = U @ V
+    W_pred.add_(E, alpha=math.sqrt(1.0 - RHO))
+    del E
+    W_other = torch.randn(F, d, generator=_gen(device, _seed(w, layer, 5)), device=device) * inv_sd
+    WdT = torch.randn(F, d, generator=_gen(device, _seed(w, layer, 6)), device=device) * inv_sd
+
+    b1_orig = torch.special.ndtri(torch.as_tensor(p_orig, dtype=torch.float64)).to(torch.float32)
+    out = {"perm": perm, "p": p_orig[perm], "thr": w.thr}
+    if w.gated:
+        out["Wg"] = _as_wtype(W_pred[perm_t], w.wtype)
+        out["Wu"] = _as_wtype(W_other[perm_t], w.wtype)
+    else:
+        out["Wg"] = None
+        out["Wu"] = _as_wtype(W_pred[perm_t], w.wtype)
+    del W_pred, W_other
+    out["WdT"] = _as_wtype(WdT[perm_t], w.wtype)
+    del WdT
+    b1 = b1_orig.to(device)[perm_t].contiguous()
+    out["b1"] = b1
+    if w.has_b2:
+        out["b2"] = (torch.randn(d, generator=_gen(device, _seed(w, layer, 7)), device=device) * 0.05).float()
+    else:
+        out["b2"] = None
+    pt = _TORCH_DT[w.ptype]
+    out["P1"] = torch.cat([V, -V], dim=0).to(pt).contiguous()
+    U_cold = U[perm_t[w.n_hot:]]
+    out["P2"] = torch.cat([U_cold, -U_cold], dim=1).to(pt).contiguous()
+    out["bp"] = (b1[w.n_hot:] + w.thr).float().contiguous()
+    return out
+
+
+def make_tokens(w: Workload, batch: int, step: int, device="cpu") -> torch.Tensor:
+    """Token block h [batch, d] for decode step `step`: N(0,1) rows scaled to ||h||^2 = d."""
+    g = _gen(device, _seed(w, 0xF0, step))
+    h = torch.randn(batch, w.d, generator=g, device=device, dtype=torch.float64)
+    h = h * (math.sqrt(w.d) / h.norm(dim=1, keepdim=True))
+    return h.to(_TORCH_DT[w.ptype]).contiguous()
+
+
+def make_int_layer(d: int, ffn: int, n_hot: int, rank: int, act: str, wtype: str, ptype: str, batch: int,
+                   seed: int, density: float = 0.05, device="cpu") -> dict:
+    """A layer whose every product and partial sum is exact in fp16/fp32/double.
+
+    Weights, predictor entries and tokens are small integers (Q4_0: s * (q - 8)
+    with s a power of two), most of them zero, so that dot products are small
+    integers and fp32 accumulation is exact in any order.  bp is an integer
+    and thr = 0.5, so no score ever ties the threshold.
+    """
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+
+    def sparse_int(shape, lo, hi, dens):
+        v = torch.randint(lo, hi + 1, shape, generator=g).float()
+        keep = torch.rand(shape, generator=g) < dens
+        return v * keep
+
+    h = sparse_int((batch, d), -2, 2, 0.5)
+    out = {"h": h.to(_TORCH_DT[ptype]).to(device), "thr": 0.5, "perm": np.arange(ffn)}
+    if wtype == "q4_0":
+        def qmat():
+            q = torch.randint(0, 16, (ffn, d), generator=g)
+            keep = torch.rand((ffn, d), generator=g) < density
+            q = torch.where(keep, q, torch.full_like(q, 8)).to(torch.uint8).reshape(ffn, d // 32, 32)
+            qs = (q[..., :16] | (q[..., 16:] << 4)).reshape(ffn, d // 2).contiguous()
+            e = torch.randint(-2, 1, (ffn, d // 32), generator=g).float()
+            sc = torch.pow(2.0, e).to(torch.float16).contiguous()
+            return qs.to(device), sc.to(device)
+        Wg, Wu, WdT = (qmat() if act == "reglu" else None), qmat(), qmat()
+    else:
+        dt = _TORCH_DT[wtype]
+        Wg = sparse_int((ffn, d), -2, 2, density).to(dt).to(device) if act == "reglu" else None
+        Wu = sparse_int((ffn, d), -2, 2, density).to(dt).to(device)
+        WdT = sparse_int((ffn, d), -2, 2, density).to(dt).to(device)
+    out.update(Wg=Wg, Wu=Wu, WdT=WdT)
+    out["b1"] = torch.randint(-1, 2, (ffn,), generator=g).float().to(device)
+    out["b2"] = torch.randint(-2, 3, (d,), generator=g).float().to(device)
+    pt = _TORCH_DT[ptype]
+    out["P1"] = sparse_int((rank, d), -1, 1, min(1.0, 8.0 / d + density)).to(pt).to(device)
+    out["P2"] = sparse_int((ffn - n_hot, rank), -1, 1, min(1.0, 4.0 / rank + density)).to(pt).to(device)
+    out["bp"] = torch.randint(-2, 2, (ffn - n_hot,), generator=g).float().to(device)
+    return out
+
+
+def layer_bytes(w: Workload, batch: int, n_active: float) -> float:
+    """Algorithmic bytes one layer must move for one token block with n_active
+    predicted-active cold neurons: both predictor matrices, the listed weight
+    rows (hot + active), their biases, the index list, and the token block in
+    and the fp32 output out."""
+    e_p = 4 if w.ptype == "f32" else 2
+    e_w = {"f32": 4.0, "f16": 2.0, "q4_0": 18.0 / 32.0}[w.wtype]
+    mats = 3 if w.gated else 2
+    n_list = w.n_hot + n_active
+    pred = (w.rank * w.d + w.n_cold * w.rank) * e_p + 4 * w.n_cold          # P1, P2, bp
+    ffn = mats * n_list * w.d * e_w + 4 * n_list                           # rows + b1
+    idx = 4 * n_active
+    io = batch * w.d * e_p + batch * w.d * 4 + (4 * w.d if w.has_b2 else 0)
+    return pred + ffn + idx + io
+
+
+def expected_active(w: Workload, batch: int) -> float:
+    """E[|union of cold actives|] under the Zipf model, for planning only."""
+    p_rank = zipf_probs(w.ffn, w.alpha, 1.0 - w.sparsity)
+    cold = p_rank[w.n_hot:]
+    return float(np.sum(1.0 - (1.0 - cold) ** batch))
