@@ -1,0 +1,265 @@
+// pi_api.cu -- the C ABI of libpi (declared in include/pi.h): argument checks,
+// workspace layout and launch sequences.  Nothing here allocates device memory.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "pi.h"
+#include "pi_common.cuh"
+#include "pi_kernels_v1.cuh"
+#include "pi_layout.h"
+
+namespace {
+
+thread_local char g_err[512] = "no error";
+
+pi_status fail(pi_status st, const char* fmt, const char* what) {
+  snprintf(g_err, sizeof(g_err), fmt, what);
+  return st;
+}
+
+pi_status cuda_fail(cudaError_t e, const char* where) {
+  snprintf(g_err, sizeof(g_err), "%s: %s", where, cudaGetErrorString(e));
+  return PI_ERR_CUDA;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+pi_status check_desc(const pi_ffn_desc* d, int32_t batch) {
+  if (!d) return fail(PI_ERR_INVALID_ARG, "%s", "desc is NULL");
+  if (d->d <= 0 || d->d % 8) return fail(PI_ERR_INVALID_ARG, "%s", "d must be a positive multiple of 8");
+  if (d->ffn <= 0) return fail(PI_ERR_INVALID_ARG, "%s", "ffn must be positive");
+  if (d->n_hot < 0 || d->n_hot > d->ffn) return fail(PI_ERR_INVALID_ARG, "%s", "n_hot must be in [0, ffn]");
+  if (d->rank <= 0 || d->rank % 8) return fail(PI_ERR_INVALID_ARG, "%s", "rank must be a positive multiple of 8");
+  if (d->wtype != PI_F32 && d->wtype != PI_F16 && d->wtype != PI_Q4_0)
+    return fail(PI_ERR_INVALID_ARG, "%s", "wtype must be PI_F32, PI_F16 or PI_Q4_0");
+  if (d->ptype != PI_F32 && d->ptype != PI_F16) return fail(PI_ERR_INVALID_ARG, "%s", "ptype must be PI_F32 or PI_F16");
+  if (d->act != PI_ACT_RELU && d->act != PI_ACT_REGLU && d->act != PI_ACT_RELU2)
+    return fail(PI_ERR_INVALID_ARG, "%s", "act must be PI_ACT_RELU, PI_ACT_REGLU or PI_ACT_RELU2");
+  if (d->wtype == PI_Q4_0 && d->d % 32) return fail(PI_ERR_INVALID_ARG, "%s", "Q4_0 needs d % 32 == 0");
+  if (batch < 1 || batch > PI_MAX_BATCH) return fail(PI_ERR_INVALID_ARG, "%s", "batch must be in [1, 16]");
+  if (d->d > 16384) return fail(PI_ERR_UNSUPPORTED, "%s", "d above 16384 is not supported");
+  if (d->rank > 65536) return fail(PI_ERR_UNSUPPORTED, "%s", "rank above 65536 is not supported");
+  return PI_OK;
+}
+
+pi_status check_ptr(const void* p, size_t align, const char* name) {
+  if (!p) return fail(PI_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned(p, align)) return fail(PI_ERR_INVALID_ARG, "%s is not aligned", name);
+  return PI_OK;
+}
+
+pi_status check_weight(const pi_ffn_desc* d, pi_weight w, const char* name) {
+  pi_status s = check_ptr(w.data, 16, name);
+  if (s) return s;
+  if (d->wtype == PI_Q4_0) {
+    s = check_ptr(w.scales, 16, "Q4_0 scales");
+    if (s) return s;
+  }
+  return PI_OK;
+}
+
+pi_status check_ws(const pi_ffn_desc* d, int32_t batch, void* ws, size_t ws_bytes) {
+  pi_status s = check_ptr(ws, 256, "ws");
+  if (s) return s;
+  if (ws_bytes < pi_workspace_bytes(d, batch))
+    return fail(PI_ERR_CAPACITY, "%s", "workspace smaller than pi_workspace_bytes()");
+  return PI_OK;
+}
+
+#define PI_TRY(x)                   \
+  do {                              \
+    pi_status _s = (x);             \
+    if (_s != PI_OK) return _s;     \
+  } while (0)
+#define PI_CUDA(x, where)                          \
+  do {                                             \
+    cudaError_t _e = (x);                          \
+    if (_e != cudaSuccess) return cuda_fail(_e, where); \
+  } while (0)
+
+pi_status predict_impl(const pi_ffn_desc* d, int32_t B, const void* h, const void* P1, const void* P2,
+                       const float* bp, float thr, int32_t* idx, int32_t* count, char* ws, cudaStream_t st) {
+  const pi::WsLayout L = pi::ws_layout(d->d, d->ffn, d->n_hot, d->rank, B);
+  float* u = reinterpret_cast<float*>(ws + L.u);
+  uint32_t* tmask = reinterpret_cast<uint32_t*>(ws + L.tile_mask);
+  int* tcount = reinterpret_cast<int*>(ws + L.tile_count);
+  const int C = d->ffn - d->n_hot;
+  const int sms = sm_count();
+  PI_CUDA(pi::launch_pred_u(d->ptype, P1, h, B, d->d, d->rank, u, sms, st), "predictor GEMV1 launch");
+  PI_CUDA(pi::launch_pred_score(d->ptype, P2, bp, u, B, d->rank, C, thr, tmask, tcount, st), "predictor score launch");
+  PI_CUDA(pi::launch_compact(tmask, tcount, C, d->n_hot, idx, count, st), "compaction launch");
+  return PI_OK;
+}
+
+pi_status ffn_impl(const pi_ffn_desc* d, int32_t B, const void* h, const int32_t* idx, const int32_t* count,
+                   pi_weight Wg, pi_weight Wu, pi_weight Wd, const float* b1, const float* b2, float* y, char* ws,
+                   cudaStream_t st) {
+  const pi::WsLayout L = pi::ws_layout(d->d, d->ffn, d->n_hot, d->rank, B);
+  int* status = reinterpret_cast<int*>(ws);
+  float* a = reinterpret_cast<float*>(ws + L.act);
+  float* partial = reinterpret_cast<float*>(ws + L.partial);
+  const int sms = sm_count();
+  const int G = L.g_max < 2 * sms ? L.g_max : 2 * sms;
+  PI_CUDA(pi::launch_ffn_act(d->wtype, d->ptype, d->act, h, B, d->d, d->ffn, d->n_hot, idx, count, Wg.data,
+                             Wg.scales, Wu.data, Wu.scales, b1, a, d->ffn, status, sms, st),
+          "FFN activation launch");
+  PI_CUDA(pi::launch_ffn_down(d->wtype, B, d->d, d->ffn, d->n_hot, idx, count, Wd.data, Wd.scales, a, d->ffn,
+                              partial, G, st),
+          "FFN down launch");
+  PI_CUDA(pi::launch_ffn_reduce(partial, G, B, d->d, b2, y, st), "split-K reduce launch");
+  return PI_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pi_last_error(void) { return g_err; }
+
+const char* pi_version(void) { return "0.1.0"; }
+
+size_t pi_workspace_bytes(const pi_ffn_desc* desc, int32_t batch) {
+  if (check_desc(desc, batch) != PI_OK) return 0;
+  return pi::ws_layout(desc->d, desc->ffn, desc->n_hot, desc->rank, batch).total;
+}
+
+pi_status pi_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  PI_TRY(check_ptr(ws, 256, "ws"));
+  if (ws_bytes < sizeof(pi::Ctrl)) return fail(PI_ERR_CAPACITY, "%s", "workspace smaller than its control block");
+  PI_CUDA(cudaMemsetAsync(ws, 0, sizeof(pi::Ctrl), (cudaStream_t)stream), "workspace init");
+  return PI_OK;
+}
+
+pi_status pi_predict(const pi_ffn_desc* desc, int32_t batch, const void* h, const void* P1, const void* P2,
+                     const float* bp, float threshold, int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,
+                     void* stream) {
+  PI_TRY(check_desc(desc, batch));
+  PI_TRY(check_ptr(h, 16, "h"));
+  PI_TRY(check_ptr(P1, 16, "P1"));
+  if (desc->ffn > desc->n_hot) PI_TRY(check_ptr(P2, 16, "P2"));
+  if (bp) PI_TRY(check_ptr(bp, 4, "bp"));
+  PI_TRY(check_ptr(idx, 4, "idx"));
+  PI_TRY(check_ptr(count, 4, "count"));
+  PI_TRY(check_ws(desc, batch, ws, ws_bytes));
+  return predict_impl(desc, batch, h, P1, P2, bp, threshold, idx, count, (char*)ws, (cudaStream_t)stream);
+}
+
+pi_status pi_sparse_ffn(const pi_ffn_desc* desc, int32_t batch, const void* h, const int32_t* idx,
+                        const int32_t* count, pi_weight W_gate, pi_weight W_up, pi_weight W_downT, const float* b1,
+                        const float* b2, float* y, void* ws, size_t ws_bytes, void* stream) {
+  PI_TRY(check_desc(desc, batch));
+  PI_TRY(check_ptr(h, 16, "h"));
+  PI_TRY(check_ptr(idx, 4, "idx"));
+  PI_TRY(check_ptr(count, 4, "count"));
+  if (desc->act == PI_ACT_REGLU) PI_TRY(check_weight(desc, W_gate, "W_gate"));
+  PI_TRY(check_weight(desc, W_up, "W_up"));
+  PI_TRY(check_weight(desc, W_downT, "W_downT"));
+  if (b1) PI_TRY(check_ptr(b1, 4, "b1"));
+  if (b2) PI_TRY(check_ptr(b2, 16, "b2"));
+  PI_TRY(check_ptr(y, 16, "y"));
+  PI_TRY(check_ws(desc, batch, ws, ws_bytes));
+  return ffn_impl(desc, batch, h, idx, count, W_gate, W_up, W_downT, b1, b2, y, (char*)ws, (cudaStream_t)stream);
+}
+
+pi_status pi_layer(const pi_ffn_desc* desc, int32_t batch, const void* h, const pi_layer_weights* w, int32_t* idx,
+                   int32_t* count, float* y, void* ws, size_t ws_bytes, void* stream) {
+  if (!w) return fail(PI_ERR_INVALID_ARG, "%s", "layer weights are NULL");
+  PI_TRY(check_desc(desc, batch));
+  PI_TRY(check_ptr(h, 16, "h"));
+  PI_TRY(check_ptr(w->P1, 16, "P1"));
+  if (desc->ffn > desc->n_hot) PI_TRY(check_ptr(w->P2, 16, "P2"));
+  if (w->bp) PI_TRY(check_ptr(w->bp, 4, "bp"));
+  PI_TRY(check_ptr(idx, 4, "idx"));
+  PI_TRY(check_ptr(count, 4, "count"));
+  if (desc->act == PI_ACT_REGLU) PI_TRY(check_weight(desc, w->W_gate, "W_gate"));
+  PI_TRY(check_weight(desc, w->W_up, "W_up"));
+  PI_TRY(check_weight(desc, w->W_downT, "W_downT"));
+  if (w->b1) PI_TRY(check_ptr(w->b1, 4, "b1"));
+  if (w->b2) PI_TRY(check_ptr(w->b2, 16, "b2"));
+  PI_TRY(check_ptr(y, 16, "y"));
+  PI_TRY(check_ws(desc, batch, ws, ws_bytes));
+  cudaStream_t st = (cudaStream_t)stream;
+  PI_TRY(predict_impl(desc, batch, h, w->P1, w->P2, w->bp, w->threshold, idx, count, (char*)ws, st));
+  return ffn_impl(desc, batch, h, idx, count, w->W_gate, w->W_up, w->W_downT, w->b1, w->b2, y, (char*)ws, st);
+}
+
+pi_status pi_residual_rmsnorm(int32_t batch, int32_t d, pi_dtype htype, const void* h, const float* y, float eps,
+                              void* h_out, void* stream) {
+  if (batch < 1 || batch > PI_MAX_BATCH) return fail(PI_ERR_INVALID_ARG, "%s", "batch must be in [1, 16]");
+  if (d <= 0 || d % 8) return fail(PI_ERR_INVALID_ARG, "%s", "d must be a positive multiple of 8");
+  if (htype != PI_F32 && htype != PI_F16) return fail(PI_ERR_INVALID_ARG, "%s", "htype must be PI_F32 or PI_F16");
+  if (!(eps >= 0.f)) return fail(PI_ERR_INVALID_ARG, "%s", "eps must be >= 0");
+  PI_TRY(check_ptr(h, 16, "h"));
+  PI_TRY(check_ptr(y, 16, "y"));
+  PI_TRY(check_ptr(h_out, 16, "h_out"));
+  PI_CUDA(pi::launch_rmsnorm(htype, h, y, batch, d, eps, h_out, (cudaStream_t)stream), "rmsnorm launch");
+  return PI_OK;
+}
+
+pi_status pi_decode_stack(const pi_ffn_desc* desc, int32_t batch, int32_t n_layers, const pi_layer_weights* layers,
+                          const void* h_in, void* h_out, int32_t* idx, int32_t* counts, float* y, void* h_trace,
+                          float eps, void* ws, size_t ws_bytes, void* stream) {
+  PI_TRY(check_desc(desc, batch));
+  if (n_layers < 1 || n_layers > PI_MAX_LAYERS) return fail(PI_ERR_INVALID_ARG, "%s", "n_layers must be in [1, 128]");
+  if (h_trace) PI_TRY(check_ptr(h_trace, 16, "h_trace"));
+  if (!layers) return fail(PI_ERR_INVALID_ARG, "%s", "layers is NULL");
+  PI_TRY(check_ptr(h_in, 16, "h_in"));
+  PI_TRY(check_ptr(h_out, 16, "h_out"));
+  if (h_in == h_out) return fail(PI_ERR_INVALID_ARG, "%s", "h_out must not alias h_in");
+  PI_TRY(check_ptr(idx, 4, "idx"));
+  PI_TRY(check_ptr(counts, 4, "counts"));
+  if (y) PI_TRY(check_ptr(y, 16, "y"));
+  if (!(eps >= 0.f)) return fail(PI_ERR_INVALID_ARG, "%s", "eps must be >= 0");
+  PI_TRY(check_ws(desc, batch, ws, ws_bytes));
+  const pi::WsLayout L = pi::ws_layout(desc->d, desc->ffn, desc->n_hot, desc->rank, batch);
+  char* wsc = (char*)ws;
+  float* ybuf = reinterpret_cast<float*>(wsc + L.ybuf);
+  void* hbuf[2] = {h_out, wsc + L.hbuf};
+  const size_t C = (size_t)(desc->ffn - desc->n_hot);
+  cudaStream_t st = (cudaStream_t)stream;
+  // h_l ping-pongs between a workspace buffer and h_out so that the last layer lands in h_out.
+  const void* cur = h_in;
+  const size_t hbytes = (size_t)batch * desc->d * (desc->ptype == PI_F32 ? 4 : 2);
+  for (int l = 0; l < n_layers; ++l) {
+    if (h_trace) PI_CUDA(cudaMemcpyAsync((char*)h_trace + l * hbytes, cur, hbytes, cudaMemcpyDeviceToDevice, st),
+                         "h trace copy");
+    float* yl = y ? y + (size_t)l * batch * desc->d : ybuf;
+    PI_TRY(pi_layer(desc, batch, cur, &layers[l], idx + (size_t)l * C, counts + l, yl, ws, ws_bytes, stream));
+    void* nxt = hbuf[(n_layers - 1 - l) & 1];
+    PI_CUDA(pi::launch_rmsnorm(desc->ptype, cur, yl, batch, desc->d, eps, nxt, st), "rmsnorm launch");
+    cur = nxt;
+  }
+  return PI_OK;
+}
+
+int32_t pi_stack_launches(const pi_ffn_desc* desc, int32_t batch, int32_t n_layers) {
+  if (check_desc(desc, batch) != PI_OK || n_layers < 1 || n_layers > PI_MAX_LAYERS) return -1;
+  const int per_layer = desc->ffn > desc->n_hot ? 7 : 5;  // predictor (3 or 1 + memset), FFN (3), glue (1)
+  return per_layer * n_layers;
+}
+
+pi_status pi_get_device_status(void* ws, int32_t* status_out, int32_t clear, void* stream) {
+  PI_TRY(check_ptr(ws, 256, "ws"));
+  if (!status_out) return fail(PI_ERR_INVALID_ARG, "%s", "status_out is NULL");
+  cudaStream_t st = (cudaStream_t)stream;
+  int32_t v = 0;
+  PI_CUDA(cudaMemcpyAsync(&v, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, st), "status read");
+  PI_CUDA(cudaStreamSynchronize(st), "status read sync");
+  if (clear) {
+    PI_CUDA(cudaMemsetAsync(ws, 0, sizeof(int32_t), st), "status clear");
+    PI_CUDA(cudaStreamSynchronize(st), "status clear sync");
+  }
+  *status_out = v;
+  return PI_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,442 @@
+// pi_kernels_v1.cu -- the stand-alone kernels behind pi_predict, pi_sparse_ffn
+// and pi_residual_rmsnorm (sm_100a).  Each step is its own launch; the fused
+// multi-layer path lives in pi_stack.cu.
+//
+// Pages: unite.ai "PowerInfer: Tüketici Düzeyinde bir GPU ile Hızlı Büyük Dil
+// Modeli Sunucusu" -- "Adaptif Sparsite Predictor’ları" (predictor),
+// "Nöron Bilinçli Operatör" (row/column operators); GeekNews "Serving model
+// bahasa besar ...", "Keterbatasan dan FAQ" (ReLU, ReGLU, squared ReLU).
+#include "pi_common.cuh"
+#include "pi_kernels_v1.cuh"
+
+namespace pi {
+
+// ---------------------------------------------------------------------------
+// Predictor step 1: u[b,k] = max(0, P1[k,:] . h[b,:]), fp32.  One warp per row.
+template <int PT, int NB>
+__global__ void __launch_bounds__(256) k_pred_u(const void* __restrict__ P1, const void* __restrict__ h, int B, int d,
+                                                int r, float* __restrict__ u) {
+  constexpr int E = Unit<PT>::E;
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  const int units = d / E;
+  for (int k = gw; k < r; k += nw) {
+    for (int b0 = 0; b0 < B; b0 += NB) {
+      const int nb = min(NB, B - b0);
+      float acc[NB];
+#pragma unroll
+      for (int i = 0; i < NB; ++i) acc[i] = 0.f;
+      for (int un = lane; un < units; un += 32) {
+        float w[E];
+        load_w_unit<PT>(P1, nullptr, k, d, un, w);
+#pragma unroll
+        for (int i = 0; i < NB; ++i) {
+          if (i < nb) {
+            float x[E];
+            load_h_unit<PT, PT>(h, b0 + i, d, un, x);
+#pragma unroll
+            for (int e = 0; e < E; ++e) acc[i] = fmaf(w[e], x[e], acc[i]);
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < NB; ++i) acc[i] = warp_sum(acc[i]);
+      if (lane == 0) {
+        for (int i = 0; i < nb; ++i) u[(int64_t)(b0 + i) * r + k] = fmaxf(acc[i], 0.f);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Predictor step 2: scores of one tile of 256 cold neurons (8 warps x 32 rows),
+// s = P2[c,:] . u[b,:] + bp[c]; active = OR_b (s > thr).  Writes the tile's
+// 8 ballot words and its popcount.
+template <int PT, int NB>
+__global__ void __launch_bounds__(256) k_pred_score(const void* __restrict__ P2, const float* __restrict__ bp,
+                                                    const float* __restrict__ u, int B, int r, int C, float thr,
+                                                    uint32_t* __restrict__ tile_mask, int* __restrict__ tile_count) {
+  constexpr int E = Unit<PT>::E;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int units = r / E;
+  bool mine = false;
+  const int c_base = blockIdx.x * 256 + warp * 32;
+  for (int t = 0; t < 32; ++t) {
+    const int c = c_base + t;
+    if (c >= C) break;
+    const float bias = bp ? __ldg(bp + c) : 0.f;
+    bool on = false;
+    for (int b0 = 0; b0 < B; b0 += NB) {
+      const int nb = min(NB, B - b0);
+      float acc[NB];
+#pragma unroll
+      for (int i = 0; i < NB; ++i) acc[i] = 0.f;
+      for (int un = lane; un < units; un += 32) {
+        float w[E];
+        load_w_unit<PT>(P2, nullptr, c, r, un, w);
+#pragma unroll
+        for (int i = 0; i < NB; ++i) {
+          if (i < nb) {
+            float x[E];
+            load_h_unit<PT, kF32>(u, b0 + i, r, un, x);
+#pragma unroll
+            for (int e = 0; e < E; ++e) acc[i] = fmaf(w[e], x[e], acc[i]);
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < NB; ++i) {
+        const float s = warp_sum(acc[i]) + bias;
+        on |= (i < nb) && (s > thr);
+      }
+    }
+    if (lane == t) mine = on;
+  }
+  const unsigned m = __ballot_sync(0xffffffffu, mine);
+  __shared__ int cnt[8];
+  if (lane == 0) {
+    tile_mask[blockIdx.x * 8 + warp] = m;
+    cnt[warp] = __popc(m);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int s = 0;
+    for (int w = 0; w < 8; ++w) s += cnt[w];
+    tile_count[blockIdx.x] = s;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Order-preserving compaction: one CTA per tile.  Each CTA sums the counts of
+// the tiles before it (no inter-CTA waiting), then writes its tile's active
+// rows in ascending order.  CTA 0 also writes the total count.
+__global__ void __launch_bounds__(256) k_compact(const uint32_t* __restrict__ tile_mask,
+                                                 const int* __restrict__ tile_count, int n_tiles, int n_hot,
+                                                 int32_t* __restrict__ idx, int32_t* __restrict__ count) {
+  __shared__ int red[8];
+  __shared__ int wpre[9];
+  const int tile = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int before = 0, total = 0;
+  for (int t = threadIdx.x; t < n_tiles; t += blockDim.x) {
+    const int c = tile_count[t];
+    total += c;
+    if (t < tile) before += c;
+  }
+  // block reduce of `before` (and of `total` for CTA 0)
+  for (int o = 16; o > 0; o >>= 1) {
+    before += __shfl_xor_sync(0xffffffffu, before, o);
+    total += __shfl_xor_sync(0xffffffffu, total, o);
+  }
+  __shared__ int redt[8];
+  if (lane == 0) { red[warp] = before; redt[warp] = total; }
+  const uint32_t m = tile_mask[tile * 8 + warp];
+  if (threadIdx.x == 0) {
+    wpre[0] = 0;
+    for (int w = 0; w < 8; ++w) wpre[w + 1] = wpre[w] + __popc(tile_mask[tile * 8 + w]);
+  }
+  __syncthreads();
+  int base = 0, tot = 0;
+  for (int w = 0; w < 8; ++w) { base += red[w]; tot += redt[w]; }
+  if ((m >> lane) & 1u) {
+    const int pos = base + wpre[warp] + __popc(m & ((1u << lane) - 1u));
+    idx[pos] = n_hot + tile * 256 + warp * 32 + lane;
+  }
+  if (tile == 0 && threadIdx.x == 0) *count = tot;
+}
+
+// ---------------------------------------------------------------------------
+// Sparse FFN step 1: activation of every listed neuron, one warp per neuron.
+// list = [0, n_hot) ++ idx[0, count); a[b, p] for list position p.
+template <int WT, int HT, int ACT, int NB>
+__global__ void __launch_bounds__(256) k_ffn_act(const void* __restrict__ h, int B, int d, int ffn, int n_hot,
+                                                 const int32_t* __restrict__ idx, const int32_t* __restrict__ count,
+                                                 const void* __restrict__ wg, const void* __restrict__ wg_sc,
+                                                 const void* __restrict__ wu, const void* __restrict__ wu_sc,
+                                                 const float* __restrict__ b1, float* __restrict__ a, int n_max,
+                                                 int* __restrict__ status) {
+  constexpr int E = Unit<WT>::E;
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  const int n_cold = ffn - n_hot;
+  int cnt = *count;
+  if (cnt < 0 || cnt > n_cold) {
+    if (gw == 0 && lane == 0) set_status(status, kStCapacity);
+    cnt = cnt < 0 ? 0 : n_cold;
+  }
+  const int n = n_hot + cnt;
+  const int units = d / E;
+  for (int p = gw; p < n; p += nw) {
+    const int j = p < n_hot ? p : idx[p - n_hot];
+    if (j < n_hot || j >= ffn) {
+      if (lane == 0) set_status(status, kStIndex);
+      if (lane < B) a[(int64_t)lane * n_max + p] = 0.f;
+      continue;
+    }
+    const float bias = b1 ? __ldg(b1 + j) : 0.f;
+    for (int b0 = 0; b0 < B; b0 += NB) {
+      const int nb = min(NB, B - b0);
+      float g[NB], v[NB];
+#pragma unroll
+      for (int i = 0; i < NB; ++i) { g[i] = 0.f; v[i] = 0.f; }
+      for (int un = lane; un < units; un += 32) {
+        float wu_[E];
+        load_w_unit<WT>(wu, wu_sc, j, d, un, wu_);
+        float wg_[E];
+        if constexpr (ACT == kReglu) load_w_unit<WT>(wg, wg_sc, j, d, un, wg_);
+#pragma unroll
+        for (int i = 0; i < NB; ++i) {
+          if (i < nb) {
+            float x[E];
+            load_h_unit<WT, HT>(h, b0 + i, d, un, x);
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+              v[i] = fmaf(wu_[e], x[e], v[i]);
+              if constexpr (ACT == kReglu) g[i] = fmaf(wg_[e], x[e], g[i]);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < NB; ++i) {
+        v[i] = warp_sum(v[i]);
+        if constexpr (ACT == kReglu) g[i] = warp_sum(g[i]);
+      }
+      if (lane == 0) {
+        for (int i = 0; i < nb; ++i) {
+          float av;
+          if constexpr (ACT == kReglu) av = activation<ACT>(g[i] + bias, v[i]);
+          else av = activation<ACT>(v[i] + bias, 0.f);
+          a[(int64_t)(b0 + i) * n_max + p] = av;
+        }
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Sparse FFN step 2: down projection.  CTA c owns a contiguous, balanced range
+// of list positions and writes its fp32 partial y [B, d] (zeros for an empty
+// range).  Thread t owns the columns of units t, t + T, ... of the W_downT
+// rows (16 elements per thread per token group of NB tokens).
+template <int WT, int NB>
+__global__ void k_ffn_down(int B, int d, int ffn, int n_hot, const int32_t* __restrict__ idx,
+                           const int32_t* __restrict__ count, const void* __restrict__ wd,
+                           const void* __restrict__ wd_sc, const float* __restrict__ a, int n_max,
+                           float* __restrict__ partial) {
+  constexpr int E = Unit<WT>::E;
+  constexpr int UPT = 16 / E;  // units per thread
+  const int n_cold = ffn - n_hot;
+  int cnt = *count;
+  cnt = cnt < 0 ? 0 : (cnt > n_cold ? n_cold : cnt);
+  const int64_t n = n_hot + cnt;
+  const int64_t p0 = n * blockIdx.x / gridDim.x, p1 = n * (blockIdx.x + 1) / gridDim.x;
+  const int units = d / E;
+  float* out = partial + (int64_t)blockIdx.x * B * d;
+  for (int b0 = 0; b0 < B; b0 += NB) {
+    const int nb = min(NB, B - b0);
+    float acc[UPT][E][NB];
+#pragma unroll
+    for (int q = 0; q < UPT; ++q)
+#pragma unroll
+      for (int e = 0; e < E; ++e)
+#pragma unroll
+        for (int i = 0; i < NB; ++i) acc[q][e][i] = 0.f;
+    for (int64_t p = p0; p < p1; ++p) {
+      const int j = p < n_hot ? (int)p : idx[p - n_hot];
+      if (j < n_hot || j >= ffn) continue;  // flagged by k_ffn_act
+      float av[NB];
+#pragma unroll
+      for (int i = 0; i < NB; ++i) av[i] = (i < nb) ? a[(int64_t)(b0 + i) * n_max + p] : 0.f;
+#pragma unroll
+      for (int q = 0; q < UPT; ++q) {
+        const int un = threadIdx.x + q * blockDim.x;
+        if (un < units) {
+          float w[E];
+          load_w_unit<WT>(wd, wd_sc, j, d, un, w);
+#pragma unroll
+          for (int e = 0; e < E; ++e)
+#pragma unroll
+            for (int i = 0; i < NB; ++i) acc[q][e][i] = fmaf(av[i], w[e], acc[q][e][i]);
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < UPT; ++q) {
+      const int un = threadIdx.x + q * blockDim.x;
+      if (un < units) {
+#pragma unroll
+        for (int i = 0; i < NB; ++i) {
+          if (i < nb) {
+            float* o = out + (int64_t)(b0 + i) * d;
+#pragma unroll
+            for (int e = 0; e < E; ++e) o[unit_col<WT>(un, e)] = acc[q][e][i];
+          }
+        }
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Split-K reduction: y = b2 + sum_g partial[g] in a fixed order.  A CTA covers
+// 32 float4 columns x 8 partial groups; group k sums partials g = k mod 8 in
+// ascending order, then the 8 group sums are added in order.
+__global__ void __launch_bounds__(256) k_ffn_reduce(const float* __restrict__ partial, int G, int BD,
+                                                    const float* __restrict__ b2, int d, float* __restrict__ y) {
+  __shared__ float4 grp[8][32];
+  const int col4 = blockIdx.x * 32 + (threadIdx.x & 31);
+  const int k = threadIdx.x >> 5;
+  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (col4 * 4 < BD) {
+    for (int g = k; g < G; g += 8) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(partial + (int64_t)g * BD) + col4);
+      s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+    }
+  }
+  grp[k][threadIdx.x & 31] = s;
+  __syncthreads();
+  if (k == 0 && col4 * 4 < BD) {
+    float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (b2) {
+      const int e = (col4 * 4) % d;
+      t = *reinterpret_cast<const float4*>(b2 + e);
+    }
+    for (int q = 0; q < 8; ++q) {
+      const float4 v = grp[q][threadIdx.x];
+      t.x += v.x; t.y += v.y; t.z += v.z; t.w += v.w;
+    }
+    reinterpret_cast<float4*>(y)[col4] = t;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Stack glue: x = h + y; h_out = x * rsqrt(mean(x^2) + eps).  One CTA per token.
+template <int HT>
+__global__ void __launch_bounds__(256) k_rmsnorm(const void* __restrict__ h, const float* __restrict__ y, int d,
+                                                 float eps, void* __restrict__ h_out) {
+  const int b = blockIdx.x;
+  __shared__ float red[8];
+  float ss = 0.f;
+  for (int e = threadIdx.x; e < d; e += blockDim.x) {
+    float hv;
+    if constexpr (HT == kF32) hv = reinterpret_cast<const float*>(h)[(int64_t)b * d + e];
+    else hv = __half2float(reinterpret_cast<const __half*>(h)[(int64_t)b * d + e]);
+    const float x = hv + y[(int64_t)b * d + e];
+    ss = fmaf(x, x, ss);
+  }
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += red[w];
+  const float inv = rsqrtf(tot / (float)d + eps);
+  __syncthreads();
+  for (int e = threadIdx.x; e < d; e += blockDim.x) {
+    float hv;
+    if constexpr (HT == kF32) hv = reinterpret_cast<const float*>(h)[(int64_t)b * d + e];
+    else hv = __half2float(reinterpret_cast<const __half*>(h)[(int64_t)b * d + e]);
+    const float x = (hv + y[(int64_t)b * d + e]) * inv;
+    if constexpr (HT == kF32) reinterpret_cast<float*>(h_out)[(int64_t)b * d + e] = x;
+    else reinterpret_cast<__half*>(h_out)[(int64_t)b * d + e] = __float2half_rn(x);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Launchers (dtype dispatch).
+
+constexpr int kNB = 4;  // tokens per pass in the CUDA-core kernels
+
+cudaError_t launch_pred_u(int ptype, const void* P1, const void* h, int B, int d, int r, float* u, int sms,
+                          cudaStream_t st) {
+  const int grid = min((r + 7) / 8, sms * 8);
+  if (ptype == kF32) k_pred_u<kF32, kNB><<<grid, 256, 0, st>>>(P1, h, B, d, r, u);
+  else k_pred_u<kF16, kNB><<<grid, 256, 0, st>>>(P1, h, B, d, r, u);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pred_score(int ptype, const void* P2, const float* bp, const float* u, int B, int r, int C,
+                              float thr, uint32_t* tile_mask, int* tile_count, cudaStream_t st) {
+  const int tiles = (C + 255) / 256;
+  if (tiles == 0) return cudaSuccess;
+  if (ptype == kF32) k_pred_score<kF32, kNB><<<tiles, 256, 0, st>>>(P2, bp, u, B, r, C, thr, tile_mask, tile_count);
+  else k_pred_score<kF16, kNB><<<tiles, 256, 0, st>>>(P2, bp, u, B, r, C, thr, tile_mask, tile_count);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_compact(const uint32_t* tile_mask, const int* tile_count, int C, int n_hot, int32_t* idx,
+                           int32_t* count, cudaStream_t st) {
+  const int tiles = (C + 255) / 256;
+  if (tiles == 0) return cudaMemsetAsync(count, 0, sizeof(int32_t), st);
+  k_compact<<<tiles, 256, 0, st>>>(tile_mask, tile_count, tiles, n_hot, idx, count);
+  return cudaGetLastError();
+}
+
+template <int WT, int HT>
+static void act_dispatch(int act, int grid, cudaStream_t st, const void* h, int B, int d, int ffn, int n_hot,
+                         const int32_t* idx, const int32_t* count, const void* wg, const void* wg_sc, const void* wu,
+                         const void* wu_sc, const float* b1, float* a, int n_max, int* status) {
+  if (act == kReglu)
+    k_ffn_act<WT, HT, kReglu, kNB><<<grid, 256, 0, st>>>(h, B, d, ffn, n_hot, idx, count, wg, wg_sc, wu, wu_sc, b1,
+                                                         a, n_max, status);
+  else if (act == kRelu2)
+    k_ffn_act<WT, HT, kRelu2, kNB><<<grid, 256, 0, st>>>(h, B, d, ffn, n_hot, idx, count, wg, wg_sc, wu, wu_sc, b1,
+                                                         a, n_max, status);
+  else
+    k_ffn_act<WT, HT, kRelu, kNB><<<grid, 256, 0, st>>>(h, B, d, ffn, n_hot, idx, count, wg, wg_sc, wu, wu_sc, b1,
+                                                        a, n_max, status);
+}
+
+cudaError_t launch_ffn_act(int wtype, int htype, int act, const void* h, int B, int d, int ffn, int n_hot,
+                           const int32_t* idx, const int32_t* count, const void* wg, const void* wg_sc,
+                           const void* wu, const void* wu_sc, const float* b1, float* a, int n_max, int* status,
+                           int sms, cudaStream_t st) {
+  const int grid = sms * 8;
+  if (htype == kF32) {
+    if (wtype == kF32) act_dispatch<kF32, kF32>(act, grid, st, h, B, d, ffn, n_hot, idx, count, wg, wg_sc, wu, wu_sc, b1, a, n_max, status);
+    else if (wtype == kF16) act_dispatch<kF16, kF32>(act, grid, st, h, B, d, ffn, n_hot, idx, count, wg, wg_sc, wu, wu_sc, b1, a, n_max, status);
+    else act_dispatch<kQ4_0, kF32>(act, grid, st, h, B, d, ffn, n_hot, idx, count, wg, wg_sc, wu, wu_sc, b1, a, n_max, status);
+  } else {
+    if (wtype == kF32) act_dispatch<kF32, kF16>(act, grid, st, h, B, d, ffn, n_hot, idx, count, wg, wg_sc, wu, wu_sc, b1, a, n_max, status);
+    else if (wtype == kF16) act_dispatch<kF16, kF16>(act, grid, st, h, B, d, ffn, n_hot, idx, count, wg, wg_sc, wu, wu_sc, b1, a, n_max, status);
+    else act_dispatch<kQ4_0, kF16>(act, grid, st, h, B, d, ffn, n_hot, idx, count, wg, wg_sc, wu, wu_sc, b1, a, n_max, status);
+  }
+  return cudaGetLastError();
+}
+
+int down_threads(int wtype, int d) {
+  const int e = wtype == kF32 ? 4 : (wtype == kF16 ? 8 : 16);
+  const int units = d / e;
+  const int upt = 16 / e;
+  int t = (units + upt - 1) / upt;
+  t = (t + 31) / 32 * 32;
+  return t < 32 ? 32 : t;
+}
+
+cudaError_t launch_ffn_down(int wtype, int B, int d, int ffn, int n_hot, const int32_t* idx, const int32_t* count,
+                            const void* wd, const void* wd_sc, const float* a, int n_max, float* partial, int G,
+                            cudaStream_t st) {
+  const int T = down_threads(wtype, d);
+  if (T > 1024) return cudaErrorInvalidValue;
+  if (wtype == kF32) k_ffn_down<kF32, kNB><<<G, T, 0, st>>>(B, d, ffn, n_hot, idx, count, wd, wd_sc, a, n_max, partial);
+  else if (wtype == kF16) k_ffn_down<kF16, kNB><<<G, T, 0, st>>>(B, d, ffn, n_hot, idx, count, wd, wd_sc, a, n_max, partial);
+  else k_ffn_down<kQ4_0, kNB><<<G, T, 0, st>>>(B, d, ffn, n_hot, idx, count, wd, wd_sc, a, n_max, partial);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ffn_reduce(const float* partial, int G, int B, int d, const float* b2, float* y, cudaStream_t st) {
+  const int BD = B * d;
+  const int grid = (BD / 4 + 31) / 32;
+  k_ffn_reduce<<<grid, 256, 0, st>>>(partial, G, BD, b2, d, y);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rmsnorm(int htype, const void* h, const float* y, int B, int d, float eps, void* h_out,
+                           cudaStream_t st) {
+  if (htype == kF32) k_rmsnorm<kF32><<<B, 256, 0, st>>>(h, y, d, eps, h_out);
+  else k_rmsnorm<kF16><<<B, 256, 0, st>>>(h, y, d, eps, h_out);
+  return cudaGetLastError();
+}
+
+}  // namespace pi

@@ -1,0 +1,27 @@
+// pi_kernels_v1.cuh -- launchers of the stand-alone libpi kernels.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace pi {
+
+cudaError_t launch_pred_u(int ptype, const void* P1, const void* h, int B, int d, int r, float* u, int sms,
+                          cudaStream_t st);
+cudaError_t launch_pred_score(int ptype, const void* P2, const float* bp, const float* u, int B, int r, int C,
+                              float thr, uint32_t* tile_mask, int* tile_count, cudaStream_t st);
+cudaError_t launch_compact(const uint32_t* tile_mask, const int* tile_count, int C, int n_hot, int32_t* idx,
+                           int32_t* count, cudaStream_t st);
+cudaError_t launch_ffn_act(int wtype, int htype, int act, const void* h, int B, int d, int ffn, int n_hot,
+                           const int32_t* idx, const int32_t* count, const void* wg, const void* wg_sc,
+                           const void* wu, const void* wu_sc, const float* b1, float* a, int n_max, int* status,
+                           int sms, cudaStream_t st);
+int down_threads(int wtype, int d);
+cudaError_t launch_ffn_down(int wtype, int B, int d, int ffn, int n_hot, const int32_t* idx, const int32_t* count,
+                            const void* wd, const void* wd_sc, const float* a, int n_max, float* partial, int G,
+                            cudaStream_t st);
+cudaError_t launch_ffn_reduce(const float* partial, int G, int B, int d, const float* b2, float* y,
+                              cudaStream_t st);
+cudaError_t launch_rmsnorm(int htype, const void* h, const float* y, int B, int d, float eps, void* h_out,
+                           cudaStream_t st);
+
+}  // namespace pi

@@ -1,0 +1,40 @@
+// pi_layout.h -- byte layout of a libpi workspace (host side).
+//
+//   [ctrl 256 B][u: B x rank fp32][tile masks][tile counts][a: B x ffn fp32]
+//   [partials: G_MAX x B x d fp32][y: B x d fp32][h: B x d fp32]
+//
+// Every region starts on a 256-byte boundary.  The layout depends only on the
+// descriptor and the batch, never on the device.
+#pragma once
+#include <stddef.h>
+#include <stdint.h>
+
+namespace pi {
+
+constexpr int kGMax = 296;  // split-K partial slots (2 x 148 SMs)
+
+struct WsLayout {
+  size_t u, tile_mask, tile_count, act, partial, ybuf, hbuf, total;
+  int n_tiles, g_max;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+inline WsLayout ws_layout(int d, int ffn, int n_hot, int rank, int B) {
+  WsLayout L;
+  size_t off = 256;
+  const int C = ffn - n_hot;
+  L.n_tiles = (C + 255) / 256;
+  L.g_max = kGMax;
+  L.u = off; off += align256((size_t)B * rank * 4);
+  L.tile_mask = off; off += align256((size_t)(L.n_tiles > 0 ? L.n_tiles : 1) * 8 * 4);
+  L.tile_count = off; off += align256((size_t)(L.n_tiles > 0 ? L.n_tiles : 1) * 4);
+  L.act = off; off += align256((size_t)B * ffn * 4);
+  L.partial = off; off += align256((size_t)kGMax * B * d * 4);
+  L.ybuf = off; off += align256((size_t)B * d * 4);
+  L.hbuf = off; off += align256((size_t)B * d * 4);
+  L.total = off;
+  return L;
+}
+
+}  // namespace pi

@@ -1,0 +1,417 @@
+"""Benchmark: sparse-FFN decode tokens/s through the whole layer stack on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--batch B]
+                    [--sparsity S] [--impl ours|reference] [--no-cpu-baseline]
+
+A step is one decode step of one token block through every layer of the
+workload: predictor, compaction, hot block, sparse up/gate + activation,
+sparse down, split-K reduction and the residual+RMSNorm glue, all in libpi's
+kernels.  Inputs (weights for every layer, the token blocks) are synthetic and
+seeded (pi_workload) and resident in HBM before timing starts; the resident
+stack is far larger than L2, and each step streams every layer's predictor and
+active rows, so no L2 flush is needed between steps.
+
+Prints ONE JSON line (rank 0).  With N > 1 (torchrun) every rank runs an
+independent replica (the path has no exchange step): weak scaling, time = max
+over ranks of the device-timed region.
+
+--impl reference times the CPU oracle (the only other implementation of this
+path) on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import pi_workload as W  # noqa: E402
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+POOL = 64         # distinct token blocks (one captured graph each), cycled over the timed steps
+E2E_STEPS = 200   # steps of the end-to-end (host buffers) measurement
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="7b-reglu-fp16", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--batch", type=int, default=None)
+    ap.add_argument("--sparsity", type=float, default=None)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=None, help="run fewer layers (smoke only; not a bench number)")
+    return ap.parse_args()
+
+
+def peak_hbm():
+    try:
+        with open(PEAKS_FILE) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.QUERY,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return None
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------
+# our arm
+
+
+def run_ours(args, rank, world, local_rank):
+    import activation_sparse_decode_predict_b200 as pi
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = W.WORKLOADS[args.workload]
+    if args.sparsity is not None:
+        wl = wl.with_(sparsity=args.sparsity)
+    B = args.batch or wl.batches[0]
+    n_layers = args.layers or wl.layers
+    desc = pi.desc_for(wl)
+
+    layers = [W.make_layer(wl, l, device=dev) for l in range(n_layers)]
+    torch.cuda.synchronize()
+    arr = pi.layer_array([pi.layer_weights(L) for L in layers])
+    n_steps = args.warmup + args.steps
+    P = min(POOL, n_steps)                    # distinct token blocks, cycled
+    h_pool = torch.stack([W.make_tokens(wl, B, rank * 100003 + t, device=dev) for t in range(P)])
+    ws = pi.workspace(desc, B, device=dev)
+    C = wl.n_cold
+    idx = torch.empty(n_layers, max(C, 1), dtype=torch.int32, device=dev)
+    counts = torch.zeros(P, n_layers, dtype=torch.int32, device=dev)
+    h_out = torch.empty(B, wl.d, dtype=h_pool.dtype, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(p, s):
+        pi.decode_stack(desc, arr, h_pool[p], h_out, idx, counts[p], None, W.RMS_EPS, ws, stream=s)
+
+    # one CUDA graph per token block; captured before timing
+    graphs = []
+    with torch.cuda.stream(stream):
+        step(0, stream)                       # warm the code path once outside capture
+        stream.synchronize()
+        for p in range(P):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step(p, stream)
+            graphs.append(g)
+    torch.cuda.synchronize()
+
+    for t in range(args.warmup):
+        graphs[t % P].replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        with torch.cuda.stream(stream):
+            torch.cuda.synchronize()
+            ev0.record(stream)
+            for t in range(args.warmup, n_steps):
+                graphs[t % P].replay()
+            ev1.record(stream)
+            torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1)
+    clocks = clk.summary()
+    if world > 1:
+        t_ = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t_, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t_.item())
+        torch.distributed.barrier()
+    status = pi.device_status(ws)
+
+    # measured active counts of the timed steps -> algorithmic bytes
+    cnt_p = counts.double().cpu().numpy()
+    cnt = np.stack([cnt_p[t % P] for t in range(args.warmup, n_steps)])
+    per_block = [sum(W.layer_bytes(wl, B, float(a)) for a in cnt_p[p]) for p in range(P)]
+    total_bytes = sum(per_block[t % P] for t in range(args.warmup, n_steps))
+    sec = ms / 1e3
+    gbs = total_bytes / sec / 1e9
+    peak, peak_kind = peak_hbm()
+    tok_s = world * B * args.steps / sec
+
+    # end to end through the public API with host buffers: H2D of the step's
+    # token block from pinned memory, the stack call, D2H of the result.
+    h_host = h_pool.cpu().pin_memory()
+    out_host = torch.empty(B, wl.d, dtype=h_pool.dtype).pin_memory()
+    h_dev_in = torch.empty(B, wl.d, dtype=h_pool.dtype, device=dev)
+    e_steps = min(args.steps, E2E_STEPS)
+    e_cnt = torch.zeros(n_layers, dtype=torch.int32, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for t in range(args.warmup):
+            h_dev_in.copy_(h_host[t % P], non_blocking=True)
+            pi.decode_stack(desc, arr, h_dev_in, h_out, idx, e_cnt, None, W.RMS_EPS, ws, stream=stream)
+            out_host.copy_(h_out, non_blocking=True)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        e0.record(stream)
+        for t in range(e_steps):
+            h_dev_in.copy_(h_host[t % P], non_blocking=True)
+            pi.decode_stack(desc, arr, h_dev_in, h_out, idx, e_cnt, None, W.RMS_EPS, ws, stream=stream)
+            out_host.copy_(h_out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t_ = torch.tensor([e_ms], device=dev)
+        torch.distributed.all_reduce(t_, op=torch.distributed.ReduceOp.MAX)
+        e_ms = float(t_.item())
+    e2e_tok_s = world * B * e_steps / (e_ms / 1e3)
+    hb = B * wl.d * h_pool.element_size()
+
+    launches_per_step = pi.stack_launches(desc, B, n_layers)
+    out = {
+        "metric": "sparse-FFN decode tokens/s",
+        "value": round(tok_s, 3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16" if wl.wtype == "f16" else wl.wtype,
+        "data": "synthetic (seeded Zipf-activity weights, low-rank predictor, RMS-normalised tokens)",
+        "config": {"workload": wl.name, "d": wl.d, "ffn": wl.ffn, "layers": n_layers, "batch": B,
+                   "sparsity": wl.sparsity, "hot": wl.n_hot, "rank": wl.rank, "act": wl.act, "weights": wl.wtype,
+                   "parallelism": "replicas" if world > 1 else "single",
+                   "l2": "no flush: resident stack %.1f GB, %.2f GB streamed per step (L2 126 MB)" % (
+                       _resident_bytes(layers) / 1e9, total_bytes / args.steps / 1e9),
+                   "mean_active_cold": round(float(cnt.mean()), 1)},
+        "gb_per_s": round(gbs, 1),
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(gbs / peak, 4), "traffic": None,
+                     "kernel": "whole decode step (%d launches)" % launches_per_step,
+                     "peak_source": peak_kind},
+        "e2e": {"value": round(e2e_tok_s, 3), "unit": "tokens/s", "h2d_bytes_per_step": hb, "d2h_bytes_per_step": hb,
+                "steps": e_steps, "how": "pinned H2D of the token block, pi_decode_stack via the binding, D2H of h_out"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "device_status": status,
+    }
+    return out, (wl, B, layers, n_layers)
+
+
+def _resident_bytes(layers):
+    n = 0
+    for L in layers:
+        for k in ("Wg", "Wu", "WdT", "P1", "P2", "bp", "b1"):
+            v = L.get(k)
+            if v is None:
+                continue
+            for t in (v if isinstance(v, tuple) else (v,)):
+                n += t.numel() * t.element_size()
+    return n
+
+
+# ----------------------------------------------------------------------------
+# the CPU oracle on the host cores
+
+
+def _host_layers(layers):
+    host = []
+    for L in layers:
+        Ln = {}
+        for k in ("Wg", "Wu", "WdT", "P1", "P2", "bp", "b1", "b2"):
+            v = L.get(k)
+            if isinstance(v, tuple):
+                Ln[k] = tuple(np.ascontiguousarray(t.cpu().numpy()) for t in v)
+            elif v is not None:
+                Ln[k] = np.ascontiguousarray(v.cpu().numpy())
+            else:
+                Ln[k] = None
+        Ln["thr"] = L["thr"]
+        host.append(Ln)
+    return host
+
+
+def _oracle_layer_step(wl, B, Ln, step):
+    import oracle
+    h = W.make_tokens(wl, B, 7_000_000 + step).numpy()
+    r = oracle.predict(h, Ln["P1"], Ln["P2"], Ln["bp"], Ln["thr"], wl.n_hot, wl.ffn)
+    y = oracle.masked_ffn(h, r["idx"], Ln["Wg"], Ln["Wu"], Ln["WdT"], Ln["b1"], Ln["b2"], wl.act, wl.n_hot, wl.ffn)
+    return oracle.residual_rmsnorm(h, y, W.RMS_EPS)
+
+
+def oracle_sample(wl, B, layers, n_sample_layers, n_steps, threads=None):
+    """Time the oracle (predictor + masked FFN + glue) on the first layers of
+    the stack for a few token blocks; returns (tokens/s scaled to the full
+    stack, seconds spent, threads used, description)."""
+    import oracle
+    if threads:
+        oracle.set_threads(threads)
+    host = _host_layers(layers[:n_sample_layers])
+    t0 = time.perf_counter()
+    for s in range(n_steps):
+        h = W.make_tokens(wl, B, 7_000_000 + s).numpy()
+        for Ln in host:
+            r = oracle.predict(h, Ln["P1"], Ln["P2"], Ln["bp"], Ln["thr"], wl.n_hot, wl.ffn)
+            y = oracle.masked_ffn(h, r["idx"], Ln["Wg"], Ln["Wu"], Ln["WdT"], Ln["b1"], Ln["b2"], wl.act, wl.n_hot,
+                                  wl.ffn)
+            hn = oracle.residual_rmsnorm(h, y, W.RMS_EPS)
+            h = hn.astype(h.dtype)
+    dt = time.perf_counter() - t0
+    n_layers = wl.layers
+    tok_s = n_steps * B / (dt * n_layers / n_sample_layers)
+    desc = "%d decode steps x %d of %d layers (B=%d), scaled by %d/%d (extrapolated)" % (
+        n_steps, n_sample_layers, n_layers, B, n_layers, n_sample_layers)
+    return tok_s, dt, oracle.get_threads(), desc
+
+
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle, as it stands, on the host cores."""
+    wl = W.WORKLOADS[args.workload]
+    if args.sparsity is not None:
+        wl = wl.with_(sparsity=args.sparsity)
+    B = args.batch or wl.batches[0]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    n_sample = 2
+    layers = [W.make_layer(wl, l, device=dev) for l in range(n_sample)]
+    import oracle
+    oracle.set_threads(os.cpu_count() or 1)
+    # Each reference step is one token block through ONE layer of the stack (the
+    # sampled layers taken in turn); tokens/s is scaled to the full stack.
+    host = _host_layers(layers)
+    for t in range(args.warmup):
+        _oracle_layer_step(wl, B, host[t % n_sample], t)
+    t0 = time.perf_counter()
+    for t in range(args.steps):
+        _oracle_layer_step(wl, B, host[t % n_sample], 1000 + t)
+    dt = time.perf_counter() - t0
+    tok_s = args.steps * B / (dt * wl.layers)
+    cores = oracle.get_threads()
+    desc = "%d steps of one token block (B=%d) through one of %d sampled layers, scaled by %d layers (extrapolated)" % (
+        args.steps, B, n_sample, wl.layers)
+    ms = dt * 1e3 / args.steps * wl.layers
+    return {
+        "impl": "reference",
+        "metric": "sparse-FFN decode tokens/s",
+        "value": round(tok_s, 4),
+        "unit": "tokens/s",
+        "n_gpus": 1,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded Zipf-activity weights, low-rank predictor, RMS-normalised tokens)",
+        "config": {"workload": wl.name, "d": wl.d, "ffn": wl.ffn, "layers": wl.layers, "batch": B,
+                   "sparsity": wl.sparsity},
+        "cpu_baseline": {"value": round(tok_s, 4), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": desc, "cpu": cpu_model()},
+        "e2e": {"value": round(tok_s, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    out, ctx = run_ours(args, rank, world, local_rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        wl, B, layers, _ = ctx
+        n_s = 2 if wl.d * wl.ffn <= 64e6 else 1
+        steps = 4 if wl.d * wl.ffn <= 64e6 else 2
+        tok_s, dt, cores, desc = oracle_sample(wl, B, layers, n_s, steps, threads=os.cpu_count())
+        out["cpu_baseline"] = {"value": round(tok_s, 4), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                               "sample": desc, "cpu": cpu_model(), "seconds": round(dt, 2)}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,239 @@
+/*
+ * pi.h -- C ABI of libpi: the activation-sparse decode FFN on one NVIDIA B200.
+ *
+ * The operation is the per-layer hot path of predictor-driven activation
+ * sparsity as the PowerInfer pages describe it:
+ *
+ *   [GN] GeekNews, "Serving model bahasa besar berkecepatan tinggi pada PC
+ *        dengan GPU konsumen"
+ *   [AB] aibars.net, "PowerInfer - Hochgeschwindigkeits-Inferenz-Engine für
+ *        große Sprachmodelle"
+ *   [UA] unite.ai, "PowerInfer: Tüketici Düzeyinde bir GPU ile Hızlı Büyük
+ *        Dil Modeli Sunucusu"
+ *
+ * A small per-layer predictor picks the FFN neurons that will fire ([UA]
+ * "Adaptif Sparsite Predictor’ları"); neuron-aware operators then read and
+ * compute only those rows of W_gate / W_up and columns of W_down ([UA] "Nöron
+ * Bilinçli Operatör"); the always-hot neurons, stored first by the offline
+ * layout ([UA] "Nöron Yerleştirme ve Yönetimi"; [AB] "Hot-Cold-Neuron-
+ * Mechanismus"), are always computed as one dense slice.
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ * - Every tensor pointer is a DEVICE pointer, owned by the caller, 16-byte
+ *   aligned, with dense row-major strides.  The library allocates nothing and
+ *   keeps no global state; all scratch lives in the caller's workspace `ws`.
+ * - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *   stream).  Calls are asynchronous and ordered on that stream.
+ * - Errors the host can see (bad descriptor, NULL or misaligned pointer,
+ *   workspace too small, unsupported shape) are returned synchronously and
+ *   nothing is launched.  A launch failure returns PI_ERR_CUDA.  Errors found
+ *   on the device (an index outside [n_hot, ffn), a count above capacity, a
+ *   bounded wait that ran out) set a sticky word in `ws`; read it with
+ *   pi_get_device_status().  The kernels never trap.
+ * - Calls are reentrant when they use different workspaces.  Calls that share
+ *   a workspace must be ordered (same stream, or synchronised).
+ * - Storage order is hot-first: neuron rows [0, n_hot) are the hot neurons,
+ *   rows [n_hot, ffn) the cold ones.  The neuron table that maps storage rows
+ *   back to the model's original rows stays with the caller.
+ *
+ * Layouts (d = hidden size, F = ffn, H = n_hot, C = F - H, r = rank, B = batch)
+ *   h        [B, d]   token block, element type `ptype` (F32 or F16)
+ *   P1       [r, d]   predictor first matrix, `ptype`
+ *   P2       [C, r]   predictor second matrix (cold neurons only), `ptype`
+ *   bp       [C]      fp32 predictor bias, may be NULL
+ *   W_gate   [F, d]   gate rows (ReGLU only), `wtype`
+ *   W_up     [F, d]   up rows, `wtype`
+ *   W_downT  [F, d]   W_down stored neuron-major (row j = column j of W_down)
+ *   b1       [F]      fp32 bias of the gate (ReGLU) or of the up projection,
+ *                     may be NULL
+ *   b2       [d]      fp32 output bias, may be NULL
+ *   y        [B, d]   fp32 output
+ *   idx      [C]      int32 active-neuron list, ascending storage rows in
+ *                     [H, F); its length lives in the device scalar `count`
+ *   Q4_0 weights use split planes: data = qs [F, d/2] uint8, scales =
+ *   sc [F, d/32] fp16; in each 32-element block, byte k holds element k in
+ *   its low nibble and element k + 16 in its high nibble, x = s * (q - 8)
+ *   ([GN] "Kuantisasi dan kompatibilitas": INT4 Q4_0).
+ */
+#ifndef PI_H_
+#define PI_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PI_API __attribute__((visibility("default")))
+#else
+#define PI_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PI_OK = 0,
+  PI_ERR_INVALID_ARG = -1,  /* bad descriptor, NULL/misaligned pointer, bad size */
+  PI_ERR_UNSUPPORTED = -2,  /* valid but not implemented (shape/dtype combination) */
+  PI_ERR_CUDA = -3,         /* a CUDA call failed; see pi_last_error() */
+  PI_ERR_CAPACITY = -4,     /* workspace too small, or a device count above capacity */
+  PI_ERR_TIMEOUT = -5,      /* a bounded device-side wait ran out */
+  PI_ERR_INDEX = -6         /* device found an active index outside [n_hot, ffn) */
+} pi_status;
+
+typedef enum { PI_F32 = 0, PI_F16 = 1, PI_Q4_0 = 2 } pi_dtype;
+
+/* [GN] "Keterbatasan dan FAQ": the supported activation families. */
+typedef enum {
+  PI_ACT_RELU = 0,   /* a = max(W_up h + b1, 0)                      */
+  PI_ACT_REGLU = 1,  /* a = max(W_gate h + b1, 0) * (W_up h)          */
+  PI_ACT_RELU2 = 2   /* a = max(W_up h + b1, 0)^2  (not gated)         */
+} pi_act;
+
+/* Shape and types of one FFN layer. */
+typedef struct {
+  int32_t d;       /* hidden size; multiple of 8 (Q4_0: of 32)            */
+  int32_t ffn;     /* neurons per layer                                   */
+  int32_t n_hot;   /* hot neurons, rows [0, n_hot); 0 <= n_hot <= ffn     */
+  int32_t rank;    /* predictor rank; multiple of 8                       */
+  pi_dtype wtype;  /* FFN weights: PI_F32, PI_F16 or PI_Q4_0             */
+  pi_dtype ptype;  /* predictor matrices and the token block: F32 or F16 */
+  pi_act act;
+} pi_ffn_desc;
+
+/* One weight matrix: `data` (fp32/fp16 rows, or Q4_0 qs), `scales` (Q4_0 sc, else NULL). */
+typedef struct {
+  const void *data;
+  const void *scales;
+} pi_weight;
+
+/* All per-layer tensors of one layer (device pointers). */
+typedef struct {
+  const void *P1;
+  const void *P2;
+  const float *bp;
+  pi_weight W_gate;   /* ignored unless act == PI_ACT_REGLU */
+  pi_weight W_up;
+  pi_weight W_downT;
+  const float *b1;
+  const float *b2;
+  float threshold;    /* predictor threshold: neuron c is active iff its score > threshold */
+  int32_t _pad;
+} pi_layer_weights;
+
+/* Maximum token-block size accepted by every call. */
+#define PI_MAX_BATCH 16
+/* Maximum number of layers of one pi_decode_stack call. */
+#define PI_MAX_LAYERS 128
+
+/*
+ * Bytes of device workspace a call with this descriptor and batch needs
+ * (the largest over pi_predict, pi_sparse_ffn, pi_layer and pi_decode_stack).
+ * Returns 0 for an invalid descriptor.  The workspace must be zeroed once
+ * (pi_workspace_init) before its first use; the library keeps it consistent
+ * afterwards.
+ */
+PI_API size_t pi_workspace_bytes(const pi_ffn_desc *desc, int32_t batch);
+
+/* Zero the workspace's control block (status word and counters), on `stream`. */
+PI_API pi_status pi_workspace_init(void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * pi_predict -- which cold neurons will fire ([UA] "Adaptif Sparsite
+ * Predictor’ları": a per-layer predictor; only predicted-active neurons are
+ * computed; [UA] "Çevrim İçi Aşama": the engine predicts active neurons and
+ * skips the rest).  The pages do not state the predictor's form; this call
+ * computes the low-rank reading
+ *     u[b,k] = max(0, sum_i P1[k,i] h[b,i])          (fp32 accumulation)
+ *     s[b,c] = sum_k P2[c,k] u[b,k] + bp[c]
+ *     active(c) = OR over b of (s[b,c] > threshold)
+ * and writes idx = ascending { n_hot + c : active(c) } and *count = |idx|.
+ * Hot neurons are not scored: they are always computed.
+ *   h [B, d] ptype; P1 [r, d]; P2 [C, r]; bp [C] or NULL;
+ *   idx: device int32 [C] (capacity C); count: device int32 scalar.
+ * The list is identical to an exact evaluation except for neurons whose
+ * score is within rounding (well under 1e-3) of the threshold.
+ */
+PI_API pi_status pi_predict(const pi_ffn_desc *desc, int32_t batch, const void *h, const void *P1, const void *P2,
+                     const float *bp, float threshold, int32_t *idx, int32_t *count, void *ws, size_t ws_bytes,
+                     void *stream);
+
+/*
+ * pi_sparse_ffn -- the neuron-aware sparse FFN over the list
+ * [0, n_hot) ++ idx[0, *count) ([UA] "Nöron Bilinçli Operatör": single rows
+ * of the up/gate matrices and single columns of the down matrix, no dense
+ * conversion at run time; [GN] "Metode inferensi hibrida CPU/GPU": the dense
+ * always-active block runs on the GPU):
+ *     for each listed neuron j and token b:
+ *         ReGLU:  a = max(W_gate[j].h_b + b1[j], 0) * (W_up[j].h_b)
+ *         ReLU:   a = max(W_up[j].h_b + b1[j], 0)
+ *         ReLU^2: a = max(W_up[j].h_b + b1[j], 0)^2
+ *     y[b, :] = b2 + sum over listed j of a * W_downT[j, :]
+ * Every token of the block uses the same list (the union mask).  Dots and the
+ * output accumulate in fp32; the activation is never rounded below fp32.
+ * `count` is read on the device (no host synchronisation); an index outside
+ * [n_hot, ffn) or a count above C sets PI_ERR_INDEX / PI_ERR_CAPACITY in the
+ * status word and is skipped.
+ */
+PI_API pi_status pi_sparse_ffn(const pi_ffn_desc *desc, int32_t batch, const void *h, const int32_t *idx,
+                        const int32_t *count, pi_weight W_gate, pi_weight W_up, pi_weight W_downT, const float *b1,
+                        const float *b2, float *y, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * pi_layer -- pi_predict followed by pi_sparse_ffn on the same token block
+ * (one decode step of one FFN layer).  Writes idx/count and y exactly as the
+ * two calls would.
+ */
+PI_API pi_status pi_layer(const pi_ffn_desc *desc, int32_t batch, const void *h, const pi_layer_weights *w, int32_t *idx,
+                   int32_t *count, float *y, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * pi_residual_rmsnorm -- glue between stacked FFN layers (the pages do not
+ * say what joins the layers; this is the plainest reading that keeps the
+ * token statistics fixed): x = h + y;  h_out = x / sqrt(mean(x^2) + eps),
+ * computed in fp32 and stored in `htype` (F32 or F16).  h_out may alias h.
+ */
+PI_API pi_status pi_residual_rmsnorm(int32_t batch, int32_t d, pi_dtype htype, const void *h, const float *y, float eps,
+                              void *h_out, void *stream);
+
+/*
+ * pi_decode_stack -- one decode step through `n_layers` layers:
+ *     h_0 = h_in;  for l: (idx_l, count_l, y_l) = pi_layer(h_l);
+ *                         h_{l+1} = pi_residual_rmsnorm(h_l, y_l, eps)
+ *     h_out = h_{n_layers}
+ * layers: HOST array of n_layers pi_layer_weights (read during the call; its
+ * device pointers are baked into the launch, so a captured CUDA graph keeps
+ * them).  idx: [n_layers, C] int32; counts: [n_layers] int32; y: optional
+ * [n_layers, B, d] fp32 (NULL: not kept); h_trace: optional [n_layers, B, d]
+ * ptype receiving each layer's input h_l (NULL: not kept).  h_out [B, d]
+ * ptype must not alias h_in.  All layers share one descriptor;
+ * n_layers <= PI_MAX_LAYERS.
+ */
+PI_API pi_status pi_decode_stack(const pi_ffn_desc *desc, int32_t batch, int32_t n_layers,
+                                 const pi_layer_weights *layers, const void *h_in, void *h_out, int32_t *idx,
+                                 int32_t *counts, float *y, void *h_trace, float eps, void *ws, size_t ws_bytes,
+                                 void *stream);
+
+/*
+ * Number of kernel launches one pi_decode_stack call with these arguments
+ * issues (for accounting; -1 for invalid arguments).
+ */
+PI_API int32_t pi_stack_launches(const pi_ffn_desc *desc, int32_t batch, int32_t n_layers);
+
+/*
+ * Read (and optionally clear) the sticky device status word of `ws`.  Waits
+ * for `stream`.  *status_out = PI_OK or the first device-side error recorded.
+ */
+PI_API pi_status pi_get_device_status(void *ws, int32_t *status_out, int32_t clear, void *stream);
+
+/* Text of the last host-side error in this thread (never NULL). */
+PI_API const char *pi_last_error(void);
+
+/* Library version, "major.minor.patch". */
+PI_API const char *pi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PI_H_ */

@@ -1,0 +1,107 @@
+"""libpi loads on a machine without a GPU, exports every symbol include/pi.h
+declares, and rejects bad arguments on the host before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import activation_sparse_decode_predict_b200 as pi
+from activation_sparse_decode_predict_b200 import _binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "pi.h"), encoding="utf-8").read()
+    return sorted(set(re.findall(r"PI_API\s+[\w\s\*]+?\b(pi_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_exports():
+    assert _declared() == sorted(B.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = pi.lib()
+    for name in _declared():
+        assert hasattr(lib, name), name
+    assert pi.version().count(".") == 2
+
+
+def _desc(**kw):
+    base = dict(d=4096, ffn=11008, n_hot=1101, rank=1024, wtype="f16", ptype="f16", act="reglu")
+    base.update(kw)
+    return pi.make_desc(**base)
+
+
+def test_workspace_bytes_is_host_only_and_grows_with_batch():
+    n1 = pi.workspace_bytes(_desc(), 1)
+    n16 = pi.workspace_bytes(_desc(), 16)
+    assert 0 < n1 < n16
+    assert n1 % 256 == 0
+
+
+@pytest.mark.parametrize("kw,batch", [
+    (dict(d=4100), 1),            # d % 8
+    (dict(ffn=0), 1),
+    (dict(n_hot=-1), 1),
+    (dict(n_hot=20000), 1),       # n_hot > ffn
+    (dict(rank=1020), 1),         # rank % 8
+    (dict(wtype="q4_0", d=4104), 1),  # Q4_0 needs d % 32
+    ({}, 0),
+    ({}, 17),
+])
+def test_invalid_descriptors_are_rejected(kw, batch):
+    lib = pi.lib()
+    assert lib.pi_workspace_bytes(ctypes.byref(_desc(**kw)), batch) == 0
+    assert lib.pi_last_error()
+
+
+def test_bad_pointers_fail_before_any_launch():
+    lib = pi.lib()
+    d = _desc()
+    fake = ctypes.c_void_p(1 << 20)        # aligned, never dereferenced: every call below fails first
+    mis = ctypes.c_void_p((1 << 20) + 4)   # misaligned for 16-byte tensors
+    P = ctypes.c_void_p
+    # NULL h
+    st = lib.pi_predict(ctypes.byref(d), 1, None, fake, fake, None, 0.5, fake, fake, fake, 1 << 40, None)
+    assert st == B.PI_ERR_INVALID_ARG and b"h" in lib.pi_last_error()
+    # misaligned P1
+    st = lib.pi_predict(ctypes.byref(d), 1, fake, mis, fake, None, 0.5, fake, fake, fake, 1 << 40, None)
+    assert st == B.PI_ERR_INVALID_ARG
+    # workspace too small
+    st = lib.pi_predict(ctypes.byref(d), 1, fake, fake, fake, None, 0.5, fake, fake, fake, 1024, None)
+    assert st == B.PI_ERR_CAPACITY
+    # NULL desc
+    st = lib.pi_predict(None, 1, fake, fake, fake, None, 0.5, fake, fake, fake, 1 << 40, None)
+    assert st == B.PI_ERR_INVALID_ARG
+    # sparse FFN: Q4_0 without scales
+    dq = _desc(wtype="q4_0", d=4096)
+    w = B.Weight(fake, None)
+    st = lib.pi_sparse_ffn(ctypes.byref(dq), 1, fake, fake, fake, w, w, w, None, None, fake, fake, 1 << 40, None)
+    assert st == B.PI_ERR_INVALID_ARG and b"scales" in lib.pi_last_error()
+    # ReGLU needs W_gate
+    w0 = B.Weight(None, None)
+    wf = B.Weight(fake, None)
+    st = lib.pi_sparse_ffn(ctypes.byref(d), 1, fake, fake, fake, w0, wf, wf, None, None, fake, fake, 1 << 40, None)
+    assert st == B.PI_ERR_INVALID_ARG and b"W_gate" in lib.pi_last_error()
+    # rmsnorm: bad batch / eps
+    assert lib.pi_residual_rmsnorm(0, 64, 1, fake, fake, 1e-6, fake, None) == B.PI_ERR_INVALID_ARG
+    assert lib.pi_residual_rmsnorm(1, 64, 1, fake, fake, -1.0, fake, None) == B.PI_ERR_INVALID_ARG
+    # decode stack: aliasing output and too many layers
+    arr = (B.LayerWeights * 1)()
+    st = lib.pi_decode_stack(ctypes.byref(d), 1, 1, arr, fake, fake, fake, fake, None, None, 1e-6, fake, 1 << 40,
+                             None)
+    assert st == B.PI_ERR_INVALID_ARG and b"alias" in lib.pi_last_error()
+    st = lib.pi_decode_stack(ctypes.byref(d), 1, 129, arr, fake, P(2 << 20), fake, fake, None, None, 1e-6, fake,
+                             1 << 40, None)
+    assert st == B.PI_ERR_INVALID_ARG
+    # status read needs an output pointer
+    assert lib.pi_get_device_status(fake, None, 0, None) == B.PI_ERR_INVALID_ARG
+
+
+def test_python_layer_refuses_cpu_tensors():
+    import torch
+    d = _desc(d=64, ffn=100, n_hot=10, rank=8)
+    with pytest.raises(ValueError, match="CUDA"):
+        pi.residual_rmsnorm(torch.zeros(1, 64), torch.zeros(1, 64), 1e-6, torch.zeros(1, 64))

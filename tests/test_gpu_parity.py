@@ -1,0 +1,227 @@
+"""GPU parity: libpi (through its C ABI) against the CPU oracle on the same
+seeded inputs, at sizes the oracle finishes in seconds that still span
+several tiles and ragged tails, plus edge cases and integer-exact layers."""
+import numpy as np
+import pytest
+import torch
+
+import activation_sparse_decode_predict_b200 as pi
+import oracle
+import pi_workload as W
+from gpu_util import (BAND, TOL, check_index_list, gpu_ffn, gpu_predict, oracle_layer, oracle_predict, rel_err,
+                      to_dev, to_np)
+
+pytestmark = pytest.mark.gpu
+
+# (name, d, ffn, hot_frac, rank, act, wtype, ptype, batch)
+SHAPES = [
+    ("tiny-relu-fp32", 512, 2048, 0.05, 64, "relu", "f32", "f32", 1),
+    ("ragged-reglu-f16-b3", 264, 777, 0.017, 24, "reglu", "f16", "f16", 3),
+    ("relu2-f16-nohot", 128, 513, 0.0, 16, "relu2", "f16", "f16", 1),
+    ("reglu-q4-b2", 160, 300, 0.10, 32, "reglu", "q4_0", "f16", 2),
+    ("relu-q4-b5", 256, 1100, 0.08, 32, "relu", "q4_0", "f16", 5),
+    ("relu-f32w-f16tok", 64, 100, 0.10, 8, "relu", "f32", "f16", 1),
+    ("reglu-f16-b16", 256, 1000, 0.10, 32, "reglu", "f16", "f16", 16),
+    ("reglu-f16-b8", 1024, 2600, 0.10, 128, "reglu", "f16", "f16", 8),
+    ("relu2-f32-b4", 96, 700, 0.05, 16, "relu2", "f32", "f32", 4),
+]
+
+
+def _workload(name, d, ffn, hot, rank, act, wt, pt, B, sparsity=0.88):
+    return W.Workload(name, 40 + len(name), d, ffn, 1, act, wt, pt, sparsity, 1.2, hot, rank, (B,), 1,
+                      has_b2=(act != "reglu"))
+
+
+def _layer(wl, layer=0):
+    L = W.make_layer(wl, layer, device="cpu")
+    return {k: to_dev(v) if k not in ("perm", "p", "thr") else v for k, v in L.items()}
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=[s[0] for s in SHAPES])
+def test_predict_and_sparse_ffn_match_oracle(shape):
+    wl = _workload(*shape)
+    B = shape[-1]
+    L = _layer(wl)
+    h = to_dev(W.make_tokens(wl, B, 0))
+    desc = pi.desc_for(wl)
+    ws = pi.workspace(desc, B)
+    gidx, idx_t, cnt_t = gpu_predict(desc, h, L, ws)
+    h_np = to_np(h)
+    orc = oracle_predict(L, h_np, wl)
+    check_index_list(gidx, orc, wl.thr, wl.n_hot, wl.ffn)
+    assert 0 < len(gidx) < wl.n_cold
+    y = gpu_ffn(desc, h, L, idx_t, cnt_t, ws)
+    ref = oracle_layer(L, h_np, wl, gidx)
+    assert rel_err(y, ref) <= TOL[wl.wtype]
+    assert pi.device_status(ws) == 0
+    # the fused layer call gives the same list and output
+    y2 = torch.zeros(B, wl.d, device="cuda")
+    idx2 = torch.zeros_like(idx_t)
+    cnt2 = torch.zeros_like(cnt_t)
+    pi.layer(desc, h, pi.layer_weights(L), idx2, cnt2, y2, ws)
+    torch.cuda.synchronize()
+    assert int(cnt2.item()) == len(gidx)
+    assert np.array_equal(idx2[: len(gidx)].cpu().numpy(), gidx)
+    assert rel_err(y2.cpu().numpy(), ref) <= TOL[wl.wtype]
+
+
+INT_CASES = [
+    (256, 600, 40, 32, "reglu", "f16", "f16", 1),
+    (256, 600, 0, 32, "relu", "f16", "f16", 4),
+    (96, 333, 33, 16, "relu2", "f32", "f32", 3),
+    (128, 520, 20, 16, "reglu", "q4_0", "f16", 2),
+    (160, 300, 300, 16, "relu", "q4_0", "f16", 1),
+    (256, 700, 70, 32, "reglu", "f16", "f16", 16),
+    (256, 700, 70, 32, "relu", "f16", "f16", 8),
+]
+
+
+@pytest.mark.parametrize("case", INT_CASES)
+def test_integer_exact_layers_are_bit_identical(case):
+    """Every product and partial sum is an exact small integer (or dyadic), so
+    the GPU must equal the oracle bit for bit in any summation order."""
+    d, ffn, n_hot, rank, act, wt, pt, B = case
+    L = W.make_int_layer(d, ffn, n_hot, rank, act, wt, pt, B, seed=d + ffn + B)
+    L = {k: to_dev(v) if k not in ("perm", "thr") else v for k, v in L.items()}
+    desc = pi.make_desc(d, ffn, n_hot, rank, wt, pt, act)
+    ws = pi.workspace(desc, B)
+    h = L["h"]
+    gidx, idx_t, cnt_t = gpu_predict(desc, h, L, ws)
+    h_np = to_np(h)
+    orc = oracle.predict(h_np, to_np(L["P1"]), to_np(L["P2"]), to_np(L["bp"]), 0.5, n_hot, ffn)
+    assert np.array_equal(gidx, orc["idx"])
+    y = gpu_ffn(desc, h, L, idx_t, cnt_t, ws)
+    ref = oracle.masked_ffn(h_np, gidx, to_np(L["Wg"]), to_np(L["Wu"]), to_np(L["WdT"]), to_np(L["b1"]),
+                            to_np(L["b2"]), act, n_hot, ffn)
+    assert np.array_equal(y, ref)
+
+
+def test_threshold_extremes_and_no_cold_neurons():
+    wl = _workload("edge", 128, 600, 0.1, 16, "reglu", "f16", "f16", 2)
+    L = _layer(wl)
+    h = to_dev(W.make_tokens(wl, 2, 3))
+    desc = pi.desc_for(wl)
+    ws = pi.workspace(desc, 2)
+    h_np = to_np(h)
+    # everything active: equals the dense FFN
+    L_all = dict(L, thr=-1e30)
+    gidx, idx_t, cnt_t = gpu_predict(desc, h, L_all, ws)
+    assert np.array_equal(gidx, np.arange(wl.n_hot, wl.ffn))
+    y = gpu_ffn(desc, h, L_all, idx_t, cnt_t, ws)
+    Ln = {k: to_np(L[k]) for k in ("Wg", "Wu", "WdT", "b1")}
+    dense = oracle.dense_ffn(h_np, Ln["Wg"], Ln["Wu"], Ln["WdT"], Ln["b1"], None, "reglu", wl.n_hot, wl.ffn)
+    assert rel_err(y, dense) <= TOL["f16"]
+    # nothing active: hot part only
+    L_none = dict(L, thr=1e30)
+    gidx, idx_t, cnt_t = gpu_predict(desc, h, L_none, ws)
+    assert len(gidx) == 0
+    y = gpu_ffn(desc, h, L_none, idx_t, cnt_t, ws)
+    hot = oracle.masked_ffn(h_np, [], Ln["Wg"], Ln["Wu"], Ln["WdT"], Ln["b1"], None, "reglu", wl.n_hot, wl.ffn)
+    assert rel_err(y, hot) <= TOL["f16"]
+    # all neurons hot: no predictor matrix at all
+    desc_h = pi.make_desc(128, 600, 600, 16, "f16", "f16", "reglu")
+    ws_h = pi.workspace(desc_h, 2)
+    idx = torch.zeros(1, dtype=torch.int32, device="cuda")
+    cnt = torch.full((1,), 5, dtype=torch.int32, device="cuda")
+    pi.predict(desc_h, h, L["P1"], None, None, 0.5, idx, cnt, ws_h)
+    torch.cuda.synchronize()
+    assert int(cnt.item()) == 0
+    y = torch.zeros(2, 128, device="cuda")
+    pi.sparse_ffn(desc_h, h, idx, cnt, L["Wg"], L["Wu"], L["WdT"], L["b1"], None, y, ws_h)
+    torch.cuda.synchronize()
+    full = oracle.masked_ffn(h_np, [], Ln["Wg"], Ln["Wu"], Ln["WdT"], Ln["b1"], None, "reglu", 600, 600)
+    assert rel_err(y.cpu().numpy(), full) <= TOL["f16"]
+
+
+def test_bad_device_list_is_flagged_and_skipped():
+    wl = _workload("badidx", 128, 500, 0.1, 16, "relu", "f16", "f16", 1)
+    L = _layer(wl)
+    h = to_dev(W.make_tokens(wl, 1, 0))
+    desc = pi.desc_for(wl)
+    ws = pi.workspace(desc, 1)
+    good = [wl.n_hot + 3, wl.n_hot + 40, wl.ffn - 1]
+    idx = torch.tensor(good[:2] + [wl.ffn + 5] + good[2:], dtype=torch.int32, device="cuda")
+    cnt = torch.tensor([4], dtype=torch.int32, device="cuda")
+    y = gpu_ffn(desc, h, L, idx, cnt, ws)
+    assert pi.device_status(ws, clear=True) == pi._binding.PI_ERR_INDEX
+    ref = oracle_layer(L, to_np(h), wl, good)
+    assert rel_err(y, ref) <= TOL["f16"]
+    assert pi.device_status(ws) == 0
+    # a count above the list's capacity is flagged and clamped
+    full = torch.arange(wl.n_hot, wl.ffn, dtype=torch.int32, device="cuda")
+    cnt = torch.tensor([wl.n_cold + 1000], dtype=torch.int32, device="cuda")
+    y = gpu_ffn(desc, h, L, full, cnt, ws)
+    assert pi.device_status(ws, clear=True) == pi._binding.PI_ERR_CAPACITY
+    ref = oracle_layer(L, to_np(h), wl, full.cpu().numpy())
+    assert rel_err(y, ref) <= TOL["f16"]
+
+
+@pytest.mark.parametrize("htype", ["f32", "f16"])
+def test_residual_rmsnorm_matches_oracle(htype):
+    g = torch.Generator().manual_seed(5)
+    B, d = 3, 520
+    h = (torch.randn(B, d, generator=g)).to(torch.float32 if htype == "f32" else torch.float16)
+    y = torch.randn(B, d, generator=g) * 0.3
+    out = torch.empty_like(h, device="cuda")
+    pi.residual_rmsnorm(h.cuda(), y.cuda(), 1e-6, out)
+    torch.cuda.synchronize()
+    ref = oracle.residual_rmsnorm(h.numpy(), y.numpy().astype(np.float64), 1e-6)
+    got = out.float().cpu().numpy()
+    tol = 2e-6 if htype == "f32" else 2 ** -10
+    assert np.abs(got - ref).max() <= tol * np.abs(ref).max()
+
+
+def _stack_check(wl, B, n_layers, cols=None, seed_step=0):
+    """pi_decode_stack (the benchmark's launch) against the oracle, teacher-forced
+    per layer on the GPU's own layer inputs (h_trace)."""
+    desc = pi.desc_for(wl)
+    layers = [W.make_layer(wl, l, device="cuda") for l in range(n_layers)]
+    arr = pi.layer_array([pi.layer_weights(L) for L in layers])
+    h0 = W.make_tokens(wl, B, seed_step, device="cuda")
+    ws = pi.workspace(desc, B)
+    C = wl.n_cold
+    idx = torch.full((n_layers, C), -1, dtype=torch.int32, device="cuda")
+    counts = torch.zeros(n_layers, dtype=torch.int32, device="cuda")
+    y = torch.zeros(n_layers, B, wl.d, device="cuda")
+    trace = torch.zeros(n_layers, B, wl.d, dtype=h0.dtype, device="cuda")
+    h_out = torch.zeros_like(h0)
+    pi.decode_stack(desc, arr, h0, h_out, idx, counts, y, W.RMS_EPS, ws, h_trace=trace)
+    torch.cuda.synchronize()
+    assert pi.device_status(ws) == 0
+    assert torch.equal(trace[0], h0)
+    n_amb = 0
+    for l, L in enumerate(layers):
+        h_l = to_np(trace[l])
+        n = int(counts[l].item())
+        gidx = idx[l, :n].cpu().numpy()
+        orc = oracle_predict(L, h_l, wl)
+        n_amb += check_index_list(gidx, orc, wl.thr, wl.n_hot, wl.ffn)
+        ref = oracle_layer(L, h_l, wl, gidx, cols=cols)
+        got = to_np(y[l]).astype(np.float64)
+        if cols is not None:
+            got = got[:, cols]
+        assert rel_err(got, ref) <= TOL[wl.wtype], "layer %d" % l
+        # glue: the next layer's input (or h_out) is RMSNorm(h_l + y_l)
+        nxt = to_np(trace[l + 1]) if l + 1 < n_layers else to_np(h_out)
+        glue = oracle.residual_rmsnorm(h_l, to_np(y[l]).astype(np.float64), W.RMS_EPS)
+        assert np.abs(nxt.astype(np.float64) - glue).max() <= 2 ** -9 * np.abs(glue).max()
+    return n_amb
+
+
+def test_decode_stack_small_matches_oracle():
+    wl = _workload("stack", 256, 900, 0.1, 32, "reglu", "f16", "f16", 2).with_(layers=3)
+    _stack_check(wl, 2, 3)
+
+
+FULL = [("7b-reglu-fp16", 1), ("13b-reglu-q4_0", 1), ("40b-relu-fp16", 1), ("40b-relu-fp16", 8),
+        ("70b-reglu-fp16", 1), ("70b-reglu-fp16", 4), ("70b-reglu-fp16", 16)]
+
+
+@pytest.mark.parametrize("name,B", FULL, ids=["%s-b%d" % f for f in FULL])
+def test_full_size_workloads_two_layers_sampled(name, B):
+    """Full workload shapes through pi_decode_stack; every active-list entry is
+    checked, y on 48 sampled columns (the oracle computes them one by one)."""
+    wl = W.WORKLOADS[name]
+    rng = np.random.default_rng(B)
+    cols = np.sort(rng.choice(wl.d, size=48, replace=False)).astype(np.int32)
+    _stack_check(wl, B, 2, cols=cols, seed_step=B)
