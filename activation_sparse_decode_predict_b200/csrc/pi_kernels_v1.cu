@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(256) k_ffn_act(const void* __restrict__ h, int
   const int units = d / E;
   for (int p = gw; p < n; p += nw) {
     const int j = p < n_hot ? p : idx[p - n_hot];
-    if (j < n_hot || j >= ffn) {
+    if (p >= n_hot && (j < n_hot || j >= ffn)) {
       if (lane == 0) set_status(status, kStIndex);
       if (lane < B) a[(int64_t)lane * n_max + p] = 0.f;
       continue;
@@ -245,7 +245,7 @@ __global__ void k_ffn_down(int B, int d, int ffn, int n_hot, const int32_t* __re
         for (int i = 0; i < NB; ++i) acc[q][e][i] = 0.f;
     for (int64_t p = p0; p < p1; ++p) {
       const int j = p < n_hot ? (int)p : idx[p - n_hot];
-      if (j < n_hot || j >= ffn) continue;  // flagged by k_ffn_act
+      if (p >= n_hot && (j < n_hot || j >= ffn)) continue;  // flagged by k_ffn_act
       float av[NB];
 #pragma unroll
       for (int i = 0; i < NB; ++i) av[i] = (i < nb) ? a[(int64_t)(b0 + i) * n_max + p] : 0.f;
