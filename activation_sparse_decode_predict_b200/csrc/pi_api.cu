@@ -9,6 +9,7 @@
 #include "pi_common.cuh"
 #include "pi_kernels_v1.cuh"
 #include "pi_layout.h"
+#include "pi_stack.cuh"
 
 namespace {
 
@@ -119,6 +120,93 @@ pi_status ffn_impl(const pi_ffn_desc* d, int32_t B, const void* h, const int32_t
   return PI_OK;
 }
 
+pi_status check_layer(const pi_ffn_desc* desc, const pi_layer_weights* w) {
+  PI_TRY(check_ptr(w->P1, 16, "P1"));
+  if (desc->ffn > desc->n_hot) PI_TRY(check_ptr(w->P2, 16, "P2"));
+  if (w->bp) PI_TRY(check_ptr(w->bp, 4, "bp"));
+  if (desc->act == PI_ACT_REGLU) PI_TRY(check_weight(desc, w->W_gate, "W_gate"));
+  PI_TRY(check_weight(desc, w->W_up, "W_up"));
+  PI_TRY(check_weight(desc, w->W_downT, "W_downT"));
+  if (w->b1) PI_TRY(check_ptr(w->b1, 4, "b1"));
+  if (w->b2) PI_TRY(check_ptr(w->b2, 16, "b2"));
+  return PI_OK;
+}
+
+int stack_grid() {
+  const int g = sm_count();
+  return g < pi::kGMax ? g : pi::kGMax;
+}
+
+// Fill the persistent kernel's parameters; PI_ERR_UNSUPPORTED if the shape
+// does not fit its constraints (the caller then runs the per-kernel path).
+pi_status fused_params(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, pi::StackParams& P, size_t& smem,
+                       int& G) {
+  if (!pi::stack_supported(desc->wtype, desc->ptype, desc->d, desc->ffn, desc->n_hot, desc->rank, B, n_layers))
+    return PI_ERR_UNSUPPORTED;
+  G = stack_grid();
+  memset(&P, 0, sizeof(P));
+  P.d = desc->d;
+  P.ffn = desc->ffn;
+  P.n_hot = desc->n_hot;
+  P.rank = desc->rank;
+  P.act = desc->act;
+  P.L = n_layers;
+  P.T = desc->d / 16;
+  smem = pi::stack_smem_layout(P, B, G);
+  if (smem == 0) return PI_ERR_UNSUPPORTED;
+  const int ep = desc->ptype == PI_F16 ? 2 : 4;
+  const size_t wrow = desc->wtype == PI_Q4_0 ? desc->d / 2 + desc->d / 16
+                                              : (size_t)desc->d * (desc->wtype == PI_F16 ? 2 : 4);
+  const size_t neuron = wrow * (desc->act == PI_ACT_REGLU ? 3 : 2);
+  const size_t p2item = (size_t)(P.T / 32) * desc->rank * ep;
+  const size_t p1item = (size_t)desc->d * ep;
+  const size_t half = (size_t)P.ring_bytes / 2;
+  if (neuron > half || p2item > half || p1item > half) return PI_ERR_UNSUPPORTED;
+  const int C = desc->ffn - desc->n_hot;
+  P.seg_cap = (C + G - 1) / G + 1;
+  return PI_OK;
+}
+
+pi_status fused_stack(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, const pi_layer_weights* layers,
+                      const void* h_in, void* h_out, int32_t* idx, int32_t* counts, float* y, void* h_trace, float eps,
+                      char* ws, const pi::WsLayout& L, cudaStream_t st) {
+  pi::StackParams P;
+  size_t smem = 0;
+  int G = 0;
+  const pi_status fs = fused_params(desc, B, n_layers, P, smem, G);
+  if (fs != PI_OK) return fs;
+  P.eps = eps;
+  P.h_in = h_in;
+  P.h_out = h_out;
+  P.idx = idx;
+  P.counts = counts;
+  P.y_out = y;
+  P.h_trace = h_trace;
+  P.ctrl = reinterpret_cast<pi::Ctrl*>(ws);
+  P.u_g = reinterpret_cast<float*>(ws + L.u);
+  P.yacc = reinterpret_cast<float*>(ws + L.yacc);
+  P.seg = reinterpret_cast<int*>(ws + L.seg);
+  P.seg_cnt = reinterpret_cast<int*>(ws + L.seg_cnt);
+  for (int l = 0; l < n_layers; ++l) {
+    const pi_layer_weights& w = layers[l];
+    pi::StackLayer& s = P.layers[l];
+    s.P1 = w.P1;
+    s.P2 = w.P2;
+    s.bp = w.bp;
+    s.wg = w.W_gate.data;
+    s.wg_sc = w.W_gate.scales;
+    s.wu = w.W_up.data;
+    s.wu_sc = w.W_up.scales;
+    s.wd = w.W_downT.data;
+    s.wd_sc = w.W_downT.scales;
+    s.b1 = w.b1;
+    s.b2 = w.b2;
+    s.thr = w.threshold;
+  }
+  PI_CUDA(pi::launch_stack(desc->wtype, desc->ptype, B, P, G, smem, st), "fused decode-step launch");
+  return PI_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -147,7 +235,7 @@ pi_status pi_predict(const pi_ffn_desc* desc, int32_t batch, const void* h, cons
   PI_TRY(check_ptr(P1, 16, "P1"));
   if (desc->ffn > desc->n_hot) PI_TRY(check_ptr(P2, 16, "P2"));
   if (bp) PI_TRY(check_ptr(bp, 4, "bp"));
-  PI_TRY(check_ptr(idx, 4, "idx"));
+  if (desc->ffn > desc->n_hot) PI_TRY(check_ptr(idx, 4, "idx"));
   PI_TRY(check_ptr(count, 4, "count"));
   PI_TRY(check_ws(desc, batch, ws, ws_bytes));
   return predict_impl(desc, batch, h, P1, P2, bp, threshold, idx, count, (char*)ws, (cudaStream_t)stream);
@@ -158,7 +246,7 @@ pi_status pi_sparse_ffn(const pi_ffn_desc* desc, int32_t batch, const void* h, c
                         const float* b2, float* y, void* ws, size_t ws_bytes, void* stream) {
   PI_TRY(check_desc(desc, batch));
   PI_TRY(check_ptr(h, 16, "h"));
-  PI_TRY(check_ptr(idx, 4, "idx"));
+  if (desc->ffn > desc->n_hot) PI_TRY(check_ptr(idx, 4, "idx"));
   PI_TRY(check_ptr(count, 4, "count"));
   if (desc->act == PI_ACT_REGLU) PI_TRY(check_weight(desc, W_gate, "W_gate"));
   PI_TRY(check_weight(desc, W_up, "W_up"));
@@ -178,7 +266,7 @@ pi_status pi_layer(const pi_ffn_desc* desc, int32_t batch, const void* h, const 
   PI_TRY(check_ptr(w->P1, 16, "P1"));
   if (desc->ffn > desc->n_hot) PI_TRY(check_ptr(w->P2, 16, "P2"));
   if (w->bp) PI_TRY(check_ptr(w->bp, 4, "bp"));
-  PI_TRY(check_ptr(idx, 4, "idx"));
+  if (desc->ffn > desc->n_hot) PI_TRY(check_ptr(idx, 4, "idx"));
   PI_TRY(check_ptr(count, 4, "count"));
   if (desc->act == PI_ACT_REGLU) PI_TRY(check_weight(desc, w->W_gate, "W_gate"));
   PI_TRY(check_weight(desc, w->W_up, "W_up"));
@@ -215,13 +303,19 @@ pi_status pi_decode_stack(const pi_ffn_desc* desc, int32_t batch, int32_t n_laye
   PI_TRY(check_ptr(h_in, 16, "h_in"));
   PI_TRY(check_ptr(h_out, 16, "h_out"));
   if (h_in == h_out) return fail(PI_ERR_INVALID_ARG, "%s", "h_out must not alias h_in");
-  PI_TRY(check_ptr(idx, 4, "idx"));
+  if (desc->ffn > desc->n_hot) PI_TRY(check_ptr(idx, 4, "idx"));
   PI_TRY(check_ptr(counts, 4, "counts"));
   if (y) PI_TRY(check_ptr(y, 16, "y"));
   if (!(eps >= 0.f)) return fail(PI_ERR_INVALID_ARG, "%s", "eps must be >= 0");
   PI_TRY(check_ws(desc, batch, ws, ws_bytes));
+  for (int l = 0; l < n_layers; ++l) PI_TRY(check_layer(desc, &layers[l]));
   const pi::WsLayout L = pi::ws_layout(desc->d, desc->ffn, desc->n_hot, desc->rank, batch);
   char* wsc = (char*)ws;
+  {
+    const pi_status fs = fused_stack(desc, batch, n_layers, layers, h_in, h_out, idx, counts, y, h_trace, eps, wsc, L,
+                                     (cudaStream_t)stream);
+    if (fs != PI_ERR_UNSUPPORTED) return fs;
+  }
   float* ybuf = reinterpret_cast<float*>(wsc + L.ybuf);
   void* hbuf[2] = {h_out, wsc + L.hbuf};
   const size_t C = (size_t)(desc->ffn - desc->n_hot);
@@ -243,6 +337,12 @@ pi_status pi_decode_stack(const pi_ffn_desc* desc, int32_t batch, int32_t n_laye
 
 int32_t pi_stack_launches(const pi_ffn_desc* desc, int32_t batch, int32_t n_layers) {
   if (check_desc(desc, batch) != PI_OK || n_layers < 1 || n_layers > PI_MAX_LAYERS) return -1;
+  {
+    pi::StackParams P;
+    size_t smem = 0;
+    int G = 0;
+    if (fused_params(desc, batch, n_layers, P, smem, G) == PI_OK) return 1;
+  }
   const int per_layer = desc->ffn > desc->n_hot ? 7 : 5;  // predictor (3 or 1 + memset), FFN (3), glue (1)
   return per_layer * n_layers;
 }

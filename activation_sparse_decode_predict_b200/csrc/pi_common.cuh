@@ -24,10 +24,12 @@ enum : int { kStOk = 0, kStCapacity = -4, kStTimeout = -5, kStIndex = -6 };
 // Workspace control block (first 256 bytes of every workspace).
 struct Ctrl {
   int status;          // sticky: first device error wins
-  int pad0[7];
-  unsigned bar_count;  // grid barrier arrivals (persistent kernels)
-  unsigned bar_gen;    // grid barrier generation
-  int pad1[54];
+  int abort;           // set when any CTA of a persistent kernel gives up a wait
+  int pad0[30];
+  unsigned bar_count;  // grid barrier arrivals (own 64-byte line)
+  unsigned pad1[15];
+  unsigned bar_gen;    // grid barrier generation (own 64-byte line)
+  unsigned pad2[15];
 };
 static_assert(sizeof(Ctrl) == 256, "control block is 256 bytes");
 

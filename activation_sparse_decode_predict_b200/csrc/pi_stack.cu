@@ -1,0 +1,811 @@
+// pi_stack.cu -- one persistent, cooperative kernel for a whole decode step
+// through every layer of the stack (token blocks of 1 or 2).
+//
+// Pages: unite.ai "PowerInfer: Tüketici Düzeyinde bir GPU ile Hızlı Büyük Dil
+// Modeli Sunucusu" -- "Adaptif Sparsite Predictor’ları" (a per-layer predictor
+// picks the active neurons), "Nöron Bilinçli Operatör" (operators on single
+// rows of the up/gate matrices and single columns of the down matrix),
+// "Nöron Yerleştirme ve Yönetimi" (hot neurons stored first, with a table back
+// to the original rows); GeekNews "Serving model bahasa besar ...",
+// "Metode inferensi hibrida CPU/GPU" (the always-active block runs densely on
+// the GPU) and "Keterbatasan dan FAQ" (ReLU, ReGLU, squared ReLU).
+//
+// Design (one CTA per SM, G CTAs, grid-wide barriers are bounded spins):
+//   * a producer warp streams every byte the CTA needs into a shared-memory
+//     byte ring with 1-D bulk copies (cp.async.bulk, mbarrier completion), in
+//     a fixed order per layer: its P1 rows, its block of P2 rows, its share
+//     of the hot neurons (gate/up/down rows of each neuron as one item), then
+//     -- once every CTA has scored its P2 rows -- its share of the predicted
+//     cold neurons.  Nothing but the cold rows depends on the predictor, so
+//     the ring keeps HBM busy across the grid barriers.
+//   * consumer warps own 16 fixed columns of d per thread: the token block
+//     and the fp32 partial output stay in registers for the whole layer.
+//   * per layer: P1 rows -> u (global) -> barrier U -> P2 scores of the CTA's
+//     cold rows -> local ascending list + count -> barrier S -> hot neurons ->
+//     cold share of the global list -> partial y reduced into an fp32
+//     accumulator with vector atomics -> barrier Y -> residual + RMSNorm glue
+//     computed redundantly by every CTA -> next layer.
+//   * the cold list is ordered: CTA c's active rows are ascending and precede
+//     CTA c+1's, so the concatenation is the ascending list pi_predict writes.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pi_common.cuh"
+#include "pi_stack.cuh"
+#include "pi_sync.cuh"
+
+namespace pi {
+
+namespace {
+
+// ----------------------------------------------------------------------------
+// column ownership: consumer thread t of T owns 16 columns of d, as NRUN runs
+// of RUN consecutive columns whose layout follows the weight type.
+
+template <int WT>
+struct Own {
+  static constexpr int RUN = (WT == kF32) ? 4 : 8;
+  static constexpr int NRUN = 16 / RUN;
+  __device__ __forceinline__ static int col(int t, int T, int k) {
+    if constexpr (WT == kQ4_0) {
+      return (t >> 1) * 32 + (t & 1) * 8 + k * 16;
+    } else {
+      return (t + k * T) * RUN;
+    }
+  }
+};
+
+// 16 owned values of a d-row of element type X (kF32/kF16) at `row` (shared or global).
+template <int WT, int X>
+__device__ __forceinline__ void row_vals(const uint8_t* row, int t, int T, float (&v)[16]) {
+  using O = Own<WT>;
+#pragma unroll
+  for (int k = 0; k < O::NRUN; ++k) {
+    const int c = O::col(t, T, k);
+    float* o = v + k * O::RUN;
+    if constexpr (X == kF16) {
+      if constexpr (O::RUN == 8) {
+        const uint4 q = *reinterpret_cast<const uint4*>(row + 2 * c);
+        float2 f;
+        f = h2f2(q.x); o[0] = f.x; o[1] = f.y;
+        f = h2f2(q.y); o[2] = f.x; o[3] = f.y;
+        f = h2f2(q.z); o[4] = f.x; o[5] = f.y;
+        f = h2f2(q.w); o[6] = f.x; o[7] = f.y;
+      } else {
+        const uint2 q = *reinterpret_cast<const uint2*>(row + 2 * c);
+        float2 f;
+        f = h2f2(q.x); o[0] = f.x; o[1] = f.y;
+        f = h2f2(q.y); o[2] = f.x; o[3] = f.y;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < O::RUN; e += 4) {
+        const float4 q = *reinterpret_cast<const float4*>(row + 4 * (c + e));
+        o[e] = q.x; o[e + 1] = q.y; o[e + 2] = q.z; o[e + 3] = q.w;
+      }
+    }
+  }
+}
+
+// 16 owned values of a Q4_0 row laid out as [qs d/2 bytes][sc d/16 bytes].
+__device__ __forceinline__ void q4_vals(const uint8_t* row, int d, int t, float (&v)[16]) {
+  const uint2 q = *reinterpret_cast<const uint2*>(row + 8 * t);
+  const uint16_t sb = *reinterpret_cast<const uint16_t*>(row + d / 2 + 2 * (t >> 1));
+  const float s = half_bits_to_float(sb);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t b0 = (q.x >> (8 * k)) & 0xffu, b1 = (q.y >> (8 * k)) & 0xffu;
+    v[k] = s * (float)((int)(b0 & 15u) - 8);
+    v[4 + k] = s * (float)((int)(b1 & 15u) - 8);
+    v[8 + k] = s * (float)((int)(b0 >> 4) - 8);
+    v[12 + k] = s * (float)((int)(b1 >> 4) - 8);
+  }
+}
+
+template <int WT>
+__device__ __forceinline__ void w_vals(const uint8_t* row, int d, int t, int T, float (&v)[16]) {
+  if constexpr (WT == kQ4_0) q4_vals(row, d, t, v);
+  else row_vals<WT, WT>(row, t, T, v);
+}
+
+template <int WT, int X>
+__device__ __forceinline__ void store_vals(uint8_t* row, int t, int T, const float (&v)[16]) {
+  using O = Own<WT>;
+#pragma unroll
+  for (int k = 0; k < O::NRUN; ++k) {
+    const int c = O::col(t, T, k);
+    const float* o = v + k * O::RUN;
+    if constexpr (X == kF16) {
+#pragma unroll
+      for (int e = 0; e < O::RUN; e += 2) {
+        *reinterpret_cast<__half2*>(row + 2 * (c + e)) = __floats2half2_rn(o[e], o[e + 1]);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < O::RUN; e += 4) {
+        *reinterpret_cast<float4*>(row + 4 * (c + e)) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ float round_to(int X, float v) {
+  return X == kF16 ? __half2float(__float2half_rn(v)) : v;
+}
+
+__device__ __forceinline__ float act_eval(int act, float g, float v) {
+  if (act == kReglu) return fmaxf(g, 0.f) * v;
+  const float r = fmaxf(g, 0.f);
+  return act == kRelu2 ? r * r : r;
+}
+
+__device__ __forceinline__ int wrow_bytes(int WT_, int d) {
+  return WT_ == kQ4_0 ? d / 2 + d / 16 : d * (WT_ == kF16 ? 2 : 4);
+}
+
+struct Smem {
+  uint8_t* ring;
+  uint64_t* full;
+  uint64_t* empty;
+  uint64_t* list_bar;
+  uint32_t* item_off;
+  uint32_t* istart;  // producer-private: start/size of the items in flight
+  uint32_t* isize;
+  float* u;          // [B][r] split layout (see load_u)
+  float* bp;
+  float* b1hot;
+  int* cidx;
+  float* cb1;
+  uint8_t* act;
+  float* red;        // [2][NW][2B]
+  int* prefix;       // [G + 1]
+  int* misc;         // [0] cold_n, [1] gen_start
+};
+
+__device__ __forceinline__ Smem carve(uint8_t* base, const StackParams& p) {
+  Smem s;
+  s.ring = base;
+  s.full = reinterpret_cast<uint64_t*>(base + p.off_bars);
+  s.empty = s.full + kNQ;
+  s.list_bar = s.empty + kNQ;
+  s.item_off = reinterpret_cast<uint32_t*>(base + p.off_itemoff);
+  s.istart = s.item_off + kNQ;
+  s.isize = s.istart + kNQ;
+  s.u = reinterpret_cast<float*>(base + p.off_u);
+  s.bp = reinterpret_cast<float*>(base + p.off_bp);
+  s.b1hot = reinterpret_cast<float*>(base + p.off_b1hot);
+  s.cidx = reinterpret_cast<int*>(base + p.off_cidx);
+  s.cb1 = reinterpret_cast<float*>(base + p.off_cb1);
+  s.act = base + p.off_act;
+  s.red = reinterpret_cast<float*>(base + p.off_red);
+  s.prefix = reinterpret_cast<int*>(base + p.off_prefix);
+  s.misc = reinterpret_cast<int*>(base + p.off_misc);
+  return s;
+}
+
+__device__ __forceinline__ int share_lo(int n, int c, int G) { return (int)((int64_t)n * c / G); }
+
+// CTA-wide (consumer warps) sum of NV values per thread; every thread gets the
+// totals, added in the same warp order.  The two scratch buffers alternate
+// (stride MAXV per warp) so that the next call's writes cannot overtake this
+// call's reads.  Returns the OR of `flag` over the consumer threads.
+template <int NV, int MAXV>
+__device__ __forceinline__ bool cta_reduce(float (&v)[NV], float* red_base, int& par, int warp, int lane, int NW,
+                                           int T, bool flag) {
+#pragma unroll
+  for (int i = 0; i < NV; ++i) v[i] = warp_sum(v[i]);
+  float* red = red_base + par * (kMaxConsumers / 32) * MAXV;
+  if (lane == 0) {
+#pragma unroll
+    for (int i = 0; i < NV; ++i) red[warp * MAXV + i] = v[i];
+  }
+  flag = named_sync_or(1, T, flag);
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    float a = 0.f;
+    for (int w = 0; w < NW; ++w) a += red[w * MAXV + i];
+    v[i] = a;
+  }
+  par ^= 1;
+  return flag;
+}
+
+// ----------------------------------------------------------------------------
+// producer (one warp; lane 0 issues the copies)
+
+struct Producer {
+  const StackParams& p;
+  Smem& s;
+  Ctrl* ctrl;
+  uint32_t item = 0;  // next item index
+  uint32_t rel = 0;   // items known consumed
+  uint32_t head = 0;  // next free ring byte
+  bool ok = true;
+
+  __device__ Producer(const StackParams& p_, Smem& s_) : p(p_), s(s_), ctrl(p_.ctrl) {}
+
+  __device__ bool wait_consumed() {
+    const uint32_t q = rel % kNQ;
+    if (!mbar_wait(&s.empty[q], (rel / kNQ) & 1u, ctrl)) return false;
+    ++rel;
+    return true;
+  }
+
+  // Reserve `bytes` contiguous ring bytes for the next item; returns the offset.
+  __device__ bool alloc(uint32_t bytes, uint32_t& pos) {
+    const uint32_t R = (uint32_t)p.ring_bytes;
+    for (;;) {
+      if (item - rel >= (uint32_t)kNQ) {
+        if (!wait_consumed()) return false;
+        continue;
+      }
+      if (rel == item) {  // ring empty
+        pos = (head + bytes <= R) ? head : 0;
+        return true;
+      }
+      const uint32_t tail = s.istart[rel % kNQ];
+      if (head > tail) {
+        if (head + bytes <= R) { pos = head; return true; }
+        if (bytes <= tail) { pos = 0; return true; }
+      } else if (head + bytes <= tail) {
+        pos = head;
+        return true;
+      }
+      if (!wait_consumed()) return false;
+    }
+  }
+
+  // One item made of up to 6 contiguous source segments, copied back to back.
+  __device__ bool issue(int nseg, const void* const* src, const uint32_t* bytes) {
+    uint32_t total = 0;
+    for (int i = 0; i < nseg; ++i) total += bytes[i];
+    uint32_t pos;
+    if (!alloc(total, pos)) return false;
+    const uint32_t q = item % kNQ;
+    s.item_off[q] = pos;
+    s.istart[q] = pos;
+    s.isize[q] = total;
+    mbar_arrive_expect_tx(&s.full[q], total);
+    uint32_t o = pos;
+    for (int i = 0; i < nseg; ++i) {
+      bulk_g2s(s.ring + o, src[i], bytes[i], &s.full[q]);
+      o += bytes[i];
+    }
+    head = pos + total;
+    ++item;
+    return true;
+  }
+
+  __device__ bool issue_neuron(const StackLayer& Ly, int j, int wt, int gated) {
+    const void* src[6];
+    uint32_t by[6];
+    int n = 0;
+    const int d = p.d;
+    auto add_row = [&](const void* data, const void* sc) {
+      if (wt == kQ4_0) {
+        src[n] = reinterpret_cast<const uint8_t*>(data) + (int64_t)j * (d / 2);
+        by[n++] = d / 2;
+        src[n] = reinterpret_cast<const uint8_t*>(sc) + (int64_t)j * (d / 16);
+        by[n++] = d / 16;
+      } else {
+        const int rb = d * (wt == kF16 ? 2 : 4);
+        src[n] = reinterpret_cast<const uint8_t*>(data) + (int64_t)j * rb;
+        by[n++] = rb;
+      }
+    };
+    if (gated) add_row(Ly.wg, Ly.wg_sc);
+    add_row(Ly.wu, Ly.wu_sc);
+    add_row(Ly.wd, Ly.wd_sc);
+    return issue(n, src, by);
+  }
+
+  // Drain: wait for every issued copy to land before the CTA may exit.
+  __device__ void drain() {
+    for (uint32_t i = rel; i < item; ++i) mbar_wait(&s.full[i % kNQ], (i / kNQ) & 1u, ctrl);
+  }
+};
+
+// ----------------------------------------------------------------------------
+
+template <int WT, int PT, int B>
+__global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_constant__ StackParams p) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  Smem s = carve(smem_raw, p);
+  Ctrl* ctrl = p.ctrl;
+  const int G = gridDim.x, c = blockIdx.x;
+  const int T = p.T, NW = T / 32;
+  const int d = p.d, r = p.rank, H = p.n_hot, C = p.ffn - p.n_hot;
+  const int gated = p.act == kReglu;
+  const int ep = PT == kF16 ? 2 : 4;
+
+  if (threadIdx.x == 0) {
+    for (int q = 0; q < kNQ; ++q) {
+      mbar_init(&s.full[q], 1);
+      mbar_init(&s.empty[q], NW);
+    }
+    mbar_init(s.list_bar, 1);
+    mbar_fence_init();
+    s.misc[1] = (int)ld_acquire_u32(&ctrl->bar_gen);
+  }
+  __syncthreads();
+  const unsigned gen0 = (unsigned)s.misc[1];
+
+  // shares that do not depend on the predictor
+  const int k0 = share_lo(r, c, G), k1 = share_lo(r, c + 1, G);
+  const int c0 = share_lo(C, c, G), c1 = share_lo(C, c + 1, G);
+  const int j0 = share_lo(H, c, G), j1 = share_lo(H, c + 1, G);
+
+  if (threadIdx.x < 32) {
+    // ======================= producer warp =======================
+    const int lane = threadIdx.x;
+    Producer pr(p, s);
+    bool ok = true;
+    for (int l = 0; l < p.L && ok; ++l) {
+      const StackLayer& Ly = p.layers[l];
+      if (lane == 0) {
+        for (int k = k0; k < k1 && ok; ++k) {
+          const void* src = reinterpret_cast<const uint8_t*>(Ly.P1) + (int64_t)k * d * ep;
+          const uint32_t by = d * ep;
+          ok = pr.issue(1, &src, &by);
+        }
+        for (int cc = c0; cc < c1 && ok; cc += NW) {
+          const int rows = min(NW, c1 - cc);
+          const void* src = reinterpret_cast<const uint8_t*>(Ly.P2) + (int64_t)cc * r * ep;
+          const uint32_t by = rows * r * ep;
+          ok = pr.issue(1, &src, &by);
+        }
+        for (int j = j0; j < j1 && ok; ++j) ok = pr.issue_neuron(Ly, j, WT, gated);
+        // the cold rows need every CTA's scores: barrier S of this layer
+        if (ok) ok = grid_wait(ctrl, gen0, 3 * l + 1);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      __syncwarp();
+      if (!ok) break;
+      // cold list: prefix over the per-CTA counts, then this CTA's share
+      for (int i = lane; i <= G; i += 32) s.prefix[i] = 0;
+      __syncwarp();
+      int run = 0;
+      for (int base = 0; base < G; base += 32) {
+        const int i = base + lane;
+        int v = i < G ? __ldcg(p.seg_cnt + i) : 0;
+        int x = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += y;
+        }
+        if (i < G) s.prefix[i + 1] = run + x;
+        run += __shfl_sync(0xffffffffu, x, 31);
+      }
+      __syncwarp();
+      const int A = run;
+      const int q0 = share_lo(A, c, G), q1 = share_lo(A, c + 1, G);
+      for (int q = q0 + lane; q < q1; q += 32) {
+        int lo = 0, hi = G;  // last cta with prefix[cta] <= q
+        while (hi - lo > 1) {
+          const int mid = (lo + hi) >> 1;
+          if (s.prefix[mid] <= q) lo = mid;
+          else hi = mid;
+        }
+        const int j = __ldcg(p.seg + (int64_t)lo * p.seg_cap + (q - s.prefix[lo]));
+        s.cidx[q - q0] = j;
+        s.cb1[q - q0] = Ly.b1 ? __ldg(Ly.b1 + j) : 0.f;
+      }
+      // outputs: this CTA's segment of the ascending list, and the count
+      const int my_n = s.prefix[c + 1] - s.prefix[c];
+      for (int i = lane; i < my_n; i += 32)
+        p.idx[(int64_t)l * C + s.prefix[c] + i] = __ldcg(p.seg + (int64_t)c * p.seg_cap + i);
+      if (c == 0 && lane == 0) p.counts[l] = A;
+      if (lane == 0) s.misc[0] = q1 - q0;
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(s.list_bar);
+        for (int q = 0; q < q1 - q0 && ok; ++q) ok = pr.issue_neuron(Ly, s.cidx[q], WT, gated);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+    }
+    if (lane == 0) pr.drain();
+    return;
+  }
+
+  // ======================= consumer warps =======================
+  const int t = threadIdx.x - 32;
+  const int warp = t >> 5, lane = t & 31;
+  uint32_t item = 0;
+  int par = 0;
+  float h[B][16], y[B][16];
+  bool bad = false;
+
+  // layer-0 input
+#pragma unroll
+  for (int b = 0; b < B; ++b)
+    row_vals<WT, PT>(reinterpret_cast<const uint8_t*>(p.h_in) + (int64_t)b * d * ep, t, T, h[b]);
+  if (c == 0 && p.h_trace) {
+#pragma unroll
+    for (int b = 0; b < B; ++b) store_vals<WT, PT>(reinterpret_cast<uint8_t*>(p.h_trace) + (int64_t)b * d * ep, t, T, h[b]);
+  }
+  // zero this CTA's slice of the layer-0 accumulator
+  {
+    const int n4 = B * d / 4;
+    const int z0 = share_lo(n4, c, G), z1 = share_lo(n4, c + 1, G);
+    for (int i = z0 + t; i < z1; i += T) reinterpret_cast<float4*>(p.yacc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+
+  auto wait_item = [&](uint32_t& off) -> bool {
+    const uint32_t q = item % kNQ;
+    const bool okw = mbar_wait(&s.full[q], (item / kNQ) & 1u, ctrl);
+    off = s.item_off[q];
+    return okw;
+  };
+  auto release_item = [&]() {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.empty[item % kNQ]);
+    ++item;
+  };
+
+
+  for (int l = 0; l < p.L; ++l) {
+    const StackLayer& Ly = p.layers[l];
+    // small per-layer vectors of this CTA's shares
+    for (int x = t; x < c1 - c0; x += T) s.bp[x] = Ly.bp ? __ldg(Ly.bp + c0 + x) : 0.f;
+    for (int x = t; x < j1 - j0; x += T) s.b1hot[x] = Ly.b1 ? __ldg(Ly.b1 + j0 + x) : 0.f;
+
+    // ---- predictor step 1: u = ReLU(P1 h) for this CTA's rows ----
+    for (int k = k0; k < k1; ++k) {
+      uint32_t off;
+      bool to = !wait_item(off);
+      float w[16];
+      row_vals<WT, PT>(s.ring + off, t, T, w);
+      float acc[B];
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) a = fmaf(w[e], h[b][e], a);
+        acc[b] = a;
+      }
+      release_item();
+      to = cta_reduce<B, 2 * B>(acc, s.red, par, warp, lane, NW, T, to);
+      if (to) { bad = true; break; }
+      if (t == 0)
+        for (int b = 0; b < B; ++b) p.u_g[(int64_t)b * r + k] = fmaxf(acc[b], 0.f);
+    }
+    if (named_sync_or(1, T, bad)) return;
+    if (t == 0) grid_arrive(ctrl, G);
+    {
+      bool okw = true;
+      if (t == 0) okw = grid_wait(ctrl, gen0, 3 * l);
+      if (named_sync_or(1, T, !okw)) return;
+    }
+    // next layer's accumulator slice is free now (its last readers passed this barrier)
+    {
+      float* nxt = p.yacc + (size_t)((l + 1) & 1) * B * d;
+      const int n4 = B * d / 4;
+      const int z0 = share_lo(n4, c, G), z1 = share_lo(n4, c + 1, G);
+      for (int i = z0 + t; i < z1; i += T) reinterpret_cast<float4*>(nxt)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    // u -> shared memory, split layout: unit m (8 values) stored as two float4
+    // planes so that lane-strided reads are conflict-free.
+    {
+      const int nu = r / 8;
+      for (int i = t; i < B * nu; i += T) {
+        const int b = i / nu, m = i % nu;
+        const float4* src = reinterpret_cast<const float4*>(p.u_g + (int64_t)b * r + 8 * m);
+        const float4 lo = __ldcg(src), hi = __ldcg(src + 1);
+        float4* dst = reinterpret_cast<float4*>(s.u + (size_t)b * r);
+        dst[m] = lo;
+        dst[nu + m] = hi;
+      }
+    }
+    named_sync(1, T);
+
+    // ---- predictor step 2: scores of this CTA's cold rows ----
+    {
+      const int nu = r / 8;  // 8-element units per row (r % 8 == 0)
+      for (int cc = c0; cc < c1; cc += NW) {
+        const int rows = min(NW, c1 - cc);
+        uint32_t off;
+        bool to = !wait_item(off);
+        if (warp < rows) {
+          const uint8_t* row = s.ring + off + (size_t)warp * r * ep;
+          float acc[B];
+#pragma unroll
+          for (int b = 0; b < B; ++b) acc[b] = 0.f;
+          for (int m = lane; m < nu; m += 32) {
+            float w[8];
+            if constexpr (PT == kF16) {
+              const uint4 q = *reinterpret_cast<const uint4*>(row + 16 * m);
+              float2 f;
+              f = h2f2(q.x); w[0] = f.x; w[1] = f.y;
+              f = h2f2(q.y); w[2] = f.x; w[3] = f.y;
+              f = h2f2(q.z); w[4] = f.x; w[5] = f.y;
+              f = h2f2(q.w); w[6] = f.x; w[7] = f.y;
+            } else {
+              const float4 a = *reinterpret_cast<const float4*>(row + 32 * m);
+              const float4 b2 = *reinterpret_cast<const float4*>(row + 32 * m + 16);
+              w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+              w[4] = b2.x; w[5] = b2.y; w[6] = b2.z; w[7] = b2.w;
+            }
+#pragma unroll
+            for (int b = 0; b < B; ++b) {
+              const float4* ub = reinterpret_cast<const float4*>(s.u + (size_t)b * r);
+              const float4 lo = ub[m], hi = ub[nu + m];
+              float a = acc[b];
+              a = fmaf(w[0], lo.x, a); a = fmaf(w[1], lo.y, a); a = fmaf(w[2], lo.z, a); a = fmaf(w[3], lo.w, a);
+              a = fmaf(w[4], hi.x, a); a = fmaf(w[5], hi.y, a); a = fmaf(w[6], hi.z, a); a = fmaf(w[7], hi.w, a);
+              acc[b] = a;
+            }
+          }
+          bool on = false;
+          const float bias = s.bp[cc - c0 + warp];
+#pragma unroll
+          for (int b = 0; b < B; ++b) on |= (warp_sum(acc[b]) + bias) > Ly.thr;
+          if (lane == 0) s.act[cc - c0 + warp] = on ? 1 : 0;
+        }
+        release_item();
+        if (named_sync_or(1, T, to)) return;
+      }
+    }
+    named_sync(1, T);
+    // local ascending list of this CTA's active cold rows (consumer warp 0)
+    if (warp == 0) {
+      int base = 0;
+      for (int x0 = 0; x0 < c1 - c0; x0 += 32) {
+        const int x = x0 + lane;
+        const bool on = x < c1 - c0 && s.act[x];
+        const unsigned m = __ballot_sync(0xffffffffu, on);
+        if (on) p.seg[(int64_t)c * p.seg_cap + base + __popc(m & ((1u << lane) - 1u))] = H + c0 + x;
+        base += __popc(m);
+      }
+      if (lane == 0) p.seg_cnt[c] = base;
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) grid_arrive(ctrl, G);
+    }
+
+    // ---- sparse FFN: hot share, then cold share ----
+#pragma unroll
+    for (int b = 0; b < B; ++b)
+#pragma unroll
+      for (int e = 0; e < 16; ++e) y[b][e] = 0.f;
+    const int wrb = wrow_bytes(WT, d);
+    auto neuron = [&](float bias, bool& to) {
+      uint32_t off;
+      to |= !wait_item(off);
+      const uint8_t* it = s.ring + off;
+      float acc[2 * B];
+      {
+        float wu[16];
+        w_vals<WT>(it + (gated ? wrb : 0), d, t, T, wu);
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+          float a = 0.f;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) a = fmaf(wu[e], h[b][e], a);
+          acc[B + b] = a;
+        }
+      }
+      if (gated) {
+        float wg[16];
+        w_vals<WT>(it, d, t, T, wg);
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+          float a = 0.f;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) a = fmaf(wg[e], h[b][e], a);
+          acc[b] = a;
+        }
+      } else {
+#pragma unroll
+        for (int b = 0; b < B; ++b) acc[b] = 0.f;
+      }
+      to = cta_reduce<2 * B, 2 * B>(acc, s.red, par, warp, lane, NW, T, to);
+      float a[B];
+#pragma unroll
+      for (int b = 0; b < B; ++b) a[b] = gated ? act_eval(kReglu, acc[b] + bias, acc[B + b]) : act_eval(p.act, acc[B + b] + bias, 0.f);
+      float wd[16];
+      w_vals<WT>(it + (gated ? 2 : 1) * wrb, d, t, T, wd);
+      release_item();
+#pragma unroll
+      for (int b = 0; b < B; ++b)
+#pragma unroll
+        for (int e = 0; e < 16; ++e) y[b][e] = fmaf(a[b], wd[e], y[b][e]);
+    };
+    for (int j = j0; j < j1; ++j) {
+      bool to = false;
+      neuron(s.b1hot[j - j0], to);
+      if (to) return;
+    }
+    {
+      const bool okw = mbar_wait(s.list_bar, l & 1, ctrl);
+      if (named_sync_or(1, T, !okw)) return;
+    }
+    const int ncold = s.misc[0];
+    for (int q = 0; q < ncold; ++q) {
+      bool to = false;
+      neuron(s.cb1[q], to);
+      if (to) return;
+    }
+
+    // ---- split-K: add the partial into the fp32 accumulator ----
+    {
+      float* acc = p.yacc + (size_t)(l & 1) * B * d;
+      using O = Own<WT>;
+#pragma unroll
+      for (int b = 0; b < B; ++b)
+#pragma unroll
+        for (int k = 0; k < O::NRUN; ++k) {
+          const int col = O::col(t, T, k);
+#pragma unroll
+          for (int e = 0; e < O::RUN; e += 4)
+            atomicAdd(reinterpret_cast<float4*>(acc + (size_t)b * d + col + e),
+                      make_float4(y[b][k * O::RUN + e], y[b][k * O::RUN + e + 1], y[b][k * O::RUN + e + 2],
+                                  y[b][k * O::RUN + e + 3]));
+        }
+      __threadfence();
+    }
+    named_sync(1, T);
+    if (t == 0) grid_arrive(ctrl, G);
+    {
+      bool okw = true;
+      if (t == 0) okw = grid_wait(ctrl, gen0, 3 * l + 2);
+      if (named_sync_or(1, T, !okw)) return;
+    }
+
+    // ---- glue: h <- RMSNorm(h + y + b2), rounded to the token type ----
+    {
+      const float* acc = p.yacc + (size_t)(l & 1) * B * d;
+      using O = Own<WT>;
+      float ss[B];
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        float yv[16];
+#pragma unroll
+        for (int k = 0; k < O::NRUN; ++k) {
+          const int col = O::col(t, T, k);
+#pragma unroll
+          for (int e = 0; e < O::RUN; e += 4) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(acc + (size_t)b * d + col + e));
+            float4 bb = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (Ly.b2) bb = __ldg(reinterpret_cast<const float4*>(Ly.b2 + col + e));
+            yv[k * O::RUN + e] = v.x + bb.x;
+            yv[k * O::RUN + e + 1] = v.y + bb.y;
+            yv[k * O::RUN + e + 2] = v.z + bb.z;
+            yv[k * O::RUN + e + 3] = v.w + bb.w;
+          }
+        }
+        if (c == 0 && p.y_out) store_vals<WT, kF32>(reinterpret_cast<uint8_t*>(p.y_out + ((size_t)l * B + b) * d), t, T, yv);
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float x = h[b][e] + yv[e];
+          h[b][e] = x;
+          a = fmaf(x, x, a);
+        }
+        ss[b] = a;
+      }
+      cta_reduce<B, 2 * B>(ss, s.red, par, warp, lane, NW, T, false);
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        const float inv = rsqrtf(ss[b] / (float)d + p.eps);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) h[b][e] = round_to(PT, h[b][e] * inv);
+      }
+      if (c == 0) {
+        uint8_t* dst = nullptr;
+        if (l + 1 < p.L) {
+          if (p.h_trace) dst = reinterpret_cast<uint8_t*>(p.h_trace) + (size_t)(l + 1) * B * d * ep;
+        } else {
+          dst = reinterpret_cast<uint8_t*>(p.h_out);
+        }
+        if (dst) {
+#pragma unroll
+          for (int b = 0; b < B; ++b) store_vals<WT, PT>(dst + (size_t)b * d * ep, t, T, h[b]);
+        }
+      }
+    }
+  }
+}
+
+template <int WT, int PT, int B>
+cudaError_t launch_t(const StackParams& p, int G, size_t smem, cudaStream_t st) {
+  auto fn = k_stack<WT, PT, B>;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(G);
+  cfg.blockDim = dim3(p.T + 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fn, p);
+}
+
+}  // namespace
+
+bool stack_supported(int wtype, int ptype, int d, int ffn, int n_hot, int rank, int B, int L) {
+  if (B < 1 || B > 2) return false;
+  if (L < 1 || L > kMaxLayers) return false;
+  if (d % 512 != 0 || d / 16 > kMaxConsumers) return false;
+  if (wtype == kQ4_0 && ptype != kF16 && ptype != kF32) return false;
+  if (rank % 8 != 0 || rank > kMaxRank) return false;
+  (void)ffn;
+  (void)n_hot;
+  return true;
+}
+
+size_t stack_smem_layout(StackParams& p, int B, int G) {
+  const int C = p.ffn - p.n_hot;
+  const int share_cap = (C + G - 1) / G + 1;
+  const int hot_cap = (p.n_hot + G - 1) / G + 1;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += (bytes + 127) & ~(size_t)127;
+    return (int)o;
+  };
+  // everything but the ring first (at the end of shared memory), then the ring
+  size_t fixed = 0;
+  {
+    size_t o = 0;
+    auto t2 = [&](size_t bytes) { o += (bytes + 127) & ~(size_t)127; };
+    t2(sizeof(uint64_t) * (2 * kNQ + 1));
+    t2(sizeof(uint32_t) * 3 * kNQ);
+    t2(sizeof(float) * (size_t)B * p.rank);
+    t2(sizeof(float) * share_cap);
+    t2(sizeof(float) * hot_cap);
+    t2(sizeof(int) * share_cap);
+    t2(sizeof(float) * share_cap);
+    t2(share_cap);
+    t2(sizeof(float) * 2 * (kMaxConsumers / 32) * 2 * B);
+    t2(sizeof(int) * (G + 1));
+    t2(sizeof(int) * 4);
+    fixed = o;
+  }
+  const size_t total = kSmemBytes;
+  if (fixed + 32768 > total) return 0;
+  const size_t ring = (total - fixed) & ~(size_t)127;
+  p.ring_bytes = (int)ring;
+  off = ring;
+  p.off_bars = take(sizeof(uint64_t) * (2 * kNQ + 1));
+  p.off_itemoff = take(sizeof(uint32_t) * 3 * kNQ);
+  p.off_u = take(sizeof(float) * (size_t)B * p.rank);
+  p.off_bp = take(sizeof(float) * share_cap);
+  p.off_b1hot = take(sizeof(float) * hot_cap);
+  p.off_cidx = take(sizeof(int) * share_cap);
+  p.off_cb1 = take(sizeof(float) * share_cap);
+  p.off_act = take(share_cap);
+  p.off_red = take(sizeof(float) * 2 * (kMaxConsumers / 32) * 2 * B);
+  p.off_prefix = take(sizeof(int) * (G + 1));
+  p.off_misc = take(sizeof(int) * 4);
+  return off;
+}
+
+cudaError_t launch_stack(int wtype, int ptype, int B, const StackParams& p, int G, size_t smem, cudaStream_t st) {
+#define PI_STACK_CASE(W_, P_, B_) \
+  if (wtype == W_ && ptype == P_ && B == B_) return launch_t<W_, P_, B_>(p, G, smem, st);
+  PI_STACK_CASE(kF16, kF16, 1)
+  PI_STACK_CASE(kF16, kF16, 2)
+  PI_STACK_CASE(kQ4_0, kF16, 1)
+  PI_STACK_CASE(kQ4_0, kF16, 2)
+  PI_STACK_CASE(kF32, kF32, 1)
+  PI_STACK_CASE(kF32, kF32, 2)
+  PI_STACK_CASE(kF16, kF32, 1)
+  PI_STACK_CASE(kF16, kF32, 2)
+  PI_STACK_CASE(kF32, kF16, 1)
+  PI_STACK_CASE(kF32, kF16, 2)
+  PI_STACK_CASE(kQ4_0, kF32, 1)
+  PI_STACK_CASE(kQ4_0, kF32, 2)
+#undef PI_STACK_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace pi

@@ -1,0 +1,61 @@
+// pi_stack.cuh -- parameters and launcher of the persistent decode-step kernel.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "pi_common.cuh"
+
+namespace pi {
+
+constexpr int kMaxLayers = 128;
+constexpr int kNQ = 64;              // items in flight per CTA (queue depth)
+constexpr int kMaxConsumers = 512;   // consumer threads per CTA (d <= 8192)
+constexpr int kMaxRank = 4096;
+constexpr size_t kSmemBytes = 232448;  // opt-in shared memory per CTA on sm_100
+
+// One layer's device pointers (a copy of pi_layer_weights).
+struct StackLayer {
+  const void* P1;
+  const void* P2;
+  const float* bp;
+  const void* wg;
+  const void* wg_sc;
+  const void* wu;
+  const void* wu_sc;
+  const void* wd;
+  const void* wd_sc;
+  const float* b1;
+  const float* b2;
+  float thr;
+  int pad;
+};
+
+struct StackParams {
+  int d, ffn, n_hot, rank, act, L;
+  float eps;
+  int T;           // consumer threads (d / 16)
+  int ring_bytes;  // shared-memory ring size
+  int seg_cap;     // per-CTA capacity of the local active lists
+  int off_bars, off_itemoff, off_u, off_bp, off_b1hot, off_cidx, off_cb1, off_act, off_red, off_prefix, off_misc;
+  const void* h_in;
+  void* h_out;
+  int32_t* idx;     // [L, C]
+  int32_t* counts;  // [L]
+  float* y_out;     // [L, B, d] or null
+  void* h_trace;    // [L, B, d] or null
+  Ctrl* ctrl;
+  float* u_g;       // [B, r]
+  float* yacc;      // [2, B, d]
+  int* seg;         // [G, seg_cap]
+  int* seg_cnt;     // [G]
+  StackLayer layers[kMaxLayers];
+};
+
+bool stack_supported(int wtype, int ptype, int d, int ffn, int n_hot, int rank, int B, int L);
+// Fills the shared-memory offsets of p (needs d, ffn, n_hot, rank); returns the
+// dynamic shared memory size, or 0 if it does not fit.
+size_t stack_smem_layout(StackParams& p, int B, int G);
+cudaError_t launch_stack(int wtype, int ptype, int B, const StackParams& p, int G, size_t smem, cudaStream_t st);
+
+}  // namespace pi

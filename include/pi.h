@@ -50,7 +50,8 @@
  *   b2       [d]      fp32 output bias, may be NULL
  *   y        [B, d]   fp32 output
  *   idx      [C]      int32 active-neuron list, ascending storage rows in
- *                     [H, F); its length lives in the device scalar `count`
+ *                     [H, F); its length lives in the device scalar `count`;
+ *                     may be NULL when C == 0
  *   Q4_0 weights use split planes: data = qs [F, d/2] uint8, scales =
  *   sc [F, d/32] fp16; in each 32-element block, byte k holds element k in
  *   its low nibble and element k + 16 in its high nibble, x = s * (q - 8)

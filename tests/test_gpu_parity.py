@@ -180,7 +180,7 @@ def _stack_check(wl, B, n_layers, cols=None, seed_step=0):
     h0 = W.make_tokens(wl, B, seed_step, device="cuda")
     ws = pi.workspace(desc, B)
     C = wl.n_cold
-    idx = torch.full((n_layers, C), -1, dtype=torch.int32, device="cuda")
+    idx = torch.full((n_layers, max(C, 1)), -1, dtype=torch.int32, device="cuda")
     counts = torch.zeros(n_layers, dtype=torch.int32, device="cuda")
     y = torch.zeros(n_layers, B, wl.d, device="cuda")
     trace = torch.zeros(n_layers, B, wl.d, dtype=h0.dtype, device="cuda")
@@ -194,6 +194,8 @@ def _stack_check(wl, B, n_layers, cols=None, seed_step=0):
         h_l = to_np(trace[l])
         n = int(counts[l].item())
         gidx = idx[l, :n].cpu().numpy()
+        if C == 0:
+            assert n == 0
         orc = oracle_predict(L, h_l, wl)
         n_amb += check_index_list(gidx, orc, wl.thr, wl.n_hot, wl.ffn)
         ref = oracle_layer(L, h_l, wl, gidx, cols=cols)
@@ -225,3 +227,88 @@ def test_full_size_workloads_two_layers_sampled(name, B):
     rng = np.random.default_rng(B)
     cols = np.sort(rng.choice(wl.d, size=48, replace=False)).astype(np.int32)
     _stack_check(wl, B, 2, cols=cols, seed_step=B)
+
+
+# Shapes the persistent decode-step kernel takes (d % 512 == 0, token blocks of 1 or 2).
+FUSED = [
+    ("fused-f32-relu", 512, 2048, 0.05, 64, "relu", "f32", "f32", 1, 2),
+    ("fused-f16-reglu-b2", 1024, 3000, 0.10, 64, "reglu", "f16", "f16", 2, 3),
+    ("fused-q4-relu2", 512, 1500, 0.08, 32, "relu2", "q4_0", "f16", 1, 2),
+    ("fused-f16-relu", 1536, 5000, 0.08, 128, "relu", "f16", "f16", 1, 2),
+    ("fused-q4-reglu-b2", 1024, 2500, 0.10, 64, "reglu", "q4_0", "f16", 2, 2),
+    ("fused-f16-reglu-allhot", 512, 700, 1.0, 32, "reglu", "f16", "f16", 1, 2),
+    ("fused-f16-relu-nohot", 512, 900, 0.0, 32, "relu", "f16", "f16", 2, 2),
+]
+
+
+@pytest.mark.parametrize("case", FUSED, ids=[f[0] for f in FUSED])
+def test_fused_stack_matches_oracle(case):
+    name, d, ffn, hot, rank, act, wt, pt, B, L = case
+    wl = _workload(name, d, ffn, hot, rank, act, wt, pt, B).with_(layers=L)
+    assert pi.stack_launches(pi.desc_for(wl), B, L) == 1
+    _stack_check(wl, B, L, seed_step=3)
+
+
+@pytest.mark.parametrize("case", [(512, 900, 60, 32, "reglu", "f16", "f16", 1),
+                                  (1024, 1200, 0, 32, "relu", "f16", "f16", 2),
+                                  (512, 640, 40, 16, "relu2", "q4_0", "f16", 1),
+                                  (512, 500, 50, 16, "relu", "f32", "f32", 2)])
+def test_fused_stack_integer_exact(case):
+    """One integer-exact layer through the persistent kernel: list and output
+    are bit-identical to the oracle (fp32 sums of small integers are exact in
+    any order, atomics included)."""
+    d, ffn, n_hot, rank, act, wt, pt, B = case
+    L = W.make_int_layer(d, ffn, n_hot, rank, act, wt, pt, B, seed=3 * d + ffn)
+    L = {k: to_dev(v) if k not in ("perm", "thr") else v for k, v in L.items()}
+    desc = pi.make_desc(d, ffn, n_hot, rank, wt, pt, act)
+    assert pi.stack_launches(desc, B, 1) == 1
+    ws = pi.workspace(desc, B)
+    arr = pi.layer_array([pi.layer_weights(L)])
+    C = ffn - n_hot
+    idx = torch.full((1, max(C, 1)), -1, dtype=torch.int32, device="cuda")
+    counts = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = torch.zeros(1, B, d, device="cuda")
+    h_out = torch.zeros_like(L["h"])
+    pi.decode_stack(desc, arr, L["h"], h_out, idx, counts, y, 1e-6, ws)
+    torch.cuda.synchronize()
+    assert pi.device_status(ws) == 0
+    h_np = to_np(L["h"])
+    orc = oracle.predict(h_np, to_np(L["P1"]), to_np(L["P2"]), to_np(L["bp"]), 0.5, n_hot, ffn)
+    n = int(counts[0].item())
+    assert np.array_equal(idx[0, :n].cpu().numpy(), orc["idx"])
+    ref = oracle.masked_ffn(h_np, orc["idx"], to_np(L["Wg"]), to_np(L["Wu"]), to_np(L["WdT"]), to_np(L["b1"]),
+                            to_np(L["b2"]), act, n_hot, ffn)
+    assert np.array_equal(y[0].cpu().numpy().astype(np.float64), ref)
+
+
+def test_fused_stack_repeated_calls_and_graph_replay():
+    """The persistent kernel leaves its barrier state clean: back-to-back calls
+    and CUDA-graph replays give identical lists and outputs."""
+    wl = _workload("replay", 1024, 3000, 0.1, 64, "reglu", "f16", "f16", 1).with_(layers=4)
+    desc = pi.desc_for(wl)
+    layers = [W.make_layer(wl, l, device="cuda") for l in range(4)]
+    arr = pi.layer_array([pi.layer_weights(L) for L in layers])
+    h0 = W.make_tokens(wl, 1, 9, device="cuda")
+    ws = pi.workspace(desc, 1)
+    outs = []
+    s = torch.cuda.Stream()
+    idx = torch.zeros(4, wl.n_cold, dtype=torch.int32, device="cuda")
+    counts = torch.zeros(4, dtype=torch.int32, device="cuda")
+    h_out = torch.zeros_like(h0)
+    with torch.cuda.stream(s):
+        for _ in range(3):
+            pi.decode_stack(desc, arr, h0, h_out, idx, counts, None, W.RMS_EPS, ws, stream=s)
+            s.synchronize()
+            outs.append((counts.clone(), h_out.clone()))
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            pi.decode_stack(desc, arr, h0, h_out, idx, counts, None, W.RMS_EPS, ws, stream=s)
+        for _ in range(3):
+            g.replay()
+            s.synchronize()
+            outs.append((counts.clone(), h_out.clone()))
+    assert pi.device_status(ws) == 0
+    for c_, h_ in outs[1:]:
+        assert torch.equal(c_, outs[0][0])
+        # atomics may change the last bits of y; the fp16 outputs agree to 1 ulp
+        assert (h_.float() - outs[0][1].float()).abs().max().item() <= 2 ** -9
