@@ -209,6 +209,10 @@ pi_status fused_stack(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, cons
 
 }  // namespace
 
+namespace pi {
+void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+}  // namespace pi
+
 extern "C" {
 
 const char* pi_last_error(void) { return g_err; }

@@ -228,6 +228,31 @@ PI_API int32_t pi_stack_launches(const pi_ffn_desc *desc, int32_t batch, int32_t
  */
 PI_API pi_status pi_get_device_status(void *ws, int32_t *status_out, int32_t clear, void *stream);
 
+/*
+ * pi_predict_static -- pi_predict for callers that cannot allocate device
+ * memory.  The paper has no counterpart to this call; it exists for hosts
+ * that hand the library only its inputs and outputs (plugin interfaces that
+ * own every allocation, or serving loops that must not call cudaMalloc once
+ * running, because an allocation can synchronise the device).
+ *
+ * Same arguments, results and rules as pi_predict, minus the workspace: the
+ * scratch lives in one library-owned device array of PI_STATIC_SCRATCH_BYTES
+ * (1 MiB), held on every GPU that loads the library until the process exits.
+ * Limit: align256(batch * rank * 4) + align256(ceil(C/256) * 32) +
+ * align256(ceil(C/256) * 4) <= 1 MiB (C = ffn - n_hot), else
+ * PI_ERR_CAPACITY and nothing is launched.  The call allocates nothing.
+ * - The first call on a device looks the array's address up on that device
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ * - Every call shares the one array and the last call's contents stay in it;
+ *   nothing in it needs to start at zero (each call writes all it reads).
+ * - Calls that can overlap on the GPU (different streams, or several host
+ *   threads) race on the array: order them on one stream.
+ */
+#define PI_STATIC_SCRATCH_BYTES ((size_t)1 << 20)
+PI_API pi_status pi_predict_static(const pi_ffn_desc *desc, int32_t batch, const void *h, const void *P1,
+                                   const void *P2, const float *bp, float threshold, int32_t *idx, int32_t *count,
+                                   void *stream);
+
 /* Text of the last host-side error in this thread (never NULL). */
 PI_API const char *pi_last_error(void);
 

@@ -1,0 +1,54 @@
+"""pi_predict_static: the predictor for callers that cannot allocate device
+memory (hosts that give the library only its inputs and outputs).  Its
+scratch is a fixed 1 MiB array inside libpi; it must give the same active
+lists as pi_predict with a caller workspace, call after call."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import activation_sparse_decode_predict_b200 as pi
+import pi_workload as W
+from activation_sparse_decode_predict_b200 import _binding as B
+
+pytestmark = pytest.mark.gpu
+
+
+def _static_predict(lib, desc, h, L, idx, count):
+    st = lib.pi_predict_static(ctypes.byref(desc), h.shape[0], h.data_ptr(), L["P1"].data_ptr(),
+                               L["P2"].data_ptr(), L["bp"].data_ptr(), float(L["thr"]), idx.data_ptr(),
+                               count.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    assert st == B.PI_OK, lib.pi_last_error()
+
+
+def test_static_scratch_predict_matches_workspace_predict_twice():
+    lib = pi.lib()
+    wl = W.Workload("noalloc", 91, 1024, 3000, 1, "reglu", "f16", "f16", 0.88, 1.2, 0.1, 128, (2,), 2)
+    L = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in W.make_layer(wl, 0).items()}
+    desc = pi.desc_for(wl)
+    ws = pi.workspace(desc, 2)
+    C = wl.n_cold
+    for step in range(2):                      # two calls in a row, different token blocks
+        h = W.make_tokens(wl, 2, 50 + step, device="cuda")
+        idx_ref = torch.full((C,), -1, dtype=torch.int32, device="cuda")
+        cnt_ref = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+        pi.predict(desc, h, L["P1"], L["P2"], L["bp"], L["thr"], idx_ref, cnt_ref, ws)
+        idx = torch.full((C,), -2, dtype=torch.int32, device="cuda")
+        cnt = torch.full((1,), -2, dtype=torch.int32, device="cuda")
+        _static_predict(lib, desc, h, L, idx, cnt)
+        torch.cuda.synchronize()
+        n = int(cnt_ref.item())
+        assert 0 < n < C
+        assert int(cnt.item()) == n
+        assert torch.equal(idx[:n], idx_ref[:n])
+        assert np.all(np.diff(idx[:n].cpu().numpy()) > 0)
+
+
+def test_static_scratch_rejects_sizes_beyond_its_limit():
+    lib = pi.lib()
+    desc = pi.make_desc(1024, 40000, 0, 32768, "f16", "f16", "relu")   # 16 x 32768 x 4 B = 2 MiB of u
+    fake = ctypes.c_void_p(1 << 20)
+    st = lib.pi_predict_static(ctypes.byref(desc), 16, fake, fake, fake, None, 0.5, fake, fake, None)
+    assert st == B.PI_ERR_CAPACITY
+    assert b"1 MiB" in lib.pi_last_error()
