@@ -132,6 +132,9 @@ pi_status check_layer(const pi_ffn_desc* desc, const pi_layer_weights* w) {
   return PI_OK;
 }
 
+static_assert(pi::kYAccCopies == pi::kYCopies, "workspace layout and kernel agree on the accumulator copies");
+static_assert(pi::kGMax == pi::kGMaxCtas, "workspace layout and kernel agree on the largest grid");
+
 int stack_grid() {
   const int g = sm_count();
   return g < pi::kGMax ? g : pi::kGMax;
@@ -151,7 +154,7 @@ pi_status fused_params(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, pi:
   P.rank = desc->rank;
   P.act = desc->act;
   P.L = n_layers;
-  P.T = desc->d / 16;
+  P.T = desc->d / pi::stack_ept(desc->d);
   smem = pi::stack_smem_layout(P, B, G);
   if (smem == 0) return PI_ERR_UNSUPPORTED;
   const int ep = desc->ptype == PI_F16 ? 2 : 4;
@@ -164,6 +167,9 @@ pi_status fused_params(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, pi:
   if (neuron > half || p2item > half || p1item > half) return PI_ERR_UNSUPPORTED;
   const int C = desc->ffn - desc->n_hot;
   P.seg_cap = (C + G - 1) / G + 1;
+  // every consumer thread holds at most kShareRegs entries of the CTA's bias shares
+  if ((C + G - 1) / G > pi::kShareRegs * P.T || (desc->n_hot + G - 1) / G > pi::kShareRegs * P.T)
+    return PI_ERR_UNSUPPORTED;
   return PI_OK;
 }
 

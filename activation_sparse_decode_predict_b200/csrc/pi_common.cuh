@@ -26,9 +26,9 @@ struct Ctrl {
   int status;          // sticky: first device error wins
   int abort;           // set when any CTA of a persistent kernel gives up a wait
   int pad0[30];
-  unsigned bar_count;  // grid barrier arrivals (own 64-byte line)
+  unsigned bar_count;  // grid barrier arrivals, monotonic (own 64-byte line)
   unsigned pad1[15];
-  unsigned bar_gen;    // grid barrier generation (own 64-byte line)
+  unsigned bar_base;   // bar_count at the start of the next persistent launch
   unsigned pad2[15];
 };
 static_assert(sizeof(Ctrl) == 256, "control block is 256 bytes");

@@ -2,7 +2,7 @@
 //
 //   [ctrl 256 B][u: B x rank fp32][tile masks][tile counts][a: B x ffn fp32]
 //   [partials: G_MAX x B x d fp32][y: B x d fp32][h: B x d fp32]
-//   [y accumulators: 2 x B x d fp32][per-CTA active lists][per-CTA counts]
+//   [y accumulators: 2 x 8 x B x d fp32][per-CTA active lists][per-CTA counts]
 //
 // Every region starts on a 256-byte boundary.  The layout depends only on the
 // descriptor and the batch, never on the device.
@@ -13,6 +13,7 @@
 namespace pi {
 
 constexpr int kGMax = 296;  // split-K partial slots (2 x 148 SMs)
+constexpr int kYAccCopies = 8;  // copies of the persistent kernel's fp32 output accumulator
 
 struct WsLayout {
   size_t u, tile_mask, tile_count, act, partial, ybuf, hbuf, yacc, seg, seg_cnt, total;
@@ -34,7 +35,7 @@ inline WsLayout ws_layout(int d, int ffn, int n_hot, int rank, int B) {
   L.partial = off; off += align256((size_t)kGMax * B * d * 4);
   L.ybuf = off; off += align256((size_t)B * d * 4);
   L.hbuf = off; off += align256((size_t)B * d * 4);
-  L.yacc = off; off += align256((size_t)2 * B * d * 4);
+  L.yacc = off; off += align256((size_t)2 * kYAccCopies * B * d * 4);
   L.seg = off; off += align256((size_t)(C + 2 * kGMax) * 4);
   L.seg_cnt = off; off += align256((size_t)kGMax * 4);
   L.total = off;

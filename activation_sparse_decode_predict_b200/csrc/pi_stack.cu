@@ -42,13 +42,16 @@ namespace {
 // column ownership: consumer thread t of T owns 16 columns of d, as NRUN runs
 // of RUN consecutive columns whose layout follows the weight type.
 
-template <int WT>
+template <int WT, int EPT>
 struct Own {
-  static constexpr int RUN = (WT == kF32) ? 4 : 8;
-  static constexpr int NRUN = 16 / RUN;
+  static_assert(EPT == 8 || EPT == 16, "8 or 16 columns per thread");
+  static constexpr int RUN = (WT == kF32) ? 4 : (WT == kQ4_0 ? EPT / 2 : 8);
+  static constexpr int NRUN = EPT / RUN;
   __device__ __forceinline__ static int col(int t, int T, int k) {
     if constexpr (WT == kQ4_0) {
-      return (t >> 1) * 32 + (t & 1) * 8 + k * 16;
+      // EPT/2 bytes of one Q4_0 block: low nibbles give a run, high nibbles the run 16 columns on
+      constexpr int PER_BLK = 32 / EPT;  // threads per 32-column block
+      return (t / PER_BLK) * 32 + (t % PER_BLK) * (EPT / 2) + k * 16;
     } else {
       return (t + k * T) * RUN;
     }
@@ -56,9 +59,9 @@ struct Own {
 };
 
 // 16 owned values of a d-row of element type X (kF32/kF16) at `row` (shared or global).
-template <int WT, int X>
-__device__ __forceinline__ void row_vals(const uint8_t* row, int t, int T, float (&v)[16]) {
-  using O = Own<WT>;
+template <int WT, int EPT, int X>
+__device__ __forceinline__ void row_vals(const uint8_t* row, int t, int T, float (&v)[EPT]) {
+  using O = Own<WT, EPT>;
 #pragma unroll
   for (int k = 0; k < O::NRUN; ++k) {
     const int c = O::col(t, T, k);
@@ -87,30 +90,42 @@ __device__ __forceinline__ void row_vals(const uint8_t* row, int t, int T, float
   }
 }
 
-// 16 owned values of a Q4_0 row laid out as [qs d/2 bytes][sc d/16 bytes].
-__device__ __forceinline__ void q4_vals(const uint8_t* row, int d, int t, float (&v)[16]) {
-  const uint2 q = *reinterpret_cast<const uint2*>(row + 8 * t);
-  const uint16_t sb = *reinterpret_cast<const uint16_t*>(row + d / 2 + 2 * (t >> 1));
+// EPT owned values of a Q4_0 row laid out as [qs d/2 bytes][sc d/16 bytes]:
+// EPT/2 consecutive qs bytes of one block; their low nibbles are the first
+// run, their high nibbles the run 16 columns on; x = s * (q - 8).
+template <int EPT>
+__device__ __forceinline__ void q4_vals(const uint8_t* row, int d, int t, float (&v)[EPT]) {
+  constexpr int NB = EPT / 2;         // qs bytes per thread
+  constexpr int PER_BLK = 32 / EPT;   // threads per block
+  uint32_t q[NB / 4];
+  if constexpr (NB == 8) {
+    const uint2 qq = *reinterpret_cast<const uint2*>(row + NB * t);
+    q[0] = qq.x;
+    q[1] = qq.y;
+  } else {
+    q[0] = *reinterpret_cast<const uint32_t*>(row + NB * t);
+  }
+  const uint16_t sb = *reinterpret_cast<const uint16_t*>(row + d / 2 + 2 * (t / PER_BLK));
   const float s = half_bits_to_float(sb);
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const uint32_t b0 = (q.x >> (8 * k)) & 0xffu, b1 = (q.y >> (8 * k)) & 0xffu;
-    v[k] = s * (float)((int)(b0 & 15u) - 8);
-    v[4 + k] = s * (float)((int)(b1 & 15u) - 8);
-    v[8 + k] = s * (float)((int)(b0 >> 4) - 8);
-    v[12 + k] = s * (float)((int)(b1 >> 4) - 8);
-  }
+  for (int w = 0; w < NB / 4; ++w)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t b = (q[w] >> (8 * k)) & 0xffu;
+      v[w * 4 + k] = s * (float)((int)(b & 15u) - 8);
+      v[NB + w * 4 + k] = s * (float)((int)(b >> 4) - 8);
+    }
 }
 
-template <int WT>
-__device__ __forceinline__ void w_vals(const uint8_t* row, int d, int t, int T, float (&v)[16]) {
-  if constexpr (WT == kQ4_0) q4_vals(row, d, t, v);
-  else row_vals<WT, WT>(row, t, T, v);
+template <int WT, int EPT>
+__device__ __forceinline__ void w_vals(const uint8_t* row, int d, int t, int T, float (&v)[EPT]) {
+  if constexpr (WT == kQ4_0) q4_vals<EPT>(row, d, t, v);
+  else row_vals<WT, EPT, WT>(row, t, T, v);
 }
 
-template <int WT, int X>
-__device__ __forceinline__ void store_vals(uint8_t* row, int t, int T, const float (&v)[16]) {
-  using O = Own<WT>;
+template <int WT, int EPT, int X>
+__device__ __forceinline__ void store_vals(uint8_t* row, int t, int T, const float (&v)[EPT]) {
+  using O = Own<WT, EPT>;
 #pragma unroll
   for (int k = 0; k < O::NRUN; ++k) {
     const int c = O::col(t, T, k);
@@ -150,7 +165,6 @@ struct Smem {
   uint64_t* list_bar;
   uint32_t* item_off;
   uint32_t* istart;  // producer-private: start/size of the items in flight
-  uint32_t* isize;
   float* u;          // [B][r] split layout (see load_u)
   float* bp;
   float* b1hot;
@@ -170,7 +184,6 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const StackParams& p) {
   s.list_bar = s.empty + kNQ;
   s.item_off = reinterpret_cast<uint32_t*>(base + p.off_itemoff);
   s.istart = s.item_off + kNQ;
-  s.isize = s.istart + kNQ;
   s.u = reinterpret_cast<float*>(base + p.off_u);
   s.bp = reinterpret_cast<float*>(base + p.off_bp);
   s.b1hot = reinterpret_cast<float*>(base + p.off_b1hot);
@@ -186,7 +199,7 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const StackParams& p) {
 __device__ __forceinline__ int share_lo(int n, int c, int G) { return (int)((int64_t)n * c / G); }
 
 // CTA-wide (consumer warps) sum of NV values per thread; every thread gets the
-// totals, added in the same warp order.  The two scratch buffers alternate
+// same totals (same butterfly order in every warp).  The two scratch buffers alternate
 // (stride MAXV per warp) so that the next call's writes cannot overtake this
 // call's reads.  Returns the OR of `flag` over the consumer threads.
 template <int NV, int MAXV>
@@ -200,10 +213,12 @@ __device__ __forceinline__ bool cta_reduce(float (&v)[NV], float* red_base, int&
     for (int i = 0; i < NV; ++i) red[warp * MAXV + i] = v[i];
   }
   flag = named_sync_or(1, T, flag);
+  // lane w reads warp w's partial; a butterfly gives every lane the total
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
-    float a = 0.f;
-    for (int w = 0; w < NW; ++w) a += red[w * MAXV + i];
+    float a = lane < NW ? red[lane * MAXV + i] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
     v[i] = a;
   }
   par ^= 1;
@@ -220,7 +235,6 @@ struct Producer {
   uint32_t item = 0;  // next item index
   uint32_t rel = 0;   // items known consumed
   uint32_t head = 0;  // next free ring byte
-  bool ok = true;
 
   __device__ Producer(const StackParams& p_, Smem& s_) : p(p_), s(s_), ctrl(p_.ctrl) {}
 
@@ -264,7 +278,6 @@ struct Producer {
     const uint32_t q = item % kNQ;
     s.item_off[q] = pos;
     s.istart[q] = pos;
-    s.isize[q] = total;
     mbar_arrive_expect_tx(&s.full[q], total);
     uint32_t o = pos;
     for (int i = 0; i < nseg; ++i) {
@@ -307,7 +320,7 @@ struct Producer {
 
 // ----------------------------------------------------------------------------
 
-template <int WT, int PT, int B>
+template <int WT, int PT, int B, int EPT>
 __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_constant__ StackParams p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   Smem s = carve(smem_raw, p);
@@ -317,6 +330,7 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
   const int d = p.d, r = p.rank, H = p.n_hot, C = p.ffn - p.n_hot;
   const int gated = p.act == kReglu;
   const int ep = PT == kF16 ? 2 : 4;
+  constexpr int K = kYCopies;
 
   if (threadIdx.x == 0) {
     for (int q = 0; q < kNQ; ++q) {
@@ -325,10 +339,10 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
     }
     mbar_init(s.list_bar, 1);
     mbar_fence_init();
-    s.misc[1] = (int)ld_acquire_u32(&ctrl->bar_gen);
+    s.misc[1] = (int)ld_acquire_u32(&ctrl->bar_base);
   }
   __syncthreads();
-  const unsigned gen0 = (unsigned)s.misc[1];
+  const unsigned base = (unsigned)s.misc[1];
 
   // shares that do not depend on the predictor
   const int k0 = share_lo(r, c, G), k1 = share_lo(r, c + 1, G);
@@ -356,24 +370,30 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
         }
         for (int j = j0; j < j1 && ok; ++j) ok = pr.issue_neuron(Ly, j, WT, gated);
         // the cold rows need every CTA's scores: barrier S of this layer
-        if (ok) ok = grid_wait(ctrl, gen0, 3 * l + 1);
+        if (ok) ok = grid_wait(ctrl, base, 3 * l + 1, G);
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       __syncwarp();
       if (!ok) break;
-      // cold list: prefix over the per-CTA counts, then this CTA's share
-      for (int i = lane; i <= G; i += 32) s.prefix[i] = 0;
-      __syncwarp();
+      // prefix over the per-CTA counts (all loads in flight at once)
+      constexpr int kMaxChunks = (kGMaxCtas + 31) / 32;
+      int cv[kMaxChunks];
+#pragma unroll 1
+      for (int m = 0; m < kMaxChunks; ++m) {
+        const int i = m * 32 + lane;
+        cv[m] = i < G ? __ldcg(p.seg_cnt + i) : 0;
+      }
+      if (lane == 0) s.prefix[0] = 0;
       int run = 0;
-      for (int base = 0; base < G; base += 32) {
-        const int i = base + lane;
-        int v = i < G ? __ldcg(p.seg_cnt + i) : 0;
-        int x = v;
+#pragma unroll 1
+      for (int m = 0; m < kMaxChunks; ++m) {
+        int x = cv[m];
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const int y = __shfl_up_sync(0xffffffffu, x, o);
           if (lane >= o) x += y;
         }
+        const int i = m * 32 + lane;
         if (i < G) s.prefix[i + 1] = run + x;
         run += __shfl_sync(0xffffffffu, x, 31);
       }
@@ -381,21 +401,14 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
       const int A = run;
       const int q0 = share_lo(A, c, G), q1 = share_lo(A, c + 1, G);
       for (int q = q0 + lane; q < q1; q += 32) {
-        int lo = 0, hi = G;  // last cta with prefix[cta] <= q
+        int lo = 0, hi = G;  // last CTA with prefix[cta] <= q
         while (hi - lo > 1) {
           const int mid = (lo + hi) >> 1;
           if (s.prefix[mid] <= q) lo = mid;
           else hi = mid;
         }
-        const int j = __ldcg(p.seg + (int64_t)lo * p.seg_cap + (q - s.prefix[lo]));
-        s.cidx[q - q0] = j;
-        s.cb1[q - q0] = Ly.b1 ? __ldg(Ly.b1 + j) : 0.f;
+        s.cidx[q - q0] = __ldcg(p.seg + (int64_t)lo * p.seg_cap + (q - s.prefix[lo]));
       }
-      // outputs: this CTA's segment of the ascending list, and the count
-      const int my_n = s.prefix[c + 1] - s.prefix[c];
-      for (int i = lane; i < my_n; i += 32)
-        p.idx[(int64_t)l * C + s.prefix[c] + i] = __ldcg(p.seg + (int64_t)c * p.seg_cap + i);
-      if (c == 0 && lane == 0) p.counts[l] = A;
       if (lane == 0) s.misc[0] = q1 - q0;
       __syncwarp();
       if (lane == 0) {
@@ -403,6 +416,12 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
         for (int q = 0; q < q1 - q0 && ok; ++q) ok = pr.issue_neuron(Ly, s.cidx[q], WT, gated);
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
+      // outputs (off the critical path): this CTA's part of the ascending list, and the count
+      const int my_n = s.prefix[c + 1] - s.prefix[c];
+      for (int i = lane; i < my_n; i += 32)
+        p.idx[(int64_t)l * C + s.prefix[c] + i] = __ldcg(p.seg + (int64_t)c * p.seg_cap + i);
+      if (c == 0 && lane == 0) p.counts[l] = A;
+      __syncwarp();
     }
     if (lane == 0) pr.drain();
     return;
@@ -411,78 +430,97 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
   // ======================= consumer warps =======================
   const int t = threadIdx.x - 32;
   const int warp = t >> 5, lane = t & 31;
-  uint32_t item = 0;
+  uint32_t witem = 0, ritem = 0;  // next item to wait for / to release
   int par = 0;
-  float h[B][16], y[B][16];
-  bool bad = false;
-
-  // layer-0 input
-#pragma unroll
-  for (int b = 0; b < B; ++b)
-    row_vals<WT, PT>(reinterpret_cast<const uint8_t*>(p.h_in) + (int64_t)b * d * ep, t, T, h[b]);
-  if (c == 0 && p.h_trace) {
-#pragma unroll
-    for (int b = 0; b < B; ++b) store_vals<WT, PT>(reinterpret_cast<uint8_t*>(p.h_trace) + (int64_t)b * d * ep, t, T, h[b]);
-  }
-  // zero this CTA's slice of the layer-0 accumulator
-  {
-    const int n4 = B * d / 4;
-    const int z0 = share_lo(n4, c, G), z1 = share_lo(n4, c + 1, G);
-    for (int i = z0 + t; i < z1; i += T) reinterpret_cast<float4*>(p.yacc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
+  float h[B][EPT], y[B][EPT];
 
   auto wait_item = [&](uint32_t& off) -> bool {
-    const uint32_t q = item % kNQ;
-    const bool okw = mbar_wait(&s.full[q], (item / kNQ) & 1u, ctrl);
+    const uint32_t q = witem % kNQ;
+    const bool okw = mbar_wait(&s.full[q], (witem / kNQ) & 1u, ctrl);
     off = s.item_off[q];
+    ++witem;
     return okw;
   };
   auto release_item = [&]() {
     __syncwarp();
-    if (lane == 0) mbar_arrive(&s.empty[item % kNQ]);
-    ++item;
+    if (lane == 0) mbar_arrive(&s.empty[ritem % kNQ]);
+    ++ritem;
   };
 
+  // layer-0 input
+#pragma unroll
+  for (int b = 0; b < B; ++b)
+    row_vals<WT, EPT, PT>(reinterpret_cast<const uint8_t*>(p.h_in) + (int64_t)b * d * ep, t, T, h[b]);
+  if (c == 0 && p.h_trace) {
+#pragma unroll
+    for (int b = 0; b < B; ++b) store_vals<WT, EPT, PT>(reinterpret_cast<uint8_t*>(p.h_trace) + (int64_t)b * d * ep, t, T, h[b]);
+  }
+  const int ybuf4 = K * B * d / 4;  // float4s per accumulator buffer (K copies)
+  {
+    const int z0 = share_lo(ybuf4, c, G), z1 = share_lo(ybuf4, c + 1, G);
+    for (int i = z0 + t; i < z1; i += T) reinterpret_cast<float4*>(p.yacc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 
   for (int l = 0; l < p.L; ++l) {
     const StackLayer& Ly = p.layers[l];
-    // small per-layer vectors of this CTA's shares
-    for (int x = t; x < c1 - c0; x += T) s.bp[x] = Ly.bp ? __ldg(Ly.bp + c0 + x) : 0.f;
-    for (int x = t; x < j1 - j0; x += T) s.b1hot[x] = Ly.b1 ? __ldg(Ly.b1 + j0 + x) : 0.f;
-
-    // ---- predictor step 1: u = ReLU(P1 h) for this CTA's rows ----
-    for (int k = k0; k < k1; ++k) {
-      uint32_t off;
-      bool to = !wait_item(off);
-      float w[16];
-      row_vals<WT, PT>(s.ring + off, t, T, w);
-      float acc[B];
+    // small per-layer vectors of this CTA's shares: loaded now, stored to
+    // shared memory after the P1 rows so that the load latency is hidden
+    float bp_v[kShareRegs], b1_v[kShareRegs];
 #pragma unroll
-      for (int b = 0; b < B; ++b) {
-        float a = 0.f;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) a = fmaf(w[e], h[b][e], a);
-        acc[b] = a;
-      }
-      release_item();
-      to = cta_reduce<B, 2 * B>(acc, s.red, par, warp, lane, NW, T, to);
-      if (to) { bad = true; break; }
-      if (t == 0)
-        for (int b = 0; b < B; ++b) p.u_g[(int64_t)b * r + k] = fmaxf(acc[b], 0.f);
+    for (int i = 0; i < kShareRegs; ++i) {
+      const int x = t + i * T;
+      bp_v[i] = (Ly.bp && x < c1 - c0) ? __ldg(Ly.bp + c0 + x) : 0.f;
+      b1_v[i] = (Ly.b1 && x < j1 - j0) ? __ldg(Ly.b1 + j0 + x) : 0.f;
     }
-    if (named_sync_or(1, T, bad)) return;
-    if (t == 0) grid_arrive(ctrl, G);
+
+    // ---- predictor step 1: u = ReLU(P1 h), up to 4 rows per CTA-wide reduction ----
+    bool to = false;
+    for (int kk = k0; kk < k1; kk += 4) {
+      const int nrow = min(4, k1 - kk);
+      float acc[4 * B];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int b = 0; b < B; ++b) acc[i * B + b] = 0.f;
+        if (i < nrow) {
+          uint32_t off;
+          to |= !wait_item(off);
+          float w[EPT];
+          row_vals<WT, EPT, PT>(s.ring + off, t, T, w);
+          release_item();
+#pragma unroll
+          for (int b = 0; b < B; ++b) {
+            float a = 0.f;
+#pragma unroll
+            for (int e = 0; e < EPT; ++e) a = fmaf(w[e], h[b][e], a);
+            acc[i * B + b] = a;
+          }
+        }
+      }
+      to = cta_reduce<4 * B, 4 * B>(acc, s.red, par, warp, lane, NW, T, to);
+      if (to) return;
+      if (t == 0)
+        for (int i = 0; i < nrow; ++i)
+          for (int b = 0; b < B; ++b) p.u_g[(int64_t)b * r + kk + i] = fmaxf(acc[i * B + b], 0.f);
+    }
+#pragma unroll
+    for (int i = 0; i < kShareRegs; ++i) {
+      const int x = t + i * T;
+      if (x < c1 - c0) s.bp[x] = bp_v[i];
+      if (x < j1 - j0) s.b1hot[x] = b1_v[i];
+    }
+    named_sync(1, T);
+    if (t == 0) grid_arrive(ctrl);
     {
       bool okw = true;
-      if (t == 0) okw = grid_wait(ctrl, gen0, 3 * l);
+      if (t == 0) okw = grid_wait(ctrl, base, 3 * l, G);
       if (named_sync_or(1, T, !okw)) return;
     }
-    // next layer's accumulator slice is free now (its last readers passed this barrier)
+    // the other accumulator buffer is free now (its last readers passed this barrier)
     {
-      float* nxt = p.yacc + (size_t)((l + 1) & 1) * B * d;
-      const int n4 = B * d / 4;
-      const int z0 = share_lo(n4, c, G), z1 = share_lo(n4, c + 1, G);
-      for (int i = z0 + t; i < z1; i += T) reinterpret_cast<float4*>(nxt)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      float4* nxt = reinterpret_cast<float4*>(p.yacc) + (size_t)((l + 1) & 1) * ybuf4;
+      const int z0 = share_lo(ybuf4, c, G), z1 = share_lo(ybuf4, c + 1, G);
+      for (int i = z0 + t; i < z1; i += T) nxt[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     // u -> shared memory, split layout: unit m (8 values) stored as two float4
     // planes so that lane-strided reads are conflict-free.
@@ -499,18 +537,63 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
     }
     named_sync(1, T);
 
-    // ---- predictor step 2: scores of this CTA's cold rows ----
+    // ---- predictor step 2: scores of this CTA's cold rows (warp per row) ----
     {
       const int nu = r / 8;  // 8-element units per row (r % 8 == 0)
+      // single token and rank <= 1024: this lane's slice of u stays in registers
+      float ureg[4][8];
+      const bool u_in_regs = (B == 1) && nu <= 128;
+      if (u_in_regs) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int m = lane + 32 * i;
+          float4 lo = make_float4(0.f, 0.f, 0.f, 0.f), hi = lo;
+          if (m < nu) {
+            lo = reinterpret_cast<const float4*>(s.u)[m];
+            hi = reinterpret_cast<const float4*>(s.u)[nu + m];
+          }
+          ureg[i][0] = lo.x; ureg[i][1] = lo.y; ureg[i][2] = lo.z; ureg[i][3] = lo.w;
+          ureg[i][4] = hi.x; ureg[i][5] = hi.y; ureg[i][6] = hi.z; ureg[i][7] = hi.w;
+        }
+      }
       for (int cc = c0; cc < c1; cc += NW) {
         const int rows = min(NW, c1 - cc);
         uint32_t off;
-        bool to = !wait_item(off);
+        to |= !wait_item(off);
         if (warp < rows) {
           const uint8_t* row = s.ring + off + (size_t)warp * r * ep;
           float acc[B];
 #pragma unroll
           for (int b = 0; b < B; ++b) acc[b] = 0.f;
+          if (u_in_regs) {
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int m = lane + 32 * i;
+              if (m < nu) {
+                float w[8];
+                if constexpr (PT == kF16) {
+                  const uint4 q = *reinterpret_cast<const uint4*>(row + 16 * m);
+                  float2 f;
+                  f = h2f2(q.x); w[0] = f.x; w[1] = f.y;
+                  f = h2f2(q.y); w[2] = f.x; w[3] = f.y;
+                  f = h2f2(q.z); w[4] = f.x; w[5] = f.y;
+                  f = h2f2(q.w); w[6] = f.x; w[7] = f.y;
+                } else {
+                  const float4 a = *reinterpret_cast<const float4*>(row + 32 * m);
+                  const float4 b2 = *reinterpret_cast<const float4*>(row + 32 * m + 16);
+                  w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+                  w[4] = b2.x; w[5] = b2.y; w[6] = b2.z; w[7] = b2.w;
+                }
+                a0 = fmaf(w[0], ureg[i][0], a0); a1 = fmaf(w[1], ureg[i][1], a1);
+                a0 = fmaf(w[2], ureg[i][2], a0); a1 = fmaf(w[3], ureg[i][3], a1);
+                a0 = fmaf(w[4], ureg[i][4], a0); a1 = fmaf(w[5], ureg[i][5], a1);
+                a0 = fmaf(w[6], ureg[i][6], a0); a1 = fmaf(w[7], ureg[i][7], a1);
+              }
+            }
+            acc[0] = a0 + a1;
+          } else
+#pragma unroll 2
           for (int m = lane; m < nu; m += 32) {
             float w[8];
             if constexpr (PT == kF16) {
@@ -543,94 +626,129 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
           if (lane == 0) s.act[cc - c0 + warp] = on ? 1 : 0;
         }
         release_item();
-        if (named_sync_or(1, T, to)) return;
       }
     }
-    named_sync(1, T);
+    if (named_sync_or(1, T, to)) return;
     // local ascending list of this CTA's active cold rows (consumer warp 0)
     if (warp == 0) {
-      int base = 0;
+      int cnt = 0;
       for (int x0 = 0; x0 < c1 - c0; x0 += 32) {
         const int x = x0 + lane;
         const bool on = x < c1 - c0 && s.act[x];
         const unsigned m = __ballot_sync(0xffffffffu, on);
-        if (on) p.seg[(int64_t)c * p.seg_cap + base + __popc(m & ((1u << lane) - 1u))] = H + c0 + x;
-        base += __popc(m);
+        if (on) p.seg[(int64_t)c * p.seg_cap + cnt + __popc(m & ((1u << lane) - 1u))] = H + c0 + x;
+        cnt += __popc(m);
       }
-      if (lane == 0) p.seg_cnt[c] = base;
-      __threadfence();
+      if (lane == 0) p.seg_cnt[c] = cnt;
       __syncwarp();
-      if (lane == 0) grid_arrive(ctrl, G);
+      if (lane == 0) grid_arrive(ctrl);
     }
 
-    // ---- sparse FFN: hot share, then cold share ----
+    // ---- sparse FFN: hot share, then cold share, two neurons in flight ----
 #pragma unroll
     for (int b = 0; b < B; ++b)
 #pragma unroll
-      for (int e = 0; e < 16; ++e) y[b][e] = 0.f;
+      for (int e = 0; e < EPT; ++e) y[b][e] = 0.f;
     const int wrb = wrow_bytes(WT, d);
-    auto neuron = [&](float bias, bool& to) {
+    const int nh = j1 - j0;
+    int n = nh;
+    bool have_list = false;
+    uint32_t itoff0 = 0u, itoff1 = 0u;
+    float* nred = s.red + 2 * (kMaxConsumers / 32) * (4 * B);  // neuron scratch: [2][NW][2B]
+    // dots of neuron k -> per-warp partial sums in nred[k & 1]
+    auto prepare = [&](int k) {
       uint32_t off;
       to |= !wait_item(off);
+      if (k & 1) itoff1 = off;
+      else itoff0 = off;
       const uint8_t* it = s.ring + off;
       float acc[2 * B];
-      {
-        float wu[16];
-        w_vals<WT>(it + (gated ? wrb : 0), d, t, T, wu);
+      float wu[EPT];
+      w_vals<WT, EPT>(it + (gated ? wrb : 0), d, t, T, wu);
 #pragma unroll
-        for (int b = 0; b < B; ++b) {
-          float a = 0.f;
+      for (int b = 0; b < B; ++b) {
+        float a = 0.f;
 #pragma unroll
-          for (int e = 0; e < 16; ++e) a = fmaf(wu[e], h[b][e], a);
-          acc[B + b] = a;
-        }
+        for (int e = 0; e < EPT; ++e) a = fmaf(wu[e], h[b][e], a);
+        acc[B + b] = a;
       }
       if (gated) {
-        float wg[16];
-        w_vals<WT>(it, d, t, T, wg);
+        float wg[EPT];
+        w_vals<WT, EPT>(it, d, t, T, wg);
 #pragma unroll
         for (int b = 0; b < B; ++b) {
           float a = 0.f;
 #pragma unroll
-          for (int e = 0; e < 16; ++e) a = fmaf(wg[e], h[b][e], a);
+          for (int e = 0; e < EPT; ++e) a = fmaf(wg[e], h[b][e], a);
           acc[b] = a;
         }
       } else {
 #pragma unroll
         for (int b = 0; b < B; ++b) acc[b] = 0.f;
       }
-      to = cta_reduce<2 * B, 2 * B>(acc, s.red, par, warp, lane, NW, T, to);
+#pragma unroll
+      for (int i = 0; i < 2 * B; ++i) acc[i] = warp_sum(acc[i]);
+      float* red = nred + (k & 1) * (kMaxConsumers / 32) * (2 * B);
+      if (lane == 0) {
+#pragma unroll
+        for (int i = 0; i < 2 * B; ++i) red[warp * 2 * B + i] = acc[i];
+      }
+    };
+    // activation and down-row accumulation of neuron k (after its barrier)
+    auto finish = [&](int k) {
+      const float* red = nred + (k & 1) * (kMaxConsumers / 32) * (2 * B);
+      float tot[2 * B];
+#pragma unroll
+      for (int i = 0; i < 2 * B; ++i) {
+        float v = lane < NW ? red[lane * 2 * B + i] : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        tot[i] = v;
+      }
+      const float bias = k < nh ? s.b1hot[k] : s.cb1[k - nh];
       float a[B];
 #pragma unroll
-      for (int b = 0; b < B; ++b) a[b] = gated ? act_eval(kReglu, acc[b] + bias, acc[B + b]) : act_eval(p.act, acc[B + b] + bias, 0.f);
-      float wd[16];
-      w_vals<WT>(it + (gated ? 2 : 1) * wrb, d, t, T, wd);
+      for (int b = 0; b < B; ++b)
+        a[b] = gated ? act_eval(kReglu, tot[b] + bias, tot[B + b]) : act_eval(p.act, tot[B + b] + bias, 0.f);
+      float wd[EPT];
+      w_vals<WT, EPT>(s.ring + ((k & 1) ? itoff1 : itoff0) + (gated ? 2 : 1) * wrb, d, t, T, wd);
       release_item();
 #pragma unroll
       for (int b = 0; b < B; ++b)
 #pragma unroll
-        for (int e = 0; e < 16; ++e) y[b][e] = fmaf(a[b], wd[e], y[b][e]);
+        for (int e = 0; e < EPT; ++e) y[b][e] = fmaf(a[b], wd[e], y[b][e]);
     };
-    for (int j = j0; j < j1; ++j) {
-      bool to = false;
-      neuron(s.b1hot[j - j0], to);
-      if (to) return;
-    }
-    {
+    // the cold list (and its biases) from the producer
+    auto take_list = [&]() -> bool {
       const bool okw = mbar_wait(s.list_bar, l & 1, ctrl);
-      if (named_sync_or(1, T, !okw)) return;
+      if (named_sync_or(1, T, !okw)) return false;
+      const int ncold = s.misc[0];
+      for (int x = t; x < ncold; x += T) s.cb1[x] = Ly.b1 ? __ldg(Ly.b1 + s.cidx[x]) : 0.f;
+      n = nh + ncold;
+      have_list = true;
+      return true;
+    };
+    if (nh == 0) {
+      if (!take_list()) return;
+      named_sync(1, T);  // cb1 visible
     }
-    const int ncold = s.misc[0];
-    for (int q = 0; q < ncold; ++q) {
-      bool to = false;
-      neuron(s.cb1[q], to);
-      if (to) return;
+    if (n > 0) prepare(0);
+    for (int k = 0; k < n; ++k) {
+      if (named_sync_or(1, T, to)) return;  // neuron k's partial sums are complete
+      if (k + 1 == nh && !have_list) {
+        if (!take_list()) return;  // cb1 becomes visible at the next neuron's barrier
+      }
+      if (k + 1 < n) prepare(k + 1);
+      finish(k);
+    }
+    if (!have_list) {  // (nh > 0 and the loop ended before the list: cannot happen, kept for safety)
+      if (!take_list()) return;
     }
 
-    // ---- split-K: add the partial into the fp32 accumulator ----
+    // ---- split-K: add the partial into one of K fp32 accumulator copies ----
     {
-      float* acc = p.yacc + (size_t)(l & 1) * B * d;
-      using O = Own<WT>;
+      float* acc = p.yacc + ((size_t)(l & 1) * K + (c % K)) * B * d;
+      using O = Own<WT, EPT>;
 #pragma unroll
       for (int b = 0; b < B; ++b)
 #pragma unroll
@@ -642,54 +760,60 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
                       make_float4(y[b][k * O::RUN + e], y[b][k * O::RUN + e + 1], y[b][k * O::RUN + e + 2],
                                   y[b][k * O::RUN + e + 3]));
         }
-      __threadfence();
     }
     named_sync(1, T);
-    if (t == 0) grid_arrive(ctrl, G);
+    if (t == 0) grid_arrive(ctrl);
     {
       bool okw = true;
-      if (t == 0) okw = grid_wait(ctrl, gen0, 3 * l + 2);
+      if (t == 0) okw = grid_wait(ctrl, base, 3 * l + 2, G);
       if (named_sync_or(1, T, !okw)) return;
     }
 
     // ---- glue: h <- RMSNorm(h + y + b2), rounded to the token type ----
     {
-      const float* acc = p.yacc + (size_t)(l & 1) * B * d;
-      using O = Own<WT>;
+      const float* acc = p.yacc + (size_t)(l & 1) * K * B * d;
+      using O = Own<WT, EPT>;
       float ss[B];
 #pragma unroll
       for (int b = 0; b < B; ++b) {
-        float yv[16];
+        float yv[EPT];
 #pragma unroll
         for (int k = 0; k < O::NRUN; ++k) {
           const int col = O::col(t, T, k);
 #pragma unroll
           for (int e = 0; e < O::RUN; e += 4) {
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(acc + (size_t)b * d + col + e));
             float4 bb = make_float4(0.f, 0.f, 0.f, 0.f);
             if (Ly.b2) bb = __ldg(reinterpret_cast<const float4*>(Ly.b2 + col + e));
-            yv[k * O::RUN + e] = v.x + bb.x;
-            yv[k * O::RUN + e + 1] = v.y + bb.y;
-            yv[k * O::RUN + e + 2] = v.z + bb.z;
-            yv[k * O::RUN + e + 3] = v.w + bb.w;
+            float4 v[K];
+#pragma unroll
+            for (int q = 0; q < K; ++q)
+              v[q] = __ldcg(reinterpret_cast<const float4*>(acc + ((size_t)q * B + b) * d + col + e));
+#pragma unroll
+            for (int q = 0; q < K; ++q) {
+              bb.x += v[q].x; bb.y += v[q].y; bb.z += v[q].z; bb.w += v[q].w;
+            }
+            yv[k * O::RUN + e] = bb.x;
+            yv[k * O::RUN + e + 1] = bb.y;
+            yv[k * O::RUN + e + 2] = bb.z;
+            yv[k * O::RUN + e + 3] = bb.w;
           }
         }
-        if (c == 0 && p.y_out) store_vals<WT, kF32>(reinterpret_cast<uint8_t*>(p.y_out + ((size_t)l * B + b) * d), t, T, yv);
+        if (c == 0 && p.y_out) store_vals<WT, EPT, kF32>(reinterpret_cast<uint8_t*>(p.y_out + ((size_t)l * B + b) * d), t, T, yv);
         float a = 0.f;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
+        for (int e = 0; e < EPT; ++e) {
           const float x = h[b][e] + yv[e];
           h[b][e] = x;
           a = fmaf(x, x, a);
         }
         ss[b] = a;
       }
-      cta_reduce<B, 2 * B>(ss, s.red, par, warp, lane, NW, T, false);
+      cta_reduce<B, 4 * B>(ss, s.red, par, warp, lane, NW, T, false);
 #pragma unroll
       for (int b = 0; b < B; ++b) {
         const float inv = rsqrtf(ss[b] / (float)d + p.eps);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) h[b][e] = round_to(PT, h[b][e] * inv);
+        for (int e = 0; e < EPT; ++e) h[b][e] = round_to(PT, h[b][e] * inv);
       }
       if (c == 0) {
         uint8_t* dst = nullptr;
@@ -700,16 +824,18 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
         }
         if (dst) {
 #pragma unroll
-          for (int b = 0; b < B; ++b) store_vals<WT, PT>(dst + (size_t)b * d * ep, t, T, h[b]);
+          for (int b = 0; b < B; ++b) store_vals<WT, EPT, PT>(dst + (size_t)b * d * ep, t, T, h[b]);
         }
       }
     }
   }
+  // every CTA has passed the last barrier: leave the count base for the next launch
+  if (c == 0 && t == 0) atomicExch(&ctrl->bar_base, base + (unsigned)(3 * p.L * G));
 }
 
-template <int WT, int PT, int B>
+template <int WT, int PT, int B, int EPT>
 cudaError_t launch_t(const StackParams& p, int G, size_t smem, cudaStream_t st) {
-  auto fn = k_stack<WT, PT, B>;
+  auto fn = k_stack<WT, PT, B, EPT>;
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -731,11 +857,17 @@ cudaError_t launch_t(const StackParams& p, int G, size_t smem, cudaStream_t st) 
 
 }  // namespace
 
+int stack_ept(int d) { return (d % 256 == 0 && d / 8 <= kMaxConsumers) ? 8 : 16; }
+
 bool stack_supported(int wtype, int ptype, int d, int ffn, int n_hot, int rank, int B, int L) {
   if (B < 1 || B > 2) return false;
   if (L < 1 || L > kMaxLayers) return false;
-  if (d % 512 != 0 || d / 16 > kMaxConsumers) return false;
-  if (wtype == kQ4_0 && ptype != kF16 && ptype != kF32) return false;
+  const bool combo = (wtype == kF16 && ptype == kF16) || (wtype == kQ4_0 && ptype == kF16) ||
+                     (wtype == kF32 && ptype == kF32);
+  if (!combo) return false;
+  const int ept = stack_ept(d);
+  if (d % (32 * ept) != 0 || d / ept > kMaxConsumers) return false;
+  if (wtype == kQ4_0 && d % 256 != 0) return false;
   if (rank % 8 != 0 || rank > kMaxRank) return false;
   (void)ffn;
   (void)n_hot;
@@ -765,7 +897,7 @@ size_t stack_smem_layout(StackParams& p, int B, int G) {
     t2(sizeof(int) * share_cap);
     t2(sizeof(float) * share_cap);
     t2(share_cap);
-    t2(sizeof(float) * 2 * (kMaxConsumers / 32) * 2 * B);
+    t2(sizeof(float) * 2 * (kMaxConsumers / 32) * 6 * B);
     t2(sizeof(int) * (G + 1));
     t2(sizeof(int) * 4);
     fixed = o;
@@ -783,27 +915,28 @@ size_t stack_smem_layout(StackParams& p, int B, int G) {
   p.off_cidx = take(sizeof(int) * share_cap);
   p.off_cb1 = take(sizeof(float) * share_cap);
   p.off_act = take(share_cap);
-  p.off_red = take(sizeof(float) * 2 * (kMaxConsumers / 32) * 2 * B);
+  p.off_red = take(sizeof(float) * 2 * (kMaxConsumers / 32) * 6 * B);
   p.off_prefix = take(sizeof(int) * (G + 1));
   p.off_misc = take(sizeof(int) * 4);
   return off;
 }
 
 cudaError_t launch_stack(int wtype, int ptype, int B, const StackParams& p, int G, size_t smem, cudaStream_t st) {
-#define PI_STACK_CASE(W_, P_, B_) \
-  if (wtype == W_ && ptype == P_ && B == B_) return launch_t<W_, P_, B_>(p, G, smem, st);
-  PI_STACK_CASE(kF16, kF16, 1)
-  PI_STACK_CASE(kF16, kF16, 2)
-  PI_STACK_CASE(kQ4_0, kF16, 1)
-  PI_STACK_CASE(kQ4_0, kF16, 2)
-  PI_STACK_CASE(kF32, kF32, 1)
-  PI_STACK_CASE(kF32, kF32, 2)
-  PI_STACK_CASE(kF16, kF32, 1)
-  PI_STACK_CASE(kF16, kF32, 2)
-  PI_STACK_CASE(kF32, kF16, 1)
-  PI_STACK_CASE(kF32, kF16, 2)
-  PI_STACK_CASE(kQ4_0, kF32, 1)
-  PI_STACK_CASE(kQ4_0, kF32, 2)
+  const int ept = p.d / p.T;
+#define PI_STACK_CASE(W_, P_, B_, E_) \
+  if (wtype == W_ && ptype == P_ && B == B_ && ept == E_) return launch_t<W_, P_, B_, E_>(p, G, smem, st);
+  PI_STACK_CASE(kF16, kF16, 1, 8)
+  PI_STACK_CASE(kF16, kF16, 2, 8)
+  PI_STACK_CASE(kF16, kF16, 1, 16)
+  PI_STACK_CASE(kF16, kF16, 2, 16)
+  PI_STACK_CASE(kQ4_0, kF16, 1, 8)
+  PI_STACK_CASE(kQ4_0, kF16, 2, 8)
+  PI_STACK_CASE(kQ4_0, kF16, 1, 16)
+  PI_STACK_CASE(kQ4_0, kF16, 2, 16)
+  PI_STACK_CASE(kF32, kF32, 1, 8)
+  PI_STACK_CASE(kF32, kF32, 2, 8)
+  PI_STACK_CASE(kF32, kF32, 1, 16)
+  PI_STACK_CASE(kF32, kF32, 2, 16)
 #undef PI_STACK_CASE
   return cudaErrorInvalidValue;
 }

@@ -13,6 +13,9 @@ constexpr int kNQ = 64;              // items in flight per CTA (queue depth)
 constexpr int kMaxConsumers = 512;   // consumer threads per CTA (d <= 8192)
 constexpr int kMaxRank = 4096;
 constexpr size_t kSmemBytes = 232448;  // opt-in shared memory per CTA on sm_100
+constexpr int kYCopies = 8;          // fp32 output accumulator copies (spreads the atomics)
+constexpr int kGMaxCtas = 296;       // largest grid (2 x 148)
+constexpr int kShareRegs = 2;        // per-thread registers for the CTA's bias shares
 
 // One layer's device pointers (a copy of pi_layer_weights).
 struct StackLayer {
@@ -34,7 +37,7 @@ struct StackLayer {
 struct StackParams {
   int d, ffn, n_hot, rank, act, L;
   float eps;
-  int T;           // consumer threads (d / 16)
+  int T;           // consumer threads (d / stack_ept(d))
   int ring_bytes;  // shared-memory ring size
   int seg_cap;     // per-CTA capacity of the local active lists
   int off_bars, off_itemoff, off_u, off_bp, off_b1hot, off_cidx, off_cb1, off_act, off_red, off_prefix, off_misc;
@@ -46,12 +49,14 @@ struct StackParams {
   void* h_trace;    // [L, B, d] or null
   Ctrl* ctrl;
   float* u_g;       // [B, r]
-  float* yacc;      // [2, B, d]
+  float* yacc;      // [2, kYCopies, B, d] fp32 output accumulators
   int* seg;         // [G, seg_cap]
   int* seg_cnt;     // [G]
   StackLayer layers[kMaxLayers];
 };
 
+// Columns of d each consumer thread owns (8 when d/8 threads fit, else 16).
+int stack_ept(int d);
 bool stack_supported(int wtype, int ptype, int d, int ffn, int n_hot, int rank, int B, int L);
 // Fills the shared-memory offsets of p (needs d, ffn, n_hot, rank); returns the
 // dynamic shared memory size, or 0 if it does not fit.

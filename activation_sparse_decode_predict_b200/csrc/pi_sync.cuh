@@ -113,37 +113,48 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Ctrl* 
   }
 }
 
-// Grid barrier over all co-resident CTAs of a cooperative launch.
-// One thread per CTA arrives; barrier k (0-based, in launch order) has
-// completed once bar_gen has advanced k + 1 times past gen_start.
-__device__ __forceinline__ void grid_arrive(Ctrl* ctrl, unsigned nctas) {
+// Grid barrier over the co-resident CTAs of a cooperative launch.  bar_count
+// only grows: barrier k (0-based, in launch order) has completed once it
+// reaches base + (k + 1) * nctas, where base is the count the previous launch
+// left (ctrl->bar_base, read once at kernel start).  One thread per CTA
+// arrives after a CTA-wide barrier: one fence, one release add (the pattern of
+// a cooperative-groups grid sync).
+__device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void grid_arrive(Ctrl* ctrl) {
   __threadfence();
-  const unsigned old = atomicAdd(&ctrl->bar_count, 1u);
-  if (old == nctas - 1) {
-    atomicExch(&ctrl->bar_count, 0u);
-    __threadfence();
-    atomicAdd(&ctrl->bar_gen, 1u);
-  }
+  red_release_add(&ctrl->bar_count, 1u);
 }
 
-__device__ __forceinline__ bool grid_done(Ctrl* ctrl, unsigned gen_start, unsigned k) {
-  return (int)(ld_acquire_u32(&ctrl->bar_gen) - gen_start) >= (int)(k + 1);
+__device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
 }
 
-__device__ __forceinline__ bool grid_wait(Ctrl* ctrl, unsigned gen_start, unsigned k) {
-  if (grid_done(ctrl, gen_start, k)) return true;
-  const uint64_t t0 = global_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (grid_done(ctrl, gen_start, k)) return true;
-    if ((it & 15u) == 0) {
-      if (ld_volatile_s32(&ctrl->abort)) return false;
-      if (global_ns() - t0 > kTimeoutNs) {
-        raise_abort(ctrl);
-        return false;
+__device__ __forceinline__ bool grid_done(Ctrl* ctrl, unsigned base, unsigned k, unsigned nctas) {
+  return (int)(ld_relaxed_u32(&ctrl->bar_count) - (base + (k + 1) * nctas)) >= 0;
+}
+
+// Polls with relaxed loads; one acquire fence once the count is reached.
+__device__ __forceinline__ bool grid_wait(Ctrl* ctrl, unsigned base, unsigned k, unsigned nctas) {
+  if (!grid_done(ctrl, base, k, nctas)) {
+    const uint64_t t0 = global_ns();
+    for (uint32_t it = 1;; ++it) {
+      if (grid_done(ctrl, base, k, nctas)) break;
+      if ((it & 31u) == 0) {
+        if (ld_volatile_s32(&ctrl->abort)) return false;
+        if (global_ns() - t0 > kTimeoutNs) {
+          raise_abort(ctrl);
+          return false;
+        }
       }
     }
-    __nanosleep(64);
   }
+  __threadfence();
+  return true;
 }
 
 }  // namespace pi
