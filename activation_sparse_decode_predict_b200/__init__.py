@@ -149,5 +149,10 @@ def device_status(ws: torch.Tensor, clear: bool = False, stream=None) -> int:
     return int(v.value)
 
 
+def selftest_bounded_wait(ws: torch.Tensor, kind: int, stream=None) -> None:
+    """Launch a wait that can only time out (kind 0: mbarrier, 1: grid barrier)."""
+    _check(lib().pi_selftest_bounded_wait(_ptr(ws), int(kind), _stream(stream)))
+
+
 def version() -> str:
     return lib().pi_version().decode()

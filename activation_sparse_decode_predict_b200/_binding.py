@@ -23,7 +23,7 @@ MAX_BATCH = 16
 
 # Every symbol include/pi.h declares.
 EXPORTS = ("pi_workspace_bytes", "pi_workspace_init", "pi_predict", "pi_sparse_ffn", "pi_layer",
-           "pi_residual_rmsnorm", "pi_decode_stack", "pi_stack_launches", "pi_get_device_status", "pi_predict_static", "pi_last_error", "pi_version")
+           "pi_residual_rmsnorm", "pi_decode_stack", "pi_stack_launches", "pi_get_device_status", "pi_predict_static", "pi_selftest_bounded_wait", "pi_last_error", "pi_version")
 
 
 class FfnDesc(ctypes.Structure):
@@ -75,6 +75,8 @@ def load(path: str = LIB_PATH):
     lib.pi_get_device_status.restype = st
     lib.pi_predict_static.argtypes = [D, i32, P, P, P, P, f32, P, P, P]
     lib.pi_predict_static.restype = st
+    lib.pi_selftest_bounded_wait.argtypes = [P, i32, P]
+    lib.pi_selftest_bounded_wait.restype = st
     lib.pi_last_error.restype = ctypes.c_char_p
     lib.pi_version.restype = ctypes.c_char_p
     return lib

@@ -160,11 +160,31 @@ pi_status fused_params(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, pi:
   const int ep = desc->ptype == PI_F16 ? 2 : 4;
   const size_t wrow = desc->wtype == PI_Q4_0 ? desc->d / 2 + desc->d / 16
                                               : (size_t)desc->d * (desc->wtype == PI_F16 ? 2 : 4);
-  const size_t neuron = wrow * (desc->act == PI_ACT_REGLU ? 3 : 2);
-  const size_t p2item = (size_t)(P.T / 32) * desc->rank * ep;
-  const size_t p1item = (size_t)desc->d * ep;
+  const size_t neuron = (wrow + 16) * (desc->act == PI_ACT_REGLU ? 3 : 2) + 256;
+  // predictor items: fp16 predictors go to the tensor cores in 16-row tiles with padded rows
+  const size_t p2item = desc->ptype == PI_F16 ? (size_t)16 * (2 * desc->rank + 16) + 256
+                                              : (size_t)(P.T / 32) * desc->rank * ep;
+  const size_t p1item = (size_t)desc->d * ep + 256;
   const size_t half = (size_t)P.ring_bytes / 2;
   if (neuron > half || p2item > half || p1item > half) return PI_ERR_UNSUPPORTED;
+  // the tensor-core P1 tile takes at most 16 rows, and the rows of one tile
+  // (each a ring item of 2d bytes plus alignment and skew) fill at most half the ring
+  P.p1rows = 16;
+  if (desc->ptype == PI_F16) {
+    const int fit = (int)(half / ((size_t)desc->d * 2 + 240));
+    if (fit < P.p1rows) P.p1rows = fit;
+    if (P.p1rows < 1) return PI_ERR_UNSUPPORTED;
+  }
+  // a tensor-core group of ng neurons stays resident while the next group
+  // streams in: ng items fill at most half the ring, and the 16-row tile
+  // holds ng neurons' gate and up rows
+  const int rpn = desc->act == PI_ACT_REGLU ? 2 : 1;
+  P.ng = 1;
+  if (desc->wtype == PI_F16 && desc->ptype == PI_F16) {
+    const int cap = (int)(half / neuron);
+    P.ng = cap < 16 / rpn ? cap : 16 / rpn;
+    if (P.ng < 1) P.ng = 1;
+  }
   const int C = desc->ffn - desc->n_hot;
   P.seg_cap = (C + G - 1) / G + 1;
   // every consumer thread holds at most kShareRegs entries of the CTA's bias shares

@@ -31,6 +31,7 @@
 #include <stdint.h>
 
 #include "pi_common.cuh"
+#include "pi_mma.cuh"
 #include "pi_stack.cuh"
 #include "pi_sync.cuh"
 
@@ -174,6 +175,10 @@ struct Smem {
   float* red;        // [2][NW][2B]
   int* prefix;       // [G + 1]
   int* misc;         // [0] cold_n, [1] gen_start
+  uint8_t* hb;       // [B][d + 8] fp16 token rows (tensor-core operand)
+  uint8_t* ub;       // [2B][r + 8] fp16 u rows: hi and lo parts of each token's u
+  uint8_t* zero;     // 16 zero bytes (operand rows beyond the token count)
+  float* redp;       // [NW][16][2] P1 partial dots
 };
 
 __device__ __forceinline__ Smem carve(uint8_t* base, const StackParams& p) {
@@ -193,6 +198,10 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const StackParams& p) {
   s.red = reinterpret_cast<float*>(base + p.off_red);
   s.prefix = reinterpret_cast<int*>(base + p.off_prefix);
   s.misc = reinterpret_cast<int*>(base + p.off_misc);
+  s.hb = base + p.off_hb;
+  s.ub = base + p.off_ub;
+  s.zero = base + p.off_zero;
+  s.redp = reinterpret_cast<float*>(base + p.off_redp);
   return s;
 }
 
@@ -269,6 +278,26 @@ struct Producer {
     }
   }
 
+  // One item of `nrows` rows of `row_bytes` each: row i comes from
+  // src + i * src_stride and lands at dst_stride * i past a 128-byte aligned
+  // start shifted by `skew` bytes (skew and padding keep ldmatrix rows of
+  // consecutive rows/items on different shared-memory banks).
+  __device__ bool issue_rows(const uint8_t* src, int64_t src_stride, int nrows, uint32_t row_bytes,
+                             uint32_t dst_stride, uint32_t skew) {
+    const uint32_t total = nrows * dst_stride + 128 + skew;
+    uint32_t pos;
+    if (!alloc(total, pos)) return false;
+    const uint32_t start = ((pos + 127u) & ~127u) + skew;
+    const uint32_t q = item % kNQ;
+    s.item_off[q] = start;
+    s.istart[q] = pos;
+    mbar_arrive_expect_tx(&s.full[q], nrows * row_bytes);
+    for (int i = 0; i < nrows; ++i) bulk_g2s(s.ring + start + i * dst_stride, src + i * src_stride, row_bytes, &s.full[q]);
+    head = pos + total;
+    ++item;
+    return true;
+  }
+
   // One item made of up to 6 contiguous source segments, copied back to back.
   __device__ bool issue(int nseg, const void* const* src, const uint32_t* bytes) {
     uint32_t total = 0;
@@ -289,27 +318,45 @@ struct Producer {
     return true;
   }
 
+  // One neuron: its gate (ReGLU only), up and down rows.  Row m of the item
+  // starts m * (wrb + 16) bytes past a 128-byte aligned base that is shifted
+  // by 32 * (neuron sequence number mod 4) bytes, so that the gate and up
+  // rows of four consecutive neurons fall on eight different shared-memory
+  // bank groups (conflict-free ldmatrix).  Q4_0 rows hold qs then sc.
+  uint32_t nseq = 0;
   __device__ bool issue_neuron(const StackLayer& Ly, int j, int wt, int gated) {
-    const void* src[6];
-    uint32_t by[6];
-    int n = 0;
     const int d = p.d;
-    auto add_row = [&](const void* data, const void* sc) {
+    const uint32_t wrb = wt == kQ4_0 ? (uint32_t)(d / 2 + d / 16) : (uint32_t)(d * (wt == kF16 ? 2 : 4));
+    const uint32_t wrp = wrb + 16;
+    const int nrow = gated ? 3 : 2;
+    const uint32_t skew = 32u * (nseq & 3u);
+    ++nseq;
+    const uint32_t total = nrow * wrp + 128 + skew;
+    uint32_t pos;
+    if (!alloc(total, pos)) return false;
+    const uint32_t start = ((pos + 127u) & ~127u) + skew;
+    const uint32_t q = item % kNQ;
+    s.item_off[q] = start;
+    s.istart[q] = pos;
+    mbar_arrive_expect_tx(&s.full[q], nrow * wrb);
+    const void* rows[3];
+    const void* scs[3];
+    int m = 0;
+    if (gated) { rows[m] = Ly.wg; scs[m++] = Ly.wg_sc; }
+    rows[m] = Ly.wu; scs[m++] = Ly.wu_sc;
+    rows[m] = Ly.wd; scs[m++] = Ly.wd_sc;
+    for (int i = 0; i < nrow; ++i) {
+      uint8_t* dst = s.ring + start + i * wrp;
       if (wt == kQ4_0) {
-        src[n] = reinterpret_cast<const uint8_t*>(data) + (int64_t)j * (d / 2);
-        by[n++] = d / 2;
-        src[n] = reinterpret_cast<const uint8_t*>(sc) + (int64_t)j * (d / 16);
-        by[n++] = d / 16;
+        bulk_g2s(dst, reinterpret_cast<const uint8_t*>(rows[i]) + (int64_t)j * (d / 2), d / 2, &s.full[q]);
+        bulk_g2s(dst + d / 2, reinterpret_cast<const uint8_t*>(scs[i]) + (int64_t)j * (d / 16), d / 16, &s.full[q]);
       } else {
-        const int rb = d * (wt == kF16 ? 2 : 4);
-        src[n] = reinterpret_cast<const uint8_t*>(data) + (int64_t)j * rb;
-        by[n++] = rb;
+        bulk_g2s(dst, reinterpret_cast<const uint8_t*>(rows[i]) + (int64_t)j * wrb, wrb, &s.full[q]);
       }
-    };
-    if (gated) add_row(Ly.wg, Ly.wg_sc);
-    add_row(Ly.wu, Ly.wu_sc);
-    add_row(Ly.wd, Ly.wd_sc);
-    return issue(n, src, by);
+    }
+    head = pos + total;
+    ++item;
+    return true;
   }
 
   // Drain: wait for every issued copy to land before the CTA may exit.
@@ -336,6 +383,8 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
     for (int q = 0; q < kNQ; ++q) {
       mbar_init(&s.full[q], 1);
       mbar_init(&s.empty[q], NW);
+      s.item_off[q] = 0u;  // in-ring offsets even before the first item of a slot
+      s.istart[q] = 0u;
     }
     mbar_init(s.list_bar, 1);
     mbar_fence_init();
@@ -357,16 +406,26 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
     for (int l = 0; l < p.L && ok; ++l) {
       const StackLayer& Ly = p.layers[l];
       if (lane == 0) {
-        for (int k = k0; k < k1 && ok; ++k) {
-          const void* src = reinterpret_cast<const uint8_t*>(Ly.P1) + (int64_t)k * d * ep;
-          const uint32_t by = d * ep;
-          ok = pr.issue(1, &src, &by);
-        }
-        for (int cc = c0; cc < c1 && ok; cc += NW) {
-          const int rows = min(NW, c1 - cc);
-          const void* src = reinterpret_cast<const uint8_t*>(Ly.P2) + (int64_t)cc * r * ep;
-          const uint32_t by = rows * r * ep;
-          ok = pr.issue(1, &src, &by);
+        if constexpr (PT == kF16) {
+          // tensor-core predictor: skewed P1 rows, P2 in 16-row tiles with padded rows
+          for (int k = k0; k < k1 && ok; ++k)
+            ok = pr.issue_rows(reinterpret_cast<const uint8_t*>(Ly.P1) + (int64_t)k * d * 2, 0, 1, d * 2, d * 2,
+                               16u * (uint32_t)((k - k0) & 7));
+          for (int cc = c0; cc < c1 && ok; cc += 16)
+            ok = pr.issue_rows(reinterpret_cast<const uint8_t*>(Ly.P2) + (int64_t)cc * r * 2, (int64_t)r * 2,
+                               min(16, c1 - cc), r * 2, r * 2 + 16, 0);
+        } else {
+          for (int k = k0; k < k1 && ok; ++k) {
+            const void* src = reinterpret_cast<const uint8_t*>(Ly.P1) + (int64_t)k * d * ep;
+            const uint32_t by = d * ep;
+            ok = pr.issue(1, &src, &by);
+          }
+          for (int cc = c0; cc < c1 && ok; cc += NW) {
+            const int rows = min(NW, c1 - cc);
+            const void* src = reinterpret_cast<const uint8_t*>(Ly.P2) + (int64_t)cc * r * ep;
+            const uint32_t by = rows * r * ep;
+            ok = pr.issue(1, &src, &by);
+          }
         }
         for (int j = j0; j < j1 && ok; ++j) ok = pr.issue_neuron(Ly, j, WT, gated);
         // the cold rows need every CTA's scores: barrier S of this layer
@@ -437,7 +496,7 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
   auto wait_item = [&](uint32_t& off) -> bool {
     const uint32_t q = witem % kNQ;
     const bool okw = mbar_wait(&s.full[q], (witem / kNQ) & 1u, ctrl);
-    off = s.item_off[q];
+    off = okw ? s.item_off[q] : 0u;  // after a timeout, reads stay inside the ring
     ++witem;
     return okw;
   };
@@ -454,6 +513,13 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
   if (c == 0 && p.h_trace) {
 #pragma unroll
     for (int b = 0; b < B; ++b) store_vals<WT, EPT, PT>(reinterpret_cast<uint8_t*>(p.h_trace) + (int64_t)b * d * ep, t, T, h[b]);
+  }
+  const int HS = 2 * d + 16;  // byte stride of the fp16 token rows in shared memory
+  const int US = 2 * r + 16;  // byte stride of the fp16 u rows
+  if constexpr (PT == kF16) {
+#pragma unroll
+    for (int b = 0; b < B; ++b) store_vals<WT, EPT, kF16>(s.hb + b * HS, t, T, h[b]);
+    if (t < 4) reinterpret_cast<uint32_t*>(s.zero)[t] = 0u;
   }
   const int ybuf4 = K * B * d / 4;  // float4s per accumulator buffer (K copies)
   {
@@ -473,8 +539,61 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
       b1_v[i] = (Ly.b1 && x < j1 - j0) ? __ldg(Ly.b1 + j0 + x) : 0.f;
     }
 
-    // ---- predictor step 1: u = ReLU(P1 h), up to 4 rows per CTA-wide reduction ----
+    // ---- predictor step 1: u = ReLU(P1 h) ----
     bool to = false;
+    if constexpr (PT == kF16) {
+      // Tensor cores: the CTA's (<= 16) P1 rows are the A tile, the fp16
+      // token rows the B tile; warps split d, partial dots meet in shared memory.
+      named_sync(1, T);  // token rows (written by the glue) are complete
+      const int bn = lane & 7;
+      const uint32_t b_base = (bn < B ? smem_u32(s.hb + bn * HS) + (uint32_t)(((lane >> 3) & 1) * 16) : smem_u32(s.zero));
+      const uint32_t b_step = bn < B ? 32u : 0u;
+      const int KS = d / 16, ks0 = warp * KS / NW, ks1 = (warp + 1) * KS / NW;
+      // rows in groups of at most p.p1rows, so that a group fits in half the ring
+      for (int g0 = k0; g0 < k1; g0 += p.p1rows) {
+        const int nrow = min(p.p1rows, k1 - g0);
+        if (g0 > k0) named_sync(1, T);  // the previous group's partial dots have been read
+        for (int i = 0; i < nrow; ++i) to |= !mbar_wait(&s.full[(witem + i) % kNQ], ((witem + i) / kNQ) & 1u, ctrl);
+        const int ar = lane & 15;
+        const uint32_t a_base =
+            smem_u32(s.ring + s.item_off[(witem + (ar < nrow ? ar : 0)) % kNQ]) + (uint32_t)((lane >> 4) * 16);
+        float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+        int ks = to ? ks1 : ks0;  // no tile is read unless all its rows have landed
+        for (; ks + 1 < ks1; ks += 2) {
+          uint32_t a0, a1, a2, a3, b0, b1, e0, e1, e2, e3, f0, f1;
+          ldsm_x4(a_base + 32u * ks, a0, a1, a2, a3);
+          ldsm_x2(b_base + b_step * ks, b0, b1);
+          ldsm_x4(a_base + 32u * (ks + 1), e0, e1, e2, e3);
+          ldsm_x2(b_base + b_step * (ks + 1), f0, f1);
+          mma_16816(acc0, a0, a1, a2, a3, b0, b1);
+          mma_16816(acc1, e0, e1, e2, e3, f0, f1);
+        }
+        if (ks < ks1) {
+          uint32_t a0, a1, a2, a3, b0, b1;
+          ldsm_x4(a_base + 32u * ks, a0, a1, a2, a3);
+          ldsm_x2(b_base + b_step * ks, b0, b1);
+          mma_16816(acc0, a0, a1, a2, a3, b0, b1);
+        }
+        witem += nrow;
+        for (int i = 0; i < nrow; ++i) release_item();
+        // thread (g = lane/4, t4 = lane%4 == 0) holds rows g and g+8, tokens 0 and 1
+        if ((lane & 3) == 0) {
+          const int g = lane >> 2;
+          float* rp = s.redp + warp * 32;
+          rp[g * 2 + 0] = acc0[0] + acc1[0];
+          rp[g * 2 + 1] = acc0[1] + acc1[1];
+          rp[(g + 8) * 2 + 0] = acc0[2] + acc1[2];
+          rp[(g + 8) * 2 + 1] = acc0[3] + acc1[3];
+        }
+        if (named_sync_or(1, T, to)) return;
+        if (t < nrow * B) {
+          const int row = t / B, b = t % B;
+          float a = 0.f;
+          for (int w = 0; w < NW; ++w) a += s.redp[w * 32 + row * 2 + b];
+          p.u_g[(int64_t)b * r + g0 + row] = fmaxf(a, 0.f);
+        }
+      }
+    } else {
     for (int kk = k0; kk < k1; kk += 4) {
       const int nrow = min(4, k1 - kk);
       float acc[4 * B];
@@ -503,6 +622,7 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
         for (int i = 0; i < nrow; ++i)
           for (int b = 0; b < B; ++b) p.u_g[(int64_t)b * r + kk + i] = fmaxf(acc[i * B + b], 0.f);
     }
+    }  // predictor step 1
 #pragma unroll
     for (int i = 0; i < kShareRegs; ++i) {
       const int x = t + i * T;
@@ -522,9 +642,19 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
       const int z0 = share_lo(ybuf4, c, G), z1 = share_lo(ybuf4, c + 1, G);
       for (int i = z0 + t; i < z1; i += T) nxt[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    // u -> shared memory, split layout: unit m (8 values) stored as two float4
-    // planes so that lane-strided reads are conflict-free.
-    {
+    if constexpr (PT == kF16) {
+      // u -> fp16 rows for the tensor cores: row 2b = hi(u_b), row 2b+1 = lo(u_b) = u_b - hi
+      for (int i = t; i < B * r; i += T) {
+        const int b = i / r, k = i % r;
+        const float v = __ldcg(p.u_g + i);
+        const __half hi = __float2half_rn(v);
+        const __half lo = __float2half_rn(v - __half2float(hi));
+        reinterpret_cast<__half*>(s.ub + (2 * b) * US)[k] = hi;
+        reinterpret_cast<__half*>(s.ub + (2 * b + 1) * US)[k] = lo;
+      }
+    } else {
+      // u -> shared memory, split layout: unit m (8 values) stored as two float4
+      // planes so that lane-strided reads are conflict-free.
       const int nu = r / 8;
       for (int i = t; i < B * nu; i += T) {
         const int b = i / nu, m = i % nu;
@@ -537,8 +667,61 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
     }
     named_sync(1, T);
 
-    // ---- predictor step 2: scores of this CTA's cold rows (warp per row) ----
-    {
+    // ---- predictor step 2: scores of this CTA's cold rows ----
+    if constexpr (PT == kF16) {
+      // Tensor cores: each 16-row tile of P2 (one ring item) against the u
+      // rows (hi, lo per token); warp w takes tiles w, w + NW, ...
+      const int nrows = c1 - c0;
+      const int ntile = (nrows + 15) / 16;
+      const int bn = lane & 7;
+      const uint32_t b_base = (bn < 2 * B ? smem_u32(s.ub + bn * US) + (uint32_t)(((lane >> 3) & 1) * 16) : smem_u32(s.zero));
+      const uint32_t b_step = bn < 2 * B ? 32u : 0u;
+      const int KS = r / 16;
+      for (int it = 0; it < ntile; ++it) {
+        const uint32_t myitem = witem + it;
+        if (it % NW == warp) {
+          to |= !mbar_wait(&s.full[myitem % kNQ], (myitem / kNQ) & 1u, ctrl);
+          const int rows = min(16, nrows - 16 * it);
+          const int ar = lane & 15;
+          const uint32_t a_base = smem_u32(s.ring + s.item_off[myitem % kNQ]) + (uint32_t)((ar < rows ? ar : 0) * US) +
+                                  (uint32_t)((lane >> 4) * 16);
+          float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+          int ks = to ? KS : 0;  // the tile is read only once it has landed
+          for (; ks + 1 < KS; ks += 2) {
+            uint32_t a0, a1, a2, a3, b0, b1, e0, e1, e2, e3, f0, f1;
+            ldsm_x4(a_base + 32u * ks, a0, a1, a2, a3);
+            ldsm_x2(b_base + b_step * ks, b0, b1);
+            ldsm_x4(a_base + 32u * (ks + 1), e0, e1, e2, e3);
+            ldsm_x2(b_base + b_step * (ks + 1), f0, f1);
+            mma_16816(acc0, a0, a1, a2, a3, b0, b1);
+            mma_16816(acc1, e0, e1, e2, e3, f0, f1);
+          }
+          if (ks < KS) {
+            uint32_t a0, a1, a2, a3, b0, b1;
+            ldsm_x4(a_base + 32u * ks, a0, a1, a2, a3);
+            ldsm_x2(b_base + b_step * ks, b0, b1);
+            mma_16816(acc0, a0, a1, a2, a3, b0, b1);
+          }
+          // thread (g, t4): rows g and g+8, columns 2*t4 (hi) and 2*t4+1 (lo) = token t4
+          const int g = lane >> 2, t4 = lane & 3;
+          const float s_g = (acc0[0] + acc1[0]) + (acc0[1] + acc1[1]);
+          const float s_g8 = (acc0[2] + acc1[2]) + (acc0[3] + acc1[3]);
+          const int r0 = 16 * it + g, r8 = r0 + 8;
+          bool on0 = t4 < B && g < rows && (s_g + s.bp[r0]) > Ly.thr;
+          bool on8 = t4 < B && g + 8 < rows && (s_g8 + s.bp[r8 < nrows ? r8 : r0]) > Ly.thr;
+          on0 |= __shfl_xor_sync(0xffffffffu, on0, 1);
+          on0 |= __shfl_xor_sync(0xffffffffu, on0, 2);
+          on8 |= __shfl_xor_sync(0xffffffffu, on8, 1);
+          on8 |= __shfl_xor_sync(0xffffffffu, on8, 2);
+          if (t4 == 0) {
+            if (g < rows) s.act[r0] = on0 ? 1 : 0;
+            if (g + 8 < rows) s.act[r8] = on8 ? 1 : 0;
+          }
+        }
+        release_item();
+      }
+      witem += ntile;
+    } else {
       const int nu = r / 8;  // 8-element units per row (r % 8 == 0)
       // single token and rank <= 1024: this lane's slice of u stays in registers
       float ureg[4][8];
@@ -649,7 +832,7 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
     for (int b = 0; b < B; ++b)
 #pragma unroll
       for (int e = 0; e < EPT; ++e) y[b][e] = 0.f;
-    const int wrb = wrow_bytes(WT, d);
+    const int wrp = wrow_bytes(WT, d) + 16;  // byte stride of a neuron item's rows
     const int nh = j1 - j0;
     int n = nh;
     bool have_list = false;
@@ -664,7 +847,7 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
       const uint8_t* it = s.ring + off;
       float acc[2 * B];
       float wu[EPT];
-      w_vals<WT, EPT>(it + (gated ? wrb : 0), d, t, T, wu);
+      w_vals<WT, EPT>(it + (gated ? wrp : 0), d, t, T, wu);
 #pragma unroll
       for (int b = 0; b < B; ++b) {
         float a = 0.f;
@@ -711,7 +894,7 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
       for (int b = 0; b < B; ++b)
         a[b] = gated ? act_eval(kReglu, tot[b] + bias, tot[B + b]) : act_eval(p.act, tot[B + b] + bias, 0.f);
       float wd[EPT];
-      w_vals<WT, EPT>(s.ring + ((k & 1) ? itoff1 : itoff0) + (gated ? 2 : 1) * wrb, d, t, T, wd);
+      w_vals<WT, EPT>(s.ring + ((k & 1) ? itoff1 : itoff0) + (gated ? 2 : 1) * wrp, d, t, T, wd);
       release_item();
 #pragma unroll
       for (int b = 0; b < B; ++b)
@@ -728,21 +911,107 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
       have_list = true;
       return true;
     };
-    if (nh == 0) {
-      if (!take_list()) return;
-      named_sync(1, T);  // cb1 visible
-    }
-    if (n > 0) prepare(0);
-    for (int k = 0; k < n; ++k) {
-      if (named_sync_or(1, T, to)) return;  // neuron k's partial sums are complete
-      if (k + 1 == nh && !have_list) {
-        if (!take_list()) return;  // cb1 becomes visible at the next neuron's barrier
+    if constexpr (WT == kF16 && PT == kF16) {
+      // Tensor cores for the gate/up dots of p.ng neurons at a time: their
+      // gate and up rows form one 16-row A tile (unused rows repeat neuron 0),
+      // the fp16 token rows the B tile; warps split d and their partial dots
+      // meet in shared memory, one thread per (neuron, token) applies the
+      // activation, then every thread adds the group's down rows into its
+      // columns of the partial output.
+      const int rpn = gated ? 2 : 1;  // tile rows per neuron
+      const int bn = lane & 7;
+      const uint32_t b_base =
+          bn < B ? smem_u32(s.hb + bn * HS) + (uint32_t)(((lane >> 3) & 1) * 16) : smem_u32(s.zero);
+      const uint32_t b_step = bn < B ? 32u : 0u;
+      const int KS = d / 16, ks0 = warp * KS / NW, ks1 = (warp + 1) * KS / NW;
+      float* gact = nred;  // [ng][B] activations of the group
+      int k = 0;
+      for (;;) {
+        if (k == nh && !have_list) {
+          if (!take_list()) return;
+          named_sync(1, T);  // cb1 visible
+        }
+        const int lim = have_list ? n : nh;
+        if (k >= lim) break;
+        const int ng = min(p.ng, lim - k);
+        for (int i = 0; i < ng; ++i) to |= !mbar_wait(&s.full[(witem + i) % kNQ], ((witem + i) / kNQ) & 1u, ctrl);
+        if (!to) {
+          const int tr = lane & 15;
+          const int jj = tr / rpn < ng ? tr / rpn : 0;
+          const int which = gated ? (tr & 1) : 0;  // item row: gate then up (ReGLU), up (otherwise)
+          const uint32_t a_base = smem_u32(s.ring + s.item_off[(witem + jj) % kNQ]) + (uint32_t)(which * wrp) +
+                                  (uint32_t)((lane >> 4) * 16);
+          float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+          int ks = ks0;
+          for (; ks + 1 < ks1; ks += 2) {
+            uint32_t a0, a1, a2, a3, b0, b1, e0, e1, e2, e3, f0, f1;
+            ldsm_x4(a_base + 32u * ks, a0, a1, a2, a3);
+            ldsm_x2(b_base + b_step * ks, b0, b1);
+            ldsm_x4(a_base + 32u * (ks + 1), e0, e1, e2, e3);
+            ldsm_x2(b_base + b_step * (ks + 1), f0, f1);
+            mma_16816(acc0, a0, a1, a2, a3, b0, b1);
+            mma_16816(acc1, e0, e1, e2, e3, f0, f1);
+          }
+          if (ks < ks1) {
+            uint32_t a0, a1, a2, a3, b0, b1;
+            ldsm_x4(a_base + 32u * ks, a0, a1, a2, a3);
+            ldsm_x2(b_base + b_step * ks, b0, b1);
+            mma_16816(acc0, a0, a1, a2, a3, b0, b1);
+          }
+          // thread (g = lane/4, lane%4 == 0) holds tile rows g and g+8, tokens 0 and 1
+          if ((lane & 3) == 0) {
+            const int g = lane >> 2;
+            float* rp = s.redp + warp * 32;
+            rp[g * 2 + 0] = acc0[0] + acc1[0];
+            rp[g * 2 + 1] = acc0[1] + acc1[1];
+            rp[(g + 8) * 2 + 0] = acc0[2] + acc1[2];
+            rp[(g + 8) * 2 + 1] = acc0[3] + acc1[3];
+          }
+        }
+        if (named_sync_or(1, T, to)) return;
+        if (t < ng * B) {
+          const int jj = t / B, b = t % B;
+          float gd = 0.f, vd = 0.f;
+          for (int w = 0; w < NW; ++w) {
+            gd += s.redp[w * 32 + (jj * rpn) * 2 + b];
+            vd += s.redp[w * 32 + (jj * rpn + rpn - 1) * 2 + b];
+          }
+          const int kk = k + jj;
+          const float bias = kk < nh ? s.b1hot[kk] : s.cb1[kk - nh];
+          gact[jj * B + b] = gated ? act_eval(kReglu, gd + bias, vd) : act_eval(p.act, vd + bias, 0.f);
+        }
+        named_sync(1, T);
+        for (int jj = 0; jj < ng; ++jj) {
+          float wd[EPT];
+          w_vals<WT, EPT>(s.ring + s.item_off[(witem + jj) % kNQ] + rpn * wrp, d, t, T, wd);
+#pragma unroll
+          for (int b = 0; b < B; ++b) {
+            const float a = gact[jj * B + b];
+#pragma unroll
+            for (int e = 0; e < EPT; ++e) y[b][e] = fmaf(a, wd[e], y[b][e]);
+          }
+        }
+        witem += ng;
+        for (int i = 0; i < ng; ++i) release_item();
+        k += ng;
       }
-      if (k + 1 < n) prepare(k + 1);
-      finish(k);
-    }
-    if (!have_list) {  // (nh > 0 and the loop ended before the list: cannot happen, kept for safety)
-      if (!take_list()) return;
+    } else {
+      if (nh == 0) {
+        if (!take_list()) return;
+        named_sync(1, T);  // cb1 visible
+      }
+      if (n > 0) prepare(0);
+      for (int k = 0; k < n; ++k) {
+        if (named_sync_or(1, T, to)) return;  // neuron k's partial sums are complete
+        if (k + 1 == nh && !have_list) {
+          if (!take_list()) return;  // cb1 becomes visible at the next neuron's barrier
+        }
+        if (k + 1 < n) prepare(k + 1);
+        finish(k);
+      }
+      if (!have_list) {  // (nh > 0 and the loop ended before the list: cannot happen, kept for safety)
+        if (!take_list()) return;
+      }
     }
 
     // ---- split-K: add the partial into one of K fp32 accumulator copies ----
@@ -814,6 +1083,10 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
         const float inv = rsqrtf(ss[b] / (float)d + p.eps);
 #pragma unroll
         for (int e = 0; e < EPT; ++e) h[b][e] = round_to(PT, h[b][e] * inv);
+      }
+      if constexpr (PT == kF16) {
+#pragma unroll
+        for (int b = 0; b < B; ++b) store_vals<WT, EPT, kF16>(s.hb + b * HS, t, T, h[b]);
       }
       if (c == 0) {
         uint8_t* dst = nullptr;
@@ -900,6 +1173,10 @@ size_t stack_smem_layout(StackParams& p, int B, int G) {
     t2(sizeof(float) * 2 * (kMaxConsumers / 32) * 6 * B);
     t2(sizeof(int) * (G + 1));
     t2(sizeof(int) * 4);
+    t2((size_t)B * (2 * p.d + 16));
+    t2((size_t)2 * B * (2 * p.rank + 16));
+    t2(16);
+    t2(sizeof(float) * (kMaxConsumers / 32) * 32);
     fixed = o;
   }
   const size_t total = kSmemBytes;
@@ -918,6 +1195,10 @@ size_t stack_smem_layout(StackParams& p, int B, int G) {
   p.off_red = take(sizeof(float) * 2 * (kMaxConsumers / 32) * 6 * B);
   p.off_prefix = take(sizeof(int) * (G + 1));
   p.off_misc = take(sizeof(int) * 4);
+  p.off_hb = take((size_t)B * (2 * p.d + 16));
+  p.off_ub = take((size_t)2 * B * (2 * p.rank + 16));
+  p.off_zero = take(16);
+  p.off_redp = take(sizeof(float) * (kMaxConsumers / 32) * 32);
   return off;
 }
 

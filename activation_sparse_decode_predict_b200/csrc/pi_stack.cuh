@@ -40,7 +40,10 @@ struct StackParams {
   int T;           // consumer threads (d / stack_ept(d))
   int ring_bytes;  // shared-memory ring size
   int seg_cap;     // per-CTA capacity of the local active lists
+  int ng;          // neurons per tensor-core group (fp16 weights and predictors)
+  int p1rows;      // P1 rows per tensor-core group (fp16 predictors)
   int off_bars, off_itemoff, off_u, off_bp, off_b1hot, off_cidx, off_cb1, off_act, off_red, off_prefix, off_misc;
+  int off_hb, off_ub, off_zero, off_redp;
   const void* h_in;
   void* h_out;
   int32_t* idx;     // [L, C]

@@ -253,6 +253,17 @@ PI_API pi_status pi_predict_static(const pi_ffn_desc *desc, int32_t batch, const
                                    const void *P2, const float *bp, float threshold, int32_t *idx, int32_t *count,
                                    void *stream);
 
+/*
+ * pi_selftest_bounded_wait -- run one bounded wait that nothing will ever
+ * satisfy, to exercise the failure path of the persistent kernel without a
+ * GPU fault: kind 0 waits on a shared-memory mbarrier nobody arrives on,
+ * kind 1 on a grid-barrier count nobody reaches.  The wait gives up after the
+ * same limit the decode kernel uses (2 s), records PI_ERR_TIMEOUT in the
+ * workspace status word, raises the workspace abort flag and returns; the
+ * CUDA context stays usable.  Call pi_workspace_init before reusing `ws`.
+ */
+PI_API pi_status pi_selftest_bounded_wait(void *ws, int32_t kind, void *stream);
+
 /* Text of the last host-side error in this thread (never NULL). */
 PI_API const char *pi_last_error(void);
 
