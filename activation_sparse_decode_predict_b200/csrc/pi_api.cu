@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include "pi.h"
+#include "pi_batch.cuh"
 #include "pi_common.cuh"
 #include "pi_kernels_v1.cuh"
 #include "pi_layout.h"
@@ -109,6 +110,16 @@ pi_status ffn_impl(const pi_ffn_desc* d, int32_t B, const void* h, const int32_t
   float* a = reinterpret_cast<float*>(ws + L.act);
   float* partial = reinterpret_cast<float*>(ws + L.partial);
   const int sms = sm_count();
+  if (pi::batch_supported(d->wtype, d->ptype, d->d, B)) {
+    // token blocks of 3..16 with fp16 weights: tensor-core gate/up and down
+    const int NR = pi::batch_ranges(d->d, sms);
+    PI_CUDA(pi::launch_batch_ffn(d->act, h, B, d->d, d->ffn, d->n_hot, idx, count, Wg.data, Wu.data, Wd.data, b1,
+                                 reinterpret_cast<float*>(ws + L.pre), partial, NR, reinterpret_cast<pi::Ctrl*>(ws),
+                                 sms, st),
+            "tensor-core FFN launch");
+    PI_CUDA(pi::launch_ffn_reduce(partial, NR, B, d->d, b2, y, st), "split-K reduce launch");
+    return PI_OK;
+  }
   const int G = L.g_max < 2 * sms ? L.g_max : 2 * sms;
   PI_CUDA(pi::launch_ffn_act(d->wtype, d->ptype, d->act, h, B, d->d, d->ffn, d->n_hot, idx, count, Wg.data,
                              Wg.scales, Wu.data, Wu.scales, b1, a, d->ffn, status, sms, st),
@@ -134,6 +145,9 @@ pi_status check_layer(const pi_ffn_desc* desc, const pi_layer_weights* w) {
 
 static_assert(pi::kYAccCopies == pi::kYCopies, "workspace layout and kernel agree on the accumulator copies");
 static_assert(pi::kGMax == pi::kGMaxCtas, "workspace layout and kernel agree on the largest grid");
+static_assert(pi::kLayersMax == pi::kMaxLayers && pi::kLayersMax == PI_MAX_LAYERS, "layer limits agree");
+static_assert(sizeof(pi::Ctrl) == pi::kCtrlBytes, "control block size");
+static_assert(sizeof(pi::Ctrl{}.pool) / sizeof(int) == pi::kLayersMax, "one claim counter per layer");
 
 int stack_grid() {
   const int g = sm_count();
@@ -160,7 +174,7 @@ pi_status fused_params(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, pi:
   const int ep = desc->ptype == PI_F16 ? 2 : 4;
   const size_t wrow = desc->wtype == PI_Q4_0 ? desc->d / 2 + desc->d / 16
                                               : (size_t)desc->d * (desc->wtype == PI_F16 ? 2 : 4);
-  const size_t neuron = (wrow + 16) * (desc->act == PI_ACT_REGLU ? 3 : 2) + 256;
+  const size_t neuron = (wrow + 16) * (desc->act == PI_ACT_REGLU ? 3 : 2) + 16 + 256;
   // predictor items: fp16 predictors go to the tensor cores in 16-row tiles with padded rows
   const size_t p2item = desc->ptype == PI_F16 ? (size_t)16 * (2 * desc->rank + 16) + 256
                                               : (size_t)(P.T / 32) * desc->rank * ep;
@@ -175,21 +189,26 @@ pi_status fused_params(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, pi:
     if (fit < P.p1rows) P.p1rows = fit;
     if (P.p1rows < 1) return PI_ERR_UNSUPPORTED;
   }
-  // a tensor-core group of ng neurons stays resident while the next group
-  // streams in: ng items fill at most half the ring, and the 16-row tile
-  // holds ng neurons' gate and up rows
+  // a group of ng neurons stays resident while the next group streams in:
+  // ng items fill at most half the ring; a tensor-core group's gate and up
+  // rows fill one 16-row tile
   const int rpn = desc->act == PI_ACT_REGLU ? 2 : 1;
-  P.ng = 1;
-  if (desc->wtype == PI_F16 && desc->ptype == PI_F16) {
+  {
     const int cap = (int)(half / neuron);
-    P.ng = cap < 16 / rpn ? cap : 16 / rpn;
+    const int lim = (desc->wtype == PI_F16 && desc->ptype == PI_F16) ? 16 / rpn : 4;
+    P.ng = cap < lim ? cap : lim;
     if (P.ng < 1) P.ng = 1;
   }
+  // about one group of hot neurons per CTA is shared out statically (it fills
+  // the wait for barrier U); the rest is claimed, which balances the CTAs
+  P.hot_static = desc->n_hot < G * P.ng ? desc->n_hot : G * P.ng;
   const int C = desc->ffn - desc->n_hot;
-  P.seg_cap = (C + G - 1) / G + 1;
-  // every consumer thread holds at most kShareRegs entries of the CTA's bias shares
-  if ((C + G - 1) / G > pi::kShareRegs * P.T || (desc->n_hot + G - 1) / G > pi::kShareRegs * P.T)
-    return PI_ERR_UNSUPPORTED;
+  // every consumer thread holds at most kShareRegs entries of the CTA's P2 bias share
+  if ((C + G - 1) / G > pi::kShareRegs * P.T) return PI_ERR_UNSUPPORTED;
+  // the final list compaction keeps cmp_layers layers of this CTA's list (and
+  // two offsets per layer) in the ring
+  P.cmp_layers = (int)((size_t)P.ring_bytes / ((size_t)P.seg_cap * 4 + 8));
+  if (P.cmp_layers < 1) return PI_ERR_UNSUPPORTED;
   return PI_OK;
 }
 
@@ -211,8 +230,8 @@ pi_status fused_stack(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, cons
   P.ctrl = reinterpret_cast<pi::Ctrl*>(ws);
   P.u_g = reinterpret_cast<float*>(ws + L.u);
   P.yacc = reinterpret_cast<float*>(ws + L.yacc);
-  P.seg = reinterpret_cast<int*>(ws + L.seg);
-  P.seg_cnt = reinterpret_cast<int*>(ws + L.seg_cnt);
+  P.pool = reinterpret_cast<pi::Ctrl*>(ws)->pool;
+  P.lcnt = reinterpret_cast<int*>(ws + L.lcnt);
   for (int l = 0; l < n_layers; ++l) {
     const pi_layer_weights& w = layers[l];
     pi::StackLayer& s = P.layers[l];
@@ -227,6 +246,8 @@ pi_status fused_stack(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, cons
     s.wd_sc = w.W_downT.scales;
     s.b1 = w.b1;
     s.b2 = w.b2;
+    // a neuron item carries the 16-byte block of b1 that holds its bias
+    if (w.b1 && (reinterpret_cast<uintptr_t>(w.b1) & 15u)) return PI_ERR_UNSUPPORTED;
     s.thr = w.threshold;
   }
   PI_CUDA(pi::launch_stack(desc->wtype, desc->ptype, B, P, G, smem, st), "fused decode-step launch");

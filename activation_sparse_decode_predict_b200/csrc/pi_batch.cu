@@ -1,0 +1,507 @@
+// pi_batch.cu -- the sparse FFN of a token block of 3..16 tokens on the
+// tensor cores (fp16 weights, fp16 tokens).
+//
+// PowerInfer (unite.ai, "Nöron Bilinçli Operatör"; aibars.net,
+// "Sparsity-Nutzung"): only the rows of the hot neurons and of the
+// predicted-active cold neurons are read.  With several tokens in a block
+// every streamed row serves all of them, so the per-neuron dots become small
+// matrix products -- [rows x d] x [d x B] for gate/up and [B x n] x [n x d] for
+// down -- done with mma.sync m16n8k16 (fp16 in, fp32 accumulate) while the
+// weight rows stream through shared memory by 1-D bulk copies.  The work is
+// HBM-bound (at most 16 FMAs per fp16 weight), so the tensor cores only have
+// to keep up with the copies; the layout rules of the bulk copies and of
+// ldmatrix decide the speed.
+//
+// k_bup    CTA = (range of list positions, part of d).  The gate and up rows
+//          of the range, columns of the part, against the tokens' columns of
+//          the part: pre-activation dots -> pre[part][pos][2][B] fp32.
+// k_bdown  CTA = (chunk of d, range of list positions).  Activations from
+//          pre (summed over the parts) and b1, split into fp16 hi + lo so the
+//          product keeps ~22 bits of each activation; fp32 partial output of
+//          the chunk -> partial[range][B][d]; the split-K reduce kernel adds
+//          the ranges and b2.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "pi_batch.cuh"
+#include "pi_common.cuh"
+#include "pi_mma.cuh"
+#include "pi_sync.cuh"
+
+namespace pi {
+
+namespace {
+
+constexpr int kBW = 8;          // consumer warps
+constexpr int kBT = kBW * 32;   // consumer threads
+constexpr int kBSmem = 227 * 1024;
+constexpr int kBMaxSlots = 8;
+
+__device__ __forceinline__ int bshare(int n, int c, int G) { return (int)((int64_t)n * c / G); }
+
+// list position -> neuron row (hot rows first, then the predicted list);
+// an entry outside [n_hot, ffn) is reported and replaced by row 0
+__device__ __forceinline__ int list_row(int pos, int n_hot, int ffn, const int32_t* idx, Ctrl* ctrl) {
+  if (pos < n_hot) return pos;
+  const int j = __ldg(idx + (pos - n_hot));
+  if (j < n_hot || j >= ffn) {
+    set_status(&ctrl->status, kStIndex);
+    return -1;
+  }
+  return j;
+}
+
+__device__ __forceinline__ int clamp_count(const int32_t* count, int C, Ctrl* ctrl, bool report) {
+  int cnt = *count;
+  if (cnt < 0 || cnt > C) {
+    if (report) set_status(&ctrl->status, kStCapacity);
+    cnt = cnt < 0 ? 0 : C;
+  }
+  return cnt;
+}
+
+// ---------------------------------------------------------------------------
+// shared-memory layouts (host and device agree through these functions)
+
+struct UpLayout {
+  int PC, KC, HS, RS, ISZ, off_h, off_red, off_ring, nslot, bytes;
+};
+
+__host__ __device__ inline UpLayout up_layout(int B8, int d, int S) {
+  UpLayout L;
+  L.PC = d / S;
+  L.KC = (L.PC % 1024 == 0) ? 1024 : (L.PC % 512 == 0) ? 512 : (L.PC % 256 == 0) ? 256 : 128;
+  L.HS = L.PC * 2 + 16;   // token row stride (bytes): +16 keeps ldmatrix rows on distinct banks
+  L.RS = L.KC * 2 + 16;   // weight row stride in a ring slot
+  L.ISZ = 16 * L.RS;      // one slot: 16 rows x KC columns
+  L.off_h = 2 * 8 * kBMaxSlots;
+  L.off_h = (L.off_h + 127) & ~127;
+  L.off_red = L.off_h + ((B8 * L.HS + 127) & ~127);
+  L.off_ring = L.off_red + 2 * kBW * 16 * 16 * 4;
+  const int room = kBSmem - L.off_ring;
+  L.nslot = room / L.ISZ;
+  if (L.nslot > kBMaxSlots) L.nslot = kBMaxSlots;
+  L.bytes = L.off_ring + L.nslot * L.ISZ;
+  return L;
+}
+
+struct DownLayout {
+  int DCOLS, RS, ISZ, off_a, off_ring, nslot, bytes;
+};
+
+constexpr int kARow = 48;  // bytes per token row of an activation tile (16 fp16 + pad: conflict-free ldmatrix)
+
+__host__ __device__ inline DownLayout down_layout(int d) {
+  DownLayout L;
+  L.DCOLS = (d % 1024 == 0) ? 1024 : (d % 512 == 0) ? 512 : 256;
+  L.RS = L.DCOLS * 2 + 16;
+  L.ISZ = 16 * L.RS;
+  L.off_a = 2 * 8 * kBMaxSlots;
+  L.off_a = (L.off_a + 127) & ~127;
+  L.off_ring = L.off_a + 2 * 2 * 16 * kARow;  // [buffer][hi, lo][16 token rows]
+  L.off_ring = (L.off_ring + 127) & ~127;
+  const int room = kBSmem - L.off_ring;
+  L.nslot = room / L.ISZ;
+  if (L.nslot > kBMaxSlots) L.nslot = kBMaxSlots;
+  L.bytes = L.off_ring + L.nslot * L.ISZ;
+  return L;
+}
+
+// ---------------------------------------------------------------------------
+
+struct BUpParams {
+  const __half* h;   // [B, d]
+  const __half* wg;  // [F, d] (ReGLU only)
+  const __half* wu;  // [F, d]
+  const int32_t* idx;
+  const int32_t* count;
+  float* pre;  // [S][F][2][B]
+  Ctrl* ctrl;
+  int B, d, ffn, n_hot, S, gated;
+};
+
+template <int NT>
+__global__ void __launch_bounds__(kBT + 32, 1) k_bup(const __grid_constant__ BUpParams p) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  const UpLayout Lay = up_layout(NT * 8, p.d, p.S);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm);
+  uint64_t* empty = full + kBMaxSlots;
+  uint8_t* hs = sm + Lay.off_h;
+  float* red = reinterpret_cast<float*>(sm + Lay.off_red);
+  uint8_t* ring = sm + Lay.off_ring;
+  Ctrl* ctrl = p.ctrl;
+
+  const int R = gridDim.x / p.S;
+  const int rho = blockIdx.x / p.S, sig = blockIdx.x % p.S;
+  const int col0 = sig * Lay.PC;
+  const int C = p.ffn - p.n_hot;
+  const int ntot = p.n_hot + clamp_count(p.count, C, ctrl, blockIdx.x == 0 && threadIdx.x == 0);
+  const int n0 = bshare(ntot, rho, R), n1 = bshare(ntot, rho + 1, R);
+  const int npt = p.gated ? 8 : 16;  // neurons per 16-row tile
+  const int ntile = (n1 - n0 + npt - 1) / npt;
+  const int nch = Lay.PC / Lay.KC;
+  const int nitems = ntile * nch;
+  const int nslot = Lay.nslot;
+
+  if (threadIdx.x == 0) {
+    for (int q = 0; q < nslot; ++q) {
+      mbar_init(&full[q], 1);
+      mbar_init(&empty[q], kBW);
+    }
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  if (threadIdx.x < 32) {
+    // ---------------- producer warp: one row per lane ----------------
+    const int lane = threadIdx.x;
+    for (int it = 0; it < nitems; ++it) {
+      const int q = it % nslot;
+      bool ok = true;
+      if (it >= nslot) ok = mbar_wait(&empty[q], ((it / nslot) - 1) & 1, ctrl);
+      if (!__all_sync(0xffffffffu, ok)) return;
+      const int tile = it / nch, ch = it % nch;
+      if (lane == 0) mbar_arrive_expect_tx(&full[q], 16u * Lay.KC * 2u);
+      __syncwarp();
+      if (lane < 16) {
+        int pos = n0 + tile * npt + (p.gated ? lane / 2 : lane);
+        if (pos >= n1) pos = n1 - 1;  // tail rows repeat the last one; their dots are dropped
+        int j = list_row(pos, p.n_hot, p.ffn, p.idx, ctrl);
+        if (j < 0) j = 0;
+        const __half* mat = p.gated ? ((lane & 1) ? p.wu : p.wg) : p.wu;
+        bulk_g2s(ring + q * Lay.ISZ + lane * Lay.RS, mat + (int64_t)j * p.d + col0 + ch * Lay.KC, Lay.KC * 2u,
+                 &full[q]);
+      }
+      __syncwarp();
+    }
+    // the CTA may exit only once its copies have landed
+    for (int it = nitems > nslot ? nitems - nslot : 0; it < nitems; ++it)
+      if (lane == 0) mbar_wait(&full[it % nslot], (it / nslot) & 1, ctrl);
+    return;
+  }
+
+  // ---------------- consumer warps ----------------
+  const int t = threadIdx.x - 32, cw = t >> 5, lane = t & 31;
+  // this part's token columns -> shared memory (rows >= B are zero)
+  {
+    const int units = Lay.PC / 8;
+    for (int i = t; i < NT * 8 * units; i += kBT) {
+      const int b = i / units, u = i % units;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (b < p.B) v = __ldg(reinterpret_cast<const uint4*>(p.h + (int64_t)b * p.d + col0) + u);
+      *reinterpret_cast<uint4*>(hs + b * Lay.HS + 16 * u) = v;
+    }
+  }
+  named_sync(1, kBT);
+
+  const int KSc = Lay.KC / 16;
+  const int ks0 = cw * KSc / kBW, ks1 = (cw + 1) * KSc / kBW;
+  const uint32_t a_lane = (uint32_t)((lane & 15) * Lay.RS + (lane >> 4) * 16);
+  const uint32_t b_lane = smem_u32(hs) + (uint32_t)((lane & 7) * Lay.HS + ((lane >> 3) & 1) * 16);
+  float acc[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+  bool to = false;
+  for (int it = 0; it < nitems; ++it) {
+    const int q = it % nslot;
+    const int tile = it / nch, ch = it % nch;
+    to |= !mbar_wait(&full[q], (it / nslot) & 1, ctrl);
+    if (!to) {
+      const uint32_t a_base = smem_u32(ring + q * Lay.ISZ) + a_lane;
+      const uint32_t b_base = b_lane + (uint32_t)(ch * Lay.KC * 2);
+      for (int ks = ks0; ks < ks1; ++ks) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(a_base + 32u * ks, a0, a1, a2, a3);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          uint32_t b0, b1;
+          ldsm_x2(b_base + (uint32_t)(nt * 8 * Lay.HS) + 32u * ks, b0, b1);
+          mma_16816(acc[nt], a0, a1, a2, a3, b0, b1);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[q]);
+    if (ch == nch - 1) {
+      // tile complete: partial dots of each warp -> shared memory, summed per (row, token)
+      float* rb = red + (tile & 1) * kBW * 256;
+      {
+        const int g = lane >> 2, c2 = 2 * (lane & 3);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          float* w = rb + cw * 256;
+          w[g * 16 + nt * 8 + c2] = acc[nt][0];
+          w[g * 16 + nt * 8 + c2 + 1] = acc[nt][1];
+          w[(g + 8) * 16 + nt * 8 + c2] = acc[nt][2];
+          w[(g + 8) * 16 + nt * 8 + c2 + 1] = acc[nt][3];
+          acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+        }
+      }
+      if (named_sync_or(1, kBT, to)) return;
+      const int row = t >> 4, tok = t & 15;
+      if (tok < p.B) {
+        const int pos = n0 + tile * npt + (p.gated ? row / 2 : row);
+        if (pos < n1) {
+          float v = 0.f;
+#pragma unroll
+          for (int w = 0; w < kBW; ++w) v += rb[w * 256 + row * 16 + tok];
+          const int which = p.gated ? (row & 1) : 1;  // 0: gate, 1: up
+          p.pre[(((int64_t)sig * p.ffn + pos) * 2 + which) * p.B + tok] = v;
+        }
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+
+struct BDownParams {
+  const float* pre;   // [S][F][2][B]
+  const float* b1;    // [F] or null
+  const __half* wd;   // [F, d] (W_down transposed: neuron-major)
+  const int32_t* idx;
+  const int32_t* count;
+  float* partial;     // [NR][B][d]
+  Ctrl* ctrl;
+  int B, d, ffn, n_hot, S, act, NR;
+};
+
+template <int NT>
+__global__ void __launch_bounds__(kBT + 32, 1) k_bdown(const __grid_constant__ BDownParams p) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  const DownLayout Lay = down_layout(p.d);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm);
+  uint64_t* empty = full + kBMaxSlots;
+  uint8_t* abuf = sm + Lay.off_a;
+  uint8_t* ring = sm + Lay.off_ring;
+  Ctrl* ctrl = p.ctrl;
+
+  const int DC = p.d / Lay.DCOLS;
+  const int chi = blockIdx.x % DC, rho = blockIdx.x / DC;
+  const int cbase = chi * Lay.DCOLS;
+  const int C = p.ffn - p.n_hot;
+  const int ntot = p.n_hot + clamp_count(p.count, C, ctrl, false);
+  const int n0 = bshare(ntot, rho, p.NR), n1 = bshare(ntot, rho + 1, p.NR);
+  const int ntile = (n1 - n0 + 15) / 16;
+  const int nslot = Lay.nslot;
+
+  if (threadIdx.x == 0) {
+    for (int q = 0; q < nslot; ++q) {
+      mbar_init(&full[q], 1);
+      mbar_init(&empty[q], kBW);
+    }
+    mbar_fence_init();
+  }
+  // activation tiles start zero (token rows >= B stay zero)
+  for (int i = threadIdx.x; i < 2 * 2 * 16 * kARow / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(abuf)[i] = make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();
+
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    for (int it = 0; it < ntile; ++it) {
+      const int q = it % nslot;
+      bool ok = true;
+      if (it >= nslot) ok = mbar_wait(&empty[q], ((it / nslot) - 1) & 1, ctrl);
+      if (!__all_sync(0xffffffffu, ok)) return;
+      if (lane == 0) mbar_arrive_expect_tx(&full[q], 16u * Lay.DCOLS * 2u);
+      __syncwarp();
+      if (lane < 16) {
+        int pos = n0 + it * 16 + lane;
+        if (pos >= n1) pos = n1 - 1;  // tail rows repeat the last one; their activations are zero
+        int j = list_row(pos, p.n_hot, p.ffn, p.idx, ctrl);
+        if (j < 0) j = 0;
+        bulk_g2s(ring + q * Lay.ISZ + lane * Lay.RS, p.wd + (int64_t)j * p.d + cbase, Lay.DCOLS * 2u, &full[q]);
+      }
+      __syncwarp();
+    }
+    for (int it = ntile > nslot ? ntile - nslot : 0; it < ntile; ++it)
+      if (lane == 0) mbar_wait(&full[it % nslot], (it / nslot) & 1, ctrl);
+    return;
+  }
+
+  const int t = threadIdx.x - 32, cw = t >> 5, lane = t & 31;
+  constexpr int kMT = 8;  // m-tiles (16 columns each) per warp at most
+  const int MT = Lay.DCOLS / (kBW * 16);
+  const int wcol = cw * MT * 16;  // this warp's first column within the chunk
+  float acc[kMT][NT][4];
+#pragma unroll
+  for (int m = 0; m < kMT; ++m)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) acc[m][nt][0] = acc[m][nt][1] = acc[m][nt][2] = acc[m][nt][3] = 0.f;
+  const int gated = p.act == kReglu;
+  const uint32_t a_lane = (uint32_t)(((lane & 7) + 8 * (lane >> 4)) * Lay.RS + ((lane >> 3) & 1) * 16 + wcol * 2);
+  const uint32_t b_lane = smem_u32(abuf) + (uint32_t)((lane & 7) * kARow + ((lane >> 3) & 1) * 16);
+  bool to = false;
+  for (int it = 0; it < ntile; ++it) {
+    // activations of the tile's 16 neurons, split into fp16 hi + lo
+    const int buf = it & 1;
+    {
+      const int i = t >> 4, b = t & 15;
+      const int pos = n0 + it * 16 + i;
+      if (b < p.B) {
+        float a = 0.f;
+        if (pos < n1) {
+          const int j = list_row(pos, p.n_hot, p.ffn, p.idx, ctrl);
+          if (j >= 0) {
+            float g = 0.f, v = 0.f;
+            for (int s = 0; s < p.S; ++s) {
+              const float* pr = p.pre + (((int64_t)s * p.ffn + pos) * 2) * p.B + b;
+              g += __ldcg(pr);
+              v += __ldcg(pr + p.B);
+            }
+            const float bias = p.b1 ? __ldg(p.b1 + j) : 0.f;
+            a = gated ? act_eval(kReglu, g + bias, v) : act_eval(p.act, v + bias, 0.f);
+          }
+        }
+        const __half hi = __float2half_rn(a);
+        const __half lo = __float2half_rn(a - __half2float(hi));
+        reinterpret_cast<__half*>(abuf + ((buf * 2 + 0) * 16 + b) * kARow)[i] = hi;
+        reinterpret_cast<__half*>(abuf + ((buf * 2 + 1) * 16 + b) * kARow)[i] = lo;
+      }
+    }
+    const int q = it % nslot;
+    to |= !mbar_wait(&full[q], (it / nslot) & 1, ctrl);
+    if (named_sync_or(1, kBT, to)) return;  // activation tile complete
+    {
+      const uint32_t a_base = smem_u32(ring + q * Lay.ISZ) + a_lane;
+      uint32_t bh[NT][2], bl[NT][2];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        ldsm_x2(b_lane + (uint32_t)(((buf * 2 + 0) * 16 + nt * 8) * kARow), bh[nt][0], bh[nt][1]);
+        ldsm_x2(b_lane + (uint32_t)(((buf * 2 + 1) * 16 + nt * 8) * kARow), bl[nt][0], bl[nt][1]);
+      }
+#pragma unroll
+      for (int m = 0; m < kMT; ++m) {
+        if (m < MT) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(a_base + 32u * m, a0, a1, a2, a3);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            mma_16816(acc[m][nt], a0, a1, a2, a3, bh[nt][0], bh[nt][1]);
+            mma_16816(acc[m][nt], a0, a1, a2, a3, bl[nt][0], bl[nt][1]);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[q]);
+  }
+  // partial output of this range and chunk (zeros for an empty range)
+  {
+    const int g = lane >> 2, c2 = 2 * (lane & 3);
+    float* out = p.partial + (int64_t)rho * p.B * p.d + cbase + wcol;
+#pragma unroll
+    for (int m = 0; m < kMT; ++m) {
+      if (m < MT) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const int b0 = nt * 8 + c2;
+          if (b0 < p.B) {
+            out[(int64_t)b0 * p.d + m * 16 + g] = acc[m][nt][0];
+            out[(int64_t)b0 * p.d + m * 16 + g + 8] = acc[m][nt][2];
+          }
+          if (b0 + 1 < p.B) {
+            out[(int64_t)(b0 + 1) * p.d + m * 16 + g] = acc[m][nt][1];
+            out[(int64_t)(b0 + 1) * p.d + m * 16 + g + 8] = acc[m][nt][3];
+          }
+        }
+      }
+    }
+  }
+}
+
+int up_parts(int B, int d) {
+  // the tokens' columns of one part stay in shared memory: at most 64 KB
+  const size_t bytes = (size_t)((B + 7) / 8 * 8) * d * 2;
+  int S = 1;
+  while ((size_t)S * 65536 < bytes) S *= 2;
+  return S;
+}
+
+}  // namespace
+
+bool batch_supported(int wtype, int ptype, int d, int B) {
+  if (wtype != kF16 || ptype != kF16) return false;
+  if (B < kBatchMin || B > 16) return false;
+  if (d % 256 != 0) return false;
+  const int S = up_parts(B, d);
+  if (S > 4 || d % (128 * S) != 0) return false;
+  const UpLayout U = up_layout((B + 7) / 8 * 8, d, S);
+  const DownLayout D = down_layout(d);
+  return U.nslot >= 2 && D.nslot >= 2;
+}
+
+size_t batch_pre_bytes(int ffn, int B) { return (size_t)4 * ffn * 2 * B * sizeof(float); }
+
+int batch_ranges(int d, int sms) {
+  const DownLayout D = down_layout(d);
+  const int DC = d / D.DCOLS;
+  const int NR = sms / DC;
+  return NR < 1 ? 1 : NR;
+}
+
+cudaError_t launch_batch_ffn(int act, const void* h, int B, int d, int ffn, int n_hot, const int32_t* idx,
+                             const int32_t* count, const void* wg, const void* wu, const void* wd, const float* b1,
+                             float* pre, float* partial, int NR, Ctrl* ctrl, int sms, cudaStream_t st) {
+  const int S = up_parts(B, d);
+  const int NT = B > 8 ? 2 : 1;
+  BUpParams U;
+  U.h = static_cast<const __half*>(h);
+  U.wg = static_cast<const __half*>(wg);
+  U.wu = static_cast<const __half*>(wu);
+  U.idx = idx;
+  U.count = count;
+  U.pre = pre;
+  U.ctrl = ctrl;
+  U.B = B;
+  U.d = d;
+  U.ffn = ffn;
+  U.n_hot = n_hot;
+  U.S = S;
+  U.gated = act == kReglu;
+  const UpLayout UL = up_layout(NT * 8, d, S);
+  const int Gu = (sms / S) * S;
+  cudaError_t e;
+  if (NT == 1) {
+    e = cudaFuncSetAttribute(k_bup<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, UL.bytes);
+    if (e != cudaSuccess) return e;
+    k_bup<1><<<Gu, kBT + 32, UL.bytes, st>>>(U);
+  } else {
+    e = cudaFuncSetAttribute(k_bup<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, UL.bytes);
+    if (e != cudaSuccess) return e;
+    k_bup<2><<<Gu, kBT + 32, UL.bytes, st>>>(U);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  BDownParams D;
+  D.pre = pre;
+  D.b1 = b1;
+  D.wd = static_cast<const __half*>(wd);
+  D.idx = idx;
+  D.count = count;
+  D.partial = partial;
+  D.ctrl = ctrl;
+  D.B = B;
+  D.d = d;
+  D.ffn = ffn;
+  D.n_hot = n_hot;
+  D.S = S;
+  D.act = act;
+  D.NR = NR;
+  const DownLayout DL = down_layout(d);
+  const int Gd = NR * (d / DL.DCOLS);
+  if (NT == 1) {
+    e = cudaFuncSetAttribute(k_bdown<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, DL.bytes);
+    if (e != cudaSuccess) return e;
+    k_bdown<1><<<Gd, kBT + 32, DL.bytes, st>>>(D);
+  } else {
+    e = cudaFuncSetAttribute(k_bdown<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, DL.bytes);
+    if (e != cudaSuccess) return e;
+    k_bdown<2><<<Gd, kBT + 32, DL.bytes, st>>>(D);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace pi

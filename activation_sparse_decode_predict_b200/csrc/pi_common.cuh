@@ -30,8 +30,9 @@ struct Ctrl {
   unsigned pad1[15];
   unsigned bar_base;   // bar_count at the start of the next persistent launch
   unsigned pad2[15];
+  int pool[128];       // per-layer claim counters of the persistent kernel (zero between launches)
 };
-static_assert(sizeof(Ctrl) == 256, "control block is 256 bytes");
+static_assert(sizeof(Ctrl) == 768, "control block is 768 bytes");
 
 __device__ __forceinline__ void set_status(int* status, int code) { atomicCAS(status, 0, code); }
 
@@ -157,6 +158,14 @@ __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
+}
+
+// The activation with the kind chosen at run time (g: gate or up
+// pre-activation incl. bias; v: up dot, used by ReGLU only).
+__device__ __forceinline__ float act_eval(int act, float g, float v) {
+  if (act == kReglu) return fmaxf(g, 0.f) * v;
+  const float r = fmaxf(g, 0.f);
+  return act == kRelu2 ? r * r : r;
 }
 
 template <int ACT>

@@ -1,8 +1,10 @@
 // pi_layout.h -- byte layout of a libpi workspace (host side).
 //
-//   [ctrl 256 B][u: B x rank fp32][tile masks][tile counts][a: B x ffn fp32]
+//   [ctrl 768 B: status, abort, barrier count and base, claim counters][u: B x rank fp32][tile masks][tile counts][a: B x ffn fp32]
 //   [partials: G_MAX x B x d fp32][y: B x d fp32][h: B x d fp32]
-//   [y accumulators: 2 x 8 x B x d fp32][per-CTA active lists][per-CTA counts]
+//   [y accumulators: 2 x 8 x B x d fp32][list counts: 128 x G_MAX]
+//   [pre-activations of the tensor-core token-block path: 4 x ffn x 2 x B fp32,
+//    token blocks of 3 or more only]
 //
 // Every region starts on a 256-byte boundary.  The layout depends only on the
 // descriptor and the batch, never on the device.
@@ -14,9 +16,11 @@ namespace pi {
 
 constexpr int kGMax = 296;  // split-K partial slots (2 x 148 SMs)
 constexpr int kYAccCopies = 8;  // copies of the persistent kernel's fp32 output accumulator
+constexpr int kLayersMax = 128;  // layers of one decode-stack call
+constexpr size_t kCtrlBytes = 768;  // the control block at the start of a workspace
 
 struct WsLayout {
-  size_t u, tile_mask, tile_count, act, partial, ybuf, hbuf, yacc, seg, seg_cnt, total;
+  size_t u, tile_mask, tile_count, act, partial, ybuf, hbuf, yacc, lcnt, pre, total;
   int n_tiles, g_max;
 };
 
@@ -24,7 +28,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 inline WsLayout ws_layout(int d, int ffn, int n_hot, int rank, int B) {
   WsLayout L;
-  size_t off = 256;
+  size_t off = kCtrlBytes;
   const int C = ffn - n_hot;
   L.n_tiles = (C + 255) / 256;
   L.g_max = kGMax;
@@ -36,8 +40,8 @@ inline WsLayout ws_layout(int d, int ffn, int n_hot, int rank, int B) {
   L.ybuf = off; off += align256((size_t)B * d * 4);
   L.hbuf = off; off += align256((size_t)B * d * 4);
   L.yacc = off; off += align256((size_t)2 * kYAccCopies * B * d * 4);
-  L.seg = off; off += align256((size_t)(C + 2 * kGMax) * 4);
-  L.seg_cnt = off; off += align256((size_t)kGMax * 4);
+  L.lcnt = off; off += align256((size_t)kLayersMax * kGMax * 4);
+  L.pre = off; off += B >= 3 ? align256((size_t)4 * ffn * 2 * B * 4) : 0;
   L.total = off;
   return L;
 }

@@ -1,8 +1,7 @@
 // pi_mma.cuh -- warp-level fp16 tensor-core helpers (ldmatrix + mma.sync
-// m16n8k16, fp32 accumulation) used for the predictor's dot products inside
-// the persistent kernel.  A: 16 weight rows x 16 columns (row-major, from the
-// shared-memory ring); B: 16 columns x 8 "tokens" (stored transposed, one
-// shared-memory row per token); D: 16 x 8 fp32.
+// m16n8k16, fp32 accumulation).  A: 16 x 16 (row-major, or loaded with the
+// transposing ldmatrix from k-major storage); B: 16 x 8, stored as one
+// shared-memory row of 16 k-values per column; D: 16 x 8 fp32.
 #pragma once
 
 #include <stdint.h>
@@ -11,6 +10,14 @@ namespace pi {
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr)
+               : "memory");
+}
+
+// Four 8x8 b16 matrices, each transposed on the way in.
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                : "r"(addr)
                : "memory");

@@ -13,20 +13,22 @@
 // Design (one CTA per SM, G CTAs, grid-wide barriers are bounded spins):
 //   * a producer warp streams every byte the CTA needs into a shared-memory
 //     byte ring with 1-D bulk copies (cp.async.bulk, mbarrier completion), in
-//     a fixed order per layer: its P1 rows, its block of P2 rows, its share
-//     of the hot neurons (gate/up/down rows of each neuron as one item), then
-//     -- once every CTA has scored its P2 rows -- its share of the predicted
-//     cold neurons.  Nothing but the cold rows depends on the predictor, so
-//     the ring keeps HBM busy across the grid barriers.
-//   * consumer warps own 16 fixed columns of d per thread: the token block
-//     and the fp32 partial output stay in registers for the whole layer.
-//   * per layer: P1 rows -> u (global) -> barrier U -> P2 scores of the CTA's
-//     cold rows -> local ascending list + count -> barrier S -> hot neurons ->
-//     cold share of the global list -> partial y reduced into an fp32
-//     accumulator with vector atomics -> barrier Y -> residual + RMSNorm glue
-//     computed redundantly by every CTA -> next layer.
-//   * the cold list is ordered: CTA c's active rows are ascending and precede
-//     CTA c+1's, so the concatenation is the ascending list pi_predict writes.
+//     consumption order per layer: its P1 rows, a static share of the hot
+//     neurons, its block of P2 rows, then a stream of neurons: the cold rows
+//     its own CTA predicted active and chunks of the remaining hot neurons
+//     claimed from a per-layer atomic counter (the claims balance the
+//     per-CTA cold counts).  A neuron item is its gate/up/down rows plus the
+//     16-byte block of b1 that holds its bias.
+//   * consumer warps own fixed columns of d: the token block and the fp32
+//     partial output stay in registers for the whole layer.
+//   * per layer: P1 rows -> u (global) -> barrier U (static hot neurons fill
+//     the wait) -> P2 scores of the CTA's cold rows -> local ascending list ->
+//     neuron stream -> partial y added into an fp32 accumulator with vector
+//     atomics -> barrier Y -> residual + RMSNorm glue computed redundantly by
+//     every CTA -> next layer.  Two grid barriers per layer.
+//   * the ascending list pi_predict would write is each CTA's local list in
+//     CTA order; every CTA parks its list in place and the lists are
+//     compacted once, after the last layer.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -149,12 +151,6 @@ __device__ __forceinline__ float round_to(int X, float v) {
   return X == kF16 ? __half2float(__float2half_rn(v)) : v;
 }
 
-__device__ __forceinline__ float act_eval(int act, float g, float v) {
-  if (act == kReglu) return fmaxf(g, 0.f) * v;
-  const float r = fmaxf(g, 0.f);
-  return act == kRelu2 ? r * r : r;
-}
-
 __device__ __forceinline__ int wrow_bytes(int WT_, int d) {
   return WT_ == kQ4_0 ? d / 2 + d / 16 : d * (WT_ == kF16 ? 2 : 4);
 }
@@ -165,16 +161,17 @@ struct Smem {
   uint64_t* empty;
   uint64_t* list_bar;
   uint32_t* item_off;
-  uint32_t* istart;  // producer-private: start/size of the items in flight
+  uint32_t* istart;  // producer-private: start of the items in flight
+  int* item_j;       // neuron row of a neuron item; -1 for an end marker
+  int* item_gs;      // on the first item of a group: the group's size (0: end marker)
   float* u;          // [B][r] split layout (see load_u)
   float* bp;
-  float* b1hot;
-  int* cidx;
-  float* cb1;
+  int* cidx;         // this CTA's predicted-active cold rows (neuron ids), ascending
   uint8_t* act;
+  float* sc;  // partial P2 scores [rows][B]
   float* red;        // [2][NW][2B]
-  int* prefix;       // [G + 1]
-  int* misc;         // [0] cold_n, [1] gen_start
+  float* gred;       // [kMaxGroup][NW][2B] per-warp gate/up dots (CUDA-core groups)
+  int* misc;         // [0] local cold count, [1] barrier base, [2] next group size, [3] scratch
   uint8_t* hb;       // [B][d + 8] fp16 token rows (tensor-core operand)
   uint8_t* ub;       // [2B][r + 8] fp16 u rows: hi and lo parts of each token's u
   uint8_t* zero;     // 16 zero bytes (operand rows beyond the token count)
@@ -189,14 +186,15 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const StackParams& p) {
   s.list_bar = s.empty + kNQ;
   s.item_off = reinterpret_cast<uint32_t*>(base + p.off_itemoff);
   s.istart = s.item_off + kNQ;
+  s.item_j = reinterpret_cast<int*>(s.item_off + 2 * kNQ);
+  s.item_gs = reinterpret_cast<int*>(s.item_off + 3 * kNQ);
   s.u = reinterpret_cast<float*>(base + p.off_u);
   s.bp = reinterpret_cast<float*>(base + p.off_bp);
-  s.b1hot = reinterpret_cast<float*>(base + p.off_b1hot);
   s.cidx = reinterpret_cast<int*>(base + p.off_cidx);
-  s.cb1 = reinterpret_cast<float*>(base + p.off_cb1);
   s.act = base + p.off_act;
+  s.sc = reinterpret_cast<float*>(base + p.off_sc);
   s.red = reinterpret_cast<float*>(base + p.off_red);
-  s.prefix = reinterpret_cast<int*>(base + p.off_prefix);
+  s.gred = reinterpret_cast<float*>(base + p.off_gred);
   s.misc = reinterpret_cast<int*>(base + p.off_misc);
   s.hb = base + p.off_hb;
   s.ub = base + p.off_ub;
@@ -318,27 +316,31 @@ struct Producer {
     return true;
   }
 
-  // One neuron: its gate (ReGLU only), up and down rows.  Row m of the item
-  // starts m * (wrb + 16) bytes past a 128-byte aligned base that is shifted
-  // by 32 * (neuron sequence number mod 4) bytes, so that the gate and up
-  // rows of four consecutive neurons fall on eight different shared-memory
-  // bank groups (conflict-free ldmatrix).  Q4_0 rows hold qs then sc.
+  // One neuron: its gate (ReGLU only), up and down rows, then (with a b1)
+  // the 16-byte block of b1 that holds its bias.  Row m of the item starts
+  // m * (wrb + 16) bytes past a 128-byte aligned base that is shifted by
+  // 32 * (neuron sequence number mod 4) bytes, so that the gate and up rows
+  // of four consecutive neurons fall on eight different shared-memory bank
+  // groups (conflict-free ldmatrix).  Q4_0 rows hold qs then sc.  gs > 0
+  // marks the first item of a group of gs neurons.
   uint32_t nseq = 0;
-  __device__ bool issue_neuron(const StackLayer& Ly, int j, int wt, int gated) {
+  __device__ bool issue_neuron(const StackLayer& Ly, int j, int wt, int gated, int gs) {
     const int d = p.d;
     const uint32_t wrb = wt == kQ4_0 ? (uint32_t)(d / 2 + d / 16) : (uint32_t)(d * (wt == kF16 ? 2 : 4));
     const uint32_t wrp = wrb + 16;
     const int nrow = gated ? 3 : 2;
     const uint32_t skew = 32u * (nseq & 3u);
     ++nseq;
-    const uint32_t total = nrow * wrp + 128 + skew;
+    const uint32_t total = nrow * wrp + 16 + 128 + skew;
     uint32_t pos;
     if (!alloc(total, pos)) return false;
     const uint32_t start = ((pos + 127u) & ~127u) + skew;
     const uint32_t q = item % kNQ;
     s.item_off[q] = start;
     s.istart[q] = pos;
-    mbar_arrive_expect_tx(&s.full[q], nrow * wrb);
+    s.item_j[q] = j;
+    s.item_gs[q] = gs;
+    mbar_arrive_expect_tx(&s.full[q], nrow * wrb + (Ly.b1 ? 16u : 0u));
     const void* rows[3];
     const void* scs[3];
     int m = 0;
@@ -354,7 +356,33 @@ struct Producer {
         bulk_g2s(dst, reinterpret_cast<const uint8_t*>(rows[i]) + (int64_t)j * wrb, wrb, &s.full[q]);
       }
     }
+    if (Ly.b1) bulk_g2s(s.ring + start + nrow * wrp, Ly.b1 + (j & ~3), 16u, &s.full[q]);
     head = pos + total;
+    ++item;
+    return true;
+  }
+
+  // neurons j0 .. j0+n-1 in groups of at most ng
+  __device__ bool issue_range(const StackLayer& Ly, int j0, int n, int wt, int gated) {
+    bool ok = true;
+    for (int i = 0; i < n && ok; ++i) {
+      const int gs = (i % p.ng == 0) ? min(p.ng, n - i) : 0;
+      ok = issue_neuron(Ly, j0 + i, wt, gated, gs);
+    }
+    return ok;
+  }
+
+  // End of a neuron stream: an item without bytes (group size 0).
+  __device__ bool issue_marker() {
+    uint32_t pos;
+    if (!alloc(0, pos)) return false;
+    const uint32_t q = item % kNQ;
+    s.item_off[q] = pos;
+    s.istart[q] = pos;
+    s.item_j[q] = -1;
+    s.item_gs[q] = 0;
+    mbar_arrive(&s.full[q]);
+    head = pos;
     ++item;
     return true;
   }
@@ -396,7 +424,11 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
   // shares that do not depend on the predictor
   const int k0 = share_lo(r, c, G), k1 = share_lo(r, c + 1, G);
   const int c0 = share_lo(C, c, G), c1 = share_lo(C, c + 1, G);
-  const int j0 = share_lo(H, c, G), j1 = share_lo(H, c + 1, G);
+
+  // static hot share (consumed while barrier U completes); the rest of the
+  // hot neurons, [HA, H), is claimed in chunks through p.pool[l]
+  const int HA = p.hot_static;
+  const int a0 = share_lo(HA, c, G), a1 = share_lo(HA, c + 1, G);
 
   if (threadIdx.x < 32) {
     // ======================= producer warp =======================
@@ -406,11 +438,14 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
     for (int l = 0; l < p.L && ok; ++l) {
       const StackLayer& Ly = p.layers[l];
       if (lane == 0) {
+        // item order = consumption order
         if constexpr (PT == kF16) {
           // tensor-core predictor: skewed P1 rows, P2 in 16-row tiles with padded rows
           for (int k = k0; k < k1 && ok; ++k)
             ok = pr.issue_rows(reinterpret_cast<const uint8_t*>(Ly.P1) + (int64_t)k * d * 2, 0, 1, d * 2, d * 2,
                                16u * (uint32_t)((k - k0) & 7));
+          if (ok) ok = pr.issue_range(Ly, a0, a1 - a0, WT, gated);
+          if (ok) ok = pr.issue_marker();
           for (int cc = c0; cc < c1 && ok; cc += 16)
             ok = pr.issue_rows(reinterpret_cast<const uint8_t*>(Ly.P2) + (int64_t)cc * r * 2, (int64_t)r * 2,
                                min(16, c1 - cc), r * 2, r * 2 + 16, 0);
@@ -420,6 +455,8 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
             const uint32_t by = d * ep;
             ok = pr.issue(1, &src, &by);
           }
+          if (ok) ok = pr.issue_range(Ly, a0, a1 - a0, WT, gated);
+          if (ok) ok = pr.issue_marker();
           for (int cc = c0; cc < c1 && ok; cc += NW) {
             const int rows = min(NW, c1 - cc);
             const void* src = reinterpret_cast<const uint8_t*>(Ly.P2) + (int64_t)cc * r * ep;
@@ -427,60 +464,28 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
             ok = pr.issue(1, &src, &by);
           }
         }
-        for (int j = j0; j < j1 && ok; ++j) ok = pr.issue_neuron(Ly, j, WT, gated);
-        // the cold rows need every CTA's scores: barrier S of this layer
-        if (ok) ok = grid_wait(ctrl, base, 3 * l + 1, G);
+        // the neuron stream: one claimed hot chunk (covers the wait for the
+        // local list), the predicted cold rows, more claimed chunks, the end marker
+        const int PN = H - HA;
+        int* pool = p.pool + l;
+        int nxt = PN > 0 ? atomicAdd(pool, p.ng) : 0;
+        if (ok && nxt < PN) {
+          const int cur = nxt;
+          nxt = atomicAdd(pool, p.ng);
+          ok = pr.issue_range(Ly, HA + cur, min(p.ng, PN - cur), WT, gated);
+        }
+        if (ok) ok = mbar_wait(s.list_bar, l & 1, ctrl);
+        const int nloc = s.misc[0];
+        for (int q = 0; q < nloc && ok; ++q)
+          ok = pr.issue_neuron(Ly, s.cidx[q], WT, gated, (q % p.ng == 0) ? min(p.ng, nloc - q) : 0);
+        while (ok && nxt < PN) {
+          const int cur = nxt;
+          nxt = atomicAdd(pool, p.ng);
+          ok = pr.issue_range(Ly, HA + cur, min(p.ng, PN - cur), WT, gated);
+        }
+        if (ok) ok = pr.issue_marker();
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      __syncwarp();
-      if (!ok) break;
-      // prefix over the per-CTA counts (all loads in flight at once)
-      constexpr int kMaxChunks = (kGMaxCtas + 31) / 32;
-      int cv[kMaxChunks];
-#pragma unroll 1
-      for (int m = 0; m < kMaxChunks; ++m) {
-        const int i = m * 32 + lane;
-        cv[m] = i < G ? __ldcg(p.seg_cnt + i) : 0;
-      }
-      if (lane == 0) s.prefix[0] = 0;
-      int run = 0;
-#pragma unroll 1
-      for (int m = 0; m < kMaxChunks; ++m) {
-        int x = cv[m];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, x, o);
-          if (lane >= o) x += y;
-        }
-        const int i = m * 32 + lane;
-        if (i < G) s.prefix[i + 1] = run + x;
-        run += __shfl_sync(0xffffffffu, x, 31);
-      }
-      __syncwarp();
-      const int A = run;
-      const int q0 = share_lo(A, c, G), q1 = share_lo(A, c + 1, G);
-      for (int q = q0 + lane; q < q1; q += 32) {
-        int lo = 0, hi = G;  // last CTA with prefix[cta] <= q
-        while (hi - lo > 1) {
-          const int mid = (lo + hi) >> 1;
-          if (s.prefix[mid] <= q) lo = mid;
-          else hi = mid;
-        }
-        s.cidx[q - q0] = __ldcg(p.seg + (int64_t)lo * p.seg_cap + (q - s.prefix[lo]));
-      }
-      if (lane == 0) s.misc[0] = q1 - q0;
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(s.list_bar);
-        for (int q = 0; q < q1 - q0 && ok; ++q) ok = pr.issue_neuron(Ly, s.cidx[q], WT, gated);
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      // outputs (off the critical path): this CTA's part of the ascending list, and the count
-      const int my_n = s.prefix[c + 1] - s.prefix[c];
-      for (int i = lane; i < my_n; i += 32)
-        p.idx[(int64_t)l * C + s.prefix[c] + i] = __ldcg(p.seg + (int64_t)c * p.seg_cap + i);
-      if (c == 0 && lane == 0) p.counts[l] = A;
-      __syncwarp();
     }
     if (lane == 0) pr.drain();
     return;
@@ -527,17 +532,26 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
     for (int i = z0 + t; i < z1; i += T) reinterpret_cast<float4*>(p.yacc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 
-  for (int l = 0; l < p.L; ++l) {
-    const StackLayer& Ly = p.layers[l];
-    // small per-layer vectors of this CTA's shares: loaded now, stored to
-    // shared memory after the P1 rows so that the load latency is hidden
-    float bp_v[kShareRegs], b1_v[kShareRegs];
+  // the P2 biases of this CTA's cold rows: loaded one layer ahead into
+  // registers, stored to shared memory after P1
+  float bp_v[kShareRegs];
+  auto load_shares = [&](const StackLayer& Lz) {
 #pragma unroll
     for (int i = 0; i < kShareRegs; ++i) {
       const int x = t + i * T;
-      bp_v[i] = (Ly.bp && x < c1 - c0) ? __ldg(Ly.bp + c0 + x) : 0.f;
-      b1_v[i] = (Ly.b1 && x < j1 - j0) ? __ldg(Ly.b1 + j0 + x) : 0.f;
+      bp_v[i] = (Lz.bp && x < c1 - c0) ? __ldg(Lz.bp + c0 + x) : 0.f;
     }
+  };
+  load_shares(p.layers[0]);
+  const int wrp = wrow_bytes(WT, d) + 16;  // byte stride of a neuron item's rows
+  const int rpn = gated ? 2 : 1;           // gate/up rows per neuron
+
+  for (int l = 0; l < p.L; ++l) {
+    const StackLayer& Ly = p.layers[l];
+#pragma unroll
+    for (int b = 0; b < B; ++b)
+#pragma unroll
+      for (int e = 0; e < EPT; ++e) y[b][e] = 0.f;
 
     // ---- predictor step 1: u = ReLU(P1 h) ----
     bool to = false;
@@ -627,13 +641,149 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
     for (int i = 0; i < kShareRegs; ++i) {
       const int x = t + i * T;
       if (x < c1 - c0) s.bp[x] = bp_v[i];
-      if (x < j1 - j0) s.b1hot[x] = b1_v[i];
     }
+    // ---- neuron streams: groups of items until an end marker ----
+    // Every warp takes the same barriers in the same order; a group's size is
+    // read by thread 0 from the group's first item and passed on through
+    // shared memory behind a barrier, so every warp agrees on it.
+    float* gact = s.gred + kMaxGroup * (kMaxConsumers / 32) * 2 * B;  // [gs][B] activations
+    auto head_size = [&](uint32_t it) -> int {  // thread 0 only
+      to |= !mbar_wait(&s.full[it % kNQ], (it / kNQ) & 1u, ctrl);
+      return to ? 0 : s.item_gs[it % kNQ];
+    };
+    auto run_stream = [&]() -> bool {
+      if (t == 0) s.misc[2] = head_size(witem);
+      if (named_sync_or(1, T, to)) return false;
+      for (;;) {
+        const int gs = s.misc[2];
+        if (gs == 0) {  // the end marker: every warp releases it
+          ++witem;
+          release_item();
+          return true;
+        }
+        for (int i = 0; i < gs; ++i) to |= !mbar_wait(&s.full[(witem + i) % kNQ], ((witem + i) / kNQ) & 1u, ctrl);
+        if (!to) {
+          if constexpr (WT == kF16 && PT == kF16) {
+            // Tensor cores: the group's gate and up rows form one 16-row A tile
+            // (unused rows repeat the first neuron), the fp16 token rows the B
+            // tile; warps split d, partial dots meet in shared memory.
+            const int bn = lane & 7;
+            const uint32_t b_base =
+                bn < B ? smem_u32(s.hb + bn * HS) + (uint32_t)(((lane >> 3) & 1) * 16) : smem_u32(s.zero);
+            const uint32_t b_step = bn < B ? 32u : 0u;
+            const int KS = d / 16, ks0 = warp * KS / NW, ks1 = (warp + 1) * KS / NW;
+            const int tr = lane & 15;
+            const int jj = tr / rpn < gs ? tr / rpn : 0;
+            const int which = gated ? (tr & 1) : 0;  // item row: gate then up (ReGLU), up (otherwise)
+            const uint32_t a_base = smem_u32(s.ring + s.item_off[(witem + jj) % kNQ]) + (uint32_t)(which * wrp) +
+                                    (uint32_t)((lane >> 4) * 16);
+            float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+            int ks = ks0;
+            for (; ks + 1 < ks1; ks += 2) {
+              uint32_t a0, a1, a2, a3, b0, b1, e0, e1, e2, e3, f0, f1;
+              ldsm_x4(a_base + 32u * ks, a0, a1, a2, a3);
+              ldsm_x2(b_base + b_step * ks, b0, b1);
+              ldsm_x4(a_base + 32u * (ks + 1), e0, e1, e2, e3);
+              ldsm_x2(b_base + b_step * (ks + 1), f0, f1);
+              mma_16816(acc0, a0, a1, a2, a3, b0, b1);
+              mma_16816(acc1, e0, e1, e2, e3, f0, f1);
+            }
+            if (ks < ks1) {
+              uint32_t a0, a1, a2, a3, b0, b1;
+              ldsm_x4(a_base + 32u * ks, a0, a1, a2, a3);
+              ldsm_x2(b_base + b_step * ks, b0, b1);
+              mma_16816(acc0, a0, a1, a2, a3, b0, b1);
+            }
+            // thread (g = lane/4, lane%4 == 0) holds tile rows g and g+8, tokens 0 and 1
+            if ((lane & 3) == 0) {
+              const int g = lane >> 2;
+              float* rp = s.redp + warp * 32;
+              rp[g * 2 + 0] = acc0[0] + acc1[0];
+              rp[g * 2 + 1] = acc0[1] + acc1[1];
+              rp[(g + 8) * 2 + 0] = acc0[2] + acc1[2];
+              rp[(g + 8) * 2 + 1] = acc0[3] + acc1[3];
+            }
+          } else {
+            // CUDA cores: each thread's columns, one warp sum per dot
+            for (int jj = 0; jj < gs; ++jj) {
+              const uint8_t* it = s.ring + s.item_off[(witem + jj) % kNQ];
+              float acc[2 * B];
+              float wu[EPT];
+              w_vals<WT, EPT>(it + (gated ? wrp : 0), d, t, T, wu);
+#pragma unroll
+              for (int b = 0; b < B; ++b) {
+                float a = 0.f;
+#pragma unroll
+                for (int e = 0; e < EPT; ++e) a = fmaf(wu[e], h[b][e], a);
+                acc[B + b] = a;
+              }
+              if (gated) {
+                float wg[EPT];
+                w_vals<WT, EPT>(it, d, t, T, wg);
+#pragma unroll
+                for (int b = 0; b < B; ++b) {
+                  float a = 0.f;
+#pragma unroll
+                  for (int e = 0; e < EPT; ++e) a = fmaf(wg[e], h[b][e], a);
+                  acc[b] = a;
+                }
+              } else {
+#pragma unroll
+                for (int b = 0; b < B; ++b) acc[b] = 0.f;
+              }
+#pragma unroll
+              for (int i = 0; i < 2 * B; ++i) acc[i] = warp_sum(acc[i]);
+              if (lane == 0) {
+#pragma unroll
+                for (int i = 0; i < 2 * B; ++i) s.gred[(jj * NW + warp) * 2 * B + i] = acc[i];
+              }
+            }
+          }
+        }
+        if (named_sync_or(1, T, to)) return false;  // every partial dot of the group is in
+        if (t < gs * B) {
+          const int jj = t / B, b = t % B;
+          float gd = 0.f, vd = 0.f;
+          if constexpr (WT == kF16 && PT == kF16) {
+            for (int w = 0; w < NW; ++w) {
+              gd += s.redp[w * 32 + (jj * rpn) * 2 + b];
+              vd += s.redp[w * 32 + (jj * rpn + rpn - 1) * 2 + b];
+            }
+          } else {
+            for (int w = 0; w < NW; ++w) {
+              gd += s.gred[(jj * NW + w) * 2 * B + b];
+              vd += s.gred[(jj * NW + w) * 2 * B + B + b];
+            }
+          }
+          const uint32_t q = (witem + jj) % kNQ;
+          const float bias =
+              Ly.b1 ? reinterpret_cast<const float*>(s.ring + s.item_off[q] + (rpn + 1) * wrp)[s.item_j[q] & 3] : 0.f;
+          gact[jj * B + b] = gated ? act_eval(kReglu, gd + bias, vd) : act_eval(p.act, vd + bias, 0.f);
+        }
+        if (t == 0) s.misc[2] = head_size(witem + gs);  // the next group (or the end marker)
+        if (named_sync_or(1, T, to)) return false;
+        for (int jj = 0; jj < gs; ++jj) {
+          float wd[EPT];
+          w_vals<WT, EPT>(s.ring + s.item_off[(witem + jj) % kNQ] + rpn * wrp, d, t, T, wd);
+#pragma unroll
+          for (int b = 0; b < B; ++b) {
+            const float a = gact[jj * B + b];
+#pragma unroll
+            for (int e = 0; e < EPT; ++e) y[b][e] = fmaf(a, wd[e], y[b][e]);
+          }
+        }
+        witem += gs;
+        for (int i = 0; i < gs; ++i) release_item();
+      }
+    };
+
     named_sync(1, T);
     if (t == 0) grid_arrive(ctrl);
+    // the static hot neurons need no predictor: they fill the wait for barrier U
+    if (!run_stream()) return;
     {
       bool okw = true;
-      if (t == 0) okw = grid_wait(ctrl, base, 3 * l, G);
+      if (t == 0) okw = grid_wait(ctrl, base, 2 * l, G);
       if (named_sync_or(1, T, !okw)) return;
     }
     // the other accumulator buffer is free now (its last readers passed this barrier)
@@ -643,6 +793,7 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
       for (int i = z0 + t; i < z1; i += T) nxt[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     if constexpr (PT == kF16) {
+      for (int x = t; x < (c1 - c0) * B; x += T) s.sc[x] = 0.f;  // partial scores accumulate here
       // u -> fp16 rows for the tensor cores: row 2b = hi(u_b), row 2b+1 = lo(u_b) = u_b - hi
       for (int i = t; i < B * r; i += T) {
         const int b = i / r, k = i % r;
@@ -669,56 +820,61 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
 
     // ---- predictor step 2: scores of this CTA's cold rows ----
     if constexpr (PT == kF16) {
-      // Tensor cores: each 16-row tile of P2 (one ring item) against the u
-      // rows (hi, lo per token); warp w takes tiles w, w + NW, ...
+      // Tensor cores: 16-row tiles of P2 (one ring item each) against the u
+      // rows (hi, lo per token).  Each tile's k-steps are cut into KQ parts
+      // so that every warp has work; partial scores meet in shared memory.
       const int nrows = c1 - c0;
       const int ntile = (nrows + 15) / 16;
       const int bn = lane & 7;
       const uint32_t b_base = (bn < 2 * B ? smem_u32(s.ub + bn * US) + (uint32_t)(((lane >> 3) & 1) * 16) : smem_u32(s.zero));
       const uint32_t b_step = bn < 2 * B ? 32u : 0u;
       const int KS = r / 16;
-      for (int it = 0; it < ntile; ++it) {
+      int KQ = ntile > 0 ? (2 * NW + ntile - 1) / ntile : 1;
+      if (KQ > KS / 4) KQ = KS / 4;
+      if (KQ < 1) KQ = 1;
+      int released = 0;  // P2 tiles this warp has released; a tile is released once the warp is past it
+      for (int un = warp; un < ntile * KQ; un += NW) {
+        const int it = un / KQ, kq = un % KQ;
+        for (; released < it; ++released) release_item();
         const uint32_t myitem = witem + it;
-        if (it % NW == warp) {
-          to |= !mbar_wait(&s.full[myitem % kNQ], (myitem / kNQ) & 1u, ctrl);
-          const int rows = min(16, nrows - 16 * it);
-          const int ar = lane & 15;
-          const uint32_t a_base = smem_u32(s.ring + s.item_off[myitem % kNQ]) + (uint32_t)((ar < rows ? ar : 0) * US) +
-                                  (uint32_t)((lane >> 4) * 16);
-          float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
-          int ks = to ? KS : 0;  // the tile is read only once it has landed
-          for (; ks + 1 < KS; ks += 2) {
-            uint32_t a0, a1, a2, a3, b0, b1, e0, e1, e2, e3, f0, f1;
-            ldsm_x4(a_base + 32u * ks, a0, a1, a2, a3);
-            ldsm_x2(b_base + b_step * ks, b0, b1);
-            ldsm_x4(a_base + 32u * (ks + 1), e0, e1, e2, e3);
-            ldsm_x2(b_base + b_step * (ks + 1), f0, f1);
-            mma_16816(acc0, a0, a1, a2, a3, b0, b1);
-            mma_16816(acc1, e0, e1, e2, e3, f0, f1);
-          }
-          if (ks < KS) {
-            uint32_t a0, a1, a2, a3, b0, b1;
-            ldsm_x4(a_base + 32u * ks, a0, a1, a2, a3);
-            ldsm_x2(b_base + b_step * ks, b0, b1);
-            mma_16816(acc0, a0, a1, a2, a3, b0, b1);
-          }
-          // thread (g, t4): rows g and g+8, columns 2*t4 (hi) and 2*t4+1 (lo) = token t4
-          const int g = lane >> 2, t4 = lane & 3;
-          const float s_g = (acc0[0] + acc1[0]) + (acc0[1] + acc1[1]);
-          const float s_g8 = (acc0[2] + acc1[2]) + (acc0[3] + acc1[3]);
-          const int r0 = 16 * it + g, r8 = r0 + 8;
-          bool on0 = t4 < B && g < rows && (s_g + s.bp[r0]) > Ly.thr;
-          bool on8 = t4 < B && g + 8 < rows && (s_g8 + s.bp[r8 < nrows ? r8 : r0]) > Ly.thr;
-          on0 |= __shfl_xor_sync(0xffffffffu, on0, 1);
-          on0 |= __shfl_xor_sync(0xffffffffu, on0, 2);
-          on8 |= __shfl_xor_sync(0xffffffffu, on8, 1);
-          on8 |= __shfl_xor_sync(0xffffffffu, on8, 2);
-          if (t4 == 0) {
-            if (g < rows) s.act[r0] = on0 ? 1 : 0;
-            if (g + 8 < rows) s.act[r8] = on8 ? 1 : 0;
-          }
+        to |= !mbar_wait(&s.full[myitem % kNQ], (myitem / kNQ) & 1u, ctrl);
+        if (to) continue;  // the tile is read only once it has landed
+        const int rows = min(16, nrows - 16 * it);
+        const int ar = lane & 15;
+        const uint32_t a_base = smem_u32(s.ring + s.item_off[myitem % kNQ]) + (uint32_t)((ar < rows ? ar : 0) * US) +
+                                (uint32_t)((lane >> 4) * 16);
+        float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+        const int ke = (kq + 1) * KS / KQ;
+        int ks = kq * KS / KQ;
+        for (; ks + 1 < ke; ks += 2) {
+          uint32_t a0, a1, a2, a3, b0, b1, e0, e1, e2, e3, f0, f1;
+          ldsm_x4(a_base + 32u * ks, a0, a1, a2, a3);
+          ldsm_x2(b_base + b_step * ks, b0, b1);
+          ldsm_x4(a_base + 32u * (ks + 1), e0, e1, e2, e3);
+          ldsm_x2(b_base + b_step * (ks + 1), f0, f1);
+          mma_16816(acc0, a0, a1, a2, a3, b0, b1);
+          mma_16816(acc1, e0, e1, e2, e3, f0, f1);
         }
-        release_item();
+        if (ks < ke) {
+          uint32_t a0, a1, a2, a3, b0, b1;
+          ldsm_x4(a_base + 32u * ks, a0, a1, a2, a3);
+          ldsm_x2(b_base + b_step * ks, b0, b1);
+          mma_16816(acc0, a0, a1, a2, a3, b0, b1);
+        }
+        // thread (g, t4): rows g and g+8, columns 2*t4 (hi) and 2*t4+1 (lo) = token t4
+        const int g = lane >> 2, t4 = lane & 3;
+        if (t4 < B) {
+          if (g < rows) atomicAdd(&s.sc[(16 * it + g) * B + t4], (acc0[0] + acc1[0]) + (acc0[1] + acc1[1]));
+          if (g + 8 < rows) atomicAdd(&s.sc[(16 * it + g + 8) * B + t4], (acc0[2] + acc1[2]) + (acc0[3] + acc1[3]));
+        }
+      }
+      for (; released < ntile; ++released) release_item();
+      if (named_sync_or(1, T, to)) return;  // every partial score is in
+      for (int x = t; x < nrows; x += T) {
+        bool on = false;
+#pragma unroll
+        for (int b = 0; b < B; ++b) on |= (s.sc[x * B + b] + s.bp[x]) > Ly.thr;
+        s.act[x] = on ? 1 : 0;
       }
       witem += ntile;
     } else {
@@ -812,207 +968,33 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
       }
     }
     if (named_sync_or(1, T, to)) return;
-    // local ascending list of this CTA's active cold rows (consumer warp 0)
+    // local ascending list of this CTA's active cold rows (consumer warp 0):
+    // to the producer through shared memory, and parked in this CTA's own
+    // stretch of idx (compacted after the last layer) with its count
     if (warp == 0) {
       int cnt = 0;
+      int32_t* park = p.idx ? p.idx + (int64_t)l * C + c0 : nullptr;
       for (int x0 = 0; x0 < c1 - c0; x0 += 32) {
         const int x = x0 + lane;
         const bool on = x < c1 - c0 && s.act[x];
         const unsigned m = __ballot_sync(0xffffffffu, on);
-        if (on) p.seg[(int64_t)c * p.seg_cap + cnt + __popc(m & ((1u << lane) - 1u))] = H + c0 + x;
+        if (on) {
+          const int at = cnt + __popc(m & ((1u << lane) - 1u));
+          s.cidx[at] = H + c0 + x;
+          if (park) park[at] = H + c0 + x;
+        }
         cnt += __popc(m);
       }
-      if (lane == 0) p.seg_cnt[c] = cnt;
+      if (lane == 0) {
+        s.misc[0] = cnt;
+        p.lcnt[l * G + c] = cnt;
+      }
       __syncwarp();
-      if (lane == 0) grid_arrive(ctrl);
+      if (lane == 0) mbar_arrive(s.list_bar);
     }
 
-    // ---- sparse FFN: hot share, then cold share, two neurons in flight ----
-#pragma unroll
-    for (int b = 0; b < B; ++b)
-#pragma unroll
-      for (int e = 0; e < EPT; ++e) y[b][e] = 0.f;
-    const int wrp = wrow_bytes(WT, d) + 16;  // byte stride of a neuron item's rows
-    const int nh = j1 - j0;
-    int n = nh;
-    bool have_list = false;
-    uint32_t itoff0 = 0u, itoff1 = 0u;
-    float* nred = s.red + 2 * (kMaxConsumers / 32) * (4 * B);  // neuron scratch: [2][NW][2B]
-    // dots of neuron k -> per-warp partial sums in nred[k & 1]
-    auto prepare = [&](int k) {
-      uint32_t off;
-      to |= !wait_item(off);
-      if (k & 1) itoff1 = off;
-      else itoff0 = off;
-      const uint8_t* it = s.ring + off;
-      float acc[2 * B];
-      float wu[EPT];
-      w_vals<WT, EPT>(it + (gated ? wrp : 0), d, t, T, wu);
-#pragma unroll
-      for (int b = 0; b < B; ++b) {
-        float a = 0.f;
-#pragma unroll
-        for (int e = 0; e < EPT; ++e) a = fmaf(wu[e], h[b][e], a);
-        acc[B + b] = a;
-      }
-      if (gated) {
-        float wg[EPT];
-        w_vals<WT, EPT>(it, d, t, T, wg);
-#pragma unroll
-        for (int b = 0; b < B; ++b) {
-          float a = 0.f;
-#pragma unroll
-          for (int e = 0; e < EPT; ++e) a = fmaf(wg[e], h[b][e], a);
-          acc[b] = a;
-        }
-      } else {
-#pragma unroll
-        for (int b = 0; b < B; ++b) acc[b] = 0.f;
-      }
-#pragma unroll
-      for (int i = 0; i < 2 * B; ++i) acc[i] = warp_sum(acc[i]);
-      float* red = nred + (k & 1) * (kMaxConsumers / 32) * (2 * B);
-      if (lane == 0) {
-#pragma unroll
-        for (int i = 0; i < 2 * B; ++i) red[warp * 2 * B + i] = acc[i];
-      }
-    };
-    // activation and down-row accumulation of neuron k (after its barrier)
-    auto finish = [&](int k) {
-      const float* red = nred + (k & 1) * (kMaxConsumers / 32) * (2 * B);
-      float tot[2 * B];
-#pragma unroll
-      for (int i = 0; i < 2 * B; ++i) {
-        float v = lane < NW ? red[lane * 2 * B + i] : 0.f;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        tot[i] = v;
-      }
-      const float bias = k < nh ? s.b1hot[k] : s.cb1[k - nh];
-      float a[B];
-#pragma unroll
-      for (int b = 0; b < B; ++b)
-        a[b] = gated ? act_eval(kReglu, tot[b] + bias, tot[B + b]) : act_eval(p.act, tot[B + b] + bias, 0.f);
-      float wd[EPT];
-      w_vals<WT, EPT>(s.ring + ((k & 1) ? itoff1 : itoff0) + (gated ? 2 : 1) * wrp, d, t, T, wd);
-      release_item();
-#pragma unroll
-      for (int b = 0; b < B; ++b)
-#pragma unroll
-        for (int e = 0; e < EPT; ++e) y[b][e] = fmaf(a[b], wd[e], y[b][e]);
-    };
-    // the cold list (and its biases) from the producer
-    auto take_list = [&]() -> bool {
-      const bool okw = mbar_wait(s.list_bar, l & 1, ctrl);
-      if (named_sync_or(1, T, !okw)) return false;
-      const int ncold = s.misc[0];
-      for (int x = t; x < ncold; x += T) s.cb1[x] = Ly.b1 ? __ldg(Ly.b1 + s.cidx[x]) : 0.f;
-      n = nh + ncold;
-      have_list = true;
-      return true;
-    };
-    if constexpr (WT == kF16 && PT == kF16) {
-      // Tensor cores for the gate/up dots of p.ng neurons at a time: their
-      // gate and up rows form one 16-row A tile (unused rows repeat neuron 0),
-      // the fp16 token rows the B tile; warps split d and their partial dots
-      // meet in shared memory, one thread per (neuron, token) applies the
-      // activation, then every thread adds the group's down rows into its
-      // columns of the partial output.
-      const int rpn = gated ? 2 : 1;  // tile rows per neuron
-      const int bn = lane & 7;
-      const uint32_t b_base =
-          bn < B ? smem_u32(s.hb + bn * HS) + (uint32_t)(((lane >> 3) & 1) * 16) : smem_u32(s.zero);
-      const uint32_t b_step = bn < B ? 32u : 0u;
-      const int KS = d / 16, ks0 = warp * KS / NW, ks1 = (warp + 1) * KS / NW;
-      float* gact = nred;  // [ng][B] activations of the group
-      int k = 0;
-      for (;;) {
-        if (k == nh && !have_list) {
-          if (!take_list()) return;
-          named_sync(1, T);  // cb1 visible
-        }
-        const int lim = have_list ? n : nh;
-        if (k >= lim) break;
-        const int ng = min(p.ng, lim - k);
-        for (int i = 0; i < ng; ++i) to |= !mbar_wait(&s.full[(witem + i) % kNQ], ((witem + i) / kNQ) & 1u, ctrl);
-        if (!to) {
-          const int tr = lane & 15;
-          const int jj = tr / rpn < ng ? tr / rpn : 0;
-          const int which = gated ? (tr & 1) : 0;  // item row: gate then up (ReGLU), up (otherwise)
-          const uint32_t a_base = smem_u32(s.ring + s.item_off[(witem + jj) % kNQ]) + (uint32_t)(which * wrp) +
-                                  (uint32_t)((lane >> 4) * 16);
-          float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
-          int ks = ks0;
-          for (; ks + 1 < ks1; ks += 2) {
-            uint32_t a0, a1, a2, a3, b0, b1, e0, e1, e2, e3, f0, f1;
-            ldsm_x4(a_base + 32u * ks, a0, a1, a2, a3);
-            ldsm_x2(b_base + b_step * ks, b0, b1);
-            ldsm_x4(a_base + 32u * (ks + 1), e0, e1, e2, e3);
-            ldsm_x2(b_base + b_step * (ks + 1), f0, f1);
-            mma_16816(acc0, a0, a1, a2, a3, b0, b1);
-            mma_16816(acc1, e0, e1, e2, e3, f0, f1);
-          }
-          if (ks < ks1) {
-            uint32_t a0, a1, a2, a3, b0, b1;
-            ldsm_x4(a_base + 32u * ks, a0, a1, a2, a3);
-            ldsm_x2(b_base + b_step * ks, b0, b1);
-            mma_16816(acc0, a0, a1, a2, a3, b0, b1);
-          }
-          // thread (g = lane/4, lane%4 == 0) holds tile rows g and g+8, tokens 0 and 1
-          if ((lane & 3) == 0) {
-            const int g = lane >> 2;
-            float* rp = s.redp + warp * 32;
-            rp[g * 2 + 0] = acc0[0] + acc1[0];
-            rp[g * 2 + 1] = acc0[1] + acc1[1];
-            rp[(g + 8) * 2 + 0] = acc0[2] + acc1[2];
-            rp[(g + 8) * 2 + 1] = acc0[3] + acc1[3];
-          }
-        }
-        if (named_sync_or(1, T, to)) return;
-        if (t < ng * B) {
-          const int jj = t / B, b = t % B;
-          float gd = 0.f, vd = 0.f;
-          for (int w = 0; w < NW; ++w) {
-            gd += s.redp[w * 32 + (jj * rpn) * 2 + b];
-            vd += s.redp[w * 32 + (jj * rpn + rpn - 1) * 2 + b];
-          }
-          const int kk = k + jj;
-          const float bias = kk < nh ? s.b1hot[kk] : s.cb1[kk - nh];
-          gact[jj * B + b] = gated ? act_eval(kReglu, gd + bias, vd) : act_eval(p.act, vd + bias, 0.f);
-        }
-        named_sync(1, T);
-        for (int jj = 0; jj < ng; ++jj) {
-          float wd[EPT];
-          w_vals<WT, EPT>(s.ring + s.item_off[(witem + jj) % kNQ] + rpn * wrp, d, t, T, wd);
-#pragma unroll
-          for (int b = 0; b < B; ++b) {
-            const float a = gact[jj * B + b];
-#pragma unroll
-            for (int e = 0; e < EPT; ++e) y[b][e] = fmaf(a, wd[e], y[b][e]);
-          }
-        }
-        witem += ng;
-        for (int i = 0; i < ng; ++i) release_item();
-        k += ng;
-      }
-    } else {
-      if (nh == 0) {
-        if (!take_list()) return;
-        named_sync(1, T);  // cb1 visible
-      }
-      if (n > 0) prepare(0);
-      for (int k = 0; k < n; ++k) {
-        if (named_sync_or(1, T, to)) return;  // neuron k's partial sums are complete
-        if (k + 1 == nh && !have_list) {
-          if (!take_list()) return;  // cb1 becomes visible at the next neuron's barrier
-        }
-        if (k + 1 < n) prepare(k + 1);
-        finish(k);
-      }
-      if (!have_list) {  // (nh > 0 and the loop ended before the list: cannot happen, kept for safety)
-        if (!take_list()) return;
-      }
-    }
+    // ---- the neuron stream: claimed hot chunks and this CTA's predicted cold rows ----
+    if (!run_stream()) return;
 
     // ---- split-K: add the partial into one of K fp32 accumulator copies ----
     {
@@ -1030,11 +1012,12 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
                                   y[b][k * O::RUN + e + 3]));
         }
     }
+    if (l + 1 < p.L) load_shares(p.layers[l + 1]);  // in flight across barrier Y and the glue
     named_sync(1, T);
     if (t == 0) grid_arrive(ctrl);
     {
       bool okw = true;
-      if (t == 0) okw = grid_wait(ctrl, base, 3 * l + 2, G);
+      if (t == 0) okw = grid_wait(ctrl, base, 2 * l + 1, G);
       if (named_sync_or(1, T, !okw)) return;
     }
 
@@ -1102,8 +1085,61 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
       }
     }
   }
-  // every CTA has passed the last barrier: leave the count base for the next launch
-  if (c == 0 && t == 0) atomicExch(&ctrl->bar_base, base + (unsigned)(3 * p.L * G));
+  // ---- the ascending lists: every CTA moves its parked list of each layer
+  // to its offset (the sum of the lower CTAs' counts); layers in chunks whose
+  // lists fit in the ring, one grid barrier per chunk between reads and writes
+  unsigned nbar = 2u * p.L;
+  if (C > 0 && p.idx) {
+    int* keep = reinterpret_cast<int*>(s.ring);                                // [chunk layers][seg_cap]
+    int* offs = reinterpret_cast<int*>(s.ring) + p.cmp_layers * p.seg_cap;    // [chunk layers][2]: offset, total
+    for (int l0 = 0; l0 < p.L; l0 += p.cmp_layers) {
+      const int l1 = min(p.L, l0 + p.cmp_layers);
+      for (int l = l0 + warp; l < l1; l += NW) {  // one warp per layer: this CTA's offset and the total
+        int below = 0, all = 0;
+        for (int i = lane; i < G; i += 32) {
+          const int v = __ldcg(p.lcnt + l * G + i);
+          all += v;
+          if (i < c) below += v;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          below += __shfl_xor_sync(0xffffffffu, below, o);
+          all += __shfl_xor_sync(0xffffffffu, all, o);
+        }
+        if (lane == 0) {
+          offs[2 * (l - l0)] = below;
+          offs[2 * (l - l0) + 1] = all;
+        }
+      }
+      for (int l = l0; l < l1; ++l) {
+        const int n = __ldcg(p.lcnt + l * G + c);
+        for (int i = t; i < n; i += T) keep[(l - l0) * p.seg_cap + i] = __ldcg(p.idx + (int64_t)l * C + c0 + i);
+      }
+      named_sync(1, T);
+      if (t == 0) grid_arrive(ctrl);
+      {
+        bool okw = true;
+        if (t == 0) okw = grid_wait(ctrl, base, nbar, G);
+        if (named_sync_or(1, T, !okw)) return;
+      }
+      ++nbar;
+      for (int l = l0; l < l1; ++l) {
+        const int n = __ldcg(p.lcnt + l * G + c);
+        const int o = offs[2 * (l - l0)];
+        for (int i = t; i < n; i += T) p.idx[(int64_t)l * C + o + i] = keep[(l - l0) * p.seg_cap + i];
+        if (c == 0 && t == 0) p.counts[l] = offs[2 * (l - l0) + 1];
+      }
+      named_sync(1, T);  // offs and keep are reused by the next chunk
+    }
+  } else if (c == 0) {
+    for (int l = t; l < p.L; l += T) p.counts[l] = 0;
+  }
+  // every CTA has passed the last barrier, so every claim is done: reset the
+  // claim counters and leave the barrier base for the next launch
+  if (c == 0) {
+    for (int l = t; l < p.L; l += T) p.pool[l] = 0;
+    if (t == 0) atomicExch(&ctrl->bar_base, base + nbar * (unsigned)G);
+  }
 }
 
 template <int WT, int PT, int B, int EPT>
@@ -1150,55 +1186,51 @@ bool stack_supported(int wtype, int ptype, int d, int ffn, int n_hot, int rank, 
 size_t stack_smem_layout(StackParams& p, int B, int G) {
   const int C = p.ffn - p.n_hot;
   const int share_cap = (C + G - 1) / G + 1;
-  const int hot_cap = (p.n_hot + G - 1) / G + 1;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
     off += (bytes + 127) & ~(size_t)127;
     return (int)o;
   };
-  // everything but the ring first (at the end of shared memory), then the ring
+  // the ring first, everything else at the end of shared memory
+  const size_t sizes[] = {
+      sizeof(uint64_t) * (2 * kNQ + 1),                                        // bars
+      sizeof(uint32_t) * 4 * kNQ,                                              // item offsets, starts, rows, groups
+      sizeof(float) * (size_t)B * p.rank,                                      // u
+      sizeof(float) * share_cap,                                               // bp
+      sizeof(int) * share_cap,                                                 // cidx
+      (size_t)share_cap,                                                       // act
+      sizeof(float) * share_cap * B,                                           // sc
+      sizeof(float) * 2 * (kMaxConsumers / 32) * 6 * B,                        // red
+      sizeof(float) * (kMaxGroup * (kMaxConsumers / 32) * 2 * B + kMaxGroup * B),  // gred + group activations
+      sizeof(int) * 4,                                                         // misc
+      (size_t)B * (2 * p.d + 16),                                              // hb
+      (size_t)2 * B * (2 * p.rank + 16),                                       // ub
+      16,                                                                      // zero
+      sizeof(float) * (kMaxConsumers / 32) * 32,                               // redp
+  };
   size_t fixed = 0;
-  {
-    size_t o = 0;
-    auto t2 = [&](size_t bytes) { o += (bytes + 127) & ~(size_t)127; };
-    t2(sizeof(uint64_t) * (2 * kNQ + 1));
-    t2(sizeof(uint32_t) * 3 * kNQ);
-    t2(sizeof(float) * (size_t)B * p.rank);
-    t2(sizeof(float) * share_cap);
-    t2(sizeof(float) * hot_cap);
-    t2(sizeof(int) * share_cap);
-    t2(sizeof(float) * share_cap);
-    t2(share_cap);
-    t2(sizeof(float) * 2 * (kMaxConsumers / 32) * 6 * B);
-    t2(sizeof(int) * (G + 1));
-    t2(sizeof(int) * 4);
-    t2((size_t)B * (2 * p.d + 16));
-    t2((size_t)2 * B * (2 * p.rank + 16));
-    t2(16);
-    t2(sizeof(float) * (kMaxConsumers / 32) * 32);
-    fixed = o;
-  }
+  for (size_t b : sizes) fixed += (b + 127) & ~(size_t)127;
   const size_t total = kSmemBytes;
   if (fixed + 32768 > total) return 0;
   const size_t ring = (total - fixed) & ~(size_t)127;
   p.ring_bytes = (int)ring;
+  p.seg_cap = share_cap;
   off = ring;
-  p.off_bars = take(sizeof(uint64_t) * (2 * kNQ + 1));
-  p.off_itemoff = take(sizeof(uint32_t) * 3 * kNQ);
-  p.off_u = take(sizeof(float) * (size_t)B * p.rank);
-  p.off_bp = take(sizeof(float) * share_cap);
-  p.off_b1hot = take(sizeof(float) * hot_cap);
-  p.off_cidx = take(sizeof(int) * share_cap);
-  p.off_cb1 = take(sizeof(float) * share_cap);
-  p.off_act = take(share_cap);
-  p.off_red = take(sizeof(float) * 2 * (kMaxConsumers / 32) * 6 * B);
-  p.off_prefix = take(sizeof(int) * (G + 1));
-  p.off_misc = take(sizeof(int) * 4);
-  p.off_hb = take((size_t)B * (2 * p.d + 16));
-  p.off_ub = take((size_t)2 * B * (2 * p.rank + 16));
-  p.off_zero = take(16);
-  p.off_redp = take(sizeof(float) * (kMaxConsumers / 32) * 32);
+  p.off_bars = take(sizes[0]);
+  p.off_itemoff = take(sizes[1]);
+  p.off_u = take(sizes[2]);
+  p.off_bp = take(sizes[3]);
+  p.off_cidx = take(sizes[4]);
+  p.off_act = take(sizes[5]);
+  p.off_sc = take(sizes[6]);
+  p.off_red = take(sizes[7]);
+  p.off_gred = take(sizes[8]);
+  p.off_misc = take(sizes[9]);
+  p.off_hb = take(sizes[10]);
+  p.off_ub = take(sizes[11]);
+  p.off_zero = take(sizes[12]);
+  p.off_redp = take(sizes[13]);
   return off;
 }
 

@@ -15,7 +15,8 @@ constexpr int kMaxRank = 4096;
 constexpr size_t kSmemBytes = 232448;  // opt-in shared memory per CTA on sm_100
 constexpr int kYCopies = 8;          // fp32 output accumulator copies (spreads the atomics)
 constexpr int kGMaxCtas = 296;       // largest grid (2 x 148)
-constexpr int kShareRegs = 2;        // per-thread registers for the CTA's bias shares
+constexpr int kShareRegs = 2;
+constexpr int kMaxGroup = 16;       // neurons per group at most        // per-thread registers for the CTA's bias shares
 
 // One layer's device pointers (a copy of pi_layer_weights).
 struct StackLayer {
@@ -40,10 +41,12 @@ struct StackParams {
   int T;           // consumer threads (d / stack_ept(d))
   int ring_bytes;  // shared-memory ring size
   int seg_cap;     // per-CTA capacity of the local active lists
-  int ng;          // neurons per tensor-core group (fp16 weights and predictors)
+  int ng;          // neurons per group (<= kMaxGroup; one tensor-core tile for fp16)
   int p1rows;      // P1 rows per tensor-core group (fp16 predictors)
-  int off_bars, off_itemoff, off_u, off_bp, off_b1hot, off_cidx, off_cb1, off_act, off_red, off_prefix, off_misc;
-  int off_hb, off_ub, off_zero, off_redp;
+  int hot_static;  // hot neurons [0, hot_static) are shared out statically; the rest are claimed
+  int cmp_layers;  // layers per chunk of the final list compaction
+  int off_bars, off_itemoff, off_u, off_bp, off_cidx, off_act, off_red, off_gred, off_misc;
+  int off_hb, off_ub, off_zero, off_redp, off_sc;
   const void* h_in;
   void* h_out;
   int32_t* idx;     // [L, C]
@@ -53,8 +56,8 @@ struct StackParams {
   Ctrl* ctrl;
   float* u_g;       // [B, r]
   float* yacc;      // [2, kYCopies, B, d] fp32 output accumulators
-  int* seg;         // [G, seg_cap]
-  int* seg_cnt;     // [G]
+  int* pool;        // [L] claim counters of the hot neurons (zero between launches)
+  int* lcnt;        // [L, G] per-CTA counts of the local active lists
   StackLayer layers[kMaxLayers];
 };
 

@@ -117,16 +117,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Ctrl* 
 // only grows: barrier k (0-based, in launch order) has completed once it
 // reaches base + (k + 1) * nctas, where base is the count the previous launch
 // left (ctrl->bar_base, read once at kernel start).  One thread per CTA
-// arrives after a CTA-wide barrier: one fence, one release add (the pattern of
-// a cooperative-groups grid sync).
+// arrives after a CTA-wide barrier with a release add; the CTA-wide barrier
+// orders the other threads' writes before it.  The waiting thread polls with
+// acquire loads, and a CTA-wide barrier after the wait passes the acquired
+// view on.  No separate fences: each costs a round trip to L2.
 __device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-__device__ __forceinline__ void grid_arrive(Ctrl* ctrl) {
-  __threadfence();
-  red_release_add(&ctrl->bar_count, 1u);
-}
+__device__ __forceinline__ void grid_arrive(Ctrl* ctrl) { red_release_add(&ctrl->bar_count, 1u); }
 
 __device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned* p) {
   unsigned v;
@@ -135,10 +134,10 @@ __device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned* p) {
 }
 
 __device__ __forceinline__ bool grid_done(Ctrl* ctrl, unsigned base, unsigned k, unsigned nctas) {
-  return (int)(ld_relaxed_u32(&ctrl->bar_count) - (base + (k + 1) * nctas)) >= 0;
+  return (int)(ld_acquire_u32(&ctrl->bar_count) - (base + (k + 1) * nctas)) >= 0;
 }
 
-// Polls with relaxed loads; one acquire fence once the count is reached.
+// Polls with acquire loads until the count is reached.
 __device__ __forceinline__ bool grid_wait(Ctrl* ctrl, unsigned base, unsigned k, unsigned nctas) {
   if (!grid_done(ctrl, base, k, nctas)) {
     const uint64_t t0 = global_ns();
@@ -153,7 +152,6 @@ __device__ __forceinline__ bool grid_wait(Ctrl* ctrl, unsigned base, unsigned k,
       }
     }
   }
-  __threadfence();
   return true;
 }
 

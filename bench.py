@@ -173,11 +173,14 @@ def run_ours(args, rank, world, local_rank):
     with ClockSampler(local_rank) as clk:
         with torch.cuda.stream(stream):
             torch.cuda.synchronize()
+            # profiler range = the timed region (ncu --profile-from-start off)
+            torch.cuda.cudart().cudaProfilerStart()
             ev0.record(stream)
             for t in range(args.warmup, n_steps):
                 graphs[t % P].replay()
             ev1.record(stream)
             torch.cuda.synchronize()
+            torch.cuda.cudart().cudaProfilerStop()
     ms = ev0.elapsed_time(ev1)
     clocks = clk.summary()
     if world > 1:

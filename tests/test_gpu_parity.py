@@ -24,6 +24,10 @@ SHAPES = [
     ("reglu-f16-b16", 256, 1000, 0.10, 32, "reglu", "f16", "f16", 16),
     ("reglu-f16-b8", 1024, 2600, 0.10, 128, "reglu", "f16", "f16", 8),
     ("relu2-f32-b4", 96, 700, 0.05, 16, "relu2", "f32", "f32", 4),
+    # tensor-core token-block path: 256-column chunks, d split in parts, no hot rows
+    ("relu2-f16-b12", 1280, 1500, 0.05, 32, "relu2", "f16", "f16", 12),
+    ("reglu-f16-b16-split", 4096, 1200, 0.10, 64, "reglu", "f16", "f16", 16),
+    ("relu-f16-b3-nohot", 512, 900, 0.0, 32, "relu", "f16", "f16", 3),
 ]
 
 
