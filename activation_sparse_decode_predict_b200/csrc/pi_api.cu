@@ -96,6 +96,17 @@ pi_status predict_impl(const pi_ffn_desc* d, int32_t B, const void* h, const voi
   int* tcount = reinterpret_cast<int*>(ws + L.tile_count);
   const int C = d->ffn - d->n_hot;
   const int sms = sm_count();
+  if (pi::batch_pred_supported(d->ptype, d->d, d->rank, B) && d->rank <= d->ffn) {
+    // token blocks of 3..16 with fp16 predictors: tensor-core P1 and P2 (scratch:
+    // P1 dots in the partials, u rows in the activations, scores in the pre-activations)
+    PI_CUDA(pi::launch_batch_predict(h, B, d->d, d->rank, C, d->n_hot, P1, P2, bp, thr,
+                                     reinterpret_cast<float*>(ws + L.partial), ws + L.act,
+                                     reinterpret_cast<float*>(ws + L.pre), tmask, tcount,
+                                     reinterpret_cast<pi::Ctrl*>(ws), sms, st),
+            "tensor-core predictor launch");
+    PI_CUDA(pi::launch_compact(tmask, tcount, C, d->n_hot, idx, count, st), "compaction launch");
+    return PI_OK;
+  }
   PI_CUDA(pi::launch_pred_u(d->ptype, P1, h, B, d->d, d->rank, u, sms, st), "predictor GEMV1 launch");
   PI_CUDA(pi::launch_pred_score(d->ptype, P2, bp, u, B, d->rank, C, thr, tmask, tcount, st), "predictor score launch");
   PI_CUDA(pi::launch_compact(tmask, tcount, C, d->n_hot, idx, count, st), "compaction launch");
@@ -337,6 +348,7 @@ pi_status pi_residual_rmsnorm(int32_t batch, int32_t d, pi_dtype htype, const vo
   if (d <= 0 || d % 8) return fail(PI_ERR_INVALID_ARG, "%s", "d must be a positive multiple of 8");
   if (htype != PI_F32 && htype != PI_F16) return fail(PI_ERR_INVALID_ARG, "%s", "htype must be PI_F32 or PI_F16");
   if (!(eps >= 0.f)) return fail(PI_ERR_INVALID_ARG, "%s", "eps must be >= 0");
+  if (d > 16384) return fail(PI_ERR_UNSUPPORTED, "%s", "d above 16384 is not supported");
   PI_TRY(check_ptr(h, 16, "h"));
   PI_TRY(check_ptr(y, 16, "y"));
   PI_TRY(check_ptr(h_out, 16, "h_out"));

@@ -12,9 +12,11 @@
 // to keep up with the copies; the layout rules of the bulk copies and of
 // ldmatrix decide the speed.
 //
-// k_bup    CTA = (range of list positions, part of d).  The gate and up rows
-//          of the range, columns of the part, against the tokens' columns of
-//          the part: pre-activation dots -> pre[part][pos][2][B] fp32.
+// k_rowdot CTA = (range of row positions, part of K).  16-row tiles of
+//          weight rows (the FFN list's gate/up rows, or P1 / P2 rows) against
+//          the token columns of the part: dots -> out[part][pos][slot][tok].
+//          It also runs the predictor of a token block: P1 rows against the
+//          tokens, then P2 rows against u split into fp16 hi + lo rows.
 // k_bdown  CTA = (chunk of d, range of list positions).  Activations from
 //          pre (summed over the parts) and b1, split into fp16 hi + lo so the
 //          product keeps ~22 bits of each activation; fp32 partial output of
@@ -70,15 +72,24 @@ struct UpLayout {
 __host__ __device__ inline UpLayout up_layout(int B8, int d, int S) {
   UpLayout L;
   L.PC = d / S;
-  L.KC = (L.PC % 1024 == 0) ? 1024 : (L.PC % 512 == 0) ? 512 : (L.PC % 256 == 0) ? 256 : 128;
   L.HS = L.PC * 2 + 16;   // token row stride (bytes): +16 keeps ldmatrix rows on distinct banks
-  L.RS = L.KC * 2 + 16;   // weight row stride in a ring slot
-  L.ISZ = 16 * L.RS;      // one slot: 16 rows x KC columns
   L.off_h = 2 * 8 * kBMaxSlots;
   L.off_h = (L.off_h + 127) & ~127;
   L.off_red = L.off_h + ((B8 * L.HS + 127) & ~127);
-  L.off_ring = L.off_red + 2 * kBW * 16 * 16 * 4;
+  L.off_ring = L.off_red + 2 * kBW * 16 * B8 * 4;
   const int room = kBSmem - L.off_ring;
+  // columns per streamed chunk: the largest PC / m (a multiple of 16) whose
+  // 16-row slot leaves room for three slots -- long row copies stream faster
+  L.KC = 16;
+  for (int m = 1; m <= L.PC / 16; ++m) {
+    if (L.PC % m || (L.PC / m) % 16) continue;
+    if (3 * 16 * ((L.PC / m) * 2 + 16) <= room) {
+      L.KC = L.PC / m;
+      break;
+    }
+  }
+  L.RS = L.KC * 2 + 16;   // weight row stride in a ring slot
+  L.ISZ = 16 * L.RS;      // one slot: 16 rows x KC columns
   L.nslot = room / L.ISZ;
   if (L.nslot > kBMaxSlots) L.nslot = kBMaxSlots;
   L.bytes = L.off_ring + L.nslot * L.ISZ;
@@ -90,6 +101,7 @@ struct DownLayout {
 };
 
 constexpr int kARow = 48;  // bytes per token row of an activation tile (16 fp16 + pad: conflict-free ldmatrix)
+constexpr int kActTiles = 16;  // activation tiles computed together (their loads are in flight at once)
 
 __host__ __device__ inline DownLayout down_layout(int d) {
   DownLayout L;
@@ -98,7 +110,7 @@ __host__ __device__ inline DownLayout down_layout(int d) {
   L.ISZ = 16 * L.RS;
   L.off_a = 2 * 8 * kBMaxSlots;
   L.off_a = (L.off_a + 127) & ~127;
-  L.off_ring = L.off_a + 2 * 2 * 16 * kARow;  // [buffer][hi, lo][16 token rows]
+  L.off_ring = L.off_a + kActTiles * 2 * 16 * kARow;  // [tile of the chunk][hi, lo][16 token rows]
   L.off_ring = (L.off_ring + 127) & ~127;
   const int room = kBSmem - L.off_ring;
   L.nslot = room / L.ISZ;
@@ -109,21 +121,32 @@ __host__ __device__ inline DownLayout down_layout(int d) {
 
 // ---------------------------------------------------------------------------
 
-struct BUpParams {
-  const __half* h;   // [B, d]
-  const __half* wg;  // [F, d] (ReGLU only)
-  const __half* wu;  // [F, d]
+// Row dots against a block of token rows: out[part][pos][slot][tok] =
+// sum over the part's columns of W[row(pos)] * x[tok].  List mode: positions
+// are the FFN list [0, n_hot) ++ idx (gate and up rows of 8 neurons per
+// 16-row tile when gated, else up rows of 16, slot 0 = gate, 1 = up); plain
+// mode: rows 0..nrows-1 of one matrix, slot 0.
+struct RowDotParams {
+  const __half* x;   // [ntok, K] token rows
+  const __half* w0;  // gate (gated list mode) or the only matrix
+  const __half* w1;  // up (gated list mode)
   const int32_t* idx;
   const int32_t* count;
-  float* pre;  // [S][F][2][B]
+  float* out;  // [S][R][W][ntok]
   Ctrl* ctrl;
-  int B, d, ffn, n_hot, S, gated;
+  int ntok, K, S;
+  int list;    // 1: FFN list mode
+  int gated;   // list mode: gate and up rows
+  int R;       // positions per part in out (ffn in list mode, nrows in plain mode)
+  int nrows;   // plain mode
+  int n_hot, ffn;
+  int W;       // slots per position
 };
 
 template <int NT>
-__global__ void __launch_bounds__(kBT + 32, 1) k_bup(const __grid_constant__ BUpParams p) {
+__global__ void __launch_bounds__(kBT + 32, 1) k_rowdot(const __grid_constant__ RowDotParams p) {
   extern __shared__ __align__(128) uint8_t sm[];
-  const UpLayout Lay = up_layout(NT * 8, p.d, p.S);
+  const UpLayout Lay = up_layout(NT * 8, p.K, p.S);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm);
   uint64_t* empty = full + kBMaxSlots;
   uint8_t* hs = sm + Lay.off_h;
@@ -134,10 +157,11 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_bup(const __grid_constant__ BUp
   const int R = gridDim.x / p.S;
   const int rho = blockIdx.x / p.S, sig = blockIdx.x % p.S;
   const int col0 = sig * Lay.PC;
-  const int C = p.ffn - p.n_hot;
-  const int ntot = p.n_hot + clamp_count(p.count, C, ctrl, blockIdx.x == 0 && threadIdx.x == 0);
+  const int ntot = p.list ? p.n_hot + clamp_count(p.count, p.ffn - p.n_hot, ctrl, blockIdx.x == 0 && threadIdx.x == 0)
+                          : p.nrows;
   const int n0 = bshare(ntot, rho, R), n1 = bshare(ntot, rho + 1, R);
-  const int npt = p.gated ? 8 : 16;  // neurons per 16-row tile
+  const int two = p.list && p.gated;  // two rows (gate, up) per position
+  const int npt = two ? 8 : 16;       // positions per 16-row tile
   const int ntile = (n1 - n0 + npt - 1) / npt;
   const int nch = Lay.PC / Lay.KC;
   const int nitems = ntile * nch;
@@ -164,12 +188,12 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_bup(const __grid_constant__ BUp
       if (lane == 0) mbar_arrive_expect_tx(&full[q], 16u * Lay.KC * 2u);
       __syncwarp();
       if (lane < 16) {
-        int pos = n0 + tile * npt + (p.gated ? lane / 2 : lane);
+        int pos = n0 + tile * npt + (two ? lane / 2 : lane);
         if (pos >= n1) pos = n1 - 1;  // tail rows repeat the last one; their dots are dropped
-        int j = list_row(pos, p.n_hot, p.ffn, p.idx, ctrl);
+        int j = p.list ? list_row(pos, p.n_hot, p.ffn, p.idx, ctrl) : pos;
         if (j < 0) j = 0;
-        const __half* mat = p.gated ? ((lane & 1) ? p.wu : p.wg) : p.wu;
-        bulk_g2s(ring + q * Lay.ISZ + lane * Lay.RS, mat + (int64_t)j * p.d + col0 + ch * Lay.KC, Lay.KC * 2u,
+        const __half* mat = (two && (lane & 1)) ? p.w1 : p.w0;
+        bulk_g2s(ring + q * Lay.ISZ + lane * Lay.RS, mat + (int64_t)j * p.K + col0 + ch * Lay.KC, Lay.KC * 2u,
                  &full[q]);
       }
       __syncwarp();
@@ -182,13 +206,13 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_bup(const __grid_constant__ BUp
 
   // ---------------- consumer warps ----------------
   const int t = threadIdx.x - 32, cw = t >> 5, lane = t & 31;
-  // this part's token columns -> shared memory (rows >= B are zero)
+  // this part's token columns -> shared memory (rows >= ntok are zero)
   {
     const int units = Lay.PC / 8;
     for (int i = t; i < NT * 8 * units; i += kBT) {
       const int b = i / units, u = i % units;
       uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (b < p.B) v = __ldg(reinterpret_cast<const uint4*>(p.h + (int64_t)b * p.d + col0) + u);
+      if (b < p.ntok) v = __ldg(reinterpret_cast<const uint4*>(p.x + (int64_t)b * p.K + col0) + u);
       *reinterpret_cast<uint4*>(hs + b * Lay.HS + 16 * u) = v;
     }
   }
@@ -224,32 +248,83 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_bup(const __grid_constant__ BUp
     if (lane == 0) mbar_arrive(&empty[q]);
     if (ch == nch - 1) {
       // tile complete: partial dots of each warp -> shared memory, summed per (row, token)
-      float* rb = red + (tile & 1) * kBW * 256;
+      constexpr int kRC = NT * 8;  // token columns of the reduction buffer
+      float* rb = red + (tile & 1) * kBW * 16 * kRC;
       {
         const int g = lane >> 2, c2 = 2 * (lane & 3);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          float* w = rb + cw * 256;
-          w[g * 16 + nt * 8 + c2] = acc[nt][0];
-          w[g * 16 + nt * 8 + c2 + 1] = acc[nt][1];
-          w[(g + 8) * 16 + nt * 8 + c2] = acc[nt][2];
-          w[(g + 8) * 16 + nt * 8 + c2 + 1] = acc[nt][3];
+          float* w = rb + cw * 16 * kRC;
+          w[g * kRC + nt * 8 + c2] = acc[nt][0];
+          w[g * kRC + nt * 8 + c2 + 1] = acc[nt][1];
+          w[(g + 8) * kRC + nt * 8 + c2] = acc[nt][2];
+          w[(g + 8) * kRC + nt * 8 + c2 + 1] = acc[nt][3];
           acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
         }
       }
       if (named_sync_or(1, kBT, to)) return;
-      const int row = t >> 4, tok = t & 15;
-      if (tok < p.B) {
-        const int pos = n0 + tile * npt + (p.gated ? row / 2 : row);
+      for (int e = t; e < 16 * p.ntok; e += kBT) {
+        const int row = e / p.ntok, tok = e % p.ntok;
+        const int pos = n0 + tile * npt + (two ? row / 2 : row);
         if (pos < n1) {
           float v = 0.f;
 #pragma unroll
-          for (int w = 0; w < kBW; ++w) v += rb[w * 256 + row * 16 + tok];
-          const int which = p.gated ? (row & 1) : 1;  // 0: gate, 1: up
-          p.pre[(((int64_t)sig * p.ffn + pos) * 2 + which) * p.B + tok] = v;
+          for (int w = 0; w < kBW; ++w) v += rb[(w * 16 + row) * kRC + tok];
+          const int slot = two ? (row & 1) : p.W - 1;
+          p.out[(((int64_t)sig * p.R + pos) * p.W + slot) * p.ntok + tok] = v;
         }
       }
     }
+  }
+}
+
+// u = ReLU(sum over the parts of the P1 dots) -> fp16 rows: row 2b = hi(u_b),
+// row 2b+1 = lo(u_b) = u_b - hi (their sum keeps ~22 bits of u).
+__global__ void __launch_bounds__(256) k_bsplit_u(const float* __restrict__ upre, int S, int r, int B,
+                                                  __half* __restrict__ x2) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= r * B) return;
+  const int k = i / B, b = i % B;
+  float u = 0.f;
+  for (int s = 0; s < S; ++s) u += __ldcg(upre + ((int64_t)s * r + k) * B + b);
+  u = fmaxf(u, 0.f);
+  const __half hi = __float2half_rn(u);
+  const __half lo = __float2half_rn(u - __half2float(hi));
+  x2[(int64_t)(2 * b) * r + k] = hi;
+  x2[(int64_t)(2 * b + 1) * r + k] = lo;
+}
+
+// score = sum over the parts of (hi + lo dots) + bp; active = OR over the
+// tokens of score > thr; one CTA per 256-row tile: 8 ballot words + count
+// (the tile format of the compaction kernel).
+__global__ void __launch_bounds__(256) k_bthresh(const float* __restrict__ sc, int S, int C, int B,
+                                                 const float* __restrict__ bp, float thr,
+                                                 uint32_t* __restrict__ tile_mask, int* __restrict__ tile_count) {
+  __shared__ int cnt[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x * 256 + threadIdx.x;
+  bool on = false;
+  if (c < C) {
+    const float bias = bp ? __ldg(bp + c) : 0.f;
+    for (int b = 0; b < B; ++b) {
+      float v = 0.f;
+      for (int s = 0; s < S; ++s) {
+        const float* q = sc + ((int64_t)s * C + c) * 2 * B + 2 * b;
+        v += __ldcg(q) + __ldcg(q + 1);
+      }
+      on |= (v + bias) > thr;
+    }
+  }
+  const unsigned m = __ballot_sync(0xffffffffu, on);
+  if (lane == 0) {
+    tile_mask[blockIdx.x * 8 + warp] = m;
+    cnt[warp] = __popc(m);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int s = 0;
+    for (int w = 0; w < 8; ++w) s += cnt[w];
+    tile_count[blockIdx.x] = s;
   }
 }
 
@@ -293,7 +368,7 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_bdown(const __grid_constant__ B
     mbar_fence_init();
   }
   // activation tiles start zero (token rows >= B stay zero)
-  for (int i = threadIdx.x; i < 2 * 2 * 16 * kARow / 16; i += blockDim.x)
+  for (int i = threadIdx.x; i < kActTiles * 2 * 16 * kARow / 16; i += blockDim.x)
     reinterpret_cast<uint4*>(abuf)[i] = make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
 
@@ -334,42 +409,62 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_bdown(const __grid_constant__ B
   const uint32_t b_lane = smem_u32(abuf) + (uint32_t)((lane & 7) * kARow + ((lane >> 3) & 1) * 16);
   bool to = false;
   for (int it = 0; it < ntile; ++it) {
-    // activations of the tile's 16 neurons, split into fp16 hi + lo
-    const int buf = it & 1;
-    {
-      const int i = t >> 4, b = t & 15;
-      const int pos = n0 + it * 16 + i;
-      if (b < p.B) {
-        float a = 0.f;
-        if (pos < n1) {
-          const int j = list_row(pos, p.n_hot, p.ffn, p.idx, ctrl);
-          if (j >= 0) {
-            float g = 0.f, v = 0.f;
-            for (int s = 0; s < p.S; ++s) {
-              const float* pr = p.pre + (((int64_t)s * p.ffn + pos) * 2) * p.B + b;
-              g += __ldcg(pr);
-              v += __ldcg(pr + p.B);
+    const int ti = it % kActTiles;
+    if (ti == 0) {
+      // activations of the next kActTiles tiles (16 neurons x B tokens each),
+      // split into fp16 hi + lo; every thread's loads go out before any is used
+      named_sync(1, kBT);  // the previous chunk's tiles have been read
+      const int nent = min(kActTiles, ntile - it) * 16 * p.B;
+      for (int e0 = t; e0 < nent; e0 += 4 * kBT) {
+        float g[4], v[4], bias[4];
+        int tv[4], iv[4], bv[4];
+        bool on[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int e = e0 + k * kBT;
+          tv[k] = e / (16 * p.B);
+          iv[k] = (e / p.B) % 16;
+          bv[k] = e % p.B;
+          const int pos = n0 + (it + tv[k]) * 16 + iv[k];
+          on[k] = e < nent && pos < n1;
+          g[k] = v[k] = bias[k] = 0.f;
+          if (on[k]) {
+            const int j = list_row(pos, p.n_hot, p.ffn, p.idx, ctrl);
+            on[k] = j >= 0;
+            if (j >= 0) {
+              for (int sp = 0; sp < p.S; ++sp) {
+                const float* pr = p.pre + (((int64_t)sp * p.ffn + pos) * 2) * p.B + bv[k];
+                g[k] += __ldcg(pr);
+                v[k] += __ldcg(pr + p.B);
+              }
+              bias[k] = p.b1 ? __ldg(p.b1 + j) : 0.f;
             }
-            const float bias = p.b1 ? __ldg(p.b1 + j) : 0.f;
-            a = gated ? act_eval(kReglu, g + bias, v) : act_eval(p.act, v + bias, 0.f);
           }
         }
-        const __half hi = __float2half_rn(a);
-        const __half lo = __float2half_rn(a - __half2float(hi));
-        reinterpret_cast<__half*>(abuf + ((buf * 2 + 0) * 16 + b) * kARow)[i] = hi;
-        reinterpret_cast<__half*>(abuf + ((buf * 2 + 1) * 16 + b) * kARow)[i] = lo;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int e = e0 + k * kBT;
+          if (e < nent) {
+            float a = 0.f;
+            if (on[k]) a = gated ? act_eval(kReglu, g[k] + bias[k], v[k]) : act_eval(p.act, v[k] + bias[k], 0.f);
+            const __half hi = __float2half_rn(a);
+            const __half lo = __float2half_rn(a - __half2float(hi));
+            reinterpret_cast<__half*>(abuf + ((tv[k] * 2 + 0) * 16 + bv[k]) * kARow)[iv[k]] = hi;
+            reinterpret_cast<__half*>(abuf + ((tv[k] * 2 + 1) * 16 + bv[k]) * kARow)[iv[k]] = lo;
+          }
+        }
       }
+      if (named_sync_or(1, kBT, to)) return;  // the chunk's activation tiles are complete
     }
     const int q = it % nslot;
     to |= !mbar_wait(&full[q], (it / nslot) & 1, ctrl);
-    if (named_sync_or(1, kBT, to)) return;  // activation tile complete
-    {
+    if (!to) {
       const uint32_t a_base = smem_u32(ring + q * Lay.ISZ) + a_lane;
       uint32_t bh[NT][2], bl[NT][2];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        ldsm_x2(b_lane + (uint32_t)(((buf * 2 + 0) * 16 + nt * 8) * kARow), bh[nt][0], bh[nt][1]);
-        ldsm_x2(b_lane + (uint32_t)(((buf * 2 + 1) * 16 + nt * 8) * kARow), bl[nt][0], bl[nt][1]);
+        ldsm_x2(b_lane + (uint32_t)(((ti * 2 + 0) * 16 + nt * 8) * kARow), bh[nt][0], bh[nt][1]);
+        ldsm_x2(b_lane + (uint32_t)(((ti * 2 + 1) * 16 + nt * 8) * kARow), bl[nt][0], bl[nt][1]);
       }
 #pragma unroll
       for (int m = 0; m < kMT; ++m) {
@@ -387,6 +482,7 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_bdown(const __grid_constant__ B
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[q]);
   }
+  if (named_sync_or(1, kBT, to)) return;
   // partial output of this range and chunk (zeros for an empty range)
   {
     const int g = lane >> 2, c2 = 2 * (lane & 3);
@@ -411,12 +507,35 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_bdown(const __grid_constant__ B
   }
 }
 
-int up_parts(int B, int d) {
-  // the tokens' columns of one part stay in shared memory: at most 64 KB
-  const size_t bytes = (size_t)((B + 7) / 8 * 8) * d * 2;
+// parts of K such that the token columns of one part (ntok rows rounded up
+// to the n-tile) stay within 64 KB of shared memory
+int row_parts(int ntok, int K) {
+  const size_t bytes = (size_t)((ntok + 7) / 8 * 8) * K * 2;
   int S = 1;
   while ((size_t)S * 65536 < bytes) S *= 2;
   return S;
+}
+
+template <int NT>
+cudaError_t launch_rowdot_t(const RowDotParams& P, int G, cudaStream_t st) {
+  const UpLayout UL = up_layout(NT * 8, P.K, P.S);
+  cudaError_t e = cudaFuncSetAttribute(k_rowdot<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, UL.bytes);
+  if (e != cudaSuccess) return e;
+  k_rowdot<NT><<<G, kBT + 32, UL.bytes, st>>>(P);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rowdot(const RowDotParams& P, int sms, cudaStream_t st) {
+  const int G = (sms / P.S) * P.S;
+  if (P.ntok <= 8) return launch_rowdot_t<1>(P, G, st);
+  if (P.ntok <= 16) return launch_rowdot_t<2>(P, G, st);
+  return launch_rowdot_t<4>(P, G, st);
+}
+
+bool rowdot_fits(int ntok, int K) {
+  const int S = row_parts(ntok, K);
+  if (S > 4 || K % (128 * S) != 0) return false;
+  return up_layout((ntok + 7) / 8 * 8, K, S).nslot >= 2;
 }
 
 }  // namespace
@@ -425,11 +544,12 @@ bool batch_supported(int wtype, int ptype, int d, int B) {
   if (wtype != kF16 || ptype != kF16) return false;
   if (B < kBatchMin || B > 16) return false;
   if (d % 256 != 0) return false;
-  const int S = up_parts(B, d);
-  if (S > 4 || d % (128 * S) != 0) return false;
-  const UpLayout U = up_layout((B + 7) / 8 * 8, d, S);
-  const DownLayout D = down_layout(d);
-  return U.nslot >= 2 && D.nslot >= 2;
+  return rowdot_fits(B, d) && down_layout(d).nslot >= 2;
+}
+
+bool batch_pred_supported(int ptype, int d, int r, int B) {
+  if (ptype != kF16 || B < kBatchMin || B > 16) return false;
+  return rowdot_fits(B, d) && rowdot_fits(2 * B, r);
 }
 
 size_t batch_pre_bytes(int ffn, int B) { return (size_t)4 * ffn * 2 * B * sizeof(float); }
@@ -441,40 +561,68 @@ int batch_ranges(int d, int sms) {
   return NR < 1 ? 1 : NR;
 }
 
+cudaError_t launch_batch_predict(const void* h, int B, int d, int r, int C, int n_hot, const void* P1,
+                                 const void* P2, const float* bp, float thr, float* upre, void* x2, float* sc,
+                                 uint32_t* tile_mask, int* tile_count, Ctrl* ctrl, int sms, cudaStream_t st) {
+  RowDotParams U{};
+  U.x = static_cast<const __half*>(h);
+  U.w0 = static_cast<const __half*>(P1);
+  U.out = upre;
+  U.ctrl = ctrl;
+  U.ntok = B;
+  U.K = d;
+  U.S = row_parts(B, d);
+  U.R = r;
+  U.nrows = r;
+  U.W = 1;
+  cudaError_t e = launch_rowdot(U, sms, st);
+  if (e != cudaSuccess) return e;
+  k_bsplit_u<<<(r * B + 255) / 256, 256, 0, st>>>(upre, U.S, r, B, static_cast<__half*>(x2));
+  e = cudaGetLastError();
+  if (e != cudaSuccess || C == 0) return e;
+  RowDotParams S{};
+  S.x = static_cast<const __half*>(x2);
+  S.w0 = static_cast<const __half*>(P2);
+  S.out = sc;
+  S.ctrl = ctrl;
+  S.ntok = 2 * B;
+  S.K = r;
+  S.S = row_parts(2 * B, r);
+  S.R = C;
+  S.nrows = C;
+  S.W = 1;
+  e = launch_rowdot(S, sms, st);
+  if (e != cudaSuccess) return e;
+  k_bthresh<<<(C + 255) / 256, 256, 0, st>>>(sc, S.S, C, B, bp, thr, tile_mask, tile_count);
+  (void)n_hot;
+  return cudaGetLastError();
+}
+
 cudaError_t launch_batch_ffn(int act, const void* h, int B, int d, int ffn, int n_hot, const int32_t* idx,
                              const int32_t* count, const void* wg, const void* wu, const void* wd, const float* b1,
                              float* pre, float* partial, int NR, Ctrl* ctrl, int sms, cudaStream_t st) {
-  const int S = up_parts(B, d);
-  const int NT = B > 8 ? 2 : 1;
-  BUpParams U;
-  U.h = static_cast<const __half*>(h);
-  U.wg = static_cast<const __half*>(wg);
-  U.wu = static_cast<const __half*>(wu);
+  const int gated = act == kReglu;
+  RowDotParams U{};
+  U.x = static_cast<const __half*>(h);
+  U.w0 = static_cast<const __half*>(gated ? wg : wu);
+  U.w1 = static_cast<const __half*>(wu);
   U.idx = idx;
   U.count = count;
-  U.pre = pre;
+  U.out = pre;
   U.ctrl = ctrl;
-  U.B = B;
-  U.d = d;
-  U.ffn = ffn;
+  U.ntok = B;
+  U.K = d;
+  U.S = row_parts(B, d);
+  U.list = 1;
+  U.gated = gated;
+  U.R = ffn;
   U.n_hot = n_hot;
-  U.S = S;
-  U.gated = act == kReglu;
-  const UpLayout UL = up_layout(NT * 8, d, S);
-  const int Gu = (sms / S) * S;
-  cudaError_t e;
-  if (NT == 1) {
-    e = cudaFuncSetAttribute(k_bup<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, UL.bytes);
-    if (e != cudaSuccess) return e;
-    k_bup<1><<<Gu, kBT + 32, UL.bytes, st>>>(U);
-  } else {
-    e = cudaFuncSetAttribute(k_bup<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, UL.bytes);
-    if (e != cudaSuccess) return e;
-    k_bup<2><<<Gu, kBT + 32, UL.bytes, st>>>(U);
-  }
-  e = cudaGetLastError();
+  U.ffn = ffn;
+  U.W = 2;
+  cudaError_t e = launch_rowdot(U, sms, st);
   if (e != cudaSuccess) return e;
 
+  const int NT = B > 8 ? 2 : 1;
   BDownParams D;
   D.pre = pre;
   D.b1 = b1;
@@ -487,7 +635,7 @@ cudaError_t launch_batch_ffn(int act, const void* h, int B, int d, int ffn, int 
   D.d = d;
   D.ffn = ffn;
   D.n_hot = n_hot;
-  D.S = S;
+  D.S = U.S;
   D.act = act;
   D.NR = NR;
   const DownLayout DL = down_layout(d);

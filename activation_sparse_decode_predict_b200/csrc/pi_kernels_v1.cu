@@ -312,19 +312,46 @@ __global__ void __launch_bounds__(256) k_ffn_reduce(const float* __restrict__ pa
 }
 
 // ---------------------------------------------------------------------------
-// Stack glue: x = h + y; h_out = x * rsqrt(mean(x^2) + eps).  One CTA per token.
+// Stack glue: x = h + y; h_out = x * rsqrt(mean(x^2) + eps).  One CTA per
+// token; each thread keeps up to kNormUnits 8-element units of x in registers
+// (16-byte loads and stores), so h and y are read once.
+constexpr int kNormUnits = 2;
+
 template <int HT>
-__global__ void __launch_bounds__(256) k_rmsnorm(const void* __restrict__ h, const float* __restrict__ y, int d,
-                                                 float eps, void* __restrict__ h_out) {
+__global__ void __launch_bounds__(1024) k_rmsnorm(const void* __restrict__ h, const float* __restrict__ y, int d,
+                                                  float eps, void* __restrict__ h_out) {
   const int b = blockIdx.x;
-  __shared__ float red[8];
+  __shared__ float red[32];
+  const int units = d / 8;
+  float x[kNormUnits][8];
   float ss = 0.f;
-  for (int e = threadIdx.x; e < d; e += blockDim.x) {
-    float hv;
-    if constexpr (HT == kF32) hv = reinterpret_cast<const float*>(h)[(int64_t)b * d + e];
-    else hv = __half2float(reinterpret_cast<const __half*>(h)[(int64_t)b * d + e]);
-    const float x = hv + y[(int64_t)b * d + e];
-    ss = fmaf(x, x, ss);
+#pragma unroll
+  for (int v = 0; v < kNormUnits; ++v) {
+    const int u = threadIdx.x + v * blockDim.x;
+    if (u < units) {
+      const int64_t e0 = (int64_t)b * d + 8 * u;
+      const float4 y0 = __ldg(reinterpret_cast<const float4*>(y + e0));
+      const float4 y1 = __ldg(reinterpret_cast<const float4*>(y + e0) + 1);
+      float hv[8];
+      if constexpr (HT == kF32) {
+        const float4 a = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(h) + e0));
+        const float4 c = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(h) + e0) + 1);
+        hv[0] = a.x; hv[1] = a.y; hv[2] = a.z; hv[3] = a.w; hv[4] = c.x; hv[5] = c.y; hv[6] = c.z; hv[7] = c.w;
+      } else {
+        const uint4 q = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __half*>(h) + e0));
+        float2 f;
+        f = h2f2(q.x); hv[0] = f.x; hv[1] = f.y;
+        f = h2f2(q.y); hv[2] = f.x; hv[3] = f.y;
+        f = h2f2(q.z); hv[4] = f.x; hv[5] = f.y;
+        f = h2f2(q.w); hv[6] = f.x; hv[7] = f.y;
+      }
+      const float yv[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        x[v][e] = hv[e] + yv[e];
+        ss = fmaf(x[v][e], x[v][e], ss);
+      }
+    }
   }
   ss = warp_sum(ss);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
@@ -332,14 +359,25 @@ __global__ void __launch_bounds__(256) k_rmsnorm(const void* __restrict__ h, con
   float tot = 0.f;
   for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += red[w];
   const float inv = rsqrtf(tot / (float)d + eps);
-  __syncthreads();
-  for (int e = threadIdx.x; e < d; e += blockDim.x) {
-    float hv;
-    if constexpr (HT == kF32) hv = reinterpret_cast<const float*>(h)[(int64_t)b * d + e];
-    else hv = __half2float(reinterpret_cast<const __half*>(h)[(int64_t)b * d + e]);
-    const float x = (hv + y[(int64_t)b * d + e]) * inv;
-    if constexpr (HT == kF32) reinterpret_cast<float*>(h_out)[(int64_t)b * d + e] = x;
-    else reinterpret_cast<__half*>(h_out)[(int64_t)b * d + e] = __float2half_rn(x);
+#pragma unroll
+  for (int v = 0; v < kNormUnits; ++v) {
+    const int u = threadIdx.x + v * blockDim.x;
+    if (u < units) {
+      const int64_t e0 = (int64_t)b * d + 8 * u;
+      if constexpr (HT == kF32) {
+        float* o = reinterpret_cast<float*>(h_out) + e0;
+        reinterpret_cast<float4*>(o)[0] = make_float4(x[v][0] * inv, x[v][1] * inv, x[v][2] * inv, x[v][3] * inv);
+        reinterpret_cast<float4*>(o)[1] = make_float4(x[v][4] * inv, x[v][5] * inv, x[v][6] * inv, x[v][7] * inv);
+      } else {
+        uint4 q;
+        __half2 t;
+        t = __floats2half2_rn(x[v][0] * inv, x[v][1] * inv); q.x = *reinterpret_cast<uint32_t*>(&t);
+        t = __floats2half2_rn(x[v][2] * inv, x[v][3] * inv); q.y = *reinterpret_cast<uint32_t*>(&t);
+        t = __floats2half2_rn(x[v][4] * inv, x[v][5] * inv); q.z = *reinterpret_cast<uint32_t*>(&t);
+        t = __floats2half2_rn(x[v][6] * inv, x[v][7] * inv); q.w = *reinterpret_cast<uint32_t*>(&t);
+        *reinterpret_cast<uint4*>(reinterpret_cast<__half*>(h_out) + e0) = q;
+      }
+    }
   }
 }
 
@@ -434,8 +472,13 @@ cudaError_t launch_ffn_reduce(const float* partial, int G, int B, int d, const f
 
 cudaError_t launch_rmsnorm(int htype, const void* h, const float* y, int B, int d, float eps, void* h_out,
                            cudaStream_t st) {
-  if (htype == kF32) k_rmsnorm<kF32><<<B, 256, 0, st>>>(h, y, d, eps, h_out);
-  else k_rmsnorm<kF16><<<B, 256, 0, st>>>(h, y, d, eps, h_out);
+  // one CTA per token, one thread per 8-element unit (at most kNormUnits units per thread)
+  const int units = d / 8;
+  int threads = (units + kNormUnits - 1) / kNormUnits;
+  threads = (threads + 31) / 32 * 32;
+  if (threads > 1024 || d % 8 != 0) return cudaErrorInvalidValue;
+  if (htype == kF32) k_rmsnorm<kF32><<<B, threads, 0, st>>>(h, y, d, eps, h_out);
+  else k_rmsnorm<kF16><<<B, threads, 0, st>>>(h, y, d, eps, h_out);
   return cudaGetLastError();
 }
 

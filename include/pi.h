@@ -194,6 +194,7 @@ PI_API pi_status pi_layer(const pi_ffn_desc *desc, int32_t batch, const void *h,
  * say what joins the layers; this is the plainest reading that keeps the
  * token statistics fixed): x = h + y;  h_out = x / sqrt(mean(x^2) + eps),
  * computed in fp32 and stored in `htype` (F32 or F16).  h_out may alias h.
+ * d <= 16384 (larger: PI_ERR_UNSUPPORTED).
  */
 PI_API pi_status pi_residual_rmsnorm(int32_t batch, int32_t d, pi_dtype htype, const void *h, const float *y, float eps,
                               void *h_out, void *stream);

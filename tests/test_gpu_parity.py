@@ -28,6 +28,9 @@ SHAPES = [
     ("relu2-f16-b12", 1280, 1500, 0.05, 32, "relu2", "f16", "f16", 12),
     ("reglu-f16-b16-split", 4096, 1200, 0.10, 64, "reglu", "f16", "f16", 16),
     ("relu-f16-b3-nohot", 512, 900, 0.0, 32, "relu", "f16", "f16", 3),
+    # tensor-core predictor of a token block (rank % 128 == 0), P2 split in parts
+    ("relu-f16-b16-bigrank", 2048, 1500, 0.10, 2048, "relu", "f16", "f16", 16),
+    ("reglu-f16-b4-pred", 512, 1200, 0.10, 128, "reglu", "f16", "f16", 4),
 ]
 
 
