@@ -38,6 +38,7 @@ constexpr int kBW = 8;          // consumer warps
 constexpr int kBT = kBW * 32;   // consumer threads
 constexpr int kBSmem = 227 * 1024;
 constexpr int kBMaxSlots = 8;
+constexpr int kMapCap = 2048;  // list rows of a CTA's range kept in shared memory
 
 __device__ __forceinline__ int bshare(int n, int c, int G) { return (int)((int64_t)n * c / G); }
 
@@ -53,6 +54,17 @@ __device__ __forceinline__ int list_row(int pos, int n_hot, int ffn, const int32
   return j;
 }
 
+// the rows of list positions n0.. (up to kMapCap of them) -> shared memory,
+// loaded by the whole CTA at once; -1 marks an invalid list entry
+__device__ __forceinline__ void load_rows(int* rmap, int n0, int n1, int n_hot, int ffn, const int32_t* idx,
+                                          Ctrl* ctrl) {
+  for (int i = threadIdx.x; i < n1 - n0 && i < kMapCap; i += blockDim.x) rmap[i] = list_row(n0 + i, n_hot, ffn, idx, ctrl);
+}
+__device__ __forceinline__ int row_at(const int* rmap, int pos, int n0, int n_hot, int ffn, const int32_t* idx,
+                                      Ctrl* ctrl) {
+  return pos - n0 < kMapCap ? rmap[pos - n0] : list_row(pos, n_hot, ffn, idx, ctrl);
+}
+
 __device__ __forceinline__ int clamp_count(const int32_t* count, int C, Ctrl* ctrl, bool report) {
   int cnt = *count;
   if (cnt < 0 || cnt > C) {
@@ -66,15 +78,15 @@ __device__ __forceinline__ int clamp_count(const int32_t* count, int C, Ctrl* ct
 // shared-memory layouts (host and device agree through these functions)
 
 struct UpLayout {
-  int PC, KC, HS, RS, ISZ, off_h, off_red, off_ring, nslot, bytes;
+  int PC, KC, HS, RS, ISZ, off_map, off_h, off_red, off_ring, nslot, bytes;
 };
 
 __host__ __device__ inline UpLayout up_layout(int B8, int d, int S) {
   UpLayout L;
   L.PC = d / S;
   L.HS = L.PC * 2 + 16;   // token row stride (bytes): +16 keeps ldmatrix rows on distinct banks
-  L.off_h = 2 * 8 * kBMaxSlots;
-  L.off_h = (L.off_h + 127) & ~127;
+  L.off_map = (2 * 8 * kBMaxSlots + 127) & ~127;
+  L.off_h = L.off_map + kMapCap * 4;
   L.off_red = L.off_h + ((B8 * L.HS + 127) & ~127);
   L.off_ring = L.off_red + 2 * kBW * 16 * B8 * 4;
   const int room = kBSmem - L.off_ring;
@@ -97,7 +109,7 @@ __host__ __device__ inline UpLayout up_layout(int B8, int d, int S) {
 }
 
 struct DownLayout {
-  int DCOLS, RS, ISZ, off_a, off_ring, nslot, bytes;
+  int DCOLS, RS, ISZ, off_map, off_a, off_ring, nslot, bytes;
 };
 
 constexpr int kARow = 48;  // bytes per token row of an activation tile (16 fp16 + pad: conflict-free ldmatrix)
@@ -108,8 +120,8 @@ __host__ __device__ inline DownLayout down_layout(int d) {
   L.DCOLS = (d % 1024 == 0) ? 1024 : (d % 512 == 0) ? 512 : 256;
   L.RS = L.DCOLS * 2 + 16;
   L.ISZ = 16 * L.RS;
-  L.off_a = 2 * 8 * kBMaxSlots;
-  L.off_a = (L.off_a + 127) & ~127;
+  L.off_map = (2 * 8 * kBMaxSlots + 127) & ~127;
+  L.off_a = L.off_map + kMapCap * 4;
   L.off_ring = L.off_a + kActTiles * 2 * 16 * kARow;  // [tile of the chunk][hi, lo][16 token rows]
   L.off_ring = (L.off_ring + 127) & ~127;
   const int room = kBSmem - L.off_ring;
@@ -149,6 +161,7 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_rowdot(const __grid_constant__ 
   const UpLayout Lay = up_layout(NT * 8, p.K, p.S);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm);
   uint64_t* empty = full + kBMaxSlots;
+  int* rmap = reinterpret_cast<int*>(sm + Lay.off_map);
   uint8_t* hs = sm + Lay.off_h;
   float* red = reinterpret_cast<float*>(sm + Lay.off_red);
   uint8_t* ring = sm + Lay.off_ring;
@@ -174,6 +187,7 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_rowdot(const __grid_constant__ 
     }
     mbar_fence_init();
   }
+  if (p.list) load_rows(rmap, n0, n1, p.n_hot, p.ffn, p.idx, ctrl);
   __syncthreads();
 
   if (threadIdx.x < 32) {
@@ -190,7 +204,7 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_rowdot(const __grid_constant__ 
       if (lane < 16) {
         int pos = n0 + tile * npt + (two ? lane / 2 : lane);
         if (pos >= n1) pos = n1 - 1;  // tail rows repeat the last one; their dots are dropped
-        int j = p.list ? list_row(pos, p.n_hot, p.ffn, p.idx, ctrl) : pos;
+        int j = p.list ? row_at(rmap, pos, n0, p.n_hot, p.ffn, p.idx, ctrl) : pos;
         if (j < 0) j = 0;
         const __half* mat = (two && (lane & 1)) ? p.w1 : p.w0;
         bulk_g2s(ring + q * Lay.ISZ + lane * Lay.RS, mat + (int64_t)j * p.K + col0 + ch * Lay.KC, Lay.KC * 2u,
@@ -347,6 +361,7 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_bdown(const __grid_constant__ B
   const DownLayout Lay = down_layout(p.d);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm);
   uint64_t* empty = full + kBMaxSlots;
+  int* rmap = reinterpret_cast<int*>(sm + Lay.off_map);
   uint8_t* abuf = sm + Lay.off_a;
   uint8_t* ring = sm + Lay.off_ring;
   Ctrl* ctrl = p.ctrl;
@@ -370,6 +385,7 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_bdown(const __grid_constant__ B
   // activation tiles start zero (token rows >= B stay zero)
   for (int i = threadIdx.x; i < kActTiles * 2 * 16 * kARow / 16; i += blockDim.x)
     reinterpret_cast<uint4*>(abuf)[i] = make_uint4(0u, 0u, 0u, 0u);
+  load_rows(rmap, n0, n1, p.n_hot, p.ffn, p.idx, ctrl);
   __syncthreads();
 
   if (threadIdx.x < 32) {
@@ -384,7 +400,7 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_bdown(const __grid_constant__ B
       if (lane < 16) {
         int pos = n0 + it * 16 + lane;
         if (pos >= n1) pos = n1 - 1;  // tail rows repeat the last one; their activations are zero
-        int j = list_row(pos, p.n_hot, p.ffn, p.idx, ctrl);
+        int j = row_at(rmap, pos, n0, p.n_hot, p.ffn, p.idx, ctrl);
         if (j < 0) j = 0;
         bulk_g2s(ring + q * Lay.ISZ + lane * Lay.RS, p.wd + (int64_t)j * p.d + cbase, Lay.DCOLS * 2u, &full[q]);
       }
@@ -429,7 +445,7 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_bdown(const __grid_constant__ B
           on[k] = e < nent && pos < n1;
           g[k] = v[k] = bias[k] = 0.f;
           if (on[k]) {
-            const int j = list_row(pos, p.n_hot, p.ffn, p.idx, ctrl);
+            const int j = row_at(rmap, pos, n0, p.n_hot, p.ffn, p.idx, ctrl);
             on[k] = j >= 0;
             if (j >= 0) {
               for (int sp = 0; sp < p.S; ++sp) {

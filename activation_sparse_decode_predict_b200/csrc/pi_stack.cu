@@ -160,6 +160,7 @@ struct Smem {
   uint64_t* full;
   uint64_t* empty;
   uint64_t* list_bar;
+  uint64_t* u_bar;   // consumers -> barrier warp: this layer's u rows are written
   uint32_t* item_off;
   uint32_t* istart;  // producer-private: start of the items in flight
   int* item_j;       // neuron row of a neuron item; -1 for an end marker
@@ -184,6 +185,7 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const StackParams& p) {
   s.full = reinterpret_cast<uint64_t*>(base + p.off_bars);
   s.empty = s.full + kNQ;
   s.list_bar = s.empty + kNQ;
+  s.u_bar = s.list_bar + 1;
   s.item_off = reinterpret_cast<uint32_t*>(base + p.off_itemoff);
   s.istart = s.item_off + kNQ;
   s.item_j = reinterpret_cast<int*>(s.item_off + 2 * kNQ);
@@ -396,7 +398,8 @@ struct Producer {
 // ----------------------------------------------------------------------------
 
 template <int WT, int PT, int B, int EPT>
-__global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_constant__ StackParams p) {
+// 96 registers: with 17 or 18 warps per CTA an SM sub-partition holds 5 warps
+__global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   Smem s = carve(smem_raw, p);
   Ctrl* ctrl = p.ctrl;
@@ -415,6 +418,7 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
       s.istart[q] = 0u;
     }
     mbar_init(s.list_bar, 1);
+    mbar_init(s.u_bar, 1);
     mbar_fence_init();
     s.misc[1] = (int)ld_acquire_u32(&ctrl->bar_base);
   }
@@ -429,6 +433,20 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
   // hot neurons, [HA, H), is claimed in chunks through p.pool[l]
   const int HA = p.hot_static;
   const int a0 = share_lo(HA, c, G), a1 = share_lo(HA, c + 1, G);
+
+  if (threadIdx.x >= 32 + T) {
+    // ======================= barrier warp =======================
+    // Arrives at barrier U for the CTA once the consumers have written u: the
+    // release waits for those writes to reach L2, and the consumers go on with
+    // the static hot neurons meanwhile.
+    if (threadIdx.x == 32 + T) {
+      for (int l = 0; l < p.L; ++l) {
+        if (!mbar_wait(s.u_bar, l & 1, ctrl)) break;
+        grid_arrive(ctrl);
+      }
+    }
+    return;
+  }
 
   if (threadIdx.x < 32) {
     // ======================= producer warp =======================
@@ -466,22 +484,30 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
         }
         // the neuron stream: one claimed hot chunk (covers the wait for the
         // local list), the predicted cold rows, more claimed chunks, the end marker
+        // claim sizes shrink with what is left (guided self-scheduling): few
+        // round trips early, fine balance at the end; one claim is in flight
+        // while the previous one is issued
         const int PN = H - HA;
         int* pool = p.pool + l;
-        int nxt = PN > 0 ? atomicAdd(pool, p.ng) : 0;
+        const int cmin = max(1, p.ng / 2), cmax = 4 * p.ng;
+        auto csize = [&](int seen) { return max(cmin, min(cmax, (PN - seen) / (2 * G))); };
+        int nsz = csize(0);
+        int nxt = PN > 0 ? atomicAdd(pool, nsz) : PN;
         if (ok && nxt < PN) {
-          const int cur = nxt;
-          nxt = atomicAdd(pool, p.ng);
-          ok = pr.issue_range(Ly, HA + cur, min(p.ng, PN - cur), WT, gated);
+          const int cur = nxt, csz = nsz;
+          nsz = csize(cur + csz);
+          nxt = atomicAdd(pool, nsz);
+          ok = pr.issue_range(Ly, HA + cur, min(csz, PN - cur), WT, gated);
         }
         if (ok) ok = mbar_wait(s.list_bar, l & 1, ctrl);
         const int nloc = s.misc[0];
         for (int q = 0; q < nloc && ok; ++q)
           ok = pr.issue_neuron(Ly, s.cidx[q], WT, gated, (q % p.ng == 0) ? min(p.ng, nloc - q) : 0);
         while (ok && nxt < PN) {
-          const int cur = nxt;
-          nxt = atomicAdd(pool, p.ng);
-          ok = pr.issue_range(Ly, HA + cur, min(p.ng, PN - cur), WT, gated);
+          const int cur = nxt, csz = nsz;
+          nsz = csize(cur + csz);
+          nxt = atomicAdd(pool, nsz);
+          ok = pr.issue_range(Ly, HA + cur, min(csz, PN - cur), WT, gated);
         }
         if (ok) ok = pr.issue_marker();
       }
@@ -778,7 +804,7 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, 1) k_stack(const __grid_co
     };
 
     named_sync(1, T);
-    if (t == 0) grid_arrive(ctrl);
+    if (t == 0) mbar_arrive(s.u_bar);  // the barrier warp arrives at barrier U
     // the static hot neurons need no predictor: they fill the wait for barrier U
     if (!run_stream()) return;
     {
@@ -1153,7 +1179,7 @@ cudaError_t launch_t(const StackParams& p, int G, size_t smem, cudaStream_t st) 
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(G);
-  cfg.blockDim = dim3(p.T + 32);
+  cfg.blockDim = dim3(p.T + 64);  // producer warp, consumer warps, barrier warp
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -1194,7 +1220,7 @@ size_t stack_smem_layout(StackParams& p, int B, int G) {
   };
   // the ring first, everything else at the end of shared memory
   const size_t sizes[] = {
-      sizeof(uint64_t) * (2 * kNQ + 1),                                        // bars
+      sizeof(uint64_t) * (2 * kNQ + 2),                                        // bars
       sizeof(uint32_t) * 4 * kNQ,                                              // item offsets, starts, rows, groups
       sizeof(float) * (size_t)B * p.rank,                                      // u
       sizeof(float) * share_cap,                                               // bp
