@@ -96,11 +96,11 @@ pi_status predict_impl(const pi_ffn_desc* d, int32_t B, const void* h, const voi
   int* tcount = reinterpret_cast<int*>(ws + L.tile_count);
   const int C = d->ffn - d->n_hot;
   const int sms = sm_count();
-  if (pi::batch_pred_supported(d->ptype, d->d, d->rank, B) && d->rank <= d->ffn) {
+  if (pi::batch_pred_supported(d->ptype, d->d, d->rank, B)) {
     // token blocks of 3..16 with fp16 predictors: tensor-core P1 and P2 (scratch:
-    // P1 dots in the partials, u rows in the activations, scores in the pre-activations)
+    // P1 dots in the partials, scores in the pre-activations)
     PI_CUDA(pi::launch_batch_predict(h, B, d->d, d->rank, C, d->n_hot, P1, P2, bp, thr,
-                                     reinterpret_cast<float*>(ws + L.partial), ws + L.act,
+                                     reinterpret_cast<float*>(ws + L.partial),
                                      reinterpret_cast<float*>(ws + L.pre), tmask, tcount,
                                      reinterpret_cast<pi::Ctrl*>(ws), sms, st),
             "tensor-core predictor launch");
@@ -205,14 +205,16 @@ pi_status fused_params(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, pi:
   // rows fill one 16-row tile
   const int rpn = desc->act == PI_ACT_REGLU ? 2 : 1;
   {
-    const int cap = (int)(half / neuron);
+    // a consumer holds one group while it waits for the first item of the next
+    // one, and a wrap of the ring can waste up to one item: ng + 2 items fit
+    const int cap = pi::kNgFull ? (int)((size_t)P.ring_bytes / neuron) - 2 : (int)(half / neuron);
     const int lim = (desc->wtype == PI_F16 && desc->ptype == PI_F16) ? 16 / rpn : 4;
     P.ng = cap < lim ? cap : lim;
     if (P.ng < 1) P.ng = 1;
   }
   // about one group of hot neurons per CTA is shared out statically (it fills
   // the wait for barrier U); the rest is claimed, which balances the CTAs
-  P.hot_static = desc->n_hot < G * P.ng ? desc->n_hot : G * P.ng;
+  P.hot_static = desc->n_hot < G * P.ng * pi::kHotStaticGroups ? desc->n_hot : G * P.ng * pi::kHotStaticGroups;
   const int C = desc->ffn - desc->n_hot;
   // every consumer thread holds at most kShareRegs entries of the CTA's P2 bias share
   if ((C + G - 1) / G > pi::kShareRegs * P.T) return PI_ERR_UNSUPPORTED;

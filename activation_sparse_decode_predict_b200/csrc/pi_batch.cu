@@ -153,6 +153,10 @@ struct RowDotParams {
   int nrows;   // plain mode
   int n_hot, ffn;
   int W;       // slots per position
+  // token rows made on the fly (P2 of a token block): x row 2b = hi(u_b),
+  // row 2b+1 = lo(u_b), u = ReLU(sum over upre_parts of upre [part][K][ntok/2])
+  const float* upre;
+  int upre_parts;
 };
 
 template <int NT>
@@ -172,9 +176,11 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_rowdot(const __grid_constant__ 
   const int col0 = sig * Lay.PC;
   const int ntot = p.list ? p.n_hot + clamp_count(p.count, p.ffn - p.n_hot, ctrl, blockIdx.x == 0 && threadIdx.x == 0)
                           : p.nrows;
-  const int n0 = bshare(ntot, rho, R), n1 = bshare(ntot, rho + 1, R);
   const int two = p.list && p.gated;  // two rows (gate, up) per position
   const int npt = two ? 8 : 16;       // positions per 16-row tile
+  // whole tiles per range: only the last tile of the list is partial
+  const int tall = (ntot + npt - 1) / npt;
+  const int n0 = min(ntot, npt * bshare(tall, rho, R)), n1 = min(ntot, npt * bshare(tall, rho + 1, R));
   const int ntile = (n1 - n0 + npt - 1) / npt;
   const int nch = Lay.PC / Lay.KC;
   const int nitems = ntile * nch;
@@ -221,7 +227,49 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_rowdot(const __grid_constant__ 
   // ---------------- consumer warps ----------------
   const int t = threadIdx.x - 32, cw = t >> 5, lane = t & 31;
   // this part's token columns -> shared memory (rows >= ntok are zero)
-  {
+  if (p.upre) {
+    // rows made from u: every upre value of the part is loaded once, with
+    // 16-byte loads that are all in flight together
+    const int nb = p.ntok / 2;
+    const int nvec = Lay.PC * nb / 4;  // float4s of one part of upre
+    for (int i0 = t; i0 < nvec; i0 += 4 * kBT) {
+      float4 a[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) a[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int sp = 0; sp < p.upre_parts; ++sp) {
+        const float4* src = reinterpret_cast<const float4*>(p.upre + ((int64_t)sp * p.K + col0) * nb);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int i = i0 + k * kBT;
+          if (i < nvec) {
+            const float4 v = __ldcg(src + i);
+            a[k].x += v.x; a[k].y += v.y; a[k].z += v.z; a[k].w += v.w;
+          }
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int i = i0 + k * kBT;
+        if (i < nvec) {
+          const float f[4] = {a[k].x, a[k].y, a[k].z, a[k].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int el = 4 * i + e, col = el / nb, tb = el % nb;
+            const float u = fmaxf(f[e], 0.f);
+            const __half hi = __float2half_rn(u);
+            const __half lo = __float2half_rn(u - __half2float(hi));
+            reinterpret_cast<__half*>(hs + (2 * tb) * Lay.HS)[col] = hi;
+            reinterpret_cast<__half*>(hs + (2 * tb + 1) * Lay.HS)[col] = lo;
+          }
+        }
+      }
+    }
+    const int units = Lay.PC / 8;
+    for (int i = t; i < (NT * 8 - p.ntok) * units; i += kBT) {
+      const int b = p.ntok + i / units, u = i % units;
+      *reinterpret_cast<uint4*>(hs + b * Lay.HS + 16 * u) = make_uint4(0u, 0u, 0u, 0u);
+    }
+  } else {
     const int units = Lay.PC / 8;
     for (int i = t; i < NT * 8 * units; i += kBT) {
       const int b = i / units, u = i % units;
@@ -292,22 +340,6 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_rowdot(const __grid_constant__ 
   }
 }
 
-// u = ReLU(sum over the parts of the P1 dots) -> fp16 rows: row 2b = hi(u_b),
-// row 2b+1 = lo(u_b) = u_b - hi (their sum keeps ~22 bits of u).
-__global__ void __launch_bounds__(256) k_bsplit_u(const float* __restrict__ upre, int S, int r, int B,
-                                                  __half* __restrict__ x2) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= r * B) return;
-  const int k = i / B, b = i % B;
-  float u = 0.f;
-  for (int s = 0; s < S; ++s) u += __ldcg(upre + ((int64_t)s * r + k) * B + b);
-  u = fmaxf(u, 0.f);
-  const __half hi = __float2half_rn(u);
-  const __half lo = __float2half_rn(u - __half2float(hi));
-  x2[(int64_t)(2 * b) * r + k] = hi;
-  x2[(int64_t)(2 * b + 1) * r + k] = lo;
-}
-
 // score = sum over the parts of (hi + lo dots) + bp; active = OR over the
 // tokens of score > thr; one CTA per 256-row tile: 8 ballot words + count
 // (the tile format of the compaction kernel).
@@ -319,15 +351,24 @@ __global__ void __launch_bounds__(256) k_bthresh(const float* __restrict__ sc, i
   const int c = blockIdx.x * 256 + threadIdx.x;
   bool on = false;
   if (c < C) {
+    // the row's (hi, lo) dot pairs of each part are contiguous: one 8-byte
+    // load per token, all in flight together
     const float bias = bp ? __ldg(bp + c) : 0.f;
-    for (int b = 0; b < B; ++b) {
-      float v = 0.f;
-      for (int s = 0; s < S; ++s) {
-        const float* q = sc + ((int64_t)s * C + c) * 2 * B + 2 * b;
-        v += __ldcg(q) + __ldcg(q + 1);
-      }
-      on |= (v + bias) > thr;
+    float v[16];
+#pragma unroll
+    for (int b = 0; b < 16; ++b) v[b] = 0.f;
+    for (int s = 0; s < S; ++s) {
+      const float2* q = reinterpret_cast<const float2*>(sc + ((int64_t)s * C + c) * 2 * B);
+      float2 x[16];
+#pragma unroll
+      for (int b = 0; b < 16; ++b)
+        if (b < B) x[b] = __ldcg(q + b);
+#pragma unroll
+      for (int b = 0; b < 16; ++b)
+        if (b < B) v[b] += x[b].x + x[b].y;
     }
+#pragma unroll
+    for (int b = 0; b < 16; ++b) on |= b < B && (v[b] + bias) > thr;
   }
   const unsigned m = __ballot_sync(0xffffffffu, on);
   if (lane == 0) {
@@ -371,7 +412,8 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_bdown(const __grid_constant__ B
   const int cbase = chi * Lay.DCOLS;
   const int C = p.ffn - p.n_hot;
   const int ntot = p.n_hot + clamp_count(p.count, C, ctrl, false);
-  const int n0 = bshare(ntot, rho, p.NR), n1 = bshare(ntot, rho + 1, p.NR);
+  const int tall = (ntot + 15) / 16;  // whole 16-neuron tiles per range
+  const int n0 = min(ntot, 16 * bshare(tall, rho, p.NR)), n1 = min(ntot, 16 * bshare(tall, rho + 1, p.NR));
   const int ntile = (n1 - n0 + 15) / 16;
   const int nslot = Lay.nslot;
 
@@ -578,7 +620,7 @@ int batch_ranges(int d, int sms) {
 }
 
 cudaError_t launch_batch_predict(const void* h, int B, int d, int r, int C, int n_hot, const void* P1,
-                                 const void* P2, const float* bp, float thr, float* upre, void* x2, float* sc,
+                                 const void* P2, const float* bp, float thr, float* upre, float* sc,
                                  uint32_t* tile_mask, int* tile_count, Ctrl* ctrl, int sms, cudaStream_t st) {
   RowDotParams U{};
   U.x = static_cast<const __half*>(h);
@@ -592,12 +634,10 @@ cudaError_t launch_batch_predict(const void* h, int B, int d, int r, int C, int 
   U.nrows = r;
   U.W = 1;
   cudaError_t e = launch_rowdot(U, sms, st);
-  if (e != cudaSuccess) return e;
-  k_bsplit_u<<<(r * B + 255) / 256, 256, 0, st>>>(upre, U.S, r, B, static_cast<__half*>(x2));
-  e = cudaGetLastError();
   if (e != cudaSuccess || C == 0) return e;
   RowDotParams S{};
-  S.x = static_cast<const __half*>(x2);
+  S.upre = upre;  // u = ReLU(sum of the P1 parts), split into hi + lo rows while staging
+  S.upre_parts = U.S;
   S.w0 = static_cast<const __half*>(P2);
   S.out = sc;
   S.ctrl = ctrl;

@@ -19,10 +19,10 @@ bool batch_pred_supported(int ptype, int d, int r, int B);
 size_t batch_pre_bytes(int ffn, int B);
 // neuron ranges of the down kernel (= split-K partial slots it writes)
 int batch_ranges(int d, int sms);
-// u = ReLU(P1 h) (dots -> upre [parts][r][B], split -> x2 [2B][r] fp16 hi/lo),
-// scores P2 x2 -> sc [parts][C][2B], threshold -> the compaction's tile masks
+// u = ReLU(P1 h) (dots -> upre [parts][r][B]), scores of P2 against u split
+// into fp16 hi + lo rows -> sc [parts][C][2B], threshold -> the compaction's tile masks
 cudaError_t launch_batch_predict(const void* h, int B, int d, int r, int C, int n_hot, const void* P1,
-                                 const void* P2, const float* bp, float thr, float* upre, void* x2, float* sc,
+                                 const void* P2, const float* bp, float thr, float* upre, float* sc,
                                  uint32_t* tile_mask, int* tile_count, Ctrl* ctrl, int sms, cudaStream_t st);
 // gate/up dots -> pre, then activations + down -> partial[ranges][B][d]
 cudaError_t launch_batch_ffn(int act, const void* h, int B, int d, int ffn, int n_hot, const int32_t* idx,

@@ -15,7 +15,10 @@
 namespace pi {
 
 constexpr int kGMax = 296;  // split-K partial slots (2 x 148 SMs)
-constexpr int kYAccCopies = 8;  // copies of the persistent kernel's fp32 output accumulator
+#ifndef PI_YCOPIES
+#define PI_YCOPIES 1
+#endif
+constexpr int kYAccCopies = PI_YCOPIES;  // copies of the persistent kernel's fp32 output accumulator
 constexpr int kLayersMax = 128;  // layers of one decode-stack call
 constexpr size_t kCtrlBytes = 768;  // the control block at the start of a workspace
 

@@ -433,6 +433,7 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
   // hot neurons, [HA, H), is claimed in chunks through p.pool[l]
   const int HA = p.hot_static;
   const int a0 = share_lo(HA, c, G), a1 = share_lo(HA, c + 1, G);
+  const int am = kHotB ? a0 + (a1 - a0) / 2 : a1;  // [a0, am) before barrier U, [am, a1) after P2
 
   if (threadIdx.x >= 32 + T) {
     // ======================= barrier warp =======================
@@ -462,7 +463,7 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
           for (int k = k0; k < k1 && ok; ++k)
             ok = pr.issue_rows(reinterpret_cast<const uint8_t*>(Ly.P1) + (int64_t)k * d * 2, 0, 1, d * 2, d * 2,
                                16u * (uint32_t)((k - k0) & 7));
-          if (ok) ok = pr.issue_range(Ly, a0, a1 - a0, WT, gated);
+          if (ok) ok = pr.issue_range(Ly, a0, am - a0, WT, gated);
           if (ok) ok = pr.issue_marker();
           for (int cc = c0; cc < c1 && ok; cc += 16)
             ok = pr.issue_rows(reinterpret_cast<const uint8_t*>(Ly.P2) + (int64_t)cc * r * 2, (int64_t)r * 2,
@@ -473,7 +474,7 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
             const uint32_t by = d * ep;
             ok = pr.issue(1, &src, &by);
           }
-          if (ok) ok = pr.issue_range(Ly, a0, a1 - a0, WT, gated);
+          if (ok) ok = pr.issue_range(Ly, a0, am - a0, WT, gated);
           if (ok) ok = pr.issue_marker();
           for (int cc = c0; cc < c1 && ok; cc += NW) {
             const int rows = min(NW, c1 - cc);
@@ -493,7 +494,9 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
         auto csize = [&](int seen) { return max(cmin, min(cmax, (PN - seen) / (2 * G))); };
         int nsz = csize(0);
         int nxt = PN > 0 ? atomicAdd(pool, nsz) : PN;
-        if (ok && nxt < PN) {
+        if (kHotB) {
+          if (ok) ok = pr.issue_range(Ly, am, a1 - am, WT, gated);
+        } else if (ok && nxt < PN) {
           const int cur = nxt, csz = nsz;
           nsz = csize(cur + csz);
           nxt = atomicAdd(pool, nsz);
@@ -1192,7 +1195,7 @@ cudaError_t launch_t(const StackParams& p, int G, size_t smem, cudaStream_t st) 
 
 }  // namespace
 
-int stack_ept(int d) { return (d % 256 == 0 && d / 8 <= kMaxConsumers) ? 8 : 16; }
+int stack_ept(int d) { return (kEptMin == 8 && d % 256 == 0 && d / 8 <= kMaxConsumers) ? 8 : 16; }
 
 bool stack_supported(int wtype, int ptype, int d, int ffn, int n_hot, int rank, int B, int L) {
   if (B < 1 || B > 2) return false;

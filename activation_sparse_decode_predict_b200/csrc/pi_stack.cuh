@@ -13,7 +13,26 @@ constexpr int kNQ = 64;              // items in flight per CTA (queue depth)
 constexpr int kMaxConsumers = 512;   // consumer threads per CTA (d <= 8192)
 constexpr int kMaxRank = 4096;
 constexpr size_t kSmemBytes = 232448;  // opt-in shared memory per CTA on sm_100
-constexpr int kYCopies = 8;          // fp32 output accumulator copies (spreads the atomics)
+#ifndef PI_YCOPIES
+#define PI_YCOPIES 1
+#endif
+#ifndef PI_HOT_STATIC_GROUPS
+#define PI_HOT_STATIC_GROUPS 2
+#endif
+#ifndef PI_STACK_EPT_MIN
+#define PI_STACK_EPT_MIN 8
+#endif
+constexpr int kYCopies = PI_YCOPIES;  // fp32 output accumulator copies (spreads the atomics)
+constexpr int kHotStaticGroups = PI_HOT_STATIC_GROUPS;  // static hot neurons per CTA, in groups
+constexpr int kEptMin = PI_STACK_EPT_MIN;  // columns of d per consumer thread (8 or 16)
+#ifndef PI_HOT_B
+#define PI_HOT_B 1
+#endif
+#ifndef PI_NG_FULL
+#define PI_NG_FULL 0
+#endif
+constexpr int kHotB = PI_HOT_B;    // 1: half of the static hot share heads the neuron stream (no early claim)
+constexpr int kNgFull = PI_NG_FULL;  // 1: groups may fill the ring but one item (else half the ring)
 constexpr int kGMaxCtas = 296;       // largest grid (2 x 148)
 constexpr int kShareRegs = 2;
 constexpr int kMaxGroup = 16;       // neurons per group at most        // per-thread registers for the CTA's bias shares

@@ -42,6 +42,11 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 POOL = 64         # distinct token blocks (one captured graph each), cycled over the timed steps
 E2E_STEPS = 200   # steps of the end-to-end (host buffers) measurement
 REF_SECONDS = 150.0  # cap on the timed oracle work of the reference arm
+# DRAM bytes (read + write) per layer of the decode-step kernel, from an ncu
+# capture of 4 layers of the workload (profiles/k_stack_<workload>_b<B>.md);
+# per-layer traffic does not depend on the layer count, so a launch over L
+# layers moves L times this.  Only for captures of the current kernel.
+TRAFFIC_PER_LAYER = {("7b-reglu-fp16", 1): 271.36e6 / 4 + 4.49e6 / 4}
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -254,7 +259,9 @@ def run_ours(args, rank, world, local_rank):
                    "mean_active_cold": round(float(cnt.mean()), 1)},
         "gb_per_s": round(gbs, 1),
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(gbs / peak, 4), "traffic": None,
+                     "frac": round(gbs / peak, 4),
+                     "traffic": (round(TRAFFIC_PER_LAYER[(wl.name, B)] * n_layers)
+                                 if (wl.name, B) in TRAFFIC_PER_LAYER and args.sparsity is None else None),
                      "kernel": "whole decode step (%d launches)" % launches_per_step,
                      "peak_source": peak_kind},
         "e2e": {"value": round(e2e_tok_s, 3), "unit": "tokens/s", "h2d_bytes_per_step": hb, "d2h_bytes_per_step": hb,
