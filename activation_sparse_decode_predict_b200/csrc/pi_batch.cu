@@ -90,12 +90,14 @@ __host__ __device__ inline UpLayout up_layout(int B8, int d, int S) {
   L.off_red = L.off_h + ((B8 * L.HS + 127) & ~127);
   L.off_ring = L.off_red + 2 * kBW * 16 * B8 * 4;
   const int room = kBSmem - L.off_ring;
-  // columns per streamed chunk: the largest PC / m (a multiple of 16) whose
-  // 16-row slot leaves room for three slots -- long row copies stream faster
+  // columns per streamed chunk: the largest PC / m (a multiple of 16, at
+  // most 2048) whose 16-row slot leaves room for two slots -- row pieces of
+  // 4 KB in 64 KB slots stream at full bandwidth, 2 KB pieces in 32 KB slots
+  // at about half of it, even with more slots in flight
   L.KC = 16;
   for (int m = 1; m <= L.PC / 16; ++m) {
-    if (L.PC % m || (L.PC / m) % 16) continue;
-    if (3 * 16 * ((L.PC / m) * 2 + 16) <= room) {
+    if (L.PC % m || (L.PC / m) % 16 || L.PC / m > 2048) continue;
+    if (2 * 16 * ((L.PC / m) * 2 + 16) <= room) {
       L.KC = L.PC / m;
       break;
     }
@@ -109,20 +111,24 @@ __host__ __device__ inline UpLayout up_layout(int B8, int d, int S) {
 }
 
 struct DownLayout {
-  int DCOLS, RS, ISZ, off_map, off_a, off_ring, nslot, bytes;
+  int DCOLS, RS, ISZ, off_pre, off_b1, off_map, off_a, off_ring, nslot, bytes;
 };
 
 constexpr int kARow = 48;  // bytes per token row of an activation tile (16 fp16 + pad: conflict-free ldmatrix)
-constexpr int kActTiles = 16;  // activation tiles computed together (their loads are in flight at once)
 
 __host__ __device__ inline DownLayout down_layout(int d) {
   DownLayout L;
-  L.DCOLS = (d % 1024 == 0) ? 1024 : (d % 512 == 0) ? 512 : 256;
+  // 4 KB row pieces where d allows (they stream at full bandwidth)
+  L.DCOLS = (d % 2048 == 0) ? 2048 : (d % 1024 == 0) ? 1024 : (d % 512 == 0) ? 512 : 256;
   L.RS = L.DCOLS * 2 + 16;
-  L.ISZ = 16 * L.RS;
+  // a slot: the 16 W_downT row pieces, the tile's pre-activation block of
+  // every part ([part][16][2][16] fp32 at most) and the 16-byte b1 blocks
+  L.off_pre = 16 * L.RS;
+  L.off_b1 = L.off_pre + 4 * 16 * 2 * 16 * 4;
+  L.ISZ = L.off_b1 + 16 * 16;
   L.off_map = (2 * 8 * kBMaxSlots + 127) & ~127;
   L.off_a = L.off_map + kMapCap * 4;
-  L.off_ring = L.off_a + kActTiles * 2 * 16 * kARow;  // [tile of the chunk][hi, lo][16 token rows]
+  L.off_ring = L.off_a + 2 * 2 * 16 * kARow;  // [tile parity][hi, lo][16 token rows]
   L.off_ring = (L.off_ring + 127) & ~127;
   const int room = kBSmem - L.off_ring;
   L.nslot = room / L.ISZ;
@@ -394,6 +400,7 @@ struct BDownParams {
   float* partial;     // [NR][B][d]
   Ctrl* ctrl;
   int B, d, ffn, n_hot, S, act, NR;
+  int R;              // positions per part of pre (ffn + 16 spare, so that a 16-position block never runs past it)
 };
 
 template <int NT>
@@ -425,7 +432,7 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_bdown(const __grid_constant__ B
     mbar_fence_init();
   }
   // activation tiles start zero (token rows >= B stay zero)
-  for (int i = threadIdx.x; i < kActTiles * 2 * 16 * kARow / 16; i += blockDim.x)
+  for (int i = threadIdx.x; i < 2 * 2 * 16 * kARow / 16; i += blockDim.x)
     reinterpret_cast<uint4*>(abuf)[i] = make_uint4(0u, 0u, 0u, 0u);
   load_rows(rmap, n0, n1, p.n_hot, p.ffn, p.idx, ctrl);
   __syncthreads();
@@ -437,14 +444,23 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_bdown(const __grid_constant__ B
       bool ok = true;
       if (it >= nslot) ok = mbar_wait(&empty[q], ((it / nslot) - 1) & 1, ctrl);
       if (!__all_sync(0xffffffffu, ok)) return;
-      if (lane == 0) mbar_arrive_expect_tx(&full[q], 16u * Lay.DCOLS * 2u);
+      const uint32_t preb = 16u * 2u * p.B * 4u;  // one part's pre-activation block of the tile
+      if (lane == 0)
+        mbar_arrive_expect_tx(&full[q], 16u * Lay.DCOLS * 2u + p.S * preb + (p.b1 ? 16u * 16u : 0u));
       __syncwarp();
+      uint8_t* slot = ring + q * Lay.ISZ;
       if (lane < 16) {
         int pos = n0 + it * 16 + lane;
         if (pos >= n1) pos = n1 - 1;  // tail rows repeat the last one; their activations are zero
         int j = row_at(rmap, pos, n0, p.n_hot, p.ffn, p.idx, ctrl);
         if (j < 0) j = 0;
-        bulk_g2s(ring + q * Lay.ISZ + lane * Lay.RS, p.wd + (int64_t)j * p.d + cbase, Lay.DCOLS * 2u, &full[q]);
+        bulk_g2s(slot + lane * Lay.RS, p.wd + (int64_t)j * p.d + cbase, Lay.DCOLS * 2u, &full[q]);
+        if (p.b1) bulk_g2s(slot + Lay.off_b1 + 16 * lane, p.b1 + (j & ~3), 16u, &full[q]);
+      } else if (lane < 16 + p.S) {
+        // pre-activations of positions n0 + 16 it .. +15 (pre has 16 spare positions)
+        const int sp = lane - 16;
+        bulk_g2s(slot + Lay.off_pre + sp * preb, p.pre + (((int64_t)sp * p.R + n0 + it * 16) * 2) * p.B, preb,
+                 &full[q]);
       }
       __syncwarp();
     }
@@ -454,7 +470,7 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_bdown(const __grid_constant__ B
   }
 
   const int t = threadIdx.x - 32, cw = t >> 5, lane = t & 31;
-  constexpr int kMT = 8;  // m-tiles (16 columns each) per warp at most
+  constexpr int kMT = 16;  // m-tiles (16 columns each) per warp at most
   const int MT = Lay.DCOLS / (kBW * 16);
   const int wcol = cw * MT * 16;  // this warp's first column within the chunk
   float acc[kMT][NT][4];
@@ -467,62 +483,41 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_bdown(const __grid_constant__ B
   const uint32_t b_lane = smem_u32(abuf) + (uint32_t)((lane & 7) * kARow + ((lane >> 3) & 1) * 16);
   bool to = false;
   for (int it = 0; it < ntile; ++it) {
-    const int ti = it % kActTiles;
-    if (ti == 0) {
-      // activations of the next kActTiles tiles (16 neurons x B tokens each),
-      // split into fp16 hi + lo; every thread's loads go out before any is used
-      named_sync(1, kBT);  // the previous chunk's tiles have been read
-      const int nent = min(kActTiles, ntile - it) * 16 * p.B;
-      for (int e0 = t; e0 < nent; e0 += 4 * kBT) {
-        float g[4], v[4], bias[4];
-        int tv[4], iv[4], bv[4];
-        bool on[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int e = e0 + k * kBT;
-          tv[k] = e / (16 * p.B);
-          iv[k] = (e / p.B) % 16;
-          bv[k] = e % p.B;
-          const int pos = n0 + (it + tv[k]) * 16 + iv[k];
-          on[k] = e < nent && pos < n1;
-          g[k] = v[k] = bias[k] = 0.f;
-          if (on[k]) {
-            const int j = row_at(rmap, pos, n0, p.n_hot, p.ffn, p.idx, ctrl);
-            on[k] = j >= 0;
-            if (j >= 0) {
-              for (int sp = 0; sp < p.S; ++sp) {
-                const float* pr = p.pre + (((int64_t)sp * p.ffn + pos) * 2) * p.B + bv[k];
-                g[k] += __ldcg(pr);
-                v[k] += __ldcg(pr + p.B);
-              }
-              bias[k] = p.b1 ? __ldg(p.b1 + j) : 0.f;
-            }
+    const int q = it % nslot;
+    const int buf = it & 1;
+    const uint8_t* slot = ring + q * Lay.ISZ;
+    to |= !mbar_wait(&full[q], (it / nslot) & 1, ctrl);
+    // activations of the tile's 16 neurons from the slot, split into fp16 hi + lo
+    if (!to && t < 16 * p.B) {
+      const int i = t / p.B, b = t % p.B;
+      const int pos = n0 + it * 16 + i;
+      float a = 0.f;
+      if (pos < n1) {
+        const int j = row_at(rmap, pos, n0, p.n_hot, p.ffn, p.idx, ctrl);
+        if (j >= 0) {
+          float g = 0.f, v = 0.f;
+          for (int sp = 0; sp < p.S; ++sp) {
+            const float* pr = reinterpret_cast<const float*>(slot + Lay.off_pre) + (sp * 16 + i) * 2 * p.B;
+            g += pr[b];
+            v += pr[p.B + b];
           }
-        }
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int e = e0 + k * kBT;
-          if (e < nent) {
-            float a = 0.f;
-            if (on[k]) a = gated ? act_eval(kReglu, g[k] + bias[k], v[k]) : act_eval(p.act, v[k] + bias[k], 0.f);
-            const __half hi = __float2half_rn(a);
-            const __half lo = __float2half_rn(a - __half2float(hi));
-            reinterpret_cast<__half*>(abuf + ((tv[k] * 2 + 0) * 16 + bv[k]) * kARow)[iv[k]] = hi;
-            reinterpret_cast<__half*>(abuf + ((tv[k] * 2 + 1) * 16 + bv[k]) * kARow)[iv[k]] = lo;
-          }
+          const float bias = p.b1 ? reinterpret_cast<const float*>(slot + Lay.off_b1 + 16 * i)[j & 3] : 0.f;
+          a = gated ? act_eval(kReglu, g + bias, v) : act_eval(p.act, v + bias, 0.f);
         }
       }
-      if (named_sync_or(1, kBT, to)) return;  // the chunk's activation tiles are complete
+      const __half hi = __float2half_rn(a);
+      const __half lo = __float2half_rn(a - __half2float(hi));
+      reinterpret_cast<__half*>(abuf + ((buf * 2 + 0) * 16 + b) * kARow)[i] = hi;
+      reinterpret_cast<__half*>(abuf + ((buf * 2 + 1) * 16 + b) * kARow)[i] = lo;
     }
-    const int q = it % nslot;
-    to |= !mbar_wait(&full[q], (it / nslot) & 1, ctrl);
-    if (!to) {
+    if (named_sync_or(1, kBT, to)) return;  // the tile's activations are in shared memory
+    {
       const uint32_t a_base = smem_u32(ring + q * Lay.ISZ) + a_lane;
       uint32_t bh[NT][2], bl[NT][2];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        ldsm_x2(b_lane + (uint32_t)(((ti * 2 + 0) * 16 + nt * 8) * kARow), bh[nt][0], bh[nt][1]);
-        ldsm_x2(b_lane + (uint32_t)(((ti * 2 + 1) * 16 + nt * 8) * kARow), bl[nt][0], bl[nt][1]);
+        ldsm_x2(b_lane + (uint32_t)(((buf * 2 + 0) * 16 + nt * 8) * kARow), bh[nt][0], bh[nt][1]);
+        ldsm_x2(b_lane + (uint32_t)(((buf * 2 + 1) * 16 + nt * 8) * kARow), bl[nt][0], bl[nt][1]);
       }
 #pragma unroll
       for (int m = 0; m < kMT; ++m) {
@@ -610,7 +605,11 @@ bool batch_pred_supported(int ptype, int d, int r, int B) {
   return rowdot_fits(B, d) && rowdot_fits(2 * B, r);
 }
 
-size_t batch_pre_bytes(int ffn, int B) { return (size_t)4 * ffn * 2 * B * sizeof(float); }
+// positions per part of the pre-activation buffer: 16 spare (even, so that
+// every 16-position block of any part starts on a 16-byte boundary)
+int pre_positions(int ffn) { return (ffn + 16 + 1) & ~1; }
+
+size_t batch_pre_bytes(int ffn, int B) { return (size_t)4 * pre_positions(ffn) * 2 * B * sizeof(float); }
 
 int batch_ranges(int d, int sms) {
   const DownLayout D = down_layout(d);
@@ -671,7 +670,7 @@ cudaError_t launch_batch_ffn(int act, const void* h, int B, int d, int ffn, int 
   U.S = row_parts(B, d);
   U.list = 1;
   U.gated = gated;
-  U.R = ffn;
+  U.R = pre_positions(ffn);
   U.n_hot = n_hot;
   U.ffn = ffn;
   U.W = 2;
@@ -694,6 +693,7 @@ cudaError_t launch_batch_ffn(int act, const void* h, int B, int d, int ffn, int 
   D.S = U.S;
   D.act = act;
   D.NR = NR;
+  D.R = U.R;
   const DownLayout DL = down_layout(d);
   const int Gd = NR * (d / DL.DCOLS);
   if (NT == 1) {

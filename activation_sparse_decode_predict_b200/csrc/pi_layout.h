@@ -3,7 +3,7 @@
 //   [ctrl 768 B: status, abort, barrier count and base, claim counters][u: B x rank fp32][tile masks][tile counts][a: B x ffn fp32]
 //   [partials: G_MAX x B x d fp32][y: B x d fp32][h: B x d fp32]
 //   [y accumulators: 2 x 8 x B x d fp32][list counts: 128 x G_MAX]
-//   [pre-activations of the tensor-core token-block path: 4 x ffn x 2 x B fp32,
+//   [pre-activations of the tensor-core token-block path: 4 x (ffn + 16) x 2 x B fp32,
 //    token blocks of 3 or more only]
 //
 // Every region starts on a 256-byte boundary.  The layout depends only on the
@@ -44,7 +44,7 @@ inline WsLayout ws_layout(int d, int ffn, int n_hot, int rank, int B) {
   L.hbuf = off; off += align256((size_t)B * d * 4);
   L.yacc = off; off += align256((size_t)2 * kYAccCopies * B * d * 4);
   L.lcnt = off; off += align256((size_t)kLayersMax * kGMax * 4);
-  L.pre = off; off += B >= 3 ? align256((size_t)4 * ffn * 2 * B * 4) : 0;
+  L.pre = off; off += B >= 3 ? align256((size_t)4 * ((ffn + 17) & ~1) * 2 * B * 4) : 0;
   L.total = off;
   return L;
 }
