@@ -50,6 +50,21 @@ TRAFFIC_PER_LAYER = {("7b-reglu-fp16", 1): 271.36e6 / 4 + 4.49e6 / 4}
 FALLBACK_HBM_GBS = 6650.0
 
 
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The job's time is the slowest rank's device time (all ranks take this
+    collective in the same order)."""
+    if world <= 1:
+        return value
+    t_ = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t_, op=torch.distributed.ReduceOp.MAX)
+    return float(t_.item())
+
+
+def job_tokens_per_s(tokens_per_rank: int, world: int, ms: float) -> float:
+    """Whole-job throughput: every rank's tokens over the max-over-ranks time."""
+    return world * tokens_per_rank / (ms / 1e3)
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -189,10 +204,8 @@ def run_ours(args, rank, world, local_rank):
             torch.cuda.cudart().cudaProfilerStop()
     ms = ev0.elapsed_time(ev1)
     clocks = clk.summary()
+    ms = max_over_ranks(ms, world, dev)
     if world > 1:
-        t_ = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t_, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t_.item())
         torch.distributed.barrier()
     status = pi.device_status(ws)
 
@@ -204,7 +217,7 @@ def run_ours(args, rank, world, local_rank):
     sec = ms / 1e3
     gbs = total_bytes / sec / 1e9
     peak, peak_kind = peak_hbm()
-    tok_s = world * B * args.steps / sec
+    tok_s = job_tokens_per_s(B * args.steps, world, ms)
 
     # end to end through the public API with host buffers: H2D of the step's
     # token block from pinned memory, the stack call, D2H of the result.
@@ -230,11 +243,8 @@ def run_ours(args, rank, world, local_rank):
         e1.record(stream)
         torch.cuda.synchronize()
     e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t_ = torch.tensor([e_ms], device=dev)
-        torch.distributed.all_reduce(t_, op=torch.distributed.ReduceOp.MAX)
-        e_ms = float(t_.item())
-    e2e_tok_s = world * B * e_steps / (e_ms / 1e3)
+    e_ms = max_over_ranks(e_ms, world, dev)
+    e2e_tok_s = job_tokens_per_s(B * e_steps, world, e_ms)
     hb = B * wl.d * h_pool.element_size()
 
     launches_per_step = pi.stack_launches(desc, B, n_layers)

@@ -1,0 +1,70 @@
+"""Host-side logic of the multi-GPU bench path (independent replicas), on CPU.
+
+The decode path does not shard: N GPUs run N replicas, the job's time is the
+slowest rank's device time and the job's throughput counts every rank's
+tokens.  These tests run that logic with world size 2 over gloo.
+"""
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import bench
+        ms = bench.max_over_ranks(1.5 + rank, world, "cpu")  # rank 1 is the slower one
+        tok = bench.job_tokens_per_s(100, world, ms)
+        dist.barrier()
+        out_q.put((rank, ms, tok))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_take_the_slowest_time_and_count_every_token():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(world))
+    for rank, ms, tok in res:
+        assert ms == pytest.approx(2.5)  # max over ranks, on every rank
+        assert tok == pytest.approx(world * 100 / 2.5e-3)
+
+
+def test_single_rank_is_unchanged():
+    import bench
+    assert bench.max_over_ranks(3.25, 1, "cpu") == 3.25
+    assert bench.job_tokens_per_s(64, 1, 2.0) == pytest.approx(32000.0)
+
+
+def test_reference_arm_prints_only_on_rank_zero():
+    """Under torchrun the reference arm runs on rank 0 alone; other ranks exit 0 silently."""
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "0"], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == ""
