@@ -103,3 +103,29 @@ def test_algorithmic_bytes_per_layer():
     assert 68 < mb < 72
     w5 = W.WORKLOADS["70b-reglu-fp16"]
     assert 330 < W.layer_bytes(w5, 1, W.expected_active(w5, 1)) / 1e6 < 345
+
+
+def test_relu_stack_keeps_the_tokens_of_a_block_apart():
+    """b2 removes the common part of the ReLU FFN output, so the stack glue does
+    not pull the tokens of a block together (their active sets stay distinct)."""
+    import torch
+    for act in ("relu", "relu2", "reglu"):
+        wl = W.Workload("apart", 93, 512, 2048, 6, act, "f32", "f32", 0.92, 1.3, 0.08, 64, (8,), 1)
+        h = W.make_tokens(wl, 8, 1).double()
+        for l in range(6):
+            L = W.make_layer(wl, l)
+            z = h @ L["Wu"].double().T
+            if act == "reglu":
+                a = torch.relu(h @ L["Wg"].double().T + L["b1"].double()) * z
+            else:
+                a = torch.relu(z + L["b1"].double())
+                if act == "relu2":
+                    a = a * a
+            y = a @ L["WdT"].double()
+            if L["b2"] is not None:
+                y = y + L["b2"].double()
+            x = h + y
+            h = x / torch.sqrt((x * x).mean(1, keepdim=True) + 1e-6)
+        hn = h / h.norm(dim=1, keepdim=True)
+        cos = (hn @ hn.T)[~torch.eye(8, dtype=torch.bool)]
+        assert cos.abs().mean().item() < 0.3, (act, cos.abs().mean().item())  # uncentred ReLU: > 0.8
