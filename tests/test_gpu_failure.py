@@ -39,6 +39,7 @@ def test_bounded_wait_times_out_and_context_survives(kind):
     assert pi.device_status(ws) == 0
     n = int(cnt.item())
     ref = oracle.masked_ffn(h0.cpu().numpy(), idx[0, :n].cpu().numpy(), None, L["Wu"].cpu().numpy(),
-                            L["WdT"].cpu().numpy(), L["b1"].cpu().numpy(), None, "relu", wl.n_hot, wl.ffn)
+                            L["WdT"].cpu().numpy(), L["b1"].cpu().numpy(),
+                            None if L["b2"] is None else L["b2"].cpu().numpy(), "relu", wl.n_hot, wl.ffn)
     err = np.abs(y[0].cpu().numpy() - ref).max() / np.abs(ref).max()
     assert err <= 2e-3
