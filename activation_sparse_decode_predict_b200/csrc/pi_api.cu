@@ -214,7 +214,11 @@ pi_status fused_params(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, pi:
   }
   // about one group of hot neurons per CTA is shared out statically (it fills
   // the wait for barrier U); the rest is claimed, which balances the CTAs
-  P.hot_static = desc->n_hot < G * P.ng * pi::kHotStaticGroups ? desc->n_hot : G * P.ng * pi::kHotStaticGroups;
+  {
+    const int per_a = pi::kHotA > 0 ? pi::kHotA : P.ng, per_b = pi::kHotB > 0 ? pi::kHotB : P.ng;
+    P.hot_a = desc->n_hot < G * per_a ? desc->n_hot : G * per_a;
+    P.hot_static = desc->n_hot - P.hot_a < G * per_b ? desc->n_hot : P.hot_a + G * per_b;
+  }
   const int C = desc->ffn - desc->n_hot;
   // every consumer thread holds at most kShareRegs entries of the CTA's P2 bias share
   if ((C + G - 1) / G > pi::kShareRegs * P.T) return PI_ERR_UNSUPPORTED;

@@ -161,6 +161,7 @@ struct Smem {
   uint64_t* empty;
   uint64_t* list_bar;
   uint64_t* u_bar;   // consumers -> barrier warp: this layer's u rows are written
+  uint64_t* u_ready; // barrier warp -> consumers: barrier U passed, every CTA's u is staged
   uint32_t* item_off;
   uint32_t* istart;  // producer-private: start of the items in flight
   int* item_j;       // neuron row of a neuron item; -1 for an end marker
@@ -186,6 +187,7 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const StackParams& p) {
   s.empty = s.full + kNQ;
   s.list_bar = s.empty + kNQ;
   s.u_bar = s.list_bar + 1;
+  s.u_ready = s.list_bar + 2;
   s.item_off = reinterpret_cast<uint32_t*>(base + p.off_itemoff);
   s.istart = s.item_off + kNQ;
   s.item_j = reinterpret_cast<int*>(s.item_off + 2 * kNQ);
@@ -419,6 +421,7 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
     }
     mbar_init(s.list_bar, 1);
     mbar_init(s.u_bar, 1);
+    mbar_init(s.u_ready, 1);
     mbar_fence_init();
     s.misc[1] = (int)ld_acquire_u32(&ctrl->bar_base);
   }
@@ -432,19 +435,76 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
   // static hot share (consumed while barrier U completes); the rest of the
   // hot neurons, [HA, H), is claimed in chunks through p.pool[l]
   const int HA = p.hot_static;
-  const int a0 = share_lo(HA, c, G), a1 = share_lo(HA, c + 1, G);
-  const int am = kHotB ? a0 + (a1 - a0) / 2 : a1;  // [a0, am) before barrier U, [am, a1) after P2
+  const int ha0 = share_lo(p.hot_a, c, G), ha1 = share_lo(p.hot_a, c + 1, G);  // before barrier U
+  const int hb0 = p.hot_a + share_lo(HA - p.hot_a, c, G), hb1 = p.hot_a + share_lo(HA - p.hot_a, c + 1, G);
 
   if (threadIdx.x >= 32 + T) {
     // ======================= barrier warp =======================
-    // Arrives at barrier U for the CTA once the consumers have written u: the
-    // release waits for those writes to reach L2, and the consumers go on with
-    // the static hot neurons meanwhile.
-    if (threadIdx.x == 32 + T) {
-      for (int l = 0; l < p.L; ++l) {
-        if (!mbar_wait(s.u_bar, l & 1, ctrl)) break;
-        grid_arrive(ctrl);
+    // Barrier U for the CTA: once the consumers have written their u rows it
+    // arrives (the release waits for those writes to reach L2), waits for the
+    // other CTAs and stages every CTA's u in shared memory, while the
+    // consumers run the first static hot neurons.
+    const int lane = threadIdx.x & 31;
+    const int US = 2 * r + 16;
+    for (int l = 0; l < p.L; ++l) {
+      bool ok = true;
+      if (lane == 0) {
+        ok = mbar_wait(s.u_bar, l & 1, ctrl);
+        if (ok) grid_arrive(ctrl);
+        if (ok) ok = grid_wait(ctrl, base, 2 * l, G);
       }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) return;
+      if constexpr (PT == kF16) {
+        // row 2b = hi(u_b), row 2b+1 = lo(u_b) = u_b - hi: the tensor cores see ~22 bits of u
+        // 16 loads per lane in flight at a time
+        const int n2 = B * r / 2;
+        for (int i0 = lane; i0 < n2; i0 += 32 * 16) {
+          float2 v[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k)
+            if (i0 + 32 * k < n2) v[k] = __ldcg(reinterpret_cast<const float2*>(p.u_g) + i0 + 32 * k);
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const int i = i0 + 32 * k;
+            if (i < n2) {
+              const int b = (2 * i) / r, col = (2 * i) % r;
+              const __half2 hi = __floats2half2_rn(v[k].x, v[k].y);
+              const float2 hf = __half22float2(hi);
+              const __half2 lo = __floats2half2_rn(v[k].x - hf.x, v[k].y - hf.y);
+              *reinterpret_cast<__half2*>(s.ub + (2 * b) * US + 2 * col) = hi;
+              *reinterpret_cast<__half2*>(s.ub + (2 * b + 1) * US + 2 * col) = lo;
+            }
+          }
+        }
+      } else {
+        // split layout: unit m (8 values) stored as two float4 planes so that
+        // lane-strided reads are conflict-free
+        const int nu = r / 8;
+        for (int i0 = lane; i0 < B * nu; i0 += 32 * 4) {
+          float4 lo[4], hi[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int i = i0 + 32 * k;
+            if (i < B * nu) {
+              const float4* src = reinterpret_cast<const float4*>(p.u_g + (int64_t)(i / nu) * r + 8 * (i % nu));
+              lo[k] = __ldcg(src);
+              hi[k] = __ldcg(src + 1);
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int i = i0 + 32 * k;
+            if (i < B * nu) {
+              const int b = i / nu, m = i % nu;
+              float4* dst = reinterpret_cast<float4*>(s.u + (size_t)b * r);
+              dst[m] = lo[k];
+              dst[nu + m] = hi[k];
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s.u_ready);
     }
     return;
   }
@@ -463,7 +523,7 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
           for (int k = k0; k < k1 && ok; ++k)
             ok = pr.issue_rows(reinterpret_cast<const uint8_t*>(Ly.P1) + (int64_t)k * d * 2, 0, 1, d * 2, d * 2,
                                16u * (uint32_t)((k - k0) & 7));
-          if (ok) ok = pr.issue_range(Ly, a0, am - a0, WT, gated);
+          if (ok) ok = pr.issue_range(Ly, ha0, ha1 - ha0, WT, gated);
           if (ok) ok = pr.issue_marker();
           for (int cc = c0; cc < c1 && ok; cc += 16)
             ok = pr.issue_rows(reinterpret_cast<const uint8_t*>(Ly.P2) + (int64_t)cc * r * 2, (int64_t)r * 2,
@@ -474,7 +534,7 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
             const uint32_t by = d * ep;
             ok = pr.issue(1, &src, &by);
           }
-          if (ok) ok = pr.issue_range(Ly, a0, am - a0, WT, gated);
+          if (ok) ok = pr.issue_range(Ly, ha0, ha1 - ha0, WT, gated);
           if (ok) ok = pr.issue_marker();
           for (int cc = c0; cc < c1 && ok; cc += NW) {
             const int rows = min(NW, c1 - cc);
@@ -494,8 +554,8 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
         auto csize = [&](int seen) { return max(cmin, min(cmax, (PN - seen) / (2 * G))); };
         int nsz = csize(0);
         int nxt = PN > 0 ? atomicAdd(pool, nsz) : PN;
-        if (kHotB) {
-          if (ok) ok = pr.issue_range(Ly, am, a1 - am, WT, gated);
+        if (hb1 > hb0) {
+          if (ok) ok = pr.issue_range(Ly, hb0, hb1 - hb0, WT, gated);
         } else if (ok && nxt < PN) {
           const int cur = nxt, csz = nsz;
           nsz = csize(cur + csz);
@@ -810,42 +870,20 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
     if (t == 0) mbar_arrive(s.u_bar);  // the barrier warp arrives at barrier U
     // the static hot neurons need no predictor: they fill the wait for barrier U
     if (!run_stream()) return;
+    if constexpr (PT == kF16) {
+      for (int x = t; x < (c1 - c0) * B; x += T) s.sc[x] = 0.f;  // partial scores accumulate here
+    }
     {
-      bool okw = true;
-      if (t == 0) okw = grid_wait(ctrl, base, 2 * l, G);
+      // barrier U has passed and u is staged (the barrier warp's signal)
+      const bool okw = mbar_wait(s.u_ready, l & 1, ctrl);
       if (named_sync_or(1, T, !okw)) return;
     }
-    // the other accumulator buffer is free now (its last readers passed this barrier)
+    // the other accumulator buffer is free now (its last readers passed barrier U)
     {
       float4* nxt = reinterpret_cast<float4*>(p.yacc) + (size_t)((l + 1) & 1) * ybuf4;
       const int z0 = share_lo(ybuf4, c, G), z1 = share_lo(ybuf4, c + 1, G);
       for (int i = z0 + t; i < z1; i += T) nxt[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    if constexpr (PT == kF16) {
-      for (int x = t; x < (c1 - c0) * B; x += T) s.sc[x] = 0.f;  // partial scores accumulate here
-      // u -> fp16 rows for the tensor cores: row 2b = hi(u_b), row 2b+1 = lo(u_b) = u_b - hi
-      for (int i = t; i < B * r; i += T) {
-        const int b = i / r, k = i % r;
-        const float v = __ldcg(p.u_g + i);
-        const __half hi = __float2half_rn(v);
-        const __half lo = __float2half_rn(v - __half2float(hi));
-        reinterpret_cast<__half*>(s.ub + (2 * b) * US)[k] = hi;
-        reinterpret_cast<__half*>(s.ub + (2 * b + 1) * US)[k] = lo;
-      }
-    } else {
-      // u -> shared memory, split layout: unit m (8 values) stored as two float4
-      // planes so that lane-strided reads are conflict-free.
-      const int nu = r / 8;
-      for (int i = t; i < B * nu; i += T) {
-        const int b = i / nu, m = i % nu;
-        const float4* src = reinterpret_cast<const float4*>(p.u_g + (int64_t)b * r + 8 * m);
-        const float4 lo = __ldcg(src), hi = __ldcg(src + 1);
-        float4* dst = reinterpret_cast<float4*>(s.u + (size_t)b * r);
-        dst[m] = lo;
-        dst[nu + m] = hi;
-      }
-    }
-    named_sync(1, T);
 
     // ---- predictor step 2: scores of this CTA's cold rows ----
     if constexpr (PT == kF16) {
@@ -1223,7 +1261,7 @@ size_t stack_smem_layout(StackParams& p, int B, int G) {
   };
   // the ring first, everything else at the end of shared memory
   const size_t sizes[] = {
-      sizeof(uint64_t) * (2 * kNQ + 2),                                        // bars
+      sizeof(uint64_t) * (2 * kNQ + 3),                                        // bars
       sizeof(uint32_t) * 4 * kNQ,                                              // item offsets, starts, rows, groups
       sizeof(float) * (size_t)B * p.rank,                                      // u
       sizeof(float) * share_cap,                                               // bp

@@ -16,22 +16,23 @@ constexpr size_t kSmemBytes = 232448;  // opt-in shared memory per CTA on sm_100
 #ifndef PI_YCOPIES
 #define PI_YCOPIES 1
 #endif
-#ifndef PI_HOT_STATIC_GROUPS
-#define PI_HOT_STATIC_GROUPS 2
+#ifndef PI_HOT_A
+#define PI_HOT_A 0
+#endif
+#ifndef PI_HOT_B
+#define PI_HOT_B 0
 #endif
 #ifndef PI_STACK_EPT_MIN
 #define PI_STACK_EPT_MIN 8
 #endif
 constexpr int kYCopies = PI_YCOPIES;  // fp32 output accumulator copies (spreads the atomics)
-constexpr int kHotStaticGroups = PI_HOT_STATIC_GROUPS;  // static hot neurons per CTA, in groups
+// static hot neurons per CTA before barrier U (A) and at the head of the
+// neuron stream (B); 0 means one neuron group
+constexpr int kHotA = PI_HOT_A, kHotB = PI_HOT_B;
 constexpr int kEptMin = PI_STACK_EPT_MIN;  // columns of d per consumer thread (8 or 16)
-#ifndef PI_HOT_B
-#define PI_HOT_B 1
-#endif
 #ifndef PI_NG_FULL
 #define PI_NG_FULL 0
 #endif
-constexpr int kHotB = PI_HOT_B;    // 1: half of the static hot share heads the neuron stream (no early claim)
 constexpr int kNgFull = PI_NG_FULL;  // 1: groups may fill the ring but one item (else half the ring)
 constexpr int kGMaxCtas = 296;       // largest grid (2 x 148)
 constexpr int kShareRegs = 2;
@@ -62,7 +63,9 @@ struct StackParams {
   int seg_cap;     // per-CTA capacity of the local active lists
   int ng;          // neurons per group (<= kMaxGroup; one tensor-core tile for fp16)
   int p1rows;      // P1 rows per tensor-core group (fp16 predictors)
-  int hot_static;  // hot neurons [0, hot_static) are shared out statically; the rest are claimed
+  int hot_a;       // hot neurons [0, hot_a) are shared out statically, consumed before barrier U
+  int hot_static;  // [hot_a, hot_static) are shared out statically, at the head of the neuron
+                   // stream; the rest, [hot_static, n_hot), are claimed
   int cmp_layers;  // layers per chunk of the final list compaction
   int off_bars, off_itemoff, off_u, off_bp, off_cidx, off_act, off_red, off_gred, off_misc;
   int off_hb, off_ub, off_zero, off_redp, off_sc;
