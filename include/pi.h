@@ -211,6 +211,12 @@ PI_API pi_status pi_residual_rmsnorm(int32_t batch, int32_t d, pi_dtype htype, c
  * ptype receiving each layer's input h_l (NULL: not kept).  h_out [B, d]
  * ptype must not alias h_in.  All layers share one descriptor;
  * n_layers <= PI_MAX_LAYERS.
+ * Token blocks of 1-2 with fp16/fp16, Q4_0/fp16 or fp32/fp32 weights and
+ * predictors run the whole step as one cooperative launch (one CTA per SM;
+ * every b1 16-byte aligned, else the per-layer kernels run); larger blocks
+ * and other shapes run per-layer kernels.  Either way the outputs are
+ * complete once the stream reaches the end of the call; one workspace
+ * serves one call at a time.
  */
 PI_API pi_status pi_decode_stack(const pi_ffn_desc *desc, int32_t batch, int32_t n_layers,
                                  const pi_layer_weights *layers, const void *h_in, void *h_out, int32_t *idx,
