@@ -249,6 +249,7 @@ pi_status fused_stack(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, cons
   P.yacc = reinterpret_cast<float*>(ws + L.yacc);
   P.pool = reinterpret_cast<pi::Ctrl*>(ws)->pool;
   P.lcnt = reinterpret_cast<int*>(ws + L.lcnt);
+  P.don = reinterpret_cast<int*>(ws + L.don);
   for (int l = 0; l < n_layers; ++l) {
     const pi_layer_weights& w = layers[l];
     pi::StackLayer& s = P.layers[l];
@@ -291,7 +292,9 @@ size_t pi_workspace_bytes(const pi_ffn_desc* desc, int32_t batch) {
 pi_status pi_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   PI_TRY(check_ptr(ws, 256, "ws"));
   if (ws_bytes < sizeof(pi::Ctrl)) return fail(PI_ERR_CAPACITY, "%s", "workspace smaller than its control block");
-  PI_CUDA(cudaMemsetAsync(ws, 0, sizeof(pi::Ctrl), (cudaStream_t)stream), "workspace init");
+  // the whole workspace: the control block and the hand-over slots of the
+  // persistent kernel must start at zero (the kernel leaves them zero)
+  PI_CUDA(cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream), "workspace init");
   return PI_OK;
 }
 

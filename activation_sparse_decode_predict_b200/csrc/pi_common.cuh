@@ -31,8 +31,11 @@ struct Ctrl {
   unsigned bar_base;   // bar_count at the start of the next persistent launch
   unsigned pad2[15];
   int pool[128];       // per-layer claim counters of the persistent kernel (zero between launches)
+  unsigned don_push[128];  // per layer: cold rows handed to other CTAs (reserved slots)
+  unsigned don_take[128];  // per layer: tickets taken on those slots
+  unsigned don_done[128];  // per layer: CTAs that have decided what to hand over
 };
-static_assert(sizeof(Ctrl) == 768, "control block is 768 bytes");
+static_assert(sizeof(Ctrl) == 2304, "control block is 2304 bytes");
 
 __device__ __forceinline__ void set_status(int* status, int code) { atomicCAS(status, 0, code); }
 

@@ -1,8 +1,9 @@
 // pi_layout.h -- byte layout of a libpi workspace (host side).
 //
-//   [ctrl 768 B: status, abort, barrier count and base, claim counters][u: B x rank fp32][tile masks][tile counts][a: B x ffn fp32]
+//   [ctrl 2304 B: status, abort, barrier count and base, claim and hand-over counters]
+//   [u: B x rank fp32][tile masks][tile counts][a: B x ffn fp32]
 //   [partials: G_MAX x B x d fp32][y: B x d fp32][h: B x d fp32]
-//   [y accumulators: 2 x 8 x B x d fp32][list counts: 128 x G_MAX]
+//   [y accumulators][list counts: 128 x G_MAX][handed-over cold rows: 128 x C]
 //   [pre-activations of the tensor-core token-block path: 4 x (ffn + 16) x 2 x B fp32,
 //    token blocks of 3 or more only]
 //
@@ -20,10 +21,10 @@ constexpr int kGMax = 296;  // split-K partial slots (2 x 148 SMs)
 #endif
 constexpr int kYAccCopies = PI_YCOPIES;  // copies of the persistent kernel's fp32 output accumulator
 constexpr int kLayersMax = 128;  // layers of one decode-stack call
-constexpr size_t kCtrlBytes = 768;  // the control block at the start of a workspace
+constexpr size_t kCtrlBytes = 2304;  // the control block at the start of a workspace
 
 struct WsLayout {
-  size_t u, tile_mask, tile_count, act, partial, ybuf, hbuf, yacc, lcnt, pre, total;
+  size_t u, tile_mask, tile_count, act, partial, ybuf, hbuf, yacc, lcnt, don, pre, total;
   int n_tiles, g_max;
 };
 
@@ -44,6 +45,7 @@ inline WsLayout ws_layout(int d, int ffn, int n_hot, int rank, int B) {
   L.hbuf = off; off += align256((size_t)B * d * 4);
   L.yacc = off; off += align256((size_t)2 * kYAccCopies * B * d * 4);
   L.lcnt = off; off += align256((size_t)kLayersMax * kGMax * 4);
+  L.don = off; off += align256((size_t)kLayersMax * (C > 0 ? C : 1) * 4);
   L.pre = off; off += B >= 3 ? align256((size_t)4 * ((ffn + 17) & ~1) * 2 * B * 4) : 0;
   L.total = off;
   return L;

@@ -376,6 +376,38 @@ struct Producer {
     return ok;
   }
 
+  // Ticket tk on layer l's handed-over cold rows: the row, or -1 once every CTA
+  // has decided and the ticket is past the last slot (bounded waits).
+  __device__ int take_donated(int l, unsigned tk, int C, int G) {
+    const uint64_t t0 = global_ns();
+    for (uint32_t it = 0;; ++it) {
+      const unsigned pushed = ld_relaxed_u32(&ctrl->don_push[l]);
+      if (tk < pushed) {
+        const int v = ld_volatile_s32(p.don + (size_t)l * C + tk);
+        if (v != 0) {
+          // a handed-over row is a cold row of this layer; anything else is
+          // reported and dropped (the workspace was not initialised)
+          if (v - 1 < p.n_hot || v - 1 >= p.ffn) {
+            set_status(&ctrl->status, kStIndex);
+            return -1;
+          }
+          return v - 1;
+        }
+      } else if (ld_acquire_u32(&ctrl->don_done[l]) == (unsigned)G) {
+        // every reservation happened before its CTA's release of don_done
+        if (tk >= ld_relaxed_u32(&ctrl->don_push[l])) return -1;
+        continue;
+      }
+      if ((it & 31u) == 0) {
+        if (ld_volatile_s32(&ctrl->abort)) return -2;
+        if (global_ns() - t0 > kTimeoutNs) {
+          raise_abort(ctrl);
+          return -2;
+        }
+      }
+    }
+  }
+
   // End of a neuron stream: an item without bytes (group size 0).
   __device__ bool issue_marker() {
     uint32_t pos;
@@ -513,6 +545,7 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
     // ======================= producer warp =======================
     const int lane = threadIdx.x;
     Producer pr(p, s);
+    float cold_avg = 0.f;  // running mean of this CTA's predicted cold rows per layer
     bool ok = true;
     for (int l = 0; l < p.L && ok; ++l) {
       const StackLayer& Ly = p.layers[l];
@@ -564,13 +597,33 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
         }
         if (ok) ok = mbar_wait(s.list_bar, l & 1, ctrl);
         const int nloc = s.misc[0];
-        for (int q = 0; q < nloc && ok; ++q)
-          ok = pr.issue_neuron(Ly, s.cidx[q], WT, gated, (q % p.ng == 0) ? min(p.ng, nloc - q) : 0);
+        // A CTA with clearly more predicted rows than it has seen on average
+        // hands the excess to the other CTAs (slots reserved with one atomic,
+        // written as row + 1); every CTA takes handed-over rows by ticket once
+        // its hot-neuron claims run out, until a ticket lands past the last
+        // slot after every CTA has decided -- so no slot is left behind.
+        int keep = nloc;
+        if (kDonate && l > 0) keep = min(nloc, (int)ceilf(cold_avg) + 2);
+        cold_avg = (l == 0) ? (float)nloc : 0.75f * cold_avg + 0.25f * (float)nloc;
+        const int give = nloc - keep;
+        if (give > 0) {
+          const unsigned at = atomicAdd(&ctrl->don_push[l], (unsigned)give);
+          for (int q = 0; q < give; ++q) st_volatile_s32(p.don + (size_t)l * C + at + q, s.cidx[keep + q] + 1);
+        }
+        red_release_add(&ctrl->don_done[l], 1u);
+        for (int q = 0; q < keep && ok; ++q)
+          ok = pr.issue_neuron(Ly, s.cidx[q], WT, gated, (q % p.ng == 0) ? min(p.ng, keep - q) : 0);
         while (ok && nxt < PN) {
           const int cur = nxt, csz = nsz;
           nsz = csize(cur + csz);
           nxt = atomicAdd(pool, nsz);
           ok = pr.issue_range(Ly, HA + cur, min(csz, PN - cur), WT, gated);
+        }
+        while (ok && C > 0) {
+          const int j = pr.take_donated(l, atomicAdd(&ctrl->don_take[l], 1u), C, G);
+          if (j == -2) ok = false;
+          if (j < 0) break;
+          ok = pr.issue_neuron(Ly, j, WT, gated, 1);
         }
         if (ok) ok = pr.issue_marker();
       }
@@ -1156,6 +1209,14 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
   // to its offset (the sum of the lower CTAs' counts); layers in chunks whose
   // lists fit in the ring, one grid barrier per chunk between reads and writes
   unsigned nbar = 2u * p.L;
+  if (C > 0) {
+    // every take of every layer is done (barrier Y): clear this CTA's share of
+    // the handed-over slots, so that the next launch finds them zero
+    for (int l = 0; l < p.L; ++l) {
+      const int n = (int)ld_relaxed_u32(&ctrl->don_push[l]);
+      for (int i = share_lo(n, c, G) + t; i < share_lo(n, c + 1, G); i += T) p.don[(size_t)l * C + i] = 0;
+    }
+  }
   if (C > 0 && p.idx) {
     int* keep = reinterpret_cast<int*>(s.ring);                                // [chunk layers][seg_cap]
     int* offs = reinterpret_cast<int*>(s.ring) + p.cmp_layers * p.seg_cap;    // [chunk layers][2]: offset, total
@@ -1204,7 +1265,12 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
   // every CTA has passed the last barrier, so every claim is done: reset the
   // claim counters and leave the barrier base for the next launch
   if (c == 0) {
-    for (int l = t; l < p.L; l += T) p.pool[l] = 0;
+    for (int l = t; l < p.L; l += T) {
+      p.pool[l] = 0;
+      ctrl->don_push[l] = 0;
+      ctrl->don_take[l] = 0;
+      ctrl->don_done[l] = 0;
+    }
     if (t == 0) atomicExch(&ctrl->bar_base, base + nbar * (unsigned)G);
   }
 }

@@ -30,6 +30,10 @@ constexpr int kYCopies = PI_YCOPIES;  // fp32 output accumulator copies (spreads
 // neuron stream (B); 0 means one neuron group
 constexpr int kHotA = PI_HOT_A, kHotB = PI_HOT_B;
 constexpr int kEptMin = PI_STACK_EPT_MIN;  // columns of d per consumer thread (8 or 16)
+#ifndef PI_DONATE
+#define PI_DONATE 1
+#endif
+constexpr int kDonate = PI_DONATE;  // 1: a CTA hands excess predicted rows to the other CTAs
 #ifndef PI_NG_FULL
 #define PI_NG_FULL 0
 #endif
@@ -80,6 +84,7 @@ struct StackParams {
   float* yacc;      // [2, kYCopies, B, d] fp32 output accumulators
   int* pool;        // [L] claim counters of the hot neurons (zero between launches)
   int* lcnt;        // [L, G] per-CTA counts of the local active lists
+  int* don;         // [L, C] cold rows handed to other CTAs (row + 1; zero = not written yet)
   StackLayer layers[kMaxLayers];
 };
 

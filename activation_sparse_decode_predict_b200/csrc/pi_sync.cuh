@@ -91,6 +91,10 @@ __device__ __forceinline__ int ld_volatile_s32(const int* p) {
   return v;
 }
 
+__device__ __forceinline__ void st_volatile_s32(int* p, int v) {
+  asm volatile("st.volatile.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // Record a timeout and tell every CTA to stop.
 __device__ __forceinline__ void raise_abort(Ctrl* ctrl) {
   set_status(&ctrl->status, kStTimeout);

@@ -137,7 +137,8 @@ typedef struct {
  */
 PI_API size_t pi_workspace_bytes(const pi_ffn_desc *desc, int32_t batch);
 
-/* Zero the workspace's control block (status word and counters), on `stream`. */
+/* Zero the workspace (ws_bytes from ws; status word, counters and the slots
+ * the decode-step kernel expects to start at zero), on `stream`. */
 PI_API pi_status pi_workspace_init(void *ws, size_t ws_bytes, void *stream);
 
 /*
