@@ -208,7 +208,7 @@ pi_status fused_params(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, pi:
     // a consumer holds one group while it waits for the first item of the next
     // one, and a wrap of the ring can waste up to one item: ng + 2 items fit
     const int cap = pi::kNgFull ? (int)((size_t)P.ring_bytes / neuron) - 2 : (int)(half / neuron);
-    const int lim = (desc->wtype == PI_F16 && desc->ptype == PI_F16) ? 16 / rpn : 4;
+    const int lim = (desc->wtype == PI_F16 && desc->ptype == PI_F16 && pi::kF16Mma) ? 16 / rpn : 4;
     P.ng = cap < lim ? cap : lim;
     if (P.ng < 1) P.ng = 1;
   }

@@ -41,6 +41,32 @@ namespace pi {
 
 namespace {
 
+// Warp sums of V values per lane with V - 1 + 5 - log2(V) shuffles: every
+// exchange step halves the values a lane keeps.  The sum of value i ends in
+// lanes whose bits 4..(5 - log2 V) spell i, so lane i * (32 / V) holds it.
+template <int V>
+__device__ __forceinline__ float warp_sums(const float (&v)[V], int lane) {
+  static_assert(V == 2 || V == 4, "2 or 4 values");
+  const bool h16 = (lane & 16) != 0;
+  if constexpr (V == 2) {
+    float k = h16 ? v[1] : v[0];
+    k += __shfl_xor_sync(0xffffffffu, h16 ? v[0] : v[1], 16);
+#pragma unroll
+    for (int o = 8; o; o >>= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
+    return k;
+  } else {
+    float k0 = h16 ? v[2] : v[0], k1 = h16 ? v[3] : v[1];
+    k0 += __shfl_xor_sync(0xffffffffu, h16 ? v[0] : v[2], 16);
+    k1 += __shfl_xor_sync(0xffffffffu, h16 ? v[1] : v[3], 16);
+    const bool h8 = (lane & 8) != 0;
+    float k = h8 ? k1 : k0;
+    k += __shfl_xor_sync(0xffffffffu, h8 ? k0 : k1, 8);
+#pragma unroll
+    for (int o = 4; o; o >>= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
+    return k;
+  }
+}
+
 // ----------------------------------------------------------------------------
 // column ownership: consumer thread t of T owns 16 columns of d, as NRUN runs
 // of RUN consecutive columns whose layout follows the weight type.
@@ -805,7 +831,7 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
         }
         for (int i = 0; i < gs; ++i) to |= !mbar_wait(&s.full[(witem + i) % kNQ], ((witem + i) / kNQ) & 1u, ctrl);
         if (!to) {
-          if constexpr (WT == kF16 && PT == kF16) {
+          if constexpr (WT == kF16 && PT == kF16 && kF16Mma) {
             // Tensor cores: the group's gate and up rows form one 16-row A tile
             // (unused rows repeat the first neuron), the fp16 token rows the B
             // tile; warps split d, partial dots meet in shared memory.
@@ -821,6 +847,24 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
                                     (uint32_t)((lane >> 4) * 16);
             float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
             int ks = ks0;
+            if (kMmaX2 && gs * rpn <= 8) {
+              // rows 8-15 of the tile are unused: load rows 0-7 only (lanes 0-7
+              // address k 0-7, lanes 8-15 k 8-15)
+              const int tr8 = lane & 7;
+              const int j8 = tr8 / rpn < gs ? tr8 / rpn : 0;
+              const int w8 = gated ? (tr8 & 1) : 0;
+              const uint32_t a8 = smem_u32(s.ring + s.item_off[(witem + j8) % kNQ]) + (uint32_t)(w8 * wrp) +
+                                  (uint32_t)(((lane >> 3) & 1) * 16);
+              for (; ks + 1 < ks1; ks += 2) {
+                uint32_t a0, a2, b0, b1, e0, e2, f0, f1;
+                ldsm_x2(a8 + 32u * ks, a0, a2);
+                ldsm_x2(b_base + b_step * ks, b0, b1);
+                ldsm_x2(a8 + 32u * (ks + 1), e0, e2);
+                ldsm_x2(b_base + b_step * (ks + 1), f0, f1);
+                mma_16816(acc0, a0, 0u, a2, 0u, b0, b1);
+                mma_16816(acc1, e0, 0u, e2, 0u, f0, f1);
+              }
+            }
             for (; ks + 1 < ks1; ks += 2) {
               uint32_t a0, a1, a2, a3, b0, b1, e0, e1, e2, e3, f0, f1;
               ldsm_x4(a_base + 32u * ks, a0, a1, a2, a3);
@@ -846,7 +890,8 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
               rp[(g + 8) * 2 + 1] = acc0[3] + acc1[3];
             }
           } else {
-            // CUDA cores: each thread's columns, one warp sum per dot
+            // CUDA cores: each thread's columns, the 2B dots of a neuron summed
+            // over the warp together
             for (int jj = 0; jj < gs; ++jj) {
               const uint8_t* it = s.ring + s.item_off[(witem + jj) % kNQ];
               float acc[2 * B];
@@ -873,12 +918,8 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
 #pragma unroll
                 for (int b = 0; b < B; ++b) acc[b] = 0.f;
               }
-#pragma unroll
-              for (int i = 0; i < 2 * B; ++i) acc[i] = warp_sum(acc[i]);
-              if (lane == 0) {
-#pragma unroll
-                for (int i = 0; i < 2 * B; ++i) s.gred[(jj * NW + warp) * 2 * B + i] = acc[i];
-              }
+              const float tot = warp_sums<2 * B>(acc, lane);
+              if ((lane & (16 / B - 1)) == 0) s.gred[(jj * NW + warp) * 2 * B + lane / (16 / B)] = tot;
             }
           }
         }
@@ -886,7 +927,7 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
         if (t < gs * B) {
           const int jj = t / B, b = t % B;
           float gd = 0.f, vd = 0.f;
-          if constexpr (WT == kF16 && PT == kF16) {
+          if constexpr (WT == kF16 && PT == kF16 && kF16Mma) {
             for (int w = 0; w < NW; ++w) {
               gd += s.redp[w * 32 + (jj * rpn) * 2 + b];
               vd += s.redp[w * 32 + (jj * rpn + rpn - 1) * 2 + b];

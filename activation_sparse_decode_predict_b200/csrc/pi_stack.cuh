@@ -34,6 +34,14 @@ constexpr int kEptMin = PI_STACK_EPT_MIN;  // columns of d per consumer thread (
 #define PI_DONATE 1
 #endif
 constexpr int kDonate = PI_DONATE;  // 1: a CTA hands excess predicted rows to the other CTAs
+#ifndef PI_F16_MMA
+#define PI_F16_MMA 0
+#endif
+#ifndef PI_MMA_X2
+#define PI_MMA_X2 0
+#endif
+constexpr bool kF16Mma = PI_F16_MMA != 0;  // fp16 neuron groups: gate/up dots on the tensor cores
+constexpr bool kMmaX2 = PI_MMA_X2 != 0;    // load only tile rows 0-7 when a group fills no more
 #ifndef PI_NG_FULL
 #define PI_NG_FULL 0
 #endif
