@@ -723,7 +723,7 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
 
     // ---- predictor step 1: u = ReLU(P1 h) ----
     bool to = false;
-    if constexpr (PT == kF16) {
+    if constexpr (PT == kF16 && (B > 1 || kP1Mma)) {
       // Tensor cores: the CTA's (<= 16) P1 rows are the A tile, the fp16
       // token rows the B tile; warps split d, partial dots meet in shared memory.
       named_sync(1, T);  // token rows (written by the glue) are complete

@@ -40,6 +40,13 @@ constexpr int kDonate = PI_DONATE;  // 1: a CTA hands excess predicted rows to t
 #ifndef PI_MMA_X2
 #define PI_MMA_X2 0
 #endif
+#ifndef PI_P1_MMA
+#define PI_P1_MMA 0
+#endif
+// fp16 predictors: the P1 dots of a single token run on CUDA cores (one token
+// fills 1 of the 8 columns of the tensor-core operand); 1 puts them on the
+// tensor cores too.  Token blocks of 2 always use the tensor cores.
+constexpr bool kP1Mma = PI_P1_MMA != 0;
 constexpr bool kF16Mma = PI_F16_MMA != 0;  // fp16 neuron groups: gate/up dots on the tensor cores
 constexpr bool kMmaX2 = PI_MMA_X2 != 0;    // load only tile rows 0-7 when a group fills no more
 #ifndef PI_NG_FULL
