@@ -146,6 +146,33 @@ __device__ __forceinline__ void q4_vals(const uint8_t* row, int d, int t, float 
     }
 }
 
+// This thread's Q4_0 codes as f = 1 + q/16 (q placed in the top mantissa
+// bits of 1.0f: exact, no integer-to-float conversion), so q - 8 = 16 f - 24;
+// sc is the block's scale.  A dot over the thread's columns is then
+// sc * (16 * sum(f h) - 24 * sum(h)).
+template <int EPT>
+__device__ __forceinline__ void q4_codes(const uint8_t* row, int d, int t, float (&f)[EPT], float& sc) {
+  constexpr int NB = EPT / 2;         // qs bytes per thread
+  constexpr int PER_BLK = 32 / EPT;   // threads per block
+  uint32_t q[NB / 4];
+  if constexpr (NB == 8) {
+    const uint2 qq = *reinterpret_cast<const uint2*>(row + NB * t);
+    q[0] = qq.x;
+    q[1] = qq.y;
+  } else {
+    q[0] = *reinterpret_cast<const uint32_t*>(row + NB * t);
+  }
+  sc = half_bits_to_float(*reinterpret_cast<const uint16_t*>(row + d / 2 + 2 * (t / PER_BLK)));
+#pragma unroll
+  for (int w = 0; w < NB / 4; ++w)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t b = q[w] >> (8 * k);
+      f[w * 4 + k] = __uint_as_float(0x3f800000u | ((b & 0xfu) << 19));
+      f[NB + w * 4 + k] = __uint_as_float(0x3f800000u | ((b & 0xf0u) << 15));
+    }
+}
+
 template <int WT, int EPT>
 __device__ __forceinline__ void w_vals(const uint8_t* row, int d, int t, int T, float (&v)[EPT]) {
   if constexpr (WT == kQ4_0) q4_vals<EPT>(row, d, t, v);
@@ -720,6 +747,15 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
     for (int b = 0; b < B; ++b)
 #pragma unroll
       for (int e = 0; e < EPT; ++e) y[b][e] = 0.f;
+    float hsum[B];  // sum of the thread's token columns (Q4_0 dots)
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      hsum[b] = 0.f;
+      if constexpr (WT == kQ4_0) {
+#pragma unroll
+        for (int e = 0; e < EPT; ++e) hsum[b] += h[b][e];
+      }
+    }
 
     // ---- predictor step 1: u = ReLU(P1 h) ----
     bool to = false;
@@ -895,25 +931,33 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
             for (int jj = 0; jj < gs; ++jj) {
               const uint8_t* it = s.ring + s.item_off[(witem + jj) % kNQ];
               float acc[2 * B];
-              float wu[EPT];
-              w_vals<WT, EPT>(it + (gated ? wrp : 0), d, t, T, wu);
+              // dots of the row at `at` with the thread's token columns
+              auto dots = [&](const uint8_t* at, int base) {
+                float wv[EPT];
+                if constexpr (WT == kQ4_0) {
+                  float sc;
+                  q4_codes<EPT>(at, d, t, wv, sc);
 #pragma unroll
-              for (int b = 0; b < B; ++b) {
-                float a = 0.f;
+                  for (int b = 0; b < B; ++b) {
+                    float a = 0.f;
 #pragma unroll
-                for (int e = 0; e < EPT; ++e) a = fmaf(wu[e], h[b][e], a);
-                acc[B + b] = a;
-              }
-              if (gated) {
-                float wg[EPT];
-                w_vals<WT, EPT>(it, d, t, T, wg);
+                    for (int e = 0; e < EPT; ++e) a = fmaf(wv[e], h[b][e], a);
+                    acc[base + b] = sc * fmaf(16.f, a, -24.f * hsum[b]);
+                  }
+                } else {
+                  w_vals<WT, EPT>(at, d, t, T, wv);
 #pragma unroll
-                for (int b = 0; b < B; ++b) {
-                  float a = 0.f;
+                  for (int b = 0; b < B; ++b) {
+                    float a = 0.f;
 #pragma unroll
-                  for (int e = 0; e < EPT; ++e) a = fmaf(wg[e], h[b][e], a);
-                  acc[b] = a;
+                    for (int e = 0; e < EPT; ++e) a = fmaf(wv[e], h[b][e], a);
+                    acc[base + b] = a;
+                  }
                 }
+              };
+              dots(it + (gated ? wrp : 0), B);
+              if (gated) {
+                dots(it, 0);
               } else {
 #pragma unroll
                 for (int b = 0; b < B; ++b) acc[b] = 0.f;
@@ -947,12 +991,26 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
         if (named_sync_or(1, T, to)) return false;
         for (int jj = 0; jj < gs; ++jj) {
           float wd[EPT];
-          w_vals<WT, EPT>(s.ring + s.item_off[(witem + jj) % kNQ] + rpn * wrp, d, t, T, wd);
+          const uint8_t* at = s.ring + s.item_off[(witem + jj) % kNQ] + rpn * wrp;
+          if constexpr (WT == kQ4_0) {
+            float sc;
+            q4_codes<EPT>(at, d, t, wd, sc);
 #pragma unroll
-          for (int b = 0; b < B; ++b) {
-            const float a = gact[jj * B + b];
+            for (int e = 0; e < EPT; ++e) wd[e] = fmaf(wd[e], 16.f, -24.f);  // q - 8, exact
 #pragma unroll
-            for (int e = 0; e < EPT; ++e) y[b][e] = fmaf(a, wd[e], y[b][e]);
+            for (int b = 0; b < B; ++b) {
+              const float a = gact[jj * B + b] * sc;
+#pragma unroll
+              for (int e = 0; e < EPT; ++e) y[b][e] = fmaf(a, wd[e], y[b][e]);
+            }
+          } else {
+            w_vals<WT, EPT>(at, d, t, T, wd);
+#pragma unroll
+            for (int b = 0; b < B; ++b) {
+              const float a = gact[jj * B + b];
+#pragma unroll
+              for (int e = 0; e < EPT; ++e) y[b][e] = fmaf(a, wd[e], y[b][e]);
+            }
           }
         }
         witem += gs;
