@@ -46,7 +46,7 @@ REF_SECONDS = 150.0  # cap on the timed oracle work of the reference arm
 # capture of 4 layers of the workload (profiles/k_stack_<workload>_b<B>.md);
 # per-layer traffic does not depend on the layer count, so a launch over L
 # layers moves L times this.  Only for captures of the current kernel.
-TRAFFIC_PER_LAYER = {("7b-reglu-fp16", 1): (271.086336e6 + 4.789760e6) / 4}
+TRAFFIC_PER_LAYER = {("7b-reglu-fp16", 1): (271.094016e6 + 3.657472e6) / 4}
 FALLBACK_HBM_GBS = 6650.0
 
 
