@@ -119,33 +119,6 @@ __device__ __forceinline__ void row_vals(const uint8_t* row, int t, int T, float
   }
 }
 
-// EPT owned values of a Q4_0 row laid out as [qs d/2 bytes][sc d/16 bytes]:
-// EPT/2 consecutive qs bytes of one block; their low nibbles are the first
-// run, their high nibbles the run 16 columns on; x = s * (q - 8).
-template <int EPT>
-__device__ __forceinline__ void q4_vals(const uint8_t* row, int d, int t, float (&v)[EPT]) {
-  constexpr int NB = EPT / 2;         // qs bytes per thread
-  constexpr int PER_BLK = 32 / EPT;   // threads per block
-  uint32_t q[NB / 4];
-  if constexpr (NB == 8) {
-    const uint2 qq = *reinterpret_cast<const uint2*>(row + NB * t);
-    q[0] = qq.x;
-    q[1] = qq.y;
-  } else {
-    q[0] = *reinterpret_cast<const uint32_t*>(row + NB * t);
-  }
-  const uint16_t sb = *reinterpret_cast<const uint16_t*>(row + d / 2 + 2 * (t / PER_BLK));
-  const float s = half_bits_to_float(sb);
-#pragma unroll
-  for (int w = 0; w < NB / 4; ++w)
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const uint32_t b = (q[w] >> (8 * k)) & 0xffu;
-      v[w * 4 + k] = s * (float)((int)(b & 15u) - 8);
-      v[NB + w * 4 + k] = s * (float)((int)(b >> 4) - 8);
-    }
-}
-
 // This thread's Q4_0 codes as f = 1 + q/16 (q placed in the top mantissa
 // bits of 1.0f: exact, no integer-to-float conversion), so q - 8 = 16 f - 24;
 // sc is the block's scale.  A dot over the thread's columns is then
@@ -173,10 +146,12 @@ __device__ __forceinline__ void q4_codes(const uint8_t* row, int d, int t, float
     }
 }
 
+// The thread's EPT values of an fp16 or fp32 weight row (Q4_0 rows are read
+// with q4_codes).
 template <int WT, int EPT>
-__device__ __forceinline__ void w_vals(const uint8_t* row, int d, int t, int T, float (&v)[EPT]) {
-  if constexpr (WT == kQ4_0) q4_vals<EPT>(row, d, t, v);
-  else row_vals<WT, EPT, WT>(row, t, T, v);
+__device__ __forceinline__ void w_vals(const uint8_t* row, int t, int T, float (&v)[EPT]) {
+  static_assert(WT != kQ4_0, "Q4_0 rows are read with q4_codes");
+  row_vals<WT, EPT, WT>(row, t, T, v);
 }
 
 template <int WT, int EPT, int X>
@@ -945,7 +920,7 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
                     acc[base + b] = sc * fmaf(16.f, a, -24.f * hsum[b]);
                   }
                 } else {
-                  w_vals<WT, EPT>(at, d, t, T, wv);
+                  w_vals<WT, EPT>(at, t, T, wv);
 #pragma unroll
                   for (int b = 0; b < B; ++b) {
                     float a = 0.f;
@@ -1004,7 +979,7 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
               for (int e = 0; e < EPT; ++e) y[b][e] = fmaf(a, wd[e], y[b][e]);
             }
           } else {
-            w_vals<WT, EPT>(at, d, t, T, wd);
+            w_vals<WT, EPT>(at, t, T, wd);
 #pragma unroll
             for (int b = 0; b < B; ++b) {
               const float a = gact[jj * B + b];
