@@ -129,3 +129,31 @@ def test_relu_stack_keeps_the_tokens_of_a_block_apart():
         hn = h / h.norm(dim=1, keepdim=True)
         cos = (hn @ hn.T)[~torch.eye(8, dtype=torch.bool)]
         assert cos.abs().mean().item() < 0.3, (act, cos.abs().mean().item())  # uncentred ReLU: > 0.8
+
+
+@pytest.mark.parametrize("act,wtype,ptype,batch", [("reglu", "f16", "f16", 1), ("relu", "f32", "f32", 2),
+                                                   ("relu2", "f16", "f16", 3), ("reglu", "q4_0", "f16", 1)])
+def test_layer_bytes_counts_the_bytes_of_the_tensors_read(act, wtype, ptype, batch):
+    """The roofline's algorithmic bytes equal the bytes of the tensors an ideal
+    pass reads and writes, counted from a generated layer: both predictor
+    matrices and bp, the listed rows of every weight matrix with their b1
+    entries, the index list, the token block in, the fp32 output out and b2."""
+    w = W.WORKLOADS["tiny-relu-fp32"].with_(d=256, ffn=1024, rank=32, act=act, wtype=wtype, ptype=ptype)
+    L = W.make_layer(w, 0)
+    n_active = 37
+
+    def row_bytes(m):
+        if isinstance(m, tuple):  # Q4_0 planes
+            return m[0][0].numel() * m[0].element_size() + m[1][0].numel() * m[1].element_size()
+        return m[0].numel() * m.element_size()
+
+    mats = [L["Wg"], L["Wu"], L["WdT"]] if w.gated else [L["Wu"], L["WdT"]]
+    n_list = w.n_hot + n_active
+    tok = torch.empty(0, dtype=L["P1"].dtype).element_size()
+    expect = (L["P1"].numel() * L["P1"].element_size() + L["P2"].numel() * L["P2"].element_size()
+              + L["bp"].numel() * 4
+              + sum(row_bytes(m) for m in mats) * n_list + 4 * n_list
+              + 4 * n_active
+              + batch * w.d * tok + batch * w.d * 4
+              + (L["b2"].numel() * 4 if L["b2"] is not None else 0))
+    assert W.layer_bytes(w, batch, n_active) == pytest.approx(expect, rel=0, abs=1e-6)
