@@ -15,12 +15,15 @@
 //     byte ring with 1-D bulk copies (cp.async.bulk, mbarrier completion), in
 //     consumption order per layer: its P1 rows, a static share of the hot
 //     neurons, its block of P2 rows, then a stream of neurons: the cold rows
-//     its own CTA predicted active and chunks of the remaining hot neurons
-//     claimed from a per-layer atomic counter (the claims balance the
-//     per-CTA cold counts).  A neuron item is its gate/up/down rows plus the
-//     16-byte block of b1 that holds its bias.
+//     its own CTA predicted active (an excess over its running mean is handed
+//     to the other CTAs) and chunks of the remaining hot neurons claimed from
+//     a per-layer atomic counter (the claims balance the per-CTA cold
+//     counts).  A neuron item is its gate/up/down rows plus the 16-byte block
+//     of b1 that holds its bias.
 //   * consumer warps own fixed columns of d: the token block and the fp32
-//     partial output stay in registers for the whole layer.
+//     partial output stay in registers for the whole layer.  The neuron dots
+//     (and the P1 dots of a single token) run on CUDA cores, P2 (and the P1
+//     of a token block of 2) on the tensor cores with mma.sync.
 //   * per layer: P1 rows -> u (global) -> barrier U (static hot neurons fill
 //     the wait) -> P2 scores of the CTA's cold rows -> local ascending list ->
 //     neuron stream -> partial y added into an fp32 accumulator with vector

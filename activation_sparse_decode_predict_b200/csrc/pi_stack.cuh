@@ -80,7 +80,7 @@ struct StackParams {
   int T;           // consumer threads (d / stack_ept(d))
   int ring_bytes;  // shared-memory ring size
   int seg_cap;     // per-CTA capacity of the local active lists
-  int ng;          // neurons per group (<= kMaxGroup; one tensor-core tile for fp16)
+  int ng;          // neurons per group (<= 4 on CUDA cores; one 16-row tile with PI_F16_MMA)
   int p1rows;      // P1 rows per tensor-core group (fp16 predictors)
   int hot_a;       // hot neurons [0, hot_a) are shared out statically, consumed before barrier U
   int hot_static;  // [hot_a, hot_static) are shared out statically, at the head of the neuron
