@@ -105,3 +105,25 @@ def test_python_layer_refuses_cpu_tensors():
     d = _desc(d=64, ffn=100, n_hot=10, rank=8)
     with pytest.raises(ValueError, match="CUDA"):
         pi.residual_rmsnorm(torch.zeros(1, 64), torch.zeros(1, 64), 1e-6, torch.zeros(1, 64))
+
+
+def test_launch_plan_is_host_only():
+    """pi_stack_launches plans a decode step without a GPU: one persistent
+    launch for token blocks of 1-2 on every workload shape, the per-layer
+    kernels (7 per layer; 5 with no cold neurons) for token blocks of 3-16 or
+    a shape the persistent kernel does not take, -1 for invalid arguments."""
+    import pi_workload as W
+    lib = pi.lib()
+    for w in W.WORKLOADS.values():
+        desc = pi.desc_for(w)
+        for batch in (1, 2):
+            assert lib.pi_stack_launches(ctypes.byref(desc), batch, w.layers) == 1, (w.name, batch)
+        for batch in (3, 8, 16):
+            assert lib.pi_stack_launches(ctypes.byref(desc), batch, w.layers) == 7 * w.layers, (w.name, batch)
+    odd = _desc(d=520, ffn=2048, n_hot=103, rank=64, act="relu")  # d not a multiple of 256
+    assert lib.pi_stack_launches(ctypes.byref(odd), 1, 4) == 28
+    all_hot = _desc(d=512, ffn=2048, n_hot=2048, rank=64, act="relu")
+    assert lib.pi_stack_launches(ctypes.byref(all_hot), 3, 4) == 20
+    assert lib.pi_stack_launches(ctypes.byref(_desc()), 1, 0) == -1
+    assert lib.pi_stack_launches(ctypes.byref(_desc()), 0, 4) == -1
+    assert lib.pi_stack_launches(ctypes.byref(_desc(d=100)), 1, 4) == -1
