@@ -222,8 +222,8 @@ def test_decode_stack_small_matches_oracle():
     _stack_check(wl, 2, 3)
 
 
-FULL = [("7b-reglu-fp16", 1), ("13b-reglu-q4_0", 1), ("40b-relu-fp16", 1), ("40b-relu-fp16", 8),
-        ("70b-reglu-fp16", 1), ("70b-reglu-fp16", 4), ("70b-reglu-fp16", 16)]
+FULL = [("7b-reglu-fp16", 1), ("13b-reglu-q4_0", 1), ("40b-relu-fp16", 1), ("40b-relu-fp16", 2),
+        ("40b-relu-fp16", 8), ("70b-reglu-fp16", 1), ("70b-reglu-fp16", 4), ("70b-reglu-fp16", 16)]
 
 
 @pytest.mark.parametrize("name,B", FULL, ids=["%s-b%d" % f for f in FULL])
