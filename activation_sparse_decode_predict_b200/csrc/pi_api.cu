@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include "pi.h"
+#include "pi_args.h"
 #include "pi_batch.cuh"
 #include "pi_common.cuh"
 #include "pi_kernels_v1.cuh"
@@ -21,19 +22,13 @@ pi_status fail(pi_status st, const char* fmt, const char* what) {
   return st;
 }
 
-pi_status cuda_fail(cudaError_t e, const char* where) {
-  snprintf(g_err, sizeof(g_err), "%s: %s", where, cudaGetErrorString(e));
-  return PI_ERR_CUDA;
-}
-
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
-  return n;
-}
+}  // namespace
+
+namespace pi {
+
+void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
 
 pi_status check_desc(const pi_ffn_desc* d, int32_t batch) {
   if (!d) return fail(PI_ERR_INVALID_ARG, "%s", "desc is NULL");
@@ -57,6 +52,30 @@ pi_status check_ptr(const void* p, size_t align, const char* name) {
   if (!p) return fail(PI_ERR_INVALID_ARG, "%s is NULL", name);
   if (!aligned(p, align)) return fail(PI_ERR_INVALID_ARG, "%s is not aligned", name);
   return PI_OK;
+}
+
+}  // namespace pi
+
+namespace {
+
+using pi::check_desc;
+using pi::check_ptr;
+
+#ifdef PI_TRACE
+// profiling builds: where the decode-step kernel writes its phase stamps
+uint64_t* g_trace = nullptr;
+#endif
+
+pi_status cuda_fail(cudaError_t e, const char* where) {
+  snprintf(g_err, sizeof(g_err), "%s: %s", where, cudaGetErrorString(e));
+  return PI_ERR_CUDA;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
 }
 
 pi_status check_weight(const pi_ffn_desc* d, pi_weight w, const char* name) {
@@ -253,6 +272,9 @@ pi_status fused_stack(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, cons
   P.pool = reinterpret_cast<pi::Ctrl*>(ws)->pool;
   P.lcnt = reinterpret_cast<int*>(ws + L.lcnt);
   P.don = reinterpret_cast<int*>(ws + L.don);
+#ifdef PI_TRACE
+  P.trace = g_trace;
+#endif
   for (int l = 0; l < n_layers; ++l) {
     const pi_layer_weights& w = layers[l];
     pi::StackLayer& s = P.layers[l];
@@ -277,11 +299,12 @@ pi_status fused_stack(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, cons
 
 }  // namespace
 
-namespace pi {
-void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
-}  // namespace pi
-
 extern "C" {
+
+#ifdef PI_TRACE
+// profiling builds only: [n_layers, grid, kTraceEvents] uint64 device buffer (or NULL)
+PI_API void pi_trace_buffer(void* buf) { g_trace = static_cast<uint64_t*>(buf); }
+#endif
 
 const char* pi_last_error(void) { return g_err; }
 

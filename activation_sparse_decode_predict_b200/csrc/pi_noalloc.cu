@@ -18,12 +18,9 @@
 #include <stdio.h>
 
 #include "pi.h"
+#include "pi_args.h"
 #include "pi_kernels_v1.cuh"
 #include "pi_layout.h"
-
-namespace pi {
-void set_last_error(const char* msg);  // pi_api.cu: text returned by pi_last_error()
-}
 
 namespace {
 
@@ -57,8 +54,6 @@ pi_status scratch_address(void** out) {
   return PI_OK;
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 }  // namespace
 
 static_assert(kStaticScratchBytes == PI_STATIC_SCRATCH_BYTES, "header and library agree on the scratch size");
@@ -67,15 +62,18 @@ extern "C" {
 
 pi_status pi_predict_static(const pi_ffn_desc* desc, int32_t batch, const void* h, const void* P1, const void* P2,
                             const float* bp, float threshold, int32_t* idx, int32_t* count, void* stream) {
-  if (!desc) return err(PI_ERR_INVALID_ARG, "desc is NULL");
-  const int d = desc->d, ffn = desc->ffn, n_hot = desc->n_hot, r = desc->rank;
-  if (d <= 0 || d % 8 || ffn <= 0 || n_hot < 0 || n_hot > ffn || r <= 0 || r % 8 ||
-      (desc->ptype != PI_F32 && desc->ptype != PI_F16) || batch < 1 || batch > PI_MAX_BATCH)
-    return err(PI_ERR_INVALID_ARG, "invalid descriptor or batch");
+  // the same checks, with the same alignments, as pi_predict: nothing is
+  // launched unless every one passes
+  pi_status s = pi::check_desc(desc, batch);
+  if (s != PI_OK) return s;
+  const int ffn = desc->ffn, n_hot = desc->n_hot, r = desc->rank;
   const int C = ffn - n_hot;
-  if (!h || !P1 || !count || (C > 0 && (!P2 || !idx))) return err(PI_ERR_INVALID_ARG, "NULL tensor pointer");
-  if (!aligned16(h) || !aligned16(P1) || (C > 0 && !aligned16(P2)))
-    return err(PI_ERR_INVALID_ARG, "h, P1 and P2 must be 16-byte aligned");
+  if ((s = pi::check_ptr(h, 16, "h")) != PI_OK) return s;
+  if ((s = pi::check_ptr(P1, 16, "P1")) != PI_OK) return s;
+  if (C > 0 && (s = pi::check_ptr(P2, 16, "P2")) != PI_OK) return s;
+  if (bp && (s = pi::check_ptr(bp, 4, "bp")) != PI_OK) return s;
+  if (C > 0 && (s = pi::check_ptr(idx, 4, "idx")) != PI_OK) return s;
+  if ((s = pi::check_ptr(count, 4, "count")) != PI_OK) return s;
   // scratch: u [batch, rank] fp32, then the tile masks and tile counts
   const int n_tiles = (C + 255) / 256;
   const size_t u_bytes = pi::align256((size_t)batch * r * 4);
@@ -85,7 +83,7 @@ pi_status pi_predict_static(const pi_ffn_desc* desc, int32_t batch, const void* 
     return err(PI_ERR_CAPACITY,
                "pi_predict_static: batch x rank x 4 bytes plus the tile masks exceed the 1 MiB static scratch");
   void* base = nullptr;
-  pi_status s = scratch_address(&base);
+  s = scratch_address(&base);
   if (s != PI_OK) return s;
   char* b = static_cast<char*>(base);
   float* u = reinterpret_cast<float*>(b);
@@ -94,7 +92,7 @@ pi_status pi_predict_static(const pi_ffn_desc* desc, int32_t batch, const void* 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaError_t e = pi::launch_pred_u(desc->ptype, P1, h, batch, d, r, u, sms, st);
+  cudaError_t e = pi::launch_pred_u(desc->ptype, P1, h, batch, desc->d, r, u, sms, st);
   if (e == cudaSuccess) e = pi::launch_pred_score(desc->ptype, P2, bp, u, batch, r, C, threshold, tmask, tcount, st);
   if (e == cudaSuccess) e = pi::launch_compact(tmask, tcount, C, n_hot, idx, count, st);
   if (e != cudaSuccess) return err(PI_ERR_CUDA, cudaGetErrorString(e));

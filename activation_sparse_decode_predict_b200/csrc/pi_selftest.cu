@@ -8,11 +8,11 @@
 #include <cuda_runtime.h>
 
 #include "pi.h"
+#include "pi_args.h"
 #include "pi_common.cuh"
 #include "pi_sync.cuh"
 
 namespace pi {
-void set_last_error(const char* msg);
 
 namespace {
 

@@ -35,10 +35,24 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "pi_common.cuh"
 #include "pi_mma.cuh"
 #include "pi_stack.cuh"
 #include "pi_sync.cuh"
+
+// PI_TRACE builds record %globaltimer stamps at the phase boundaries of every
+// layer and CTA into p.trace (a profiling aid; the default build has none).
+#ifdef PI_TRACE
+#define PI_STAMP(l, e) \
+  do { if (p.trace) p.trace[((size_t)(l) * gridDim.x + blockIdx.x) * kTraceEvents + (e)] = global_ns(); } while (0)
+#define PI_STAMP_VAL(l, e, v) \
+  do { if (p.trace) p.trace[((size_t)(l) * gridDim.x + blockIdx.x) * kTraceEvents + (e)] = (uint64_t)(v); } while (0)
+#else
+#define PI_STAMP(l, e) do { } while (0)
+#define PI_STAMP_VAL(l, e, v) do { } while (0)
+#endif
 
 namespace pi {
 
@@ -513,8 +527,10 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
       bool ok = true;
       if (lane == 0) {
         ok = mbar_wait(s.u_bar, l & 1, ctrl);
+        PI_STAMP(l, 10);
         if (ok) grid_arrive(ctrl);
         if (ok) ok = grid_wait(ctrl, base, 2 * l, G);
+        PI_STAMP(l, 11);
       }
       if (!__shfl_sync(0xffffffffu, ok, 0)) return;
       if constexpr (PT == kF16) {
@@ -628,6 +644,8 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
         }
         if (ok) ok = mbar_wait(s.list_bar, l & 1, ctrl);
         const int nloc = s.misc[0];
+        PI_STAMP(l, 12);
+        PI_STAMP_VAL(l, 15, nloc);
         // A CTA with clearly more predicted rows than it has seen on average
         // hands the excess to the other CTAs (slots reserved with one atomic,
         // written as row + 1); every CTA takes handed-over rows by ticket once
@@ -657,6 +675,7 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
           ok = pr.issue_neuron(Ly, j, WT, gated, 1);
         }
         if (ok) ok = pr.issue_marker();
+        PI_STAMP(l, 13);
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
     }
@@ -721,6 +740,7 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
 
   for (int l = 0; l < p.L; ++l) {
     const StackLayer& Ly = p.layers[l];
+    if (t == 0) PI_STAMP(l, 0);
 #pragma unroll
     for (int b = 0; b < B; ++b)
 #pragma unroll
@@ -819,6 +839,7 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
           for (int b = 0; b < B; ++b) p.u_g[(int64_t)b * r + kk + i] = fmaxf(acc[i * B + b], 0.f);
     }
     }  // predictor step 1
+    if (t == 0) PI_STAMP(l, 1);
 #pragma unroll
     for (int i = 0; i < kShareRegs; ++i) {
       const int x = t + i * T;
@@ -1000,6 +1021,7 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
     if (t == 0) mbar_arrive(s.u_bar);  // the barrier warp arrives at barrier U
     // the static hot neurons need no predictor: they fill the wait for barrier U
     if (!run_stream()) return;
+    if (t == 0) PI_STAMP(l, 2);
     if constexpr (PT == kF16) {
       for (int x = t; x < (c1 - c0) * B; x += T) s.sc[x] = 0.f;  // partial scores accumulate here
     }
@@ -1008,6 +1030,7 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
       const bool okw = mbar_wait(s.u_ready, l & 1, ctrl);
       if (named_sync_or(1, T, !okw)) return;
     }
+    if (t == 0) PI_STAMP(l, 3);
     // the other accumulator buffer is free now (its last readers passed barrier U)
     {
       float4* nxt = reinterpret_cast<float4*>(p.yacc) + (size_t)((l + 1) & 1) * ybuf4;
@@ -1165,6 +1188,7 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
       }
     }
     if (named_sync_or(1, T, to)) return;
+    if (t == 0) PI_STAMP(l, 4);
     // local ascending list of this CTA's active cold rows (consumer warp 0):
     // to the producer through shared memory, and parked in this CTA's own
     // stretch of idx (compacted after the last layer) with its count
@@ -1188,10 +1212,12 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(s.list_bar);
+      if (lane == 0) PI_STAMP(l, 5);
     }
 
     // ---- the neuron stream: claimed hot chunks and this CTA's predicted cold rows ----
     if (!run_stream()) return;
+    if (t == 0) PI_STAMP(l, 6);
 
     // ---- split-K: add the partial into one of K fp32 accumulator copies ----
     {
@@ -1211,12 +1237,14 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
     }
     if (l + 1 < p.L) load_shares(p.layers[l + 1]);  // in flight across barrier Y and the glue
     named_sync(1, T);
+    if (t == 0) PI_STAMP(l, 7);
     if (t == 0) grid_arrive(ctrl);
     {
       bool okw = true;
       if (t == 0) okw = grid_wait(ctrl, base, 2 * l + 1, G);
       if (named_sync_or(1, T, !okw)) return;
     }
+    if (t == 0) PI_STAMP(l, 8);
 
     // ---- glue: h <- RMSNorm(h + y + b2), rounded to the token type ----
     {
@@ -1281,6 +1309,7 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
         }
       }
     }
+    if (t == 0) PI_STAMP(l, 9);
   }
   // ---- the ascending lists: every CTA moves its parked list of each layer
   // to its offset (the sum of the lower CTAs' counts); layers in chunks whose
@@ -1355,11 +1384,22 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
 template <int WT, int PT, int B, int EPT>
 cudaError_t launch_t(const StackParams& p, int G, size_t smem, cudaStream_t st) {
   auto fn = k_stack<WT, PT, B, EPT>;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = true;
+  // the dynamic shared-memory limit is a per-device attribute of the kernel:
+  // set it once on every device that launches it (the first launch on a
+  // device should come before any stream capture)
+  static std::mutex mu;
+  static bool configured[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!configured[dev]) {
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+      if (e != cudaSuccess) return e;
+      configured[dev] = true;
+    }
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(G);

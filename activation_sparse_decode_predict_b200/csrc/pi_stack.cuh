@@ -9,6 +9,8 @@
 namespace pi {
 
 constexpr int kMaxLayers = 128;
+constexpr int kMaxDevices = 64;      // devices per process the launcher keeps state for
+constexpr int kTraceEvents = 16;     // phase stamps per (layer, CTA) of a PI_TRACE build
 constexpr int kNQ = 64;              // items in flight per CTA (queue depth)
 constexpr int kMaxConsumers = 512;   // consumer threads per CTA (d <= 8192)
 constexpr int kMaxRank = 4096;
@@ -100,6 +102,7 @@ struct StackParams {
   int* pool;        // [L] claim counters of the hot neurons (zero between launches)
   int* lcnt;        // [L, G] per-CTA counts of the local active lists
   int* don;         // [L, C] cold rows handed to other CTAs (row + 1; zero = not written yet)
+  uint64_t* trace;  // [L, G, kTraceEvents] phase stamps (PI_TRACE builds only; else unused)
   StackLayer layers[kMaxLayers];
 };
 

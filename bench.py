@@ -43,7 +43,7 @@ POOL = 64         # distinct token blocks (one captured graph each), cycled over
 E2E_STEPS = 200   # steps of the end-to-end (host buffers) measurement
 REF_SECONDS = 150.0  # cap on the timed oracle work of the reference arm
 # DRAM bytes (read + write) per layer of the decode-step kernel, from an ncu
-# capture of 4 layers of the workload (profiles/k_stack_<workload>_b<B>.md);
+# capture of a few layers of the workload (the committed ncu summaries);
 # per-layer traffic does not depend on the layer count, so a launch over L
 # layers moves L times this.  Only for captures of the current kernel.
 TRAFFIC_PER_LAYER = {("7b-reglu-fp16", 1): (271.094016e6 + 3.657472e6) / 4}
@@ -70,7 +70,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="7b-reglu-fp16", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--workload", default="70b-reglu-fp16", choices=sorted(W.WORKLOADS))
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--sparsity", type=float, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -92,54 +92,113 @@ def peak_hbm():
 
 
 class ClockSampler:
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock, power and clock-event reasons of one GPU, sampled through NVML
+    every few milliseconds while the timed region runs (a background thread),
+    so that even a region of a few tens of milliseconds gets samples.  One
+    extra sample is always taken when the region ends.  Without NVML it falls
+    back to nvidia-smi's loop."""
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+    PERIOD_S = 0.005
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
+
+    def __init__(self, device):
+        self.device = device
+        self.rows = []
+        self._stop = None
+        self._thread = None
+        self._nv = None
+        self._h = None
+        self._smi = None
+
+    def _handle(self):
+        import pynvml as nv
+        nv.nvmlInit()
+        props = torch.cuda.get_device_properties(self.device)
+        uuid = getattr(props, "uuid", None)
+        if uuid is not None:
+            try:
+                return nv, nv.nvmlDeviceGetHandleByUUID("GPU-" + str(uuid))
+            except Exception:
+                pass
+        return nv, nv.nvmlDeviceGetHandleByIndex(torch.cuda.current_device() if self.device is None else
+                                                 torch.device(self.device).index or 0)
+
+    def sample(self):
+        nv, h = self._nv, self._h
+        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+        smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+        try:
+            power = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+        except Exception:
+            power = None
+        self.rows.append((float(sm), float(smax), int(reasons), power))
+
+    def _loop(self):
+        while not self._stop.is_set():
+            try:
+                self.sample()
+            except Exception:
+                return
+            self._stop.wait(self.PERIOD_S)
 
     def __enter__(self):
+        import threading
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.QUERY,
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            self._nv, self._h = self._handle()
+            self._stop = threading.Event()
+            self._thread = threading.Thread(target=self._loop, daemon=True)
+            self._thread.start()
         except Exception:
-            self.proc = None
+            self._nv = None
+            try:
+                fd, path = tempfile.mkstemp(suffix=".csv")
+                os.close(fd)
+                q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+                     "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                     "clocks_event_reasons.sw_power_cap")
+                self._smi = (subprocess.Popen(["nvidia-smi", "--query-gpu=" + q, "--format=csv,noheader,nounits",
+                                               "-lms", "200"], stdout=open(path, "w"), stderr=subprocess.DEVNULL),
+                             path)
+            except Exception:
+                self._smi = None
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
             try:
-                self.proc.wait(timeout=5)
+                self.sample()   # the end of the region is always sampled
             except Exception:
-                self.proc.kill()
+                pass
+        if self._smi is not None:
+            proc, path = self._smi
+            proc.terminate()
+            try:
+                proc.wait(timeout=5)
+            except Exception:
+                proc.kill()
+            for line in open(path):
+                p = [x.strip() for x in line.split(",")]
+                try:
+                    bits = sum(m for (_, m), v in zip(self.REASONS[:4], p[3:7]) if v.lower() == "active")
+                    self.rows.append((float(p[0]), float(p[1]), bits, float(p[2])))
+                except (ValueError, IndexError):
+                    continue
+            os.unlink(path)
         return False
 
     def summary(self):
-        if not self.path or not os.path.exists(self.path):
+        if not self.rows:
             return None
-        rows = []
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
-            except ValueError:
-                continue
-        os.unlink(self.path)
-        if not rows:
-            return None
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
-        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": reasons, "samples": len(rows)}
+        reasons = sorted({name for _, _, bits, _ in self.rows for name, m in self.REASONS if bits & m})
+        powers = [p for *_, p in self.rows if p is not None]
+        return {"sm_mhz": statistics.median(r[0] for r in self.rows), "sm_max_mhz": max(r[1] for r in self.rows),
+                "reasons": reasons, "samples": len(self.rows),
+                "source": "nvml" if self._nv is not None else "nvidia-smi",
+                "power_w_max": round(max(powers), 1) if powers else None}
 
 
 # ----------------------------------------------------------------------------
@@ -191,7 +250,7 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local_rank) as clk:
+    with ClockSampler(dev) as clk:
         with torch.cuda.stream(stream):
             torch.cuda.synchronize()
             # profiler range = the timed region (ncu --profile-from-start off)
@@ -324,7 +383,7 @@ def _oracle_layer_step(wl, B, Ln, step):
     return oracle.residual_rmsnorm(h, y, W.RMS_EPS)
 
 
-def oracle_sample(wl, B, layers, n_sample_layers, min_seconds=10.0, max_steps=200, threads=None):
+def oracle_sample(wl, B, layers, n_sample_layers, min_seconds=10.0, max_steps=200, threads=None, host=None):
     """Time the oracle (predictor + masked FFN + glue) on the first layers of
     the stack for token blocks until about `min_seconds` of CPU work are done;
     returns (tokens/s scaled to the full stack, seconds spent, threads used,
@@ -332,7 +391,8 @@ def oracle_sample(wl, B, layers, n_sample_layers, min_seconds=10.0, max_steps=20
     import oracle
     if threads:
         oracle.set_threads(threads)
-    host = _host_layers(layers[:n_sample_layers])
+    if host is None:
+        host = _host_layers(layers[:n_sample_layers])
     t0 = time.perf_counter()
     n_steps = 0
     while n_steps < max_steps and (n_steps == 0 or time.perf_counter() - t0 < min_seconds):
@@ -434,9 +494,13 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         wl, B, layers, _ = ctx
         n_s = 2 if wl.d * wl.ffn <= 64e6 else 1
-        tok_s, dt, cores, desc = oracle_sample(wl, B, layers, n_s, threads=os.cpu_count())
+        host = _host_layers(layers[:n_s])
+        tok_s, dt, cores, desc = oracle_sample(wl, B, layers, n_s, threads=os.cpu_count(), host=host)
+        tok_1, dt_1, _, desc_1 = oracle_sample(wl, B, layers, n_s, min_seconds=5.0, threads=1, host=host)
         out["cpu_baseline"] = {"value": round(tok_s, 4), "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                               "sample": desc, "cpu": cpu_model(), "seconds": round(dt, 2)}
+                               "sample": desc, "cpu": cpu_model(), "seconds": round(dt, 2),
+                               "single_thread": {"value": round(tok_1, 4), "unit": "tokens/s", "cores": 1,
+                                                 "sample": desc_1, "seconds": round(dt_1, 2)}}
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:

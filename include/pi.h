@@ -243,14 +243,23 @@ PI_API pi_status pi_get_device_status(void *ws, int32_t *status_out, int32_t cle
  * own every allocation, or serving loops that must not call cudaMalloc once
  * running, because an allocation can synchronise the device).
  *
- * Same arguments, results and rules as pi_predict, minus the workspace: the
- * scratch lives in one library-owned device array of PI_STATIC_SCRATCH_BYTES
- * (1 MiB), held on every GPU that loads the library until the process exits.
+ * Same arguments, argument checks and rules as pi_predict, minus the
+ * workspace: the scratch lives in one library-owned device array of
+ * PI_STATIC_SCRATCH_BYTES (1 MiB), held on every GPU that loads the library
+ * until the process exits.  The list equals pi_predict's except for neurons
+ * whose score lies within rounding (well under 1e-3) of the threshold: for
+ * fp16 predictors and token blocks of 3-16 pi_predict runs its tensor-core
+ * predictor, this call always the CUDA-core one.
  * Limit: align256(batch * rank * 4) + align256(ceil(C/256) * 32) +
  * align256(ceil(C/256) * 4) <= 1 MiB (C = ffn - n_hot), else
- * PI_ERR_CAPACITY and nothing is launched.  The call allocates nothing.
+ * PI_ERR_CAPACITY and nothing is launched.  The call itself never calls
+ * cudaMalloc.
  * - The first call on a device looks the array's address up on that device
- *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   (cudaGetSymbolAddress).  Under CUDA's lazy module loading (the default)
+ *   that first call may also load the library's device code on the device
+ *   and create the array there, which can allocate and synchronise: make it
+ *   during set-up, before any stream capture and before the loop that must
+ *   not allocate (CUDA_MODULE_LOADING=EAGER loads it when the process starts).
  * - Every call shares the one array and the last call's contents stay in it;
  *   nothing in it needs to start at zero (each call writes all it reads).
  * - Calls that can overlap on the GPU (different streams, or several host

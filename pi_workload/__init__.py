@@ -106,23 +106,6 @@ SPARSITY_SWEEP_70B = (0.80, 0.90, 0.95)
 _TORCH_DT = {"f32": torch.float32, "f16": torch.float16}
 
 
-def _decode_rows(t, d: int) -> torch.Tensor:
-    """fp32 rows of a weight in any stored form (fp32/fp16 tensor or Q4_0 planes)."""
-    if isinstance(t, tuple):
-        qs, sc = t
-        F = qs.shape[0]
-        q = qs.to(torch.int32)
-        lo = (q & 15) - 8
-        hi = (q >> 4) - 8
-        blocks = torch.cat([lo.view(F, d // 32, 16), hi.view(F, d // 32, 16)], dim=2).float()
-        return (blocks * sc.float().view(F, d // 32, 1)).view(F, d)
-    return t.float()
-
-
-def _row_norms(t, d: int) -> torch.Tensor:
-    return _decode_rows(t, d).norm(dim=1)
-
-
 def _seed(w: Workload, layer: int, tensor: int) -> int:
     key = (w.cfg_id * 1_000_003 + int(round(w.sparsity * 1000))) * 10_007 + layer
     return (key * 131 + tensor) & 0x7FFF_FFFF_FFFF
@@ -213,6 +196,32 @@ def make_layer(w: Workload, layer: int, device="cpu") -> dict:
     WdT = torch.randn(F, d, generator=_gen(device, _seed(w, layer, 6)), device=device) * inv_sd
 
     b1_orig = torch.special.ndtri(torch.as_tensor(p_orig, dtype=torch.float64)).to(torch.float32)
+    b1 = b1_orig.to(device)[perm_t].contiguous()
+    b2 = None
+    if w.has_b2:
+        b2 = (torch.randn(d, generator=_gen(device, _seed(w, layer, 7)), device=device) * 0.05).float()
+    if not w.gated:
+        # ReLU / squared ReLU: every token's output has a common part, the
+        # expected activations (positive for the often-firing neurons) times
+        # their down rows.  Added layer after layer it would pull the tokens of
+        # a block onto one direction, and the union of their active sets would
+        # shrink to a single token's.  b2 removes it: b2 -= sum_j E[a_j] WdT[j],
+        # with z_j = w_j . h + b1_j ~ N(b1_j, |w_j|^2) for ||h||^2 = d, taken on
+        # the rows before they are rounded to their storage type.  (ReGLU
+        # needs nothing: its up dot has mean zero.)
+        z_sd = W_pred.norm(dim=1).double()[perm_t]
+        bz = b1.double()
+        t = bz / z_sd
+        pdf = torch.exp(-0.5 * t * t) / math.sqrt(2.0 * math.pi)
+        cdf = 0.5 * torch.erfc(-t / math.sqrt(2.0))
+        if w.act == "relu2":
+            ea = (bz * bz + z_sd * z_sd) * cdf + bz * z_sd * pdf
+        else:
+            ea = bz * cdf + z_sd * pdf
+        ea_orig = torch.zeros(F, dtype=torch.float32, device=device)
+        ea_orig[perm_t] = ea.float()
+        common = (ea_orig.unsqueeze(0) @ WdT).squeeze(0)
+        b2 = (-common if b2 is None else b2 - common).float().contiguous()
     out = {"perm": perm, "p": p_orig[perm], "thr": w.thr}
     if w.gated:
         out["Wg"] = _as_wtype(W_pred[perm_t], w.wtype)
@@ -223,30 +232,7 @@ def make_layer(w: Workload, layer: int, device="cpu") -> dict:
     del W_pred, W_other
     out["WdT"] = _as_wtype(WdT[perm_t], w.wtype)
     del WdT
-    b1 = b1_orig.to(device)[perm_t].contiguous()
     out["b1"] = b1
-    b2 = None
-    if w.has_b2:
-        b2 = (torch.randn(d, generator=_gen(device, _seed(w, layer, 7)), device=device) * 0.05).float()
-    if not w.gated:
-        # ReLU / squared ReLU: every token's output has a common part, the
-        # expected activations (positive for the often-firing neurons) times
-        # their down rows.  Added layer after layer it would pull the tokens of
-        # a block onto one direction, and the union of their active sets would
-        # shrink to a single token's.  b2 removes it: b2 -= sum_j E[a_j] WdT[j],
-        # with z_j = w_j . h + b1_j ~ N(b1_j, |w_j|^2) for ||h||^2 = d.  (ReGLU
-        # needs nothing: its up dot has mean zero.)
-        z_sd = _row_norms(out["Wu"], d).to(device).double()
-        bz = b1.double()
-        t = bz / z_sd
-        pdf = torch.exp(-0.5 * t * t) / math.sqrt(2.0 * math.pi)
-        cdf = 0.5 * torch.erfc(-t / math.sqrt(2.0))
-        if w.act == "relu2":
-            ea = (bz * bz + z_sd * z_sd) * cdf + bz * z_sd * pdf
-        else:
-            ea = bz * cdf + z_sd * pdf
-        common = (ea.float().unsqueeze(0) @ _decode_rows(out["WdT"], d).to(device).float()).squeeze(0)
-        b2 = (-common if b2 is None else b2 - common).float().contiguous()
     out["b2"] = b2
     pt = _TORCH_DT[w.ptype]
     out["P1"] = torch.cat([V, -V], dim=0).to(pt).contiguous()

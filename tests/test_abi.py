@@ -127,3 +127,33 @@ def test_launch_plan_is_host_only():
     assert lib.pi_stack_launches(ctypes.byref(_desc()), 1, 0) == -1
     assert lib.pi_stack_launches(ctypes.byref(_desc()), 0, 4) == -1
     assert lib.pi_stack_launches(ctypes.byref(_desc(d=100)), 1, 4) == -1
+
+
+def test_static_predict_checks_like_predict_before_any_launch():
+    """pi_predict_static applies pi_predict's descriptor and pointer checks
+    (same alignments: h, P1, P2 16 bytes; bp, idx, count 4 bytes) and returns
+    before touching the device.  The addresses are never dereferenced: every
+    call here fails on the host."""
+    lib = pi.lib()
+    d = _desc(d=512, ffn=2048, n_hot=100, rank=64)
+    fake = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 2)   # not 4-byte aligned
+    mis16 = ctypes.c_void_p((1 << 20) + 4)  # 4- but not 16-byte aligned
+
+    def call(desc=d, batch=1, h=fake, P1=fake, P2=fake, bp=None, idx=fake, count=fake):
+        return lib.pi_predict_static(ctypes.byref(desc) if desc is not None else None, batch, h, P1, P2, bp, 0.5,
+                                     idx, count, None)
+
+    assert call(bp=odd) == B.PI_ERR_INVALID_ARG and b"bp" in lib.pi_last_error()
+    assert call(count=odd) == B.PI_ERR_INVALID_ARG and b"count" in lib.pi_last_error()
+    assert call(idx=odd) == B.PI_ERR_INVALID_ARG and b"idx" in lib.pi_last_error()
+    assert call(h=mis16) == B.PI_ERR_INVALID_ARG and b"h" in lib.pi_last_error()
+    assert call(P2=mis16) == B.PI_ERR_INVALID_ARG and b"P2" in lib.pi_last_error()
+    assert call(desc=None) == B.PI_ERR_INVALID_ARG
+    assert call(batch=17) == B.PI_ERR_INVALID_ARG
+    # the limits pi_predict enforces through its descriptor check
+    assert call(desc=_desc(d=16392, ffn=2048, n_hot=100, rank=64)) == B.PI_ERR_UNSUPPORTED
+    assert call(desc=_desc(d=512, ffn=2048, n_hot=100, rank=65544)) == B.PI_ERR_UNSUPPORTED
+    bad_act = _desc(d=512, ffn=2048, n_hot=100, rank=64)
+    bad_act.act = 7
+    assert call(desc=bad_act) == B.PI_ERR_INVALID_ARG

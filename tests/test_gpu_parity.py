@@ -178,11 +178,18 @@ def test_residual_rmsnorm_matches_oracle(htype):
     assert np.abs(got - ref).max() <= tol * np.abs(ref).max()
 
 
-def _stack_check(wl, B, n_layers, cols=None, seed_step=0):
+def _stack_check(wl, B, n_layers, cols=None, seed_step=0, thr=None, dense=False):
     """pi_decode_stack (the benchmark's launch) against the oracle, teacher-forced
-    per layer on the GPU's own layer inputs (h_trace)."""
+    per layer on the GPU's own layer inputs (h_trace).  `thr` overrides every
+    layer's threshold; `dense` also compares each layer with the oracle's dense
+    FFN (every neuron listed).  Returns the number of (layer, cold row) pairs
+    whose score fell in the 1e-3 band, which is bounded so that the list check
+    never becomes vacuous."""
     desc = pi.desc_for(wl)
     layers = [W.make_layer(wl, l, device="cuda") for l in range(n_layers)]
+    if thr is not None:
+        for L in layers:
+            L["thr"] = thr
     arr = pi.layer_array([pi.layer_weights(L) for L in layers])
     h0 = W.make_tokens(wl, B, seed_step, device="cuda")
     ws = pi.workspace(desc, B)
@@ -204,17 +211,27 @@ def _stack_check(wl, B, n_layers, cols=None, seed_step=0):
         if C == 0:
             assert n == 0
         orc = oracle_predict(L, h_l, wl)
-        n_amb += check_index_list(gidx, orc, wl.thr, wl.n_hot, wl.ffn)
+        n_amb += check_index_list(gidx, orc, L["thr"], wl.n_hot, wl.ffn)
         ref = oracle_layer(L, h_l, wl, gidx, cols=cols)
         got = to_np(y[l]).astype(np.float64)
         if cols is not None:
             got = got[:, cols]
         assert rel_err(got, ref) <= TOL[wl.wtype], "layer %d" % l
+        if dense:
+            Ln = {k: to_np(L[k]) for k in ("Wg", "Wu", "WdT", "b1", "b2")}
+            ref_d = oracle.dense_ffn(h_l, Ln["Wg"], Ln["Wu"], Ln["WdT"], Ln["b1"], Ln["b2"], wl.act, wl.n_hot,
+                                     wl.ffn)
+            assert rel_err(to_np(y[l]).astype(np.float64), ref_d) <= TOL[wl.wtype], "layer %d (dense)" % l
         # glue: the next layer's input (or h_out) is RMSNorm(h_l + y_l)
         nxt = to_np(trace[l + 1]) if l + 1 < n_layers else to_np(h_out)
         glue = oracle.residual_rmsnorm(h_l, to_np(y[l]).astype(np.float64), W.RMS_EPS)
         assert np.abs(nxt.astype(np.float64) - glue).max() <= 2 ** -9 * np.abs(glue).max()
-    return n_amb
+    # about 2e-3 of N(0, 1)-like scores fall within 1e-3 of the threshold; a
+    # much larger count would mean the band hides real disagreements
+    amb_max = 0.01 * max(C, 1) * n_layers + 8
+    print("%s B=%d: %d of %d (layer, cold row) pairs in the 1e-3 band" % (wl.name, B, n_amb, C * n_layers))
+    assert n_amb <= amb_max, "%d (layer, cold row) pairs in the band, bound %d" % (n_amb, amb_max)
+    return n_amb, counts.cpu().numpy()
 
 
 def test_decode_stack_small_matches_oracle():
@@ -254,6 +271,53 @@ def test_fused_stack_matches_oracle(case):
     wl = _workload(name, d, ffn, hot, rank, act, wt, pt, B).with_(layers=L)
     assert pi.stack_launches(pi.desc_for(wl), B, L) == 1
     _stack_check(wl, B, L, seed_step=3)
+
+
+# (name, d, ffn, hot_frac, rank, act, wtype, ptype, batch, layers)
+EXTREMES = [
+    ("ext-f16-reglu", 1024, 3000, 0.10, 64, "reglu", "f16", "f16", 1, 3),
+    ("ext-f16-relu-b2", 1536, 5000, 0.08, 128, "relu", "f16", "f16", 2, 3),
+    ("ext-q4-reglu-b2", 1024, 2500, 0.10, 64, "reglu", "q4_0", "f16", 2, 3),
+    ("ext-f32-relu2", 512, 2048, 0.05, 64, "relu2", "f32", "f32", 1, 3),
+]
+
+
+@pytest.mark.parametrize("case", EXTREMES, ids=[e[0] for e in EXTREMES])
+def test_fused_stack_every_cold_neuron_active_equals_dense(case):
+    """Threshold -1e30 on every layer: the persistent kernel's lists are every
+    cold row, so each layer must equal the dense FFN (skipping no neuron leaves
+    the output unchanged: unite.ai, "Nöron Bilinçli Operatör").  Every CTA's
+    local list is its whole P2 share: the longest lists the kernel can see."""
+    name, d, ffn, hot, rank, act, wt, pt, B, L = case
+    wl = _workload(name, d, ffn, hot, rank, act, wt, pt, B).with_(layers=L)
+    assert pi.stack_launches(pi.desc_for(wl), B, L) == 1
+    n_amb, counts = _stack_check(wl, B, L, seed_step=5, thr=-1e30, dense=True)
+    assert n_amb == 0
+    assert np.all(counts == wl.n_cold)
+
+
+@pytest.mark.parametrize("case", EXTREMES, ids=[e[0] for e in EXTREMES])
+def test_fused_stack_no_cold_neuron_active_is_hot_slice(case):
+    """Threshold +1e30 on every layer: empty lists, and each layer's output is
+    the hot slice alone."""
+    name, d, ffn, hot, rank, act, wt, pt, B, L = case
+    wl = _workload(name, d, ffn, hot, rank, act, wt, pt, B).with_(layers=L)
+    assert pi.stack_launches(pi.desc_for(wl), B, L) == 1
+    n_amb, counts = _stack_check(wl, B, L, seed_step=6, thr=1e30)
+    assert n_amb == 0
+    assert np.all(counts == 0)
+
+
+def test_full_size_70b_sparsity_80_token_block_of_2():
+    """The densest full-size setting of the persistent kernel: 70B-shaped
+    layers at 80 % sparsity with a token block of 2 (the longest per-CTA lists
+    and hand-overs); every list entry checked, y on 48 sampled columns."""
+    wl = W.WORKLOADS["70b-reglu-fp16"].with_(sparsity=0.80)
+    assert pi.stack_launches(pi.desc_for(wl), 2, 2) == 1
+    rng = np.random.default_rng(80)
+    cols = np.sort(rng.choice(wl.d, size=48, replace=False)).astype(np.int32)
+    _, counts = _stack_check(wl, 2, 2, cols=cols, seed_step=2)
+    assert np.all(counts > 0.1 * wl.n_cold)
 
 
 @pytest.mark.parametrize("case", [(512, 900, 60, 32, "reglu", "f16", "f16", 1),

@@ -76,8 +76,11 @@ def test_reference_arm_prints_the_contract_line_on_rank_zero():
     describes the run and an e2e object with no host-device bytes."""
     import json
     env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    # the 7B-shaped workload keeps this CPU test within seconds (the default,
+    # 70B-shaped, generates 1.5 GB layers)
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
-                        "--warmup", "0"], env=env, capture_output=True, text=True, timeout=600)
+                        "--warmup", "0", "--workload", "7b-reglu-fp16"], env=env, capture_output=True, text=True,
+                       timeout=600)
     assert r.returncode == 0, r.stderr
     lines = [l for l in r.stdout.splitlines() if l.strip()]
     assert len(lines) == 1
