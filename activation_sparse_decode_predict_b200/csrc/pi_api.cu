@@ -12,6 +12,7 @@
 #include "pi_kernels_v1.cuh"
 #include "pi_layout.h"
 #include "pi_stack.cuh"
+#include "pi_tc.cuh"
 
 namespace {
 
@@ -140,6 +141,14 @@ pi_status ffn_impl(const pi_ffn_desc* d, int32_t B, const void* h, const int32_t
   float* a = reinterpret_cast<float*>(ws + L.act);
   float* partial = reinterpret_cast<float*>(ws + L.partial);
   const int sms = sm_count();
+  if (pi::kTcFfn && pi::tc_ffn_supported(d->wtype, d->ptype, d->d, B)) {
+    // token blocks of 3..16 with fp16 weights: gathered tiles on tcgen05, fp32
+    // accumulators in tensor memory, y (with b2) written by the last kernel
+    PI_CUDA(pi::launch_tc_ffn(d->act, h, B, d->d, d->ffn, d->n_hot, idx, count, Wg.data, Wu.data, Wd.data, b1, b2, y,
+                              ws + L.tc, reinterpret_cast<pi::Ctrl*>(ws), sms, st),
+            "tcgen05 FFN launch");
+    return PI_OK;
+  }
   if (pi::batch_supported(d->wtype, d->ptype, d->d, B)) {
     // token blocks of 3..16 with fp16 weights: tensor-core gate/up and down
     const int NR = pi::batch_ranges(d->d, sms);
@@ -199,7 +208,7 @@ pi_status fused_params(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, pi:
   P.act = desc->act;
   P.L = n_layers;
   P.T = desc->d / pi::stack_ept(desc->d);
-  smem = pi::stack_smem_layout(P, B, G);
+  smem = pi::stack_smem_layout(P, desc->ptype, B, G);
   if (smem == 0) return PI_ERR_UNSUPPORTED;
   const int ep = desc->ptype == PI_F16 ? 2 : 4;
   const size_t wrow = desc->wtype == PI_Q4_0 ? desc->d / 2 + desc->d / 16
@@ -226,7 +235,12 @@ pi_status fused_params(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, pi:
   {
     // a consumer holds one group while it waits for the first item of the next
     // one, and a wrap of the ring can waste up to one item: ng + 2 items fit
-    const int cap = pi::kNgFull ? (int)((size_t)P.ring_bytes / neuron) - 2 : (int)(half / neuron);
+    int cap = pi::kNgFull ? (int)((size_t)P.ring_bytes / neuron) - 2 : (int)(half / neuron);
+    if (pi::kNgInflight > 0) {
+      // leave kNgInflight items streaming while a group is held
+      const int inflight_cap = (int)((size_t)P.ring_bytes / neuron) - pi::kNgInflight;
+      cap = inflight_cap > 1 ? inflight_cap : 1;
+    }
     const int lim = (desc->wtype == PI_F16 && desc->ptype == PI_F16 && pi::kF16Mma) ? 16 / rpn : 4;
     P.ng = cap < lim ? cap : lim;
     if (P.ng < 1) P.ng = 1;
@@ -441,8 +455,20 @@ int32_t pi_stack_launches(const pi_ffn_desc* desc, int32_t batch, int32_t n_laye
     int G = 0;
     if (fused_params(desc, batch, n_layers, P, smem, G) == PI_OK) return 1;
   }
-  const int per_layer = desc->ffn > desc->n_hot ? 7 : 5;  // predictor (3 or 1 + memset), FFN (3), glue (1)
-  return per_layer * n_layers;
+  // the per-layer path: the kernels predict_impl, ffn_impl and the glue launch
+  // (memsets are not kernels)
+  const bool cold = desc->ffn > desc->n_hot;
+  int pred;
+  if (pi::batch_pred_supported(desc->ptype, desc->d, desc->rank, batch))
+    pred = cold ? 4 : 1;  // P1 and P2 row dots, threshold, compaction
+  else
+    pred = cold ? 3 : 1;  // u, scores, compaction
+  int ffn;
+  if (pi::kTcFfn && pi::tc_ffn_supported(desc->wtype, desc->ptype, desc->d, batch))
+    ffn = 4;  // up, activations, down, reduce
+  else
+    ffn = 3;  // gate/up (or row dots), down, reduce
+  return (pred + ffn + 1) * n_layers;
 }
 
 pi_status pi_get_device_status(void* ws, int32_t* status_out, int32_t clear, void* stream) {

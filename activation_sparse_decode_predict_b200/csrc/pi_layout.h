@@ -6,6 +6,7 @@
 //   [y accumulators][list counts: 128 x G_MAX][handed-over cold rows: 128 x C]
 //   [pre-activations of the tensor-core token-block path: 4 x (ffn + 16) x 2 x B fp32,
 //    token blocks of 3 or more only]
+//   [scratch of the tcgen05 token-block FFN (tc_ws_bytes), token blocks of 3 or more only]
 //
 // Every region starts on a 256-byte boundary.  The layout depends only on the
 // descriptor and the batch, never on the device.
@@ -14,6 +15,9 @@
 #include <stdint.h>
 
 namespace pi {
+
+// workspace bytes of the tcgen05 token-block FFN (pi_tc.cu)
+size_t tc_ws_bytes(int d, int ffn, int B);
 
 constexpr int kGMax = 296;  // split-K partial slots (2 x 148 SMs)
 #ifndef PI_YCOPIES
@@ -24,7 +28,7 @@ constexpr int kLayersMax = 128;  // layers of one decode-stack call
 constexpr size_t kCtrlBytes = 2304;  // the control block at the start of a workspace
 
 struct WsLayout {
-  size_t u, tile_mask, tile_count, act, partial, ybuf, hbuf, yacc, lcnt, don, pre, total;
+  size_t u, tile_mask, tile_count, act, partial, ybuf, hbuf, yacc, lcnt, don, pre, tc, total;
   int n_tiles, g_max;
 };
 
@@ -47,6 +51,7 @@ inline WsLayout ws_layout(int d, int ffn, int n_hot, int rank, int B) {
   L.lcnt = off; off += align256((size_t)kLayersMax * kGMax * 4);
   L.don = off; off += align256((size_t)kLayersMax * (C > 0 ? C : 1) * 4);
   L.pre = off; off += B >= 3 ? align256((size_t)4 * ((ffn + 17) & ~1) * 2 * B * 4) : 0;
+  L.tc = off; off += B >= 3 ? align256(tc_ws_bytes(d, ffn, B)) : 0;
   L.total = off;
   return L;
 }

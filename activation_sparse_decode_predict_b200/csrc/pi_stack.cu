@@ -215,7 +215,7 @@ struct Smem {
   float* bp;
   int* cidx;         // this CTA's predicted-active cold rows (neuron ids), ascending
   uint8_t* act;
-  float* sc;  // partial P2 scores [rows][B]
+  float* sc;         // partial P2 scores [k-part][rows][B]
   float* red;        // [2][NW][2B]
   float* gred;       // [kMaxGroup][NW][2B] per-warp gate/up dots (CUDA-core groups)
   int* misc;         // [0] local cold count, [1] barrier base, [2] next group size, [3] scratch
@@ -488,6 +488,9 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
   const int gated = p.act == kReglu;
   const int ep = PT == kF16 ? 2 : 4;
   constexpr int K = kYCopies;
+  // the fp16 token rows in shared memory feed only the tensor-core P1 (token
+  // blocks of 2) and tensor-core neuron groups; otherwise they take no space
+  constexpr bool kTokRows = stack_token_rows(PT, B);
 
   if (threadIdx.x == 0) {
     for (int q = 0; q < kNQ; ++q) {
@@ -713,9 +716,11 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
   }
   const int HS = 2 * d + 16;  // byte stride of the fp16 token rows in shared memory
   const int US = 2 * r + 16;  // byte stride of the fp16 u rows
-  if constexpr (PT == kF16) {
+  if constexpr (kTokRows) {
 #pragma unroll
     for (int b = 0; b < B; ++b) store_vals<WT, EPT, kF16>(s.hb + b * HS, t, T, h[b]);
+  }
+  if constexpr (PT == kF16) {
     if (t < 4) reinterpret_cast<uint32_t*>(s.zero)[t] = 0u;
   }
   const int ybuf4 = K * B * d / 4;  // float4s per accumulator buffer (K copies)
@@ -1022,10 +1027,7 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
     // the static hot neurons need no predictor: they fill the wait for barrier U
     if (!run_stream()) return;
     if (t == 0) PI_STAMP(l, 2);
-    if constexpr (PT == kF16) {
-      for (int x = t; x < (c1 - c0) * B; x += T) s.sc[x] = 0.f;  // partial scores accumulate here
-    }
-    {
+      {
       // barrier U has passed and u is staged (the barrier warp's signal)
       const bool okw = mbar_wait(s.u_ready, l & 1, ctrl);
       if (named_sync_or(1, T, !okw)) return;
@@ -1051,7 +1053,9 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
       const int KS = r / 16;
       int KQ = ntile > 0 ? (2 * NW + ntile - 1) / ntile : 1;
       if (KQ > KS / 4) KQ = KS / 4;
+      if (KQ > kMaxKQ) KQ = kMaxKQ;
       if (KQ < 1) KQ = 1;
+      const int cap = p.seg_cap;  // rows per k-part slot of the partial scores
       int released = 0;  // P2 tiles this warp has released; a tile is released once the warp is past it
       for (int un = warp; un < ntile * KQ; un += NW) {
         const int it = un / KQ, kq = un % KQ;
@@ -1081,11 +1085,14 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
           ldsm_x2(b_base + b_step * ks, b0, b1);
           mma_16816(acc0, a0, a1, a2, a3, b0, b1);
         }
-        // thread (g, t4): rows g and g+8, columns 2*t4 (hi) and 2*t4+1 (lo) = token t4
+        // thread (g, t4): rows g and g+8, columns 2*t4 (hi) and 2*t4+1 (lo) = token t4;
+        // each k-part has its own slot, summed in k-part order below, so the
+        // scores do not depend on which warp finished first
         const int g = lane >> 2, t4 = lane & 3;
         if (t4 < B) {
-          if (g < rows) atomicAdd(&s.sc[(16 * it + g) * B + t4], (acc0[0] + acc1[0]) + (acc0[1] + acc1[1]));
-          if (g + 8 < rows) atomicAdd(&s.sc[(16 * it + g + 8) * B + t4], (acc0[2] + acc1[2]) + (acc0[3] + acc1[3]));
+          float* slot = s.sc + (size_t)kq * cap * B;
+          if (g < rows) slot[(16 * it + g) * B + t4] = (acc0[0] + acc1[0]) + (acc0[1] + acc1[1]);
+          if (g + 8 < rows) slot[(16 * it + g + 8) * B + t4] = (acc0[2] + acc1[2]) + (acc0[3] + acc1[3]);
         }
       }
       for (; released < ntile; ++released) release_item();
@@ -1093,7 +1100,11 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
       for (int x = t; x < nrows; x += T) {
         bool on = false;
 #pragma unroll
-        for (int b = 0; b < B; ++b) on |= (s.sc[x * B + b] + s.bp[x]) > Ly.thr;
+        for (int b = 0; b < B; ++b) {
+          float sc = 0.f;
+          for (int q = 0; q < KQ; ++q) sc += s.sc[((size_t)q * cap + x) * B + b];
+          on |= (sc + s.bp[x]) > Ly.thr;
+        }
         s.act[x] = on ? 1 : 0;
       }
       witem += ntile;
@@ -1292,7 +1303,7 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
 #pragma unroll
         for (int e = 0; e < EPT; ++e) h[b][e] = round_to(PT, h[b][e] * inv);
       }
-      if constexpr (PT == kF16) {
+      if constexpr (kTokRows) {
 #pragma unroll
         for (int b = 0; b < B; ++b) store_vals<WT, EPT, kF16>(s.hb + b * HS, t, T, h[b]);
       }
@@ -1433,7 +1444,7 @@ bool stack_supported(int wtype, int ptype, int d, int ffn, int n_hot, int rank, 
   return true;
 }
 
-size_t stack_smem_layout(StackParams& p, int B, int G) {
+size_t stack_smem_layout(StackParams& p, int ptype, int B, int G) {
   const int C = p.ffn - p.n_hot;
   const int share_cap = (C + G - 1) / G + 1;
   size_t off = 0;
@@ -1446,18 +1457,18 @@ size_t stack_smem_layout(StackParams& p, int B, int G) {
   const size_t sizes[] = {
       sizeof(uint64_t) * (2 * kNQ + 3),                                        // bars
       sizeof(uint32_t) * 4 * kNQ,                                              // item offsets, starts, rows, groups
-      sizeof(float) * (size_t)B * p.rank,                                      // u
+      ptype == kF32 ? sizeof(float) * (size_t)B * p.rank : 0,                  // u (fp32 predictors)
       sizeof(float) * share_cap,                                               // bp
       sizeof(int) * share_cap,                                                 // cidx
       (size_t)share_cap,                                                       // act
-      sizeof(float) * share_cap * B,                                           // sc
+      sizeof(float) * share_cap * B * kMaxKQ,                                  // sc (one slot per k-part)
       sizeof(float) * 2 * (kMaxConsumers / 32) * 6 * B,                        // red
       sizeof(float) * (kMaxGroup * (kMaxConsumers / 32) * 2 * B + kMaxGroup * B),  // gred + group activations
       sizeof(int) * 4,                                                         // misc
-      (size_t)B * (2 * p.d + 16),                                              // hb
-      (size_t)2 * B * (2 * p.rank + 16),                                       // ub
+      stack_token_rows(ptype, B) ? (size_t)B * (2 * p.d + 16) : 0,             // hb
+      ptype == kF16 ? (size_t)2 * B * (2 * p.rank + 16) : 0,                   // ub (fp16 predictors)
       16,                                                                      // zero
-      sizeof(float) * (kMaxConsumers / 32) * 32,                               // redp
+      stack_token_rows(ptype, B) ? sizeof(float) * (kMaxConsumers / 32) * 32 : 0,  // redp
   };
   size_t fixed = 0;
   for (size_t b : sizes) fixed += (b + 127) & ~(size_t)127;

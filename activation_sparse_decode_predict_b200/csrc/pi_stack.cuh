@@ -54,9 +54,14 @@ constexpr bool kMmaX2 = PI_MMA_X2 != 0;    // load only tile rows 0-7 when a gro
 #ifndef PI_NG_FULL
 #define PI_NG_FULL 0
 #endif
-constexpr int kNgFull = PI_NG_FULL;  // 1: groups may fill the ring but one item (else half the ring)
+constexpr int kNgFull = PI_NG_FULL;
+#ifndef PI_NG_INFLIGHT
+#define PI_NG_INFLIGHT 0
+#endif
+constexpr int kNgInflight = PI_NG_INFLIGHT;  // > 0: groups leave this many ring items streaming  // 1: groups may fill the ring but one item (else half the ring)
 constexpr int kGMaxCtas = 296;       // largest grid (2 x 148)
 constexpr int kShareRegs = 2;
+constexpr int kMaxKQ = 4;          // k-parts of a P2 tile at most (each has its own score slot)
 constexpr int kMaxGroup = 16;       // neurons per group at most        // per-thread registers for the CTA's bias shares
 
 // One layer's device pointers (a copy of pi_layer_weights).
@@ -106,12 +111,19 @@ struct StackParams {
   StackLayer layers[kMaxLayers];
 };
 
+// Whether the kernel keeps the token block as fp16 rows in shared memory (the
+// tensor-core operand of the P1 dots of a token block of 2, or of tensor-core
+// neuron groups).
+__host__ __device__ constexpr bool stack_token_rows(int ptype, int B) {
+  return ptype == kF16 && (B > 1 || kP1Mma || kF16Mma);
+}
+
 // Columns of d each consumer thread owns (8 when d/8 threads fit, else 16).
 int stack_ept(int d);
 bool stack_supported(int wtype, int ptype, int d, int ffn, int n_hot, int rank, int B, int L);
 // Fills the shared-memory offsets of p (needs d, ffn, n_hot, rank); returns the
 // dynamic shared memory size, or 0 if it does not fit.
-size_t stack_smem_layout(StackParams& p, int B, int G);
+size_t stack_smem_layout(StackParams& p, int ptype, int B, int G);
 cudaError_t launch_stack(int wtype, int ptype, int B, const StackParams& p, int G, size_t smem, cudaStream_t st);
 
 }  // namespace pi

@@ -1,0 +1,670 @@
+// pi_tc.cu -- the sparse FFN of a token block of 3..16 tokens on the fifth-
+// generation tensor cores: tcgen05.mma with fp32 accumulators in tensor memory,
+// operands gathered into shared memory by TMA (fp16 weights and tokens).
+//
+// PowerInfer (unite.ai, "Nöron Bilinçli Operatör"; aibars.net,
+// "Sparsity-Nutzung"): only the rows of the hot neurons and of the
+// predicted-active cold neurons are read.  With several tokens in a block each
+// streamed row serves all of them, so the neuron-aware operator becomes a
+// product of gathered tiles:
+//
+//   up    D[128 listed neurons x 16 tokens] = W_rows[128 x d] . h^T[d x 16]
+//         (gate and up rows: two accumulators), tiles of 128 list positions
+//   down  D[128 output columns x 32] = W_downT^T[128 x listed] . A^T[listed x 32]
+//         where A holds each activation as an fp16 pair hi + lo (hi rows 0-15,
+//         lo rows 16-31), so the product keeps ~22 bits of the fp32 activation.
+//
+// Gathers: a 2-D tensor map over a weight matrix with a one-row box of 64
+// columns; tile::gather4 brings four arbitrary rows per instruction into a
+// 128-byte-swizzled operand tile (the swizzle follows the shared-memory
+// address, so a row may land at any row of an aligned 1024-byte atom).
+//
+// Work split, both kernels: a flat sequence of units (up: tile x 64-column
+// block of d; down: 256-column chunk of d x 64-position block of the list) is
+// cut into G contiguous ranges of equal length, one per CTA; a CTA accumulates
+// consecutive units of the same tile (chunk) in tensor memory and writes one
+// partial per (CTA, tile) segment.  Readers find the writers of a tile from
+// the same arithmetic, and sum them in CTA order: deterministic.
+//
+// Kernels per call: k_tc_up -> k_tc_act (sum of the up partials, bias,
+// activation, fp16 hi/lo rows) -> k_tc_down -> k_tc_reduce (+ b2).
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cstring>
+#include <mutex>
+
+#include "pi_common.cuh"
+#include "pi_sync.cuh"
+#include "pi_tc.cuh"
+
+namespace pi {
+
+namespace {
+
+constexpr int kTcThreads = 192;     // warp 0: TMA producer; warp 1: MMA issuer (owns tensor memory); 2-5: epilogue
+constexpr int kTcSlots = 8;         // up partials per tile at most
+constexpr int kChunk = 256;         // output columns per down chunk (two M = 128 products)
+constexpr int kUpStage = 35 * 1024;  // [gate 16 KB][up 16 KB][tokens 2 KB], 1024-aligned
+constexpr int kUpNS = 6;
+constexpr int kDnStage = 36 * 1024;  // [4 column blocks x 64 positions x 128 B = 32 KB][activations 32 x 128 B]
+constexpr int kDnNS = 6;
+constexpr int kBarBytes = 1024;      // mbarriers and the tensor-memory address, after the stages
+
+// ---------------------------------------------------------------------------
+// the flat unit sequence and its split into contiguous per-CTA ranges
+
+struct Split {
+  int64_t U;  // units
+  int G;      // CTAs that get a (non-empty) range
+};
+
+__device__ __forceinline__ int64_t range_lo(const Split& s, int c) { return s.U * c / s.G; }
+
+// CTA whose range holds unit u (0 <= u < U)
+__device__ __forceinline__ int range_owner(const Split& s, int64_t u) {
+  int c = (int)((u * s.G) / s.U);
+  while (c > 0 && range_lo(s, c) > u) --c;
+  while (c + 1 < s.G && range_lo(s, c + 1) <= u) ++c;
+  return c;
+}
+
+// the list length (hot rows + predicted) with the count clamped to [0, C]
+__device__ __forceinline__ int list_total(const int32_t* count, int n_hot, int ffn, Ctrl* ctrl, bool report) {
+  int cnt = *count;
+  const int C = ffn - n_hot;
+  if (cnt < 0 || cnt > C) {
+    if (report) set_status(&ctrl->status, kStCapacity);
+    cnt = cnt < 0 ? 0 : C;
+  }
+  return n_hot + cnt;
+}
+
+// up: units = 128-position tiles x 64-column blocks of d; every range holds at
+// least a quarter of a tile, so a tile has at most 5 writers
+__device__ __forceinline__ Split up_split(int ntot, int d, int G) {
+  const int KB = d / 64;
+  Split s;
+  s.U = (int64_t)((ntot + 127) / 128) * KB;
+  const int64_t per = KB / 4 > 0 ? KB / 4 : 1;
+  const int64_t g = s.U / per;
+  s.G = g < G ? (g > 0 ? (int)g : 1) : G;
+  return s;
+}
+
+// down: units = 256-column chunks of d x 64-position blocks of the list;
+// d / 256 <= G, so a range spans at most two chunks
+__device__ __forceinline__ Split down_split(int ntot, int d, int G) {
+  const int KBp = (ntot + 63) / 64;
+  Split s;
+  s.U = (int64_t)(d / kChunk) * KBp;
+  s.G = s.U < G ? (s.U > 0 ? (int)s.U : 1) : G;
+  return s;
+}
+
+// storage row of list position pos (hot rows first); an entry outside
+// [n_hot, ffn) is reported and replaced by row 0
+__device__ __forceinline__ int list_row_at(int pos, int ntot, int n_hot, int ffn, const int32_t* idx, Ctrl* ctrl) {
+  if (pos < n_hot) return pos;
+  if (pos >= ntot) return 0;  // beyond the list: any valid row, its products are dropped or multiplied by zero
+  const int j = __ldg(idx + (pos - n_hot));
+  if (j < n_hot || j >= ffn) {
+    set_status(&ctrl->status, kStIndex);
+    return 0;
+  }
+  return j;
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  const uint32_t a = smem_u32(p);
+  return p + ((1024u - (a & 1023u)) & 1023u);
+}
+
+// ---------------------------------------------------------------------------
+// up: gate/up dots of 128-neuron tiles -> pre[slot][pos][2][16]
+
+struct TcUpParams {
+  CUtensorMap tm_h;   // token block [B, d] fp16; box 64 x 16 (rows past B read as zero)
+  CUtensorMap tm_w0;  // gate rows (ReGLU) or up rows [F, d] fp16; box 64 x 1
+  CUtensorMap tm_w1;  // up rows (ReGLU); box 64 x 1
+  const int32_t* idx;
+  const int32_t* count;
+  float* pre;  // [kTcSlots][ffn][2][16]
+  Ctrl* ctrl;
+  int d, ffn, n_hot, gated;
+};
+
+__global__ void __launch_bounds__(kTcThreads, 1) k_tc_up(const __grid_constant__ TcUpParams p) {
+  extern __shared__ uint8_t smraw[];
+  uint8_t* sm = align1024(smraw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + kUpNS * kUpStage);
+  uint64_t* empty = full + kUpNS;
+  uint64_t* accf = empty + kUpNS;  // [2] accumulators ready
+  uint64_t* acce = accf + 2;       // [2] accumulators drained
+  uint64_t* done = acce + 2;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
+  Ctrl* ctrl = p.ctrl;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x;
+  const int ntot = list_total(p.count, p.n_hot, p.ffn, ctrl, c == 0 && threadIdx.x == 0);
+  const int KB = p.d / 64;
+  const Split sp = up_split(ntot, p.d, gridDim.x);
+  const int64_t u0 = c < sp.G ? range_lo(sp, c) : 0, u1 = c < sp.G ? range_lo(sp, c + 1) : 0;
+  const int nmat = p.gated ? 2 : 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kUpNS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accf[b], 1);
+      mbar_init(&acce[b], 4);
+    }
+    mbar_init(done, 1);
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tslot, 64);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+
+  if (warp == 0) {
+    // ---------------- TMA producer: lane l gathers list positions 4l..4l+3 of the tile ----------------
+    int r[4] = {0, 0, 0, 0};
+    int cur = -1;
+    int64_t issued = 0;
+    bool ok = true;
+    for (int64_t u = u0; u < u1 && ok; ++u) {
+      const int it = (int)(u - u0), s = it % kUpNS;
+      const int tile = (int)(u / KB), kb = (int)(u % KB);
+      if (tile != cur) {
+        cur = tile;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) r[i] = list_row_at(tile * 128 + 4 * lane + i, ntot, p.n_hot, p.ffn, p.idx, ctrl);
+      }
+      if (it >= kUpNS) ok = mbar_wait(&empty[s], ((it / kUpNS) - 1) & 1, ctrl);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(nmat * 16384 + 2048));
+      __syncwarp();
+      uint8_t* st = sm + s * kUpStage;
+      const int x = kb * 64;
+      tma_gather4(st + lane * 512, &p.tm_w0, x, r[0], r[1], r[2], r[3], &full[s]);
+      if (p.gated) tma_gather4(st + 16384 + lane * 512, &p.tm_w1, x, r[0], r[1], r[2], r[3], &full[s]);
+      if (lane == 0) tma_load_2d(st + 32768, &p.tm_h, x, 0, &full[s]);
+      ++issued;
+    }
+    // the CTA leaves only once every issued stage has landed
+    if (lane == 0)
+      for (int64_t it = issued > kUpNS ? issued - kUpNS : 0; it < issued; ++it)
+        mbar_wait(&full[it % kUpNS], (uint32_t)((it / kUpNS) & 1), ctrl);
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16(128, 16, 0, 0);
+      int buf = 0, nseg = 0, cur = -1;
+      bool ok = true;
+      for (int64_t u = u0; u < u1; ++u) {
+        const int it = (int)(u - u0), s = it % kUpNS;
+        const int tile = (int)(u / KB);
+        const bool first = tile != cur;
+        const bool last = (u + 1 == u1) || ((u + 1) / KB != tile);
+        if (first) {
+          cur = tile;
+          // this accumulator buffer was last used two segments ago: wait until it is drained
+          if (nseg >= 2) ok = mbar_wait(&acce[buf], (uint32_t)(((nseg - 2) / 2) & 1), ctrl);
+        }
+        if (ok) ok = mbar_wait(&full[s], (uint32_t)((it / kUpNS) & 1), ctrl);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t st = smem_u32(sm + s * kUpStage);
+        const uint32_t dg = tmem + (uint32_t)(buf * 32);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t bd = sw128_desc(st + 32768 + kk * 32, 16, 1024);
+          const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+          tc_mma_f16(dg, sw128_desc(st + kk * 32, 16, 1024), bd, idesc, acc);
+          if (p.gated) tc_mma_f16(dg + 16, sw128_desc(st + 16384 + kk * 32, 16, 1024), bd, idesc, acc);
+        }
+        tc_commit(&empty[s]);
+        if (last) {
+          tc_commit(&accf[buf]);
+          buf ^= 1;
+          ++nseg;
+        }
+      }
+      // every MMA of this thread has completed before tensor memory is freed
+      tc_commit(done);
+      mbar_wait(done, 0, ctrl);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue: warp quarter q reads tensor-memory lanes 32q..32q+31 ----------------
+    const int q = warp & 3;
+    int buf = 0, nseg = 0, cur = -1;
+    for (int64_t u = u0; u < u1; ++u) {
+      const int tile = (int)(u / KB);
+      if (tile != cur) cur = tile;
+      const bool last = (u + 1 == u1) || ((u + 1) / KB != tile);
+      if (!last) continue;
+      if (!mbar_wait(&accf[buf], (uint32_t)((nseg / 2) & 1), ctrl)) break;
+      tc_fence_after();
+      float g[16], v[16];
+      const uint32_t ta = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * 32);
+      tmem_ld16(ta, g);
+      if (p.gated) tmem_ld16(ta + 16, v);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce[buf]);
+      const int pos = tile * 128 + q * 32 + lane;
+      const int slot = c - range_owner(sp, (int64_t)tile * KB);
+      if (slot >= kTcSlots) {
+        set_status(&ctrl->status, kStCapacity);
+      } else if (pos < ntot) {
+        float4* dst = reinterpret_cast<float4*>(p.pre + (((size_t)slot * p.ffn + pos) * 2) * 16);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[i] = make_float4(g[4 * i], g[4 * i + 1], g[4 * i + 2], g[4 * i + 3]);
+        if (p.gated) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[4 + i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+      }
+      buf ^= 1;
+      ++nseg;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// activations: sum of a tile's up partials (in CTA order) + b1, activation,
+// fp16 hi/lo rows act16[32][fpad] (hi: rows 0-15, lo: rows 16-31; zero for
+// tokens past B and positions past the list up to the next 64)
+
+struct TcActParams {
+  const float* pre;
+  const float* b1;
+  __half* act16;
+  const int32_t* idx;
+  const int32_t* count;
+  Ctrl* ctrl;
+  int d, ffn, n_hot, act, gated, B, fpad, G;
+};
+
+__global__ void __launch_bounds__(128) k_tc_act(const TcActParams p) {
+  const int pos = blockIdx.x * blockDim.x + threadIdx.x;
+  const int ntot = list_total(p.count, p.n_hot, p.ffn, p.ctrl, false);
+  if (pos >= ((ntot + 63) & ~63) || pos >= p.fpad) return;
+  float a[16];
+#pragma unroll
+  for (int b = 0; b < 16; ++b) a[b] = 0.f;
+  if (pos < ntot) {
+    const int KB = p.d / 64;
+    const Split sp = up_split(ntot, p.d, p.G);
+    const int tile = pos / 128;
+    const int c_lo = range_owner(sp, (int64_t)tile * KB), c_hi = range_owner(sp, (int64_t)tile * KB + KB - 1);
+    float g[16], v[16];
+#pragma unroll
+    for (int b = 0; b < 16; ++b) g[b] = v[b] = 0.f;
+    for (int slot = 0; slot <= c_hi - c_lo && slot < kTcSlots; ++slot) {
+      const float4* src = reinterpret_cast<const float4*>(p.pre + (((size_t)slot * p.ffn + pos) * 2) * 16);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 x = __ldcg(src + i);
+        g[4 * i] += x.x; g[4 * i + 1] += x.y; g[4 * i + 2] += x.z; g[4 * i + 3] += x.w;
+      }
+      if (p.gated) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4 x = __ldcg(src + 4 + i);
+          v[4 * i] += x.x; v[4 * i + 1] += x.y; v[4 * i + 2] += x.z; v[4 * i + 3] += x.w;
+        }
+      }
+    }
+    const int row = list_row_at(pos, ntot, p.n_hot, p.ffn, p.idx, p.ctrl);
+    const float bias = p.b1 ? __ldg(p.b1 + row) : 0.f;
+#pragma unroll
+    for (int b = 0; b < 16; ++b)
+      if (b < p.B) a[b] = p.gated ? act_eval(kReglu, g[b] + bias, v[b]) : act_eval(p.act, g[b] + bias, 0.f);
+  }
+#pragma unroll
+  for (int b = 0; b < 16; ++b) {
+    const __half hi = __float2half_rn(a[b]);
+    const __half lo = __float2half_rn(a[b] - __half2float(hi));
+    p.act16[(size_t)b * p.fpad + pos] = hi;
+    p.act16[(size_t)(16 + b) * p.fpad + pos] = lo;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// down: partial outputs of 256-column chunks -> part[cta][segment][16][256]
+
+struct TcDownParams {
+  CUtensorMap tm_wd;   // W_downT [F, d] fp16; box 64 x 1
+  CUtensorMap tm_act;  // act16 [32, fpad] fp16; box 64 x 32
+  const int32_t* idx;
+  const int32_t* count;
+  float* part;  // [G][2][16][kChunk]
+  Ctrl* ctrl;
+  int d, ffn, n_hot;
+};
+
+__global__ void __launch_bounds__(kTcThreads, 1) k_tc_down(const __grid_constant__ TcDownParams p) {
+  extern __shared__ uint8_t smraw[];
+  uint8_t* sm = align1024(smraw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + kDnNS * kDnStage);
+  uint64_t* empty = full + kDnNS;
+  uint64_t* accf = empty + kDnNS;
+  uint64_t* acce = accf + 2;
+  uint64_t* done = acce + 2;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
+  Ctrl* ctrl = p.ctrl;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x;
+  const int ntot = list_total(p.count, p.n_hot, p.ffn, ctrl, false);
+  const int KBp = (ntot + 63) / 64;
+  const Split sp = down_split(ntot, p.d, gridDim.x);
+  const int64_t u0 = c < sp.G ? range_lo(sp, c) : 0, u1 = c < sp.G ? range_lo(sp, c + 1) : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDnNS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accf[b], 1);
+      mbar_init(&acce[b], 4);
+    }
+    mbar_init(done, 1);
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tslot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+
+  if (warp == 0) {
+    // ---------------- TMA producer: lane l gathers positions 4(l%16)..+3 for column blocks 2(l/16), 2(l/16)+1 ----------------
+    int64_t issued = 0;
+    bool ok = true;
+    for (int64_t u = u0; u < u1 && ok; ++u) {
+      const int it = (int)(u - u0), s = it % kDnNS;
+      const int chunk = (int)(u / KBp), kb = (int)(u % KBp);
+      int r[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) r[i] = list_row_at(kb * 64 + 4 * (lane & 15) + i, ntot, p.n_hot, p.ffn, p.idx, ctrl);
+      if (it >= kDnNS) ok = mbar_wait(&empty[s], ((it / kDnNS) - 1) & 1, ctrl);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], 32768u + 4096u);
+      __syncwarp();
+      uint8_t* st = sm + s * kDnStage;
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int cb = 2 * (lane >> 4) + h2;
+        tma_gather4(st + cb * 8192 + 4 * (lane & 15) * 128, &p.tm_wd, chunk * kChunk + cb * 64, r[0], r[1], r[2], r[3],
+                    &full[s]);
+      }
+      if (lane == 0) tma_load_2d(st + 32768, &p.tm_act, kb * 64, 0, &full[s]);
+      ++issued;
+    }
+    if (lane == 0)
+      for (int64_t it = issued > kDnNS ? issued - kDnNS : 0; it < issued; ++it)
+        mbar_wait(&full[it % kDnNS], (uint32_t)((it / kDnNS) & 1), ctrl);
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16(128, 32, 1, 0);
+      int buf = 0, nseg = 0, cur = -1;
+      bool ok = true;
+      for (int64_t u = u0; u < u1; ++u) {
+        const int it = (int)(u - u0), s = it % kDnNS;
+        const int chunk = (int)(u / KBp);
+        const bool first = chunk != cur;
+        const bool last = (u + 1 == u1) || ((u + 1) / KBp != chunk);
+        if (first) {
+          cur = chunk;
+          if (nseg >= 2) ok = mbar_wait(&acce[buf], (uint32_t)(((nseg - 2) / 2) & 1), ctrl);
+        }
+        if (ok) ok = mbar_wait(&full[s], (uint32_t)((it / kDnNS) & 1), ctrl);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t st = smem_u32(sm + s * kDnStage);
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            // A: MN-major, 64-column blocks 8 KB apart, 8-position groups 1 KB apart;
+            // k-step kk = positions 16kk..16kk+15
+            const uint64_t ad = sw128_desc(st + (2 * m) * 8192 + kk * 2048, 8192, 1024);
+            const uint64_t bd = sw128_desc(st + 32768 + kk * 32, 16, 1024);
+            tc_mma_f16(tmem + (uint32_t)(buf * 64 + m * 32), ad, bd, idesc, (first && kk == 0) ? 0u : 1u);
+          }
+        }
+        tc_commit(&empty[s]);
+        if (last) {
+          tc_commit(&accf[buf]);
+          buf ^= 1;
+          ++nseg;
+        }
+      }
+      tc_commit(done);
+      mbar_wait(done, 0, ctrl);
+    }
+    __syncwarp();
+  } else {
+    const int q = warp & 3;
+    int buf = 0, nseg = 0;
+    for (int64_t u = u0; u < u1; ++u) {
+      const int chunk = (int)(u / KBp);
+      const bool last = (u + 1 == u1) || ((u + 1) / KBp != chunk);
+      if (!last) continue;
+      if (!mbar_wait(&accf[buf], (uint32_t)((nseg / 2) & 1), ctrl)) break;
+      tc_fence_after();
+      float hv[2][16], lv[2][16];
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const uint32_t ta = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * 64 + m * 32);
+        tmem_ld16(ta, hv[m]);
+        tmem_ld16(ta + 16, lv[m]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce[buf]);
+      // segment 0: the chunk of this CTA's first unit; segment 1: the next one
+      const int seg = (u0 / KBp == chunk) ? 0 : 1;
+      float* dst = p.part + ((size_t)c * 2 + seg) * 16 * kChunk;
+#pragma unroll
+      for (int m = 0; m < 2; ++m)
+#pragma unroll
+        for (int b = 0; b < 16; ++b) dst[b * kChunk + m * 128 + q * 32 + lane] = hv[m][b] + lv[m][b];
+      buf ^= 1;
+      ++nseg;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// y[b, col] = b2[col] + sum over the chunk's writers (CTA order) of their partials
+__global__ void __launch_bounds__(256) k_tc_reduce(const float* __restrict__ part, const int32_t* count, int n_hot,
+                                                   int ffn, int d, int B, int G, const float* __restrict__ b2,
+                                                   float* __restrict__ y, Ctrl* ctrl) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= B * d) return;
+  const int b = i / d, col = i % d;
+  const int ntot = list_total(count, n_hot, ffn, ctrl, false);
+  const int KBp = (ntot + 63) / 64;
+  float acc = b2 ? __ldg(b2 + col) : 0.f;
+  if (KBp > 0) {
+    const Split sp = down_split(ntot, d, G);
+    const int chunk = col / kChunk;
+    const int c_lo = range_owner(sp, (int64_t)chunk * KBp), c_hi = range_owner(sp, (int64_t)chunk * KBp + KBp - 1);
+    for (int c = c_lo; c <= c_hi; ++c) {
+      const int64_t lo = range_lo(sp, c);
+      if (range_lo(sp, c + 1) == lo) continue;  // an empty range wrote nothing
+      const int seg = (lo / KBp == chunk) ? 0 : 1;
+      acc += __ldcg(part + (((size_t)c * 2 + seg) * 16 + b) * kChunk + (col % kChunk));
+    }
+  }
+  y[i] = acc;
+}
+
+// ---------------------------------------------------------------------------
+// host: tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D fp16 tensor [rows, cols] (row pitch `pitch` bytes), box box_cols x box_rows, 128-byte swizzle
+cudaError_t make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t pitch, uint32_t box_cols,
+                     uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;  // no driver entry point: the launch fails with PI_ERR_CUDA
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {pitch};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+int tc_fpad(int ffn) { return (ffn + 63) & ~63; }
+
+struct TcScratch {
+  float* pre;
+  __half* act16;
+  float* part;
+};
+
+TcScratch tc_carve(void* scratch, int ffn) {
+  TcScratch s;
+  char* b = static_cast<char*>(scratch);
+  s.pre = reinterpret_cast<float*>(b);
+  b += ((size_t)kTcSlots * ffn * 2 * 16 * 4 + 1023) & ~(size_t)1023;
+  s.act16 = reinterpret_cast<__half*>(b);
+  b += ((size_t)32 * tc_fpad(ffn) * 2 + 1023) & ~(size_t)1023;
+  s.part = reinterpret_cast<float*>(b);
+  return s;
+}
+
+}  // namespace
+
+bool tc_ffn_supported(int wtype, int ptype, int d, int B) {
+  if (wtype != kF16 || ptype != kF16) return false;
+  if (B < 3 || B > 16) return false;
+  return d % kChunk == 0 && d / kChunk <= 148;
+}
+
+size_t tc_ws_bytes(int d, int ffn, int B) {
+  (void)d;
+  (void)B;
+  size_t n = ((size_t)kTcSlots * ffn * 2 * 16 * 4 + 1023) & ~(size_t)1023;
+  n += ((size_t)32 * tc_fpad(ffn) * 2 + 1023) & ~(size_t)1023;
+  n += (size_t)296 * 2 * 16 * kChunk * 4;
+  return n;
+}
+
+cudaError_t launch_tc_ffn(int act, const void* h, int B, int d, int ffn, int n_hot, const int32_t* idx,
+                          const int32_t* count, const void* wg, const void* wu, const void* wd, const float* b1,
+                          const float* b2, float* y, void* scratch, Ctrl* ctrl, int sms, cudaStream_t st) {
+  const int G = sms < 296 ? sms : 296;
+  const int gated = act == kReglu;
+  const TcScratch S = tc_carve(scratch, ffn);
+  const int fpad = tc_fpad(ffn);
+  cudaError_t e;
+
+  TcUpParams U;
+  memset(&U, 0, sizeof(U));
+  if ((e = make_map(&U.tm_h, h, d, B, (uint64_t)d * 2, 64, 16)) != cudaSuccess) return e;
+  if ((e = make_map(&U.tm_w0, gated ? wg : wu, d, ffn, (uint64_t)d * 2, 64, 1)) != cudaSuccess) return e;
+  if ((e = make_map(&U.tm_w1, wu, d, ffn, (uint64_t)d * 2, 64, 1)) != cudaSuccess) return e;
+  U.idx = idx;
+  U.count = count;
+  U.pre = S.pre;
+  U.ctrl = ctrl;
+  U.d = d;
+  U.ffn = ffn;
+  U.n_hot = n_hot;
+  U.gated = gated;
+  const int up_smem = kUpNS * kUpStage + kBarBytes + 1024;
+  if ((e = cudaFuncSetAttribute(k_tc_up, cudaFuncAttributeMaxDynamicSharedMemorySize, up_smem)) != cudaSuccess)
+    return e;
+  k_tc_up<<<G, kTcThreads, up_smem, st>>>(U);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  TcActParams A;
+  A.pre = S.pre;
+  A.b1 = b1;
+  A.act16 = S.act16;
+  A.idx = idx;
+  A.count = count;
+  A.ctrl = ctrl;
+  A.d = d;
+  A.ffn = ffn;
+  A.n_hot = n_hot;
+  A.act = act;
+  A.gated = gated;
+  A.B = B;
+  A.fpad = fpad;
+  A.G = G;
+  k_tc_act<<<(fpad + 127) / 128, 128, 0, st>>>(A);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  TcDownParams D;
+  memset(&D, 0, sizeof(D));
+  if ((e = make_map(&D.tm_wd, wd, d, ffn, (uint64_t)d * 2, 64, 1)) != cudaSuccess) return e;
+  if ((e = make_map(&D.tm_act, S.act16, fpad, 32, (uint64_t)fpad * 2, 64, 32)) != cudaSuccess) return e;
+  D.idx = idx;
+  D.count = count;
+  D.part = S.part;
+  D.ctrl = ctrl;
+  D.d = d;
+  D.ffn = ffn;
+  D.n_hot = n_hot;
+  const int dn_smem = kDnNS * kDnStage + kBarBytes + 1024;
+  if ((e = cudaFuncSetAttribute(k_tc_down, cudaFuncAttributeMaxDynamicSharedMemorySize, dn_smem)) != cudaSuccess)
+    return e;
+  k_tc_down<<<G, kTcThreads, dn_smem, st>>>(D);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  k_tc_reduce<<<(B * d + 255) / 256, 256, 0, st>>>(S.part, count, n_hot, ffn, d, B, G, b2, y, ctrl);
+  return cudaGetLastError();
+}
+
+}  // namespace pi

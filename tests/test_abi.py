@@ -109,20 +109,28 @@ def test_python_layer_refuses_cpu_tensors():
 
 def test_launch_plan_is_host_only():
     """pi_stack_launches plans a decode step without a GPU: one persistent
-    launch for token blocks of 1-2 on every workload shape, the per-layer
-    kernels (7 per layer; 5 with no cold neurons) for token blocks of 3-16 or
-    a shape the persistent kernel does not take, -1 for invalid arguments."""
+    launch for token blocks of 1-2 on every workload shape; for token blocks of
+    3-16 an fp16 predictor runs on the tensor cores (P1 and P2 row dots,
+    threshold, compaction), fp16 weights (d % 256 == 0) on the tcgen05 FFN
+    (up, activations, down, reduce), then the glue: 9 per layer (8 with Q4_0
+    weights, whose FFN runs on CUDA cores); a shape the
+    persistent kernel does not take runs the CUDA-core kernels (u, scores,
+    compaction; gate/up, down, reduce; glue: 7 per layer, 5 with no cold
+    neurons); -1 for invalid arguments."""
     import pi_workload as W
     lib = pi.lib()
     for w in W.WORKLOADS.values():
         desc = pi.desc_for(w)
         for batch in (1, 2):
             assert lib.pi_stack_launches(ctypes.byref(desc), batch, w.layers) == 1, (w.name, batch)
+        pred = 4 if w.ptype == "f16" else 3
+        ffn = 4 if (w.wtype == "f16" and w.ptype == "f16") else 3
         for batch in (3, 8, 16):
-            assert lib.pi_stack_launches(ctypes.byref(desc), batch, w.layers) == 7 * w.layers, (w.name, batch)
+            want = (pred + ffn + 1) * w.layers
+            assert lib.pi_stack_launches(ctypes.byref(desc), batch, w.layers) == want, (w.name, batch)
     odd = _desc(d=520, ffn=2048, n_hot=103, rank=64, act="relu")  # d not a multiple of 256
     assert lib.pi_stack_launches(ctypes.byref(odd), 1, 4) == 28
-    all_hot = _desc(d=512, ffn=2048, n_hot=2048, rank=64, act="relu")
+    all_hot = _desc(d=512, ffn=2048, n_hot=2048, rank=64, act="relu", wtype="f32", ptype="f32")
     assert lib.pi_stack_launches(ctypes.byref(all_hot), 3, 4) == 20
     assert lib.pi_stack_launches(ctypes.byref(_desc()), 1, 0) == -1
     assert lib.pi_stack_launches(ctypes.byref(_desc()), 0, 4) == -1
