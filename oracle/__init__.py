@@ -47,7 +47,7 @@ def _bind(path: str):
     lib.orc_half_to_double.restype = f64
     lib.orc_elem.argtypes = [i32, P, P, i64, i64, i64]
     lib.orc_elem.restype = f64
-    lib.orc_predict.argtypes = [i32, i32, i32, i32, i32, i32, i32, P, P, P, P, f64, P, P, P, P]
+    lib.orc_predict.argtypes = [i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, f64, P, P, P, P]
     lib.orc_predict.restype = i64
     lib.orc_masked_ffn.argtypes = [i32, i32, i32, i32, i32, i32, i32, P, P, i64, P, P, P, P, P, P, P, P,
                                    P, i32, P, P]
@@ -151,20 +151,29 @@ def decode_matrix(w, d: int) -> np.ndarray:
 
 
 def predict(h, P1, P2, bp, thr, n_hot: int, ffn: int):
-    """Returns dict(u [B,r], s [B,C], mask [C] uint8, idx int32 ascending)."""
+    """Returns dict(u [B,r], s [B,C], mask [C] uint8, idx int32 ascending).
+
+    P1 [r, d] and P2 [C, r] are fp32/fp16 arrays, or Q4_0 pairs (qs uint8
+    [rows, cols/2], sc float16 [rows, cols/32]) with blocks along d (P1) and
+    along the rank (P2)."""
     lib = _load()
     h = np.ascontiguousarray(h)
     B, d = h.shape
-    r = P1.shape[0]
+    p1, p1_sc = _wparts(P1)
+    p2, p2_sc = _wparts(P2)
+    q4 = isinstance(P1, tuple)
+    r = p1.shape[0]
     C = ffn - n_hot
-    assert P1.shape == (r, d) and P2.shape == (C, r)
+    assert p1.shape == ((r, d // 2) if q4 else (r, d))
+    assert P2 is None and C == 0 or p2.shape == ((C, r // 2) if q4 else (C, r))
+    assert (P2 is None) or isinstance(P2, tuple) == q4
     u = np.empty((B, r), np.float64)
     s = np.empty((B, C), np.float64)
     mask = np.empty((C,), np.uint8)
     idx = np.empty((max(C, 1),), np.int32)
     bp_ = None if bp is None else np.ascontiguousarray(bp, dtype=np.float32)
-    n = lib.orc_predict(d, ffn, n_hot, r, _htype(h), _htype(P1), B, _ptr(h), _ptr(P1), _ptr(P2), _ptr(bp_),
-                        float(thr), _ptr(u), _ptr(s), _ptr(mask), _ptr(idx))
+    n = lib.orc_predict(d, ffn, n_hot, r, _htype(h), _wtype_of(P1), B, _ptr(h), _ptr(p1), _ptr(p1_sc), _ptr(p2),
+                        _ptr(p2_sc), _ptr(bp_), float(thr), _ptr(u), _ptr(s), _ptr(mask), _ptr(idx))
     return {"u": u, "s": s, "mask": mask, "idx": idx[:n].copy()}
 
 

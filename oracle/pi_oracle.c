@@ -118,11 +118,16 @@ static double *decode_tokens(int htype, const void *h, int batch, int d) {
  *   s[b,c] = sum_k P2[c,k] u[b,k] + bp[c]                  c < ffn - n_hot
  *   active(c) = OR_b (s[b,c] > thr)
  *   idx = ascending { n_hot + c : active(c) }
- * Any output pointer may be NULL.  Returns the number of active neurons.
+ * The predictor matrices are fp32, fp16 or Q4_0 ([UA] "Adaptif Sparsite
+ * Predictor’ları": the predictor's size is chosen per layer; a Q4_0 predictor
+ * decodes like a Q4_0 weight: P1 in 32-element blocks along d, P2 along the
+ * rank, split planes with the scales in P1_sc / P2_sc, NULL otherwise).  Any
+ * output pointer may be NULL.  Returns the number of active neurons.
  */
 int64_t orc_predict(int d, int ffn, int n_hot, int rank, int htype, int ptype, int batch,
-                    const void *h, const void *P1, const void *P2, const float *bp, double thr,
-                    double *u_out, double *s_out, uint8_t *mask_out, int32_t *idx_out) {
+                    const void *h, const void *P1, const void *P1_sc, const void *P2, const void *P2_sc,
+                    const float *bp, double thr, double *u_out, double *s_out, uint8_t *mask_out,
+                    int32_t *idx_out) {
   const int n_cold = ffn - n_hot;
   double *hd = decode_tokens(htype, h, batch, d);
   double *u = (double *)malloc(sizeof(double) * (size_t)batch * (size_t)rank);
@@ -132,7 +137,7 @@ int64_t orc_predict(int d, int ffn, int n_hot, int rank, int htype, int ptype, i
 #pragma omp parallel for schedule(static)
     for (int k = 0; k < rank; ++k) {
       double acc = 0.0;
-      for (int i = 0; i < d; ++i) acc += orc_elem(ptype, P1, NULL, k, i, d) * hd[(size_t)b * d + i];
+      for (int i = 0; i < d; ++i) acc += orc_elem(ptype, P1, P1_sc, k, i, d) * hd[(size_t)b * d + i];
       u[(size_t)b * rank + k] = acc > 0.0 ? acc : 0.0;
     }
   }
@@ -140,7 +145,7 @@ int64_t orc_predict(int d, int ffn, int n_hot, int rank, int htype, int ptype, i
 #pragma omp parallel for schedule(static)
     for (int c = 0; c < n_cold; ++c) {
       double acc = 0.0;
-      for (int k = 0; k < rank; ++k) acc += orc_elem(ptype, P2, NULL, c, k, rank) * u[(size_t)b * rank + k];
+      for (int k = 0; k < rank; ++k) acc += orc_elem(ptype, P2, P2_sc, c, k, rank) * u[(size_t)b * rank + k];
       if (bp) acc += (double)bp[c];
       s[(size_t)b * n_cold + c] = acc;
     }

@@ -430,3 +430,52 @@ def test_pins_reject_planted_mistake(name, tmp_path):
                 caught = True
                 break
     assert caught, "no pin rejects the planted mistake: " + name
+
+
+# ----------------------------------------------------------------------------
+# Q4_0 predictor (a smaller predictor; the pages size it per layer)
+
+
+def _hexrow(s, dtype):
+    return np.array([int(x, 16) for x in s.split()], dtype=dtype)
+
+
+def test_q4_0_predictor_golden():
+    """Hand-worked Q4_0 predictor (tests/golden/predictor_q4_0_d32_r32.txt)."""
+    g = read("predictor_q4_0_d32_r32.txt")
+    d, r, ffn, n_hot, thr = int(g["d"]), int(g["rank"]), int(g["ffn"]), int(g["n_hot"]), float(g["thr"])
+    p1_qs = np.tile(_hexrow(g["P1_rest_qs"], np.uint8), (r, 1))
+    p1_sc = np.full((r, 1), int(g["P1_rest_scale"], 16), dtype=np.uint16)
+    for row in (0, 1):
+        p1_qs[row] = _hexrow(g["P1_row%d_qs" % row], np.uint8)
+        p1_sc[row, 0] = int(g["P1_row%d_scale" % row], 16)
+    p2_qs = np.stack([_hexrow(g["P2_row%d_qs" % c], np.uint8) for c in (0, 1)])
+    p2_sc = np.array([[int(g["P2_row%d_scale" % c], 16)] for c in (0, 1)], dtype=np.uint16)
+    P1 = (np.ascontiguousarray(p1_qs), np.ascontiguousarray(p1_sc.view(np.float16)))
+    P2 = (np.ascontiguousarray(p2_qs), np.ascontiguousarray(p2_sc.view(np.float16)))
+    h = np.zeros((1, d), np.float16)
+    for i, v in mat(g["h_nonzero"]):
+        h[0, int(i)] = v
+    u = np.zeros(r)
+    for k, v in mat(g["u_nonzero"]):
+        u[int(k)] = v
+    res = oracle.predict(h, P1, P2, mat(g["bp"]).astype(np.float32), thr, n_hot, ffn)
+    assert np.array_equal(res["u"][0], u)
+    assert np.array_equal(res["s"][0], mat(g["s"]))
+    assert res["idx"].tolist() == ints(g["idx"])
+
+
+def test_q4_0_predictor_equals_its_fp16_twin():
+    """A Q4_0 predictor whose values s * (q - 8) are exact in fp16 gives the
+    same u, scores and list as the fp16 predictor holding those values (the
+    fp16 path is pinned by the hand-worked fixtures above)."""
+    rng = np.random.default_rng(31)
+    d, r, ffn, n_hot = 96, 64, 40, 6
+    P1q, P1x = _q4_twin(rng, r, d)
+    P2q, P2x = _q4_twin(rng, ffn - n_hot, r)
+    bp = (rng.standard_normal(ffn - n_hot) * 0.5).astype(np.float32)
+    h = _tokens(rng, 3, d).astype(np.float16)
+    a = oracle.predict(h, P1q, P2q, bp, 0.5, n_hot, ffn)
+    b = oracle.predict(h, P1x, P2x, bp, 0.5, n_hot, ffn)
+    assert np.array_equal(a["u"], b["u"]) and np.array_equal(a["s"], b["s"])
+    assert np.array_equal(a["idx"], b["idx"]) and 0 < len(a["idx"]) < ffn - n_hot
