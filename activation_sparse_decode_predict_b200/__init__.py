@@ -91,15 +91,29 @@ def weight(w: Optional[WeightT]) -> Weight:
     return Weight(_ptr(w), None)
 
 
+def _pred_ptr(P):
+    """Device pointer of a predictor matrix: a tensor, or a Q4_0 pair (codes,
+    scales) whose scales follow its codes in one buffer (the C ABI's layout)."""
+    if isinstance(P, tuple):
+        qs, sc = P
+        if sc.data_ptr() != qs.data_ptr() + qs.numel():
+            raise ValueError("Q4_0 predictor scales must follow its codes in the same buffer")
+        return _ptr(qs)
+    return _ptr(P)
+
+
 def layer_weights(L: dict) -> LayerWeights:
-    """pi_layer_weights from a dict with keys P1, P2, bp, Wg, Wu, WdT, b1, b2, thr."""
-    return LayerWeights(_ptr(L["P1"]), _ptr(L["P2"]), _ptr(L.get("bp")), weight(L.get("Wg")), weight(L["Wu"]),
-                        weight(L["WdT"]), _ptr(L.get("b1")), _ptr(L.get("b2")), float(L["thr"]), 0)
+    """pi_layer_weights from a dict with keys P1, P2, bp, Wg, Wu, WdT, b1, b2,
+    thr and optionally rank (this layer's predictor rank; 0 = the descriptor's)."""
+    return LayerWeights(_pred_ptr(L["P1"]), _pred_ptr(L["P2"]), _ptr(L.get("bp")), weight(L.get("Wg")),
+                        weight(L["Wu"]), weight(L["WdT"]), _ptr(L.get("b1")), _ptr(L.get("b2")), float(L["thr"]),
+                        int(L.get("rank", 0)))
 
 
 def predict(desc: FfnDesc, h: torch.Tensor, P1, P2, bp, threshold: float, idx: torch.Tensor, count: torch.Tensor,
             ws: torch.Tensor, stream=None) -> None:
-    _check(lib().pi_predict(ctypes.byref(desc), h.shape[0], _ptr(h), _ptr(P1), _ptr(P2), _ptr(bp), float(threshold),
+    _check(lib().pi_predict(ctypes.byref(desc), h.shape[0], _ptr(h), _pred_ptr(P1), _pred_ptr(P2), _ptr(bp),
+                            float(threshold),
                             _ptr(idx), _ptr(count), _ptr(ws), ws.numel(), _stream(stream)))
 
 

@@ -39,7 +39,7 @@ class LayerWeights(ctypes.Structure):
     _fields_ = [("P1", ctypes.c_void_p), ("P2", ctypes.c_void_p), ("bp", ctypes.c_void_p),
                 ("W_gate", Weight), ("W_up", Weight), ("W_downT", Weight),
                 ("b1", ctypes.c_void_p), ("b2", ctypes.c_void_p), ("threshold", ctypes.c_float),
-                ("_pad", ctypes.c_int32)]
+                ("rank", ctypes.c_int32)]
 
 
 class PiError(RuntimeError):

@@ -39,7 +39,10 @@ pi_status check_desc(const pi_ffn_desc* d, int32_t batch) {
   if (d->rank <= 0 || d->rank % 8) return fail(PI_ERR_INVALID_ARG, "%s", "rank must be a positive multiple of 8");
   if (d->wtype != PI_F32 && d->wtype != PI_F16 && d->wtype != PI_Q4_0)
     return fail(PI_ERR_INVALID_ARG, "%s", "wtype must be PI_F32, PI_F16 or PI_Q4_0");
-  if (d->ptype != PI_F32 && d->ptype != PI_F16) return fail(PI_ERR_INVALID_ARG, "%s", "ptype must be PI_F32 or PI_F16");
+  if (d->ptype != PI_F32 && d->ptype != PI_F16 && d->ptype != PI_Q4_0)
+    return fail(PI_ERR_INVALID_ARG, "%s", "ptype must be PI_F32, PI_F16 or PI_Q4_0");
+  if (d->ptype == PI_Q4_0 && (d->d % 32 || d->rank % 32))
+    return fail(PI_ERR_INVALID_ARG, "%s", "a Q4_0 predictor needs d % 32 == 0 and rank % 32 == 0");
   if (d->act != PI_ACT_RELU && d->act != PI_ACT_REGLU && d->act != PI_ACT_RELU2)
     return fail(PI_ERR_INVALID_ARG, "%s", "act must be PI_ACT_RELU, PI_ACT_REGLU or PI_ACT_RELU2");
   if (d->wtype == PI_Q4_0 && d->d % 32) return fail(PI_ERR_INVALID_ARG, "%s", "Q4_0 needs d % 32 == 0");
@@ -127,8 +130,11 @@ pi_status predict_impl(const pi_ffn_desc* d, int32_t B, const void* h, const voi
     PI_CUDA(pi::launch_compact(tmask, tcount, C, d->n_hot, idx, count, st), "compaction launch");
     return PI_OK;
   }
-  PI_CUDA(pi::launch_pred_u(d->ptype, P1, h, B, d->d, d->rank, u, sms, st), "predictor GEMV1 launch");
-  PI_CUDA(pi::launch_pred_score(d->ptype, P2, bp, u, B, d->rank, C, thr, tmask, tcount, st), "predictor score launch");
+  PI_CUDA(pi::launch_pred_u(d->ptype, P1, pi::pred_scales(d, P1, d->rank, d->d), h, B, d->d, d->rank, u, sms, st),
+          "predictor GEMV1 launch");
+  PI_CUDA(pi::launch_pred_score(d->ptype, P2, pi::pred_scales(d, P2, C, d->rank), bp, u, B, d->rank, C, thr, tmask,
+                                tcount, st),
+          "predictor score launch");
   PI_CUDA(pi::launch_compact(tmask, tcount, C, d->n_hot, idx, count, st), "compaction launch");
   return PI_OK;
 }
@@ -141,7 +147,8 @@ pi_status ffn_impl(const pi_ffn_desc* d, int32_t B, const void* h, const int32_t
   float* a = reinterpret_cast<float*>(ws + L.act);
   float* partial = reinterpret_cast<float*>(ws + L.partial);
   const int sms = sm_count();
-  if (pi::kTcFfn && pi::tc_ffn_supported(d->wtype, d->ptype, d->d, B)) {
+  const int ht = pi::token_type(d);
+  if (pi::kTcFfn && pi::tc_ffn_supported(d->wtype, ht, d->d, B)) {
     // token blocks of 3..16 with fp16 weights: gathered tiles on tcgen05, fp32
     // accumulators in tensor memory, y (with b2) written by the last kernel
     PI_CUDA(pi::launch_tc_ffn(d->act, h, B, d->d, d->ffn, d->n_hot, idx, count, Wg.data, Wu.data, Wd.data, b1, b2, y,
@@ -149,7 +156,7 @@ pi_status ffn_impl(const pi_ffn_desc* d, int32_t B, const void* h, const int32_t
             "tcgen05 FFN launch");
     return PI_OK;
   }
-  if (pi::batch_supported(d->wtype, d->ptype, d->d, B)) {
+  if (pi::batch_supported(d->wtype, ht, d->d, B)) {
     // token blocks of 3..16 with fp16 weights: tensor-core gate/up and down
     const int NR = pi::batch_ranges(d->d, sms);
     PI_CUDA(pi::launch_batch_ffn(d->act, h, B, d->d, d->ffn, d->n_hot, idx, count, Wg.data, Wu.data, Wd.data, b1,
@@ -160,7 +167,7 @@ pi_status ffn_impl(const pi_ffn_desc* d, int32_t B, const void* h, const int32_t
     return PI_OK;
   }
   const int G = L.g_max < 2 * sms ? L.g_max : 2 * sms;
-  PI_CUDA(pi::launch_ffn_act(d->wtype, d->ptype, d->act, h, B, d->d, d->ffn, d->n_hot, idx, count, Wg.data,
+  PI_CUDA(pi::launch_ffn_act(d->wtype, ht, d->act, h, B, d->d, d->ffn, d->n_hot, idx, count, Wg.data,
                              Wg.scales, Wu.data, Wu.scales, b1, a, d->ffn, status, sms, st),
           "FFN activation launch");
   PI_CUDA(pi::launch_ffn_down(d->wtype, B, d->d, d->ffn, d->n_hot, idx, count, Wd.data, Wd.scales, a, d->ffn,
@@ -179,7 +186,21 @@ pi_status check_layer(const pi_ffn_desc* desc, const pi_layer_weights* w) {
   PI_TRY(check_weight(desc, w->W_downT, "W_downT"));
   if (w->b1) PI_TRY(check_ptr(w->b1, 4, "b1"));
   if (w->b2) PI_TRY(check_ptr(w->b2, 16, "b2"));
+  if (w->rank != 0) {
+    const int unit = desc->ptype == PI_Q4_0 ? 32 : 8;
+    if (w->rank < 0 || w->rank % unit || w->rank > desc->rank)
+      return fail(PI_ERR_INVALID_ARG, "%s",
+                  "a layer's rank must be 0 (the descriptor's) or a multiple of 8 (Q4_0 predictors: 32) "
+                  "no larger than the descriptor's rank");
+  }
   return PI_OK;
+}
+
+// The descriptor of one layer: the layer's own predictor rank when it has one.
+pi_ffn_desc layer_desc(const pi_ffn_desc* desc, const pi_layer_weights* w) {
+  pi_ffn_desc d = *desc;
+  if (w->rank > 0) d.rank = w->rank;
+  return d;
 }
 
 static_assert(pi::kYAccCopies == pi::kYCopies, "workspace layout and kernel agree on the accumulator copies");
@@ -214,10 +235,12 @@ pi_status fused_params(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, pi:
   const size_t wrow = desc->wtype == PI_Q4_0 ? desc->d / 2 + desc->d / 16
                                               : (size_t)desc->d * (desc->wtype == PI_F16 ? 2 : 4);
   const size_t neuron = (wrow + 16) * (desc->act == PI_ACT_REGLU ? 3 : 2) + 16 + 256;
-  // predictor items: fp16 predictors go to the tensor cores in 16-row tiles with padded rows
-  const size_t p2item = desc->ptype == PI_F16 ? (size_t)16 * (2 * desc->rank + 16) + 256
-                                              : (size_t)(P.T / 32) * desc->rank * ep;
-  const size_t p1item = (size_t)desc->d * ep + 256;
+  // predictor items (the largest rank): fp16 predictors go to the tensor cores
+  // in 16-row tiles with padded rows; Q4_0 rows carry codes and scales
+  const size_t p2item = desc->ptype == PI_F16    ? (size_t)16 * (2 * desc->rank + 16) + 256
+                        : desc->ptype == PI_Q4_0 ? (size_t)(P.T / 32) * (desc->rank / 2 + desc->rank / 16) + 256
+                                                 : (size_t)(P.T / 32) * desc->rank * ep;
+  const size_t p1item = desc->ptype == PI_Q4_0 ? (size_t)desc->d / 2 + desc->d / 16 + 256 : (size_t)desc->d * ep + 256;
   const size_t half = (size_t)P.ring_bytes / 2;
   if (neuron > half || p2item > half || p1item > half) return PI_ERR_UNSUPPORTED;
   // the tensor-core P1 tile takes at most 16 rows, and the rows of one tile
@@ -306,6 +329,11 @@ pi_status fused_stack(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, cons
     // a neuron item carries the 16-byte block of b1 that holds its bias
     if (w.b1 && (reinterpret_cast<uintptr_t>(w.b1) & 15u)) return PI_ERR_UNSUPPORTED;
     s.thr = w.threshold;
+    s.rank = w.rank > 0 ? w.rank : desc->rank;
+    if (!pi::stack_rank_ok(desc->ptype, s.rank)) return PI_ERR_UNSUPPORTED;
+    const pi_ffn_desc ld = layer_desc(desc, &w);
+    s.P1_sc = pi::pred_scales(&ld, w.P1, s.rank, desc->d);
+    s.P2_sc = pi::pred_scales(&ld, w.P2, desc->ffn - desc->n_hot, s.rank);
   }
   PI_CUDA(pi::launch_stack(desc->wtype, desc->ptype, B, P, G, smem, st), "fused decode-step launch");
   return PI_OK;
@@ -386,8 +414,10 @@ pi_status pi_layer(const pi_ffn_desc* desc, int32_t batch, const void* h, const 
   if (w->b2) PI_TRY(check_ptr(w->b2, 16, "b2"));
   PI_TRY(check_ptr(y, 16, "y"));
   PI_TRY(check_ws(desc, batch, ws, ws_bytes));
+  PI_TRY(check_layer(desc, w));
   cudaStream_t st = (cudaStream_t)stream;
-  PI_TRY(predict_impl(desc, batch, h, w->P1, w->P2, w->bp, w->threshold, idx, count, (char*)ws, st));
+  const pi_ffn_desc ld = layer_desc(desc, w);
+  PI_TRY(predict_impl(&ld, batch, h, w->P1, w->P2, w->bp, w->threshold, idx, count, (char*)ws, st));
   return ffn_impl(desc, batch, h, idx, count, w->W_gate, w->W_up, w->W_downT, w->b1, w->b2, y, (char*)ws, st);
 }
 
@@ -441,7 +471,7 @@ pi_status pi_decode_stack(const pi_ffn_desc* desc, int32_t batch, int32_t n_laye
     float* yl = y ? y + (size_t)l * batch * desc->d : ybuf;
     PI_TRY(pi_layer(desc, batch, cur, &layers[l], idx + (size_t)l * C, counts + l, yl, ws, ws_bytes, stream));
     void* nxt = hbuf[(n_layers - 1 - l) & 1];
-    PI_CUDA(pi::launch_rmsnorm(desc->ptype, cur, yl, batch, desc->d, eps, nxt, st), "rmsnorm launch");
+    PI_CUDA(pi::launch_rmsnorm(pi::token_type(desc), cur, yl, batch, desc->d, eps, nxt, st), "rmsnorm launch");
     cur = nxt;
   }
   return PI_OK;
@@ -464,7 +494,7 @@ int32_t pi_stack_launches(const pi_ffn_desc* desc, int32_t batch, int32_t n_laye
   else
     pred = cold ? 3 : 1;  // u, scores, compaction
   int ffn;
-  if (pi::kTcFfn && pi::tc_ffn_supported(desc->wtype, desc->ptype, desc->d, batch))
+  if (pi::kTcFfn && pi::tc_ffn_supported(desc->wtype, pi::token_type(desc), desc->d, batch))
     ffn = 4;  // up, activations, down, reduce
   else
     ffn = 3;  // gate/up (or row dots), down, reduce

@@ -13,10 +13,14 @@ namespace pi {
 
 // ---------------------------------------------------------------------------
 // Predictor step 1: u[b,k] = max(0, P1[k,:] . h[b,:]), fp32.  One warp per row.
+// PT: predictor matrix type (fp32, fp16 or Q4_0 with its scales in P1_sc); the
+// token block is fp32 with fp32 predictors and fp16 otherwise.
 template <int PT, int NB>
-__global__ void __launch_bounds__(256) k_pred_u(const void* __restrict__ P1, const void* __restrict__ h, int B, int d,
-                                                int r, float* __restrict__ u) {
+__global__ void __launch_bounds__(256) k_pred_u(const void* __restrict__ P1, const void* __restrict__ P1_sc,
+                                                const void* __restrict__ h, int B, int d, int r,
+                                                float* __restrict__ u) {
   constexpr int E = Unit<PT>::E;
+  constexpr int HT = PT == kF32 ? kF32 : kF16;
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nw = (gridDim.x * blockDim.x) >> 5;
@@ -29,12 +33,12 @@ __global__ void __launch_bounds__(256) k_pred_u(const void* __restrict__ P1, con
       for (int i = 0; i < NB; ++i) acc[i] = 0.f;
       for (int un = lane; un < units; un += 32) {
         float w[E];
-        load_w_unit<PT>(P1, nullptr, k, d, un, w);
+        load_w_unit<PT>(P1, P1_sc, k, d, un, w);
 #pragma unroll
         for (int i = 0; i < NB; ++i) {
           if (i < nb) {
             float x[E];
-            load_h_unit<PT, PT>(h, b0 + i, d, un, x);
+            load_h_unit<PT, HT>(h, b0 + i, d, un, x);
 #pragma unroll
             for (int e = 0; e < E; ++e) acc[i] = fmaf(w[e], x[e], acc[i]);
           }
@@ -54,7 +58,8 @@ __global__ void __launch_bounds__(256) k_pred_u(const void* __restrict__ P1, con
 // s = P2[c,:] . u[b,:] + bp[c]; active = OR_b (s > thr).  Writes the tile's
 // 8 ballot words and its popcount.
 template <int PT, int NB>
-__global__ void __launch_bounds__(256) k_pred_score(const void* __restrict__ P2, const float* __restrict__ bp,
+__global__ void __launch_bounds__(256) k_pred_score(const void* __restrict__ P2, const void* __restrict__ P2_sc,
+                                                    const float* __restrict__ bp,
                                                     const float* __restrict__ u, int B, int r, int C, float thr,
                                                     uint32_t* __restrict__ tile_mask, int* __restrict__ tile_count) {
   constexpr int E = Unit<PT>::E;
@@ -74,7 +79,7 @@ __global__ void __launch_bounds__(256) k_pred_score(const void* __restrict__ P2,
       for (int i = 0; i < NB; ++i) acc[i] = 0.f;
       for (int un = lane; un < units; un += 32) {
         float w[E];
-        load_w_unit<PT>(P2, nullptr, c, r, un, w);
+        load_w_unit<PT>(P2, P2_sc, c, r, un, w);
 #pragma unroll
         for (int i = 0; i < NB; ++i) {
           if (i < nb) {
@@ -386,20 +391,25 @@ __global__ void __launch_bounds__(1024) k_rmsnorm(const void* __restrict__ h, co
 
 constexpr int kNB = 4;  // tokens per pass in the CUDA-core kernels
 
-cudaError_t launch_pred_u(int ptype, const void* P1, const void* h, int B, int d, int r, float* u, int sms,
-                          cudaStream_t st) {
+cudaError_t launch_pred_u(int ptype, const void* P1, const void* P1_sc, const void* h, int B, int d, int r, float* u,
+                          int sms, cudaStream_t st) {
   const int grid = min((r + 7) / 8, sms * 8);
-  if (ptype == kF32) k_pred_u<kF32, kNB><<<grid, 256, 0, st>>>(P1, h, B, d, r, u);
-  else k_pred_u<kF16, kNB><<<grid, 256, 0, st>>>(P1, h, B, d, r, u);
+  if (ptype == kF32) k_pred_u<kF32, kNB><<<grid, 256, 0, st>>>(P1, nullptr, h, B, d, r, u);
+  else if (ptype == kF16) k_pred_u<kF16, kNB><<<grid, 256, 0, st>>>(P1, nullptr, h, B, d, r, u);
+  else k_pred_u<kQ4_0, kNB><<<grid, 256, 0, st>>>(P1, P1_sc, h, B, d, r, u);
   return cudaGetLastError();
 }
 
-cudaError_t launch_pred_score(int ptype, const void* P2, const float* bp, const float* u, int B, int r, int C,
-                              float thr, uint32_t* tile_mask, int* tile_count, cudaStream_t st) {
+cudaError_t launch_pred_score(int ptype, const void* P2, const void* P2_sc, const float* bp, const float* u, int B,
+                              int r, int C, float thr, uint32_t* tile_mask, int* tile_count, cudaStream_t st) {
   const int tiles = (C + 255) / 256;
   if (tiles == 0) return cudaSuccess;
-  if (ptype == kF32) k_pred_score<kF32, kNB><<<tiles, 256, 0, st>>>(P2, bp, u, B, r, C, thr, tile_mask, tile_count);
-  else k_pred_score<kF16, kNB><<<tiles, 256, 0, st>>>(P2, bp, u, B, r, C, thr, tile_mask, tile_count);
+  if (ptype == kF32)
+    k_pred_score<kF32, kNB><<<tiles, 256, 0, st>>>(P2, nullptr, bp, u, B, r, C, thr, tile_mask, tile_count);
+  else if (ptype == kF16)
+    k_pred_score<kF16, kNB><<<tiles, 256, 0, st>>>(P2, nullptr, bp, u, B, r, C, thr, tile_mask, tile_count);
+  else
+    k_pred_score<kQ4_0, kNB><<<tiles, 256, 0, st>>>(P2, P2_sc, bp, u, B, r, C, thr, tile_mask, tile_count);
   return cudaGetLastError();
 }
 

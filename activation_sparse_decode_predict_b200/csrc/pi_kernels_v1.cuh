@@ -5,10 +5,11 @@
 
 namespace pi {
 
-cudaError_t launch_pred_u(int ptype, const void* P1, const void* h, int B, int d, int r, float* u, int sms,
-                          cudaStream_t st);
-cudaError_t launch_pred_score(int ptype, const void* P2, const float* bp, const float* u, int B, int r, int C,
-                              float thr, uint32_t* tile_mask, int* tile_count, cudaStream_t st);
+// ptype: fp32, fp16 or Q4_0 predictor matrices (Q4_0: scales in P1_sc / P2_sc, else unused)
+cudaError_t launch_pred_u(int ptype, const void* P1, const void* P1_sc, const void* h, int B, int d, int r, float* u,
+                          int sms, cudaStream_t st);
+cudaError_t launch_pred_score(int ptype, const void* P2, const void* P2_sc, const float* bp, const float* u, int B,
+                              int r, int C, float thr, uint32_t* tile_mask, int* tile_count, cudaStream_t st);
 cudaError_t launch_compact(const uint32_t* tile_mask, const int* tile_count, int C, int n_hot, int32_t* idx,
                            int32_t* count, cudaStream_t st);
 cudaError_t launch_ffn_act(int wtype, int htype, int act, const void* h, int B, int d, int ffn, int n_hot,

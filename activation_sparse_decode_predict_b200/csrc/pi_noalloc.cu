@@ -92,8 +92,11 @@ pi_status pi_predict_static(const pi_ffn_desc* desc, int32_t batch, const void* 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaError_t e = pi::launch_pred_u(desc->ptype, P1, h, batch, desc->d, r, u, sms, st);
-  if (e == cudaSuccess) e = pi::launch_pred_score(desc->ptype, P2, bp, u, batch, r, C, threshold, tmask, tcount, st);
+  cudaError_t e =
+      pi::launch_pred_u(desc->ptype, P1, pi::pred_scales(desc, P1, r, desc->d), h, batch, desc->d, r, u, sms, st);
+  if (e == cudaSuccess)
+    e = pi::launch_pred_score(desc->ptype, P2, pi::pred_scales(desc, P2, C, r), bp, u, batch, r, C, threshold, tmask,
+                              tcount, st);
   if (e == cudaSuccess) e = pi::launch_compact(tmask, tcount, C, n_hot, idx, count, st);
   if (e != cudaSuccess) return err(PI_ERR_CUDA, cudaGetErrorString(e));
   return PI_OK;

@@ -484,9 +484,11 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
   Ctrl* ctrl = p.ctrl;
   const int G = gridDim.x, c = blockIdx.x;
   const int T = p.T, NW = T / 32;
-  const int d = p.d, r = p.rank, H = p.n_hot, C = p.ffn - p.n_hot;
+  const int d = p.d, H = p.n_hot, C = p.ffn - p.n_hot;
   const int gated = p.act == kReglu;
-  const int ep = PT == kF16 ? 2 : 4;
+  // the token block is fp32 with fp32 predictors, fp16 with fp16 or Q4_0 ones
+  constexpr int HT = PT == kF32 ? kF32 : kF16;
+  const int ep = HT == kF16 ? 2 : 4;  // bytes per token element (and per fp16/fp32 predictor element)
   constexpr int K = kYCopies;
   // the fp16 token rows in shared memory feed only the tensor-core P1 (token
   // blocks of 2) and tensor-core neuron groups; otherwise they take no space
@@ -508,8 +510,8 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
   __syncthreads();
   const unsigned base = (unsigned)s.misc[1];
 
-  // shares that do not depend on the predictor
-  const int k0 = share_lo(r, c, G), k1 = share_lo(r, c + 1, G);
+  // shares that do not depend on the predictor (the P1 rows, a share of the
+  // layer's rank, are taken per layer: each layer has its own rank)
   const int c0 = share_lo(C, c, G), c1 = share_lo(C, c + 1, G);
 
   // static hot share (consumed while barrier U completes); the rest of the
@@ -525,8 +527,9 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
     // other CTAs and stages every CTA's u in shared memory, while the
     // consumers run the first static hot neurons.
     const int lane = threadIdx.x & 31;
-    const int US = 2 * r + 16;
     for (int l = 0; l < p.L; ++l) {
+      const int r = p.layers[l].rank;
+      const int US = 2 * r + 16;
       bool ok = true;
       if (lane == 0) {
         ok = mbar_wait(s.u_bar, l & 1, ctrl);
@@ -557,6 +560,24 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
               *reinterpret_cast<__half2*>(s.ub + (2 * b + 1) * US + 2 * col) = lo;
             }
           }
+        }
+      } else if constexpr (PT == kQ4_0) {
+        // Q4_0 P2 rows: lane m of a warp takes 32-element block m of a row, so
+        // u is stored block-transposed, s.u[b][k][m] = u[b][32 m + k] with a
+        // row stride of nblk + 1 (conflict-free writes and reads), and each
+        // block's sum of u goes to s.usum[b][m] (see the Q4_0 row dot)
+        const int nblk = r / 32, RS = 32 * (nblk + 1);
+        float* usum = s.u + (size_t)B * (p.rank + 32);
+        for (int i = lane; i < B * r; i += 32) {
+          const int b = i / r, j = i % r;
+          s.u[(size_t)b * RS + (j % 32) * (nblk + 1) + j / 32] = __ldcg(p.u_g + i);
+        }
+        __syncwarp();
+        for (int i = lane; i < B * nblk; i += 32) {
+          const int b = i / nblk, m = i % nblk;
+          float a = 0.f;
+          for (int kk = 0; kk < 32; ++kk) a += s.u[(size_t)b * RS + kk * (nblk + 1) + m];
+          usum[i] = a;
         }
       } else {
         // split layout: unit m (8 values) stored as two float4 planes so that
@@ -599,6 +620,8 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
     bool ok = true;
     for (int l = 0; l < p.L && ok; ++l) {
       const StackLayer& Ly = p.layers[l];
+      const int r = Ly.rank;
+      const int k0 = share_lo(r, c, G), k1 = share_lo(r, c + 1, G);
       if (lane == 0) {
         // item order = consumption order
         if constexpr (PT == kF16) {
@@ -611,6 +634,24 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
           for (int cc = c0; cc < c1 && ok; cc += 16)
             ok = pr.issue_rows(reinterpret_cast<const uint8_t*>(Ly.P2) + (int64_t)cc * r * 2, (int64_t)r * 2,
                                min(16, c1 - cc), r * 2, r * 2 + 16, 0);
+        } else if constexpr (PT == kQ4_0) {
+          // Q4_0 predictor rows: codes then scales, like a Q4_0 weight row
+          for (int k = k0; k < k1 && ok; ++k) {
+            const void* src[2] = {reinterpret_cast<const uint8_t*>(Ly.P1) + (int64_t)k * (d / 2),
+                                  reinterpret_cast<const uint8_t*>(Ly.P1_sc) + (int64_t)k * (d / 16)};
+            const uint32_t by[2] = {(uint32_t)(d / 2), (uint32_t)(d / 16)};
+            ok = pr.issue(2, src, by);
+          }
+          if (ok) ok = pr.issue_range(Ly, ha0, ha1 - ha0, WT, gated);
+          if (ok) ok = pr.issue_marker();
+          // P2 items of NW rows: the rows' codes, then the rows' scales
+          for (int cc = c0; cc < c1 && ok; cc += NW) {
+            const int rows = min(NW, c1 - cc);
+            const void* src[2] = {reinterpret_cast<const uint8_t*>(Ly.P2) + (int64_t)cc * (r / 2),
+                                  reinterpret_cast<const uint8_t*>(Ly.P2_sc) + (int64_t)cc * (r / 16)};
+            const uint32_t by[2] = {(uint32_t)(rows * (r / 2)), (uint32_t)(rows * (r / 16))};
+            ok = pr.issue(2, src, by);
+          }
         } else {
           for (int k = k0; k < k1 && ok; ++k) {
             const void* src = reinterpret_cast<const uint8_t*>(Ly.P1) + (int64_t)k * d * ep;
@@ -709,13 +750,12 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
   // layer-0 input
 #pragma unroll
   for (int b = 0; b < B; ++b)
-    row_vals<WT, EPT, PT>(reinterpret_cast<const uint8_t*>(p.h_in) + (int64_t)b * d * ep, t, T, h[b]);
+    row_vals<WT, EPT, HT>(reinterpret_cast<const uint8_t*>(p.h_in) + (int64_t)b * d * ep, t, T, h[b]);
   if (c == 0 && p.h_trace) {
 #pragma unroll
-    for (int b = 0; b < B; ++b) store_vals<WT, EPT, PT>(reinterpret_cast<uint8_t*>(p.h_trace) + (int64_t)b * d * ep, t, T, h[b]);
+    for (int b = 0; b < B; ++b) store_vals<WT, EPT, HT>(reinterpret_cast<uint8_t*>(p.h_trace) + (int64_t)b * d * ep, t, T, h[b]);
   }
   const int HS = 2 * d + 16;  // byte stride of the fp16 token rows in shared memory
-  const int US = 2 * r + 16;  // byte stride of the fp16 u rows
   if constexpr (kTokRows) {
 #pragma unroll
     for (int b = 0; b < B; ++b) store_vals<WT, EPT, kF16>(s.hb + b * HS, t, T, h[b]);
@@ -745,6 +785,9 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
 
   for (int l = 0; l < p.L; ++l) {
     const StackLayer& Ly = p.layers[l];
+    const int r = Ly.rank;
+    const int US = 2 * r + 16;  // byte stride of the fp16 u rows
+    const int k0 = share_lo(r, c, G), k1 = share_lo(r, c + 1, G);
     if (t == 0) PI_STAMP(l, 0);
 #pragma unroll
     for (int b = 0; b < B; ++b)
@@ -826,13 +869,19 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
           uint32_t off;
           to |= !wait_item(off);
           float w[EPT];
-          row_vals<WT, EPT, PT>(s.ring + off, t, T, w);
+          float psc = 1.f;
+          if constexpr (PT == kQ4_0) {
+            q4_codes<EPT>(s.ring + off, d, t, w, psc);  // same column ownership as Q4_0 weight rows
+          } else {
+            row_vals<WT, EPT, PT>(s.ring + off, t, T, w);
+          }
           release_item();
 #pragma unroll
           for (int b = 0; b < B; ++b) {
             float a = 0.f;
 #pragma unroll
             for (int e = 0; e < EPT; ++e) a = fmaf(w[e], h[b][e], a);
+            if constexpr (PT == kQ4_0) a = psc * fmaf(16.f, a, -24.f * hsum[b]);
             acc[i * B + b] = a;
           }
         }
@@ -1108,6 +1157,55 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
         s.act[x] = on ? 1 : 0;
       }
       witem += ntile;
+    } else if constexpr (PT == kQ4_0) {
+      // Q4_0 P2 rows, one warp per row: lane m takes 32-element blocks m,
+      // m + 32, ...; a code q is placed in the top mantissa bits of 1.0f
+      // (f = 1 + q/16, exact), so a block's dot is s (16 sum(f u) - 24 sum(u))
+      // with the block sums of u staged with u
+      const int nblk = r / 32, US1 = nblk + 1, RS = 32 * US1;
+      const float* usum = s.u + (size_t)B * (p.rank + 32);
+      for (int cc = c0; cc < c1; cc += NW) {
+        const int rows = min(NW, c1 - cc);
+        uint32_t off;
+        to |= !wait_item(off);
+        if (warp < rows) {
+          const uint8_t* qrow = s.ring + off + (size_t)warp * (r / 2);
+          const uint8_t* srow = s.ring + off + (size_t)rows * (r / 2) + (size_t)warp * (r / 16);
+          float acc[B];
+#pragma unroll
+          for (int b = 0; b < B; ++b) acc[b] = 0.f;
+          for (int m = lane; m < nblk; m += 32) {
+            const uint4 q = *reinterpret_cast<const uint4*>(qrow + 16 * m);
+            const float bsc = half_bits_to_float(*reinterpret_cast<const uint16_t*>(srow + 2 * m));
+            const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+            float dot[B];
+#pragma unroll
+            for (int b = 0; b < B; ++b) dot[b] = 0.f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t byte = qw[w] >> (8 * kk);
+                const float flo = __uint_as_float(0x3f800000u | ((byte & 0xfu) << 19));
+                const float fhi = __uint_as_float(0x3f800000u | ((byte & 0xf0u) << 15));
+                const int e = 4 * w + kk;  // element e (low nibble) and e + 16 (high nibble)
+#pragma unroll
+                for (int b = 0; b < B; ++b) {
+                  dot[b] = fmaf(flo, s.u[(size_t)b * RS + e * US1 + m], dot[b]);
+                  dot[b] = fmaf(fhi, s.u[(size_t)b * RS + (e + 16) * US1 + m], dot[b]);
+                }
+              }
+#pragma unroll
+            for (int b = 0; b < B; ++b) acc[b] = fmaf(bsc, fmaf(16.f, dot[b], -24.f * usum[b * nblk + m]), acc[b]);
+          }
+          bool on = false;
+          const float bias = s.bp[cc - c0 + warp];
+#pragma unroll
+          for (int b = 0; b < B; ++b) on |= (warp_sum(acc[b]) + bias) > Ly.thr;
+          if (lane == 0) s.act[cc - c0 + warp] = on ? 1 : 0;
+        }
+        release_item();
+      }
     } else {
       const int nu = r / 8;  // 8-element units per row (r % 8 == 0)
       // single token and rank <= 1024: this lane's slice of u stays in registers
@@ -1301,7 +1399,7 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
       for (int b = 0; b < B; ++b) {
         const float inv = rsqrtf(ss[b] / (float)d + p.eps);
 #pragma unroll
-        for (int e = 0; e < EPT; ++e) h[b][e] = round_to(PT, h[b][e] * inv);
+        for (int e = 0; e < EPT; ++e) h[b][e] = round_to(HT, h[b][e] * inv);
       }
       if constexpr (kTokRows) {
 #pragma unroll
@@ -1316,7 +1414,7 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
         }
         if (dst) {
 #pragma unroll
-          for (int b = 0; b < B; ++b) store_vals<WT, EPT, PT>(dst + (size_t)b * d * ep, t, T, h[b]);
+          for (int b = 0; b < B; ++b) store_vals<WT, EPT, HT>(dst + (size_t)b * d * ep, t, T, h[b]);
         }
       }
     }
@@ -1433,12 +1531,13 @@ bool stack_supported(int wtype, int ptype, int d, int ffn, int n_hot, int rank, 
   if (B < 1 || B > 2) return false;
   if (L < 1 || L > kMaxLayers) return false;
   const bool combo = (wtype == kF16 && ptype == kF16) || (wtype == kQ4_0 && ptype == kF16) ||
-                     (wtype == kF32 && ptype == kF32);
+                     (wtype == kF32 && ptype == kF32) || (wtype == kQ4_0 && ptype == kQ4_0);
   if (!combo) return false;
   const int ept = stack_ept(d);
   if (d % (32 * ept) != 0 || d / ept > kMaxConsumers) return false;
   if (wtype == kQ4_0 && d % 256 != 0) return false;
   if (rank % 8 != 0 || rank > kMaxRank) return false;
+  if (!stack_rank_ok(ptype, rank)) return false;
   (void)ffn;
   (void)n_hot;
   return true;
@@ -1457,7 +1556,9 @@ size_t stack_smem_layout(StackParams& p, int ptype, int B, int G) {
   const size_t sizes[] = {
       sizeof(uint64_t) * (2 * kNQ + 3),                                        // bars
       sizeof(uint32_t) * 4 * kNQ,                                              // item offsets, starts, rows, groups
-      ptype == kF32 ? sizeof(float) * (size_t)B * p.rank : 0,                  // u (fp32 predictors)
+      ptype == kF32 ? sizeof(float) * (size_t)B * p.rank                       // u (fp32 predictors)
+      : ptype == kQ4_0 ? sizeof(float) * (size_t)B * (p.rank + 32 + p.rank / 32)  // u block-transposed + block sums
+                       : 0,
       sizeof(float) * share_cap,                                               // bp
       sizeof(int) * share_cap,                                                 // cidx
       (size_t)share_cap,                                                       // act
@@ -1511,6 +1612,10 @@ cudaError_t launch_stack(int wtype, int ptype, int B, const StackParams& p, int 
   PI_STACK_CASE(kF32, kF32, 2, 8)
   PI_STACK_CASE(kF32, kF32, 1, 16)
   PI_STACK_CASE(kF32, kF32, 2, 16)
+  PI_STACK_CASE(kQ4_0, kQ4_0, 1, 8)
+  PI_STACK_CASE(kQ4_0, kQ4_0, 2, 8)
+  PI_STACK_CASE(kQ4_0, kQ4_0, 1, 16)
+  PI_STACK_CASE(kQ4_0, kQ4_0, 2, 16)
 #undef PI_STACK_CASE
   return cudaErrorInvalidValue;
 }

@@ -77,8 +77,10 @@ struct StackLayer {
   const void* wd_sc;
   const float* b1;
   const float* b2;
+  const void* P1_sc;  // Q4_0 predictors: scales of P1 [rank, d/32] and P2 [C, rank/32] (else null)
+  const void* P2_sc;
   float thr;
-  int pad;
+  int rank;           // this layer's predictor rank (<= the descriptor's)
 };
 
 struct StackParams {
@@ -116,6 +118,14 @@ struct StackParams {
 // neuron groups).
 __host__ __device__ constexpr bool stack_token_rows(int ptype, int B) {
   return ptype == kF16 && (B > 1 || kP1Mma || kF16Mma);
+}
+
+// Whether a layer of this predictor rank fits the kernel: fp16 predictors feed
+// the tensor cores in 16-element steps; Q4_0 predictor rows go to shared
+// memory as whole rows of codes and of scales, 16-byte multiples when the
+// rank is a multiple of 256.
+__host__ __device__ constexpr bool stack_rank_ok(int ptype, int rank) {
+  return rank > 0 && rank <= kMaxRank && (ptype == kF16 ? rank % 16 == 0 : ptype == kQ4_0 ? rank % 256 == 0 : rank % 8 == 0);
 }
 
 // Columns of d each consumer thread owns (8 when d/8 threads fit, else 16).

@@ -271,7 +271,8 @@ def run_ours(args, rank, world, local_rank):
     # measured active counts of the timed steps -> algorithmic bytes
     cnt_p = counts.double().cpu().numpy()
     cnt = np.stack([cnt_p[t % P] for t in range(args.warmup, n_steps)])
-    per_block = [sum(W.layer_bytes(wl, B, float(a)) for a in cnt_p[p]) for p in range(P)]
+    per_block = [sum(W.layer_bytes(wl, B, float(a), wl.layer_rank(l)) for l, a in enumerate(cnt_p[p]))
+                 for p in range(P)]
     total_bytes = sum(per_block[t % P] for t in range(args.warmup, n_steps))
     sec = ms / 1e3
     gbs = total_bytes / sec / 1e9

@@ -38,9 +38,13 @@
  *   back to the model's original rows stays with the caller.
  *
  * Layouts (d = hidden size, F = ffn, H = n_hot, C = F - H, r = rank, B = batch)
- *   h        [B, d]   token block, element type `ptype` (F32 or F16)
+ *   h        [B, d]   token block: fp32 when ptype is F32, else fp16
  *   P1       [r, d]   predictor first matrix, `ptype`
  *   P2       [C, r]   predictor second matrix (cold neurons only), `ptype`
+ *   A Q4_0 predictor matrix [rows, cols] is ONE buffer: the codes
+ *   qs [rows, cols/2] then, right after them, the scales sc [rows, cols/32]
+ *   fp16 (32-element blocks along d for P1 and along the rank for P2; the
+ *   same block format as the Q4_0 weights below).
  *   bp       [C]      fp32 predictor bias, may be NULL
  *   W_gate   [F, d]   gate rows (ReGLU only), `wtype`
  *   W_up     [F, d]   up rows, `wtype`
@@ -97,9 +101,13 @@ typedef struct {
   int32_t d;       /* hidden size; multiple of 8 (Q4_0: of 32)            */
   int32_t ffn;     /* neurons per layer                                   */
   int32_t n_hot;   /* hot neurons, rows [0, n_hot); 0 <= n_hot <= ffn     */
-  int32_t rank;    /* predictor rank; multiple of 8                       */
+  int32_t rank;    /* predictor rank (the largest of a stack's layers);
+                      multiple of 8 (Q4_0 predictors: of 32)               */
   pi_dtype wtype;  /* FFN weights: PI_F32, PI_F16 or PI_Q4_0             */
-  pi_dtype ptype;  /* predictor matrices and the token block: F32 or F16 */
+  pi_dtype ptype;  /* predictor matrices: PI_F32 (fp32 token block), PI_F16
+                      or PI_Q4_0 (fp16 token block); PI_Q4_0 needs d % 32 == 0
+                      ([UA] "Adaptif Sparsite Predictor’ları": the predictor's
+                      size is chosen per layer; a Q4_0 one is the smallest) */
   pi_act act;
 } pi_ffn_desc;
 
@@ -120,7 +128,10 @@ typedef struct {
   const float *b1;
   const float *b2;
   float threshold;    /* predictor threshold: neuron c is active iff its score > threshold */
-  int32_t _pad;
+  int32_t rank;       /* this layer's predictor rank, P1 [rank, d] and P2 [C, rank]; 0 = the
+                         descriptor's; else a multiple of 8 (Q4_0: 32) no larger than it
+                         ([UA] "Adaptif Sparsite Predictor’ları": each layer's predictor has its
+                         own size) */
 } pi_layer_weights;
 
 /* Maximum token-block size accepted by every call. */
@@ -209,12 +220,14 @@ PI_API pi_status pi_residual_rmsnorm(int32_t batch, int32_t d, pi_dtype htype, c
  * device pointers are baked into the launch, so a captured CUDA graph keeps
  * them).  idx: [n_layers, C] int32; counts: [n_layers] int32; y: optional
  * [n_layers, B, d] fp32 (NULL: not kept); h_trace: optional [n_layers, B, d]
- * ptype receiving each layer's input h_l (NULL: not kept).  h_out [B, d]
- * ptype must not alias h_in.  All layers share one descriptor;
+ * in the token type, receiving each layer's input h_l (NULL: not kept).
+ * h_in and h_out [B, d] are in the token type; h_out must not alias h_in.  All layers share one descriptor, except that
+ * each layer may have its own (smaller) predictor rank (layers[l].rank);
  * n_layers <= PI_MAX_LAYERS.
- * Token blocks of 1-2 with fp16/fp16, Q4_0/fp16 or fp32/fp32 weights and
- * predictors run the whole step as one cooperative launch (one CTA per SM;
- * every b1 16-byte aligned, else the per-layer kernels run); larger blocks
+ * Token blocks of 1-2 run the whole step as one cooperative launch (one CTA
+ * per SM) for fp16/fp16, Q4_0/fp16, Q4_0/Q4_0 and fp32/fp32 weights and
+ * predictors, when every b1 is 16-byte aligned and every layer's rank is a
+ * multiple of 16 (fp16 predictors) or 256 (Q4_0 predictors); larger blocks
  * and other shapes run per-layer kernels.  Either way the outputs are
  * complete once the stream reaches the end of the call; one workspace
  * serves one call at a time.

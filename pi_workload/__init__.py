@@ -60,7 +60,7 @@ class Workload:
     layers: int
     act: str          # "relu" | "reglu" | "relu2"
     wtype: str        # "f32" | "f16" | "q4_0"
-    ptype: str        # "f32" | "f16" (predictor and token dtype)
+    ptype: str        # "f32" | "f16" | "q4_0" (predictor dtype; tokens are fp32 with fp32 predictors, else fp16)
     sparsity: float
     alpha: float
     hot_frac: float
@@ -69,6 +69,8 @@ class Workload:
     steps: int
     has_b2: bool = False
     thr: float = THRESHOLD
+    # per-layer predictor ranks (layer l takes rank_steps[l % len]); empty: every layer has `rank`
+    rank_steps: tuple = ()
 
     @property
     def n_hot(self) -> int:
@@ -81,6 +83,20 @@ class Workload:
     @property
     def gated(self) -> bool:
         return self.act == "reglu"
+
+    @property
+    def htype(self) -> str:
+        """Token-block dtype: fp32 with fp32 predictors, fp16 otherwise."""
+        return "f32" if self.ptype == "f32" else "f16"
+
+    def layer_rank(self, layer: int) -> int:
+        """Predictor rank of a layer ([UA] "Adaptif Sparsite Predictor’ları":
+        the predictor's size is chosen per layer); never above `rank`."""
+        if not self.rank_steps:
+            return self.rank
+        r = int(self.rank_steps[layer % len(self.rank_steps)])
+        assert 0 < r <= self.rank
+        return r
 
     def with_(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -166,6 +182,25 @@ def quantize_q4_0(x: torch.Tensor):
     return qs, sc
 
 
+def pack_q4_0(x: torch.Tensor):
+    """Q4_0 planes of a [rows, cols] matrix in ONE buffer, scales after the
+    codes (the C ABI's layout of a Q4_0 predictor matrix); returns the pair
+    (qs, sc) of views into that buffer."""
+    qs, sc = quantize_q4_0(x.to(torch.float16))
+    n = qs.numel()
+    buf = torch.empty(n + 2 * sc.numel(), dtype=torch.uint8, device=x.device)
+    buf[:n] = qs.reshape(-1)
+    buf[n:] = sc.reshape(-1).view(torch.uint8)
+    rows, cols = x.shape
+    return buf[:n].view(rows, cols // 2), buf[n:].view(torch.float16).view(rows, cols // 32)
+
+
+def _as_ptype(x: torch.Tensor, ptype: str):
+    if ptype == "q4_0":
+        return pack_q4_0(x)
+    return x.to(_TORCH_DT[ptype]).contiguous()
+
+
 def _as_wtype(x: torch.Tensor, wtype: str):
     if wtype == "q4_0":
         return quantize_q4_0(x.to(torch.float16))
@@ -179,7 +214,7 @@ def make_layer(w: Workload, layer: int, device="cpu") -> dict:
     b1 fp32 [ffn], b2 fp32 [d] or None, P1 [rank, d], P2 [n_cold, rank], bp fp32
     [n_cold], perm int64 [ffn], p fp64 [ffn] (storage order), thr.
     """
-    d, F, r = w.d, w.ffn, w.rank
+    d, F, r = w.d, w.ffn, w.layer_rank(layer)
     assert r % 2 == 0
     rh = r // 2
     p_orig, perm = neuron_layout(w, layer)
@@ -234,10 +269,10 @@ def make_layer(w: Workload, layer: int, device="cpu") -> dict:
     del WdT
     out["b1"] = b1
     out["b2"] = b2
-    pt = _TORCH_DT[w.ptype]
-    out["P1"] = torch.cat([V, -V], dim=0).to(pt).contiguous()
+    out["P1"] = _as_ptype(torch.cat([V, -V], dim=0), w.ptype)
     U_cold = U[perm_t[w.n_hot:]]
-    out["P2"] = torch.cat([U_cold, -U_cold], dim=1).to(pt).contiguous()
+    out["P2"] = _as_ptype(torch.cat([U_cold, -U_cold], dim=1), w.ptype) if w.n_cold > 0 else None
+    out["rank"] = r
     out["bp"] = (b1[w.n_hot:] + w.thr).float().contiguous()
     return out
 
@@ -247,7 +282,7 @@ def make_tokens(w: Workload, batch: int, step: int, device="cpu") -> torch.Tenso
     g = _gen(device, _seed(w, 0xF0, step))
     h = torch.randn(batch, w.d, generator=g, device=device, dtype=torch.float64)
     h = h * (math.sqrt(w.d) / h.norm(dim=1, keepdim=True))
-    return h.to(_TORCH_DT[w.ptype]).contiguous()
+    return h.to(_TORCH_DT[w.htype]).contiguous()
 
 
 def make_int_layer(d: int, ffn: int, n_hot: int, rank: int, act: str, wtype: str, ptype: str, batch: int,
@@ -294,19 +329,22 @@ def make_int_layer(d: int, ffn: int, n_hot: int, rank: int, act: str, wtype: str
     return out
 
 
-def layer_bytes(w: Workload, batch: int, n_active: float) -> float:
+def layer_bytes(w: Workload, batch: int, n_active: float, rank: Optional[int] = None) -> float:
     """Algorithmic bytes one layer must move for one token block with n_active
-    predicted-active cold neurons: both predictor matrices, the listed weight
-    rows (hot + active), their biases, the index list, and the token block in
-    and the fp32 output out."""
-    e_p = 4 if w.ptype == "f32" else 2
-    e_w = {"f32": 4.0, "f16": 2.0, "q4_0": 18.0 / 32.0}[w.wtype]
+    predicted-active cold neurons: both predictor matrices (of the layer's
+    rank), the listed weight rows (hot + active), their biases, the index
+    list, and the token block in and the fp32 output out."""
+    e = {"f32": 4.0, "f16": 2.0, "q4_0": 18.0 / 32.0}
+    e_p = e[w.ptype]
+    e_h = 4 if w.htype == "f32" else 2
+    e_w = e[w.wtype]
+    r = w.rank if rank is None else rank
     mats = 3 if w.gated else 2
     n_list = w.n_hot + n_active
-    pred = (w.rank * w.d + w.n_cold * w.rank) * e_p + 4 * w.n_cold          # P1, P2, bp
+    pred = (r * w.d + w.n_cold * r) * e_p + 4 * w.n_cold                   # P1, P2, bp
     ffn = mats * n_list * w.d * e_w + 4 * n_list                           # rows + b1
     idx = 4 * n_active
-    io = batch * w.d * e_p + batch * w.d * 4 + (4 * w.d if (w.has_b2 or not w.gated) else 0)
+    io = batch * w.d * e_h + batch * w.d * 4 + (4 * w.d if (w.has_b2 or not w.gated) else 0)
     return pred + ffn + idx + io
 
 
