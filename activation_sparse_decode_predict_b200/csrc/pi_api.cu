@@ -234,7 +234,9 @@ pi_status fused_params(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, pi:
   const int ep = desc->ptype == PI_F16 ? 2 : 4;
   const size_t wrow = desc->wtype == PI_Q4_0 ? desc->d / 2 + desc->d / 16
                                               : (size_t)desc->d * (desc->wtype == PI_F16 ? 2 : 4);
-  const size_t neuron = (wrow + 16) * (desc->act == PI_ACT_REGLU ? 3 : 2) + 16 + 256;
+  // ring bytes of one neuron (a whole item, or its gate/up and down items)
+  const size_t neuron = pi::kSplitGU ? (wrow + 16) * (desc->act == PI_ACT_REGLU ? 3 : 2) + 2 * (16 + 256)
+                                     : (wrow + 16) * (desc->act == PI_ACT_REGLU ? 3 : 2) + 16 + 256;
   // predictor items (the largest rank): fp16 predictors go to the tensor cores
   // in 16-row tiles with padded rows; Q4_0 rows carry codes and scales
   const size_t p2item = desc->ptype == PI_F16    ? (size_t)16 * (2 * desc->rank + 16) + 256

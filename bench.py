@@ -73,6 +73,8 @@ def parse():
     ap.add_argument("--workload", default="70b-reglu-fp16", choices=sorted(W.WORKLOADS))
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--sparsity", type=float, default=None)
+    ap.add_argument("--ptype", default=None, choices=["f16", "q4_0"],
+                    help="predictor dtype instead of the workload's (q4_0: a quantised predictor, fp16 tokens)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=None, help="run fewer layers (smoke only; not a bench number)")
@@ -212,6 +214,8 @@ def run_ours(args, rank, world, local_rank):
     wl = W.WORKLOADS[args.workload]
     if args.sparsity is not None:
         wl = wl.with_(sparsity=args.sparsity)
+    if args.ptype is not None:
+        wl = wl.with_(ptype=args.ptype)
     B = args.batch or wl.batches[0]
     n_layers = args.layers or wl.layers
     desc = pi.desc_for(wl)
@@ -281,7 +285,7 @@ def run_ours(args, rank, world, local_rank):
 
     # end to end through the public API with host buffers: H2D of the step's
     # token block from pinned memory, the stack call, D2H of the result.
-    h_host = h_pool.cpu().pin_memory()
+    h_host = h_pool.cpu().pin_memory()  # token block in its own dtype (fp16 unless fp32 predictors)
     out_host = torch.empty(B, wl.d, dtype=h_pool.dtype).pin_memory()
     h_dev_in = torch.empty(B, wl.d, dtype=h_pool.dtype, device=dev)
     e_steps = min(args.steps, E2E_STEPS)
@@ -323,6 +327,7 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic (seeded Zipf-activity weights, low-rank predictor, RMS-normalised tokens)",
         "config": {"workload": wl.name, "d": wl.d, "ffn": wl.ffn, "layers": n_layers, "batch": B,
                    "sparsity": wl.sparsity, "hot": wl.n_hot, "rank": wl.rank, "act": wl.act, "weights": wl.wtype,
+                   "predictor": wl.ptype,
                    "parallelism": "replicas" if world > 1 else "single",
                    "l2": "no flush: resident stack %.1f GB, %.2f GB streamed per step (L2 126 MB)" % (
                        _resident_bytes(layers) / 1e9, total_bytes / args.steps / 1e9),
@@ -429,6 +434,8 @@ def run_reference(args):
     wl = W.WORKLOADS[args.workload]
     if args.sparsity is not None:
         wl = wl.with_(sparsity=args.sparsity)
+    if args.ptype is not None:
+        wl = wl.with_(ptype=args.ptype)
     B = args.batch or wl.batches[0]
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     n_sample = 2
