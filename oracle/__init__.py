@@ -54,6 +54,9 @@ def _bind(path: str):
     lib.orc_masked_ffn.restype = None
     lib.orc_true_support.argtypes = [i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P]
     lib.orc_true_support.restype = None
+    lib.orc_attention.argtypes = [i32, i32, i32, i32, i32, i32, i32, P, P, i64, P, P, P, P, P, P, i32, i32, P, P,
+                                  P]
+    lib.orc_attention.restype = None
     lib.orc_residual_rmsnorm.argtypes = [i32, i32, i32, P, P, f64, P]
     lib.orc_residual_rmsnorm.restype = None
     lib.orc_set_threads.argtypes = [i32]
@@ -222,6 +225,31 @@ def true_support(h, Wg, Wu, b1, act: str, ffn: int) -> np.ndarray:
     lib.orc_true_support(d, ffn, _wtype_of(Wu), ACTS[act], _htype(h), B, _ptr(h), _ptr(wg), _ptr(wg_sc), _ptr(wu),
                          _ptr(wu_sc), _ptr(b1_), _ptr(out))
     return out
+
+
+def attention(x, idx, Wq, Wk, Wv, WoT, K, V, length: int, n_heads: int, n_hot: int):
+    """Head-sparse decode attention over the heads [0, n_hot) ++ idx: dict(y [B, d],
+    k [B, n_list, dh], v [B, n_list, dh]) in float64.  K, V: caches [B, n_heads, s_max, dh]."""
+    lib = _load()
+    x = np.ascontiguousarray(x)
+    B, d = x.shape
+    idx = np.ascontiguousarray(np.asarray(idx, dtype=np.int32))
+    K = np.ascontiguousarray(K)
+    V = np.ascontiguousarray(V)
+    assert K.shape == V.shape and K.shape[0] == B and K.shape[1] == n_heads and K.shape[3] == d // n_heads
+    assert 0 <= length <= K.shape[2]
+    wt = _htype(Wq)
+    for w in (Wk, Wv, WoT):
+        assert _htype(w) == wt and w.shape == (d, d)
+    n_list = n_hot + len(idx)
+    dh = d // n_heads
+    y = np.empty((B, d), np.float64)
+    k = np.empty((B, max(n_list, 1), dh), np.float64)
+    v = np.empty((B, max(n_list, 1), dh), np.float64)
+    lib.orc_attention(d, n_heads, n_hot, wt, _htype(x), _htype(K), B, _ptr(x), _ptr(idx), len(idx), _ptr(Wq),
+                      _ptr(Wk), _ptr(Wv), _ptr(WoT), _ptr(K), _ptr(V), K.shape[2], int(length), _ptr(y), _ptr(k),
+                      _ptr(v))
+    return {"y": y, "k": k[:, :n_list], "v": v[:, :n_list]}
 
 
 def residual_rmsnorm(h, y, eps: float) -> np.ndarray:

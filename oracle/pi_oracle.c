@@ -251,6 +251,96 @@ void orc_true_support(int d, int ffn, int wtype, int act, int htype, int batch, 
 }
 
 /*
+ * Head-sparse decode self-attention ([UA] "Adaptif Sparsite Predictor’ları":
+ * besides the FFN predictor, each layer has a predictor for its
+ * self-attention block; only the heads it picks are computed).  One decode
+ * step of `batch` independent sequences, multi-head attention with n_heads
+ * heads of dh = d / n_heads dimensions:
+ *   heads = [0, n_hot) ++ idx[0, count)   (always-computed heads, then the predicted ones)
+ *   for every listed head h and token b (rows h*dh .. h*dh+dh-1 of Wq, Wk, Wv, WoT):
+ *     q = Wq[h] x_b,  k = Wk[h] x_b,  v = Wv[h] x_b
+ *     score_t = q . K[b,h,t] / sqrt(dh) for t < len,  score_len = q . k / sqrt(dh)
+ *     p = softmax(score_0 .. score_len)
+ *     o = sum_{t < len} p_t V[b,h,t] + p_len v
+ *     y_b += sum_i o_i WoT[h*dh + i, :]
+ * The new position uses this step's k and v themselves (the caller's cache
+ * keeps them in its own type).  Caches K, V: [batch, n_heads, s_max, dh] of
+ * type ctype; positions 0 .. len-1 are read.  Heads are added in list order,
+ * every other sum in ascending index order.  k_out / v_out (optional):
+ * [batch, n_list, dh], the new k and v of each listed head.
+ */
+void orc_attention(int d, int n_heads, int n_hot, int wtype, int htype, int ctype, int batch, const void *x,
+                   const int32_t *idx, int64_t count, const void *Wq, const void *Wk, const void *Wv,
+                   const void *WoT, const void *Kc, const void *Vc, int s_max, int len, double *y_out,
+                   double *k_out, double *v_out) {
+  const int dh = d / n_heads;
+  const int64_t n_list = (int64_t)n_hot + count;
+  const double scale = 1.0 / sqrt((double)dh);
+  double *xd = decode_tokens(htype, x, batch, d);
+  double *o = (double *)malloc(sizeof(double) * (size_t)batch * (size_t)(n_list > 0 ? n_list : 1) * (size_t)dh);
+  for (int b = 0; b < batch; ++b) {
+#pragma omp parallel for schedule(static)
+    for (int64_t p = 0; p < n_list; ++p) {
+      const int64_t h = p < n_hot ? p : (int64_t)idx[p - n_hot];
+      const double *xb = xd + (size_t)b * d;
+      double *q = (double *)malloc(sizeof(double) * (size_t)dh * 3);
+      double *k = q + dh, *v = q + 2 * dh;
+      for (int i = 0; i < dh; ++i) {
+        double aq = 0.0, ak = 0.0, av = 0.0;
+        for (int e = 0; e < d; ++e) {
+          aq += orc_elem(wtype, Wq, NULL, h * dh + i, e, d) * xb[e];
+          ak += orc_elem(wtype, Wk, NULL, h * dh + i, e, d) * xb[e];
+          av += orc_elem(wtype, Wv, NULL, h * dh + i, e, d) * xb[e];
+        }
+        q[i] = aq;
+        k[i] = ak;
+        v[i] = av;
+      }
+      double *sc = (double *)malloc(sizeof(double) * (size_t)(len + 1));
+      const int64_t crow = ((int64_t)b * n_heads + h) * s_max;
+      for (int t = 0; t <= len; ++t) {
+        double acc = 0.0;
+        for (int i = 0; i < dh; ++i) acc += q[i] * (t < len ? orc_elem(ctype, Kc, NULL, crow + t, i, dh) : k[i]);
+        sc[t] = acc * scale;
+      }
+      double m = sc[0];
+      for (int t = 1; t <= len; ++t) m = sc[t] > m ? sc[t] : m;
+      double sum = 0.0;
+      for (int t = 0; t <= len; ++t) {
+        sc[t] = exp(sc[t] - m);
+        sum += sc[t];
+      }
+      double *ob = o + ((size_t)b * n_list + p) * dh;
+      for (int i = 0; i < dh; ++i) {
+        double acc = 0.0;
+        for (int t = 0; t <= len; ++t) acc += sc[t] * (t < len ? orc_elem(ctype, Vc, NULL, crow + t, i, dh) : v[i]);
+        ob[i] = acc / sum;
+      }
+      if (k_out)
+        for (int i = 0; i < dh; ++i) k_out[((size_t)b * n_list + p) * dh + i] = k[i];
+      if (v_out)
+        for (int i = 0; i < dh; ++i) v_out[((size_t)b * n_list + p) * dh + i] = v[i];
+      free(sc);
+      free(q);
+    }
+  }
+  for (int b = 0; b < batch; ++b) {
+#pragma omp parallel for schedule(static)
+    for (int e = 0; e < d; ++e) {
+      double acc = 0.0;
+      for (int64_t p = 0; p < n_list; ++p) {
+        const int64_t h = p < n_hot ? p : (int64_t)idx[p - n_hot];
+        for (int i = 0; i < dh; ++i)
+          acc += o[((size_t)b * n_list + p) * dh + i] * orc_elem(wtype, WoT, NULL, h * dh + i, e, d);
+      }
+      y_out[(size_t)b * d + e] = acc;
+    }
+  }
+  free(xd);
+  free(o);
+}
+
+/*
  * Stack glue between layers (the pages are silent; residual + RMSNorm with
  * unit gain): x = h + y;  out = x / sqrt(mean_e x[e]^2 + eps).
  */

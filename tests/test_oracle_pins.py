@@ -479,3 +479,119 @@ def test_q4_0_predictor_equals_its_fp16_twin():
     b = oracle.predict(h, P1x, P2x, bp, 0.5, n_hot, ffn)
     assert np.array_equal(a["u"], b["u"]) and np.array_equal(a["s"], b["s"])
     assert np.array_equal(a["idx"], b["idx"]) and 0 < len(a["idx"]) < ffn - n_hot
+
+
+# ----------------------------------------------------------------------------
+# head-sparse decode attention (the self-attention predictor's operator)
+
+
+def _attn_golden():
+    g = read("attention_d4_h2.txt")
+    d, H, n = int(g["d"]), int(g["n_heads"]), int(g["len"])
+    W = {k: mat(g[k]).astype(np.float32) for k in ("Wq", "Wk", "Wv", "WoT")}
+    x = mat(g["x"]).astype(np.float32).reshape(1, d)
+    K = np.zeros((1, H, 4, d // H), np.float32)
+    V = np.zeros((1, H, 4, d // H), np.float32)
+    K[0, :, 0] = mat(g["K0"])
+    V[0, :, 0] = mat(g["V0"])
+    return g, d, H, n, W, x, K, V
+
+
+def test_attention_golden_per_head_and_union():
+    g, d, H, n, W, x, K, V = _attn_golden()
+    r0 = oracle.attention(x, [0], W["Wq"], W["Wk"], W["Wv"], W["WoT"], K, V, n, H, 0)
+    assert np.array_equal(r0["y"][0], mat(g["y_head0"]))
+    assert np.array_equal(r0["k"][0, 0], mat(g["k_head0"])) and np.array_equal(r0["v"][0, 0], mat(g["v_head0"]))
+    r1 = oracle.attention(x, [1], W["Wq"], W["Wk"], W["Wv"], W["WoT"], K, V, n, H, 0)
+    assert np.array_equal(r1["y"][0], mat(g["y_head1"]))
+    both = oracle.attention(x, [1], W["Wq"], W["Wk"], W["Wv"], W["WoT"], K, V, n, H, 1)   # head 0 hot, 1 listed
+    assert np.array_equal(both["y"][0], mat(g["y_both"]))
+    assert oracle.attention(x, [], W["Wq"], W["Wk"], W["Wv"], W["WoT"], K, V, n, H, 0)["y"].tolist() == [[0, 0, 0, 0]]
+
+
+def _attn_rand(rng, B, d, H, s_max, dtype=np.float16):
+    W = {k: (rng.standard_normal((d, d)) / np.sqrt(d)).astype(dtype) for k in ("Wq", "Wk", "Wv", "WoT")}
+    x = _tokens(rng, B, d).astype(dtype)
+    K = rng.standard_normal((B, H, s_max, d // H)).astype(dtype)
+    V = rng.standard_normal((B, H, s_max, d // H)).astype(dtype)
+    return W, x, K, V
+
+
+def test_attention_empty_cache_is_the_value_projection():
+    """len = 0: the new token attends to itself alone (softmax of one score is
+    1), so each head's output is its own v and y = sum_h WoT[h]^T v_h."""
+    rng = np.random.default_rng(41)
+    B, d, H = 2, 32, 4
+    W, x, K, V = _attn_rand(rng, B, d, H, 3)
+    r = oracle.attention(x, [1, 3], W["Wq"], W["Wk"], W["Wv"], W["WoT"], K, V, 0, H, 0)
+    dh = d // H
+    Wv, WoT = W["Wv"].astype(np.float64), W["WoT"].astype(np.float64)
+    xd = x.astype(np.float64)
+    for b in range(B):
+        ref = sum(WoT[h * dh:(h + 1) * dh].T @ (Wv[h * dh:(h + 1) * dh] @ xd[b]) for h in (1, 3))
+        assert np.allclose(r["y"][b], ref, rtol=0, atol=1e-12)
+
+
+def test_attention_equal_scores_average_the_values():
+    """Wq = 0: every score is 0, p is uniform over the len + 1 positions, and
+    o is the mean of the cached values and the new v."""
+    rng = np.random.default_rng(42)
+    B, d, H, n = 1, 16, 2, 5
+    W, x, K, V = _attn_rand(rng, B, d, H, 8)
+    W["Wq"][:] = 0
+    r = oracle.attention(x, [0, 1], W["Wq"], W["Wk"], W["Wv"], W["WoT"], K, V, n, H, 0)
+    dh = d // H
+    for h in range(H):
+        o = (V[0, h, :n].astype(np.float64).sum(axis=0) + r["v"][0, h]) / (n + 1)
+        y_h = W["WoT"][h * dh:(h + 1) * dh].astype(np.float64).T @ o
+        y_one = oracle.attention(x, [h], W["Wq"], W["Wk"], W["Wv"], W["WoT"], K, V, n, H, 0)["y"][0]
+        assert np.allclose(y_one, y_h, rtol=0, atol=1e-12)
+
+
+def test_attention_is_additive_over_heads_and_invariant_to_cache_order():
+    """Heads contribute independently (y of a set = sum of single heads, up
+    to rounding); permuting the cached positions (K and V together) leaves
+    every head's softmax-weighted average unchanged; listing a head as hot
+    or as predicted gives the same y."""
+    rng = np.random.default_rng(43)
+    B, d, H, n = 2, 32, 4, 6
+    W, x, K, V = _attn_rand(rng, B, d, H, 9)
+    args = (W["Wq"], W["Wk"], W["Wv"], W["WoT"])
+    y = oracle.attention(x, [0, 2, 3], *args, K, V, n, H, 0)["y"]
+    parts = sum(oracle.attention(x, [h], *args, K, V, n, H, 0)["y"] for h in (0, 2, 3))
+    assert np.allclose(y, parts, rtol=0, atol=1e-12)
+    perm = rng.permutation(n)
+    Kp, Vp = K.copy(), V.copy()
+    Kp[:, :, :n] = K[:, :, perm]
+    Vp[:, :, :n] = V[:, :, perm]
+    assert np.allclose(oracle.attention(x, [0, 2, 3], *args, Kp, Vp, n, H, 0)["y"], y, rtol=0, atol=1e-12)
+    assert np.array_equal(oracle.attention(x, [2, 3], *args, K, V, n, H, 1)["y"],
+                          oracle.attention(x, [0, 2, 3], *args, K, V, n, H, 0)["y"])
+    # positions past len are never read
+    K2, V2 = K.copy(), V.copy()
+    K2[:, :, n:] = 1e4
+    V2[:, :, n:] = -1e4
+    assert np.array_equal(oracle.attention(x, [0, 2, 3], *args, K2, V2, n, H, 0)["y"], y)
+
+
+def test_attention_two_positions_is_a_logistic_of_the_scaled_score():
+    """One cached position with key K0 and a new token whose k and v are 0:
+    the softmax over two scores reduces to p0 = 1 / (1 + exp(-q.K0 / sqrt(dh))),
+    so o = p0 V0 -- this fixes the 1/sqrt(dh) scale."""
+    d, H = 8, 2
+    dh = d // H
+    x = np.zeros((1, d), np.float32)
+    x[0, 0] = 1.0
+    Wq = np.zeros((d, d), np.float32)
+    Wq[0, 0] = 3.0                      # head 0: q = [3, 0, 0, 0]
+    Wk = np.zeros((d, d), np.float32)   # k_new = 0
+    Wv = np.zeros((d, d), np.float32)   # v_new = 0
+    WoT = np.eye(d, dtype=np.float32)   # y = o of head 0 in columns 0..3
+    K = np.zeros((1, H, 2, dh), np.float32)
+    V = np.zeros((1, H, 2, dh), np.float32)
+    K[0, 0, 0] = [1.0, 0, 0, 0]
+    V[0, 0, 0] = [2.0, -1.0, 0, 0.5]
+    r = oracle.attention(x, [0], Wq, Wk, Wv, WoT, K, V, 1, H, 0)
+    p0 = 1.0 / (1.0 + math.exp(-3.0 / math.sqrt(dh)))
+    assert np.allclose(r["y"][0, :dh], p0 * V[0, 0, 0].astype(np.float64), rtol=0, atol=1e-15)
+    assert np.all(r["y"][0, dh:] == 0)
