@@ -19,7 +19,7 @@ from typing import Optional, Sequence, Tuple, Union
 import torch
 
 from . import _binding as _b
-from ._binding import ACTS, DTYPES, EXPORTS, MAX_BATCH, FfnDesc, LayerWeights, PiError, Weight
+from ._binding import ACTS, DTYPES, EXPORTS, MAX_BATCH, AttnDesc, FfnDesc, LayerWeights, PiError, Weight
 
 _lib = None
 
@@ -166,6 +166,30 @@ def device_status(ws: torch.Tensor, clear: bool = False, stream=None) -> int:
 def selftest_bounded_wait(ws: torch.Tensor, kind: int, stream=None) -> None:
     """Launch a wait that can only time out (kind 0: mbarrier, 1: grid barrier)."""
     _check(lib().pi_selftest_bounded_wait(_ptr(ws), int(kind), _stream(stream)))
+
+
+def attn_desc(d: int, n_heads: int, n_hot: int, s_max: int, wtype: str = "f16", xtype: str = "f16",
+              ctype: str = "f16") -> AttnDesc:
+    return AttnDesc(d, n_heads, n_hot, s_max, DTYPES[wtype], DTYPES[xtype], DTYPES[ctype])
+
+
+def attn_workspace(desc: AttnDesc, batch: int, device=None, stream=None) -> torch.Tensor:
+    """A zero-initialised workspace for pi_sparse_attention (allocated by torch)."""
+    n = lib().pi_attn_workspace_bytes(ctypes.byref(desc), int(batch))
+    if n == 0:
+        raise PiError(_b.PI_ERR_INVALID_ARG, lib().pi_last_error().decode())
+    ws = torch.empty(int(n), dtype=torch.uint8, device=device or "cuda")
+    _check(lib().pi_workspace_init(_ptr(ws), int(n), _stream(stream)))
+    return ws
+
+
+def sparse_attention(desc: AttnDesc, x: torch.Tensor, head_idx, head_count: torch.Tensor, Wq, Wk, Wv, WoT,
+                     K: torch.Tensor, V: torch.Tensor, length: int, y: torch.Tensor, ws: torch.Tensor,
+                     stream=None) -> None:
+    """One decode step of the self-attention block over the listed heads (pi_sparse_attention)."""
+    _check(lib().pi_sparse_attention(ctypes.byref(desc), x.shape[0], _ptr(x), _ptr(head_idx), _ptr(head_count),
+                                     _ptr(Wq), _ptr(Wk), _ptr(Wv), _ptr(WoT), _ptr(K), _ptr(V), int(length), _ptr(y),
+                                     _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def version() -> str:

@@ -23,7 +23,9 @@ MAX_BATCH = 16
 
 # Every symbol include/pi.h declares.
 EXPORTS = ("pi_workspace_bytes", "pi_workspace_init", "pi_predict", "pi_sparse_ffn", "pi_layer",
-           "pi_residual_rmsnorm", "pi_decode_stack", "pi_stack_launches", "pi_get_device_status", "pi_predict_static", "pi_selftest_bounded_wait", "pi_last_error", "pi_version")
+           "pi_residual_rmsnorm", "pi_decode_stack", "pi_stack_launches", "pi_get_device_status",
+           "pi_attn_workspace_bytes", "pi_sparse_attention", "pi_predict_static", "pi_selftest_bounded_wait",
+           "pi_last_error", "pi_version")
 
 
 class FfnDesc(ctypes.Structure):
@@ -40,6 +42,11 @@ class LayerWeights(ctypes.Structure):
                 ("W_gate", Weight), ("W_up", Weight), ("W_downT", Weight),
                 ("b1", ctypes.c_void_p), ("b2", ctypes.c_void_p), ("threshold", ctypes.c_float),
                 ("rank", ctypes.c_int32)]
+
+
+class AttnDesc(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int32), ("n_heads", ctypes.c_int32), ("n_hot", ctypes.c_int32),
+                ("s_max", ctypes.c_int32), ("wtype", ctypes.c_int), ("xtype", ctypes.c_int), ("ctype", ctypes.c_int)]
 
 
 class PiError(RuntimeError):
@@ -73,6 +80,11 @@ def load(path: str = LIB_PATH):
     lib.pi_stack_launches.restype = i32
     lib.pi_get_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32), i32, P]
     lib.pi_get_device_status.restype = st
+    A = ctypes.POINTER(AttnDesc)
+    lib.pi_attn_workspace_bytes.argtypes = [A, i32]
+    lib.pi_attn_workspace_bytes.restype = S
+    lib.pi_sparse_attention.argtypes = [A, i32, P, P, P, P, P, P, P, P, P, i32, P, P, S, P]
+    lib.pi_sparse_attention.restype = st
     lib.pi_predict_static.argtypes = [D, i32, P, P, P, P, f32, P, P, P]
     lib.pi_predict_static.restype = st
     lib.pi_selftest_bounded_wait.argtypes = [P, i32, P]

@@ -7,6 +7,7 @@
 
 #include "pi.h"
 #include "pi_args.h"
+#include "pi_attn.cuh"
 #include "pi_batch.cuh"
 #include "pi_common.cuh"
 #include "pi_kernels_v1.cuh"
@@ -201,6 +202,43 @@ pi_ffn_desc layer_desc(const pi_ffn_desc* desc, const pi_layer_weights* w) {
   pi_ffn_desc d = *desc;
   if (w->rank > 0) d.rank = w->rank;
   return d;
+}
+
+pi_status check_attn(const pi_attn_desc* d, int32_t batch) {
+  if (!d) return fail(PI_ERR_INVALID_ARG, "%s", "desc is NULL");
+  if (d->d <= 0 || d->d % 8) return fail(PI_ERR_INVALID_ARG, "%s", "d must be a positive multiple of 8");
+  if (d->n_heads <= 0 || d->d % d->n_heads) return fail(PI_ERR_INVALID_ARG, "%s", "n_heads must divide d");
+  if (!pi::attn_head_dim_ok(d->d / d->n_heads))
+    return fail(PI_ERR_UNSUPPORTED, "%s", "head dimension must be 32, 64, 128 or 256");
+  if (d->n_hot < 0 || d->n_hot > d->n_heads) return fail(PI_ERR_INVALID_ARG, "%s", "n_hot must be in [0, n_heads]");
+  if (d->s_max <= 0) return fail(PI_ERR_INVALID_ARG, "%s", "s_max must be positive");
+  if (d->wtype != PI_F16 && d->wtype != PI_F32) return fail(PI_ERR_INVALID_ARG, "%s", "wtype must be PI_F16 or PI_F32");
+  if (d->xtype != PI_F16 && d->xtype != PI_F32) return fail(PI_ERR_INVALID_ARG, "%s", "xtype must be PI_F16 or PI_F32");
+  if (d->ctype != PI_F16 && d->ctype != PI_F32) return fail(PI_ERR_INVALID_ARG, "%s", "ctype must be PI_F16 or PI_F32");
+  if (d->wtype == PI_F16 && d->xtype == PI_F32)
+    return fail(PI_ERR_UNSUPPORTED, "%s", "fp32 tokens need fp32 weights");
+  if (batch < 1 || batch > PI_MAX_BATCH) return fail(PI_ERR_INVALID_ARG, "%s", "batch must be in [1, 16]");
+  return PI_OK;
+}
+
+// Workspace of pi_sparse_attention: [ctrl][q, k, v of the listed heads][chunk
+// partials][head outputs][W_o^T row list][its count][split-K partial outputs]
+struct AttnLayout {
+  size_t qkv, part, a, orow, ocount, partial, total;
+};
+
+AttnLayout attn_layout(const pi_attn_desc* d, int32_t B) {
+  AttnLayout L;
+  const size_t dh = (size_t)(d->d / d->n_heads);
+  size_t off = pi::kCtrlBytes;
+  L.qkv = off; off += pi::align256((size_t)B * d->n_heads * 3 * dh * 4);
+  L.part = off; off += pi::align256((size_t)B * d->n_heads * pi::kAttnMaxSplit * (dh + 4) * 4);
+  L.a = off; off += pi::align256((size_t)B * d->d * 4);
+  L.orow = off; off += pi::align256((size_t)d->d * 4);
+  L.ocount = off; off += 256;
+  L.partial = off; off += pi::align256((size_t)pi::kGMax * B * d->d * 4);
+  L.total = off;
+  return L;
 }
 
 static_assert(pi::kYAccCopies == pi::kYCopies, "workspace layout and kernel agree on the accumulator copies");
@@ -476,6 +514,60 @@ pi_status pi_decode_stack(const pi_ffn_desc* desc, int32_t batch, int32_t n_laye
     PI_CUDA(pi::launch_rmsnorm(pi::token_type(desc), cur, yl, batch, desc->d, eps, nxt, st), "rmsnorm launch");
     cur = nxt;
   }
+  return PI_OK;
+}
+
+size_t pi_attn_workspace_bytes(const pi_attn_desc* desc, int32_t batch) {
+  if (check_attn(desc, batch) != PI_OK) return 0;
+  return attn_layout(desc, batch).total;
+}
+
+pi_status pi_sparse_attention(const pi_attn_desc* desc, int32_t batch, const void* x, const int32_t* head_idx,
+                              const int32_t* head_count, const void* Wq, const void* Wk, const void* Wv,
+                              const void* WoT, void* K, void* V, int32_t len, float* y, void* ws, size_t ws_bytes,
+                              void* stream) {
+  PI_TRY(check_attn(desc, batch));
+  if (len < 0 || len >= desc->s_max) return fail(PI_ERR_INVALID_ARG, "%s", "len must be in [0, s_max)");
+  PI_TRY(check_ptr(x, 16, "x"));
+  if (desc->n_heads > desc->n_hot) PI_TRY(check_ptr(head_idx, 4, "head_idx"));
+  PI_TRY(check_ptr(head_count, 4, "head_count"));
+  PI_TRY(check_ptr(Wq, 16, "Wq"));
+  PI_TRY(check_ptr(Wk, 16, "Wk"));
+  PI_TRY(check_ptr(Wv, 16, "Wv"));
+  PI_TRY(check_ptr(WoT, 16, "WoT"));
+  PI_TRY(check_ptr(K, 16, "K"));
+  PI_TRY(check_ptr(V, 16, "V"));
+  PI_TRY(check_ptr(y, 16, "y"));
+  PI_TRY(check_ptr(ws, 256, "ws"));
+  const AttnLayout L = attn_layout(desc, batch);
+  if (ws_bytes < L.total) return fail(PI_ERR_CAPACITY, "%s", "workspace smaller than pi_attn_workspace_bytes()");
+  char* w = static_cast<char*>(ws);
+  const int sms = sm_count();
+  pi::AttnParams P;
+  P.d = desc->d;
+  P.n_heads = desc->n_heads;
+  P.n_hot = desc->n_hot;
+  P.B = batch;
+  P.s_max = desc->s_max;
+  P.len = len;
+  P.nsplit = pi::attn_splits(len, batch, desc->n_heads, sms);
+  P.x = x;
+  P.head_idx = head_idx;
+  P.head_count = head_count;
+  P.Wq = Wq;
+  P.Wk = Wk;
+  P.Wv = Wv;
+  P.WoT = WoT;
+  P.K = K;
+  P.V = V;
+  P.qkv = reinterpret_cast<float*>(w + L.qkv);
+  P.part = reinterpret_cast<float*>(w + L.part);
+  P.ctrl = reinterpret_cast<pi::Ctrl*>(w);
+  const int G = 2 * sms < pi::kGMax ? 2 * sms : pi::kGMax;
+  PI_CUDA(pi::launch_attention(P, desc->wtype, desc->xtype, desc->ctype, reinterpret_cast<float*>(w + L.a),
+                               reinterpret_cast<int32_t*>(w + L.orow), reinterpret_cast<int32_t*>(w + L.ocount),
+                               reinterpret_cast<float*>(w + L.partial), G, y, sms, (cudaStream_t)stream),
+          "sparse attention launch");
   return PI_OK;
 }
 

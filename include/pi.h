@@ -250,6 +250,53 @@ PI_API int32_t pi_stack_launches(const pi_ffn_desc *desc, int32_t batch, int32_t
 PI_API pi_status pi_get_device_status(void *ws, int32_t *status_out, int32_t clear, void *stream);
 
 /*
+ * Head-sparse decode self-attention ([UA] "Adaptif Sparsite Predictor’ları":
+ * besides the FFN predictor, each layer has a predictor for its
+ * self-attention block that picks the heads to compute; the other heads are
+ * skipped).  The head predictor is pi_predict itself, with the heads as its
+ * neurons: a pi_ffn_desc {d, ffn = n_heads, n_hot, rank, ..., ptype} (wtype
+ * and act are not used by pi_predict) gives head_idx / head_count.
+ */
+typedef struct {
+  int32_t d;        /* hidden size, multiple of 8                                 */
+  int32_t n_heads;  /* heads; head dimension dh = d / n_heads: 32, 64, 128 or 256 */
+  int32_t n_hot;    /* always-computed heads [0, n_hot); 0 <= n_hot <= n_heads    */
+  int32_t s_max;    /* cache positions per (sequence, head)                      */
+  pi_dtype wtype;   /* Wq, Wk, Wv, WoT: PI_F16 or PI_F32                           */
+  pi_dtype xtype;   /* token block: PI_F16, or PI_F32 with fp32 weights            */
+  pi_dtype ctype;   /* KV cache: PI_F16 or PI_F32                                  */
+} pi_attn_desc;
+
+/* Workspace bytes of pi_sparse_attention for this descriptor and batch (0: invalid). */
+PI_API size_t pi_attn_workspace_bytes(const pi_attn_desc *desc, int32_t batch);
+
+/*
+ * pi_sparse_attention -- one decode step of the self-attention block over the
+ * heads [0, n_hot) ++ head_idx[0, *head_count), for a token block of `batch`
+ * independent sequences, each with its own cache of `len` positions:
+ *     for every listed head h and token b (rows h*dh .. h*dh+dh-1 of each matrix):
+ *         q = Wq[h] x_b,  k = Wk[h] x_b,  v = Wv[h] x_b          (fp32)
+ *         p = softmax over t = 0..len of q.K[b,h,t] / sqrt(dh), with
+ *             K[b,h,len] = k (this step's own k and v are used as computed)
+ *         o = sum_t p_t V[b,h,t]
+ *         y_b += sum_i o_i WoT[h*dh + i, :]
+ *     and k, v are stored (rounded to ctype) at K[b,h,len], V[b,h,len].
+ * Unlisted heads are not computed and their cache rows are not written.
+ *   x [B, d] xtype; Wq, Wk, Wv [d, d] wtype (head-major rows); WoT [d, d]
+ *   wtype = W_o transposed (row h*dh + i is column h*dh + i of W_o);
+ *   K, V [B, n_heads, s_max, dh] ctype; 0 <= len < s_max (host value);
+ *   head_idx [n_heads - n_hot] int32 (may be NULL when n_hot == n_heads);
+ *   head_count: device int32 scalar; y [B, d] fp32 (overwritten).
+ * A listed head outside [n_hot, n_heads) sets PI_ERR_INDEX in the workspace
+ * status word and is skipped; a count above n_heads - n_hot sets
+ * PI_ERR_CAPACITY and is clamped.
+ */
+PI_API pi_status pi_sparse_attention(const pi_attn_desc *desc, int32_t batch, const void *x,
+                                     const int32_t *head_idx, const int32_t *head_count, const void *Wq,
+                                     const void *Wk, const void *Wv, const void *WoT, void *K, void *V,
+                                     int32_t len, float *y, void *ws, size_t ws_bytes, void *stream);
+
+/*
  * pi_predict_static -- pi_predict for callers that cannot allocate device
  * memory.  The paper has no counterpart to this call; it exists for hosts
  * that hand the library only its inputs and outputs (plugin interfaces that

@@ -353,3 +353,29 @@ def expected_active(w: Workload, batch: int) -> float:
     p_rank = zipf_probs(w.ffn, w.alpha, 1.0 - w.sparsity)
     cold = p_rank[w.n_hot:]
     return float(np.sum(1.0 - (1.0 - cold) ** batch))
+
+
+def make_attention(d: int, n_heads: int, n_hot: int, rank: int, batch: int, s_max: int, seed: int,
+                   wtype: str = "f16", ctype: str = "f16", device="cpu") -> dict:
+    """Inputs of one head-sparse attention step: Wq, Wk, Wv, WoT [d, d] with
+    rows of variance 1/d (head h = rows h*dh .. h*dh+dh-1), caches K, V
+    [batch, n_heads, s_max, dh] ~ N(0, 1), and a head predictor built like
+    the FFN's (P1 = [V; -V], P2 = [U, -U] for the cold heads, bp = thr), so
+    each cold head's score sits around the threshold and about half of them
+    are active for a token."""
+    g = _gen(device, seed)
+    dh = d // n_heads
+    wdt = _TORCH_DT[wtype]
+    out = {}
+    for k in ("Wq", "Wk", "Wv", "WoT"):
+        out[k] = (torch.randn(d, d, generator=g, device=device) / math.sqrt(d)).to(wdt).contiguous()
+    for k in ("K", "V"):
+        out[k] = torch.randn(batch, n_heads, s_max, dh, generator=g, device=device).to(_TORCH_DT[ctype]).contiguous()
+    rh = rank // 2
+    U = torch.randn(n_heads - n_hot, rh, generator=g, device=device) * math.sqrt(RHO / rh)
+    V = torch.randn(rh, d, generator=g, device=device) / math.sqrt(d)
+    out["P1"] = torch.cat([V, -V], dim=0).to(torch.float16).contiguous()
+    out["P2"] = torch.cat([U, -U], dim=1).to(torch.float16).contiguous() if n_heads > n_hot else None
+    out["bp"] = torch.full((n_heads - n_hot,), THRESHOLD, dtype=torch.float32, device=device)
+    out["thr"] = THRESHOLD
+    return out

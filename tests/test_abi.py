@@ -165,3 +165,26 @@ def test_static_predict_checks_like_predict_before_any_launch():
     bad_act = _desc(d=512, ffn=2048, n_hot=100, rank=64)
     bad_act.act = 7
     assert call(desc=bad_act) == B.PI_ERR_INVALID_ARG
+
+
+def test_sparse_attention_checks_before_any_launch():
+    """pi_sparse_attention's descriptor, length and pointer checks run on the
+    host; the fake addresses below are never dereferenced."""
+    lib = pi.lib()
+    fake = ctypes.c_void_p(1 << 20)
+    good = pi.attn_desc(4096, 32, 4, 512)
+    assert lib.pi_attn_workspace_bytes(ctypes.byref(good), 1) > 0
+    assert lib.pi_attn_workspace_bytes(ctypes.byref(good), 17) == 0
+
+    def call(desc, length=10, x=fake, hidx=fake, y=fake, ws_bytes=1 << 40):
+        return lib.pi_sparse_attention(ctypes.byref(desc), 1, x, hidx, fake, fake, fake, fake, fake, fake, fake,
+                                       length, y, fake, ws_bytes, None)
+
+    assert call(pi.attn_desc(96, 2, 0, 16)) == B.PI_ERR_UNSUPPORTED          # head dimension 48
+    assert call(pi.attn_desc(4096, 3, 0, 16)) == B.PI_ERR_INVALID_ARG        # 3 does not divide 4096
+    assert call(pi.attn_desc(512, 4, 0, 16, "f16", "f32")) == B.PI_ERR_UNSUPPORTED  # fp32 tokens, fp16 weights
+    assert call(good, length=512) == B.PI_ERR_INVALID_ARG                    # len must be < s_max
+    assert call(good, length=-1) == B.PI_ERR_INVALID_ARG
+    assert call(good, x=ctypes.c_void_p((1 << 20) + 8)) == B.PI_ERR_INVALID_ARG and b"x" in lib.pi_last_error()
+    assert call(good, hidx=None) == B.PI_ERR_INVALID_ARG and b"head_idx" in lib.pi_last_error()
+    assert call(good, ws_bytes=4096) == B.PI_ERR_CAPACITY
