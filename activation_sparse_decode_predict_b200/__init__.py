@@ -19,7 +19,8 @@ from typing import Optional, Sequence, Tuple, Union
 import torch
 
 from . import _binding as _b
-from ._binding import ACTS, DTYPES, EXPORTS, MAX_BATCH, AttnDesc, FfnDesc, LayerWeights, PiError, Weight
+from ._binding import (ACTS, DTYPES, EXPORTS, MAX_BATCH, AttnDesc, BlockWeights, FfnDesc, LayerWeights, PiError,
+                       Weight)
 
 _lib = None
 
@@ -190,6 +191,32 @@ def sparse_attention(desc: AttnDesc, x: torch.Tensor, head_idx, head_count: torc
     _check(lib().pi_sparse_attention(ctypes.byref(desc), x.shape[0], _ptr(x), _ptr(head_idx), _ptr(head_count),
                                      _ptr(Wq), _ptr(Wk), _ptr(Wv), _ptr(WoT), _ptr(K), _ptr(V), int(length), _ptr(y),
                                      _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def block_weights(L: dict, A: dict, head_rank: int) -> BlockWeights:
+    """pi_block_weights from an FFN layer dict (layer_weights) and an attention
+    dict with keys P1, P2, bp, thr (head predictor), Wq, Wk, Wv, WoT, K, V."""
+    return BlockWeights(layer_weights(L), _pred_ptr(A["P1"]), _pred_ptr(A.get("P2")), _ptr(A.get("bp")), _ptr(A["Wq"]),
+                        _ptr(A["Wk"]), _ptr(A["Wv"]), _ptr(A["WoT"]), _ptr(A["K"]), _ptr(A["V"]), float(A["thr"]),
+                        int(head_rank))
+
+
+def blocks_workspace(fdesc: FfnDesc, adesc: AttnDesc, batch: int, device=None, stream=None) -> torch.Tensor:
+    n = lib().pi_blocks_workspace_bytes(ctypes.byref(fdesc), ctypes.byref(adesc), int(batch))
+    if n == 0:
+        raise PiError(_b.PI_ERR_INVALID_ARG, lib().pi_last_error().decode())
+    ws = torch.empty(int(n), dtype=torch.uint8, device=device or "cuda")
+    _check(lib().pi_workspace_init(_ptr(ws), int(n), _stream(stream)))
+    return ws
+
+
+def decode_blocks(fdesc: FfnDesc, adesc: AttnDesc, blocks, h_in: torch.Tensor, h_out: torch.Tensor, length: int,
+                  head_idx: torch.Tensor, head_counts: torch.Tensor, idx: torch.Tensor, counts: torch.Tensor,
+                  eps: float, ws: torch.Tensor, trace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """One decode step through len(blocks) attention + FFN blocks (blocks: a ctypes array of BlockWeights)."""
+    _check(lib().pi_decode_blocks(ctypes.byref(fdesc), ctypes.byref(adesc), h_in.shape[0], len(blocks), blocks,
+                                  _ptr(h_in), _ptr(h_out), int(length), _ptr(head_idx), _ptr(head_counts), _ptr(idx),
+                                  _ptr(counts), _ptr(trace), float(eps), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def version() -> str:

@@ -24,7 +24,8 @@ MAX_BATCH = 16
 # Every symbol include/pi.h declares.
 EXPORTS = ("pi_workspace_bytes", "pi_workspace_init", "pi_predict", "pi_sparse_ffn", "pi_layer",
            "pi_residual_rmsnorm", "pi_decode_stack", "pi_stack_launches", "pi_get_device_status",
-           "pi_attn_workspace_bytes", "pi_sparse_attention", "pi_predict_static", "pi_selftest_bounded_wait",
+           "pi_attn_workspace_bytes", "pi_sparse_attention", "pi_blocks_workspace_bytes", "pi_decode_blocks",
+           "pi_predict_static", "pi_selftest_bounded_wait",
            "pi_last_error", "pi_version")
 
 
@@ -47,6 +48,12 @@ class LayerWeights(ctypes.Structure):
 class AttnDesc(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int32), ("n_heads", ctypes.c_int32), ("n_hot", ctypes.c_int32),
                 ("s_max", ctypes.c_int32), ("wtype", ctypes.c_int), ("xtype", ctypes.c_int), ("ctype", ctypes.c_int)]
+
+
+class BlockWeights(ctypes.Structure):
+    _fields_ = [("ffn", LayerWeights), ("P1h", ctypes.c_void_p), ("P2h", ctypes.c_void_p), ("bph", ctypes.c_void_p),
+                ("Wq", ctypes.c_void_p), ("Wk", ctypes.c_void_p), ("Wv", ctypes.c_void_p), ("WoT", ctypes.c_void_p),
+                ("K", ctypes.c_void_p), ("V", ctypes.c_void_p), ("thr_h", ctypes.c_float), ("head_rank", ctypes.c_int32)]
 
 
 class PiError(RuntimeError):
@@ -85,6 +92,11 @@ def load(path: str = LIB_PATH):
     lib.pi_attn_workspace_bytes.restype = S
     lib.pi_sparse_attention.argtypes = [A, i32, P, P, P, P, P, P, P, P, P, i32, P, P, S, P]
     lib.pi_sparse_attention.restype = st
+    lib.pi_blocks_workspace_bytes.argtypes = [D, A, i32]
+    lib.pi_blocks_workspace_bytes.restype = S
+    lib.pi_decode_blocks.argtypes = [D, A, i32, i32, ctypes.POINTER(BlockWeights), P, P, i32, P, P, P, P, P, f32, P,
+                                     S, P]
+    lib.pi_decode_blocks.restype = st
     lib.pi_predict_static.argtypes = [D, i32, P, P, P, P, f32, P, P, P]
     lib.pi_predict_static.restype = st
     lib.pi_selftest_bounded_wait.argtypes = [P, i32, P]

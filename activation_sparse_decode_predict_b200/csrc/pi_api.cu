@@ -241,6 +241,45 @@ AttnLayout attn_layout(const pi_attn_desc* d, int32_t B) {
   return L;
 }
 
+// The head predictor as pi_predict sees it: the heads are its neurons.
+pi_ffn_desc head_desc(const pi_ffn_desc* f, const pi_attn_desc* a, int32_t head_rank) {
+  pi_ffn_desc h = *f;
+  h.ffn = a->n_heads;
+  h.n_hot = a->n_hot;
+  h.rank = head_rank;
+  return h;
+}
+
+// Workspace of pi_decode_blocks: [FFN workspace][head predictor workspace]
+// [attention workspace][attention output B x d fp32][g, h: B x d tokens each]
+struct BlocksLayout {
+  size_t ffn, head, attn, ya, g, h, total, ffn_bytes, attn_bytes;
+};
+
+pi_status blocks_layout(const pi_ffn_desc* f, const pi_attn_desc* a, int32_t B, BlocksLayout& L) {
+  PI_TRY(check_desc(f, B));
+  PI_TRY(check_attn(a, B));
+  if (a->d != f->d) return fail(PI_ERR_INVALID_ARG, "%s", "the attention and FFN descriptors must share d");
+  if (a->xtype != pi::token_type(f)) return fail(PI_ERR_INVALID_ARG, "%s", "adesc->xtype must be the token type");
+  const pi_ffn_desc hd = head_desc(f, a, f->rank);
+  PI_TRY(check_desc(&hd, B));
+  size_t off = 0;
+  L.ffn = off;
+  L.ffn_bytes = pi_workspace_bytes(f, B);
+  off += pi::align256(L.ffn_bytes);
+  L.head = off;
+  off += pi::align256(pi_workspace_bytes(&hd, B));
+  L.attn = off;
+  L.attn_bytes = attn_layout(a, B).total;
+  off += pi::align256(L.attn_bytes);
+  const size_t tok = (size_t)B * f->d * (pi::token_type(f) == PI_F32 ? 4 : 2);
+  L.ya = off; off += pi::align256((size_t)B * f->d * 4);
+  L.g = off; off += pi::align256(tok);
+  L.h = off; off += pi::align256(tok);
+  L.total = off;
+  return PI_OK;
+}
+
 static_assert(pi::kYAccCopies == pi::kYCopies, "workspace layout and kernel agree on the accumulator copies");
 static_assert(pi::kGMax == pi::kGMaxCtas, "workspace layout and kernel agree on the largest grid");
 static_assert(pi::kLayersMax == pi::kMaxLayers && pi::kLayersMax == PI_MAX_LAYERS, "layer limits agree");
@@ -272,9 +311,7 @@ pi_status fused_params(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, pi:
   const int ep = desc->ptype == PI_F16 ? 2 : 4;
   const size_t wrow = desc->wtype == PI_Q4_0 ? desc->d / 2 + desc->d / 16
                                               : (size_t)desc->d * (desc->wtype == PI_F16 ? 2 : 4);
-  // ring bytes of one neuron (a whole item, or its gate/up and down items)
-  const size_t neuron = pi::kSplitGU ? (wrow + 16) * (desc->act == PI_ACT_REGLU ? 3 : 2) + 2 * (16 + 256)
-                                     : (wrow + 16) * (desc->act == PI_ACT_REGLU ? 3 : 2) + 16 + 256;
+  const size_t neuron = (wrow + 16) * (desc->act == PI_ACT_REGLU ? 3 : 2) + 16 + 256;
   // predictor items (the largest rank): fp16 predictors go to the tensor cores
   // in 16-row tiles with padded rows; Q4_0 rows carry codes and scales
   const size_t p2item = desc->ptype == PI_F16    ? (size_t)16 * (2 * desc->rank + 16) + 256
@@ -298,12 +335,7 @@ pi_status fused_params(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, pi:
   {
     // a consumer holds one group while it waits for the first item of the next
     // one, and a wrap of the ring can waste up to one item: ng + 2 items fit
-    int cap = pi::kNgFull ? (int)((size_t)P.ring_bytes / neuron) - 2 : (int)(half / neuron);
-    if (pi::kNgInflight > 0) {
-      // leave kNgInflight items streaming while a group is held
-      const int inflight_cap = (int)((size_t)P.ring_bytes / neuron) - pi::kNgInflight;
-      cap = inflight_cap > 1 ? inflight_cap : 1;
-    }
+    const int cap = pi::kNgFull ? (int)((size_t)P.ring_bytes / neuron) - 2 : (int)(half / neuron);
     const int lim = (desc->wtype == PI_F16 && desc->ptype == PI_F16 && pi::kF16Mma) ? 16 / rpn : 4;
     P.ng = cap < lim ? cap : lim;
     if (P.ng < 1) P.ng = 1;
@@ -568,6 +600,76 @@ pi_status pi_sparse_attention(const pi_attn_desc* desc, int32_t batch, const voi
                                reinterpret_cast<int32_t*>(w + L.orow), reinterpret_cast<int32_t*>(w + L.ocount),
                                reinterpret_cast<float*>(w + L.partial), G, y, sms, (cudaStream_t)stream),
           "sparse attention launch");
+  return PI_OK;
+}
+
+size_t pi_blocks_workspace_bytes(const pi_ffn_desc* fdesc, const pi_attn_desc* adesc, int32_t batch) {
+  BlocksLayout L;
+  if (blocks_layout(fdesc, adesc, batch, L) != PI_OK) return 0;
+  return L.total;
+}
+
+pi_status pi_decode_blocks(const pi_ffn_desc* fdesc, const pi_attn_desc* adesc, int32_t batch, int32_t n_layers,
+                           const pi_block_weights* layers, const void* h_in, void* h_out, int32_t len,
+                           int32_t* head_idx, int32_t* head_counts, int32_t* idx, int32_t* counts, void* trace,
+                           float eps, void* ws, size_t ws_bytes, void* stream) {
+  BlocksLayout L;
+  PI_TRY(blocks_layout(fdesc, adesc, batch, L));
+  if (n_layers < 1 || n_layers > PI_MAX_LAYERS) return fail(PI_ERR_INVALID_ARG, "%s", "n_layers must be in [1, 128]");
+  if (!layers) return fail(PI_ERR_INVALID_ARG, "%s", "layers is NULL");
+  if (len < 0 || len >= adesc->s_max) return fail(PI_ERR_INVALID_ARG, "%s", "len must be in [0, s_max)");
+  PI_TRY(check_ptr(h_in, 16, "h_in"));
+  PI_TRY(check_ptr(h_out, 16, "h_out"));
+  if (h_in == h_out) return fail(PI_ERR_INVALID_ARG, "%s", "h_out must not alias h_in");
+  PI_TRY(check_ptr(head_idx, 4, "head_idx"));
+  PI_TRY(check_ptr(head_counts, 4, "head_counts"));
+  if (fdesc->ffn > fdesc->n_hot) PI_TRY(check_ptr(idx, 4, "idx"));
+  PI_TRY(check_ptr(counts, 4, "counts"));
+  if (trace) PI_TRY(check_ptr(trace, 16, "trace"));
+  if (!(eps >= 0.f)) return fail(PI_ERR_INVALID_ARG, "%s", "eps must be >= 0");
+  PI_TRY(check_ptr(ws, 256, "ws"));
+  if (ws_bytes < L.total) return fail(PI_ERR_CAPACITY, "%s", "workspace smaller than pi_blocks_workspace_bytes()");
+  for (int l = 0; l < n_layers; ++l) {
+    const pi_block_weights& w = layers[l];
+    PI_TRY(check_layer(fdesc, &w.ffn));
+    const pi_ffn_desc hd = head_desc(fdesc, adesc, w.head_rank);
+    PI_TRY(check_desc(&hd, batch));
+    if (w.head_rank > fdesc->rank) return fail(PI_ERR_INVALID_ARG, "%s", "head_rank above the FFN descriptor's rank");
+    PI_TRY(check_ptr(w.P1h, 16, "P1h"));
+    if (adesc->n_heads > adesc->n_hot) PI_TRY(check_ptr(w.P2h, 16, "P2h"));
+    if (w.bph) PI_TRY(check_ptr(w.bph, 4, "bph"));
+  }
+  char* wsc = static_cast<char*>(ws);
+  char* ws_ffn = wsc + L.ffn;
+  char* ws_head = wsc + L.head;
+  char* ws_attn = wsc + L.attn;
+  float* ya = reinterpret_cast<float*>(wsc + L.ya);
+  void* gbuf = wsc + L.g;
+  void* hbuf[2] = {h_out, wsc + L.h};
+  cudaStream_t st = (cudaStream_t)stream;
+  const int ht = pi::token_type(fdesc);
+  const size_t hbytes = (size_t)batch * fdesc->d * (ht == PI_F32 ? 4 : 2);
+  const size_t C = (size_t)(fdesc->ffn - fdesc->n_hot);
+  const void* cur = h_in;
+  for (int l = 0; l < n_layers; ++l) {
+    const pi_block_weights& w = layers[l];
+    if (trace)
+      PI_CUDA(cudaMemcpyAsync((char*)trace + (size_t)(2 * l) * hbytes, cur, hbytes, cudaMemcpyDeviceToDevice, st),
+              "trace copy");
+    const pi_ffn_desc hd = head_desc(fdesc, adesc, w.head_rank);
+    int32_t* hidx = head_idx + (size_t)l * adesc->n_heads;
+    PI_TRY(predict_impl(&hd, batch, cur, w.P1h, w.P2h, w.bph, w.thr_h, hidx, head_counts + l, ws_head, st));
+    PI_TRY(pi_sparse_attention(adesc, batch, cur, hidx, head_counts + l, w.Wq, w.Wk, w.Wv, w.WoT, w.K, w.V, len, ya,
+                               ws_attn, L.attn_bytes, stream));
+    PI_CUDA(pi::launch_rmsnorm(ht, cur, ya, batch, fdesc->d, eps, gbuf, st), "rmsnorm launch");
+    if (trace)
+      PI_CUDA(cudaMemcpyAsync((char*)trace + (size_t)(2 * l + 1) * hbytes, gbuf, hbytes, cudaMemcpyDeviceToDevice, st),
+              "trace copy");
+    void* nxt = hbuf[(n_layers - 1 - l) & 1];
+    PI_TRY(pi_decode_stack(fdesc, batch, 1, &w.ffn, gbuf, nxt, idx ? idx + (size_t)l * C : nullptr, counts + l,
+                           nullptr, nullptr, eps, ws_ffn, L.ffn_bytes, stream));
+    cur = nxt;
+  }
   return PI_OK;
 }
 

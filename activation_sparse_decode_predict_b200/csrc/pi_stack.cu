@@ -365,34 +365,21 @@ struct Producer {
     return true;
   }
 
-  // One neuron as ring items.  A whole item (kPartAll): its gate (ReGLU
-  // only), up and down rows, then (with a b1) the 16-byte block of b1 that
-  // holds its bias.  Split (kSplitGU): a gate/up item (kPartGU: gate, up,
-  // the b1 block) and a down item (kPartDn: the down row).  Row m of an item
-  // starts m * (wrb + 16) bytes past a 128-byte aligned base; a gate/up base
-  // is shifted by 32 * (neuron sequence number mod 4) bytes, so that the gate
-  // and up rows of four consecutive neurons fall on eight different
-  // shared-memory bank groups (conflict-free ldmatrix).  Q4_0 rows hold qs
-  // then sc.  gs > 0 marks the first item of a group of gs neurons.
+  // One neuron: its gate (ReGLU only), up and down rows, then (with a b1)
+  // the 16-byte block of b1 that holds its bias.  Row m of the item starts
+  // m * (wrb + 16) bytes past a 128-byte aligned base that is shifted by
+  // 32 * (neuron sequence number mod 4) bytes, so that the gate and up rows
+  // of four consecutive neurons fall on eight different shared-memory bank
+  // groups (conflict-free ldmatrix).  Q4_0 rows hold qs then sc.  gs > 0
+  // marks the first item of a group of gs neurons.
   uint32_t nseq = 0;
-  __device__ bool issue_neuron(const StackLayer& Ly, int j, int wt, int gated, int gs, int part) {
+  __device__ bool issue_neuron(const StackLayer& Ly, int j, int wt, int gated, int gs) {
     const int d = p.d;
     const uint32_t wrb = wt == kQ4_0 ? (uint32_t)(d / 2 + d / 16) : (uint32_t)(d * (wt == kF16 ? 2 : 4));
     const uint32_t wrp = wrb + 16;
-    const void* rows[3];
-    const void* scs[3];
-    int nrow = 0;
-    if (part != kPartDn) {
-      if (gated) { rows[nrow] = Ly.wg; scs[nrow++] = Ly.wg_sc; }
-      rows[nrow] = Ly.wu; scs[nrow++] = Ly.wu_sc;
-    }
-    if (part != kPartGU) { rows[nrow] = Ly.wd; scs[nrow++] = Ly.wd_sc; }
-    const bool with_b1 = part != kPartDn && Ly.b1;
-    uint32_t skew = 0;
-    if (part != kPartDn) {
-      skew = 32u * (nseq & 3u);
-      ++nseq;
-    }
+    const int nrow = gated ? 3 : 2;
+    const uint32_t skew = 32u * (nseq & 3u);
+    ++nseq;
     const uint32_t total = nrow * wrp + 16 + 128 + skew;
     uint32_t pos;
     if (!alloc(total, pos)) return false;
@@ -402,7 +389,13 @@ struct Producer {
     s.istart[q] = pos;
     s.item_j[q] = j;
     s.item_gs[q] = gs;
-    mbar_arrive_expect_tx(&s.full[q], nrow * wrb + (with_b1 ? 16u : 0u));
+    mbar_arrive_expect_tx(&s.full[q], nrow * wrb + (Ly.b1 ? 16u : 0u));
+    const void* rows[3];
+    const void* scs[3];
+    int m = 0;
+    if (gated) { rows[m] = Ly.wg; scs[m++] = Ly.wg_sc; }
+    rows[m] = Ly.wu; scs[m++] = Ly.wu_sc;
+    rows[m] = Ly.wd; scs[m++] = Ly.wd_sc;
     for (int i = 0; i < nrow; ++i) {
       uint8_t* dst = s.ring + start + i * wrp;
       if (wt == kQ4_0) {
@@ -412,22 +405,16 @@ struct Producer {
         bulk_g2s(dst, reinterpret_cast<const uint8_t*>(rows[i]) + (int64_t)j * wrb, wrb, &s.full[q]);
       }
     }
-    if (with_b1) bulk_g2s(s.ring + start + nrow * wrp, Ly.b1 + (j & ~3), 16u, &s.full[q]);
+    if (Ly.b1) bulk_g2s(s.ring + start + nrow * wrp, Ly.b1 + (j & ~3), 16u, &s.full[q]);
     head = pos + total;
     ++item;
     return true;
   }
 
-  // One group of gs neurons (rows j0 .. j0+gs-1, or list[0 .. gs)): whole
-  // items, or all gate/up items first and then all down items.
+  // One group of gs neurons: rows j0 .. j0+gs-1, or list[0 .. gs)
   __device__ bool issue_group(const StackLayer& Ly, int j0, const int* list, int gs, int wt, int gated) {
     bool ok = true;
-    if constexpr (!kSplitGU) {
-      for (int i = 0; i < gs && ok; ++i) ok = issue_neuron(Ly, list ? list[i] : j0 + i, wt, gated, i == 0 ? gs : 0, kPartAll);
-    } else {
-      for (int i = 0; i < gs && ok; ++i) ok = issue_neuron(Ly, list ? list[i] : j0 + i, wt, gated, i == 0 ? gs : 0, kPartGU);
-      for (int i = 0; i < gs && ok; ++i) ok = issue_neuron(Ly, list ? list[i] : j0 + i, wt, gated, 0, kPartDn);
-    }
+    for (int i = 0; i < gs && ok; ++i) ok = issue_neuron(Ly, list ? list[i] : j0 + i, wt, gated, i == 0 ? gs : 0);
     return ok;
   }
 
@@ -798,10 +785,8 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
   load_shares(p.layers[0]);
   const int wrp = wrow_bytes(WT, d) + 16;  // byte stride of a neuron item's rows
   const int rpn = gated ? 2 : 1;           // gate/up rows per neuron
-  // where the b1 block and the down row sit: after the gate/up rows of a
-  // whole neuron item, or in the gate/up item and at the start of the down item
-  const int b1_off = kSplitGU ? rpn * wrp : (rpn + 1) * wrp;
-  const int dn_off = kSplitGU ? 0 : rpn * wrp;
+  const int b1_off = (rpn + 1) * wrp;  // the b1 block, after the gate/up/down rows
+  const int dn_off = rpn * wrp;        // the down row
 
   for (int l = 0; l < p.L; ++l) {
     const StackLayer& Ly = p.layers[l];
@@ -1060,18 +1045,9 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
               Ly.b1 ? reinterpret_cast<const float*>(s.ring + s.item_off[q] + b1_off)[s.item_j[q] & 3] : 0.f;
           gact[jj * B + b] = gated ? act_eval(kReglu, gd + bias, vd) : act_eval(p.act, vd + bias, 0.f);
         }
-        // the next group (or the end marker) starts after this group's items
-        if (t == 0) s.misc[2] = head_size(witem + (kSplitGU ? 2 * gs : gs));
+        if (t == 0) s.misc[2] = head_size(witem + gs);  // the next group (or the end marker)
         if (named_sync_or(1, T, to)) return false;
-        if constexpr (kSplitGU) {
-          // the gate/up items are read: release them, then take the down
-          // items (after a wait that ran out they are not read; the next
-          // barrier passes the failure on)
-          witem += gs;
-          for (int i = 0; i < gs; ++i) release_item();
-          for (int i = 0; i < gs; ++i) to |= !mbar_wait(&s.full[(witem + i) % kNQ], ((witem + i) / kNQ) & 1u, ctrl);
-        }
-        for (int jj = 0; jj < gs && !to; ++jj) {
+        for (int jj = 0; jj < gs; ++jj) {
           float wd[EPT];
           const uint8_t* at = s.ring + s.item_off[(witem + jj) % kNQ] + dn_off;
           if constexpr (WT == kQ4_0) {

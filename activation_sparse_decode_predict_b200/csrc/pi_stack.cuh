@@ -54,23 +54,11 @@ constexpr bool kMmaX2 = PI_MMA_X2 != 0;    // load only tile rows 0-7 when a gro
 #ifndef PI_NG_FULL
 #define PI_NG_FULL 0
 #endif
-constexpr int kNgFull = PI_NG_FULL;
-#ifndef PI_NG_INFLIGHT
-#define PI_NG_INFLIGHT 0
-#endif
-constexpr int kNgInflight = PI_NG_INFLIGHT;  // > 0: groups leave this many ring items streaming  // 1: groups may fill the ring but one item (else half the ring)
-#ifndef PI_SPLIT_GU
-#define PI_SPLIT_GU 0
-#endif
-// 1: a neuron group streams as its gate/up items, then its down items, so the
-// gate/up bytes are released before the down rows are used
-constexpr bool kSplitGU = PI_SPLIT_GU != 0;
-static_assert(!(kSplitGU && kF16Mma), "tensor-core neuron groups read whole neuron items");
-enum { kPartAll = 0, kPartGU = 1, kPartDn = 2 };  // parts of a neuron a ring item holds
+constexpr int kNgFull = PI_NG_FULL;  // 1: groups may fill the ring but one item (else half the ring)
 constexpr int kGMaxCtas = 296;       // largest grid (2 x 148)
-constexpr int kShareRegs = 2;
-constexpr int kMaxKQ = 4;          // k-parts of a P2 tile at most (each has its own score slot)
-constexpr int kMaxGroup = 16;       // neurons per group at most        // per-thread registers for the CTA's bias shares
+constexpr int kShareRegs = 2;        // per-thread registers for the CTA's bias shares
+constexpr int kMaxKQ = 4;            // k-parts of a P2 tile at most (each has its own score slot)
+constexpr int kMaxGroup = 16;        // neurons per group at most
 
 // One layer's device pointers (a copy of pi_layer_weights).
 struct StackLayer {

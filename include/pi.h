@@ -297,6 +297,47 @@ PI_API pi_status pi_sparse_attention(const pi_attn_desc *desc, int32_t batch, co
                                      int32_t len, float *y, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * A whole decode step through transformer blocks: per layer the head-sparse
+ * self-attention and the activation-sparse FFN, each followed by the stack
+ * glue ([UA] "Çevrim İçi Aşama": the engine predicts the active neurons of
+ * each layer and computes only those; [UA] "Adaptif Sparsite Predictor’ları":
+ * one predictor for the attention heads and one for the FFN neurons).
+ */
+typedef struct {
+  pi_layer_weights ffn;            /* the FFN layer, as for pi_decode_stack                  */
+  const void *P1h;                 /* head predictor [head_rank, d], the FFN descriptor's ptype */
+  const void *P2h;                 /* [n_heads - n_hot, head_rank] (NULL when every head is hot) */
+  const float *bph;                /* [n_heads - n_hot] fp32 or NULL                          */
+  const void *Wq, *Wk, *Wv, *WoT;  /* [d, d] each, the attention descriptor's wtype          */
+  void *K, *V;                     /* this layer's caches [B, n_heads, s_max, dh]            */
+  float thr_h;                     /* head predictor threshold                                */
+  int32_t head_rank;               /* head predictor rank: a multiple of 8 (Q4_0: 32), at most
+                                      the FFN descriptor's rank                                */
+} pi_block_weights;
+
+/* Workspace bytes of pi_decode_blocks (0: invalid descriptors). */
+PI_API size_t pi_blocks_workspace_bytes(const pi_ffn_desc *fdesc, const pi_attn_desc *adesc, int32_t batch);
+
+/*
+ * pi_decode_blocks -- one decode step of a token block through n_layers blocks:
+ *     for l:  heads_l = pi_predict over the heads of h_l (head predictor of layer l)
+ *             a_l = pi_sparse_attention(h_l, heads_l, caches of layer l at position len)
+ *             g_l = RMSNorm(h_l + a_l)
+ *             (idx_l, y_l) = the FFN layer on g_l;  h_{l+1} = RMSNorm(g_l + y_l)
+ *     h_out = h_{n_layers}
+ * fdesc and adesc share d; the token type (fdesc) equals adesc->xtype.
+ * layers: HOST array; head_idx [n_layers, n_heads] and head_counts [n_layers]
+ * receive the head lists; idx [n_layers, C] and counts [n_layers] the FFN
+ * lists; trace (optional) [n_layers, 2, B, d] in the token type receives each
+ * layer's h_l and g_l.  h_out must not alias h_in.  Each layer appends its
+ * listed heads' k and v at position len of its caches.
+ */
+PI_API pi_status pi_decode_blocks(const pi_ffn_desc *fdesc, const pi_attn_desc *adesc, int32_t batch,
+                                  int32_t n_layers, const pi_block_weights *layers, const void *h_in, void *h_out,
+                                  int32_t len, int32_t *head_idx, int32_t *head_counts, int32_t *idx,
+                                  int32_t *counts, void *trace, float eps, void *ws, size_t ws_bytes, void *stream);
+
+/*
  * pi_predict_static -- pi_predict for callers that cannot allocate device
  * memory.  The paper has no counterpart to this call; it exists for hosts
  * that hand the library only its inputs and outputs (plugin interfaces that

@@ -20,8 +20,9 @@ def _wl(name, d, ffn, hot, rank, act, wt, pt, B, layers=1, steps=(), sparsity=0.
 
 
 def _layer(wl, layer=0):
-    L = W.make_layer(wl, layer, device="cpu")
-    return {k: to_dev(v) if k not in ("perm", "p", "thr", "rank") else v for k, v in L.items()}
+    # made on the device: a Q4_0 predictor's scales must stay right after its
+    # codes in one buffer, which a per-tensor copy would not keep
+    return W.make_layer(wl, layer, device="cuda")
 
 
 # (name, d, ffn, hot, rank, act, wtype, ptype, batch)
