@@ -711,11 +711,25 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
         for (int q = 0; q < keep && ok; q += p.ng) ok = pr.issue_group(Ly, 0, s.cidx + q, min(p.ng, keep - q), WT, gated);
         while (ok && nxt < PN) {
           const int cur = nxt, csz = nsz;
-          nsz = csize(cur + csz);
-          nxt = atomicAdd(pool, nsz);
+          // in the last round of chunks a CTA claims its next chunk only once
+          // its own queue is short, so the last chunks go to the CTAs that are
+          // about to run dry (kLazyTail)
+          const bool tail = kLazyTail && PN - (cur + csz) < G * cmax;
+          if (!tail) {
+            nsz = csize(cur + csz);
+            nxt = atomicAdd(pool, nsz);
+          }
           ok = pr.issue_range(Ly, HA + cur, min(csz, PN - cur), WT, gated);
+          if (tail) {
+            while (ok && pr.item - pr.rel > (uint32_t)(kTailGroups * p.ng)) ok = pr.wait_consumed();
+            nsz = csize(cur + csz);
+            nxt = atomicAdd(pool, nsz);
+          }
         }
         while (ok && C > 0) {
+          if constexpr (kLazyTail)
+            while (ok && pr.item - pr.rel > (uint32_t)(kTailGroups * p.ng)) ok = pr.wait_consumed();
+          if (!ok) break;
           const int j = pr.take_donated(l, atomicAdd(&ctrl->don_take[l], 1u), C, G);
           if (j == -2) ok = false;
           if (j < 0) break;

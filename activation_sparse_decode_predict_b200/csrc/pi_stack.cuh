@@ -55,6 +55,16 @@ constexpr bool kMmaX2 = PI_MMA_X2 != 0;    // load only tile rows 0-7 when a gro
 #define PI_NG_FULL 0
 #endif
 constexpr int kNgFull = PI_NG_FULL;  // 1: groups may fill the ring but one item (else half the ring)
+#ifndef PI_LAZY_TAIL
+#define PI_LAZY_TAIL 0
+#endif
+#ifndef PI_TAIL_GROUPS
+#define PI_TAIL_GROUPS 1
+#endif
+// 1: the last claims of a layer wait until the CTA's own queue holds at most
+// kTailGroups neuron groups
+constexpr bool kLazyTail = PI_LAZY_TAIL != 0;
+constexpr int kTailGroups = PI_TAIL_GROUPS;
 constexpr int kGMaxCtas = 296;       // largest grid (2 x 148)
 constexpr int kShareRegs = 2;        // per-thread registers for the CTA's bias shares
 constexpr int kMaxKQ = 4;            // k-parts of a P2 tile at most (each has its own score slot)
