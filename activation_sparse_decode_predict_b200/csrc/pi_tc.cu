@@ -44,14 +44,30 @@ namespace pi {
 
 namespace {
 
+#ifndef PI_TC_KBS
+#define PI_TC_KBS 1
+#endif
+#ifndef PI_TC_CHUNK
+#define PI_TC_CHUNK 256
+#endif
 constexpr int kTcThreads = 192;     // warp 0: TMA producer; warp 1: MMA issuer (owns tensor memory); 2-5: epilogue
 constexpr int kTcSlots = 8;         // up partials per tile at most
-constexpr int kChunk = 256;         // output columns per down chunk (two M = 128 products)
-constexpr int kUpStage = 35 * 1024;  // [gate 16 KB][up 16 KB][tokens 2 KB], 1024-aligned
-constexpr int kUpNS = 6;
-constexpr int kDnStage = 36 * 1024;  // [4 column blocks x 64 positions x 128 B = 32 KB][activations 32 x 128 B]
-constexpr int kDnNS = 6;
+constexpr int kSmemAvail = 227 * 1024 - 2048;  // stages fit below this (barriers + alignment slack after them)
+// up: 64-column blocks of d per stage; each block is [gate 16 KB][up 16 KB][tokens 2 KB]
+constexpr int kUpKBS = PI_TC_KBS;
+constexpr int kUpBlock = 34 * 1024;
+constexpr int kUpStage = kUpKBS * kUpBlock;
+constexpr int kUpNS = kSmemAvail / kUpStage;
+// down: output columns per chunk (kChunk / 128 products of M = 128); a stage is
+// [kChunk/64 column blocks x 64 positions x 128 B][activations 32 x 128 B]
+constexpr int kChunk = PI_TC_CHUNK;
+constexpr int kDnCB = kChunk / 64;
+constexpr int kDnStage = kDnCB * 8192 + 4096;
+constexpr int kDnNS = kSmemAvail / kDnStage;
+constexpr int kDnCols = 2 * 32 * (kChunk / 128);  // tensor-memory columns: two buffers x (kChunk/128) x N = 32
 constexpr int kBarBytes = 1024;      // mbarriers and the tensor-memory address, after the stages
+static_assert(kUpNS >= 3 && kDnNS >= 3, "at least three stages in flight");
+static_assert(kChunk == 256 || kChunk == 512, "down chunks of 256 or 512 columns");
 
 // ---------------------------------------------------------------------------
 // the flat unit sequence and its split into contiguous per-CTA ranges
@@ -85,7 +101,7 @@ __device__ __forceinline__ int list_total(const int32_t* count, int n_hot, int f
 // up: units = 128-position tiles x 64-column blocks of d; every range holds at
 // least a quarter of a tile, so a tile has at most 5 writers
 __device__ __forceinline__ Split up_split(int ntot, int d, int G) {
-  const int KB = d / 64;
+  const int KB = d / (64 * kUpKBS);
   Split s;
   s.U = (int64_t)((ntot + 127) / 128) * KB;
   const int64_t per = KB / 4 > 0 ? KB / 4 : 1;
@@ -149,7 +165,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_up(const __grid_constant__
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = blockIdx.x;
   const int ntot = list_total(p.count, p.n_hot, p.ffn, ctrl, c == 0 && threadIdx.x == 0);
-  const int KB = p.d / 64;
+  const int KB = p.d / (64 * kUpKBS);  // units per tile
   const Split sp = up_split(ntot, p.d, gridDim.x);
   const int64_t u0 = c < sp.G ? range_lo(sp, c) : 0, u1 = c < sp.G ? range_lo(sp, c + 1) : 0;
   const int nmat = p.gated ? 2 : 1;
@@ -192,13 +208,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_up(const __grid_constant__
       if (it >= kUpNS) ok = mbar_wait(&empty[s], ((it / kUpNS) - 1) & 1, ctrl);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(nmat * 16384 + 2048));
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(kUpKBS * (nmat * 16384 + 2048)));
       __syncwarp();
-      uint8_t* st = sm + s * kUpStage;
-      const int x = kb * 64;
-      tma_gather4(st + lane * 512, &p.tm_w0, x, r[0], r[1], r[2], r[3], &full[s]);
-      if (p.gated) tma_gather4(st + 16384 + lane * 512, &p.tm_w1, x, r[0], r[1], r[2], r[3], &full[s]);
-      if (lane == 0) tma_load_2d(st + 32768, &p.tm_h, x, 0, &full[s]);
+      // the unit's column blocks back to back, so that a row's pieces are requested together
+#pragma unroll
+      for (int k = 0; k < kUpKBS; ++k) {
+        uint8_t* st = sm + s * kUpStage + k * kUpBlock;
+        const int x = (kb * kUpKBS + k) * 64;
+        tma_gather4(st + lane * 512, &p.tm_w0, x, r[0], r[1], r[2], r[3], &full[s]);
+        if (p.gated) tma_gather4(st + 16384 + lane * 512, &p.tm_w1, x, r[0], r[1], r[2], r[3], &full[s]);
+        if (lane == 0) tma_load_2d(st + 32768, &p.tm_h, x, 0, &full[s]);
+      }
       ++issued;
     }
     // the CTA leaves only once every issued stage has landed
@@ -224,14 +244,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_up(const __grid_constant__
         if (ok) ok = mbar_wait(&full[s], (uint32_t)((it / kUpNS) & 1), ctrl);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t st = smem_u32(sm + s * kUpStage);
         const uint32_t dg = tmem + (uint32_t)(buf * 32);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bd = sw128_desc(st + 32768 + kk * 32, 16, 1024);
-          const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-          tc_mma_f16(dg, sw128_desc(st + kk * 32, 16, 1024), bd, idesc, acc);
-          if (p.gated) tc_mma_f16(dg + 16, sw128_desc(st + 16384 + kk * 32, 16, 1024), bd, idesc, acc);
+        for (int k = 0; k < kUpKBS; ++k) {
+          const uint32_t st = smem_u32(sm + s * kUpStage + k * kUpBlock);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bd = sw128_desc(st + 32768 + kk * 32, 16, 1024);
+            const uint32_t acc = (first && k == 0 && kk == 0) ? 0u : 1u;
+            tc_mma_f16(dg, sw128_desc(st + kk * 32, 16, 1024), bd, idesc, acc);
+            if (p.gated) tc_mma_f16(dg + 16, sw128_desc(st + 16384 + kk * 32, 16, 1024), bd, idesc, acc);
+          }
         }
         tc_commit(&empty[s]);
         if (last) {
@@ -311,7 +334,7 @@ __global__ void __launch_bounds__(128) k_tc_act(const TcActParams p) {
 #pragma unroll
   for (int b = 0; b < 16; ++b) a[b] = 0.f;
   if (pos < ntot) {
-    const int KB = p.d / 64;
+    const int KB = p.d / (64 * kUpKBS);
     const Split sp = up_split(ntot, p.d, p.G);
     const int tile = pos / 128;
     const int c_lo = range_owner(sp, (int64_t)tile * KB), c_hi = range_owner(sp, (int64_t)tile * KB + KB - 1);
@@ -391,7 +414,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_down(const __grid_constant
     mbar_fence_init();
   }
   if (warp == 1) {
-    tmem_alloc(tslot, 128);
+    tmem_alloc(tslot, kDnCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -400,7 +423,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_down(const __grid_constant
   const uint32_t tmem = *tslot;
 
   if (warp == 0) {
-    // ---------------- TMA producer: lane l gathers positions 4(l%16)..+3 for column blocks 2(l/16), 2(l/16)+1 ----------------
+    // ---------------- TMA producer: lane l gathers positions 4(l%16)..+3 for half of the column blocks ----------------
     int64_t issued = 0;
     bool ok = true;
     for (int64_t u = u0; u < u1 && ok; ++u) {
@@ -412,16 +435,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_down(const __grid_constant
       if (it >= kDnNS) ok = mbar_wait(&empty[s], ((it / kDnNS) - 1) & 1, ctrl);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      if (lane == 0) mbar_arrive_expect_tx(&full[s], 32768u + 4096u);
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(kDnCB * 8192 + 4096));
       __syncwarp();
       uint8_t* st = sm + s * kDnStage;
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        const int cb = 2 * (lane >> 4) + h2;
+      for (int h2 = 0; h2 < kDnCB / 2; ++h2) {
+        const int cb = (kDnCB / 2) * (lane >> 4) + h2;
         tma_gather4(st + cb * 8192 + 4 * (lane & 15) * 128, &p.tm_wd, chunk * kChunk + cb * 64, r[0], r[1], r[2], r[3],
                     &full[s]);
       }
-      if (lane == 0) tma_load_2d(st + 32768, &p.tm_act, kb * 64, 0, &full[s]);
+      if (lane == 0) tma_load_2d(st + kDnCB * 8192, &p.tm_act, kb * 64, 0, &full[s]);
       ++issued;
     }
     if (lane == 0)
@@ -446,14 +469,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_down(const __grid_constant
         tc_fence_after();
         const uint32_t st = smem_u32(sm + s * kDnStage);
 #pragma unroll
-        for (int m = 0; m < 2; ++m) {
+        for (int m = 0; m < kChunk / 128; ++m) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             // A: MN-major, 64-column blocks 8 KB apart, 8-position groups 1 KB apart;
             // k-step kk = positions 16kk..16kk+15
             const uint64_t ad = sw128_desc(st + (2 * m) * 8192 + kk * 2048, 8192, 1024);
-            const uint64_t bd = sw128_desc(st + 32768 + kk * 32, 16, 1024);
-            tc_mma_f16(tmem + (uint32_t)(buf * 64 + m * 32), ad, bd, idesc, (first && kk == 0) ? 0u : 1u);
+            const uint64_t bd = sw128_desc(st + kDnCB * 8192 + kk * 32, 16, 1024);
+            tc_mma_f16(tmem + (uint32_t)(buf * (kDnCols / 2) + m * 32), ad, bd, idesc, (first && kk == 0) ? 0u : 1u);
           }
         }
         tc_commit(&empty[s]);
@@ -476,23 +499,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_down(const __grid_constant
       if (!last) continue;
       if (!mbar_wait(&accf[buf], (uint32_t)((nseg / 2) & 1), ctrl)) break;
       tc_fence_after();
-      float hv[2][16], lv[2][16];
-#pragma unroll
-      for (int m = 0; m < 2; ++m) {
-        const uint32_t ta = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * 64 + m * 32);
-        tmem_ld16(ta, hv[m]);
-        tmem_ld16(ta + 16, lv[m]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acce[buf]);
       // segment 0: the chunk of this CTA's first unit; segment 1: the next one
       const int seg = (u0 / KBp == chunk) ? 0 : 1;
       float* dst = p.part + ((size_t)c * 2 + seg) * 16 * kChunk;
 #pragma unroll
-      for (int m = 0; m < 2; ++m)
+      for (int m = 0; m < kChunk / 128; ++m) {
+        float hv[16], lv[16];
+        const uint32_t ta = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * (kDnCols / 2) + m * 32);
+        tmem_ld16(ta, hv);
+        tmem_ld16(ta + 16, lv);
 #pragma unroll
-        for (int b = 0; b < 16; ++b) dst[b * kChunk + m * 128 + q * 32 + lane] = hv[m][b] + lv[m][b];
+        for (int b = 0; b < 16; ++b) dst[b * kChunk + m * 128 + q * 32 + lane] = hv[b] + lv[b];
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce[buf]);
       buf ^= 1;
       ++nseg;
     }
@@ -501,7 +522,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_down(const __grid_constant
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, kDnCols);
   }
 }
 
@@ -596,7 +617,7 @@ size_t tc_ws_bytes(int d, int ffn, int B) {
   (void)B;
   size_t n = ((size_t)kTcSlots * ffn * 2 * 16 * 4 + 1023) & ~(size_t)1023;
   n += ((size_t)32 * tc_fpad(ffn) * 2 + 1023) & ~(size_t)1023;
-  n += (size_t)296 * 2 * 16 * kChunk * 4;
+  n += (size_t)296 * 2 * 16 * kChunk * 4;  // partial outputs: two segments per CTA
   return n;
 }
 
