@@ -46,7 +46,9 @@ REF_SECONDS = 150.0  # cap on the timed oracle work of the reference arm
 # capture of a few layers of the workload (the committed ncu summaries);
 # per-layer traffic does not depend on the layer count, so a launch over L
 # layers moves L times this.  Only for captures of the current kernel.
-TRAFFIC_PER_LAYER = {("7b-reglu-fp16", 1): (271.094016e6 + 3.657472e6) / 4}
+TRAFFIC_PER_LAYER = {("7b-reglu-fp16", 1): (276943360 + 3626496) / 4,
+                     ("13b-reglu-q4_0", 1): (208071680 + 3443968) / 4,
+                     ("70b-reglu-fp16", 1): (1316775424 + 3609856) / 4}
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -336,7 +338,8 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(gbs / peak, 4),
                      "traffic": (round(TRAFFIC_PER_LAYER[(wl.name, B)] * n_layers)
-                                 if (wl.name, B) in TRAFFIC_PER_LAYER and args.sparsity is None else None),
+                                 if (wl.name, B) in TRAFFIC_PER_LAYER and args.sparsity is None
+                                 and args.ptype is None else None),
                      "kernel": "whole decode step (%d launches)" % launches_per_step,
                      "peak_source": peak_kind},
         "e2e": {"value": round(e2e_tok_s, 3), "unit": "tokens/s", "h2d_bytes_per_step": hb, "d2h_bytes_per_step": hb,
