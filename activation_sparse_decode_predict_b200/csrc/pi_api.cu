@@ -691,7 +691,7 @@ int32_t pi_stack_launches(const pi_ffn_desc* desc, int32_t batch, int32_t n_laye
     pred = cold ? 3 : 1;  // u, scores, compaction
   int ffn;
   if (pi::kTcFfn && pi::tc_ffn_supported(desc->wtype, pi::token_type(desc), desc->d, batch))
-    ffn = 4;  // up, activations, down, reduce
+    ffn = 2;  // up (+ bias and activation), down (+ the sum over writers and b2)
   else
     ffn = 3;  // gate/up (or row dots), down, reduce
   return (pred + ffn + 1) * n_layers;

@@ -23,11 +23,14 @@
 // block of d; down: 256-column chunk of d x 64-position block of the list) is
 // cut into G contiguous ranges of equal length, one per CTA; a CTA accumulates
 // consecutive units of the same tile (chunk) in tensor memory and writes one
-// partial per (CTA, tile) segment.  Readers find the writers of a tile from
-// the same arithmetic, and sum them in CTA order: deterministic.
+// partial per (CTA, tile) segment.  The writers of a tile (chunk) follow from
+// the same arithmetic; each counts itself on a per-tile (per-chunk) counter,
+// and the last one to count sums the partials in CTA order -- the same sum
+// whichever CTA is last: deterministic.
 //
-// Kernels per call: k_tc_up -> k_tc_act (sum of the up partials, bias,
-// activation, fp16 hi/lo rows) -> k_tc_down -> k_tc_reduce (+ b2).
+// Kernels per call: k_tc_up (gate/up dots; the last writer of a tile adds b1,
+// applies the activation and writes the fp16 hi/lo rows) -> k_tc_down (down
+// products; the last writer of a chunk adds b2 and writes y).
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -50,8 +53,20 @@ namespace {
 #ifndef PI_TC_CHUNK
 #define PI_TC_CHUNK 256
 #endif
-constexpr int kTcThreads = 192;     // warp 0: TMA producer; warp 1: MMA issuer (owns tensor memory); 2-5: epilogue
+// Warps 0-3 issue the TMA gathers, one warp per SM sub-partition: the
+// gathers of one warp are issued lane after lane, and a single warp cannot
+// issue them fast enough to keep HBM busy (about a third of the rate of four
+// warps).  Warp 4 issues the MMAs and owns the tensor memory; warps 5-8 are
+// the epilogue (warp w reads tensor-memory lanes 32 (w % 4) .. + 31).
+#ifndef PI_TC_PW
+#define PI_TC_PW 8
+#endif
+constexpr int kProdWarps = PI_TC_PW;
+static_assert(kProdWarps == 2 || kProdWarps == 4 || kProdWarps == 8, "2, 4 or 8 producer warps");
+constexpr int kMmaWarp = kProdWarps;
+constexpr int kTcThreads = 32 * (kProdWarps + 5);
 constexpr int kTcSlots = 8;         // up partials per tile at most
+constexpr int kGMaxWriters = 296;   // CTAs of the largest grid: writers of a down chunk at most
 constexpr int kSmemAvail = 227 * 1024 - 2048;  // stages fit below this (barriers + alignment slack after them)
 // up: 64-column blocks of d per stage; each block is [gate 16 KB][up 16 KB][tokens 2 KB]
 constexpr int kUpKBS = PI_TC_KBS;
@@ -133,6 +148,21 @@ __device__ __forceinline__ int list_row_at(int pos, int ntot, int n_hot, int ffn
   return j;
 }
 
+// The same in two steps: the raw entry (a load that may still be in flight),
+// then its check once the value is needed.
+__device__ __forceinline__ int list_raw(int pos, int ntot, int n_hot, const int32_t* idx) {
+  if (pos < n_hot) return pos;
+  if (pos >= ntot) return 0;
+  return __ldg(idx + (pos - n_hot));
+}
+__device__ __forceinline__ int list_checked(int j, int pos, int ntot, int n_hot, int ffn, Ctrl* ctrl) {
+  if (pos >= n_hot && pos < ntot && (j < n_hot || j >= ffn)) {
+    set_status(&ctrl->status, kStIndex);
+    return 0;
+  }
+  return j;
+}
+
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   const uint32_t a = smem_u32(p);
   return p + ((1024u - (a & 1023u)) & 1023u);
@@ -145,15 +175,21 @@ struct TcUpParams {
   CUtensorMap tm_h;   // token block [B, d] fp16; box 64 x 16 (rows past B read as zero)
   CUtensorMap tm_w0;  // gate rows (ReGLU) or up rows [F, d] fp16; box 64 x 1
   CUtensorMap tm_w1;  // up rows (ReGLU); box 64 x 1
+  CUtensorMap tm_t0;  // the same two matrices with a box of 64 x 128: a tile of hot rows in one load
+  CUtensorMap tm_t1;
   const int32_t* idx;
   const int32_t* count;
-  float* pre;  // [kTcSlots][ffn][2][16]
+  float* pre;      // [kTcSlots][ffn][2][16] partial dots of tiles with several writers
+  const float* b1;
+  __half* act16;   // [32][fpad] activations as fp16 hi / lo rows
+  int* tcnt;       // [tiles] writers counted so far (zero between calls)
   Ctrl* ctrl;
-  int d, ffn, n_hot, gated;
+  int d, ffn, n_hot, gated, act, B, fpad;
 };
 
 __global__ void __launch_bounds__(kTcThreads, 1) k_tc_up(const __grid_constant__ TcUpParams p) {
   extern __shared__ uint8_t smraw[];
+  __shared__ int s_last;  // set by the epilogue: this CTA finishes the tile
   uint8_t* sm = align1024(smraw);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + kUpNS * kUpStage);
   uint64_t* empty = full + kUpNS;
@@ -182,7 +218,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_up(const __grid_constant__
     mbar_init(done, 1);
     mbar_fence_init();
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tslot, 64);
     tmem_relinquish();
   }
@@ -191,8 +227,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_up(const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = *tslot;
 
-  if (warp == 0) {
-    // ---------------- TMA producer: lane l gathers list positions 4l..4l+3 of the tile ----------------
+  if (warp < kProdWarps) {
+    // ---------------- TMA producers: a tile's 32 four-row groups are split
+    // evenly over the producer warps; lane l < 2 gpw of warp w gathers group
+    // g = w gpw + l % gpw from the gate (l < gpw) or up (l >= gpw) rows ----------------
+    constexpr int gpw = 32 / kProdWarps;
+    const int g = gpw * warp + lane % gpw, m = lane / gpw;
+    const bool mine = m == 0 || (m == 1 && p.gated);
     int r[4] = {0, 0, 0, 0};
     int cur = -1;
     int64_t issued = 0;
@@ -200,32 +241,43 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_up(const __grid_constant__
     for (int64_t u = u0; u < u1 && ok; ++u) {
       const int it = (int)(u - u0), s = it % kUpNS;
       const int tile = (int)(u / KB), kb = (int)(u % KB);
+      // a tile of hot rows only is 128 consecutive storage rows: one tiled load per matrix
+      const bool hot_tile = tile * 128 + 128 <= p.n_hot;
       if (tile != cur) {
         cur = tile;
+        if (mine && !hot_tile) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) r[i] = list_row_at(tile * 128 + 4 * lane + i, ntot, p.n_hot, p.ffn, p.idx, ctrl);
+          for (int i = 0; i < 4; ++i) r[i] = list_row_at(tile * 128 + 4 * g + i, ntot, p.n_hot, p.ffn, p.idx, ctrl);
+        }
       }
       if (it >= kUpNS) ok = mbar_wait(&empty[s], ((it / kUpNS) - 1) & 1, ctrl);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(kUpKBS * (nmat * 16384 + 2048)));
+      // the stage's byte count is posted once; copies of the other warps that
+      // land first leave the count below zero until then, and the phase cannot
+      // complete before this arrival
+      if (warp == 0 && lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(kUpKBS * (nmat * 16384 + 2048)));
       __syncwarp();
       // the unit's column blocks back to back, so that a row's pieces are requested together
 #pragma unroll
       for (int k = 0; k < kUpKBS; ++k) {
         uint8_t* st = sm + s * kUpStage + k * kUpBlock;
         const int x = (kb * kUpKBS + k) * 64;
-        tma_gather4(st + lane * 512, &p.tm_w0, x, r[0], r[1], r[2], r[3], &full[s]);
-        if (p.gated) tma_gather4(st + 16384 + lane * 512, &p.tm_w1, x, r[0], r[1], r[2], r[3], &full[s]);
-        if (lane == 0) tma_load_2d(st + 32768, &p.tm_h, x, 0, &full[s]);
+        if (hot_tile) {
+          if (warp == 0 && lane < nmat) tma_load_2d(st + lane * 16384, lane ? &p.tm_t1 : &p.tm_t0, x, tile * 128, &full[s]);
+        } else if (mine) {
+          tma_gather4(st + m * 16384 + g * 512, m ? &p.tm_w1 : &p.tm_w0, x, r[0], r[1], r[2], r[3], &full[s]);
+        }
+        if (warp == kProdWarps - 1 && lane == 31) tma_load_2d(st + 32768, &p.tm_h, x, 0, &full[s]);
       }
       ++issued;
     }
-    // the CTA leaves only once every issued stage has landed
-    if (lane == 0)
+    // the CTA leaves only once every issued stage has landed (every producer
+    // warp's copies count toward the same phases)
+    if (warp == 0 && lane == 0)
       for (int64_t it = issued > kUpNS ? issued - kUpNS : 0; it < issued; ++it)
         mbar_wait(&full[it % kUpNS], (uint32_t)((it / kUpNS) & 1), ctrl);
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16(128, 16, 0, 0);
@@ -270,104 +322,108 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_up(const __grid_constant__
     __syncwarp();
   } else {
     // ---------------- epilogue: warp quarter q reads tensor-memory lanes 32q..32q+31 ----------------
-    const int q = warp & 3;
-    int buf = 0, nseg = 0, cur = -1;
+    // A tile written by one CTA is finished from registers.  A tile split
+    // between CTAs: each writer stores its partial dots in its slot and counts
+    // itself; the last writer to count sums the slots in CTA order (the same
+    // sum whoever is last) and finishes the tile.
+    const int q = warp & 3, et = threadIdx.x - 32 * (kMmaWarp + 1);
+    int buf = 0, nseg = 0;
     for (int64_t u = u0; u < u1; ++u) {
       const int tile = (int)(u / KB);
-      if (tile != cur) cur = tile;
       const bool last = (u + 1 == u1) || ((u + 1) / KB != tile);
       if (!last) continue;
-      if (!mbar_wait(&accf[buf], (uint32_t)((nseg / 2) & 1), ctrl)) break;
+      const bool okw = mbar_wait(&accf[buf], (uint32_t)((nseg / 2) & 1), ctrl);
+      if (named_sync_or(1, 128, !okw)) break;  // all epilogue warps leave together
       tc_fence_after();
       float g[16], v[16];
       const uint32_t ta = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * 32);
       tmem_ld16(ta, g);
-      if (p.gated) tmem_ld16(ta + 16, v);
+      if (p.gated) {
+        tmem_ld16(ta + 16, v);
+      } else {
+#pragma unroll
+        for (int b = 0; b < 16; ++b) v[b] = 0.f;
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acce[buf]);
-      const int pos = tile * 128 + q * 32 + lane;
-      const int slot = c - range_owner(sp, (int64_t)tile * KB);
-      if (slot >= kTcSlots) {
-        set_status(&ctrl->status, kStCapacity);
-      } else if (pos < ntot) {
-        float4* dst = reinterpret_cast<float4*>(p.pre + (((size_t)slot * p.ffn + pos) * 2) * 16);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) dst[i] = make_float4(g[4 * i], g[4 * i + 1], g[4 * i + 2], g[4 * i + 3]);
-        if (p.gated) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) dst[4 + i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-        }
-      }
       buf ^= 1;
       ++nseg;
+      const int pos = tile * 128 + q * 32 + lane;
+      const int c_lo = range_owner(sp, (int64_t)tile * KB);
+      const int nw = range_owner(sp, (int64_t)tile * KB + KB - 1) - c_lo + 1, slot = c - c_lo;
+      if (nw > 1) {
+        if (slot >= kTcSlots) {
+          if (et == 0) set_status(&ctrl->status, kStCapacity);
+        } else if (pos < ntot) {
+          float4* dst = reinterpret_cast<float4*>(p.pre + (((size_t)slot * p.ffn + pos) * 2) * 16);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_float4(g[4 * i], g[4 * i + 1], g[4 * i + 2], g[4 * i + 3]);
+          if (p.gated) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[4 + i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          }
+        }
+        __threadfence();
+        named_sync(1, 128);
+        if (et == 0) {
+          const int prev = atomicAdd(p.tcnt + tile, 1);
+          s_last = prev == nw - 1;
+          if (prev == nw - 1) p.tcnt[tile] = 0;  // every writer has counted: ready for the next call
+        }
+        named_sync(1, 128);
+        if (!s_last) continue;
+        __threadfence();
+#pragma unroll
+        for (int b = 0; b < 16; ++b) g[b] = v[b] = 0.f;
+        if (pos < ntot) {
+#pragma unroll
+          for (int sl = 0; sl < kTcSlots; ++sl) {
+            if (sl >= nw) break;
+            const float4* src = reinterpret_cast<const float4*>(p.pre + (((size_t)sl * p.ffn + pos) * 2) * 16);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float4 x = __ldcg(src + i);
+              g[4 * i] += x.x; g[4 * i + 1] += x.y; g[4 * i + 2] += x.z; g[4 * i + 3] += x.w;
+            }
+            if (p.gated) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float4 x = __ldcg(src + 4 + i);
+                v[4 * i] += x.x; v[4 * i + 1] += x.y; v[4 * i + 2] += x.z; v[4 * i + 3] += x.w;
+              }
+            }
+          }
+        }
+      }
+      // bias + activation; fp16 hi/lo rows of the down operand, zero for tokens
+      // past B and for positions past the list up to the next 64
+      if (pos < ((ntot + 63) & ~63) && pos < p.fpad) {
+        float a[16];
+#pragma unroll
+        for (int b = 0; b < 16; ++b) a[b] = 0.f;
+        if (pos < ntot) {
+          const int row = list_row_at(pos, ntot, p.n_hot, p.ffn, p.idx, ctrl);
+          const float bias = p.b1 ? __ldg(p.b1 + row) : 0.f;
+#pragma unroll
+          for (int b = 0; b < 16; ++b)
+            if (b < p.B) a[b] = p.gated ? act_eval(kReglu, g[b] + bias, v[b]) : act_eval(p.act, g[b] + bias, 0.f);
+        }
+#pragma unroll
+        for (int b = 0; b < 16; ++b) {
+          const __half hi = __float2half_rn(a[b]);
+          const __half lo = __float2half_rn(a[b] - __half2float(hi));
+          p.act16[(size_t)b * p.fpad + pos] = hi;
+          p.act16[(size_t)(16 + b) * p.fpad + pos] = lo;
+        }
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 64);
-  }
-}
-
-// ---------------------------------------------------------------------------
-// activations: sum of a tile's up partials (in CTA order) + b1, activation,
-// fp16 hi/lo rows act16[32][fpad] (hi: rows 0-15, lo: rows 16-31; zero for
-// tokens past B and positions past the list up to the next 64)
-
-struct TcActParams {
-  const float* pre;
-  const float* b1;
-  __half* act16;
-  const int32_t* idx;
-  const int32_t* count;
-  Ctrl* ctrl;
-  int d, ffn, n_hot, act, gated, B, fpad, G;
-};
-
-__global__ void __launch_bounds__(128) k_tc_act(const TcActParams p) {
-  const int pos = blockIdx.x * blockDim.x + threadIdx.x;
-  const int ntot = list_total(p.count, p.n_hot, p.ffn, p.ctrl, false);
-  if (pos >= ((ntot + 63) & ~63) || pos >= p.fpad) return;
-  float a[16];
-#pragma unroll
-  for (int b = 0; b < 16; ++b) a[b] = 0.f;
-  if (pos < ntot) {
-    const int KB = p.d / (64 * kUpKBS);
-    const Split sp = up_split(ntot, p.d, p.G);
-    const int tile = pos / 128;
-    const int c_lo = range_owner(sp, (int64_t)tile * KB), c_hi = range_owner(sp, (int64_t)tile * KB + KB - 1);
-    float g[16], v[16];
-#pragma unroll
-    for (int b = 0; b < 16; ++b) g[b] = v[b] = 0.f;
-    for (int slot = 0; slot <= c_hi - c_lo && slot < kTcSlots; ++slot) {
-      const float4* src = reinterpret_cast<const float4*>(p.pre + (((size_t)slot * p.ffn + pos) * 2) * 16);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 x = __ldcg(src + i);
-        g[4 * i] += x.x; g[4 * i + 1] += x.y; g[4 * i + 2] += x.z; g[4 * i + 3] += x.w;
-      }
-      if (p.gated) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float4 x = __ldcg(src + 4 + i);
-          v[4 * i] += x.x; v[4 * i + 1] += x.y; v[4 * i + 2] += x.z; v[4 * i + 3] += x.w;
-        }
-      }
-    }
-    const int row = list_row_at(pos, ntot, p.n_hot, p.ffn, p.idx, p.ctrl);
-    const float bias = p.b1 ? __ldg(p.b1 + row) : 0.f;
-#pragma unroll
-    for (int b = 0; b < 16; ++b)
-      if (b < p.B) a[b] = p.gated ? act_eval(kReglu, g[b] + bias, v[b]) : act_eval(p.act, g[b] + bias, 0.f);
-  }
-#pragma unroll
-  for (int b = 0; b < 16; ++b) {
-    const __half hi = __float2half_rn(a[b]);
-    const __half lo = __float2half_rn(a[b] - __half2float(hi));
-    p.act16[(size_t)b * p.fpad + pos] = hi;
-    p.act16[(size_t)(16 + b) * p.fpad + pos] = lo;
   }
 }
 
@@ -376,16 +432,22 @@ __global__ void __launch_bounds__(128) k_tc_act(const TcActParams p) {
 
 struct TcDownParams {
   CUtensorMap tm_wd;   // W_downT [F, d] fp16; box 64 x 1
+  CUtensorMap tm_wdt;  // the same with a box of 64 x 64: a block of hot positions in one load per column block
   CUtensorMap tm_act;  // act16 [32, fpad] fp16; box 64 x 32
   const int32_t* idx;
   const int32_t* count;
   float* part;  // [G][2][16][kChunk]
+  const float* b2;
+  float* y;     // [B][d]
+  int* ccnt;    // [d / kChunk] writers counted so far (zero between calls)
   Ctrl* ctrl;
-  int d, ffn, n_hot;
+  int d, ffn, n_hot, B;
 };
 
 __global__ void __launch_bounds__(kTcThreads, 1) k_tc_down(const __grid_constant__ TcDownParams p) {
   extern __shared__ uint8_t smraw[];
+  __shared__ int s_last;  // set by the epilogue: this CTA finishes the chunk
+  __shared__ int s_woff[kGMaxWriters];  // the chunk's partial outputs, by writer (offsets into part)
   uint8_t* sm = align1024(smraw);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + kDnNS * kDnStage);
   uint64_t* empty = full + kDnNS;
@@ -413,7 +475,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_down(const __grid_constant
     mbar_init(done, 1);
     mbar_fence_init();
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tslot, kDnCols);
     tmem_relinquish();
   }
@@ -422,35 +484,62 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_down(const __grid_constant
   tc_fence_after();
   const uint32_t tmem = *tslot;
 
-  if (warp == 0) {
-    // ---------------- TMA producer: lane l gathers positions 4(l%16)..+3 for half of the column blocks ----------------
+  if (warp < kProdWarps) {
+    // ---------------- TMA producers: a unit's kDnCB x 16 four-position gathers
+    // are split evenly over the producer warps; lane l < opw of warp w does
+    // gather o = w opw + l: column block o / 16, list positions 4 (o % 16) .. + 3 ----------------
+    constexpr int opw = kDnCB * 16 / kProdWarps;
+    static_assert(opw <= 32, "one gather per lane and unit");
+    const int o = opw * warp + lane, cbo = o / 16, pg = o % 16;
+    const bool mine = lane < opw;
     int64_t issued = 0;
     bool ok = true;
+    // the list entries of a unit are loaded two units ahead and checked when
+    // the unit is issued, so that no lookup waits on the path from a free
+    // stage to its copies
+    int ra[4] = {0, 0, 0, 0}, rb[4] = {0, 0, 0, 0};
+    if (mine) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (u0 < u1) ra[i] = list_raw(((int)(u0 % KBp)) * 64 + 4 * pg + i, ntot, p.n_hot, p.idx);
+        if (u0 + 1 < u1) rb[i] = list_raw(((int)((u0 + 1) % KBp)) * 64 + 4 * pg + i, ntot, p.n_hot, p.idx);
+      }
+    }
     for (int64_t u = u0; u < u1 && ok; ++u) {
       const int it = (int)(u - u0), s = it % kDnNS;
       const int chunk = (int)(u / KBp), kb = (int)(u % KBp);
       int r[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) r[i] = list_row_at(kb * 64 + 4 * (lane & 15) + i, ntot, p.n_hot, p.ffn, p.idx, ctrl);
+      for (int i = 0; i < 4; ++i) {
+        r[i] = ra[i];
+        ra[i] = rb[i];
+        if (mine && u + 2 < u1) rb[i] = list_raw(((int)((u + 2) % KBp)) * 64 + 4 * pg + i, ntot, p.n_hot, p.idx);
+      }
       if (it >= kDnNS) ok = mbar_wait(&empty[s], ((it / kDnNS) - 1) & 1, ctrl);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(kDnCB * 8192 + 4096));
+      if (warp == 0 && lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(kDnCB * 8192 + 4096));
       __syncwarp();
       uint8_t* st = sm + s * kDnStage;
+      if (mine) {
 #pragma unroll
-      for (int h2 = 0; h2 < kDnCB / 2; ++h2) {
-        const int cb = (kDnCB / 2) * (lane >> 4) + h2;
-        tma_gather4(st + cb * 8192 + 4 * (lane & 15) * 128, &p.tm_wd, chunk * kChunk + cb * 64, r[0], r[1], r[2], r[3],
+        for (int i = 0; i < 4; ++i) r[i] = list_checked(r[i], kb * 64 + 4 * pg + i, ntot, p.n_hot, p.ffn, ctrl);
+      }
+      if (kb * 64 + 64 <= p.n_hot) {
+        // 64 hot positions are 64 consecutive storage rows
+        if (warp == 0 && lane < kDnCB)
+          tma_load_2d(st + lane * 8192, &p.tm_wdt, chunk * kChunk + lane * 64, kb * 64, &full[s]);
+      } else if (mine) {
+        tma_gather4(st + cbo * 8192 + 4 * pg * 128, &p.tm_wd, chunk * kChunk + cbo * 64, r[0], r[1], r[2], r[3],
                     &full[s]);
       }
-      if (lane == 0) tma_load_2d(st + kDnCB * 8192, &p.tm_act, kb * 64, 0, &full[s]);
+      if (warp == kProdWarps - 1 && lane == 31) tma_load_2d(st + kDnCB * 8192, &p.tm_act, kb * 64, 0, &full[s]);
       ++issued;
     }
-    if (lane == 0)
+    if (warp == 0 && lane == 0)
       for (int64_t it = issued > kDnNS ? issued - kDnNS : 0; it < issued; ++it)
         mbar_wait(&full[it % kDnNS], (uint32_t)((it / kDnNS) & 1), ctrl);
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16(128, 32, 1, 0);
       int buf = 0, nseg = 0, cur = -1;
@@ -491,13 +580,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_down(const __grid_constant
     }
     __syncwarp();
   } else {
-    const int q = warp & 3;
+    // ---------------- epilogue: partial outputs of the CTA's chunk segments;
+    // the last writer of a chunk to count itself sums the chunk's partials in
+    // CTA order, adds b2 and writes y ----------------
+    const int q = warp & 3, et = threadIdx.x - 32 * (kMmaWarp + 1);
+    if (KBp == 0 && c < p.d / kChunk) {
+      // an empty list: y = b2 (CTA c writes chunk c)
+      for (int i = et; i < p.B * kChunk; i += 128) {
+        const int col = c * kChunk + i % kChunk;
+        p.y[(size_t)(i / kChunk) * p.d + col] = p.b2 ? __ldg(p.b2 + col) : 0.f;
+      }
+    }
     int buf = 0, nseg = 0;
     for (int64_t u = u0; u < u1; ++u) {
       const int chunk = (int)(u / KBp);
       const bool last = (u + 1 == u1) || ((u + 1) / KBp != chunk);
       if (!last) continue;
-      if (!mbar_wait(&accf[buf], (uint32_t)((nseg / 2) & 1), ctrl)) break;
+      const bool okw = mbar_wait(&accf[buf], (uint32_t)((nseg / 2) & 1), ctrl);
+      if (named_sync_or(1, 128, !okw)) break;  // all epilogue warps leave together
       tc_fence_after();
       // segment 0: the chunk of this CTA's first unit; segment 1: the next one
       const int seg = (u0 / KBp == chunk) ? 0 : 1;
@@ -516,38 +616,64 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_down(const __grid_constant
       if (lane == 0) mbar_arrive(&acce[buf]);
       buf ^= 1;
       ++nseg;
+      const int c_lo = range_owner(sp, (int64_t)chunk * KBp);
+      const int nw = range_owner(sp, (int64_t)chunk * KBp + KBp - 1) - c_lo + 1;
+      __threadfence();
+      named_sync(1, 128);
+      if (et == 0) {
+        const int prev = atomicAdd(p.ccnt + chunk, 1);
+        s_last = prev == nw - 1;
+        if (prev == nw - 1) p.ccnt[chunk] = 0;  // every writer has counted: ready for the next call
+      }
+      named_sync(1, 128);
+      if (!s_last) continue;
+      __threadfence();
+      for (int k = et; k < nw && k < kGMaxWriters; k += 128) {
+        const int cw = c_lo + k;
+        const int sg = (range_lo(sp, cw) / KBp == chunk) ? 0 : 1;
+        s_woff[k] = (cw * 2 + sg) * 16 * kChunk;
+      }
+      named_sync(1, 128);
+      // four columns per item and eight items per thread at once, so that the
+      // loads of all of them are in flight together (this sum ends the kernel)
+      const int nit = p.B * (kChunk / 4), nk = nw < kGMaxWriters ? nw : kGMaxWriters;
+      for (int i0 = et; i0 < nit; i0 += 128 * 8) {
+        float4 acc[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int i = i0 + 128 * j, col = chunk * kChunk + 4 * (i % (kChunk / 4));
+          acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (i < nit && p.b2) acc[j] = make_float4(__ldg(p.b2 + col), __ldg(p.b2 + col + 1), __ldg(p.b2 + col + 2),
+                                                    __ldg(p.b2 + col + 3));
+        }
+        for (int k = 0; k < nk; ++k) {
+          const float* src = p.part + s_woff[k];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int i = i0 + 128 * j;
+            if (i < nit) {
+              const float4 x = __ldcg(reinterpret_cast<const float4*>(src + (i / (kChunk / 4)) * kChunk) + i % (kChunk / 4));
+              acc[j].x += x.x; acc[j].y += x.y; acc[j].z += x.z; acc[j].w += x.w;
+            }
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int i = i0 + 128 * j;
+          if (i < nit) {
+            float* dst = p.y + (size_t)(i / (kChunk / 4)) * p.d + chunk * kChunk + 4 * (i % (kChunk / 4));
+            dst[0] = acc[j].x; dst[1] = acc[j].y; dst[2] = acc[j].z; dst[3] = acc[j].w;
+          }
+        }
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kDnCols);
   }
-}
-
-// y[b, col] = b2[col] + sum over the chunk's writers (CTA order) of their partials
-__global__ void __launch_bounds__(256) k_tc_reduce(const float* __restrict__ part, const int32_t* count, int n_hot,
-                                                   int ffn, int d, int B, int G, const float* __restrict__ b2,
-                                                   float* __restrict__ y, Ctrl* ctrl) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= B * d) return;
-  const int b = i / d, col = i % d;
-  const int ntot = list_total(count, n_hot, ffn, ctrl, false);
-  const int KBp = (ntot + 63) / 64;
-  float acc = b2 ? __ldg(b2 + col) : 0.f;
-  if (KBp > 0) {
-    const Split sp = down_split(ntot, d, G);
-    const int chunk = col / kChunk;
-    const int c_lo = range_owner(sp, (int64_t)chunk * KBp), c_hi = range_owner(sp, (int64_t)chunk * KBp + KBp - 1);
-    for (int c = c_lo; c <= c_hi; ++c) {
-      const int64_t lo = range_lo(sp, c);
-      if (range_lo(sp, c + 1) == lo) continue;  // an empty range wrote nothing
-      const int seg = (lo / KBp == chunk) ? 0 : 1;
-      acc += __ldcg(part + (((size_t)c * 2 + seg) * 16 + b) * kChunk + (col % kChunk));
-    }
-  }
-  y[i] = acc;
 }
 
 // ---------------------------------------------------------------------------
@@ -587,20 +713,33 @@ cudaError_t make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t r
 
 int tc_fpad(int ffn) { return (ffn + 63) & ~63; }
 
+int tc_tiles(int ffn) { return (ffn + 127) / 128; }
+
+// The token-block scratch: up partials, the activation rows, down partials and
+// the per-tile / per-chunk writer counters (zero from pi_workspace_init on;
+// each call leaves them at zero again).
 struct TcScratch {
   float* pre;
   __half* act16;
   float* part;
+  int* tcnt;
+  int* ccnt;
 };
+
+size_t tc_align(size_t n) { return (n + 1023) & ~(size_t)1023; }
 
 TcScratch tc_carve(void* scratch, int ffn) {
   TcScratch s;
   char* b = static_cast<char*>(scratch);
   s.pre = reinterpret_cast<float*>(b);
-  b += ((size_t)kTcSlots * ffn * 2 * 16 * 4 + 1023) & ~(size_t)1023;
+  b += tc_align((size_t)kTcSlots * ffn * 2 * 16 * 4);
   s.act16 = reinterpret_cast<__half*>(b);
-  b += ((size_t)32 * tc_fpad(ffn) * 2 + 1023) & ~(size_t)1023;
+  b += tc_align((size_t)32 * tc_fpad(ffn) * 2);
   s.part = reinterpret_cast<float*>(b);
+  b += tc_align((size_t)296 * 2 * 16 * kChunk * 4);  // two segments per CTA
+  s.tcnt = reinterpret_cast<int*>(b);
+  b += tc_align((size_t)tc_tiles(ffn) * 4);
+  s.ccnt = reinterpret_cast<int*>(b);
   return s;
 }
 
@@ -615,9 +754,11 @@ bool tc_ffn_supported(int wtype, int ptype, int d, int B) {
 size_t tc_ws_bytes(int d, int ffn, int B) {
   (void)d;
   (void)B;
-  size_t n = ((size_t)kTcSlots * ffn * 2 * 16 * 4 + 1023) & ~(size_t)1023;
-  n += ((size_t)32 * tc_fpad(ffn) * 2 + 1023) & ~(size_t)1023;
-  n += (size_t)296 * 2 * 16 * kChunk * 4;  // partial outputs: two segments per CTA
+  size_t n = tc_align((size_t)kTcSlots * ffn * 2 * 16 * 4);
+  n += tc_align((size_t)32 * tc_fpad(ffn) * 2);
+  n += tc_align((size_t)296 * 2 * 16 * kChunk * 4);
+  n += tc_align((size_t)tc_tiles(ffn) * 4);
+  n += tc_align((size_t)(148 + 1) * 4);  // chunk counters: d / kChunk <= 148
   return n;
 }
 
@@ -635,56 +776,48 @@ cudaError_t launch_tc_ffn(int act, const void* h, int B, int d, int ffn, int n_h
   if ((e = make_map(&U.tm_h, h, d, B, (uint64_t)d * 2, 64, 16)) != cudaSuccess) return e;
   if ((e = make_map(&U.tm_w0, gated ? wg : wu, d, ffn, (uint64_t)d * 2, 64, 1)) != cudaSuccess) return e;
   if ((e = make_map(&U.tm_w1, wu, d, ffn, (uint64_t)d * 2, 64, 1)) != cudaSuccess) return e;
+  if ((e = make_map(&U.tm_t0, gated ? wg : wu, d, ffn, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
+  if ((e = make_map(&U.tm_t1, wu, d, ffn, (uint64_t)d * 2, 64, 128)) != cudaSuccess) return e;
   U.idx = idx;
   U.count = count;
   U.pre = S.pre;
+  U.b1 = b1;
+  U.act16 = S.act16;
+  U.tcnt = S.tcnt;
   U.ctrl = ctrl;
   U.d = d;
   U.ffn = ffn;
   U.n_hot = n_hot;
   U.gated = gated;
+  U.act = act;
+  U.B = B;
+  U.fpad = fpad;
   const int up_smem = kUpNS * kUpStage + kBarBytes + 1024;
   if ((e = cudaFuncSetAttribute(k_tc_up, cudaFuncAttributeMaxDynamicSharedMemorySize, up_smem)) != cudaSuccess)
     return e;
   k_tc_up<<<G, kTcThreads, up_smem, st>>>(U);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-  TcActParams A;
-  A.pre = S.pre;
-  A.b1 = b1;
-  A.act16 = S.act16;
-  A.idx = idx;
-  A.count = count;
-  A.ctrl = ctrl;
-  A.d = d;
-  A.ffn = ffn;
-  A.n_hot = n_hot;
-  A.act = act;
-  A.gated = gated;
-  A.B = B;
-  A.fpad = fpad;
-  A.G = G;
-  k_tc_act<<<(fpad + 127) / 128, 128, 0, st>>>(A);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-
   TcDownParams D;
   memset(&D, 0, sizeof(D));
   if ((e = make_map(&D.tm_wd, wd, d, ffn, (uint64_t)d * 2, 64, 1)) != cudaSuccess) return e;
+  if ((e = make_map(&D.tm_wdt, wd, d, ffn, (uint64_t)d * 2, 64, 64)) != cudaSuccess) return e;
   if ((e = make_map(&D.tm_act, S.act16, fpad, 32, (uint64_t)fpad * 2, 64, 32)) != cudaSuccess) return e;
   D.idx = idx;
   D.count = count;
   D.part = S.part;
+  D.b2 = b2;
+  D.y = y;
+  D.ccnt = S.ccnt;
   D.ctrl = ctrl;
   D.d = d;
   D.ffn = ffn;
   D.n_hot = n_hot;
+  D.B = B;
   const int dn_smem = kDnNS * kDnStage + kBarBytes + 1024;
   if ((e = cudaFuncSetAttribute(k_tc_down, cudaFuncAttributeMaxDynamicSharedMemorySize, dn_smem)) != cudaSuccess)
     return e;
   k_tc_down<<<G, kTcThreads, dn_smem, st>>>(D);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-
-  k_tc_reduce<<<(B * d + 255) / 256, 256, 0, st>>>(S.part, count, n_hot, ffn, d, B, G, b2, y, ctrl);
   return cudaGetLastError();
 }
 

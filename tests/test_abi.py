@@ -112,8 +112,8 @@ def test_launch_plan_is_host_only():
     launch for token blocks of 1-2 on every workload shape; for token blocks of
     3-16 an fp16 predictor runs on the tensor cores (P1 and P2 row dots,
     threshold, compaction), fp16 weights (d % 256 == 0) on the tcgen05 FFN
-    (up, activations, down, reduce), then the glue: 9 per layer (8 with Q4_0
-    weights, whose FFN runs on CUDA cores); a shape the
+    (up with the activation, down with the reduction), then the glue: 7 per
+    layer (8 with Q4_0 weights, whose FFN runs on CUDA cores); a shape the
     persistent kernel does not take runs the CUDA-core kernels (u, scores,
     compaction; gate/up, down, reduce; glue: 7 per layer, 5 with no cold
     neurons); -1 for invalid arguments."""
@@ -124,7 +124,7 @@ def test_launch_plan_is_host_only():
         for batch in (1, 2):
             assert lib.pi_stack_launches(ctypes.byref(desc), batch, w.layers) == 1, (w.name, batch)
         pred = 4 if w.ptype == "f16" else 3
-        ffn = 4 if (w.wtype == "f16" and w.ptype == "f16") else 3
+        ffn = 2 if (w.wtype == "f16" and w.ptype == "f16") else 3
         for batch in (3, 8, 16):
             want = (pred + ffn + 1) * w.layers
             assert lib.pi_stack_launches(ctypes.byref(desc), batch, w.layers) == want, (w.name, batch)

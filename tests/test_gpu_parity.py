@@ -140,6 +140,31 @@ def test_threshold_extremes_and_no_cold_neurons():
     assert rel_err(y.cpu().numpy(), full) <= TOL["f16"]
 
 
+def test_token_block_extremes_on_tensor_cores():
+    """Token blocks on the tcgen05 FFN (fp16, d % 256 == 0, B = 3..16): an
+    empty list (no hot rows and nothing predicted: y = b2), every neuron
+    active (the dense FFN), and one workspace reused by calls whose lists
+    differ in length (the per-tile and per-chunk writer counters are back at
+    zero after every call)."""
+    for act, B in (("relu", 4), ("reglu", 16)):
+        wl = _workload("tc-edge-" + act, 512, 1000, 0.0, 32, act, "f16", "f16", B)
+        L = _layer(wl)
+        h = to_dev(W.make_tokens(wl, B, 5))
+        h_np = to_np(h)
+        desc = pi.desc_for(wl)
+        ws = pi.workspace(desc, B)
+        for thr in (1e30, -1e30, wl.thr, 1e30, wl.thr, -1e30):
+            Lt = dict(L, thr=thr)
+            gidx, idx_t, cnt_t = gpu_predict(desc, h, Lt, ws)
+            if thr == 1e30:
+                assert len(gidx) == 0
+            if thr == -1e30:
+                assert len(gidx) == wl.n_cold
+            y = gpu_ffn(desc, h, Lt, idx_t, cnt_t, ws)
+            assert rel_err(y, oracle_layer(Lt, h_np, wl, gidx)) <= TOL["f16"], (act, thr)
+            assert pi.device_status(ws) == 0
+
+
 def test_bad_device_list_is_flagged_and_skipped():
     wl = _workload("badidx", 128, 500, 0.1, 16, "relu", "f16", "f16", 1)
     L = _layer(wl)
