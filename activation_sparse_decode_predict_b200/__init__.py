@@ -151,6 +151,21 @@ def decode_stack(desc: FfnDesc, layers, h_in: torch.Tensor, h_out: torch.Tensor,
                                  _stream(stream)))
 
 
+def set_token_block_ffn(path: str) -> None:
+    """Kernels for the sparse FFN of token blocks of 3-16 (fp16 weights):
+    "warp_mma" (row dots on warp-level mma.sync, the default) or "tcgen05"
+    (gathered tiles on the fifth-generation tensor cores).  Process-wide."""
+    if path not in _b.TOKEN_FFN:
+        raise ValueError("path must be one of %s" % sorted(_b.TOKEN_FFN))
+    _check(lib().pi_set_token_block_ffn(_b.TOKEN_FFN[path]))
+
+
+def token_block_ffn() -> str:
+    """The current token-block FFN kernels ("warp_mma" or "tcgen05")."""
+    v = lib().pi_get_token_block_ffn()
+    return {i: k for k, i in _b.TOKEN_FFN.items()}[v]
+
+
 def stack_launches(desc: FfnDesc, batch: int, n_layers: int) -> int:
     n = lib().pi_stack_launches(ctypes.byref(desc), int(batch), int(n_layers))
     if n < 0:

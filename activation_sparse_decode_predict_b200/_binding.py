@@ -20,10 +20,12 @@ STATUS_NAMES = {0: "PI_OK", -1: "PI_ERR_INVALID_ARG", -2: "PI_ERR_UNSUPPORTED", 
 DTYPES = {"f32": 0, "f16": 1, "q4_0": 2}
 ACTS = {"relu": 0, "reglu": 1, "relu2": 2}
 MAX_BATCH = 16
+TOKEN_FFN = {"warp_mma": 0, "tcgen05": 1}
 
 # Every symbol include/pi.h declares.
 EXPORTS = ("pi_workspace_bytes", "pi_workspace_init", "pi_predict", "pi_sparse_ffn", "pi_layer",
-           "pi_residual_rmsnorm", "pi_decode_stack", "pi_stack_launches", "pi_get_device_status",
+           "pi_residual_rmsnorm", "pi_decode_stack", "pi_stack_launches", "pi_set_token_block_ffn",
+           "pi_get_token_block_ffn", "pi_get_device_status",
            "pi_attn_workspace_bytes", "pi_sparse_attention", "pi_blocks_workspace_bytes", "pi_decode_blocks",
            "pi_predict_static", "pi_selftest_bounded_wait",
            "pi_last_error", "pi_version")
@@ -85,6 +87,10 @@ def load(path: str = LIB_PATH):
     lib.pi_decode_stack.restype = st
     lib.pi_stack_launches.argtypes = [D, i32, i32]
     lib.pi_stack_launches.restype = i32
+    lib.pi_set_token_block_ffn.argtypes = [i32]
+    lib.pi_set_token_block_ffn.restype = ctypes.c_int
+    lib.pi_get_token_block_ffn.argtypes = []
+    lib.pi_get_token_block_ffn.restype = i32
     lib.pi_get_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32), i32, P]
     lib.pi_get_device_status.restype = st
     A = ctypes.POINTER(AttnDesc)

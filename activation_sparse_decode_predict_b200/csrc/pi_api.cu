@@ -5,6 +5,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "pi.h"
 #include "pi_args.h"
 #include "pi_attn.cuh"
@@ -25,6 +27,14 @@ pi_status fail(pi_status st, const char* fmt, const char* what) {
 }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// the token-block FFN kernels (pi_set_token_block_ffn); process-wide
+std::atomic<int> g_token_ffn{PI_TOKEN_FFN_WARP_MMA};
+
+// whether a token block of this shape takes the tcgen05 FFN
+bool use_tc_ffn(int wtype, int ttype, int d, int B) {
+  return g_token_ffn.load(std::memory_order_relaxed) == PI_TOKEN_FFN_TCGEN05 && pi::tc_ffn_supported(wtype, ttype, d, B);
+}
 
 }  // namespace
 
@@ -149,7 +159,7 @@ pi_status ffn_impl(const pi_ffn_desc* d, int32_t B, const void* h, const int32_t
   float* partial = reinterpret_cast<float*>(ws + L.partial);
   const int sms = sm_count();
   const int ht = pi::token_type(d);
-  if (pi::kTcFfn && pi::tc_ffn_supported(d->wtype, ht, d->d, B)) {
+  if (use_tc_ffn(d->wtype, ht, d->d, B)) {
     // token blocks of 3..16 with fp16 weights: gathered tiles on tcgen05, fp32
     // accumulators in tensor memory, y (with b2) written by the last kernel
     PI_CUDA(pi::launch_tc_ffn(d->act, h, B, d->d, d->ffn, d->n_hot, idx, count, Wg.data, Wu.data, Wd.data, b1, b2, y,
@@ -673,6 +683,15 @@ pi_status pi_decode_blocks(const pi_ffn_desc* fdesc, const pi_attn_desc* adesc, 
   return PI_OK;
 }
 
+pi_status pi_set_token_block_ffn(int32_t path) {
+  if (path != PI_TOKEN_FFN_WARP_MMA && path != PI_TOKEN_FFN_TCGEN05)
+    return fail(PI_ERR_INVALID_ARG, "%s", "path must be PI_TOKEN_FFN_WARP_MMA or PI_TOKEN_FFN_TCGEN05");
+  g_token_ffn.store(path, std::memory_order_relaxed);
+  return PI_OK;
+}
+
+int32_t pi_get_token_block_ffn(void) { return g_token_ffn.load(std::memory_order_relaxed); }
+
 int32_t pi_stack_launches(const pi_ffn_desc* desc, int32_t batch, int32_t n_layers) {
   if (check_desc(desc, batch) != PI_OK || n_layers < 1 || n_layers > PI_MAX_LAYERS) return -1;
   {
@@ -690,7 +709,7 @@ int32_t pi_stack_launches(const pi_ffn_desc* desc, int32_t batch, int32_t n_laye
   else
     pred = cold ? 3 : 1;  // u, scores, compaction
   int ffn;
-  if (pi::kTcFfn && pi::tc_ffn_supported(desc->wtype, pi::token_type(desc), desc->d, batch))
+  if (use_tc_ffn(desc->wtype, pi::token_type(desc), desc->d, batch))
     ffn = 2;  // up (+ bias and activation), down (+ the sum over writers and b2)
   else
     ffn = 3;  // gate/up (or row dots), down, reduce

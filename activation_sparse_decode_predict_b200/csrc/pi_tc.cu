@@ -48,7 +48,7 @@ namespace pi {
 namespace {
 
 #ifndef PI_TC_KBS
-#define PI_TC_KBS 1
+#define PI_TC_KBS 2
 #endif
 #ifndef PI_TC_CHUNK
 #define PI_TC_CHUNK 256
@@ -238,9 +238,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_up(const __grid_constant__
     int cur = -1;
     int64_t issued = 0;
     bool ok = true;
+    // units: (tile, column block) pairs counted along the range without divisions
+    int t_nx = (int)(u0 / KB), k_nx = (int)(u0 % KB);
     for (int64_t u = u0; u < u1 && ok; ++u) {
       const int it = (int)(u - u0), s = it % kUpNS;
-      const int tile = (int)(u / KB), kb = (int)(u % KB);
+      const int tile = t_nx, kb = k_nx;
+      if (++k_nx == KB) { k_nx = 0; ++t_nx; }
       // a tile of hot rows only is 128 consecutive storage rows: one tiled load per matrix
       const bool hot_tile = tile * 128 + 128 <= p.n_hot;
       if (tile != cur) {
@@ -283,11 +286,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_up(const __grid_constant__
       constexpr uint32_t idesc = idesc_f16(128, 16, 0, 0);
       int buf = 0, nseg = 0, cur = -1;
       bool ok = true;
+      int t_nx = (int)(u0 / KB), k_nx = (int)(u0 % KB);
       for (int64_t u = u0; u < u1; ++u) {
         const int it = (int)(u - u0), s = it % kUpNS;
-        const int tile = (int)(u / KB);
+        const int tile = t_nx;
+        if (++k_nx == KB) { k_nx = 0; ++t_nx; }
         const bool first = tile != cur;
-        const bool last = (u + 1 == u1) || ((u + 1) / KB != tile);
+        const bool last = (u + 1 == u1) || k_nx == 0;
         if (first) {
           cur = tile;
           // this accumulator buffer was last used two segments ago: wait until it is drained
@@ -328,10 +333,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_up(const __grid_constant__
     // sum whoever is last) and finishes the tile.
     const int q = warp & 3, et = threadIdx.x - 32 * (kMmaWarp + 1);
     int buf = 0, nseg = 0;
+    int t_nx = (int)(u0 / KB), k_nx = (int)(u0 % KB);
     for (int64_t u = u0; u < u1; ++u) {
-      const int tile = (int)(u / KB);
-      const bool last = (u + 1 == u1) || ((u + 1) / KB != tile);
+      const int tile = t_nx;
+      if (++k_nx == KB) { k_nx = 0; ++t_nx; }
+      const bool last = (u + 1 == u1) || k_nx == 0;
       if (!last) continue;
+      // the segment's bookkeeping and this position's bias are looked up while
+      // the accumulators are still being filled
+      const int pos = tile * 128 + q * 32 + lane;
+      const int c_lo = range_owner(sp, (int64_t)tile * KB);
+      const int nw = range_owner(sp, (int64_t)tile * KB + KB - 1) - c_lo + 1, slot = c - c_lo;
+      float bias = 0.f;
+      if (pos < ntot && p.b1) bias = __ldg(p.b1 + list_row_at(pos, ntot, p.n_hot, p.ffn, p.idx, ctrl));
       const bool okw = mbar_wait(&accf[buf], (uint32_t)((nseg / 2) & 1), ctrl);
       if (named_sync_or(1, 128, !okw)) break;  // all epilogue warps leave together
       tc_fence_after();
@@ -349,9 +363,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_up(const __grid_constant__
       if (lane == 0) mbar_arrive(&acce[buf]);
       buf ^= 1;
       ++nseg;
-      const int pos = tile * 128 + q * 32 + lane;
-      const int c_lo = range_owner(sp, (int64_t)tile * KB);
-      const int nw = range_owner(sp, (int64_t)tile * KB + KB - 1) - c_lo + 1, slot = c - c_lo;
       if (nw > 1) {
         if (slot >= kTcSlots) {
           if (et == 0) set_status(&ctrl->status, kStCapacity);
@@ -364,16 +375,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_up(const __grid_constant__
             for (int i = 0; i < 4; ++i) dst[4 + i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
           }
         }
-        __threadfence();
+        // the CTA barrier orders every epilogue thread's stores before thread 0's
+        // fence and count (release); the last writer's thread 0 fences after
+        // its count (acquire) before the barrier that lets the others read
         named_sync(1, 128);
         if (et == 0) {
+          __threadfence();
           const int prev = atomicAdd(p.tcnt + tile, 1);
           s_last = prev == nw - 1;
-          if (prev == nw - 1) p.tcnt[tile] = 0;  // every writer has counted: ready for the next call
+          if (prev == nw - 1) {
+            p.tcnt[tile] = 0;  // every writer has counted: ready for the next call
+            __threadfence();
+          }
         }
         named_sync(1, 128);
         if (!s_last) continue;
-        __threadfence();
 #pragma unroll
         for (int b = 0; b < 16; ++b) g[b] = v[b] = 0.f;
         if (pos < ntot) {
@@ -403,8 +419,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_up(const __grid_constant__
 #pragma unroll
         for (int b = 0; b < 16; ++b) a[b] = 0.f;
         if (pos < ntot) {
-          const int row = list_row_at(pos, ntot, p.n_hot, p.ffn, p.idx, ctrl);
-          const float bias = p.b1 ? __ldg(p.b1 + row) : 0.f;
 #pragma unroll
           for (int b = 0; b < 16; ++b)
             if (b < p.B) a[b] = p.gated ? act_eval(kReglu, g[b] + bias, v[b]) : act_eval(p.act, g[b] + bias, 0.f);
@@ -485,12 +499,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_down(const __grid_constant
   const uint32_t tmem = *tslot;
 
   if (warp < kProdWarps) {
-    // ---------------- TMA producers: a unit's kDnCB x 16 four-position gathers
+    // ---------------- TMA producers: a unit's 16 x kDnCB four-position gathers
     // are split evenly over the producer warps; lane l < opw of warp w does
-    // gather o = w opw + l: column block o / 16, list positions 4 (o % 16) .. + 3 ----------------
+    // gather o = w opw + l: list positions 4 (o / kDnCB) .. + 3, column block
+    // o % kDnCB (neighbouring lanes ask for neighbouring pieces of the same rows) ----------------
     constexpr int opw = kDnCB * 16 / kProdWarps;
     static_assert(opw <= 32, "one gather per lane and unit");
-    const int o = opw * warp + lane, cbo = o / 16, pg = o % 16;
+    const int o = opw * warp + lane, cbo = o % kDnCB, pg = o / kDnCB;
     const bool mine = lane < opw;
     int64_t issued = 0;
     bool ok = true;
@@ -498,22 +513,34 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_down(const __grid_constant
     // the unit is issued, so that no lookup waits on the path from a free
     // stage to its copies
     int ra[4] = {0, 0, 0, 0}, rb[4] = {0, 0, 0, 0};
+    // units: (chunk, position block) pairs counted along the range without
+    // divisions; kb2 is the position block two units ahead
+    int c_nx = KBp > 0 ? (int)(u0 / KBp) : 0, k_nx = KBp > 0 ? (int)(u0 % KBp) : 0;
+    int kb2 = k_nx;
     if (mine) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        if (u0 < u1) ra[i] = list_raw(((int)(u0 % KBp)) * 64 + 4 * pg + i, ntot, p.n_hot, p.idx);
-        if (u0 + 1 < u1) rb[i] = list_raw(((int)((u0 + 1) % KBp)) * 64 + 4 * pg + i, ntot, p.n_hot, p.idx);
+        if (u0 < u1) ra[i] = list_raw(kb2 * 64 + 4 * pg + i, ntot, p.n_hot, p.idx);
+      }
+    }
+    if (++kb2 == KBp) kb2 = 0;
+    if (mine) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (u0 + 1 < u1) rb[i] = list_raw(kb2 * 64 + 4 * pg + i, ntot, p.n_hot, p.idx);
       }
     }
     for (int64_t u = u0; u < u1 && ok; ++u) {
       const int it = (int)(u - u0), s = it % kDnNS;
-      const int chunk = (int)(u / KBp), kb = (int)(u % KBp);
+      const int chunk = c_nx, kb = k_nx;
+      if (++k_nx == KBp) { k_nx = 0; ++c_nx; }
+      if (++kb2 == KBp) kb2 = 0;
       int r[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         r[i] = ra[i];
         ra[i] = rb[i];
-        if (mine && u + 2 < u1) rb[i] = list_raw(((int)((u + 2) % KBp)) * 64 + 4 * pg + i, ntot, p.n_hot, p.idx);
+        if (mine && u + 2 < u1) rb[i] = list_raw(kb2 * 64 + 4 * pg + i, ntot, p.n_hot, p.idx);
       }
       if (it >= kDnNS) ok = mbar_wait(&empty[s], ((it / kDnNS) - 1) & 1, ctrl);
       ok = __all_sync(0xffffffffu, ok);
@@ -544,11 +571,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_down(const __grid_constant
       constexpr uint32_t idesc = idesc_f16(128, 32, 1, 0);
       int buf = 0, nseg = 0, cur = -1;
       bool ok = true;
+      int c_nx = KBp > 0 ? (int)(u0 / KBp) : 0, k_nx = KBp > 0 ? (int)(u0 % KBp) : 0;
       for (int64_t u = u0; u < u1; ++u) {
         const int it = (int)(u - u0), s = it % kDnNS;
-        const int chunk = (int)(u / KBp);
+        const int chunk = c_nx;
+        if (++k_nx == KBp) { k_nx = 0; ++c_nx; }
         const bool first = chunk != cur;
-        const bool last = (u + 1 == u1) || ((u + 1) / KBp != chunk);
+        const bool last = (u + 1 == u1) || k_nx == 0;
         if (first) {
           cur = chunk;
           if (nseg >= 2) ok = mbar_wait(&acce[buf], (uint32_t)(((nseg - 2) / 2) & 1), ctrl);
@@ -592,10 +621,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_down(const __grid_constant
       }
     }
     int buf = 0, nseg = 0;
+    int c_nx = KBp > 0 ? (int)(u0 / KBp) : 0, k_nx = KBp > 0 ? (int)(u0 % KBp) : 0;
     for (int64_t u = u0; u < u1; ++u) {
-      const int chunk = (int)(u / KBp);
-      const bool last = (u + 1 == u1) || ((u + 1) / KBp != chunk);
+      const int chunk = c_nx;
+      if (++k_nx == KBp) { k_nx = 0; ++c_nx; }
+      const bool last = (u + 1 == u1) || k_nx == 0;
       if (!last) continue;
+      const int c_lo = range_owner(sp, (int64_t)chunk * KBp);
+      const int nw = range_owner(sp, (int64_t)chunk * KBp + KBp - 1) - c_lo + 1;
       const bool okw = mbar_wait(&accf[buf], (uint32_t)((nseg / 2) & 1), ctrl);
       if (named_sync_or(1, 128, !okw)) break;  // all epilogue warps leave together
       tc_fence_after();
@@ -609,25 +642,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_down(const __grid_constant
         tmem_ld16(ta, hv);
         tmem_ld16(ta + 16, lv);
 #pragma unroll
-        for (int b = 0; b < 16; ++b) dst[b * kChunk + m * 128 + q * 32 + lane] = hv[b] + lv[b];
+        for (int b = 0; b < 16; ++b)
+          if (b < p.B) dst[b * kChunk + m * 128 + q * 32 + lane] = hv[b] + lv[b];  // token rows past B are not read
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acce[buf]);
       buf ^= 1;
       ++nseg;
-      const int c_lo = range_owner(sp, (int64_t)chunk * KBp);
-      const int nw = range_owner(sp, (int64_t)chunk * KBp + KBp - 1) - c_lo + 1;
-      __threadfence();
-      named_sync(1, 128);
+      named_sync(1, 128);  // as in the up kernel: release by thread 0 after the barrier
       if (et == 0) {
+        __threadfence();
         const int prev = atomicAdd(p.ccnt + chunk, 1);
         s_last = prev == nw - 1;
-        if (prev == nw - 1) p.ccnt[chunk] = 0;  // every writer has counted: ready for the next call
+        if (prev == nw - 1) {
+          p.ccnt[chunk] = 0;  // every writer has counted: ready for the next call
+          __threadfence();
+        }
       }
       named_sync(1, 128);
       if (!s_last) continue;
-      __threadfence();
       for (int k = et; k < nw && k < kGMaxWriters; k += 128) {
         const int cw = c_lo + k;
         const int sg = (range_lo(sp, cw) / KBp == chunk) ? 0 : 1;

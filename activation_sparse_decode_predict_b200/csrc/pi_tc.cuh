@@ -115,11 +115,6 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* tm, in
 // ---------------------------------------------------------------------------
 // launcher of the token-block FFN on tcgen05 (pi_tc.cu)
 
-#ifndef PI_TC_FFN
-#define PI_TC_FFN 1
-#endif
-constexpr bool kTcFfn = PI_TC_FFN != 0;  // 0: token blocks keep the mma.sync kernels of pi_batch.cu
-
 // true if the shape takes the tcgen05 token-block path
 bool tc_ffn_supported(int wtype, int ptype, int d, int B);
 // workspace bytes of that path: split-K dots, fp16 activation rows, partial outputs

@@ -80,6 +80,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=None, help="run fewer layers (smoke only; not a bench number)")
+    ap.add_argument("--token-ffn", default=None, choices=["warp_mma", "tcgen05"],
+                    help="FFN kernels for token blocks of 3-16 (default: the library's, warp_mma)")
     return ap.parse_args()
 
 
@@ -221,6 +223,8 @@ def run_ours(args, rank, world, local_rank):
     B = args.batch or wl.batches[0]
     n_layers = args.layers or wl.layers
     desc = pi.desc_for(wl)
+    if args.token_ffn is not None:
+        pi.set_token_block_ffn(args.token_ffn)
 
     layers = [W.make_layer(wl, l, device=dev) for l in range(n_layers)]
     torch.cuda.synchronize()
@@ -330,6 +334,7 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": wl.name, "d": wl.d, "ffn": wl.ffn, "layers": n_layers, "batch": B,
                    "sparsity": wl.sparsity, "hot": wl.n_hot, "rank": wl.rank, "act": wl.act, "weights": wl.wtype,
                    "predictor": wl.ptype,
+                   "token_ffn": pi.token_block_ffn() if B >= 3 else None,
                    "parallelism": "replicas" if world > 1 else "single",
                    "l2": "no flush: resident stack %.1f GB, %.2f GB streamed per step (L2 126 MB)" % (
                        _resident_bytes(layers) / 1e9, total_bytes / args.steps / 1e9),

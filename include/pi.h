@@ -244,6 +244,25 @@ PI_API pi_status pi_decode_stack(const pi_ffn_desc *desc, int32_t batch, int32_t
 PI_API int32_t pi_stack_launches(const pi_ffn_desc *desc, int32_t batch, int32_t n_layers);
 
 /*
+ * Which kernels run the sparse FFN of a token block of 3-16 tokens with fp16
+ * weights and fp16 tokens (d % 256 == 0, d / 256 <= 148):
+ *   PI_TOKEN_FFN_WARP_MMA  row-dot kernels on warp-level mma.sync, whole
+ *                          contiguous rows per copy (the default: the faster
+ *                          of the two on B200 at the 40B/70B shapes)
+ *   PI_TOKEN_FFN_TCGEN05   128-neuron tiles gathered by TMA into shared memory,
+ *                          tcgen05.mma with fp32 accumulators in tensor memory
+ * Both add every sum in a fixed order, so each is deterministic; they differ
+ * in rounding order only.  The choice is process-wide and holds for calls
+ * issued after it returns (pi_sparse_ffn, pi_layer, pi_decode_stack,
+ * pi_decode_blocks and pi_stack_launches).  PI_ERR_INVALID_ARG for any other
+ * value.
+ */
+#define PI_TOKEN_FFN_WARP_MMA 0
+#define PI_TOKEN_FFN_TCGEN05 1
+PI_API pi_status pi_set_token_block_ffn(int32_t path);
+PI_API int32_t pi_get_token_block_ffn(void);
+
+/*
  * Read (and optionally clear) the sticky device status word of `ws`.  Waits
  * for `stream`.  *status_out = PI_OK or the first device-side error recorded.
  */

@@ -1,5 +1,7 @@
 """Helpers shared by the GPU parity tests: run libpi through its C ABI and
 compare with the CPU oracle on the same seeded inputs."""
+import contextlib
+
 import numpy as np
 import torch
 
@@ -79,3 +81,15 @@ def oracle_layer(L, h_np, wl, idx, cols=None):
 
 def oracle_predict(L, h_np, wl):
     return oracle.predict(h_np, to_np(L["P1"]), to_np(L["P2"]), to_np(L["bp"]), L["thr"], wl.n_hot, wl.ffn)
+
+
+@contextlib.contextmanager
+def token_ffn(path):
+    """Run the body with the token-block FFN kernels `path` ("warp_mma" or
+    "tcgen05"), then restore the previous choice."""
+    old = pi.token_block_ffn()
+    pi.set_token_block_ffn(path)
+    try:
+        yield
+    finally:
+        pi.set_token_block_ffn(old)

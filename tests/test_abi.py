@@ -111,9 +111,10 @@ def test_launch_plan_is_host_only():
     """pi_stack_launches plans a decode step without a GPU: one persistent
     launch for token blocks of 1-2 on every workload shape; for token blocks of
     3-16 an fp16 predictor runs on the tensor cores (P1 and P2 row dots,
-    threshold, compaction), fp16 weights (d % 256 == 0) on the tcgen05 FFN
-    (up with the activation, down with the reduction), then the glue: 7 per
-    layer (8 with Q4_0 weights, whose FFN runs on CUDA cores); a shape the
+    threshold, compaction), the FFN on the warp-level kernels (gate/up row
+    dots, down, reduce) or, when chosen, fp16 weights (d % 256 == 0) on the
+    tcgen05 kernels (up with the activation, down with the reduction), then
+    the glue: 8 per layer (7 on tcgen05; 8 with Q4_0 weights); a shape the
     persistent kernel does not take runs the CUDA-core kernels (u, scores,
     compaction; gate/up, down, reduce; glue: 7 per layer, 5 with no cold
     neurons); -1 for invalid arguments."""
@@ -124,10 +125,13 @@ def test_launch_plan_is_host_only():
         for batch in (1, 2):
             assert lib.pi_stack_launches(ctypes.byref(desc), batch, w.layers) == 1, (w.name, batch)
         pred = 4 if w.ptype == "f16" else 3
-        ffn = 2 if (w.wtype == "f16" and w.ptype == "f16") else 3
-        for batch in (3, 8, 16):
-            want = (pred + ffn + 1) * w.layers
-            assert lib.pi_stack_launches(ctypes.byref(desc), batch, w.layers) == want, (w.name, batch)
+        for path in ("warp_mma", "tcgen05"):
+            pi.set_token_block_ffn(path)
+            ffn = 2 if (path == "tcgen05" and w.wtype == "f16" and w.ptype == "f16") else 3
+            for batch in (3, 8, 16):
+                want = (pred + ffn + 1) * w.layers
+                assert lib.pi_stack_launches(ctypes.byref(desc), batch, w.layers) == want, (w.name, batch, path)
+        pi.set_token_block_ffn("warp_mma")
     odd = _desc(d=520, ffn=2048, n_hot=103, rank=64, act="relu")  # d not a multiple of 256
     assert lib.pi_stack_launches(ctypes.byref(odd), 1, 4) == 28
     all_hot = _desc(d=512, ffn=2048, n_hot=2048, rank=64, act="relu", wtype="f32", ptype="f32")
@@ -188,3 +192,18 @@ def test_sparse_attention_checks_before_any_launch():
     assert call(good, x=ctypes.c_void_p((1 << 20) + 8)) == B.PI_ERR_INVALID_ARG and b"x" in lib.pi_last_error()
     assert call(good, hidx=None) == B.PI_ERR_INVALID_ARG and b"head_idx" in lib.pi_last_error()
     assert call(good, ws_bytes=4096) == B.PI_ERR_CAPACITY
+
+
+def test_token_block_ffn_switch():
+    """The token-block FFN kernels are chosen process-wide; warp_mma is the
+    default, any other value than the two paths is refused."""
+    lib = pi.lib()
+    assert pi.token_block_ffn() == "warp_mma"
+    pi.set_token_block_ffn("tcgen05")
+    assert lib.pi_get_token_block_ffn() == 1
+    assert lib.pi_set_token_block_ffn(7) == B.PI_ERR_INVALID_ARG
+    assert pi.token_block_ffn() == "tcgen05"
+    pi.set_token_block_ffn("warp_mma")
+    assert lib.pi_get_token_block_ffn() == 0
+    with pytest.raises(ValueError):
+        pi.set_token_block_ffn("cuda_cores")

@@ -9,7 +9,7 @@ import activation_sparse_decode_predict_b200 as pi
 import oracle
 import pi_workload as W
 from gpu_util import (BAND, TOL, check_index_list, gpu_ffn, gpu_predict, oracle_layer, oracle_predict, rel_err,
-                      to_dev, to_np)
+                      to_dev, to_np, token_ffn)
 
 pytestmark = pytest.mark.gpu
 
@@ -44,8 +44,23 @@ def _layer(wl, layer=0):
     return {k: to_dev(v) if k not in ("perm", "p", "thr") else v for k, v in L.items()}
 
 
+# the shapes whose FFN the tcgen05 token-block kernels take (fp16, d % 256 == 0, B = 3..16)
+TC_SHAPES = [s for s in SHAPES if s[6] == "f16" and s[7] == "f16" and s[1] % 256 == 0 and 3 <= s[-1] <= 16]
+
+
 @pytest.mark.parametrize("shape", SHAPES, ids=[s[0] for s in SHAPES])
 def test_predict_and_sparse_ffn_match_oracle(shape):
+    _shape_check(shape)
+
+
+@pytest.mark.parametrize("shape", TC_SHAPES, ids=[s[0] for s in TC_SHAPES])
+def test_token_blocks_on_tcgen05_match_oracle(shape):
+    """The same checks with the token-block FFN on the tcgen05 kernels."""
+    with token_ffn("tcgen05"):
+        _shape_check(shape)
+
+
+def _shape_check(shape):
     wl = _workload(*shape)
     B = shape[-1]
     L = _layer(wl)
@@ -83,10 +98,17 @@ INT_CASES = [
 ]
 
 
+@pytest.mark.parametrize("path", ["warp_mma", "tcgen05"])
 @pytest.mark.parametrize("case", INT_CASES)
-def test_integer_exact_layers_are_bit_identical(case):
+def test_integer_exact_layers_are_bit_identical(case, path):
     """Every product and partial sum is an exact small integer (or dyadic), so
-    the GPU must equal the oracle bit for bit in any summation order."""
+    the GPU must equal the oracle bit for bit in any summation order (token
+    blocks through either FFN kernel family)."""
+    with token_ffn(path):
+        _int_check(case)
+
+
+def _int_check(case):
     d, ffn, n_hot, rank, act, wt, pt, B = case
     L = W.make_int_layer(d, ffn, n_hot, rank, act, wt, pt, B, seed=d + ffn + B)
     L = {k: to_dev(v) if k not in ("perm", "thr") else v for k, v in L.items()}
@@ -140,12 +162,18 @@ def test_threshold_extremes_and_no_cold_neurons():
     assert rel_err(y.cpu().numpy(), full) <= TOL["f16"]
 
 
-def test_token_block_extremes_on_tensor_cores():
-    """Token blocks on the tcgen05 FFN (fp16, d % 256 == 0, B = 3..16): an
-    empty list (no hot rows and nothing predicted: y = b2), every neuron
-    active (the dense FFN), and one workspace reused by calls whose lists
-    differ in length (the per-tile and per-chunk writer counters are back at
-    zero after every call)."""
+@pytest.mark.parametrize("path", ["warp_mma", "tcgen05"])
+def test_token_block_extremes(path):
+    """Token blocks (fp16, d % 256 == 0, B = 3..16) through either FFN kernel
+    family: an empty list (no hot rows and nothing predicted: y = b2), every
+    neuron active (the dense FFN), and one workspace reused by calls whose
+    lists differ in length (on tcgen05 the per-tile and per-chunk writer
+    counters are back at zero after every call)."""
+    with token_ffn(path):
+        _token_block_extremes()
+
+
+def _token_block_extremes():
     for act, B in (("relu", 4), ("reglu", 16)):
         wl = _workload("tc-edge-" + act, 512, 1000, 0.0, 32, act, "f16", "f16", B)
         L = _layer(wl)
@@ -272,6 +300,20 @@ FULL = [("7b-reglu-fp16", 1), ("13b-reglu-q4_0", 1), ("40b-relu-fp16", 1), ("40b
 def test_full_size_workloads_two_layers_sampled(name, B):
     """Full workload shapes through pi_decode_stack; every active-list entry is
     checked, y on 48 sampled columns (the oracle computes them one by one)."""
+    _full_check(name, B)
+
+
+FULL_TB = [f for f in FULL if f[1] >= 3]
+
+
+@pytest.mark.parametrize("name,B", FULL_TB, ids=["%s-b%d" % f for f in FULL_TB])
+def test_full_size_token_blocks_on_tcgen05(name, B):
+    """The full-size token blocks with their FFN on the tcgen05 kernels."""
+    with token_ffn("tcgen05"):
+        _full_check(name, B)
+
+
+def _full_check(name, B):
     wl = W.WORKLOADS[name]
     rng = np.random.default_rng(B)
     cols = np.sort(rng.choice(wl.d, size=48, replace=False)).astype(np.int32)
