@@ -98,6 +98,18 @@ def main(argv=None) -> int:
     se = (t[lo:, :, 6] - t[lo:, :, 6].min(1, keepdims=True)) / 1e3
     print("stream end after the first CTA's: median %.2f  p90 %.2f  max %.2f" % (
         med(se), np.percentile(se, 90), med(se.max(1))))
+    last = np.argmax(t[lo:, :, 6], axis=1)
+    ids, cnt = np.unique(last, return_counts=True)
+    top = sorted(zip(cnt, ids), reverse=True)[:5]
+    print("CTAs ending the stream last (layers %d..%d): %s" % (lo, NL - 1, ", ".join("%d x%d" % (i, c) for c, i in top)))
+    # stream end vs the CTA's own predicted cold rows and its SM's position
+    se_ctas = np.median(se, axis=0)
+    nl = np.median(t[lo:, :, 15], axis=0)
+    if np.std(nl) > 0:
+        print("stream end vs local predicted rows: correlation %.2f" % float(np.corrcoef(se_ctas, nl)[0, 1]))
+    half = G // 2
+    print("median stream end after the first, CTAs 0..%d: %.2f  CTAs %d..%d: %.2f" % (
+        half - 1, med(se[:, :half]), half, G - 1, med(se[:, half:])))
     nloc = t[lo:, :, 15]
     print("local predicted cold rows per CTA: mean %.1f  max %.1f (median over layers)" % (
         nloc.mean(), med(nloc.max(1))))
