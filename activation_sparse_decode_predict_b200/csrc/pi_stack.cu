@@ -694,13 +694,13 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
         const int nloc = s.misc[0];
         PI_STAMP(l, 12);
         PI_STAMP_VAL(l, 15, nloc);
-        // A CTA with clearly more predicted rows than it has seen on average
-        // hands the excess to the other CTAs (slots reserved with one atomic,
+        // A CTA with more predicted rows than its running mean (rounded up,
+        // plus p.don_slack) hands the excess to the other CTAs (slots reserved with one atomic,
         // written as row + 1); every CTA takes handed-over rows by ticket once
         // its hot-neuron claims run out, until a ticket lands past the last
         // slot after every CTA has decided -- so no slot is left behind.
         int keep = nloc;
-        if (kDonate && l > 0) keep = min(nloc, (int)ceilf(cold_avg) + 2);
+        if (kDonate && l > 0) keep = min(nloc, (int)ceilf(cold_avg) + p.don_slack);
         cold_avg = (l == 0) ? (float)nloc : 0.75f * cold_avg + 0.25f * (float)nloc;
         const int give = nloc - keep;
         if (give > 0) {

@@ -100,6 +100,7 @@ struct StackParams {
   int hot_a;       // hot neurons [0, hot_a) are shared out statically, consumed before barrier U
   int hot_static;  // [hot_a, hot_static) are shared out statically, at the head of the neuron
                    // stream; the rest, [hot_static, n_hot), are claimed
+  int don_slack;   // a CTA keeps its predicted cold rows up to its running mean + don_slack
   int cmp_layers;  // layers per chunk of the final list compaction
   int off_bars, off_itemoff, off_u, off_bp, off_cidx, off_act, off_red, off_gred, off_misc;
   int off_hb, off_ub, off_zero, off_redp, off_sc;

@@ -47,9 +47,9 @@ REF_SECONDS = 150.0  # cap on the timed oracle work of the reference arm
 # capture of a few layers of the workload (the committed ncu summaries);
 # per-layer traffic does not depend on the layer count, so a launch over L
 # layers moves L times this.  Only for captures of the current kernel.
-TRAFFIC_PER_LAYER = {("7b-reglu-fp16", 1): (276943360 + 3626496) / 4,
-                     ("13b-reglu-q4_0", 1): (208071680 + 3443968) / 4,
-                     ("70b-reglu-fp16", 1): (1316775424 + 3609856) / 4}
+TRAFFIC_PER_LAYER = {("7b-reglu-fp16", 1): (271105792 + 3212032) / 4,
+                     ("13b-reglu-q4_0", 1): (208271616 + 3159808) / 4,
+                     ("70b-reglu-fp16", 1): (1318978816 + 4201984) / 4}
 FALLBACK_HBM_GBS = 6650.0
 
 

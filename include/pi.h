@@ -184,7 +184,9 @@ PI_API pi_status pi_predict(const pi_ffn_desc *desc, int32_t batch, const void *
  *         ReLU^2: a = max(W_up[j].h_b + b1[j], 0)^2
  *     y[b, :] = b2 + sum over listed j of a * W_downT[j, :]
  * Every token of the block uses the same list (the union mask).  Dots and the
- * output accumulate in fp32; the activation is never rounded below fp32.
+ * output accumulate in fp32; the activation is kept in fp32, except that
+ * token blocks of 3-16 with fp16 weights feed it to the tensor cores as an
+ * fp16 pair hi + lo (hi = round(a), lo = round(a - hi), about 22 bits).
  * `count` is read on the device (no host synchronisation); an index outside
  * [n_hot, ffn) or a count above C sets PI_ERR_INDEX / PI_ERR_CAPACITY in the
  * status word and is skipped.
