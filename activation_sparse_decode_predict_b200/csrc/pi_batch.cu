@@ -27,6 +27,7 @@
 
 #include "pi_batch.cuh"
 #include "pi_common.cuh"
+#include "pi_launch.h"
 #include "pi_mma.cuh"
 #include "pi_sync.cuh"
 
@@ -177,6 +178,11 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_rowdot(const __grid_constant__ 
   uint8_t* ring = sm + Lay.off_ring;
   Ctrl* ctrl = p.ctrl;
 
+  pdl_trigger();
+  // list mode: the rows to stream come from the kernels before; plain mode
+  // streams rows that no kernel writes, so the producer starts before the
+  // previous kernel has finished and only the consumers wait (for the token rows)
+  if (p.list) pdl_wait();
   const int R = gridDim.x / p.S;
   const int rho = blockIdx.x / p.S, sig = blockIdx.x % p.S;
   const int col0 = sig * Lay.PC;
@@ -231,6 +237,7 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_rowdot(const __grid_constant__ 
   }
 
   // ---------------- consumer warps ----------------
+  if (!p.list) pdl_wait();
   const int t = threadIdx.x - 32, cw = t >> 5, lane = t & 31;
   // this part's token columns -> shared memory (rows >= ntok are zero)
   if (p.upre) {
@@ -353,6 +360,8 @@ __global__ void __launch_bounds__(256) k_bthresh(const float* __restrict__ sc, i
                                                  const float* __restrict__ bp, float thr,
                                                  uint32_t* __restrict__ tile_mask, int* __restrict__ tile_count) {
   __shared__ int cnt[8];
+  pdl_trigger();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = blockIdx.x * 256 + threadIdx.x;
   bool on = false;
@@ -413,6 +422,8 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_bdown(const __grid_constant__ B
   uint8_t* abuf = sm + Lay.off_a;
   uint8_t* ring = sm + Lay.off_ring;
   Ctrl* ctrl = p.ctrl;
+  pdl_trigger();
+  pdl_wait();  // the list, its count and the pre-activations come from the kernels before
 
   const int DC = p.d / Lay.DCOLS;
   const int chi = blockIdx.x % DC, rho = blockIdx.x / DC;
@@ -574,8 +585,8 @@ cudaError_t launch_rowdot_t(const RowDotParams& P, int G, cudaStream_t st) {
   const UpLayout UL = up_layout(NT * 8, P.K, P.S);
   cudaError_t e = cudaFuncSetAttribute(k_rowdot<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, UL.bytes);
   if (e != cudaSuccess) return e;
-  k_rowdot<NT><<<G, kBT + 32, UL.bytes, st>>>(P);
-  return cudaGetLastError();
+  e = launch_pdl(k_rowdot<NT>, dim3(G), dim3(kBT + 32), UL.bytes, st, P);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_rowdot(const RowDotParams& P, int sms, cudaStream_t st) {
@@ -648,7 +659,9 @@ cudaError_t launch_batch_predict(const void* h, int B, int d, int r, int C, int 
   S.W = 1;
   e = launch_rowdot(S, sms, st);
   if (e != cudaSuccess) return e;
-  k_bthresh<<<(C + 255) / 256, 256, 0, st>>>(sc, S.S, C, B, bp, thr, tile_mask, tile_count);
+  e = launch_pdl(k_bthresh, dim3((C + 255) / 256), dim3(256), 0, st, static_cast<const float*>(sc), S.S, C, B, bp, thr,
+                 tile_mask, tile_count);
+  if (e != cudaSuccess) return e;
   (void)n_hot;
   return cudaGetLastError();
 }
@@ -699,11 +712,13 @@ cudaError_t launch_batch_ffn(int act, const void* h, int B, int d, int ffn, int 
   if (NT == 1) {
     e = cudaFuncSetAttribute(k_bdown<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, DL.bytes);
     if (e != cudaSuccess) return e;
-    k_bdown<1><<<Gd, kBT + 32, DL.bytes, st>>>(D);
+    e = launch_pdl(k_bdown<1>, dim3(Gd), dim3(kBT + 32), DL.bytes, st, D);
+    if (e != cudaSuccess) return e;
   } else {
     e = cudaFuncSetAttribute(k_bdown<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, DL.bytes);
     if (e != cudaSuccess) return e;
-    k_bdown<2><<<Gd, kBT + 32, DL.bytes, st>>>(D);
+    e = launch_pdl(k_bdown<2>, dim3(Gd), dim3(kBT + 32), DL.bytes, st, D);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }

@@ -39,6 +39,16 @@ static_assert(sizeof(Ctrl) == 2304, "control block is 2304 bytes");
 
 __device__ __forceinline__ void set_status(int* status, int code) { atomicCAS(status, 0, code); }
 
+// Programmatic dependent launch (kernels launched with launch_pdl): a kernel
+// lets the next kernel on its stream be scheduled before it ends
+// (pdl_trigger), and a thread waits for the previous kernel to complete with
+// its memory visible (pdl_wait) before it reads anything that kernel wrote
+// or writes global memory.  Work that depends on neither (barrier set-up,
+// copies of weights nobody writes) may come before the wait.  Both are
+// no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Elements per access unit.
 template <int T> struct Unit;
 template <> struct Unit<kF32> { static constexpr int E = 4; };

@@ -8,6 +8,7 @@
 // bahasa besar ...", "Keterbatasan dan FAQ" (ReLU, ReGLU, squared ReLU).
 #include "pi_common.cuh"
 #include "pi_kernels_v1.cuh"
+#include "pi_launch.h"
 
 namespace pi {
 
@@ -121,6 +122,8 @@ __global__ void __launch_bounds__(256) k_compact(const uint32_t* __restrict__ ti
                                                  int32_t* __restrict__ idx, int32_t* __restrict__ count) {
   __shared__ int red[8];
   __shared__ int wpre[9];
+  pdl_trigger();
+  pdl_wait();
   const int tile = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int before = 0, total = 0;
   for (int t = threadIdx.x; t < n_tiles; t += blockDim.x) {
@@ -291,6 +294,8 @@ __global__ void k_ffn_down(int B, int d, int ffn, int n_hot, const int32_t* __re
 __global__ void __launch_bounds__(256) k_ffn_reduce(const float* __restrict__ partial, int G, int BD,
                                                     const float* __restrict__ b2, int d, float* __restrict__ y) {
   __shared__ float4 grp[8][32];
+  pdl_trigger();
+  pdl_wait();
   const int col4 = blockIdx.x * 32 + (threadIdx.x & 31);
   const int k = threadIdx.x >> 5;
   float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -325,6 +330,8 @@ constexpr int kNormUnits = 2;
 template <int HT>
 __global__ void __launch_bounds__(1024) k_rmsnorm(const void* __restrict__ h, const float* __restrict__ y, int d,
                                                   float eps, void* __restrict__ h_out) {
+  pdl_trigger();
+  pdl_wait();
   const int b = blockIdx.x;
   __shared__ float red[32];
   const int units = d / 8;
@@ -417,8 +424,8 @@ cudaError_t launch_compact(const uint32_t* tile_mask, const int* tile_count, int
                            int32_t* count, cudaStream_t st) {
   const int tiles = (C + 255) / 256;
   if (tiles == 0) return cudaMemsetAsync(count, 0, sizeof(int32_t), st);
-  k_compact<<<tiles, 256, 0, st>>>(tile_mask, tile_count, tiles, n_hot, idx, count);
-  return cudaGetLastError();
+  const cudaError_t e = launch_pdl(k_compact, dim3(tiles), dim3(256), 0, st, tile_mask, tile_count, tiles, n_hot, idx, count);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <int WT, int HT>
@@ -476,8 +483,8 @@ cudaError_t launch_ffn_down(int wtype, int B, int d, int ffn, int n_hot, const i
 cudaError_t launch_ffn_reduce(const float* partial, int G, int B, int d, const float* b2, float* y, cudaStream_t st) {
   const int BD = B * d;
   const int grid = (BD / 4 + 31) / 32;
-  k_ffn_reduce<<<grid, 256, 0, st>>>(partial, G, BD, b2, d, y);
-  return cudaGetLastError();
+  const cudaError_t e = launch_pdl(k_ffn_reduce, dim3(grid), dim3(256), 0, st, partial, G, BD, b2, d, y);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_rmsnorm(int htype, const void* h, const float* y, int B, int d, float eps, void* h_out,
@@ -487,9 +494,9 @@ cudaError_t launch_rmsnorm(int htype, const void* h, const float* y, int B, int 
   int threads = (units + kNormUnits - 1) / kNormUnits;
   threads = (threads + 31) / 32 * 32;
   if (threads > 1024 || d % 8 != 0) return cudaErrorInvalidValue;
-  if (htype == kF32) k_rmsnorm<kF32><<<B, threads, 0, st>>>(h, y, d, eps, h_out);
-  else k_rmsnorm<kF16><<<B, threads, 0, st>>>(h, y, d, eps, h_out);
-  return cudaGetLastError();
+  const cudaError_t e = htype == kF32 ? launch_pdl(k_rmsnorm<kF32>, dim3(B), dim3(threads), 0, st, h, y, d, eps, h_out)
+                                      : launch_pdl(k_rmsnorm<kF16>, dim3(B), dim3(threads), 0, st, h, y, d, eps, h_out);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace pi

@@ -40,6 +40,7 @@
 #include <mutex>
 
 #include "pi_common.cuh"
+#include "pi_launch.h"
 #include "pi_sync.cuh"
 #include "pi_tc.cuh"
 
@@ -190,6 +191,8 @@ struct TcUpParams {
 __global__ void __launch_bounds__(kTcThreads, 1) k_tc_up(const __grid_constant__ TcUpParams p) {
   extern __shared__ uint8_t smraw[];
   __shared__ int s_last;  // set by the epilogue: this CTA finishes the tile
+  pdl_trigger();
+  pdl_wait();  // the list, its count and the token block come from the kernels before
   uint8_t* sm = align1024(smraw);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + kUpNS * kUpStage);
   uint64_t* empty = full + kUpNS;
@@ -462,6 +465,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_down(const __grid_constant
   extern __shared__ uint8_t smraw[];
   __shared__ int s_last;  // set by the epilogue: this CTA finishes the chunk
   __shared__ int s_woff[kGMaxWriters];  // the chunk's partial outputs, by writer (offsets into part)
+  pdl_trigger();
+  pdl_wait();  // the list, its count and the activation rows come from the kernels before
   uint8_t* sm = align1024(smraw);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + kDnNS * kDnStage);
   uint64_t* empty = full + kDnNS;
@@ -829,7 +834,7 @@ cudaError_t launch_tc_ffn(int act, const void* h, int B, int d, int ffn, int n_h
   const int up_smem = kUpNS * kUpStage + kBarBytes + 1024;
   if ((e = cudaFuncSetAttribute(k_tc_up, cudaFuncAttributeMaxDynamicSharedMemorySize, up_smem)) != cudaSuccess)
     return e;
-  k_tc_up<<<G, kTcThreads, up_smem, st>>>(U);
+  if ((e = launch_pdl(k_tc_up, dim3(G), dim3(kTcThreads), up_smem, st, U)) != cudaSuccess) return e;
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   TcDownParams D;
@@ -851,7 +856,7 @@ cudaError_t launch_tc_ffn(int act, const void* h, int B, int d, int ffn, int n_h
   const int dn_smem = kDnNS * kDnStage + kBarBytes + 1024;
   if ((e = cudaFuncSetAttribute(k_tc_down, cudaFuncAttributeMaxDynamicSharedMemorySize, dn_smem)) != cudaSuccess)
     return e;
-  k_tc_down<<<G, kTcThreads, dn_smem, st>>>(D);
+  if ((e = launch_pdl(k_tc_down, dim3(G), dim3(kTcThreads), dn_smem, st, D)) != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
