@@ -47,7 +47,7 @@ __device__ __forceinline__ int bshare(int n, int c, int G) { return (int)((int64
 // an entry outside [n_hot, ffn) is reported and replaced by row 0
 __device__ __forceinline__ int list_row(int pos, int n_hot, int ffn, const int32_t* idx, Ctrl* ctrl) {
   if (pos < n_hot) return pos;
-  const int j = __ldg(idx + (pos - n_hot));
+  const int j = __ldcg(idx + (pos - n_hot));
   if (j < n_hot || j >= ffn) {
     set_status(&ctrl->status, kStIndex);
     return -1;
@@ -67,7 +67,7 @@ __device__ __forceinline__ int row_at(const int* rmap, int pos, int n0, int n_ho
 }
 
 __device__ __forceinline__ int clamp_count(const int32_t* count, int C, Ctrl* ctrl, bool report) {
-  int cnt = *count;
+  int cnt = __ldcg(count);
   if (cnt < 0 || cnt > C) {
     if (report) set_status(&ctrl->status, kStCapacity);
     cnt = cnt < 0 ? 0 : C;
@@ -287,7 +287,7 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_rowdot(const __grid_constant__ 
     for (int i = t; i < NT * 8 * units; i += kBT) {
       const int b = i / units, u = i % units;
       uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (b < p.ntok) v = __ldg(reinterpret_cast<const uint4*>(p.x + (int64_t)b * p.K + col0) + u);
+      if (b < p.ntok) v = __ldcg(reinterpret_cast<const uint4*>(p.x + (int64_t)b * p.K + col0) + u);
       *reinterpret_cast<uint4*>(hs + b * Lay.HS + 16 * u) = v;
     }
   }
@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_rowdot(const __grid_constant__ 
 // score = sum over the parts of (hi + lo dots) + bp; active = OR over the
 // tokens of score > thr; one CTA per 256-row tile: 8 ballot words + count
 // (the tile format of the compaction kernel).
-__global__ void __launch_bounds__(256) k_bthresh(const float* __restrict__ sc, int S, int C, int B,
+__global__ void __launch_bounds__(256) k_bthresh(const float* sc, int S, int C, int B,
                                                  const float* __restrict__ bp, float thr,
                                                  uint32_t* __restrict__ tile_mask, int* __restrict__ tile_count) {
   __shared__ int cnt[8];

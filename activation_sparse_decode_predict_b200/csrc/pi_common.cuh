@@ -45,7 +45,11 @@ __device__ __forceinline__ void set_status(int* status, int code) { atomicCAS(st
 // its memory visible (pdl_wait) before it reads anything that kernel wrote
 // or writes global memory.  Work that depends on neither (barrier set-up,
 // copies of weights nobody writes) may come before the wait.  Both are
-// no-ops for a kernel launched without the attribute.
+// no-ops for a kernel launched without the attribute.  A kernel launched this
+// way overlaps the previous one, so data that kernel writes is not read-only
+// for this kernel's lifetime: it is read with plain or .cg loads after the
+// wait, never through __ldg / const __restrict__ (the non-coherent read-only
+// path, which the compiler may also move above the wait).
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
@@ -121,7 +125,9 @@ __device__ __forceinline__ void load_w_unit(const void* __restrict__ data, const
 }
 
 // Token values at the columns of unit u (layout of weight type WT) for token
-// row `b` of h [*, ld] of type HT (kF32 or kF16).  Cached loads: h is reused.
+// row `b` of h [*, ld] of type HT (kF32 or kF16).  Read-only cached loads
+// (h is reused by every warp of a CTA), so the kernels that call this are
+// launched without the dependent-launch attribute (see pdl_wait).
 template <int WT, int HT>
 __device__ __forceinline__ void load_h_unit(const void* __restrict__ h, int b, int ld, int u,
                                             float (&x)[Unit<WT>::E]) {

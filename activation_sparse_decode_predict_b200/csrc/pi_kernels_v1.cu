@@ -117,8 +117,8 @@ __global__ void __launch_bounds__(256) k_pred_score(const void* __restrict__ P2,
 // Order-preserving compaction: one CTA per tile.  Each CTA sums the counts of
 // the tiles before it (no inter-CTA waiting), then writes its tile's active
 // rows in ascending order.  CTA 0 also writes the total count.
-__global__ void __launch_bounds__(256) k_compact(const uint32_t* __restrict__ tile_mask,
-                                                 const int* __restrict__ tile_count, int n_tiles, int n_hot,
+__global__ void __launch_bounds__(256) k_compact(const uint32_t* tile_mask,
+                                                 const int* tile_count, int n_tiles, int n_hot,
                                                  int32_t* __restrict__ idx, int32_t* __restrict__ count) {
   __shared__ int red[8];
   __shared__ int wpre[9];
@@ -127,7 +127,7 @@ __global__ void __launch_bounds__(256) k_compact(const uint32_t* __restrict__ ti
   const int tile = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int before = 0, total = 0;
   for (int t = threadIdx.x; t < n_tiles; t += blockDim.x) {
-    const int c = tile_count[t];
+    const int c = __ldcg(tile_count + t);
     total += c;
     if (t < tile) before += c;
   }
@@ -138,10 +138,10 @@ __global__ void __launch_bounds__(256) k_compact(const uint32_t* __restrict__ ti
   }
   __shared__ int redt[8];
   if (lane == 0) { red[warp] = before; redt[warp] = total; }
-  const uint32_t m = tile_mask[tile * 8 + warp];
+  const uint32_t m = __ldcg(tile_mask + tile * 8 + warp);
   if (threadIdx.x == 0) {
     wpre[0] = 0;
-    for (int w = 0; w < 8; ++w) wpre[w + 1] = wpre[w] + __popc(tile_mask[tile * 8 + w]);
+    for (int w = 0; w < 8; ++w) wpre[w + 1] = wpre[w] + __popc(__ldcg(tile_mask + tile * 8 + w));
   }
   __syncthreads();
   int base = 0, tot = 0;
@@ -291,7 +291,7 @@ __global__ void k_ffn_down(int B, int d, int ffn, int n_hot, const int32_t* __re
 // Split-K reduction: y = b2 + sum_g partial[g] in a fixed order.  A CTA covers
 // 32 float4 columns x 8 partial groups; group k sums partials g = k mod 8 in
 // ascending order, then the 8 group sums are added in order.
-__global__ void __launch_bounds__(256) k_ffn_reduce(const float* __restrict__ partial, int G, int BD,
+__global__ void __launch_bounds__(256) k_ffn_reduce(const float* partial, int G, int BD,
                                                     const float* __restrict__ b2, int d, float* __restrict__ y) {
   __shared__ float4 grp[8][32];
   pdl_trigger();
@@ -328,7 +328,7 @@ __global__ void __launch_bounds__(256) k_ffn_reduce(const float* __restrict__ pa
 constexpr int kNormUnits = 2;
 
 template <int HT>
-__global__ void __launch_bounds__(1024) k_rmsnorm(const void* __restrict__ h, const float* __restrict__ y, int d,
+__global__ void __launch_bounds__(1024) k_rmsnorm(const void* h, const float* y, int d,
                                                   float eps, void* __restrict__ h_out) {
   pdl_trigger();
   pdl_wait();
@@ -342,15 +342,15 @@ __global__ void __launch_bounds__(1024) k_rmsnorm(const void* __restrict__ h, co
     const int u = threadIdx.x + v * blockDim.x;
     if (u < units) {
       const int64_t e0 = (int64_t)b * d + 8 * u;
-      const float4 y0 = __ldg(reinterpret_cast<const float4*>(y + e0));
-      const float4 y1 = __ldg(reinterpret_cast<const float4*>(y + e0) + 1);
+      const float4 y0 = __ldcg(reinterpret_cast<const float4*>(y + e0));
+      const float4 y1 = __ldcg(reinterpret_cast<const float4*>(y + e0) + 1);
       float hv[8];
       if constexpr (HT == kF32) {
-        const float4 a = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(h) + e0));
-        const float4 c = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(h) + e0) + 1);
+        const float4 a = __ldcg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(h) + e0));
+        const float4 c = __ldcg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(h) + e0) + 1);
         hv[0] = a.x; hv[1] = a.y; hv[2] = a.z; hv[3] = a.w; hv[4] = c.x; hv[5] = c.y; hv[6] = c.z; hv[7] = c.w;
       } else {
-        const uint4 q = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __half*>(h) + e0));
+        const uint4 q = __ldcg(reinterpret_cast<const uint4*>(reinterpret_cast<const __half*>(h) + e0));
         float2 f;
         f = h2f2(q.x); hv[0] = f.x; hv[1] = f.y;
         f = h2f2(q.y); hv[2] = f.x; hv[3] = f.y;

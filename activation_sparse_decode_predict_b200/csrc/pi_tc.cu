@@ -105,7 +105,7 @@ __device__ __forceinline__ int range_owner(const Split& s, int64_t u) {
 
 // the list length (hot rows + predicted) with the count clamped to [0, C]
 __device__ __forceinline__ int list_total(const int32_t* count, int n_hot, int ffn, Ctrl* ctrl, bool report) {
-  int cnt = *count;
+  int cnt = __ldcg(count);
   const int C = ffn - n_hot;
   if (cnt < 0 || cnt > C) {
     if (report) set_status(&ctrl->status, kStCapacity);
@@ -141,7 +141,7 @@ __device__ __forceinline__ Split down_split(int ntot, int d, int G) {
 __device__ __forceinline__ int list_row_at(int pos, int ntot, int n_hot, int ffn, const int32_t* idx, Ctrl* ctrl) {
   if (pos < n_hot) return pos;
   if (pos >= ntot) return 0;  // beyond the list: any valid row, its products are dropped or multiplied by zero
-  const int j = __ldg(idx + (pos - n_hot));
+  const int j = __ldcg(idx + (pos - n_hot));
   if (j < n_hot || j >= ffn) {
     set_status(&ctrl->status, kStIndex);
     return 0;
@@ -154,7 +154,7 @@ __device__ __forceinline__ int list_row_at(int pos, int ntot, int n_hot, int ffn
 __device__ __forceinline__ int list_raw(int pos, int ntot, int n_hot, const int32_t* idx) {
   if (pos < n_hot) return pos;
   if (pos >= ntot) return 0;
-  return __ldg(idx + (pos - n_hot));
+  return __ldcg(idx + (pos - n_hot));
 }
 __device__ __forceinline__ int list_checked(int j, int pos, int ntot, int n_hot, int ffn, Ctrl* ctrl) {
   if (pos >= n_hot && pos < ntot && (j < n_hot || j >= ffn)) {
