@@ -571,10 +571,14 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_bdown(const __grid_constant__ B
   }
 }
 
-// parts of K such that the token columns of one part (ntok rows rounded up
-// to the n-tile) stay within 64 KB of shared memory
+// n-tiles of 8 token rows the row-dot kernel stages (1, 2 or 4)
+int rowdot_nt(int ntok) { return ntok <= 8 ? 1 : (ntok <= 16 ? 2 : 4); }
+
+// parts of K such that the staged token columns of one part stay within
+// 64 KB of shared memory
+
 int row_parts(int ntok, int K) {
-  const size_t bytes = (size_t)((ntok + 7) / 8 * 8) * K * 2;
+  const size_t bytes = (size_t)(8 * rowdot_nt(ntok)) * K * 2;
   int S = 1;
   while ((size_t)S * 65536 < bytes) S *= 2;
   return S;
@@ -591,15 +595,16 @@ cudaError_t launch_rowdot_t(const RowDotParams& P, int G, cudaStream_t st) {
 
 cudaError_t launch_rowdot(const RowDotParams& P, int sms, cudaStream_t st) {
   const int G = (sms / P.S) * P.S;
-  if (P.ntok <= 8) return launch_rowdot_t<1>(P, G, st);
-  if (P.ntok <= 16) return launch_rowdot_t<2>(P, G, st);
+  const int NT = rowdot_nt(P.ntok);
+  if (NT == 1) return launch_rowdot_t<1>(P, G, st);
+  if (NT == 2) return launch_rowdot_t<2>(P, G, st);
   return launch_rowdot_t<4>(P, G, st);
 }
 
 bool rowdot_fits(int ntok, int K) {
   const int S = row_parts(ntok, K);
   if (S > 4 || K % (128 * S) != 0) return false;
-  return up_layout((ntok + 7) / 8 * 8, K, S).nslot >= 2;
+  return up_layout(8 * rowdot_nt(ntok), K, S).nslot >= 2;  // the token tile the kernel stages
 }
 
 }  // namespace
