@@ -177,7 +177,7 @@ pi_status ffn_impl(const pi_ffn_desc* d, int32_t B, const void* h, const int32_t
     PI_CUDA(pi::launch_ffn_reduce(partial, NR, B, d->d, b2, y, st), "split-K reduce launch");
     return PI_OK;
   }
-  const int G = L.g_max < 2 * sms ? L.g_max : 2 * sms;
+  const int G = pi::down_ranges(d->d, sms);
   PI_CUDA(pi::launch_ffn_act(d->wtype, ht, d->act, h, B, d->d, d->ffn, d->n_hot, idx, count, Wg.data,
                              Wg.scales, Wu.data, Wu.scales, b1, a, d->ffn, status, sms, st),
           "FFN activation launch");
@@ -611,7 +611,7 @@ pi_status pi_sparse_attention(const pi_attn_desc* desc, int32_t batch, const voi
   P.qkv = reinterpret_cast<float*>(w + L.qkv);
   P.part = reinterpret_cast<float*>(w + L.part);
   P.ctrl = reinterpret_cast<pi::Ctrl*>(w);
-  const int G = 2 * sms < pi::kGMax ? 2 * sms : pi::kGMax;
+  const int G = pi::down_ranges(desc->d, sms);
   PI_CUDA(pi::launch_attention(P, desc->wtype, desc->xtype, desc->ctype, reinterpret_cast<float*>(w + L.a),
                                reinterpret_cast<int32_t*>(w + L.orow), reinterpret_cast<int32_t*>(w + L.ocount),
                                reinterpret_cast<float*>(w + L.partial), G, y, sms, (cudaStream_t)stream),

@@ -93,35 +93,56 @@ __device__ __forceinline__ float half_bits_to_float(uint16_t v) {
   return __half2float(*reinterpret_cast<__half*>(&v));
 }
 
-// Load unit u of row `row` of a [rows, d] matrix of type T, decoded to floats.
-// Weights are streamed once, so loads bypass L1.
+// The raw bytes of unit u of row `row` of a [rows, d] matrix of type T
+// (Q4_0: the 8 code bytes and the block's fp16 scale), and their decoding to
+// floats.  Weights are streamed once, so loads bypass L1; a kernel that
+// wants several units in flight loads them all before decoding any.
+template <int T> struct WRaw { uint4 v; };
+template <> struct WRaw<kQ4_0> { uint2 q; uint16_t s; };
+
 template <int T>
-__device__ __forceinline__ void load_w_unit(const void* __restrict__ data, const void* __restrict__ scales, int64_t row,
-                                            int d, int u, float (&w)[Unit<T>::E]) {
+__device__ __forceinline__ WRaw<T> load_w_raw(const void* __restrict__ data, const void* __restrict__ scales,
+                                              int64_t row, int d, int u) {
+  WRaw<T> r;
   if constexpr (T == kF32) {
-    const uint4 v = ld_nc_v4(reinterpret_cast<const float*>(data) + row * d + u * 4);
-    w[0] = __uint_as_float(v.x); w[1] = __uint_as_float(v.y); w[2] = __uint_as_float(v.z); w[3] = __uint_as_float(v.w);
+    r.v = ld_nc_v4(reinterpret_cast<const float*>(data) + row * d + u * 4);
   } else if constexpr (T == kF16) {
-    const uint4 v = ld_nc_v4(reinterpret_cast<const __half*>(data) + row * d + u * 8);
-    float2 f;
-    f = h2f2(v.x); w[0] = f.x; w[1] = f.y;
-    f = h2f2(v.y); w[2] = f.x; w[3] = f.y;
-    f = h2f2(v.z); w[4] = f.x; w[5] = f.y;
-    f = h2f2(v.w); w[6] = f.x; w[7] = f.y;
+    r.v = ld_nc_v4(reinterpret_cast<const __half*>(data) + row * d + u * 8);
   } else {
-    const uint8_t* qs = reinterpret_cast<const uint8_t*>(data) + row * (d / 2) + u * 8;
-    const uint16_t* sc = reinterpret_cast<const uint16_t*>(scales) + row * (d / 32) + (u >> 1);
-    const uint2 q = ld_nc_v2(qs);
-    const float s = half_bits_to_float(__ldg(sc));
+    r.q = ld_nc_v2(reinterpret_cast<const uint8_t*>(data) + row * (d / 2) + u * 8);
+    r.s = __ldg(reinterpret_cast<const uint16_t*>(scales) + row * (d / 32) + (u >> 1));
+  }
+  return r;
+}
+
+template <int T>
+__device__ __forceinline__ void decode_w(const WRaw<T>& r, float (&w)[Unit<T>::E]) {
+  if constexpr (T == kF32) {
+    w[0] = __uint_as_float(r.v.x); w[1] = __uint_as_float(r.v.y); w[2] = __uint_as_float(r.v.z); w[3] = __uint_as_float(r.v.w);
+  } else if constexpr (T == kF16) {
+    float2 f;
+    f = h2f2(r.v.x); w[0] = f.x; w[1] = f.y;
+    f = h2f2(r.v.y); w[2] = f.x; w[3] = f.y;
+    f = h2f2(r.v.z); w[4] = f.x; w[5] = f.y;
+    f = h2f2(r.v.w); w[6] = f.x; w[7] = f.y;
+  } else {
+    const float s = half_bits_to_float(r.s);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const uint32_t b0 = (q.x >> (8 * k)) & 0xffu, b1 = (q.y >> (8 * k)) & 0xffu;
+      const uint32_t b0 = (r.q.x >> (8 * k)) & 0xffu, b1 = (r.q.y >> (8 * k)) & 0xffu;
       w[k] = s * (float)((int)(b0 & 15u) - 8);
       w[4 + k] = s * (float)((int)(b1 & 15u) - 8);
       w[8 + k] = s * (float)((int)(b0 >> 4) - 8);
       w[12 + k] = s * (float)((int)(b1 >> 4) - 8);
     }
   }
+}
+
+// Load unit u of row `row` of a [rows, d] matrix of type T, decoded to floats.
+template <int T>
+__device__ __forceinline__ void load_w_unit(const void* __restrict__ data, const void* __restrict__ scales, int64_t row,
+                                            int d, int u, float (&w)[Unit<T>::E]) {
+  decode_w<T>(load_w_raw<T>(data, scales, row, d, u), w);
 }
 
 // Token values at the columns of unit u (layout of weight type WT) for token

@@ -9,6 +9,7 @@
 #include "pi_common.cuh"
 #include "pi_kernels_v1.cuh"
 #include "pi_launch.h"
+#include "pi_layout.h"
 
 namespace pi {
 
@@ -155,7 +156,10 @@ __global__ void __launch_bounds__(256) k_compact(const uint32_t* tile_mask,
 
 // ---------------------------------------------------------------------------
 // Sparse FFN step 1: activation of every listed neuron, one warp per neuron.
-// list = [0, n_hot) ++ idx[0, count); a[b, p] for list position p.
+// list = [0, n_hot) ++ idx[0, count); a[b, p] for list position p.  A lane
+// loads kActU units of the up (and gate) row before it decodes any of them.
+constexpr int kActU = 4;
+
 template <int WT, int HT, int ACT, int NB>
 __global__ void __launch_bounds__(256) k_ffn_act(const void* __restrict__ h, int B, int d, int ffn, int n_hot,
                                                  const int32_t* __restrict__ idx, const int32_t* __restrict__ count,
@@ -188,20 +192,34 @@ __global__ void __launch_bounds__(256) k_ffn_act(const void* __restrict__ h, int
       float g[NB], v[NB];
 #pragma unroll
       for (int i = 0; i < NB; ++i) { g[i] = 0.f; v[i] = 0.f; }
-      for (int un = lane; un < units; un += 32) {
-        float wu_[E];
-        load_w_unit<WT>(wu, wu_sc, j, d, un, wu_);
-        float wg_[E];
-        if constexpr (ACT == kReglu) load_w_unit<WT>(wg, wg_sc, j, d, un, wg_);
+      for (int u0 = lane; u0 < units; u0 += 32 * kActU) {
+        WRaw<WT> ru[kActU], rg[kActU];
 #pragma unroll
-        for (int i = 0; i < NB; ++i) {
-          if (i < nb) {
-            float x[E];
-            load_h_unit<WT, HT>(h, b0 + i, d, un, x);
+        for (int k = 0; k < kActU; ++k) {
+          const int un = u0 + 32 * k;
+          if (un < units) {
+            ru[k] = load_w_raw<WT>(wu, wu_sc, j, d, un);
+            if constexpr (ACT == kReglu) rg[k] = load_w_raw<WT>(wg, wg_sc, j, d, un);
+          }
+        }
 #pragma unroll
-            for (int e = 0; e < E; ++e) {
-              v[i] = fmaf(wu_[e], x[e], v[i]);
-              if constexpr (ACT == kReglu) g[i] = fmaf(wg_[e], x[e], g[i]);
+        for (int k = 0; k < kActU; ++k) {
+          const int un = u0 + 32 * k;
+          if (un < units) {
+            float wu_[E], wg_[E];
+            decode_w<WT>(ru[k], wu_);
+            if constexpr (ACT == kReglu) decode_w<WT>(rg[k], wg_);
+#pragma unroll
+            for (int i = 0; i < NB; ++i) {
+              if (i < nb) {
+                float x[E];
+                load_h_unit<WT, HT>(h, b0 + i, d, un, x);
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                  v[i] = fmaf(wu_[e], x[e], v[i]);
+                  if constexpr (ACT == kReglu) g[i] = fmaf(wg_[e], x[e], g[i]);
+                }
+              }
             }
           }
         }
@@ -224,24 +242,40 @@ __global__ void __launch_bounds__(256) k_ffn_act(const void* __restrict__ h, int
 }
 
 // ---------------------------------------------------------------------------
-// Sparse FFN step 2: down projection.  CTA c owns a contiguous, balanced range
-// of list positions and writes its fp32 partial y [B, d] (zeros for an empty
-// range).  Thread t owns the columns of units t, t + T, ... of the W_downT
-// rows (16 elements per thread per token group of NB tokens).
+// Sparse FFN step 2: down projection.  CTA (c, r) covers chunk c of d -- 32
+// lanes x 16 columns, a lane owning the same columns in every row -- for the
+// list positions of range r (contiguous and balanced over the ranges).  The
+// range's rows and activations are staged in shared memory; the 8 warps take
+// its positions in turn with kDnU rows in flight per lane, and their sums are
+// added in warp order through shared memory into the fp32 partial y[r]
+// [B, d] (zeros for an empty range).
+constexpr int kDnWarps = 8;
+constexpr int kDnU = 4;
+constexpr int kDnCap = 1024;  // positions staged at a time
+
 template <int WT, int NB>
-__global__ void k_ffn_down(int B, int d, int ffn, int n_hot, const int32_t* __restrict__ idx,
-                           const int32_t* __restrict__ count, const void* __restrict__ wd,
-                           const void* __restrict__ wd_sc, const float* __restrict__ a, int n_max,
-                           float* __restrict__ partial) {
+__global__ void __launch_bounds__(kDnWarps * 32) k_ffn_down(int B, int d, int ffn, int n_hot,
+                                                            const int32_t* __restrict__ idx,
+                                                            const int32_t* __restrict__ count,
+                                                            const void* __restrict__ wd, const void* __restrict__ wd_sc,
+                                                            const float* __restrict__ a, int n_max,
+                                                            float* __restrict__ partial) {
   constexpr int E = Unit<WT>::E;
-  constexpr int UPT = 16 / E;  // units per thread
+  constexpr int UPT = 16 / E;      // units per lane
+  constexpr int V = 16 * NB;       // sums per lane
+  extern __shared__ float dsm[];
+  int* srow = reinterpret_cast<int*>(dsm);  // [kDnCap] rows of the staged positions
+  float* sact = dsm + kDnCap;               // [NB][kDnCap] their activations
+  float* red = dsm;                         // [warps][V][32] after the stream (aliases the staging)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x, r = blockIdx.y, R = gridDim.y;
   const int n_cold = ffn - n_hot;
   int cnt = *count;
   cnt = cnt < 0 ? 0 : (cnt > n_cold ? n_cold : cnt);
   const int64_t n = n_hot + cnt;
-  const int64_t p0 = n * blockIdx.x / gridDim.x, p1 = n * (blockIdx.x + 1) / gridDim.x;
+  const int p0 = (int)(n * r / R), p1 = (int)(n * (r + 1) / R);
   const int units = d / E;
-  float* out = partial + (int64_t)blockIdx.x * B * d;
+  const int ub = c * 32 * UPT + lane;  // this lane's first unit
   for (int b0 = 0; b0 < B; b0 += NB) {
     const int nb = min(NB, B - b0);
     float acc[UPT][E][NB];
@@ -251,38 +285,68 @@ __global__ void k_ffn_down(int B, int d, int ffn, int n_hot, const int32_t* __re
       for (int e = 0; e < E; ++e)
 #pragma unroll
         for (int i = 0; i < NB; ++i) acc[q][e][i] = 0.f;
-    for (int64_t p = p0; p < p1; ++p) {
-      const int j = p < n_hot ? (int)p : idx[p - n_hot];
-      if (p >= n_hot && (j < n_hot || j >= ffn)) continue;  // flagged by k_ffn_act
-      float av[NB];
+    for (int s0 = p0; s0 < p1; s0 += kDnCap) {
+      const int len = min(kDnCap, p1 - s0);
+      __syncthreads();  // the previous segment (or reduction) is done with the buffer
+      for (int i = threadIdx.x; i < len; i += blockDim.x) {
+        const int p = s0 + i;
+        const int j = p < n_hot ? p : idx[p - n_hot];
+        const bool ok = p < n_hot || (j >= n_hot && j < ffn);  // a bad entry is flagged by k_ffn_act
+        srow[i] = ok ? j : 0;
 #pragma unroll
-      for (int i = 0; i < NB; ++i) av[i] = (i < nb) ? a[(int64_t)(b0 + i) * n_max + p] : 0.f;
-#pragma unroll
-      for (int q = 0; q < UPT; ++q) {
-        const int un = threadIdx.x + q * blockDim.x;
-        if (un < units) {
-          float w[E];
-          load_w_unit<WT>(wd, wd_sc, j, d, un, w);
-#pragma unroll
-          for (int e = 0; e < E; ++e)
-#pragma unroll
-            for (int i = 0; i < NB; ++i) acc[q][e][i] = fmaf(av[i], w[e], acc[q][e][i]);
-        }
+        for (int q = 0; q < NB; ++q) sact[q * kDnCap + i] = (ok && q < nb) ? a[(int64_t)(b0 + q) * n_max + p] : 0.f;
       }
-    }
+      __syncthreads();
+      for (int m0 = warp; m0 < len; m0 += kDnWarps * kDnU) {
+        WRaw<WT> raw[kDnU][UPT] = {};
 #pragma unroll
-    for (int q = 0; q < UPT; ++q) {
-      const int un = threadIdx.x + q * blockDim.x;
-      if (un < units) {
+        for (int k = 0; k < kDnU; ++k) {
+          const int m = m0 + kDnWarps * k;
+          if (m < len) {
+            const int j = srow[m];
 #pragma unroll
-        for (int i = 0; i < NB; ++i) {
-          if (i < nb) {
-            float* o = out + (int64_t)(b0 + i) * d;
+            for (int q = 0; q < UPT; ++q)
+              if (ub + 32 * q < units) raw[k][q] = load_w_raw<WT>(wd, wd_sc, j, d, ub + 32 * q);
+          }
+        }
 #pragma unroll
-            for (int e = 0; e < E; ++e) o[unit_col<WT>(un, e)] = acc[q][e][i];
+        for (int k = 0; k < kDnU; ++k) {
+          const int m = m0 + kDnWarps * k;
+          if (m < len) {
+            float av[NB];
+#pragma unroll
+            for (int i = 0; i < NB; ++i) av[i] = sact[i * kDnCap + m];
+#pragma unroll
+            for (int q = 0; q < UPT; ++q) {
+              if (ub + 32 * q < units) {
+                float w[E];
+                decode_w<WT>(raw[k][q], w);
+#pragma unroll
+                for (int e = 0; e < E; ++e)
+#pragma unroll
+                  for (int i = 0; i < NB; ++i) acc[q][e][i] = fmaf(av[i], w[e], acc[q][e][i]);
+              }
+            }
           }
         }
       }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < UPT; ++q)
+#pragma unroll
+      for (int e = 0; e < E; ++e)
+#pragma unroll
+        for (int i = 0; i < NB; ++i) red[((size_t)warp * V + (q * E + e) * NB + i) * 32 + lane] = acc[q][e][i];
+    __syncthreads();
+    for (int x = threadIdx.x; x < V * 32; x += blockDim.x) {
+      const int ln = x & 31, y = x >> 5;
+      const int i = y % NB, q = (y / NB) / E, e = (y / NB) % E;
+      float sum = 0.f;
+#pragma unroll
+      for (int w = 0; w < kDnWarps; ++w) sum += red[((size_t)w * V + y) * 32 + ln];
+      const int un = c * 32 * UPT + ln + 32 * q;
+      if (un < units && i < nb) partial[((int64_t)r * B + b0 + i) * d + unit_col<WT>(un, e)] = sum;
     }
   }
 }
@@ -460,23 +524,34 @@ cudaError_t launch_ffn_act(int wtype, int htype, int act, const void* h, int B, 
   return cudaGetLastError();
 }
 
-int down_threads(int wtype, int d) {
-  const int e = wtype == kF32 ? 4 : (wtype == kF16 ? 8 : 16);
-  const int units = d / e;
-  const int upt = 16 / e;
-  int t = (units + upt - 1) / upt;
-  t = (t + 31) / 32 * 32;
-  return t < 32 ? 32 : t;
+int down_ranges(int d, int sms) {
+  const int chunks = (d + 511) / 512;
+  const int R = (3 * sms) / chunks;
+  return R < 1 ? 1 : (R > kGMax ? kGMax : R);
 }
 
 cudaError_t launch_ffn_down(int wtype, int B, int d, int ffn, int n_hot, const int32_t* idx, const int32_t* count,
                             const void* wd, const void* wd_sc, const float* a, int n_max, float* partial, int G,
                             cudaStream_t st) {
-  const int T = down_threads(wtype, d);
-  if (T > 1024) return cudaErrorInvalidValue;
-  if (wtype == kF32) k_ffn_down<kF32, kNB><<<G, T, 0, st>>>(B, d, ffn, n_hot, idx, count, wd, wd_sc, a, n_max, partial);
-  else if (wtype == kF16) k_ffn_down<kF16, kNB><<<G, T, 0, st>>>(B, d, ffn, n_hot, idx, count, wd, wd_sc, a, n_max, partial);
-  else k_ffn_down<kQ4_0, kNB><<<G, T, 0, st>>>(B, d, ffn, n_hot, idx, count, wd, wd_sc, a, n_max, partial);
+  if (G < 1 || G > kGMax) return cudaErrorInvalidValue;
+  const dim3 grid((d + 511) / 512, G);
+  const size_t smem = (size_t)kDnWarps * 16 * kNB * 32 * sizeof(float);
+  static_assert((size_t)kDnWarps * 16 * kNB * 32 >= (size_t)(1 + kNB) * kDnCap, "the staging fits the reduction buffer");
+  cudaError_t e;
+  if (wtype == kF32) {
+    if ((e = cudaFuncSetAttribute(k_ffn_down<kF32, kNB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+      return e;
+    k_ffn_down<kF32, kNB><<<grid, kDnWarps * 32, smem, st>>>(B, d, ffn, n_hot, idx, count, wd, wd_sc, a, n_max, partial);
+  } else if (wtype == kF16) {
+    if ((e = cudaFuncSetAttribute(k_ffn_down<kF16, kNB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+      return e;
+    k_ffn_down<kF16, kNB><<<grid, kDnWarps * 32, smem, st>>>(B, d, ffn, n_hot, idx, count, wd, wd_sc, a, n_max, partial);
+  } else {
+    if ((e = cudaFuncSetAttribute(k_ffn_down<kQ4_0, kNB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+      return e;
+    k_ffn_down<kQ4_0, kNB><<<grid, kDnWarps * 32, smem, st>>>(B, d, ffn, n_hot, idx, count, wd, wd_sc, a, n_max,
+                                                              partial);
+  }
   return cudaGetLastError();
 }
 

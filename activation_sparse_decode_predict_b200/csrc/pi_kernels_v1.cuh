@@ -16,7 +16,8 @@ cudaError_t launch_ffn_act(int wtype, int htype, int act, const void* h, int B, 
                            const int32_t* idx, const int32_t* count, const void* wg, const void* wg_sc,
                            const void* wu, const void* wu_sc, const float* b1, float* a, int n_max, int* status,
                            int sms, cudaStream_t st);
-int down_threads(int wtype, int d);
+// position ranges (split-K partials, at most kGMax) of the down projection
+int down_ranges(int d, int sms);
 cudaError_t launch_ffn_down(int wtype, int B, int d, int ffn, int n_hot, const int32_t* idx, const int32_t* count,
                             const void* wd, const void* wd_sc, const float* a, int n_max, float* partial, int G,
                             cudaStream_t st);
