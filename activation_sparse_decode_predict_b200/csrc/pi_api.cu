@@ -168,11 +168,12 @@ pi_status ffn_impl(const pi_ffn_desc* d, int32_t B, const void* h, const int32_t
     return PI_OK;
   }
   if (pi::batch_supported(d->wtype, ht, d->d, B)) {
-    // token blocks of 3..16 with fp16 weights: tensor-core gate/up and down
-    const int NR = pi::batch_ranges(d->d, sms);
-    PI_CUDA(pi::launch_batch_ffn(d->act, h, B, d->d, d->ffn, d->n_hot, idx, count, Wg.data, Wu.data, Wd.data, b1,
-                                 reinterpret_cast<float*>(ws + L.pre), partial, NR, reinterpret_cast<pi::Ctrl*>(ws),
-                                 sms, st),
+    // token blocks of 3..16: tensor-core gate/up, down on the tensor cores
+    // (fp16 weights) or on the CUDA cores (Q4_0)
+    const int NR = d->wtype == PI_Q4_0 ? pi::down_ranges(d->d, sms) : pi::batch_ranges(d->d, sms);
+    PI_CUDA(pi::launch_batch_ffn(d->act, d->wtype, h, B, d->d, d->ffn, d->n_hot, idx, count, Wg.data, Wg.scales,
+                                 Wu.data, Wu.scales, Wd.data, Wd.scales, b1, reinterpret_cast<float*>(ws + L.pre),
+                                 partial, NR, reinterpret_cast<pi::Ctrl*>(ws), sms, st),
             "tensor-core FFN launch");
     PI_CUDA(pi::launch_ffn_reduce(partial, NR, B, d->d, b2, y, st), "split-K reduce launch");
     return PI_OK;

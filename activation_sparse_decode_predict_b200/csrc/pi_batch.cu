@@ -27,6 +27,7 @@
 
 #include "pi_batch.cuh"
 #include "pi_common.cuh"
+#include "pi_kernels_v1.cuh"
 #include "pi_launch.h"
 #include "pi_mma.cuh"
 #include "pi_sync.cuh"
@@ -79,10 +80,16 @@ __device__ __forceinline__ int clamp_count(const int32_t* count, int C, Ctrl* ct
 // shared-memory layouts (host and device agree through these functions)
 
 struct UpLayout {
-  int PC, KC, HS, RS, ISZ, off_map, off_h, off_red, off_ring, nslot, bytes;
+  int PC, KC, HS, RS, SRS, SOFF, ISZ, off_map, off_h, off_red, off_ring, nslot, bytes;
 };
 
-__host__ __device__ inline UpLayout up_layout(int B8, int d, int S) {
+// bytes of one 16-row slot of KC columns: fp16 rows, or Q4_0 rows as the
+// KC / 2 code bytes then (SOFF on) the KC / 16 scale bytes of every row
+__host__ __device__ inline int up_slot_bytes(int wt, int kc) {
+  return wt == kQ4_0 ? 16 * (kc / 2 + 16) + 16 * (kc / 16 + 16) : 16 * (kc * 2 + 16);
+}
+
+__host__ __device__ inline UpLayout up_layout(int B8, int d, int S, int wt = kF16) {
   UpLayout L;
   L.PC = d / S;
   L.HS = L.PC * 2 + 16;   // token row stride (bytes): +16 keeps ldmatrix rows on distinct banks
@@ -92,19 +99,29 @@ __host__ __device__ inline UpLayout up_layout(int B8, int d, int S) {
   L.off_ring = L.off_red + 2 * kBW * 16 * B8 * 4;
   const int room = kBSmem - L.off_ring;
   // columns per streamed chunk: the largest PC / m (a multiple of 16, at
-  // most 2048) whose 16-row slot leaves room for two slots -- row pieces of
-  // 4 KB in 64 KB slots stream at full bandwidth, 2 KB pieces in 32 KB slots
-  // at about half of it, even with more slots in flight
-  L.KC = 16;
-  for (int m = 1; m <= L.PC / 16; ++m) {
-    if (L.PC % m || (L.PC / m) % 16 || L.PC / m > 2048) continue;
-    if (2 * 16 * ((L.PC / m) * 2 + 16) <= room) {
+  // most 2048; Q4_0: of 256, whole scale pieces, at most 4096) whose 16-row
+  // slot leaves room for two slots -- fp16 row pieces of 4 KB in 64 KB slots
+  // stream at full bandwidth, 2 KB pieces in 32 KB slots at about half of it,
+  // even with more slots in flight
+  const int step = wt == kQ4_0 ? 256 : 16, cap = wt == kQ4_0 ? 4096 : 2048;
+  L.KC = step;
+  for (int m = 1; m <= L.PC / step; ++m) {
+    if (L.PC % m || (L.PC / m) % step || L.PC / m > cap) continue;
+    if (2 * up_slot_bytes(wt, L.PC / m) <= room) {
       L.KC = L.PC / m;
       break;
     }
   }
-  L.RS = L.KC * 2 + 16;   // weight row stride in a ring slot
-  L.ISZ = 16 * L.RS;      // one slot: 16 rows x KC columns
+  if (wt == kQ4_0) {
+    L.RS = L.KC / 2 + 16;   // code row stride: rows start 4 banks apart
+    L.SRS = L.KC / 16 + 16;
+    L.SOFF = 16 * L.RS;
+  } else {
+    L.RS = L.KC * 2 + 16;   // weight row stride in a ring slot
+    L.SRS = 0;
+    L.SOFF = 0;
+  }
+  L.ISZ = up_slot_bytes(wt, L.KC);
   L.nslot = room / L.ISZ;
   if (L.nslot > kBMaxSlots) L.nslot = kBMaxSlots;
   L.bytes = L.off_ring + L.nslot * L.ISZ;
@@ -147,8 +164,10 @@ __host__ __device__ inline DownLayout down_layout(int d) {
 // mode: rows 0..nrows-1 of one matrix, slot 0.
 struct RowDotParams {
   const __half* x;   // [ntok, K] token rows
-  const __half* w0;  // gate (gated list mode) or the only matrix
-  const __half* w1;  // up (gated list mode)
+  const void* w0;    // gate (gated list mode) or the only matrix: fp16 rows, or Q4_0 codes
+  const void* w1;    // up (gated list mode)
+  const void* w0_sc;  // Q4_0 scales of w0 / w1 (list mode only)
+  const void* w1_sc;
   const int32_t* idx;
   const int32_t* count;
   float* out;  // [S][R][W][ntok]
@@ -166,10 +185,30 @@ struct RowDotParams {
   int upre_parts;
 };
 
-template <int NT>
+// Q4_0 rows (list mode): a lane's 4 code bytes 4t..4t+3 of a row's 32-column
+// block, as the exact fp16 pairs (q - 8) of the block's k-step 0 (low
+// nibbles: columns 4t, 4t+1 and 4t+2, 4t+3) and k-step 1 (high nibbles:
+// the same + 16).  The token rows are staged in that column order, so the
+// products pair up; each block's scale multiplies its two steps' sums in fp32.
+__device__ __forceinline__ void q4_frag(uint32_t w, uint32_t& lo01, uint32_t& lo23, uint32_t& hi01, uint32_t& hi23) {
+  const uint32_t p01 = __byte_perm(w, 0u, 0x4140), p23 = __byte_perm(w, 0u, 0x4342);
+  const __half2 k1032 = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));  // 1024 + 8
+  const __half2 k16th = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));  // 1 / 16
+  const __half2 km72 = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));   // -72
+  auto h2 = [](uint32_t v) { return *reinterpret_cast<__half2*>(&v); };
+  auto u32 = [](__half2 v) { return *reinterpret_cast<uint32_t*>(&v); };
+  // (v | 0x6400) read as fp16 is 1024 + v for v < 1024: nibble q -> 1024 + q, high nibble -> 1024 + 16 q
+  lo01 = u32(__hsub2(h2((p01 & 0x000F000Fu) | 0x64006400u), k1032));
+  lo23 = u32(__hsub2(h2((p23 & 0x000F000Fu) | 0x64006400u), k1032));
+  hi01 = u32(__hfma2(h2((p01 & 0x00F000F0u) | 0x64006400u), k16th, km72));
+  hi23 = u32(__hfma2(h2((p23 & 0x00F000F0u) | 0x64006400u), k16th, km72));
+}
+
+template <int NT, int WT>
 __global__ void __launch_bounds__(kBT + 32, 1) k_rowdot(const __grid_constant__ RowDotParams p) {
+  static_assert(WT == kF16 || WT == kQ4_0, "fp16 or Q4_0 rows");
   extern __shared__ __align__(128) uint8_t sm[];
-  const UpLayout Lay = up_layout(NT * 8, p.K, p.S);
+  const UpLayout Lay = up_layout(NT * 8, p.K, p.S, WT);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm);
   uint64_t* empty = full + kBMaxSlots;
   int* rmap = reinterpret_cast<int*>(sm + Lay.off_map);
@@ -217,16 +256,37 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_rowdot(const __grid_constant__ 
       if (it >= nslot) ok = mbar_wait(&empty[q], ((it / nslot) - 1) & 1, ctrl);
       if (!__all_sync(0xffffffffu, ok)) return;
       const int tile = it / nch, ch = it % nch;
-      if (lane == 0) mbar_arrive_expect_tx(&full[q], 16u * Lay.KC * 2u);
-      __syncwarp();
-      if (lane < 16) {
-        int pos = n0 + tile * npt + (two ? lane / 2 : lane);
+      if constexpr (WT == kQ4_0) {
+        // lanes 0-15: the rows' code pieces; lanes 16-31: their scale pieces
+        if (lane == 0) mbar_arrive_expect_tx(&full[q], 16u * (uint32_t)(Lay.KC / 2 + Lay.KC / 16));
+        __syncwarp();
+        const int r16 = lane & 15;
+        int pos = n0 + tile * npt + (two ? r16 / 2 : r16);
         if (pos >= n1) pos = n1 - 1;  // tail rows repeat the last one; their dots are dropped
-        int j = p.list ? row_at(rmap, pos, n0, p.n_hot, p.ffn, p.idx, ctrl) : pos;
+        int j = row_at(rmap, pos, n0, p.n_hot, p.ffn, p.idx, ctrl);
         if (j < 0) j = 0;
-        const __half* mat = (two && (lane & 1)) ? p.w1 : p.w0;
-        bulk_g2s(ring + q * Lay.ISZ + lane * Lay.RS, mat + (int64_t)j * p.K + col0 + ch * Lay.KC, Lay.KC * 2u,
-                 &full[q]);
+        const bool up = two && (r16 & 1);
+        const int64_t c0 = col0 + (int64_t)ch * Lay.KC;
+        if (lane < 16)
+          bulk_g2s(ring + q * Lay.ISZ + r16 * Lay.RS,
+                   static_cast<const uint8_t*>(up ? p.w1 : p.w0) + (int64_t)j * (p.K / 2) + c0 / 2, Lay.KC / 2u,
+                   &full[q]);
+        else
+          bulk_g2s(ring + q * Lay.ISZ + Lay.SOFF + r16 * Lay.SRS,
+                   static_cast<const uint8_t*>(up ? p.w1_sc : p.w0_sc) + (int64_t)j * (p.K / 16) + c0 / 16,
+                   Lay.KC / 16u, &full[q]);
+      } else {
+        if (lane == 0) mbar_arrive_expect_tx(&full[q], 16u * Lay.KC * 2u);
+        __syncwarp();
+        if (lane < 16) {
+          int pos = n0 + tile * npt + (two ? lane / 2 : lane);
+          if (pos >= n1) pos = n1 - 1;  // tail rows repeat the last one; their dots are dropped
+          int j = p.list ? row_at(rmap, pos, n0, p.n_hot, p.ffn, p.idx, ctrl) : pos;
+          if (j < 0) j = 0;
+          const __half* mat = static_cast<const __half*>((two && (lane & 1)) ? p.w1 : p.w0);
+          bulk_g2s(ring + q * Lay.ISZ + lane * Lay.RS, mat + (int64_t)j * p.K + col0 + ch * Lay.KC, Lay.KC * 2u,
+                   &full[q]);
+        }
       }
       __syncwarp();
     }
@@ -288,7 +348,18 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_rowdot(const __grid_constant__ 
       const int b = i / units, u = i % units;
       uint4 v = make_uint4(0u, 0u, 0u, 0u);
       if (b < p.ntok) v = __ldcg(reinterpret_cast<const uint4*>(p.x + (int64_t)b * p.K + col0) + u);
-      *reinterpret_cast<uint4*>(hs + b * Lay.HS + 16 * u) = v;
+      if constexpr (WT == kQ4_0) {
+        // column pairs in the order of q4_frag: within each 16 columns, pair w
+        // goes to pair 4 (w % 2) + w / 2
+        uint32_t* dst = reinterpret_cast<uint32_t*>(hs + b * Lay.HS + 32 * (u >> 1));
+        const int h = 2 * (u & 1);
+        dst[h] = v.x;
+        dst[4 + h] = v.y;
+        dst[h + 1] = v.z;
+        dst[5 + h] = v.w;
+      } else {
+        *reinterpret_cast<uint4*>(hs + b * Lay.HS + 16 * u) = v;
+      }
     }
   }
   named_sync(1, kBT);
@@ -305,7 +376,36 @@ __global__ void __launch_bounds__(kBT + 32, 1) k_rowdot(const __grid_constant__ 
     const int q = it % nslot;
     const int tile = it / nch, ch = it % nch;
     to |= !mbar_wait(&full[q], (it / nslot) & 1, ctrl);
-    if (!to) {
+    if (!to && WT == kQ4_0) {
+      // this warp's 32-column blocks of the slot (KC / 32 is a multiple of 8)
+      const int nblk = Lay.KC / 32, kb0 = cw * (nblk / kBW), kb1 = kb0 + nblk / kBW;
+      const int g = lane >> 2, t4 = lane & 3;
+      const uint8_t* slot = ring + q * Lay.ISZ;
+      const uint8_t* cg = slot + g * Lay.RS + 4 * t4;
+      const uint8_t* cg8 = cg + 8 * Lay.RS;
+      const __half* sg = reinterpret_cast<const __half*>(slot + Lay.SOFF + g * Lay.SRS);
+      const __half* sg8 = reinterpret_cast<const __half*>(slot + Lay.SOFF + (g + 8) * Lay.SRS);
+      const uint32_t b_base = b_lane + (uint32_t)(ch * Lay.KC * 2);
+      for (int kb = kb0; kb < kb1; ++kb) {
+        uint32_t a0, a2, e0, e2, a1, a3, e1, e3;  // a: k-step 2 kb (low nibbles), e: 2 kb + 1 (high)
+        q4_frag(*reinterpret_cast<const uint32_t*>(cg + 16 * kb), a0, a2, e0, e2);
+        q4_frag(*reinterpret_cast<const uint32_t*>(cg8 + 16 * kb), a1, a3, e1, e3);
+        const float s0 = __half2float(sg[kb]), s8 = __half2float(sg8[kb]);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          uint32_t b0, b1, f0, f1;
+          ldsm_x2(b_base + (uint32_t)(nt * 8 * Lay.HS) + 64u * kb, b0, b1);
+          ldsm_x2(b_base + (uint32_t)(nt * 8 * Lay.HS) + 64u * kb + 32u, f0, f1);
+          float d4[4] = {0.f, 0.f, 0.f, 0.f};
+          mma_16816(d4, a0, a1, a2, a3, b0, b1);
+          mma_16816(d4, e0, e1, e2, e3, f0, f1);
+          acc[nt][0] = fmaf(s0, d4[0], acc[nt][0]);
+          acc[nt][1] = fmaf(s0, d4[1], acc[nt][1]);
+          acc[nt][2] = fmaf(s8, d4[2], acc[nt][2]);
+          acc[nt][3] = fmaf(s8, d4[3], acc[nt][3]);
+        }
+      }
+    } else if (!to) {
       const uint32_t a_base = smem_u32(ring + q * Lay.ISZ) + a_lane;
       const uint32_t b_base = b_lane + (uint32_t)(ch * Lay.KC * 2);
       for (int ks = ks0; ks < ks1; ++ks) {
@@ -584,36 +684,43 @@ int row_parts(int ntok, int K) {
   return S;
 }
 
-template <int NT>
+template <int NT, int WT>
 cudaError_t launch_rowdot_t(const RowDotParams& P, int G, cudaStream_t st) {
-  const UpLayout UL = up_layout(NT * 8, P.K, P.S);
-  cudaError_t e = cudaFuncSetAttribute(k_rowdot<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, UL.bytes);
+  const UpLayout UL = up_layout(NT * 8, P.K, P.S, WT);
+  cudaError_t e = cudaFuncSetAttribute(k_rowdot<NT, WT>, cudaFuncAttributeMaxDynamicSharedMemorySize, UL.bytes);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(k_rowdot<NT>, dim3(G), dim3(kBT + 32), UL.bytes, st, P);
+  e = launch_pdl(k_rowdot<NT, WT>, dim3(G), dim3(kBT + 32), UL.bytes, st, P);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-cudaError_t launch_rowdot(const RowDotParams& P, int sms, cudaStream_t st) {
+// wt: kF16 rows, or Q4_0 rows (list mode only)
+cudaError_t launch_rowdot(const RowDotParams& P, int wt, int sms, cudaStream_t st) {
   const int G = (sms / P.S) * P.S;
   const int NT = rowdot_nt(P.ntok);
-  if (NT == 1) return launch_rowdot_t<1>(P, G, st);
-  if (NT == 2) return launch_rowdot_t<2>(P, G, st);
-  return launch_rowdot_t<4>(P, G, st);
+  if (wt == kQ4_0) {
+    if (!P.list) return cudaErrorInvalidValue;
+    if (NT == 1) return launch_rowdot_t<1, kQ4_0>(P, G, st);
+    if (NT == 2) return launch_rowdot_t<2, kQ4_0>(P, G, st);
+    return launch_rowdot_t<4, kQ4_0>(P, G, st);
+  }
+  if (NT == 1) return launch_rowdot_t<1, kF16>(P, G, st);
+  if (NT == 2) return launch_rowdot_t<2, kF16>(P, G, st);
+  return launch_rowdot_t<4, kF16>(P, G, st);
 }
 
-bool rowdot_fits(int ntok, int K) {
+bool rowdot_fits(int ntok, int K, int wt = kF16) {
   const int S = row_parts(ntok, K);
-  if (S > 4 || K % (128 * S) != 0) return false;
-  return up_layout(8 * rowdot_nt(ntok), K, S).nslot >= 2;  // the token tile the kernel stages
+  if (S > 4 || K % ((wt == kQ4_0 ? 256 : 128) * S) != 0) return false;
+  return up_layout(8 * rowdot_nt(ntok), K, S, wt).nslot >= 2;  // the token tile the kernel stages
 }
 
 }  // namespace
 
-bool batch_supported(int wtype, int ptype, int d, int B) {
-  if (wtype != kF16 || ptype != kF16) return false;
-  if (B < kBatchMin || B > 16) return false;
-  if (d % 256 != 0) return false;
-  return rowdot_fits(B, d) && down_layout(d).nslot >= 2;
+bool batch_supported(int wtype, int htype, int d, int B) {
+  if (htype != kF16 || B < kBatchMin || B > 16 || d % 256 != 0) return false;
+  if (wtype == kF16) return rowdot_fits(B, d) && down_layout(d).nslot >= 2;
+  if (wtype == kQ4_0) return rowdot_fits(B, d, kQ4_0);
+  return false;
 }
 
 bool batch_pred_supported(int ptype, int d, int r, int B) {
@@ -648,7 +755,7 @@ cudaError_t launch_batch_predict(const void* h, int B, int d, int r, int C, int 
   U.R = r;
   U.nrows = r;
   U.W = 1;
-  cudaError_t e = launch_rowdot(U, sms, st);
+  cudaError_t e = launch_rowdot(U, kF16, sms, st);
   if (e != cudaSuccess || C == 0) return e;
   RowDotParams S{};
   S.upre = upre;  // u = ReLU(sum of the P1 parts), split into hi + lo rows while staging
@@ -662,7 +769,7 @@ cudaError_t launch_batch_predict(const void* h, int B, int d, int r, int C, int 
   S.R = C;
   S.nrows = C;
   S.W = 1;
-  e = launch_rowdot(S, sms, st);
+  e = launch_rowdot(S, kF16, sms, st);
   if (e != cudaSuccess) return e;
   e = launch_pdl(k_bthresh, dim3((C + 255) / 256), dim3(256), 0, st, static_cast<const float*>(sc), S.S, C, B, bp, thr,
                  tile_mask, tile_count);
@@ -671,14 +778,17 @@ cudaError_t launch_batch_predict(const void* h, int B, int d, int r, int C, int 
   return cudaGetLastError();
 }
 
-cudaError_t launch_batch_ffn(int act, const void* h, int B, int d, int ffn, int n_hot, const int32_t* idx,
-                             const int32_t* count, const void* wg, const void* wu, const void* wd, const float* b1,
-                             float* pre, float* partial, int NR, Ctrl* ctrl, int sms, cudaStream_t st) {
+cudaError_t launch_batch_ffn(int act, int wtype, const void* h, int B, int d, int ffn, int n_hot, const int32_t* idx,
+                             const int32_t* count, const void* wg, const void* wg_sc, const void* wu,
+                             const void* wu_sc, const void* wd, const void* wd_sc, const float* b1, float* pre,
+                             float* partial, int NR, Ctrl* ctrl, int sms, cudaStream_t st) {
   const int gated = act == kReglu;
   RowDotParams U{};
   U.x = static_cast<const __half*>(h);
-  U.w0 = static_cast<const __half*>(gated ? wg : wu);
-  U.w1 = static_cast<const __half*>(wu);
+  U.w0 = gated ? wg : wu;
+  U.w1 = wu;
+  U.w0_sc = gated ? wg_sc : wu_sc;
+  U.w1_sc = wu_sc;
   U.idx = idx;
   U.count = count;
   U.out = pre;
@@ -692,8 +802,11 @@ cudaError_t launch_batch_ffn(int act, const void* h, int B, int d, int ffn, int 
   U.n_hot = n_hot;
   U.ffn = ffn;
   U.W = 2;
-  cudaError_t e = launch_rowdot(U, sms, st);
+  cudaError_t e = launch_rowdot(U, wtype, sms, st);
   if (e != cudaSuccess) return e;
+  if (wtype == kQ4_0)  // down on the CUDA cores, activations from the dots of every part
+    return launch_ffn_down(kQ4_0, B, d, ffn, n_hot, idx, count, wd, wd_sc, nullptr, 0, partial, NR, st, pre, U.S, U.R,
+                           b1, act);
 
   const int NT = B > 8 ? 2 : 1;
   BDownParams D;

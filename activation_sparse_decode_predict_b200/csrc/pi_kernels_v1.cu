@@ -248,7 +248,9 @@ __global__ void __launch_bounds__(256) k_ffn_act(const void* __restrict__ h, int
 // range's rows and activations are staged in shared memory; the 8 warps take
 // its positions in turn with kDnU rows in flight per lane, and their sums are
 // added in warp order through shared memory into the fp32 partial y[r]
-// [B, d] (zeros for an empty range).
+// [B, d] (zeros for an empty range).  With `pre` the activations are made
+// while staging, from the gate/up dots of the token-block row-dot kernel
+// (pre [parts][pre_R][2][B], the parts added in order) and b1.
 constexpr int kDnWarps = 8;
 constexpr int kDnU = 4;
 constexpr int kDnCap = 1024;  // positions staged at a time
@@ -259,7 +261,9 @@ __global__ void __launch_bounds__(kDnWarps * 32) k_ffn_down(int B, int d, int ff
                                                             const int32_t* __restrict__ count,
                                                             const void* __restrict__ wd, const void* __restrict__ wd_sc,
                                                             const float* __restrict__ a, int n_max,
-                                                            float* __restrict__ partial) {
+                                                            float* __restrict__ partial, const float* __restrict__ pre,
+                                                            int pre_S, int pre_R, const float* __restrict__ b1,
+                                                            int act) {
   constexpr int E = Unit<WT>::E;
   constexpr int UPT = 16 / E;      // units per lane
   constexpr int V = 16 * NB;       // sums per lane
@@ -293,8 +297,25 @@ __global__ void __launch_bounds__(kDnWarps * 32) k_ffn_down(int B, int d, int ff
         const int j = p < n_hot ? p : idx[p - n_hot];
         const bool ok = p < n_hot || (j >= n_hot && j < ffn);  // a bad entry is flagged by k_ffn_act
         srow[i] = ok ? j : 0;
+        if (pre) {
+          const float bias = (ok && b1) ? b1[j] : 0.f;
 #pragma unroll
-        for (int q = 0; q < NB; ++q) sact[q * kDnCap + i] = (ok && q < nb) ? a[(int64_t)(b0 + q) * n_max + p] : 0.f;
+          for (int q = 0; q < NB; ++q) {
+            float g = 0.f, v = 0.f;
+            if (ok && q < nb) {
+              for (int sp = 0; sp < pre_S; ++sp) {
+                const float* pp = pre + ((int64_t)sp * pre_R + p) * 2 * B + b0 + q;
+                g += pp[0];
+                v += pp[B];
+              }
+            }
+            sact[q * kDnCap + i] =
+                !(ok && q < nb) ? 0.f : (act == kReglu ? act_eval(kReglu, g + bias, v) : act_eval(act, v + bias, 0.f));
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < NB; ++q) sact[q * kDnCap + i] = (ok && q < nb) ? a[(int64_t)(b0 + q) * n_max + p] : 0.f;
+        }
       }
       __syncthreads();
       for (int m0 = warp; m0 < len; m0 += kDnWarps * kDnU) {
@@ -532,7 +553,7 @@ int down_ranges(int d, int sms) {
 
 cudaError_t launch_ffn_down(int wtype, int B, int d, int ffn, int n_hot, const int32_t* idx, const int32_t* count,
                             const void* wd, const void* wd_sc, const float* a, int n_max, float* partial, int G,
-                            cudaStream_t st) {
+                            cudaStream_t st, const float* pre, int pre_S, int pre_R, const float* b1, int act) {
   if (G < 1 || G > kGMax) return cudaErrorInvalidValue;
   const dim3 grid((d + 511) / 512, G);
   const size_t smem = (size_t)kDnWarps * 16 * kNB * 32 * sizeof(float);
@@ -541,16 +562,16 @@ cudaError_t launch_ffn_down(int wtype, int B, int d, int ffn, int n_hot, const i
   if (wtype == kF32) {
     if ((e = cudaFuncSetAttribute(k_ffn_down<kF32, kNB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
       return e;
-    k_ffn_down<kF32, kNB><<<grid, kDnWarps * 32, smem, st>>>(B, d, ffn, n_hot, idx, count, wd, wd_sc, a, n_max, partial);
+    k_ffn_down<kF32, kNB><<<grid, kDnWarps * 32, smem, st>>>(B, d, ffn, n_hot, idx, count, wd, wd_sc, a, n_max, partial, pre, pre_S, pre_R, b1, act);
   } else if (wtype == kF16) {
     if ((e = cudaFuncSetAttribute(k_ffn_down<kF16, kNB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
       return e;
-    k_ffn_down<kF16, kNB><<<grid, kDnWarps * 32, smem, st>>>(B, d, ffn, n_hot, idx, count, wd, wd_sc, a, n_max, partial);
+    k_ffn_down<kF16, kNB><<<grid, kDnWarps * 32, smem, st>>>(B, d, ffn, n_hot, idx, count, wd, wd_sc, a, n_max, partial, pre, pre_S, pre_R, b1, act);
   } else {
     if ((e = cudaFuncSetAttribute(k_ffn_down<kQ4_0, kNB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
       return e;
     k_ffn_down<kQ4_0, kNB><<<grid, kDnWarps * 32, smem, st>>>(B, d, ffn, n_hot, idx, count, wd, wd_sc, a, n_max,
-                                                              partial);
+                                                              partial, pre, pre_S, pre_R, b1, act);
   }
   return cudaGetLastError();
 }

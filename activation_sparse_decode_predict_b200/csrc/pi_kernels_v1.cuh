@@ -18,9 +18,13 @@ cudaError_t launch_ffn_act(int wtype, int htype, int act, const void* h, int B, 
                            int sms, cudaStream_t st);
 // position ranges (split-K partials, at most kGMax) of the down projection
 int down_ranges(int d, int sms);
+// down projection of the listed rows into G split-K partials; the activations
+// come from a [B][n_max], or with `pre` from the token-block gate/up dots
+// (pre [pre_S][pre_R][2][B]) and b1 with activation kind `act`
 cudaError_t launch_ffn_down(int wtype, int B, int d, int ffn, int n_hot, const int32_t* idx, const int32_t* count,
                             const void* wd, const void* wd_sc, const float* a, int n_max, float* partial, int G,
-                            cudaStream_t st);
+                            cudaStream_t st, const float* pre = nullptr, int pre_S = 0, int pre_R = 0,
+                            const float* b1 = nullptr, int act = 0);
 cudaError_t launch_ffn_reduce(const float* partial, int G, int B, int d, const float* b2, float* y,
                               cudaStream_t st);
 cudaError_t launch_rmsnorm(int htype, const void* h, const float* y, int B, int d, float eps, void* h_out,

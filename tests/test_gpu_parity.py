@@ -31,6 +31,10 @@ SHAPES = [
     # tensor-core predictor of a token block (rank % 128 == 0), P2 split in parts
     ("relu-f16-b16-bigrank", 2048, 1500, 0.10, 2048, "relu", "f16", "f16", 16),
     ("reglu-f16-b4-pred", 512, 1200, 0.10, 128, "reglu", "f16", "f16", 4),
+    # Q4_0 token blocks: gate/up rows decoded onto the tensor cores, d in parts, ragged lists
+    ("reglu-q4-b8", 512, 1300, 0.10, 64, "reglu", "q4_0", "f16", 8),
+    ("relu2-q4-b16-parts", 4096, 900, 0.05, 32, "relu2", "q4_0", "f16", 16),
+    ("reglu-q4-b3-ragged", 768, 999, 0.02, 48, "reglu", "q4_0", "f16", 3),
 ]
 
 
@@ -292,8 +296,9 @@ def test_decode_stack_small_matches_oracle():
     _stack_check(wl, 2, 3)
 
 
-FULL = [("7b-reglu-fp16", 1), ("13b-reglu-q4_0", 1), ("40b-relu-fp16", 1), ("40b-relu-fp16", 2),
-        ("40b-relu-fp16", 8), ("70b-reglu-fp16", 1), ("70b-reglu-fp16", 4), ("70b-reglu-fp16", 16)]
+FULL = [("7b-reglu-fp16", 1), ("13b-reglu-q4_0", 1), ("13b-reglu-q4_0", 4), ("13b-reglu-q4_0", 16),
+        ("40b-relu-fp16", 1), ("40b-relu-fp16", 2), ("40b-relu-fp16", 8), ("70b-reglu-fp16", 1),
+        ("70b-reglu-fp16", 4), ("70b-reglu-fp16", 16)]
 
 
 @pytest.mark.parametrize("name,B", FULL, ids=["%s-b%d" % f for f in FULL])
@@ -303,7 +308,7 @@ def test_full_size_workloads_two_layers_sampled(name, B):
     _full_check(name, B)
 
 
-FULL_TB = [f for f in FULL if f[1] >= 3]
+FULL_TB = [f for f in FULL if f[1] >= 3 and "q4" not in f[0]]  # the switch is for fp16 weights
 
 
 @pytest.mark.parametrize("name,B", FULL_TB, ids=["%s-b%d" % f for f in FULL_TB])
