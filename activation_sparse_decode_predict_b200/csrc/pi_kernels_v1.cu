@@ -283,12 +283,15 @@ __global__ void __launch_bounds__(kDnWarps * 32) k_ffn_down(int B, int d, int ff
   for (int b0 = 0; b0 < B; b0 += NB) {
     const int nb = min(NB, B - b0);
     float acc[UPT][E][NB];
+    float corr[NB];  // Q4_0: the sum of 24 s a over the rows, taken off every column at the end
 #pragma unroll
     for (int q = 0; q < UPT; ++q)
 #pragma unroll
       for (int e = 0; e < E; ++e)
 #pragma unroll
         for (int i = 0; i < NB; ++i) acc[q][e][i] = 0.f;
+#pragma unroll
+    for (int i = 0; i < NB; ++i) corr[i] = 0.f;
     for (int s0 = p0; s0 < p1; s0 += kDnCap) {
       const int len = min(kDnCap, p1 - s0);
       __syncthreads();  // the previous segment (or reduction) is done with the buffer
@@ -340,12 +343,37 @@ __global__ void __launch_bounds__(kDnWarps * 32) k_ffn_down(int B, int d, int ff
 #pragma unroll
             for (int q = 0; q < UPT; ++q) {
               if (ub + 32 * q < units) {
-                float w[E];
-                decode_w<WT>(raw[k][q], w);
+                if constexpr (WT == kQ4_0) {
+                  // s (q - 8) = 16 s f - 24 s with f = 1 + q / 16, made by setting
+                  // the exponent bits of 1.0 around the nibble (exact)
+                  const WRaw<WT>& r = raw[k][q];
+                  const float sc = half_bits_to_float(r.s);
+                  float as[NB];
 #pragma unroll
-                for (int e = 0; e < E; ++e)
+                  for (int i = 0; i < NB; ++i) {
+                    as[i] = 16.f * sc * av[i];
+                    corr[i] = fmaf(24.f * sc, av[i], corr[i]);
+                  }
+                  float f[16];
 #pragma unroll
-                  for (int i = 0; i < NB; ++i) acc[q][e][i] = fmaf(av[i], w[e], acc[q][e][i]);
+                  for (int kk = 0; kk < 4; ++kk) {
+                    f[kk] = __uint_as_float(0x3f800000u | (((r.q.x >> (8 * kk)) << 19) & 0x00780000u));
+                    f[4 + kk] = __uint_as_float(0x3f800000u | (((r.q.y >> (8 * kk)) << 19) & 0x00780000u));
+                    f[8 + kk] = __uint_as_float(0x3f800000u | (((r.q.x >> (8 * kk)) << 15) & 0x00780000u));
+                    f[12 + kk] = __uint_as_float(0x3f800000u | (((r.q.y >> (8 * kk)) << 15) & 0x00780000u));
+                  }
+#pragma unroll
+                  for (int e = 0; e < E; ++e)
+#pragma unroll
+                    for (int i = 0; i < NB; ++i) acc[q][e][i] = fmaf(as[i], f[e], acc[q][e][i]);
+                } else {
+                  float w[E];
+                  decode_w<WT>(raw[k][q], w);
+#pragma unroll
+                  for (int e = 0; e < E; ++e)
+#pragma unroll
+                    for (int i = 0; i < NB; ++i) acc[q][e][i] = fmaf(av[i], w[e], acc[q][e][i]);
+                }
               }
             }
           }
@@ -358,7 +386,8 @@ __global__ void __launch_bounds__(kDnWarps * 32) k_ffn_down(int B, int d, int ff
 #pragma unroll
       for (int e = 0; e < E; ++e)
 #pragma unroll
-        for (int i = 0; i < NB; ++i) red[((size_t)warp * V + (q * E + e) * NB + i) * 32 + lane] = acc[q][e][i];
+        for (int i = 0; i < NB; ++i)
+          red[((size_t)warp * V + (q * E + e) * NB + i) * 32 + lane] = WT == kQ4_0 ? acc[q][e][i] - corr[i] : acc[q][e][i];
     __syncthreads();
     for (int x = threadIdx.x; x < V * 32; x += blockDim.x) {
       const int ln = x & 31, y = x >> 5;
