@@ -318,6 +318,18 @@ def test_full_size_token_blocks_on_tcgen05(name, B):
         _full_check(name, B)
 
 
+FULL_DEPTH = [("7b-reglu-fp16", 1), ("13b-reglu-q4_0", 1)]
+
+
+@pytest.mark.parametrize("name,B", FULL_DEPTH, ids=["%s-b%d" % f for f in FULL_DEPTH])
+def test_full_depth_stack_every_column(name, B):
+    """Every layer of a full-depth stack in the benchmark's one launch (32 and
+    40 layers), every output column, each layer against the oracle fed that
+    layer's GPU input; the glue between layers is checked too."""
+    wl = W.WORKLOADS[name]
+    _stack_check(wl, B, wl.layers, seed_step=7)
+
+
 def _full_check(name, B):
     wl = W.WORKLOADS[name]
     rng = np.random.default_rng(B)
