@@ -347,7 +347,12 @@ pi_status fused_params(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, pi:
     // a consumer holds one group while it waits for the first item of the next
     // one, and a wrap of the ring can waste up to one item: ng + 2 items fit
     const int cap = pi::kNgFull ? (int)((size_t)P.ring_bytes / neuron) - 2 : (int)(half / neuron);
-    const int lim = (desc->wtype == PI_F16 && desc->ptype == PI_F16 && pi::kF16Mma) ? 16 / rpn : 4;
+    // CUDA-core groups: 4 neurons; Q4_0 rows with a Q4_0 predictor or a token
+    // block of 2: 6 (13B-shaped stack: +2.8 % and +4.7 %; with an fp16
+    // predictor and one token 6 lost 3 % and 8 lost 3-6 % everywhere)
+    const int lim = (desc->wtype == PI_F16 && desc->ptype == PI_F16 && pi::kF16Mma) ? 16 / rpn
+                    : (desc->wtype == PI_Q4_0 && (desc->ptype == PI_Q4_0 || B == 2)) ? 6
+                                                                                         : 4;
     P.ng = cap < lim ? cap : lim;
     if (P.ng < 1) P.ng = 1;
   }
