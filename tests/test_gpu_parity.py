@@ -318,6 +318,19 @@ def test_full_size_token_blocks_on_tcgen05(name, B):
         _full_check(name, B)
 
 
+def test_down_projection_ranges_longer_than_one_staging_pass():
+    """The CUDA-core down kernel stages at most 1024 list positions of its
+    range at a time: wide rows (d = 8192: 16 column chunks, 27 ranges) and a
+    list of every neuron (30000) give ranges of ~1111 positions, so every
+    range takes two passes.  Q4_0 token block of 3 through the decode stack,
+    every neuron active (the dense FFN), sampled columns."""
+    wl = _workload("q4-long-ranges", 8192, 30000, 0.05, 128, "reglu", "q4_0", "f16", 3)
+    rng = np.random.default_rng(11)
+    cols = np.sort(rng.choice(wl.d, size=48, replace=False)).astype(np.int32)
+    _, counts = _stack_check(wl, 3, 1, cols=cols, thr=-1e30)
+    assert int(counts[0]) == wl.n_cold
+
+
 FULL_DEPTH = [("7b-reglu-fp16", 1), ("13b-reglu-q4_0", 1)]
 
 
