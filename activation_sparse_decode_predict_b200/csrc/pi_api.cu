@@ -359,9 +359,11 @@ pi_status fused_params(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, pi:
   // about one group of hot neurons per CTA is shared out statically (it fills
   // the wait for barrier U); the rest is claimed, which balances the CTAs
   {
-    // wide rows (d >= 8192) leave only 1-2 neurons per group, and barrier U
-    // takes longer there: three groups fill its wait
-    const int def_a = desc->d >= 8192 ? 3 * P.ng : P.ng;
+    // wide rows (d >= 8192) leave only 2-3 neurons per group, and barrier U
+    // takes longer there: three groups fill its wait, six with gated rows
+    // (measured: 70B-shaped ReGLU 12 neurons per CTA against 6: +0.7-0.9 % at
+    // sparsity 0.80-0.95, 24 -2 %; 40B-shaped ReLU: 9 best, 12 -0.6 %, 3 -3.4 %)
+    const int def_a = desc->d >= 8192 ? (rpn == 2 ? 6 : 3) * P.ng : P.ng;
     const int per_a = pi::kHotA > 0 ? pi::kHotA : def_a, per_b = pi::kHotB > 0 ? pi::kHotB : P.ng;
     P.hot_a = desc->n_hot < G * per_a ? desc->n_hot : G * per_a;
     P.hot_static = desc->n_hot - P.hot_a < G * per_b ? desc->n_hot : P.hot_a + G * per_b;
