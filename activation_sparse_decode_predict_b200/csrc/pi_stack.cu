@@ -678,7 +678,9 @@ __global__ void __maxnreg__(96) k_stack(const __grid_constant__ StackParams p) {
         // while the previous one is issued
         const int PN = H - HA;
         int* pool = p.pool + l;
-        const int cmin = max(1, p.ng / 2), cmax = 4 * p.ng;
+        // a claim is at least half a group, a whole one on wide rows (d >= 8192:
+        // 40B-shaped +1.5 %, 70B-shaped +0.35 %; at 13B a whole group lost 2 %)
+        const int cmin = d >= 8192 ? p.ng : max(1, p.ng / 2), cmax = 4 * p.ng;
         auto csize = [&](int seen) { return max(cmin, min(cmax, (PN - seen) / (2 * G))); };
         int nsz = csize(0);
         int nxt = PN > 0 ? atomicAdd(pool, nsz) : PN;
