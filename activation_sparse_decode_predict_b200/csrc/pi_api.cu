@@ -374,8 +374,9 @@ pi_status fused_params(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, pi:
     // even out the CTAs' predicted cold rows, so every row above a CTA's
     // running mean is handed over; with a larger pool a slack of two rows
     // saves the hand-over round trips (measured: 7B / 13B +2 %, 40B / 70B -1 %
-    // and -0.4 % with no slack)
-    P.don_slack = desc->n_hot - P.hot_static < G * P.ng ? 0 : 2;
+    // and -0.4 % with no slack); one row on gated rows (70B-shaped: +0.35 %
+    // over two, -1.7 % with four; 40B-shaped ReLU keeps two: one lost 0.6 %)
+    P.don_slack = desc->n_hot - P.hot_static < G * P.ng ? 0 : (rpn == 2 ? 1 : 2);
   }
   const int C = desc->ffn - desc->n_hot;
   // every consumer thread holds at most kShareRegs entries of the CTA's P2 bias share
