@@ -356,8 +356,9 @@ pi_status fused_params(const pi_ffn_desc* desc, int32_t B, int32_t n_layers, pi:
     P.ng = cap < lim ? cap : lim;
     if (P.ng < 1) P.ng = 1;
   }
-  // about one group of hot neurons per CTA is shared out statically (it fills
-  // the wait for barrier U); the rest is claimed, which balances the CTAs
+  // a few groups of hot neurons per CTA are shared out statically (they fill
+  // the wait for barrier U and the list's latency after P2); the rest is
+  // claimed, which balances the CTAs
   {
     // wide rows (d >= 8192) leave only 2-3 neurons per group, and barrier U
     // takes longer there: three groups fill its wait, six with gated rows
