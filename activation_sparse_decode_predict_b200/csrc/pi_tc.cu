@@ -347,8 +347,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_up(const __grid_constant__
       const int pos = tile * 128 + q * 32 + lane;
       const int c_lo = range_owner(sp, (int64_t)tile * KB);
       const int nw = range_owner(sp, (int64_t)tile * KB + KB - 1) - c_lo + 1, slot = c - c_lo;
+      // an entry outside [n_hot, ffn) (reported by the producers) adds nothing:
+      // its activation is zero
+      bool valid = false;
       float bias = 0.f;
-      if (pos < ntot && p.b1) bias = __ldg(p.b1 + list_row_at(pos, ntot, p.n_hot, p.ffn, p.idx, ctrl));
+      if (pos < ntot) {
+        const int j = list_raw(pos, ntot, p.n_hot, p.idx);
+        valid = pos < p.n_hot || (j >= p.n_hot && j < p.ffn);
+        if (valid && p.b1) bias = __ldg(p.b1 + j);
+      }
       const bool okw = mbar_wait(&accf[buf], (uint32_t)((nseg / 2) & 1), ctrl);
       if (named_sync_or(1, 128, !okw)) break;  // all epilogue warps leave together
       tc_fence_after();
@@ -421,7 +428,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_up(const __grid_constant__
         float a[16];
 #pragma unroll
         for (int b = 0; b < 16; ++b) a[b] = 0.f;
-        if (pos < ntot) {
+        if (valid) {
 #pragma unroll
           for (int b = 0; b < 16; ++b)
             if (b < p.B) a[b] = p.gated ? act_eval(kReglu, g[b] + bias, v[b]) : act_eval(p.act, g[b] + bias, 0.f);

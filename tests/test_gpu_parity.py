@@ -197,27 +197,39 @@ def _token_block_extremes():
             assert pi.device_status(ws) == 0
 
 
-def test_bad_device_list_is_flagged_and_skipped():
-    wl = _workload("badidx", 128, 500, 0.1, 16, "relu", "f16", "f16", 1)
+BAD_LIST = [("per-kernel", 128, "relu", "f16", 1, "warp_mma"),
+            ("token-block", 256, "reglu", "f16", 4, "warp_mma"),
+            ("token-block-tcgen05", 256, "reglu", "f16", 4, "tcgen05"),
+            ("token-block-q4", 256, "relu", "q4_0", 4, "warp_mma")]
+
+
+@pytest.mark.parametrize("name,d,act,wt,B,path", BAD_LIST, ids=[c[0] for c in BAD_LIST])
+def test_bad_device_list_is_flagged_and_skipped(name, d, act, wt, B, path):
+    """An entry of the list outside [n_hot, ffn) sets PI_ERR_INDEX and adds
+    nothing; a count above the capacity sets PI_ERR_CAPACITY and is clamped
+    -- on every FFN path."""
+    wl = _workload("badidx-" + name, d, 500, 0.1, 16, act, wt, "f16", B)
     L = _layer(wl)
-    h = to_dev(W.make_tokens(wl, 1, 0))
+    h = to_dev(W.make_tokens(wl, B, 0))
     desc = pi.desc_for(wl)
-    ws = pi.workspace(desc, 1)
+    ws = pi.workspace(desc, B)
     good = [wl.n_hot + 3, wl.n_hot + 40, wl.ffn - 1]
     idx = torch.tensor(good[:2] + [wl.ffn + 5] + good[2:], dtype=torch.int32, device="cuda")
     cnt = torch.tensor([4], dtype=torch.int32, device="cuda")
-    y = gpu_ffn(desc, h, L, idx, cnt, ws)
+    with token_ffn(path):
+        y = gpu_ffn(desc, h, L, idx, cnt, ws)
     assert pi.device_status(ws, clear=True) == pi._binding.PI_ERR_INDEX
     ref = oracle_layer(L, to_np(h), wl, good)
-    assert rel_err(y, ref) <= TOL["f16"]
+    assert rel_err(y, ref) <= TOL[wt]
     assert pi.device_status(ws) == 0
     # a count above the list's capacity is flagged and clamped
     full = torch.arange(wl.n_hot, wl.ffn, dtype=torch.int32, device="cuda")
     cnt = torch.tensor([wl.n_cold + 1000], dtype=torch.int32, device="cuda")
-    y = gpu_ffn(desc, h, L, full, cnt, ws)
+    with token_ffn(path):
+        y = gpu_ffn(desc, h, L, full, cnt, ws)
     assert pi.device_status(ws, clear=True) == pi._binding.PI_ERR_CAPACITY
     ref = oracle_layer(L, to_np(h), wl, full.cpu().numpy())
-    assert rel_err(y, ref) <= TOL["f16"]
+    assert rel_err(y, ref) <= TOL[wt]
 
 
 @pytest.mark.parametrize("htype", ["f32", "f16"])
