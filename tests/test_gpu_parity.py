@@ -177,9 +177,16 @@ def test_token_block_extremes(path):
         _token_block_extremes()
 
 
-def _token_block_extremes():
+def test_q4_token_block_extremes():
+    """The Q4_0 token-block path (gate/up codes on the tensor cores, down on the
+    CUDA cores) with an empty list, every neuron active, and one workspace
+    reused by lists of different lengths."""
+    _token_block_extremes("q4_0")
+
+
+def _token_block_extremes(wt="f16"):
     for act, B in (("relu", 4), ("reglu", 16)):
-        wl = _workload("tc-edge-" + act, 512, 1000, 0.0, 32, act, "f16", "f16", B)
+        wl = _workload("tc-edge-" + act + "-" + wt, 512, 1000, 0.0, 32, act, wt, "f16", B)
         L = _layer(wl)
         h = to_dev(W.make_tokens(wl, B, 5))
         h_np = to_np(h)
@@ -193,7 +200,7 @@ def _token_block_extremes():
             if thr == -1e30:
                 assert len(gidx) == wl.n_cold
             y = gpu_ffn(desc, h, Lt, idx_t, cnt_t, ws)
-            assert rel_err(y, oracle_layer(Lt, h_np, wl, gidx)) <= TOL["f16"], (act, thr)
+            assert rel_err(y, oracle_layer(Lt, h_np, wl, gidx)) <= TOL[wt], (act, thr)
             assert pi.device_status(ws) == 0
 
 
