@@ -99,6 +99,9 @@ INT_CASES = [
     (160, 300, 300, 16, "relu", "q4_0", "f16", 1),
     (256, 700, 70, 32, "reglu", "f16", "f16", 16),
     (256, 700, 70, 32, "relu", "f16", "f16", 8),
+    # Q4_0 token blocks: codes decoded into tensor-core fragments, down on the CUDA cores
+    (256, 600, 30, 32, "reglu", "q4_0", "f16", 4),
+    (512, 700, 50, 32, "relu", "q4_0", "f16", 16),
 ]
 
 
