@@ -14,10 +14,10 @@ from gpu_util import check_index_list, oracle_layer, oracle_predict, to_np
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("B", [1, 3])
-def test_decode_blocks_match_oracle(B):
+@pytest.mark.parametrize("wt,B", [("f16", 1), ("f16", 3), ("q4_0", 3)])
+def test_decode_blocks_match_oracle(wt, B):
     n_layers, L, s_max = 2, 40, 64
-    wl = W.Workload("blocks", 88, 512, 1500, n_layers, "reglu", "f16", "f16", 0.88, 1.2, 0.1, 64, (B,), 1)
+    wl = W.Workload("blocks-" + wt, 88, 512, 1500, n_layers, "reglu", wt, "f16", 0.88, 1.2, 0.1, 64, (B,), 1)
     H, n_hot_h, head_rank = 8, 1, 32
     fdesc = pi.desc_for(wl)
     adesc = pi.attn_desc(wl.d, H, n_hot_h, s_max)
