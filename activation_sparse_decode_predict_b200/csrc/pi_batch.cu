@@ -1,5 +1,6 @@
 // pi_batch.cu -- the sparse FFN of a token block of 3..16 tokens on the
-// tensor cores (fp16 weights, fp16 tokens).
+// tensor cores (fp16 tokens; fp16 weights, or Q4_0 gate/up rows whose codes
+// are decoded in registers into the mma fragments).
 //
 // PowerInfer (unite.ai, "Nöron Bilinçli Operatör"; aibars.net,
 // "Sparsity-Nutzung"): only the rows of the hot neurons and of the
@@ -17,6 +18,10 @@
 //          the token columns of the part: dots -> out[part][pos][slot][tok].
 //          It also runs the predictor of a token block: P1 rows against the
 //          tokens, then P2 rows against u split into fp16 hi + lo rows.
+//          Q4_0 rows (list mode): codes and scales stream per row piece; the
+//          codes become exact fp16 integers q - 8 in fragment order and each
+//          block's scale multiplies its two k-steps' fp32 sums (the down
+//          projection of Q4_0 blocks runs on the CUDA cores, pi_kernels_v1.cu).
 // k_bdown  CTA = (chunk of d, range of list positions).  Activations from
 //          pre (summed over the parts) and b1, split into fp16 hi + lo so the
 //          product keeps ~22 bits of each activation; fp32 partial output of
